@@ -1,0 +1,232 @@
+"""CPU oracle for the MoE layer forward -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may import
+this package.  The library path never touches it: the CUDA path and the oracle
+share no code.  The arithmetic lives in ``moe_oracle.c`` (plain C, IEEE double,
+plain loops); this module compiles it with gcc and wraps it with numpy.
+
+Every function cites the passage it follows in the C source.  Inputs are numpy
+arrays: bf16 tensors are passed as their uint16 bit patterns (dtype code 0),
+fp32 tensors as float32 (dtype code 1).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+BF16, FP32 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so from moe_oracle.c (gcc, OpenMP)."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        L.oracle_router_logits.argtypes = [i, i, i, i, P, P, P]
+        L.oracle_topk.argtypes = [i, i, i, P, P]
+        L.oracle_gate_weights.argtypes = [i, i, i, i, i, P, P, P]
+        L.oracle_align.argtypes = [i, i, i, i, P, ctypes.c_int64, P, P, P, P, P, P, P]
+        L.oracle_swiglu_ffn.argtypes = [i, i, i, P, P, P, P]
+        L.oracle_dense_ffn.argtypes = [i, i, i, i, P, P, P, P, i]
+        L.oracle_moe_layer.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, i, P, P, P, i]
+        for f in (L.oracle_router_logits, L.oracle_topk, L.oracle_gate_weights, L.oracle_align,
+                  L.oracle_swiglu_ffn, L.oracle_dense_ffn, L.oracle_moe_layer):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _typed(a):
+    """Return (contiguous array, dtype code) for a bf16-as-uint16 or fp32 array."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return a, BF16
+    if a.dtype == np.float32:
+        return a, FP32
+    raise TypeError(f"oracle inputs are uint16 (bf16 bits) or float32, got {a.dtype}")
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its input (rc={rc})")
+
+
+def nthreads_default() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def router_logits(x, w_r):
+    """logits[T,E] (float64) = x . W_r^T."""
+    x, dt = _typed(x)
+    w_r, dt2 = _typed(w_r)
+    assert dt == dt2
+    T, H = x.shape
+    E = w_r.shape[0]
+    out = np.empty((T, E), np.float64)
+    _check(lib().oracle_router_logits(T, H, E, dt, _ptr(x), _ptr(w_r), _ptr(out)), "router_logits")
+    return out
+
+
+def topk(logits, K):
+    """ids[T,K] int32: K largest fp32 logits per token, lower index on ties."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    ids = np.empty((T, K), np.int32)
+    _check(lib().oracle_topk(T, E, K, _ptr(logits), _ptr(ids)), "topk")
+    return ids
+
+
+def gate_weights(logits, ids, score_fn=0, renorm=1):
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, E = logits.shape
+    K = ids.shape[1]
+    w = np.empty((T, K), np.float64)
+    _check(lib().oracle_gate_weights(T, E, K, score_fn, renorm, _ptr(logits), _ptr(ids), _ptr(w)),
+           "gate_weights")
+    return w
+
+
+def expected_active(E: int, K: int, m: int) -> float:
+    """E[E_active] = E * (1 - (1 - K/E)^m): expected number of experts that
+    receive at least one of m tokens under uniform top-K routing (talk notes,
+    "Balls-Bins-Buckets" model construction)."""
+    return E * (1.0 - (1.0 - K / E) ** m)
+
+
+def p_max(T, K, E, B):
+    """Upper bound on padded rows: A + min(E, A) * (B - 1), A = T*K."""
+    A = T * K
+    return A + min(E, A) * (B - 1)
+
+
+def align(ids, E, B, P_max=None):
+    """Block-wise alignment of the assignments; returns a dict of int32 arrays."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, K = ids.shape
+    if P_max is None:
+        P_max = p_max(T, K, E, B)
+    nblk = (P_max + B - 1) // B
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    sorted_ids = np.empty(max(P_max, 1), np.int32)
+    block_expert = np.empty(max(nblk, 1), np.int32)
+    pos = np.empty(max(T * K, 1), np.int32)
+    P = np.zeros(1, np.int32)
+    ea = np.zeros(1, np.int32)
+    _check(lib().oracle_align(T, K, E, B, _ptr(ids), P_max, _ptr(counts), _ptr(offsets),
+                              _ptr(sorted_ids), _ptr(block_expert), _ptr(pos), _ptr(P), _ptr(ea)),
+           "align")
+    return dict(counts=counts, offsets=offsets, sorted_ids=sorted_ids[:P_max],
+                block_expert=block_expert[:nblk], pos=pos[:T * K], P=int(P[0]), E_active=int(ea[0]))
+
+
+def swiglu_ffn(x_row, w13, w2):
+    """y[H] for one token through one SwiGLU expert (w13 [2I,H], w2 [H,I])."""
+    x_row, dt = _typed(x_row)
+    w13, _ = _typed(w13)
+    w2, _ = _typed(w2)
+    H = x_row.shape[-1]
+    I = w2.shape[1]
+    y = np.empty(H, np.float64)
+    _check(lib().oracle_swiglu_ffn(H, I, dt, _ptr(x_row), _ptr(w13), _ptr(w2), _ptr(y)), "swiglu_ffn")
+    return y
+
+
+def dense_ffn(x, w13, w2, nthreads=None):
+    """out[T,H] (float64) of a dense SwiGLU FFN (DenseFA / DensePA / shared)."""
+    x, dt = _typed(x)
+    w13, _ = _typed(w13)
+    w2, _ = _typed(w2)
+    T, H = x.shape
+    I = w2.shape[1]
+    out = np.empty((T, H), np.float64)
+    _check(lib().oracle_dense_ffn(T, H, I, dt, _ptr(x), _ptr(w13), _ptr(w2), _ptr(out),
+                                  nthreads or nthreads_default()), "dense_ffn")
+    return out
+
+
+def moe_layer(x, w_r, w13, w2, K, score_fn=0, renorm=1, w13_sh=None, w2_sh=None,
+              logits=None, tokens=None, nthreads=None, return_routing=False):
+    """MoE layer output rows (float64) for the listed tokens (all if None).
+
+    w13 / w2: either stacked arrays [E,2I,H] / [E,H,I], or lists of per-expert
+    arrays (None allowed for experts that no listed token selects).
+    """
+    x, dt = _typed(x)
+    T, H = x.shape
+    if isinstance(w13, np.ndarray):
+        E = w13.shape[0]
+        w13_list = [np.ascontiguousarray(w13[e]) for e in range(E)]
+        w2_list = [np.ascontiguousarray(w2[e]) for e in range(E)]
+    else:
+        w13_list, w2_list = list(w13), list(w2)
+        E = len(w13_list)
+    I = next(w.shape[1] for w in w2_list if w is not None)
+    keep = []
+    p13 = (ctypes.c_void_p * E)()
+    p2 = (ctypes.c_void_p * E)()
+    for e in range(E):
+        for arr, tab in ((w13_list[e], p13), (w2_list[e], p2)):
+            if arr is None:
+                tab[e] = None
+            else:
+                a, d = _typed(arr)
+                assert d == dt
+                keep.append(a)
+                tab[e] = a.ctypes.data
+    w_r_c = None
+    if w_r is not None:
+        w_r_c, d = _typed(w_r)
+        assert d == dt
+    I_sh = 0
+    if w13_sh is not None:
+        w13_sh, _ = _typed(w13_sh)
+        w2_sh, _ = _typed(w2_sh)
+        I_sh = w2_sh.shape[1]
+    lg = None
+    if logits is not None:
+        lg = np.ascontiguousarray(logits, dtype=np.float32)
+    elif w_r_c is None:
+        raise ValueError("need router weights or logits")
+    tok = None
+    n = T
+    if tokens is not None:
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = tok.shape[0]
+    out = np.empty((n, H), np.float64)
+    ids = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float64)
+    rc = lib().oracle_moe_layer(T, H, E, K, I, I_sh, score_fn, renorm, dt, _ptr(x), _ptr(w_r_c),
+                                p13, p2, _ptr(w13_sh), _ptr(w2_sh), _ptr(lg), _ptr(tok), n,
+                                _ptr(out), _ptr(ids), _ptr(w), nthreads or nthreads_default())
+    _check(rc, "moe_layer")
+    if return_routing:
+        return out, ids, w
+    return out

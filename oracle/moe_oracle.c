@@ -1,0 +1,364 @@
+/*
+ * moe_oracle.c -- plain, slow, obviously-correct CPU reference for one
+ * Mixture-of-Experts FFN layer forward and its dense baselines.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library path may link, import or
+ * call this file: it exists so that tests, the smoke check and the CPU
+ * baseline of the benchmark can check the CUDA path against the definitions.
+ * It shares no code, header, table or helper with the CUDA sources.
+ *
+ * Arithmetic is IEEE double throughout (inputs are widened exactly: a bf16
+ * value is the upper 16 bits of an fp32 value), plain loops in the order the
+ * definitions are written, no blocking or fusion.
+ *
+ * Sources (web pages on "Demystifying the Mixture of Experts Serving Tax",
+ * MLSys 2026):
+ *   - notes.yuuk.io talk notes, section "MoE serving tax: definition"
+ *     (Eq. 1, DenseFA / DensePA definitions);
+ *   - same page, "Key findings 5" (the stages of the MoE block: router, top-K
+ *     selection, alignment, GroupGEMM, local sum);
+ *   - same page, "Padding model (Section 5.1)" (block-wise padding
+ *     P = sum_i ceil(N_i / B) * B);
+ *   - same page, "Balls-Bins-Buckets" (token-count vector N = [N_1..N_E],
+ *     m tokens x K assignments);
+ *   - same page, Table 2 (shared experts).
+ * Concrete gating (softmax renormalised over the selected K, or sigmoid
+ * normalised over the selected K), SwiGLU experts and the tile size come from
+ * the layer definitions of the workloads (Mixtral-, Qwen2-MoE-,
+ * DeepSeek-V3-shaped layers).  Readings where the pages are silent:
+ *   - top-K is taken on the fp32 router logit, descending, ties broken by
+ *     the lower expert index, IEEE comparison (so -0.0 ties +0.0); a NaN
+ *     logit is rejected (return -1);
+ *   - the K outputs of a token are listed in that order, which fixes k;
+ *   - shared experts have weight 1 and no gate; S experts of width I_s are
+ *     one dense SwiGLU FFN of width S*I_s;
+ *   - padding slots of sorted_ids are -1; blocks past P in block_expert are
+ *     -1; experts with N_e = 0 get no rows.
+ *
+ * Parity status: every function below is pinned by the CPU tests (brute force
+ * over subsets, closed forms, invariants, hand-worked fixtures, reductions).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* dtype codes: 0 = bf16 (uint16 bit patterns), 1 = fp32 */
+static double ld(const void* p, size_t i, int dtype)
+{
+    if (dtype == 0) {
+        uint32_t bits = ((uint32_t)((const uint16_t*)p)[i]) << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float*)p)[i];
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* ---------------------------------------------------------------- router */
+/* logits[t][e] = sum_h x[t][h] * w_r[e][h]  (router GEMM, x.W_r^T) */
+int oracle_router_logits(int T, int H, int E, int dtype, const void* x,
+                         const void* w_r, double* logits)
+{
+    if (T < 0 || H <= 0 || E <= 0) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int h = 0; h < H; ++h)
+                s += ld(x, (size_t)t * H + h, dtype) * ld(w_r, (size_t)e * H + h, dtype);
+            logits[(size_t)t * E + e] = s;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ top-K */
+/* K passes; each pass picks the not-yet-selected expert with the largest
+ * logit, the lowest index winning a tie.  ids[t][0..K-1] in selection order. */
+int oracle_topk(int T, int E, int K, const float* logits, int32_t* ids)
+{
+    if (T < 0 || E <= 0 || K <= 0 || K > E) return -1;
+    char* taken = (char*)malloc((size_t)E);
+    if (!taken) return -2;
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + (size_t)t * E;
+        for (int e = 0; e < E; ++e) {
+            if (isnan(l[e])) { free(taken); return -1; }
+            taken[e] = 0;
+        }
+        for (int k = 0; k < K; ++k) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e; /* strict: ties keep lower e */
+            }
+            taken[best] = 1;
+            ids[(size_t)t * K + k] = best;
+        }
+    }
+    free(taken);
+    return 0;
+}
+
+/* ---------------------------------------------------------------- weights */
+/* score_fn 0 = softmax, 1 = sigmoid.
+ * softmax, renorm=1: w_j = exp(l_j - m) / sum_{i in sel} exp(l_i - m), m = max over sel
+ * softmax, renorm=0: w_j = exp(l_j - m) / sum_{all e} exp(l_e - m), m = max over all
+ * sigmoid, renorm=1: w_j = s_j / sum_{i in sel} s_i,  s = 1/(1+exp(-l))
+ * sigmoid, renorm=0: w_j = s_j */
+int oracle_gate_weights(int T, int E, int K, int score_fn, int renorm,
+                        const float* logits, const int32_t* ids, double* w)
+{
+    if (T < 0 || E <= 0 || K <= 0 || K > E) return -1;
+    if (score_fn != 0 && score_fn != 1) return -1;
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + (size_t)t * E;
+        const int32_t* id = ids + (size_t)t * K;
+        double* wt = w + (size_t)t * K;
+        if (score_fn == 0) {
+            double m = -INFINITY, den = 0.0;
+            if (renorm) {
+                for (int k = 0; k < K; ++k) if ((double)l[id[k]] > m) m = l[id[k]];
+                for (int k = 0; k < K; ++k) den += exp((double)l[id[k]] - m);
+            } else {
+                for (int e = 0; e < E; ++e) if ((double)l[e] > m) m = l[e];
+                for (int e = 0; e < E; ++e) den += exp((double)l[e] - m);
+            }
+            for (int k = 0; k < K; ++k) wt[k] = exp((double)l[id[k]] - m) / den;
+        } else {
+            double den = 0.0;
+            for (int k = 0; k < K; ++k) den += sigmoid((double)l[id[k]]);
+            for (int k = 0; k < K; ++k)
+                wt[k] = renorm ? sigmoid((double)l[id[k]]) / den : sigmoid((double)l[id[k]]);
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------- align + pad */
+/* Assignments a = t*K + k, expert e(a) = ids[a], A = T*K.
+ *   counts[e]  = N_e = #{a : e(a) = e}
+ *   padded N^_e = ceil(N_e / B) * B                    (block-wise padding)
+ *   offsets    = exclusive scan of N^, offsets[E] = P = sum_e N^_e
+ *   sorted_ids[p] = a, a ascending within each expert's segment; -1 elsewhere
+ *   pos[a]     = the slot p holding a
+ *   block_expert[b] = e for b in [offsets[e]/B, offsets[e+1]/B), -1 for b >= P/B
+ *   E_active   = #{e : N_e > 0}
+ * sorted_ids has P_max slots, block_expert ceil(P_max/B) entries. */
+int oracle_align(int T, int K, int E, int B, const int32_t* ids, int64_t P_max,
+                 int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                 int32_t* block_expert, int32_t* pos, int32_t* P_out,
+                 int32_t* E_active_out)
+{
+    if (T < 0 || K <= 0 || E <= 0 || B <= 0) return -1;
+    int64_t A = (int64_t)T * K;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t a = 0; a < A; ++a) {
+        if (ids[a] < 0 || ids[a] >= E) return -1;
+        counts[ids[a]] += 1;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        int32_t padded = ((counts[e] + B - 1) / B) * B;
+        offsets[e + 1] = offsets[e] + padded;
+    }
+    int32_t P = offsets[E];
+    if (P > P_max) return -1;
+    for (int64_t p = 0; p < P_max; ++p) sorted_ids[p] = -1;
+    int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+    if (!cursor) return -2;
+    for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
+    for (int64_t a = 0; a < A; ++a) {
+        int e = ids[a];
+        sorted_ids[cursor[e]] = (int32_t)a;
+        pos[a] = cursor[e];
+        cursor[e] += 1;
+    }
+    free(cursor);
+    int64_t nblk = (P_max + B - 1) / B;
+    for (int64_t b = 0; b < nblk; ++b) block_expert[b] = -1;
+    for (int e = 0; e < E; ++e)
+        for (int32_t b = offsets[e] / B; b < offsets[e + 1] / B; ++b) block_expert[b] = e;
+    int ea = 0;
+    for (int e = 0; e < E; ++e) if (counts[e] > 0) ++ea;
+    *P_out = P;
+    *E_active_out = ea;
+    return 0;
+}
+
+/* ------------------------------------------------------------- SwiGLU FFN */
+/* One token through one SwiGLU expert.  w13 is [2I, H]: rows 0..I-1 are the
+ * gate projection W1, rows I..2I-1 the up projection W3; w2 is [H, I].
+ *   g_i = sum_h W1[i][h] x[h];  u_i = sum_h W3[i][h] x[h]
+ *   a_i = silu(g_i) * u_i,      silu(v) = v * sigmoid(v)
+ *   y_h = sum_i W2[h][i] a_i
+ * x is given as an element offset into a typed array. */
+static void ffn_one(int H, int I, int dtype, const void* x, size_t x_off,
+                    const void* w13, const void* w2, double* a_scratch, double* y)
+{
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = ld(x, x_off + h, dtype);
+            g += ld(w13, (size_t)i * H + h, dtype) * xv;
+            u += ld(w13, (size_t)(I + i) * H + h, dtype) * xv;
+        }
+        a_scratch[i] = g * sigmoid(g) * u;
+    }
+    for (int h = 0; h < H; ++h) {
+        double s = 0.0;
+        for (int i = 0; i < I; ++i) s += ld(w2, (size_t)h * I + i, dtype) * a_scratch[i];
+        y[h] = s;
+    }
+}
+
+/* y[H] for one token row x[H] through one expert (exported for the tests). */
+int oracle_swiglu_ffn(int H, int I, int dtype, const void* x, const void* w13,
+                      const void* w2, double* y)
+{
+    if (H <= 0 || I <= 0) return -1;
+    double* a = (double*)malloc(sizeof(double) * (size_t)I);
+    if (!a) return -2;
+    ffn_one(H, I, dtype, x, 0, w13, w2, a, y);
+    free(a);
+    return 0;
+}
+
+/* Dense SwiGLU FFN over T tokens (DenseFA / DensePA / shared experts):
+ * out[t] = W2 (silu(W1 x_t) * (W3 x_t)).  Its own loops: no routing. */
+int oracle_dense_ffn(int T, int H, int I, int dtype, const void* x,
+                     const void* w13, const void* w2, double* out, int nthreads)
+{
+    if (T < 0 || H <= 0 || I <= 0) return -1;
+    int err = 0;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        double* g = (double*)malloc(sizeof(double) * (size_t)I);
+        double* u = (double*)malloc(sizeof(double) * (size_t)I);
+        if (!g || !u) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int t = 0; t < T; ++t) {
+                for (int i = 0; i < I; ++i) {
+                    g[i] = 0.0;
+                    u[i] = 0.0;
+                }
+                for (int i = 0; i < I; ++i)
+                    for (int h = 0; h < H; ++h) {
+                        double xv = ld(x, (size_t)t * H + h, dtype);
+                        g[i] += ld(w13, (size_t)i * H + h, dtype) * xv;
+                        u[i] += ld(w13, (size_t)(I + i) * H + h, dtype) * xv;
+                    }
+                for (int h = 0; h < H; ++h) {
+                    double s = 0.0;
+                    for (int i = 0; i < I; ++i)
+                        s += ld(w2, (size_t)h * I + i, dtype) * (g[i] * sigmoid(g[i]) * u[i]);
+                    out[(size_t)t * H + h] = s;
+                }
+            }
+        }
+        free(g);
+        free(u);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------- MoE layer */
+/* Full layer forward for the tokens listed in `tokens` (n_tok of them; NULL
+ * means all T in order).  For each listed token t:
+ *   1. l = logits_in[t] if given, else fp32(x_t . W_r^T) from the router GEMM;
+ *   2. top-K ids (descending logit, lower index on ties);
+ *   3. gate weights (softmax / sigmoid, renormalised or not);
+ *   4. y_k = SwiGLU expert ids[k] applied to x_t directly (no permutation);
+ *   5. shared: y_s = SwiGLU with the shared weights (I_sh = S*I_s; 0 = none);
+ *   6. out[j] = sum_k w_k y_k + y_s.
+ * w13[e] / w2[e] point at expert e's [2I,H] and [H,I] weights (entries for
+ * experts no listed token selects may be NULL).  ids_out / w_out (nullable)
+ * receive the routing of each listed token.  Returns -1 on bad input
+ * (NaN logit, NULL weight of a selected expert). */
+int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
+                     int renorm, int dtype, const void* x, const void* w_r,
+                     const void* const* w13, const void* const* w2,
+                     const void* w13_sh, const void* w2_sh, const float* logits_in,
+                     const int32_t* tokens, int n_tok, double* out,
+                     int32_t* ids_out, double* w_out, int nthreads)
+{
+    if (T < 0 || H <= 0 || E <= 0 || K <= 0 || K > E || I <= 0 || I_sh < 0) return -1;
+    if (n_tok < 0) return -1;
+    int err = 0;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        float* l = (float*)malloc(sizeof(float) * (size_t)E);
+        double* ld_logits = (double*)malloc(sizeof(double) * (size_t)E);
+        int32_t* id = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+        double* w = (double*)malloc(sizeof(double) * (size_t)K);
+        int Imax = I > I_sh ? I : I_sh;
+        double* a = (double*)malloc(sizeof(double) * (size_t)(Imax > 0 ? Imax : 1));
+        double* y = (double*)malloc(sizeof(double) * (size_t)H);
+        if (!l || !ld_logits || !id || !w || !a || !y) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int j = 0; j < n_tok; ++j) {
+                int t = tokens ? tokens[j] : j;
+                if (t < 0 || t >= T) {
+#pragma omp atomic write
+                    err = -1;
+                    continue;
+                }
+                size_t xo = (size_t)t * H;
+                if (logits_in) {
+                    for (int e = 0; e < E; ++e) l[e] = logits_in[(size_t)t * E + e];
+                } else {
+                    for (int e = 0; e < E; ++e) {
+                        double s = 0.0;
+                        for (int h = 0; h < H; ++h)
+                            s += ld(x, xo + h, dtype) * ld(w_r, (size_t)e * H + h, dtype);
+                        ld_logits[e] = s;
+                        l[e] = (float)s;
+                    }
+                }
+                if (oracle_topk(1, E, K, l, id) != 0 ||
+                    oracle_gate_weights(1, E, K, score_fn, renorm, l, id, w) != 0) {
+#pragma omp atomic write
+                    err = -1;
+                    continue;
+                }
+                double* o = out + (size_t)j * H;
+                for (int h = 0; h < H; ++h) o[h] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    int e = id[k];
+                    if (!w13[e] || !w2[e]) {
+#pragma omp atomic write
+                        err = -1;
+                        break;
+                    }
+                    ffn_one(H, I, dtype, x, xo, w13[e], w2[e], a, y);
+                    for (int h = 0; h < H; ++h) o[h] += w[k] * y[h];
+                }
+                if (I_sh > 0) {
+                    ffn_one(H, I_sh, dtype, x, xo, w13_sh, w2_sh, a, y);
+                    for (int h = 0; h < H; ++h) o[h] += y[h];
+                }
+                if (ids_out)
+                    for (int k = 0; k < K; ++k) ids_out[(size_t)j * K + k] = id[k];
+                if (w_out)
+                    for (int k = 0; k < K; ++k) w_out[(size_t)j * K + k] = w[k];
+            }
+        }
+        free(l);
+        free(ld_logits);
+        free(id);
+        free(w);
+        free(a);
+        free(y);
+    }
+    return err;
+}

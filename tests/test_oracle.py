@@ -1,0 +1,430 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- brute force, closed forms, hand-worked fixtures, invariants and
+special cases that reduce to a library routine -- so that a dropped term, a
+wrong index, a transposed operand or a swapped gate/up fails at least one."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+import moe_inputs as mi
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f32(v):
+    if isinstance(v, str):
+        return {"-0.0": np.float32(-0.0), "inf": np.float32(np.inf), "-inf": np.float32(-np.inf),
+                "ln3": np.float32(math.log(3.0)), "-ln3": np.float32(-math.log(3.0))}[v]
+    return np.float32(v)
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------- top-K
+
+def brute_topk(row, K):
+    """Subset whose (descending logit, ascending index) key list is the
+    lexicographic maximum over all C(E,K) subsets."""
+    E = len(row)
+    best, best_key = None, None
+    for sub in itertools.combinations(range(E), K):
+        order = sorted(sub, key=lambda e: (-float(row[e]), e))
+        key = [(float(row[e]), -e) for e in order]
+        if best_key is None or key > best_key:
+            best, best_key = order, key
+    return best
+
+
+@pytest.mark.parametrize("kind", ["gauss", "ties", "inf"])
+def test_topk_matches_subset_bruteforce(kind):
+    rng = np.random.default_rng(11)
+    for E in range(1, 11):
+        for K in range(1, min(E, 4) + 1):
+            T = 12
+            if kind == "gauss":
+                lg = rng.standard_normal((T, E)).astype(np.float32)
+            elif kind == "ties":
+                lg = mi.tie_heavy_logits(T, E, seed=E * 10 + K, levels=1)
+            else:
+                lg = mi.tie_heavy_logits(T, E, seed=E * 7 + K, levels=2)
+                lg[lg == 2] = np.inf
+                lg[lg == -2] = -np.inf
+            ids = oracle.topk(lg, K)
+            for t in range(T):
+                assert list(ids[t]) == brute_topk(lg[t], K), (E, K, lg[t], ids[t])
+
+
+def test_topk_matches_stable_argsort():
+    # A stable sort on the negated logit keeps the lower index first on ties;
+    # numpy compares -0.0 equal to +0.0, as IEEE does.
+    rng = np.random.default_rng(3)
+    for E, K in [(8, 2), (64, 8), (256, 8), (37, 5)]:
+        lg = np.concatenate([rng.standard_normal((20, E)).astype(np.float32),
+                             mi.tie_heavy_logits(20, E, seed=E)], 0)
+        ids = oracle.topk(lg, K)
+        ref = np.argsort(-lg, axis=1, kind="stable")[:, :K]
+        assert np.array_equal(ids, ref.astype(np.int32))
+
+
+def test_topk_golden_ties():
+    g = _load("topk_ties.json")
+    lg = np.array([[_f32(v) for v in r["logits"]] for r in g["rows"]], np.float32)
+    ids = oracle.topk(lg, g["K"])
+    assert ids.tolist() == [r["ids"] for r in g["rows"]]
+
+
+def test_topk_K_equals_E_is_a_permutation():
+    lg = mi.tie_heavy_logits(30, 9, seed=5)
+    ids = oracle.topk(lg, 9)
+    for t in range(30):
+        assert sorted(ids[t]) == list(range(9))
+        vals = lg[t, ids[t]]
+        assert np.all(vals[:-1] >= vals[1:])
+
+
+def test_topk_rejects_nan():
+    lg = np.zeros((2, 4), np.float32)
+    lg[1, 2] = np.nan
+    with pytest.raises(ValueError):
+        oracle.topk(lg, 2)
+
+
+# ---------------------------------------------------------------- weights
+
+def test_gate_weights_golden():
+    for c in _load("gate_weights.json")["cases"]:
+        lg = np.array([[_f32(v) for v in c["logits"]]], np.float32)
+        ids = oracle.topk(lg, c["K"])
+        assert ids[0].tolist() == c["ids"]
+        w = oracle.gate_weights(lg, ids, c["score_fn"], c["renorm"])
+        assert np.allclose(w[0], c["w"], rtol=1e-6, atol=1e-7), (c, w)
+
+
+def test_softmax_K_equals_E_is_full_softmax():
+    rng = np.random.default_rng(4)
+    lg = (3 * rng.standard_normal((16, 7))).astype(np.float32)
+    ids = oracle.topk(lg, 7)
+    for renorm in (0, 1):
+        w = oracle.gate_weights(lg, ids, 0, renorm)
+        ref = scipy.special.softmax(lg.astype(np.float64), axis=1)
+        assert np.allclose(w, np.take_along_axis(ref, ids, 1), rtol=1e-12)
+
+
+def test_softmax_renorm_is_topk_slice_renormalised():
+    # renorm=0 gives the full softmax restricted to the selected experts; its
+    # renormalisation over the K selected equals the renorm=1 weights.
+    rng = np.random.default_rng(5)
+    lg = (2 * rng.standard_normal((32, 16))).astype(np.float32)
+    ids = oracle.topk(lg, 4)
+    w0 = oracle.gate_weights(lg, ids, 0, 0)
+    w1 = oracle.gate_weights(lg, ids, 0, 1)
+    ref = scipy.special.softmax(lg.astype(np.float64), axis=1)
+    assert np.allclose(w0, np.take_along_axis(ref, ids, 1), rtol=1e-12)
+    assert np.allclose(w1, w0 / w0.sum(1, keepdims=True), rtol=1e-12)
+    assert np.all(w1[:, :-1] >= w1[:, 1:])
+
+
+def test_softmax_shift_invariance_and_sigmoid_values():
+    lg = mi.tie_heavy_logits(16, 8, seed=9, levels=4).astype(np.float32)
+    ids = oracle.topk(lg, 3)
+    w = oracle.gate_weights(lg, ids, 0, 1)
+    w_shift = oracle.gate_weights(lg + np.float32(5.0), ids, 0, 1)
+    assert np.allclose(w, w_shift, rtol=1e-12)
+    ws = oracle.gate_weights(lg, ids, 1, 0)
+    ref = scipy.special.expit(np.take_along_axis(lg, ids, 1).astype(np.float64))
+    assert np.allclose(ws, ref, rtol=1e-12)
+    wsn = oracle.gate_weights(lg, ids, 1, 1)
+    assert np.allclose(wsn.sum(1), 1.0, rtol=1e-12)
+
+
+# ------------------------------------------------------------------ align
+
+def _check_align_invariants(ids, E, B, r):
+    T, K = ids.shape
+    A = T * K
+    counts, offsets, sid, be, pos = r["counts"], r["offsets"], r["sorted_ids"], r["block_expert"], r["pos"]
+    assert counts.sum() == A
+    assert np.array_equal(counts, np.bincount(ids.ravel(), minlength=E))
+    padded = np.diff(offsets)
+    assert offsets[0] == 0 and np.all(padded >= 0)
+    assert np.all(padded % B == 0)
+    assert np.all((padded - counts >= 0) & (padded - counts < B))
+    assert np.all((padded == 0) == (counts == 0))
+    assert offsets[E] == r["P"]
+    # section 5.1 closed form of the padded rows
+    assert r["P"] == int(sum(-(-int(n) // B) * B for n in counts))
+    assert len(sid) == oracle.p_max(T, K, E, B)
+    valid = sid[sid >= 0]
+    assert np.array_equal(np.sort(valid), np.arange(A))          # bijection onto [0, A)
+    assert np.all(sid[r["P"]:] == -1)
+    for a in range(A):
+        assert sid[pos[a]] == a
+    for e in range(E):
+        seg = sid[offsets[e]:offsets[e + 1]]
+        real = seg[:counts[e]]
+        assert np.all(seg[counts[e]:] == -1)
+        assert np.all(np.diff(real) > 0)                         # ascending a
+        assert np.all(ids.ravel()[real] == e)
+        assert np.all(be[offsets[e] // B:offsets[e + 1] // B] == e)
+    assert np.all(be[r["P"] // B:] == -1)
+    assert r["E_active"] == int((counts > 0).sum())
+
+
+def test_align_golden():
+    g = _load("align_small.json")
+    ids = np.array(g["ids"], np.int32)
+    r = oracle.align(ids, g["E"], g["B"])
+    assert oracle.p_max(g["T"], g["K"], g["E"], g["B"]) == g["P_max"]
+    for key in ("counts", "offsets", "sorted_ids", "pos", "block_expert"):
+        assert r[key].tolist() == g[key], key
+    assert r["P"] == g["P"] and r["E_active"] == g["E_active"]
+    _check_align_invariants(ids, g["E"], g["B"], r)
+
+
+@pytest.mark.parametrize("B", [1, 4, 16, 128])
+def test_align_invariants_random(B):
+    rng = np.random.default_rng(B)
+    for T, E, K in [(1, 8, 2), (37, 8, 2), (64, 64, 8), (50, 256, 8), (3, 5, 5), (0, 4, 2)]:
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+        ids = oracle.topk(lg, K) if T else np.zeros((0, K), np.int32)
+        r = oracle.align(ids, E, B)
+        _check_align_invariants(ids, E, B, r)
+
+
+def test_align_single_expert_closed_form():
+    # every token on expert 0 (K=1): P = ceil(A/B)*B, one active expert
+    for T, B in [(1, 16), (16, 16), (17, 16), (300, 128)]:
+        ids = np.zeros((T, 1), np.int32)
+        r = oracle.align(ids, 4, B)
+        assert r["P"] == -(-T // B) * B
+        assert r["E_active"] == 1
+        assert r["sorted_ids"][:T].tolist() == list(range(T))
+
+
+def test_align_rejects_bad_ids():
+    with pytest.raises(ValueError):
+        oracle.align(np.array([[0, 5]], np.int32), 4, 4)
+
+
+# -------------------------------------------------------------- FFN math
+
+def _perm_matrix(perm):
+    n = len(perm)
+    m = np.zeros((n, n), np.float32)
+    m[np.arange(n), perm] = 1.0     # (M v)[i] = v[perm[i]]
+    return m
+
+
+def test_swiglu_closed_form_on_permutation_weights():
+    # W1, W3, W2 permutation matrices: g_i = x[s1(i)], u_i = x[s3(i)],
+    # y_h = a[s2(h)] = silu(x[s1(s2(h))]) * x[s3(s2(h))], silu(v) = v/(1+e^-v).
+    # A transposed W2 (s2^-1), a swapped gate/up or a dropped term fails.
+    H = 7
+    rng = np.random.default_rng(0)
+    s1, s2, s3 = (rng.permutation(H) for _ in range(3))
+    assert not np.array_equal(s2, np.argsort(s2))
+    x = np.array([0.0, math.log(3.0), -1.5, 2.0, 0.25, -0.5, 3.0], np.float32)
+    w13 = np.concatenate([_perm_matrix(s1), _perm_matrix(s3)], 0)
+    w2 = _perm_matrix(s2)
+    y = oracle.swiglu_ffn(x, w13, w2)
+    xd = x.astype(np.float64)
+    for h in range(H):
+        v = xd[s1[s2[h]]]
+        u = xd[s3[s2[h]]]
+        assert y[h] == pytest.approx(v / (1.0 + math.exp(-v)) * u, rel=1e-14, abs=1e-15)
+
+
+def test_swiglu_known_sigmoid_value():
+    # sigmoid(ln 3) = 3/4: with H = I = 1 and unit weights, y = ln3 * 3/4 * ln3
+    x = np.array([math.log(3.0)], np.float32)
+    w13 = np.array([[1.0], [1.0]], np.float32)
+    w2 = np.array([[1.0]], np.float32)
+    l3 = float(np.float32(math.log(3.0)))
+    assert oracle.swiglu_ffn(x, w13, w2)[0] == pytest.approx(l3 * l3 / (1 + math.exp(-l3)), rel=1e-14)
+    assert oracle.swiglu_ffn(x, np.array([[0.0], [1.0]], np.float32), w2)[0] == 0.0
+
+
+def test_swiglu_invariants():
+    rng = np.random.default_rng(1)
+    H, I = 24, 40
+    x = rng.standard_normal(H).astype(np.float32)
+    w13 = rng.standard_normal((2 * I, H)).astype(np.float32)
+    w2 = rng.standard_normal((H, I)).astype(np.float32)
+    y = oracle.swiglu_ffn(x, w13, w2)
+    # linear in W2 and in W3 (exact power-of-two scaling)
+    assert np.allclose(oracle.swiglu_ffn(x, w13, 2 * w2), 2 * y, rtol=1e-13)
+    w13u = w13.copy()
+    w13u[I:] *= 4
+    assert np.allclose(oracle.swiglu_ffn(x, w13u, w2), 4 * y, rtol=1e-13)
+    # permuting the intermediate dimension consistently changes nothing
+    p = rng.permutation(I)
+    w13p = np.concatenate([w13[:I][p], w13[I:][p]], 0)
+    assert np.allclose(oracle.swiglu_ffn(x, w13p, np.ascontiguousarray(w2[:, p])), y, rtol=1e-12)
+    # additive over a split of the intermediate dimension (shared-expert concatenation)
+    J = 15
+    ya = oracle.swiglu_ffn(x, np.concatenate([w13[:J], w13[I:I + J]]), np.ascontiguousarray(w2[:, :J]))
+    yb = oracle.swiglu_ffn(x, np.concatenate([w13[J:I], w13[I + J:]]), np.ascontiguousarray(w2[:, J:]))
+    assert np.allclose(ya + yb, y, rtol=1e-12, atol=1e-12)
+    # gate/up are not interchangeable
+    w13s = np.concatenate([w13[I:], w13[:I]])
+    assert not np.allclose(oracle.swiglu_ffn(x, w13s, w2), y)
+
+
+def test_dense_ffn_equals_per_token_expert_ffn():
+    rng = np.random.default_rng(2)
+    T, H, I = 9, 32, 48
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w13 = (rng.standard_normal((2 * I, H)) / np.sqrt(H)).astype(np.float32)
+    w2 = (rng.standard_normal((H, I)) / np.sqrt(I)).astype(np.float32)
+    out = oracle.dense_ffn(x, w13, w2, nthreads=2)
+    for t in range(T):
+        assert np.allclose(out[t], oracle.swiglu_ffn(x[t], w13, w2), rtol=1e-13, atol=1e-14)
+
+
+def test_bf16_inputs_are_widened_exactly():
+    rng = np.random.default_rng(3)
+    x32 = rng.standard_normal((3, 16)).astype(np.float32)
+    w32 = rng.standard_normal((5, 16)).astype(np.float32)
+    xb = torch.from_numpy(x32).to(torch.bfloat16)
+    wb = torch.from_numpy(w32).to(torch.bfloat16)
+    lb = oracle.router_logits(mi.to_oracle(xb), mi.to_oracle(wb))
+    lf = oracle.router_logits(xb.float().numpy(), wb.float().numpy())
+    assert np.array_equal(lb, lf)
+
+
+def test_router_logits_on_unit_vectors():
+    rng = np.random.default_rng(6)
+    E, H = 5, 11
+    w = rng.standard_normal((E, H)).astype(np.float32)
+    x = np.eye(H, dtype=np.float32)
+    assert np.array_equal(oracle.router_logits(x, w), w.T.astype(np.float64))
+
+
+# ------------------------------------------------------------- the layer
+
+def _small_layer(seed, T=12, H=32, E=6, K=2, I=40, I_sh=0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w_r = (rng.standard_normal((E, H)) / np.sqrt(H)).astype(np.float32)
+    w13 = (rng.standard_normal((E, 2 * I, H)) / np.sqrt(H)).astype(np.float32)
+    w2 = (rng.standard_normal((E, H, I)) / np.sqrt(I)).astype(np.float32)
+    sh = {}
+    if I_sh:
+        sh = dict(w13_sh=(rng.standard_normal((2 * I_sh, H)) / np.sqrt(H)).astype(np.float32),
+                  w2_sh=(rng.standard_normal((H, I_sh)) / np.sqrt(I_sh)).astype(np.float32))
+    return x, w_r, w13, w2, sh
+
+
+@pytest.mark.parametrize("score_fn", [0, 1])
+def test_layer_E1_K1_is_dense_ffn(score_fn):
+    x, w_r, w13, w2, _ = _small_layer(0, E=1)
+    out = oracle.moe_layer(x, w_r, w13, w2, K=1, score_fn=score_fn, renorm=1)
+    assert np.allclose(out, oracle.dense_ffn(x, w13[0], w2[0]), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("score_fn", [0, 1])
+def test_layer_identical_experts_is_dense_ffn(score_fn):
+    x, w_r, w13, w2, _ = _small_layer(1, E=5, K=3)
+    w13[:] = w13[0]
+    w2[:] = w2[0]
+    out = oracle.moe_layer(x, w_r, w13, w2, K=3, score_fn=score_fn, renorm=1)
+    assert np.allclose(out, oracle.dense_ffn(x, w13[0], w2[0]), rtol=1e-12, atol=1e-13)
+
+
+def test_layer_is_per_token_concatenated_dense_ffn():
+    # out[t] = one dense FFN whose W1/W3 concatenate the selected experts (and
+    # the shared FFN) along I and whose W2 columns are scaled by the gate
+    # weights: DenseFA's shape with per-token weights.  The scaled W2 is
+    # rounded to fp32, hence the 1e-6 tolerance.
+    x, w_r, w13, w2, sh = _small_layer(2, E=6, K=3, I_sh=24)
+    I = w2.shape[2]
+    out, ids, w = oracle.moe_layer(x, w_r, w13, w2, K=3, score_fn=0, renorm=1, return_routing=True, **sh)
+    for t in range(x.shape[0]):
+        g = np.concatenate([w13[e][:I] for e in ids[t]] + [sh["w13_sh"][:24]])
+        u = np.concatenate([w13[e][I:] for e in ids[t]] + [sh["w13_sh"][24:]])
+        d = np.concatenate([(w2[e].astype(np.float64) * w[t, k]).astype(np.float32)
+                            for k, e in enumerate(ids[t])] + [sh["w2_sh"]], 1)
+        ref = oracle.dense_ffn(x[t:t + 1], np.concatenate([g, u]), np.ascontiguousarray(d))[0]
+        assert np.allclose(out[t], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+def test_layer_all_experts_then_mask():
+    # brute force: evaluate every expert for every token, weight by a mask
+    # that keeps only the brute-force top-K subset
+    x, w_r, w13, w2, _ = _small_layer(3, T=8, E=6, K=2)
+    logits = oracle.router_logits(x, w_r).astype(np.float32)
+    out = oracle.moe_layer(x, w_r, w13, w2, K=2, score_fn=0, renorm=1)
+    for t in range(8):
+        sel = brute_topk(logits[t], 2)
+        l = logits[t].astype(np.float64)
+        den = sum(math.exp(l[e] - l[sel[0]]) for e in sel)
+        ref = np.zeros(x.shape[1])
+        for e in range(6):
+            mask = math.exp(l[e] - l[sel[0]]) / den if e in sel else 0.0
+            ref += mask * oracle.swiglu_ffn(x[t], w13[e], w2[e])
+        assert np.allclose(out[t], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_layer_linear_in_w2_and_token_permutation():
+    x, w_r, w13, w2, sh = _small_layer(4, T=10, E=4, K=2, I_sh=16)
+    out = oracle.moe_layer(x, w_r, w13, w2, K=2, **sh)
+    routed_only = out - oracle.dense_ffn(x, sh["w13_sh"], sh["w2_sh"])
+    out2 = oracle.moe_layer(x, w_r, w13, 2 * w2, K=2, **sh)
+    assert np.allclose(out2 - oracle.dense_ffn(x, sh["w13_sh"], sh["w2_sh"]), 2 * routed_only,
+                       rtol=1e-12, atol=1e-12)
+    p = np.random.default_rng(0).permutation(10)
+    outp = oracle.moe_layer(np.ascontiguousarray(x[p]), w_r, w13, w2, K=2, **sh)
+    assert np.allclose(outp, out[p], rtol=1e-14, atol=1e-15)
+
+
+def test_layer_token_subset_and_supplied_logits():
+    x, w_r, w13, w2, _ = _small_layer(5, T=16, E=8, K=2)
+    full = oracle.moe_layer(x, w_r, w13, w2, K=2)
+    sub = np.array([15, 0, 7], np.int32)
+    assert np.array_equal(oracle.moe_layer(x, w_r, w13, w2, K=2, tokens=sub), full[sub])
+    lg = oracle.router_logits(x, w_r).astype(np.float32)
+    assert np.array_equal(oracle.moe_layer(x, None, w13, w2, K=2, logits=lg), full)
+
+
+# -------------------------------------------------------------- generator
+
+def test_uniform_gumbel_routing_matches_expected_active():
+    # s = 0: each token draws K distinct experts uniformly, so the number of
+    # experts receiving at least one of m tokens has mean E(1-(1-K/E)^m).
+    for E, K, m in [(8, 2, 1), (8, 2, 4), (64, 8, 8), (256, 8, 32)]:
+        vals = []
+        for seed in range(200):
+            lg = mi.zipf_gumbel_logits(E, m, 0.0, seed=seed).numpy()
+            vals.append(len(np.unique(oracle.topk(lg, K))))
+        mean = float(np.mean(vals))
+        sem = float(np.std(vals)) / math.sqrt(len(vals)) + 1e-9
+        assert abs(mean - oracle.expected_active(E, K, m)) < 3 * sem + 1e-9, (E, K, m, mean)
+
+
+def test_zipf_skew_reduces_active_experts():
+    E, K, m = 256, 8, 32
+    means = []
+    for s in (0.0, 0.5, 1.0, 1.5):
+        means.append(np.mean([len(np.unique(oracle.topk(mi.zipf_gumbel_logits(E, m, s, seed=q).numpy(), K)))
+                              for q in range(20)]))
+    assert all(a > b for a, b in zip(means, means[1:])), means
+
+
+def test_router_generator_is_near_uniform():
+    shape = mi.SHAPES["mixtral"]
+    w = mi.make_weights(shape, seed=1, experts=False)
+    x = mi.make_x(shape, 256, seed=2)
+    lg = oracle.router_logits(mi.to_oracle(x), mi.to_oracle(w["w_r"])).astype(np.float32)
+    counts = np.bincount(oracle.topk(lg, shape.K).ravel(), minlength=shape.E)
+    expect = 256 * shape.K / shape.E
+    assert np.all(np.abs(counts - expect) < 5 * math.sqrt(expect)), counts
