@@ -1,0 +1,552 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoE layer forward (one step = one forward of the whole
+layer: router GEMM, top-K gating, alignment + padding, permute, grouped
+gate/up + SwiGLU, grouped down, shared FFN, combine) on synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral:2048]
+                    [--impl ours|reference] [--sweep]
+
+One JSON line on rank 0.  `value` is whole-job tokens/s with inputs resident in
+HBM (device time from CUDA events, L2 flushed between steps, max over ranks);
+`e2e` is the same through the C-ABI with the input copied from pinned host
+memory and the output read back inside the timed region.  Also reported: the
+roofline of the dominant kernel (grouped gate/up), the per-stage breakdown, the
+tax tau against the same library's DenseFA and DensePA FFNs, the clocks seen
+during the timed region, and the CPU oracle timed on a bounded token sample.
+Multi-GPU runs are data-parallel replicas (each rank runs its own batch on its
+own full copy of the weights; no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moe_inputs as mi  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HBM_NOMINAL_GBS = 8000.0
+METRIC = "MoE layer tokens/s; % HBM BW (decode) / % tensor peak (prefill); tau vs DenseFA"
+# DRAM bytes per launch of the dominant kernel from ncu (dram__bytes_read.sum + dram__bytes_write.sum);
+# None until a capture of the current kernel exists.
+NCU_TRAFFIC = {}
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU through NVML (read only)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id if hasattr(
+                torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
+            if bus:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            else:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- workload
+
+def parse_workload(s):
+    name, T = s.split(":")
+    return mi.SHAPES[name], int(T)
+
+
+class Workload:
+    def __init__(self, shape, T, rank=0, device="cuda", skew=None):
+        import mixture_experts_layer_61_b200 as moe
+        self.moe = moe
+        self.shape, self.T = shape, T
+        seed = mi.seed_for(shape, T)
+        self.w = mi.make_weights(shape, seed, device=device)
+        self.x = mi.make_x(shape, T, seed + 100 * rank, device=device)
+        self.logits = None
+        if skew is not None:
+            self.logits = mi.zipf_gumbel_logits(shape.E, T, skew, seed=seed + 17 + 100 * rank, device=device)
+        n_sh, I_s = (1, shape.I_sh) if shape.I_sh else (0, 0)
+        self.cfg = moe.config(T, shape.H, shape.E, shape.K, shape.I, n_shared=n_sh, I_shared=I_s,
+                              tile_B=shape.tile_B, score_fn=shape.score_fn, renorm=shape.renorm,
+                              dtype=moe.BF16 if shape.dtype == "bf16" else moe.FP32)
+        self.ws = moe.alloc_workspace(moe.workspace_size(self.cfg), device)
+        self.stats = torch.zeros(4, dtype=torch.int32, device=device)
+        self.out = torch.empty((T, shape.H), dtype=shape.torch_dtype, device=device)
+        Pm = moe.padded_rows_max(self.cfg)
+        self.Pm = Pm
+        dt = shape.torch_dtype
+        # buffers of the staged run (the same kernels, one ABI call per stage)
+        self.gws = moe.alloc_workspace(moe.gemm_workspace_size(), device)
+        self.s_logits = torch.empty((T, shape.E), dtype=torch.float32, device=device)
+        self.s_ids = torch.empty((T, shape.K), dtype=torch.int32, device=device)
+        self.s_w = torch.empty((T, shape.K), dtype=torch.float32, device=device)
+        self.s_xp = torch.empty((Pm, shape.H), dtype=dt, device=device)
+        self.s_act = torch.empty((Pm, shape.I), dtype=dt, device=device)
+        self.s_y = torch.empty((Pm, shape.H), dtype=dt, device=device)
+        self.s_sh = torch.empty((T, shape.H), dtype=dt, device=device) if shape.I_sh else None
+        self.s_shws = (moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, shape.I_sh, self.cfg.dtype), device)
+                       if shape.I_sh else None)
+
+    def step(self):
+        m = self.moe
+        m.layer_forward(self.cfg, self.x, self.w["w_r"], self.w["w13"], self.w["w2"], self.ws,
+                        self.w.get("w13_sh"), self.w.get("w2_sh"), self.logits, self.out, self.stats)
+
+    def staged_step(self, ev):
+        """The same kernels as step(), one ABI call per stage, events in between."""
+        m, c = self.moe, self.cfg
+        ev[0].record()
+        m.router_gemm(c, self.x, self.w["w_r"], self.gws, self.s_logits)
+        ev[1].record()
+        m.route(c, self.logits if self.logits is not None else self.s_logits, self.s_ids, self.s_w)
+        ev[2].record()
+        self.al = m.align_pad(c, self.s_ids)
+        ev[3].record()
+        m.permute(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
+        ev[4].record()
+        m.grouped_gate_up(c, self.s_xp, self.w["w13"], self.al["offsets"], self.gws, self.s_act)
+        ev[5].record()
+        m.grouped_down(c, self.s_act, self.w["w2"], self.al["offsets"], self.gws, self.s_y)
+        ev[6].record()
+        if self.s_sh is not None:
+            m.dense_ffn(self.x, self.w["w13_sh"], self.w["w2_sh"], self.s_shws, self.s_sh)
+        ev[7].record()
+        m.combine(c, self.s_y, self.al["pos"], self.s_w, self.s_sh, self.out)
+        ev[8].record()
+
+    STAGES = ("router", "topk", "align", "permute", "gate_up", "down", "shared", "combine")
+
+
+def l2_flush_buffer(device):
+    size = max(512 << 20, 4 * torch.cuda.get_device_properties(device).L2_cache_size)
+    return torch.empty(size // 4, dtype=torch.float32, device=device)
+
+
+def time_steps(fn, steps, flush, stream_sync=True):
+    """Per-step CUDA-event durations (ms), L2 flushed before each step (outside the events)."""
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return times
+
+
+# ------------------------------------------------------------ accounting
+
+def algorithmic(shape, T, E_active):
+    """Algorithmic bytes and flops of one layer forward (padding excluded):
+    bytes = weights of the activated experts + shared weights + router weights,
+    flops = 2 T (H E + K 3 H I + 3 H I_sh)."""
+    eb = 2 if shape.dtype == "bf16" else 4
+    H, I, E, K = shape.H, shape.I, shape.E, shape.K
+    B = E_active * 3 * H * I * eb + 3 * H * shape.I_sh * eb + E * H * eb
+    F = 2.0 * T * (H * E + K * 3 * H * I + 3 * H * shape.I_sh)
+    return B, F
+
+
+def gate_up_work(shape, T, E_active):
+    """Dominant kernel (grouped gate/up + SwiGLU): weight bytes of the activated
+    experts' W1/W3, flops 2 * T K * H * 2I."""
+    eb = 2 if shape.dtype == "bf16" else 4
+    return E_active * 2 * shape.I * shape.H * eb, 2.0 * T * shape.K * shape.H * 2 * shape.I
+
+
+def dense_times(shape, T, I_d, steps, warmup, flush, device, seed):
+    import mixture_experts_layer_61_b200 as moe
+    w13, w2 = mi.make_dense_weights(shape.H, I_d, shape.torch_dtype, seed=seed, device=device)
+    x = mi.make_x(shape, T, seed, device=device)
+    ws = moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, I_d, 0 if shape.dtype == "bf16" else 1), device)
+    out = torch.empty_like(x)
+    fn = lambda: moe.dense_ffn(x, w13, w2, ws, out)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    t = time_steps(fn, steps, flush)
+    moe.check_status(ws)
+    del w13, w2, ws
+    return statistics.median(t)
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_tokens_per_s(wl, budget_s=15.0, max_tokens=None):
+    """The oracle as it stands on a bounded sample of the workload's tokens,
+    all host cores, routing on the GPU path's logits (read back)."""
+    import numpy as np
+    import oracle
+    shape = wl.shape
+    nthreads = os.cpu_count() or 1
+    logits = wl.logits
+    if logits is None:
+        logits = wl.moe.router_gemm(wl.cfg, wl.x, wl.w["w_r"], wl.gws, wl.s_logits)
+    lg = logits.float().cpu().numpy()
+    xh = mi.to_oracle(wl.x)
+    w13 = mi.to_oracle(wl.w["w13"])
+    w2 = mi.to_oracle(wl.w["w2"])
+    sh = {}
+    if shape.I_sh:
+        sh = dict(w13_sh=mi.to_oracle(wl.w["w13_sh"]), w2_sh=mi.to_oracle(wl.w["w2_sh"]))
+    T = wl.T
+
+    def run(n):
+        tok = np.arange(n, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_layer(xh, None, w13, w2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok,
+                         nthreads=nthreads, **sh)
+        return time.perf_counter() - t0
+
+    n = min(T, nthreads)
+    t1 = run(n)
+    per_tok = t1 / n
+    n2 = int(max(1, min(T if max_tokens is None else max_tokens, budget_s / max(per_tok, 1e-9))))
+    n2 = max(n2 - n2 % nthreads, min(T, nthreads)) if n2 >= nthreads else n2
+    t2 = run(n2)
+    return {"value": n2 / t2, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"first {n2} of the {T} tokens of the workload (all {nthreads} host threads, "
+                      f"{t2:.1f} s), routing on the GPU path's fp32 logits"}
+
+
+# ------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="mixtral:2048")
+    ap.add_argument("--skew", type=float, default=None, help="Zipf exponent of Gumbel router logits")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tau", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="also time every configured workload")
+    ap.add_argument("--sweep-out", default=None)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    shape, T = parse_workload(args.workload)
+
+    if args.impl == "reference":
+        return reference_arm(args, shape, T, rank, world, local, dist)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pk, pk_kind = peaks()
+    wl = Workload(shape, T, rank, device, skew=args.skew)
+    flush = l2_flush_buffer(device)
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    wl.moe.check_status(wl.ws)
+
+    # ---- timed region: K steps of the fused layer call
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = wl.moe.kernel_launch_count()
+    with ClockSampler(local) as clk:
+        times = time_steps(wl.step, args.steps, flush)
+    torch.cuda.synchronize()
+    launches = wl.moe.kernel_launch_count() - n0
+    if dist:
+        dist.barrier()
+    total_ms = sum(times)
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    wl.moe.check_status(wl.ws)
+    stats = wl.stats.cpu().tolist()
+    P, E_active = stats[0], stats[1]
+    ms_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # ---- per-stage breakdown (same kernels, one ABI call per stage)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+    stage_ms = {s: [] for s in Workload.STAGES}
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        wl.staged_step(ev)
+        ev[8].synchronize()
+        if i >= args.warmup:
+            for j, s in enumerate(Workload.STAGES):
+                stage_ms[s].append(ev[j].elapsed_time(ev[j + 1]))
+    wl.moe.check_status(wl.gws)
+    stages = {s: round(statistics.median(v), 4) for s, v in stage_ms.items()}
+
+    # ---- roofline of the dominant kernel (grouped gate/up + SwiGLU)
+    gu_bytes, gu_flops = gate_up_work(shape, T, E_active)
+    t_gu = stages["gate_up"] * 1e-3
+    hbm_peak = pk["hbm_gbs"]
+    tc_peak = pk["bf16_tflops"] * (0.5 if shape.dtype == "fp32" else 1.0)  # tf32 is half the bf16 rate
+    bound = "tensor" if gu_flops / (tc_peak * 1e12) > gu_bytes / (hbm_peak * 1e9) else "hbm"
+    if bound == "hbm":
+        ach = gu_bytes / t_gu / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(ach / hbm_peak, 4), "frac_of_8TBs": round(ach / HBM_NOMINAL_GBS, 4)}
+    else:
+        ach = gu_flops / t_gu / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": round(ach / tc_peak, 4), "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4)}
+    roof["kernel"] = "moe_gemm_kernel (grouped gate/up + SwiGLU)"
+    roof["peak_source"] = f"{pk_kind} ({'MEASURED_PEAKS.json' if pk_kind == 'measured' else 'fallback'})"
+    roof["traffic"] = NCU_TRAFFIC.get(f"{shape.name}:{T}")
+    B_alg, F_alg = algorithmic(shape, T, E_active)
+    t_layer = ms_step * 1e-3
+    layer_roof = max(F_alg / (tc_peak * 1e12), B_alg / (hbm_peak * 1e9)) / t_layer
+
+    # ---- e2e through the C-ABI with host buffers
+    x_host = torch.empty(wl.x.shape, dtype=wl.x.dtype, pin_memory=True)
+    x_host.copy_(wl.x)
+    out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
+
+    def e2e_step():
+        wl.x.copy_(x_host, non_blocking=True)
+        wl.step()
+        out_host.copy_(wl.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e2e_times = time_steps(e2e_step, args.steps, flush)
+    e2e_total = sum(e2e_times)
+    if dist:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e = {"value": world * T * args.steps / (e2e_total / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+           "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+
+    # ---- tau against DenseFA / DensePA (same library, same T)
+    tau = None
+    if not args.no_tau:
+        seed = mi.seed_for(shape, T, 50)
+        t_fa = dense_times(shape, T, shape.I_FA, args.steps, args.warmup, flush, device, seed)
+        t_pa = dense_times(shape, T, shape.I_PA, args.steps, args.warmup, flush, device, seed + 1)
+        t_moe = statistics.median(times)
+        tau = {"tau_FA": round(t_moe / t_fa, 4), "tau_PA": round(t_moe / t_pa, 4),
+               "t_moe_ms": round(t_moe, 4), "t_DenseFA_ms": round(t_fa, 4), "t_DensePA_ms": round(t_pa, 4),
+               "I_FA": shape.I_FA, "I_PA": shape.I_PA}
+
+    sweep = None
+    if args.sweep:
+        sweep = run_sweep(args, device, flush, pk)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_tokens_per_s(wl)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if shape.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded Gaussian weights/activations of the layer's shape; "
+                + ("router logits x.W_r" if args.skew is None else f"Zipf({args.skew}) Gumbel logits") + ")",
+        "config": {"workload": f"{shape.name}-shaped MoE layer forward, T={T}", "T": T, "H": shape.H,
+                   "E": shape.E, "K": shape.K, "I": shape.I, "I_shared": shape.I_sh, "tile_B": shape.tile_B,
+                   "score_fn": "softmax" if shape.score_fn == 0 else "sigmoid", "global_batch": T * world,
+                   "parallelism": f"replicas x{world} (data parallel, no collective)",
+                   "l2": "flushed between steps (512 MiB write outside the events); weights exceed L2"},
+        "roofline": roof,
+        "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - T * shape.K) / max(P, 1), 4),
+                  "bytes_alg": B_alg, "flops_alg": F_alg, "roofline_frac": round(layer_roof, 4),
+                  "hbm_GBs_alg": round(B_alg / t_layer / 1e9, 1), "tflops_alg": round(F_alg / t_layer / 1e12, 2)},
+        "stages_ms": stages,
+        "staged_total_ms": round(sum(stages.values()), 4),
+        "tau": tau,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    if sweep is not None:
+        line["sweep"] = sweep
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_sweep(args, device, flush, pk):
+    """Every configured workload (decode and prefill T of each layer shape, and
+    the DeepSeek-V3 routing-skew sweep): tokens/s, roofline fractions and tau."""
+    import mixture_experts_layer_61_b200 as moe
+    rows = []
+    plan = []
+    for name in ("mixtral", "qwen2moe", "deepseekv3"):
+        sh = mi.SHAPES[name]
+        for T in sh.decode_T + sh.prefill_T:
+            plan.append((sh, T, None))
+    for s in (0.0, 0.5, 1.0, 1.5):
+        for T in (1, 8, 64, 512, 4096):
+            plan.append((mi.SHAPES["deepseekv3"], T, s))
+    steps = max(5, args.steps // 2)
+    fa_cache = {}
+    for sh, T, s in plan:
+        wl = Workload(sh, T, 0, device, skew=s)
+        for _ in range(3):
+            wl.step()
+        torch.cuda.synchronize()
+        t = statistics.median(time_steps(wl.step, steps, flush))
+        moe.check_status(wl.ws)
+        st = wl.stats.cpu().tolist()
+        B, F = algorithmic(sh, T, st[1])
+        key = (sh.name, T)
+        if key not in fa_cache:
+            fa_cache[key] = dense_times(sh, T, sh.I_FA, steps, 3, flush, device, mi.seed_for(sh, T, 50))
+        row = {"layer": sh.name, "T": T, "skew": s, "ms": round(t, 4), "tokens_per_s": round(T / t * 1e3, 1),
+               "E_active": st[1], "P": st[0], "padded_fraction": round((st[0] - T * sh.K) / max(st[0], 1), 4),
+               "hbm_frac_8TBs": round(B / (t * 1e-3) / 8e12, 4),
+               "hbm_frac_measured": round(B / (t * 1e-3) / (pk["hbm_gbs"] * 1e9), 4),
+               "tensor_frac": round(F / (t * 1e-3) / (pk["bf16_tflops"] * 1e12), 4),
+               "tau_FA": round(t / fa_cache[key], 4)}
+        rows.append(row)
+        del wl
+        torch.cuda.empty_cache()
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            for r in rows:
+                f.write(json.dumps(r) + "\n")
+    return rows
+
+
+def reference_arm(args, shape, T, rank, world, local, dist):
+    """The CPU oracle as the reference implementation, on rank 0 only: each step
+    runs the oracle over a bounded sample of the workload's tokens."""
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return
+    import numpy as np
+    import oracle
+    seed = mi.seed_for(shape, T)
+    w = mi.make_weights(shape, seed, device="cuda" if torch.cuda.is_available() else "cpu")
+    x = mi.make_x(shape, T, seed, device=w["w_r"].device)
+    xh, wr = mi.to_oracle(x), mi.to_oracle(w["w_r"])
+    w13, w2 = mi.to_oracle(w["w13"]), mi.to_oracle(w["w2"])
+    sh = {}
+    if shape.I_sh:
+        sh = dict(w13_sh=mi.to_oracle(w["w13_sh"]), w2_sh=mi.to_oracle(w["w2_sh"]))
+    nthreads = os.cpu_count() or 1
+    # size the per-step sample so that warmup + steps stay within ~2 minutes
+    t0 = time.perf_counter()
+    oracle.moe_layer(xh, wr, w13, w2, shape.K, shape.score_fn, shape.renorm,
+                     tokens=np.arange(min(T, nthreads), dtype=np.int32), nthreads=nthreads, **sh)
+    per_tok = (time.perf_counter() - t0) / min(T, nthreads)
+    n = int(max(1, min(T, 120.0 / (args.steps + args.warmup) / per_tok)))
+    tok = np.arange(n, dtype=np.int32)
+    for _ in range(args.warmup):
+        oracle.moe_layer(xh, wr, w13, w2, shape.K, shape.score_fn, shape.renorm, tokens=tok, nthreads=nthreads, **sh)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.moe_layer(xh, wr, w13, w2, shape.K, shape.score_fn, shape.renorm, tokens=tok, nthreads=nthreads, **sh)
+        ts.append(time.perf_counter() - t0)
+    total = sum(ts)
+    value = n * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{shape.name}-shaped MoE layer forward, T={T}", "T": T, "H": shape.H,
+                       "E": shape.E, "K": shape.K, "I": shape.I, "I_shared": shape.I_sh},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                             "sample": f"first {n} of the {T} tokens per step, router GEMM included"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

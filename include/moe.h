@@ -1,0 +1,210 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the single-GPU forward of one
+ * Mixture-of-Experts FFN layer on NVIDIA B200 (sm_100a), and the dense SwiGLU
+ * FFN used as its FLOP-aligned (DenseFA) and parameter-aligned (DensePA)
+ * baselines.
+ *
+ * The operations follow the pages on "Demystifying the Mixture of Experts
+ * Serving Tax" (MLSys 2026):
+ *   - talk notes, "Key findings 5": the MoE block runs a router, top-K
+ *     selection, alignment, a grouped GEMM (GroupGEMM) and a local sum
+ *     (combine);
+ *   - talk notes, "Padding model (Section 5.1)": block-wise padding, each
+ *     expert's token count N_i rounded up to the block size B,
+ *     P = sum_i ceil(N_i / B) * B padded rows;
+ *   - talk notes, "Definition": tax tau = T(MoE, b) / T(DenseFA, b) (Eq. 1);
+ *     DenseFA = the MoE layer replaced by an FFN whose intermediate size is
+ *     scaled by K (same FLOPs per token); DensePA = a dense FFN with the MoE
+ *     layer's total parameters;
+ *   - talk notes, Table 2: shared experts (always-on FFNs).
+ *
+ * Symbols: T tokens, H hidden size, E routed experts, K experts per token,
+ * I expert intermediate size, S shared experts of width I_s (one dense FFN
+ * of width S * I_s), B padding tile, A = T * K assignments, a = t * K + k.
+ *
+ * Conventions (every entry point):
+ *   - Every pointer is a DEVICE pointer unless stated; all arrays are
+ *     row-major and contiguous.  The caller owns all memory: the library
+ *     never allocates or frees device memory.
+ *   - Work is enqueued on `stream`; no call synchronises the stream except
+ *     moe_check_status().  A return of MOE_OK means "enqueued".
+ *   - Activations and weights are bf16 (dtype 0) or fp32 (dtype 1); router
+ *     logits and gate weights are always fp32; indices are int32.
+ *   - Weights are laid out like nn.Linear ([out, in]):
+ *       w_router [E, H];
+ *       w13 [E, 2I, H]: rows 0..I-1 the gate projection W1, rows I..2I-1 the
+ *         up projection W3;   w2 [E, H, I];
+ *       shared / dense FFN: w13 [2*I_d, H], w2 [H, I_d].
+ *   - Row strides must be multiples of 16 bytes: H and I multiples of 8
+ *     (bf16) or 4 (fp32).  Device pointers must be 16-byte aligned.
+ *   - Errors are returned, never thrown; no CUDA error is left pending.
+ *   - T = 0 is a valid no-op (pointers may then be NULL), except that
+ *     moe_align_pad still writes zero counts, offsets and scalars.
+ *   - The device must be sm_100 (B200); other devices get MOE_ERR_DEVICE.
+ *   - Kernel waits are bounded: a wait that exceeds the limit sets a status
+ *     word in the workspace and the kernel returns; moe_check_status()
+ *     reports it as MOE_ERR_TIMEOUT.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (the same type as cudaStream_t / CUstream). */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = -1,        /* NULL pointer, bad size or unsupported option */
+    MOE_ERR_WORKSPACE = -2,  /* workspace smaller than the *_workspace_size() query */
+    MOE_ERR_CUDA = -3,       /* a CUDA launch or runtime call failed */
+    MOE_ERR_TIMEOUT = -4,    /* a device-side wait ran out (reported by moe_check_status) */
+    MOE_ERR_DEVICE = -5      /* current device is not sm_100 */
+} moe_status_t;
+
+typedef struct {
+    int T;          /* tokens, >= 0 */
+    int H;          /* hidden size */
+    int E;          /* routed experts, 1..1024 */
+    int K;          /* experts per token, 1..min(E, 16) */
+    int I;          /* routed expert intermediate size */
+    int n_shared;   /* shared experts S (0 = none) */
+    int I_shared;   /* intermediate size of one shared expert I_s */
+    int tile_B;     /* padding tile B, 1..256 */
+    int score_fn;   /* 0 = softmax, 1 = sigmoid */
+    int renorm;     /* 1: weights normalised over the selected K */
+    int dtype;      /* 0 = bf16, 1 = fp32 (activations and weights) */
+} moe_config_t;
+
+/* Text for a status code (static storage). */
+const char* moe_status_string(int status);
+
+/* Upper bound on padded rows: P_max = A + min(E, A) * (B - 1), A = T * K. */
+int64_t moe_padded_rows_max(const moe_config_t* cfg);
+
+/* Bytes of workspace moe_layer_forward needs for this configuration on the
+ * current device (0 on a bad configuration).  The workspace must be zeroed
+ * once before its first use (e.g. cudaMemsetAsync); the library leaves its
+ * control words zero after every call that completes without a timeout. */
+size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Bytes of workspace moe_router_gemm / moe_grouped_ffn / dense_ffn need (the
+ * control words and stream-K partial tiles only), same zeroing rule. */
+size_t moe_gemm_workspace_size(void);
+
+/* Router GEMM (stage "router"): logits[T,E] (fp32) = x[T,H] . w_router[E,H]^T,
+ * products of the inputs accumulated in fp32 on the tensor cores (fp32
+ * inputs: tf32 products).  `workspace` as returned by
+ * moe_gemm_workspace_size(). */
+int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router,
+                    float* logits, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* Top-K gating (stage "top-K selection"), one token per warp:
+ *   topk_ids[T,K]: the K largest logits[t,:], descending, the lower expert
+ *     index first on equal values (IEEE comparison: -0.0 ties +0.0; +-inf are
+ *     ordered normally; NaN logits give unspecified but in-range ids);
+ *   topk_w[T,K]: softmax (score_fn 0) or sigmoid (score_fn 1) weights,
+ *     renormalised over the selected K when cfg->renorm (softmax without
+ *     renorm: the full softmax over E, restricted to the selected experts;
+ *     sigmoid without renorm: the raw sigmoid), computed in fp32. */
+int moe_route(const moe_config_t* cfg, const float* logits, int32_t* topk_ids,
+              float* topk_w, moe_stream_t stream);
+
+/* Token-to-expert alignment with block-wise padding (stage "alignment",
+ * Section 5.1 padding model).  With e(a) = topk_ids[a]:
+ *   counts[E]        N_e = #{a : e(a) = e}
+ *   offsets[E+1]     exclusive scan of ceil(N_e / B) * B; offsets[E] = P
+ *   sorted_ids[P_max] the assignments of expert e in ascending a at
+ *                    offsets[e] .. offsets[e] + N_e - 1; every other slot -1
+ *   block_expert[ceil(P_max/B)]  e for blocks inside expert e's segment, -1 after P
+ *   pos[A]           the slot p with sorted_ids[p] = a
+ *   scalars[4]       {P, E_active = #{e : N_e > 0}, 0, 0}
+ * Bit-exact and deterministic.  Out-of-range ids are skipped and flagged in
+ * scalars[2] (nonzero = bad input). */
+int moe_align_pad(const moe_config_t* cfg, const int32_t* topk_ids, int32_t* counts,
+                  int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert,
+                  int32_t* pos, int32_t* scalars, moe_stream_t stream);
+
+/* Permute (gather): x_perm[p] = x[sorted_ids[p] / K] for p < P, a zero row
+ * where sorted_ids[p] = -1; rows >= P are left untouched.  x_perm has P_max
+ * rows of H. */
+int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids,
+                const int32_t* scalars, void* x_perm, moe_stream_t stream);
+
+/* Grouped expert FFN over the padded segments (stage "GroupGEMM"): for each
+ * expert e and each row p in [offsets[e], offsets[e+1]):
+ *   act[p]    = silu(x_perm[p] . W1_e^T) * (x_perm[p] . W3_e^T)   ([P_max, I])
+ *   y_perm[p] = act[p] . W2_e^T                                    ([P_max, H])
+ * fp32 accumulation on the tensor cores; act and y_perm are stored in the
+ * activation dtype.  `act` is caller-provided scratch of P_max * I elements. */
+int moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const void* w13,
+                    const void* w2, const int32_t* offsets, void* act, void* y_perm,
+                    void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* The two launches of moe_grouped_ffn, separately (same arguments):
+ * gate/up + SwiGLU writes act[P_max, I]; down reads act and writes
+ * y_perm[P_max, H]. */
+int moe_grouped_gate_up(const moe_config_t* cfg, const void* x_perm, const void* w13,
+                        const int32_t* offsets, void* act, void* workspace, size_t ws_bytes,
+                        moe_stream_t stream);
+int moe_grouped_down(const moe_config_t* cfg, const void* act, const void* w2,
+                     const int32_t* offsets, void* y_perm, void* workspace, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/* Weighted un-permute and combine (stage "local sum"):
+ *   out[t] = sum_{k=0..K-1} topk_w[t,k] * y_perm[pos[t*K+k]]  (+ shared_out[t])
+ * summed in fp32 in ascending k, the shared output added last, one final
+ * rounding to the activation dtype.  shared_out may be NULL. */
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* pos,
+                const float* topk_w, const void* shared_out, void* out,
+                moe_stream_t stream);
+
+/* Whole layer: router GEMM (or logits_override), top-K gating, alignment,
+ * permute, grouped gate/up + SwiGLU, grouped down, shared FFN (when
+ * n_shared > 0), combine.  out[T,H].  logits_override (nullable, fp32 [T,E])
+ * replaces the router output for the routing decision; the router GEMM still
+ * runs so its cost is kept.  stats_out (nullable, device int32[4]) receives
+ * {P, E_active, bad_ids, 0}.  Nothing is synchronised. */
+int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router,
+                      const void* w13, const void* w2, const void* w13_shared,
+                      const void* w2_shared, const float* logits_override, void* out,
+                      void* workspace, size_t ws_bytes, int32_t* stats_out,
+                      moe_stream_t stream);
+
+/* Bytes of workspace dense_ffn needs for T tokens of width I (0 if invalid). */
+size_t dense_ffn_workspace_size(int T, int H, int I, int dtype);
+
+/* Dense SwiGLU FFN (DenseFA with I = K*I + S*I_s, DensePA with
+ * I = E*I + S*I_s, or the shared experts): out[t] = W2 (silu(W1 x_t) * (W3 x_t)),
+ * w13 [2I, H], w2 [H, I], same numerics as moe_grouped_ffn. */
+int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13,
+              const void* w2, void* out, void* workspace, size_t ws_bytes,
+              moe_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the workspace status word.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT (a device wait ran out; the control words
+ * are re-zeroed so the workspace stays usable) or MOE_ERR_CUDA. */
+int moe_check_status(void* workspace, moe_stream_t stream);
+
+/* Device-side wait limit in nanoseconds for subsequent launches (default
+ * 2e9 = 2 s; 0 restores the default).  Process-wide. */
+void moe_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook: when nonzero, the next GEMM launch withholds the first operand
+ * load of block 0, so that block's waits run out and report
+ * MOE_ERR_TIMEOUT through moe_check_status().  Cleared after one launch. */
+void moe_debug_withhold_first_load(int enable);
+
+/* Number of kernels this library launched since load (all entry points). */
+uint64_t moe_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,279 @@
+"""Python binding of libmoe.so -- the B200 (sm_100a) MoE layer forward.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors; the work is enqueued on the current
+torch stream.  There is no CPU fallback: without the built library, or on a
+device other than sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+_lib = None
+
+BF16, FP32 = 0, 1
+SOFTMAX, SIGMOID = 0, 1
+STATUS = {0: "MOE_OK", -1: "MOE_ERR_ARG", -2: "MOE_ERR_WORKSPACE", -3: "MOE_ERR_CUDA",
+          -4: "MOE_ERR_TIMEOUT", -5: "MOE_ERR_DEVICE"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({_lib.moe_status_string(code).decode()})")
+
+
+class MoeConfig(ctypes.Structure):
+    """moe_config_t (include/moe.h)."""
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("T", "H", "E", "K", "I", "n_shared", "I_shared", "tile_B", "score_fn", "renorm", "dtype")]
+
+    def __repr__(self):
+        return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def config(T, H, E, K, I, n_shared=0, I_shared=0, tile_B=16, score_fn=SOFTMAX, renorm=1, dtype=BF16):
+    if isinstance(dtype, torch.dtype):
+        dtype = BF16 if dtype == torch.bfloat16 else FP32
+    return MoeConfig(T, H, E, K, I, n_shared, I_shared, tile_B, score_fn, renorm, dtype)
+
+
+def lib():
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m mixture_experts_layer_61_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        C = ctypes.POINTER(MoeConfig)
+        sig = {
+            "moe_status_string": (ctypes.c_char_p, [I]),
+            "moe_padded_rows_max": (ctypes.c_int64, [C]),
+            "moe_workspace_size": (S, [C]),
+            "moe_gemm_workspace_size": (S, []),
+            "moe_router_gemm": (I, [C, P, P, P, P, S, P]),
+            "moe_route": (I, [C, P, P, P, P]),
+            "moe_align_pad": (I, [C, P, P, P, P, P, P, P, P]),
+            "moe_permute": (I, [C, P, P, P, P, P]),
+            "moe_grouped_ffn": (I, [C, P, P, P, P, P, P, P, S, P]),
+            "moe_grouped_gate_up": (I, [C, P, P, P, P, P, S, P]),
+            "moe_grouped_down": (I, [C, P, P, P, P, P, S, P]),
+            "moe_combine": (I, [C, P, P, P, P, P, P]),
+            "moe_layer_forward": (I, [C, P, P, P, P, P, P, P, P, P, S, P, P]),
+            "dense_ffn_workspace_size": (S, [I, I, I, I]),
+            "dense_ffn": (I, [I, I, I, I, P, P, P, P, P, S, P]),
+            "moe_check_status": (I, [P, P]),
+            "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+            "moe_debug_withhold_first_load": (None, [I]),
+            "moe_kernel_launch_count": (ctypes.c_uint64, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_functions():
+    """Names of the functions include/moe.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_\w+|dense_ffn\w*)\s*\(", text)))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise MoeError(rc, what)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def _act_dtype(cfg):
+    return torch.bfloat16 if cfg.dtype == BF16 else torch.float32
+
+
+# ------------------------------------------------------------ workspaces
+
+def workspace_size(cfg):
+    n = lib().moe_workspace_size(ctypes.byref(cfg))
+    if n == 0:
+        raise MoeError(-1, "moe_workspace_size")
+    return n
+
+
+def gemm_workspace_size():
+    return lib().moe_gemm_workspace_size()
+
+
+def dense_workspace_size(T, H, I, dtype=BF16):
+    return lib().dense_ffn_workspace_size(T, H, I, dtype)
+
+
+def alloc_workspace(nbytes, device="cuda"):
+    """A zeroed workspace (the library keeps its control words zero after each call)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def padded_rows_max(cfg):
+    return int(lib().moe_padded_rows_max(ctypes.byref(cfg)))
+
+
+# ------------------------------------------------------------- the steps
+
+def router_gemm(cfg, x, w_r, ws, logits=None):
+    _need_cuda(x, w_r, ws)
+    if logits is None:
+        logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=x.device)
+    _check(lib().moe_router_gemm(ctypes.byref(cfg), _p(x), _p(w_r), _p(logits), _p(ws), ws.numel(), _stream()),
+           "moe_router_gemm")
+    return logits
+
+
+def route(cfg, logits, ids=None, w=None):
+    _need_cuda(logits)
+    if ids is None:
+        ids = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device=logits.device)
+        w = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device=logits.device)
+    _check(lib().moe_route(ctypes.byref(cfg), _p(logits), _p(ids), _p(w), _stream()), "moe_route")
+    return ids, w
+
+
+def align_pad(cfg, ids):
+    _need_cuda(ids)
+    dev = ids.device
+    Pm = padded_rows_max(cfg)
+    nblk = (Pm + cfg.tile_B - 1) // cfg.tile_B
+    out = dict(counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
+               sorted_ids=torch.empty(max(Pm, 1), dtype=torch.int32, device=dev),
+               block_expert=torch.empty(max(nblk, 1), dtype=torch.int32, device=dev),
+               pos=torch.empty(max(cfg.T * cfg.K, 1), dtype=torch.int32, device=dev),
+               scalars=torch.zeros(4, dtype=torch.int32, device=dev))
+    _check(lib().moe_align_pad(ctypes.byref(cfg), _p(ids), _p(out["counts"]), _p(out["offsets"]),
+                               _p(out["sorted_ids"]), _p(out["block_expert"]), _p(out["pos"]),
+                               _p(out["scalars"]), _stream()), "moe_align_pad")
+    out["sorted_ids"] = out["sorted_ids"][:Pm]
+    out["block_expert"] = out["block_expert"][:nblk]
+    out["pos"] = out["pos"][:cfg.T * cfg.K]
+    return out
+
+
+def permute(cfg, x, sorted_ids, scalars, x_perm=None):
+    _need_cuda(x, sorted_ids, scalars)
+    if x_perm is None:
+        x_perm = torch.empty((max(padded_rows_max(cfg), 1), cfg.H), dtype=x.dtype, device=x.device)
+    _check(lib().moe_permute(ctypes.byref(cfg), _p(x), _p(sorted_ids), _p(scalars), _p(x_perm), _stream()),
+           "moe_permute")
+    return x_perm
+
+
+def grouped_ffn(cfg, x_perm, w13, w2, offsets, ws, act=None, y_perm=None):
+    _need_cuda(x_perm, w13, w2, offsets, ws)
+    Pm = max(padded_rows_max(cfg), 1)
+    if act is None:
+        act = torch.empty((Pm, cfg.I), dtype=x_perm.dtype, device=x_perm.device)
+    if y_perm is None:
+        y_perm = torch.empty((Pm, cfg.H), dtype=x_perm.dtype, device=x_perm.device)
+    _check(lib().moe_grouped_ffn(ctypes.byref(cfg), _p(x_perm), _p(w13), _p(w2), _p(offsets), _p(act), _p(y_perm),
+                                 _p(ws), ws.numel(), _stream()), "moe_grouped_ffn")
+    return y_perm, act
+
+
+def grouped_gate_up(cfg, x_perm, w13, offsets, ws, act):
+    _need_cuda(x_perm, w13, offsets, ws, act)
+    _check(lib().moe_grouped_gate_up(ctypes.byref(cfg), _p(x_perm), _p(w13), _p(offsets), _p(act), _p(ws),
+                                     ws.numel(), _stream()), "moe_grouped_gate_up")
+    return act
+
+
+def grouped_down(cfg, act, w2, offsets, ws, y_perm):
+    _need_cuda(act, w2, offsets, ws, y_perm)
+    _check(lib().moe_grouped_down(ctypes.byref(cfg), _p(act), _p(w2), _p(offsets), _p(y_perm), _p(ws),
+                                  ws.numel(), _stream()), "moe_grouped_down")
+    return y_perm
+
+
+def combine(cfg, y_perm, pos, w, shared_out=None, out=None):
+    _need_cuda(y_perm, pos, w, shared_out)
+    if out is None:
+        out = torch.empty((cfg.T, cfg.H), dtype=y_perm.dtype, device=y_perm.device)
+    _check(lib().moe_combine(ctypes.byref(cfg), _p(y_perm), _p(pos), _p(w), _p(shared_out), _p(out), _stream()),
+           "moe_combine")
+    return out
+
+
+def layer_forward(cfg, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, logits_override=None, out=None,
+                  stats=None):
+    _need_cuda(x, w_r, w13, w2, ws, w13_sh, w2_sh, logits_override, stats)
+    if out is None:
+        out = torch.empty((cfg.T, cfg.H), dtype=x.dtype, device=x.device)
+    _check(lib().moe_layer_forward(ctypes.byref(cfg), _p(x), _p(w_r), _p(w13), _p(w2), _p(w13_sh), _p(w2_sh),
+                                   _p(logits_override), _p(out), _p(ws), ws.numel(), _p(stats), _stream()),
+           "moe_layer_forward")
+    return out
+
+
+def dense_ffn(x, w13, w2, ws, out=None):
+    _need_cuda(x, w13, w2, ws)
+    T, H = x.shape
+    I = w2.shape[1]
+    dt = BF16 if x.dtype == torch.bfloat16 else FP32
+    if out is None:
+        out = torch.empty((T, H), dtype=x.dtype, device=x.device)
+    _check(lib().dense_ffn(T, H, I, dt, _p(x), _p(w13), _p(w2), _p(out), _p(ws), ws.numel(), _stream()),
+           "dense_ffn")
+    return out
+
+
+def check_status(ws):
+    """Synchronise the current stream; raise MoeError if a device wait timed out."""
+    _check(lib().moe_check_status(_p(ws), _stream()), "moe_check_status")
+
+
+def set_wait_limit_ns(ns):
+    lib().moe_set_wait_limit_ns(int(ns))
+
+
+def debug_withhold_first_load(enable=True):
+    lib().moe_debug_withhold_first_load(1 if enable else 0)
+
+
+def kernel_launch_count():
+    return int(lib().moe_kernel_launch_count())
+
+
+class MoELayer:
+    """Owns a configuration and its workspace; forward() runs the whole layer."""
+
+    def __init__(self, cfg, weights, device="cuda"):
+        self.cfg = cfg
+        self.w = weights
+        self.ws = alloc_workspace(workspace_size(cfg), device)
+        self.stats = torch.zeros(4, dtype=torch.int32, device=device)
+
+    def forward(self, x, logits_override=None, out=None):
+        return layer_forward(self.cfg, x, self.w["w_r"], self.w["w13"], self.w["w2"], self.ws,
+                             self.w.get("w13_sh"), self.w.get("w2_sh"), logits_override, out, self.stats)

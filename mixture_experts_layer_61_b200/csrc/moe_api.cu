@@ -1,0 +1,477 @@
+// moe_api.cu -- the extern "C" entry points of libmoe.so (declared in
+// include/moe.h): argument checks, workspace layout and the launch sequence of
+// the MoE layer forward.  Every compute step runs in the kernels of
+// moe_kernels.cu and moe_gemm.cu; nothing here touches tensor data.
+#include <atomic>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_limit{2000000000ull};
+std::atomic<int> g_withhold{0};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, -1 unsupported
+std::mutex g_dev_mu;
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+uint64_t wait_limit_ns() { return g_wait_limit.load(std::memory_order_relaxed); }
+int take_withhold_flag() { return g_withhold.exchange(0); }
+
+int current_device(DeviceInfo* info) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return -3;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return -5;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_dev_state[dev] == 0) {
+        DeviceInfo d;
+        d.device = dev;
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return -3;
+        }
+        g_dev[dev] = d;
+        g_dev_state[dev] = (d.cc_major == 10 && d.cc_minor == 0) ? 1 : -1;
+    }
+    if (g_dev_state[dev] < 0) return -5;
+    *info = g_dev[dev];
+    return 0;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int elt_bytes(int dtype) { return dtype == 0 ? 2 : (dtype == 1 ? 4 : 0); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const moe_config_t* c) {
+    if (!c) return MOE_ERR_ARG;
+    const int eb = elt_bytes(c->dtype);
+    if (eb == 0) return MOE_ERR_ARG;
+    const int vec = 16 / eb;
+    if (c->T < 0 || c->H <= 0 || c->E < 1 || c->E > 1024 || c->K < 1 || c->K > 16 || c->K > c->E || c->I <= 0)
+        return MOE_ERR_ARG;
+    if (c->n_shared < 0 || c->I_shared < 0 || (c->n_shared > 0 && c->I_shared <= 0)) return MOE_ERR_ARG;
+    if (c->tile_B < 1 || c->tile_B > 256) return MOE_ERR_ARG;
+    if (c->score_fn != 0 && c->score_fn != 1) return MOE_ERR_ARG;
+    if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_ARG;
+    if (c->H % vec != 0 || c->I % vec != 0) return MOE_ERR_ARG;
+    const long long I_sh = (long long)c->n_shared * c->I_shared;
+    if (I_sh % vec != 0 || I_sh > (1LL << 30)) return MOE_ERR_ARG;
+    const long long A = (long long)c->T * c->K;
+    if (A > (1LL << 30)) return MOE_ERR_ARG;
+    if ((long long)c->E * 2 * c->I >= (1LL << 31) || (long long)c->E * c->H >= (1LL << 31)) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+long long p_max(const moe_config_t* c) {
+    const long long A = (long long)c->T * c->K;
+    return A + (A < c->E ? A : c->E) * (long long)(c->tile_B - 1);
+}
+
+struct Layout {
+    size_t ctl, logits, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm, act, act_sh, sh_out;
+    size_t total;
+};
+
+Layout layout(const moe_config_t* c, int num_sms) {
+    Layout L;
+    const size_t eb = elt_bytes(c->dtype);
+    const long long P = p_max(c);
+    const long long A = (long long)c->T * c->K;
+    const long long I_sh = (long long)c->n_shared * c->I_shared;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t r = o;
+        o = align256(o + bytes);
+        return r;
+    };
+    L.ctl = take(gemm_ctl_bytes(num_sms));
+    L.logits = take(sizeof(float) * (size_t)c->T * c->E);
+    L.ids = take(sizeof(int32_t) * (size_t)A);
+    L.w = take(sizeof(float) * (size_t)A);
+    L.counts = take(sizeof(int32_t) * (size_t)c->E);
+    L.offsets = take(sizeof(int32_t) * ((size_t)c->E + 1));
+    L.scalars = take(sizeof(int32_t) * 4);
+    L.sorted_ids = take(sizeof(int32_t) * (size_t)P);
+    L.block_expert = take(sizeof(int32_t) * (size_t)((P + c->tile_B - 1) / c->tile_B));
+    L.pos = take(sizeof(int32_t) * (size_t)A);
+    L.x_perm = take(eb * (size_t)P * c->H);  // also holds y_perm once x_perm is consumed
+    L.act = take(eb * (size_t)P * c->I);
+    L.act_sh = take(I_sh > 0 ? eb * (size_t)c->T * I_sh : 0);
+    L.sh_out = take(I_sh > 0 ? eb * (size_t)c->T * c->H : 0);
+    L.total = o;
+    return L;
+}
+
+template <typename P>
+P* at(void* base, size_t off) {
+    return reinterpret_cast<P*>(static_cast<uint8_t*>(base) + off);
+}
+
+int status_of(int rc) { return rc == 0 ? MOE_OK : (rc == -5 ? MOE_ERR_DEVICE : (rc == -1 ? MOE_ERR_ARG : MOE_ERR_CUDA)); }
+
+GemmLaunch gate_up_launch(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows,
+                          int H, int I, int dtype, const void* w13, void* act, int max_n) {
+    GemmLaunch g{};
+    g.x = x;
+    g.x_rows = x_rows;
+    g.w = w13;
+    g.w_rows = (long long)n_groups * 2 * I;
+    g.kdim = H;
+    g.n_out = I;
+    g.seg_offsets = seg_offsets;
+    g.n_groups = n_groups;
+    g.seg_rows = seg_rows;
+    g.w_group_stride = 2 * I;
+    g.up_offset = I;
+    g.swiglu = true;
+    g.out_f32 = false;
+    g.out = act;
+    g.out_ld = I;
+    g.dtype = dtype;
+    g.max_n = max_n;
+    return g;
+}
+
+GemmLaunch down_launch(const void* act, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows,
+                       int H, int I, int dtype, const void* w2, void* y, int max_n) {
+    GemmLaunch d{};
+    d.x = act;
+    d.x_rows = x_rows;
+    d.w = w2;
+    d.w_rows = (long long)n_groups * H;
+    d.kdim = I;
+    d.n_out = H;
+    d.seg_offsets = seg_offsets;
+    d.n_groups = n_groups;
+    d.seg_rows = seg_rows;
+    d.w_group_stride = H;
+    d.up_offset = 0;
+    d.swiglu = false;
+    d.out_f32 = false;
+    d.out = y;
+    d.out_ld = H;
+    d.dtype = dtype;
+    d.max_n = max_n;
+    return d;
+}
+
+// gate/up (SwiGLU) + down over `n_groups` segments of X
+int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows, int H, int I,
+            int dtype, const void* w13, const void* w2, void* act, void* y, int max_n, const GemmCtl& ctl,
+            cudaStream_t s) {
+    int rc = launch_gemm(gate_up_launch(x, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w13, act, max_n),
+                         ctl, s);
+    if (rc != 0) return rc;
+    return launch_gemm(down_launch(act, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w2, y, max_n), ctl, s);
+}
+
+int routed_max_n(const moe_config_t* c) {
+    return pick_max_n((double)c->T * c->K / (double)c->E);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_DEVICE: return "unsupported device (needs sm_100)";
+        default: return "unknown status";
+    }
+}
+
+int64_t moe_padded_rows_max(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return -1;
+    return p_max(cfg);
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    DeviceInfo d;
+    if (current_device(&d) != 0) return 0;
+    return layout(cfg, d.num_sms).total;
+}
+
+size_t moe_gemm_workspace_size(void) {
+    DeviceInfo d;
+    if (current_device(&d) != 0) return 0;
+    return gemm_ctl_bytes(d.num_sms);
+}
+
+size_t dense_ffn_workspace_size(int T, int H, int I, int dtype) {
+    const int eb = elt_bytes(dtype);
+    if (eb == 0 || T < 0 || H <= 0 || I <= 0) return 0;
+    DeviceInfo d;
+    if (current_device(&d) != 0) return 0;
+    return align256(gemm_ctl_bytes(d.num_sms)) + align256((size_t)eb * T * I);
+}
+
+int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router, float* logits, void* workspace,
+                    size_t ws_bytes, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!x || !w_router || !logits || !workspace) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    GemmLaunch g{};
+    g.x = x;
+    g.x_rows = cfg->T;
+    g.w = w_router;
+    g.w_rows = cfg->E;
+    g.kdim = cfg->H;
+    g.n_out = cfg->E;
+    g.n_groups = 1;
+    g.seg_rows = cfg->T;
+    g.swiglu = false;
+    g.out_f32 = true;
+    g.out = logits;
+    g.out_ld = cfg->E;
+    g.dtype = cfg->dtype;
+    g.max_n = pick_max_n(cfg->T);
+    return status_of(launch_gemm(g, gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+}
+
+int moe_route(const moe_config_t* cfg, const float* logits, int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!logits || !topk_ids || !topk_w) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    return status_of(launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, logits, topk_ids, topk_w,
+                                 (cudaStream_t)stream));
+}
+
+int moe_align_pad(const moe_config_t* cfg, const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
+                  int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!counts || !offsets || !scalars || !block_expert) return MOE_ERR_ARG;
+    if (cfg->T > 0 && (!topk_ids || !sorted_ids || !pos)) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    return status_of(launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, p_max(cfg), topk_ids, counts, offsets,
+                                  sorted_ids, block_expert, pos, scalars, nullptr, (cudaStream_t)stream));
+}
+
+int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids, const int32_t* scalars,
+                void* x_perm, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!x || !sorted_ids || !scalars || !x_perm || !aligned16(x) || !aligned16(x_perm)) return MOE_ERR_ARG;
+    return status_of(launch_permute(cfg->H, cfg->K, cfg->dtype, p_max(cfg), x, sorted_ids, scalars, x_perm,
+                                    (cudaStream_t)stream));
+}
+
+int moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const void* w13, const void* w2,
+                    const int32_t* offsets, void* act, void* y_perm, void* workspace, size_t ws_bytes,
+                    moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!x_perm || !w13 || !w2 || !offsets || !act || !y_perm || !workspace) return MOE_ERR_ARG;
+    if (!aligned16(x_perm) || !aligned16(w13) || !aligned16(w2) || !aligned16(act) || !aligned16(y_perm) ||
+        !aligned16(workspace))
+        return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    return status_of(run_ffn(x_perm, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act,
+                             y_perm, routed_max_n(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+}
+
+int moe_grouped_gate_up(const moe_config_t* cfg, const void* x_perm, const void* w13, const int32_t* offsets,
+                        void* act, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!x_perm || !w13 || !offsets || !act || !workspace) return MOE_ERR_ARG;
+    if (!aligned16(x_perm) || !aligned16(w13) || !aligned16(act) || !aligned16(workspace)) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    return status_of(launch_gemm(gate_up_launch(x_perm, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype,
+                                                w13, act, routed_max_n(cfg)),
+                                 gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+}
+
+int moe_grouped_down(const moe_config_t* cfg, const void* act, const void* w2, const int32_t* offsets, void* y_perm,
+                     void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!act || !w2 || !offsets || !y_perm || !workspace) return MOE_ERR_ARG;
+    if (!aligned16(act) || !aligned16(w2) || !aligned16(y_perm) || !aligned16(workspace)) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    return status_of(launch_gemm(down_launch(act, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w2,
+                                             y_perm, routed_max_n(cfg)),
+                                 gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+}
+
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* pos, const float* topk_w,
+                const void* shared_out, void* out, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    if (!y_perm || !pos || !topk_w || !out || !aligned16(y_perm) || !aligned16(out) ||
+        (shared_out && !aligned16(shared_out)))
+        return MOE_ERR_ARG;
+    return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, topk_w, shared_out, out,
+                                    (cudaStream_t)stream));
+}
+
+int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13, const void* w2,
+                      const void* w13_shared, const void* w2_shared, const float* logits_override, void* out,
+                      void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->T == 0) return MOE_OK;
+    const long long I_sh = (long long)cfg->n_shared * cfg->I_shared;
+    if (!x || !w_router || !w13 || !w2 || !out || !workspace) return MOE_ERR_ARG;
+    if (I_sh > 0 && (!w13_shared || !w2_shared)) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) ||
+        !aligned16(workspace) || (I_sh > 0 && (!aligned16(w13_shared) || !aligned16(w2_shared))))
+        return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    const Layout L = layout(cfg, d.num_sms);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const GemmCtl ctl = gemm_ctl(at<uint8_t>(workspace, L.ctl), d.num_sms);
+    float* logits = at<float>(workspace, L.logits);
+    int32_t* ids = at<int32_t>(workspace, L.ids);
+    float* w = at<float>(workspace, L.w);
+    int32_t* counts = at<int32_t>(workspace, L.counts);
+    int32_t* offsets = at<int32_t>(workspace, L.offsets);
+    int32_t* scalars = at<int32_t>(workspace, L.scalars);
+    int32_t* sorted_ids = at<int32_t>(workspace, L.sorted_ids);
+    int32_t* block_expert = at<int32_t>(workspace, L.block_expert);
+    int32_t* pos = at<int32_t>(workspace, L.pos);
+    void* x_perm = at<void>(workspace, L.x_perm);
+    void* act = at<void>(workspace, L.act);
+    void* y_perm = x_perm;
+    const long long P = p_max(cfg);
+
+    // router
+    {
+        GemmLaunch g{};
+        g.x = x;
+        g.x_rows = cfg->T;
+        g.w = w_router;
+        g.w_rows = cfg->E;
+        g.kdim = cfg->H;
+        g.n_out = cfg->E;
+        g.n_groups = 1;
+        g.seg_rows = cfg->T;
+        g.out_f32 = true;
+        g.out = logits;
+        g.out_ld = cfg->E;
+        g.dtype = cfg->dtype;
+        g.max_n = pick_max_n(cfg->T);
+        if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
+    }
+    if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, logits_override ? logits_override : logits,
+                          ids, w, s)) != 0)
+        return status_of(rc);
+    if ((rc = launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, P, ids, counts, offsets, sorted_ids, block_expert, pos,
+                           scalars, stats_out, s)) != 0)
+        return status_of(rc);
+    if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s)) != 0)
+        return status_of(rc);
+    if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
+                      routed_max_n(cfg), ctl, s)) != 0)
+        return status_of(rc);
+    const void* sh = nullptr;
+    if (I_sh > 0) {
+        void* act_sh = at<void>(workspace, L.act_sh);
+        void* sh_out = at<void>(workspace, L.sh_out);
+        if ((rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared, act_sh,
+                          sh_out, pick_max_n(cfg->T), ctl, s)) != 0)
+            return status_of(rc);
+        sh = sh_out;
+    }
+    return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, w, sh, out, s));
+}
+
+int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13, const void* w2, void* out,
+              void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    const int eb = elt_bytes(dtype);
+    if (eb == 0 || T < 0 || H <= 0 || I <= 0 || H % (16 / eb) || I % (16 / eb)) return MOE_ERR_ARG;
+    if ((long long)2 * I >= (1LL << 31)) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !w13 || !w2 || !out || !workspace) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) || !aligned16(workspace))
+        return MOE_ERR_ARG;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return status_of(rc);
+    const size_t ctl_bytes = align256(gemm_ctl_bytes(d.num_sms));
+    if (ws_bytes < ctl_bytes + (size_t)eb * T * I) return MOE_ERR_WORKSPACE;
+    void* act = at<void>(workspace, ctl_bytes);
+    return status_of(run_ffn(x, T, nullptr, 1, T, H, I, dtype, w13, w2, act, out, pick_max_n(T),
+                             gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+}
+
+int moe_check_status(void* workspace, moe_stream_t stream) {
+    if (!workspace) return MOE_ERR_ARG;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return status_of(rc);
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    unsigned st = 0;
+    if (cudaMemcpy(&st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (st & kStatusTimeout) {
+        if (cudaMemset(workspace, 0, gemm_ctl_zero_bytes(d.num_sms)) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        return MOE_ERR_TIMEOUT;
+    }
+    return MOE_OK;
+}
+
+void moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit.store(ns ? ns : 2000000000ull); }
+
+void moe_debug_withhold_first_load(int enable) { g_withhold.store(enable ? 1 : 0); }
+
+uint64_t moe_kernel_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+// moe_gemm.cu -- host side of the tcgen05 grouped GEMM: TMA tensor maps,
+// variant dispatch (operand dtype, SwiGLU or plain epilogue, token-tile cap)
+// and the persistent launch.
+#include <mutex>
+
+#include "moe_gemm.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// [rows, kdim] row-major, box = box_rows x (128 bytes), 128-byte swizzle,
+// out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void* base, long long rows, int kdim,
+              int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kdim), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kdim) * elt_bytes};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt_bytes), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T, typename OutT, bool kSwiGLU, int kMaxN>
+int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t stream) {
+    using C = GemmCfg<T, kSwiGLU, kMaxN>;
+    auto kern = moe_gemm_kernel<T, OutT, kSwiGLU, kMaxN>;
+    static bool attr_done = false;  // per instantiation
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return -3;
+        }
+        attr_done = true;
+    }
+    CUtensorMap tm_w, tm_x;
+    if (!make_map(&tm_w, Elt<T>::kTma, Elt<T>::kBytes, L.w, L.w_rows, L.kdim, 128)) return -3;
+    if (!make_map(&tm_x, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxRows)) return -3;
+    GemmParams p;
+    p.seg_offsets = L.seg_offsets;
+    p.n_groups = L.n_groups;
+    p.seg_rows = L.seg_rows;
+    p.n_out = L.n_out;
+    p.kdim = L.kdim;
+    p.w_group_stride = L.w_group_stride;
+    p.up_offset = L.up_offset;
+    p.out = L.out;
+    p.out_ld = L.out_ld;
+    p.counters = ctl.counters;
+    p.partials = ctl.partials;
+    p.status = ctl.status;
+    p.wait_limit_ns = wait_limit_ns();
+    p.withhold_first_load = take_withhold_flag();
+    p.sk_min_units = 4;
+    kern<<<num_sms, kGemmThreads, C::kSmemBytes, stream>>>(tm_w, tm_x, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+template <typename T, typename OutT, bool kSwiGLU>
+int dispatch_n(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t s) {
+    switch (L.max_n) {
+        case 32: return launch_variant<T, OutT, kSwiGLU, 32>(L, ctl, num_sms, s);
+        case 64: return launch_variant<T, OutT, kSwiGLU, 64>(L, ctl, num_sms, s);
+        case 128: return launch_variant<T, OutT, kSwiGLU, 128>(L, ctl, num_sms, s);
+        case 256: return launch_variant<T, OutT, kSwiGLU, 256>(L, ctl, num_sms, s);
+        default: return -1;
+    }
+}
+
+}  // namespace
+
+size_t gemm_ctl_bytes(int num_sms) {
+    return kCtlHeaderBytes + sizeof(int) * 2 * (size_t)num_sms + kSlotBytesMax * 2 * (size_t)num_sms + 256;
+}
+
+size_t gemm_ctl_zero_bytes(int num_sms) { return kCtlHeaderBytes + sizeof(int) * 2 * (size_t)num_sms; }
+
+GemmCtl gemm_ctl(void* workspace, int num_sms) {
+    uint8_t* b = static_cast<uint8_t*>(workspace);
+    GemmCtl c;
+    c.status = reinterpret_cast<unsigned*>(b);
+    c.counters = reinterpret_cast<int*>(b + kCtlHeaderBytes);
+    size_t off = kCtlHeaderBytes + sizeof(int) * 2 * (size_t)num_sms;
+    off = (off + 255) & ~size_t(255);
+    c.partials = reinterpret_cast<float*>(b + off);
+    return c;
+}
+
+int pick_max_n(double rows_per_group) {
+    if (rows_per_group <= 24.0) return 32;
+    if (rows_per_group <= 56.0) return 64;
+    if (rows_per_group <= 112.0) return 128;
+    return 256;
+}
+
+int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream) {
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    if (L.n_groups < 1 || L.n_groups > kMaxGroups || L.kdim <= 0 || L.n_out <= 0) return -1;
+    if (L.x_rows <= 0 || L.w_rows <= 0) return 0;
+    if (L.dtype == 0) {
+        if (L.out_f32) {
+            if (L.swiglu) return -1;
+            return dispatch_n<__nv_bfloat16, float, false>(L, ctl, d.num_sms, stream);
+        }
+        return L.swiglu ? dispatch_n<__nv_bfloat16, __nv_bfloat16, true>(L, ctl, d.num_sms, stream)
+                        : dispatch_n<__nv_bfloat16, __nv_bfloat16, false>(L, ctl, d.num_sms, stream);
+    }
+    if (L.dtype == 1) {
+        return L.swiglu ? dispatch_n<float, float, true>(L, ctl, d.num_sms, stream)
+                        : dispatch_n<float, float, false>(L, ctl, d.num_sms, stream);
+    }
+    return -1;
+}
+
+}  // namespace moe

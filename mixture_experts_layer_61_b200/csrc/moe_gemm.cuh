@@ -1,0 +1,513 @@
+// moe_gemm.cuh -- persistent grouped GEMM on the sm_100a tensor cores
+// (tcgen05.mma, accumulators in TMEM, operands staged by TMA with the
+// 128-byte swizzle), used for every contraction of the layer:
+//   * the routed experts' gate/up projections with the SwiGLU epilogue and
+//     their down projections (the "GroupGEMM" of the talk notes' Table 1 and
+//     "Key findings 5"), one group per expert segment of the padded rows;
+//   * the dense SwiGLU FFN (shared experts, DenseFA, DensePA) as one group;
+//   * the router GEMM (fp32 logits) as one group.
+//
+// Orientation.  The weight rows are the MMA's M side (128 output features
+// per tile) and the token rows its N side (16..kMaxN tokens per tile, a
+// multiple of 16).  Decode (one or two tokens per expert) then costs a
+// 128 x 16 MMA per 128 weight rows instead of a 128-row tile of padding, and
+// prefill uses N up to 256.  The accumulator D[feature][token] lives in TMEM
+// (lane = feature, column = token).
+//
+// Tiles.  A group g owns rows [seg[g], seg[g+1]) of the token matrix X.  The
+// rows are cut into chunks of at most kMaxN rows (in units of 16, balanced);
+// a tile is (group, 128-feature block f, chunk j), ordered f-major inside a
+// group so that the chunks sharing one weight block run side by side and
+// reuse it from L2.  Each tile reduces over K = kdim in steps of 128 bytes.
+//
+// Schedule.  gridDim.x persistent blocks (one per SM).  Whole waves of tiles
+// are dealt round-robin; the remaining one to two waves are split evenly by
+// k-iterations across the blocks (stream-K), so every block streams the same
+// number of weight bytes even when there are fewer tiles than SMs (decode).
+// A tile split across blocks is finished by the last block to arrive: each
+// contributor stores its fp32 partial tile, then increments the tile's
+// counter; the block that brings the counter to the number of contributors
+// sums all partials in block order (deterministic) and runs the epilogue.
+// No block ever waits on another block.
+//
+// Roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// the MMAs, warps 2..5 run the epilogue (TMEM -> registers -> global).  All
+// waits are bounded by a deadline; a wait that runs out sets the status word
+// and every role winds down (in-flight copies and MMAs are drained first).
+#pragma once
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kMaxGroups = 1024;
+constexpr int kGemmThreads = 192;
+
+struct GemmParams {
+    const int32_t* seg_offsets;  // [n_groups + 1] row offsets into X, or nullptr: one group [0, seg_rows)
+    int n_groups;
+    int seg_rows;
+    int n_out;            // output features
+    int kdim;             // reduction length
+    int w_group_stride;   // weight rows from one group to the next
+    int up_offset;        // weight rows from a gate row to its up row (SwiGLU)
+    void* out;            // output rows (same row index as X), out_ld elements apart
+    int out_ld;
+    int* counters;        // >= 2 * gridDim.x ints; zero on entry and on exit
+    float* partials;      // 2 * gridDim.x slots of 128 * kAccCols floats
+    unsigned* status;     // status word (bit kStatusTimeout)
+    uint64_t wait_limit_ns;
+    int withhold_first_load;
+    int sk_min_units;     // minimum k-iterations per stream-K block
+};
+
+template <typename T, bool kSwiGLU, int kMaxN>
+struct GemmCfg {
+    static constexpr int kBK = 128 / Elt<T>::kBytes;   // K elements per stage (one swizzle row)
+    static constexpr int kMmaK = 32 / Elt<T>::kBytes;  // K per MMA instruction
+    static constexpr int kNW = kSwiGLU ? 2 : 1;        // weight tiles per stage (gate, up)
+    static constexpr int kWTileBytes = 128 * 128;
+    static constexpr int kXBoxRows = 16;
+    static constexpr int kXBoxBytes = kXBoxRows * 128;
+    static constexpr int kXTileBytes = kMaxN * 128;
+    static constexpr int kStageBytes = kNW * kWTileBytes + kXTileBytes;
+    static constexpr int kAccCols = kSwiGLU ? 2 * kMaxN : kMaxN;
+    static constexpr int kNumAcc = (512 / kAccCols) >= 2 ? 2 : 1;
+    static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
+    static constexpr int kMiscBytes = 512;
+    static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes;
+    static constexpr int kStagesRaw = kBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
+    static_assert(kStages >= 2, "pipeline needs two stages");
+    static_assert(kMaxN % 16 == 0 && kMaxN >= 16 && kMaxN <= 256, "MMA N range");
+    static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
+};
+
+// ------------------------------------------------------------- scheduling
+struct Tile {
+    int group, f0, row0, nrows, mma_n, wrow;
+};
+
+struct Sched {
+    int n_groups, NF, KI, G, cta;
+    long long total_tiles, dp_waves, dp_tiles, sk_tiles, U;
+    int G_sk;
+    // iteration state
+    long long w;        // next DP wave
+    long long u, u_end; // stream-K cursor
+    bool sk_first;
+
+    __device__ long long beg(int c) const { return (long long)c * U / G_sk; }
+    // block owning stream-K unit q
+    __device__ int owner(long long q) const { return (int)(((q + 1) * (long long)G_sk - 1) / U); }
+};
+
+struct Item {
+    long long tile;
+    int kb, ke;
+    bool split;   // partial tile (stream-K fixup)
+    int slot;     // partial slot of this block (0 or 1)
+    long long sk_tile;
+};
+
+__device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int total_chunks, int NF, int KI) {
+    s.n_groups = p.n_groups;
+    s.NF = NF;
+    s.KI = KI;
+    s.G = gridDim.x;
+    s.cta = blockIdx.x;
+    s.total_tiles = (long long)total_chunks * NF;
+    s.dp_waves = s.total_tiles >= 2LL * s.G ? s.total_tiles / s.G - 1 : 0;
+    s.dp_tiles = s.dp_waves * s.G;
+    s.sk_tiles = s.total_tiles - s.dp_tiles;
+    s.U = s.sk_tiles * KI;
+    long long gsk = p.sk_min_units > 0 ? s.U / p.sk_min_units : s.U;
+    if (gsk < 1) gsk = 1;
+    if (gsk > s.G) gsk = s.G;
+    s.G_sk = (int)gsk;
+    s.w = 0;
+    if (s.U > 0 && s.cta < s.G_sk) {
+        s.u = s.beg(s.cta);
+        s.u_end = s.beg(s.cta + 1);
+    } else {
+        s.u = s.u_end = 0;
+    }
+    s.sk_first = true;
+}
+
+__device__ __forceinline__ bool sched_next(Sched& s, Item& it) {
+    if (s.w < s.dp_waves) {
+        it.tile = s.w * s.G + s.cta;
+        it.kb = 0;
+        it.ke = s.KI;
+        it.split = false;
+        it.slot = 0;
+        it.sk_tile = -1;
+        ++s.w;
+        return true;
+    }
+    if (s.u < s.u_end) {
+        long long st = s.u / s.KI;
+        int kb = (int)(s.u - st * s.KI);
+        long long left = s.u_end - s.u;
+        int ke = (int)((long long)kb + left < s.KI ? kb + left : s.KI);
+        it.tile = s.dp_tiles + st;
+        it.kb = kb;
+        it.ke = ke;
+        it.sk_tile = st;
+        it.split = !(kb == 0 && ke == s.KI);
+        it.slot = s.sk_first ? 0 : 1;
+        s.sk_first = false;
+        s.u += ke - kb;
+        return true;
+    }
+    return false;
+}
+
+// Rows of chunk j of a group of `rows` rows cut into `nch` chunks, in units of 16.
+__device__ __forceinline__ void chunk_rows(int rows, int nch, int j, int& start, int& n, int& mma_n) {
+    int units = (rows + 15) >> 4;
+    int base = units / nch, extra = units % nch;
+    int su = j * base + (j < extra ? j : extra);
+    int mu = base + (j < extra ? 1 : 0);
+    start = su * 16;
+    mma_n = mu * 16;
+    int left = rows - start;
+    n = mma_n < left ? mma_n : left;
+}
+
+__device__ __forceinline__ int chunks_of(int rows, int max_n) {
+    if (rows <= 0) return 0;
+    int units = (rows + 15) >> 4;
+    int per = max_n >> 4;
+    return (units + per - 1) / per;
+}
+
+__device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, const int* cbase, int n_groups, int NF,
+                                            const GemmParams& p) {
+    // group: largest g with cbase[g] * NF <= tile
+    int lo = 0, hi = n_groups - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if ((long long)cbase[mid] * NF <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    int g = lo;
+    int nch = cbase[g + 1] - cbase[g];
+    long long local = tile - (long long)cbase[g] * NF;
+    int f = (int)(local / nch);
+    int j = (int)(local - (long long)f * nch);
+    Tile t;
+    int start, n, mn;
+    chunk_rows(seg[g + 1] - seg[g], nch, j, start, n, mn);
+    t.group = g;
+    t.f0 = f * 128;
+    t.row0 = seg[g] + start;
+    t.nrows = n;
+    t.mma_n = mn;
+    t.wrow = g * p.w_group_stride + f * 128;
+    return t;
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_out(OutT* ptr, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(float* ptr, float v) { *ptr = v; }
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* ptr, float v) {
+    *ptr = __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// ------------------------------------------------------------------ kernel
+template <typename T, typename OutT, bool kSwiGLU, int kMaxN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                    const GemmParams p) {
+    using C = GemmCfg<T, kSwiGLU, kMaxN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stage_base = smem;
+    int* seg = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes);
+    int* cbase = seg + (kMaxGroups + 1);
+    uint8_t* misc = reinterpret_cast<uint8_t*>(cbase + (kMaxGroups + 1));
+    uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + C::kNumAcc;
+    uint64_t* drain_bar = tempty + C::kNumAcc;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    int* bcast = const_cast<int*>(abort_flag) + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_groups = p.n_groups;
+    const uint64_t deadline = p.wait_limit_ns;  // per-wait limit
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < C::kNumAcc; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(drain_bar, 1);
+        fence_barrier_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&tm_w);
+        tma_prefetch_desc(&tm_x);
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, 512);
+    // segment table
+    for (int g = threadIdx.x; g <= n_groups; g += blockDim.x)
+        seg[g] = p.seg_offsets ? p.seg_offsets[g] : (g == 0 ? 0 : p.seg_rows);
+    __syncthreads();
+    if (warp == 0) {
+        int running = 0;
+        for (int base = 0; base < n_groups; base += 32) {
+            int g = base + lane;
+            int n = g < n_groups ? chunks_of(seg[g + 1] - seg[g], kMaxN) : 0;
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (g < n_groups) cbase[g] = running + incl - n;
+            running += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) cbase[n_groups] = running;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int NF = (p.n_out + 127) / 128;
+    const int KI = (p.kdim + C::kBK - 1) / C::kBK;
+    Sched sch;
+    sched_init(sch, p, cbase[n_groups], NF, KI);
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            int fills[C::kStages];
+#pragma unroll
+            for (int s = 0; s < C::kStages; ++s) fills[s] = 0;
+            uint32_t kc = 0;
+            bool withhold = p.withhold_first_load && blockIdx.x == 0;
+            bool ok = true;
+            Item it;
+            while (ok && sched_next(sch, it)) {
+                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, p);
+                const uint32_t bytes = C::kNW * C::kWTileBytes + (t.mma_n / 16) * C::kXBoxBytes;
+                for (int k = it.kb; k < it.ke; ++k, ++kc) {
+                    const int s = kc % C::kStages;
+                    const uint32_t ph = (kc / C::kStages) & 1u;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, deadline, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (withhold) {  // test hook: this stage is never filled
+                        withhold = false;
+                        continue;
+                    }
+                    uint8_t* st = stage_base + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    const int kx = k * C::kBK;
+                    tma_load_2d(st, &tm_w, &full[s], kx, t.wrow, pol_w);
+                    if (kSwiGLU) tma_load_2d(st + C::kWTileBytes, &tm_w, &full[s], kx, t.wrow + p.up_offset, pol_w);
+                    uint8_t* xs = st + C::kNW * C::kWTileBytes;
+                    for (int r = 0; r < t.mma_n; r += C::kXBoxRows)
+                        tma_load_2d(xs + r * 128, &tm_x, &full[s], kx, t.row0 + r, pol_x);
+                    ++fills[s];
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+            }
+            // every issued copy lands before the block exits
+            for (int s = 0; s < C::kStages; ++s)
+                if (fills[s] > 0) mbar_drain(&full[s], (uint32_t)(fills[s] - 1) & 1u, p.wait_limit_ns);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t kc = 0, ac = 0;
+            bool ok = true;
+            Item it;
+            while (ok && sched_next(sch, it)) {
+                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, p);
+                const int b = ac % C::kNumAcc;
+                const uint32_t aph = (ac / C::kNumAcc) & 1u;
+                if (!mbar_wait_bounded(&tempty[b], aph ^ 1u, deadline, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_gate = tmem_base + b * C::kAccCols;
+                const uint32_t d_up = d_gate + kMaxN;
+                const uint32_t idesc = umma_idesc(Elt<T>::kMmaFmt, 128, t.mma_n);
+                for (int k = it.kb; k < it.ke; ++k, ++kc) {
+                    const int s = kc % C::kStages;
+                    const uint32_t ph = (kc / C::kStages) & 1u;
+                    if (!mbar_wait_bounded(&full[s], ph, deadline, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t* st = stage_base + s * C::kStageBytes;
+                    const uint64_t a0 = umma_desc_sw128(smem_u32(st));
+                    const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
+                    const uint64_t bx = umma_desc_sw128(smem_u32(st + C::kNW * C::kWTileBytes));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
+                        umma<T>(d_gate, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        if (kSwiGLU) umma<T>(d_up, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&tfull[b]);
+                ++ac;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+                umma_commit(drain_bar);
+                mbar_drain(drain_bar, 0, p.wait_limit_ns);
+            }
+        }
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // TMEM lane = feature row within the tile
+        OutT* out = reinterpret_cast<OutT*>(p.out);
+        uint32_t ac = 0;
+        Item it;
+        while (sched_next(sch, it)) {
+            Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, p);
+            const int b = ac % C::kNumAcc;
+            const uint32_t aph = (ac / C::kNumAcc) & 1u;
+            if (!mbar_wait_bounded(&tfull[b], aph, deadline, abort_flag)) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * C::kAccCols;
+            const int f = t.f0 + r;
+            const bool fvalid = f < p.n_out;
+            OutT* orow = out + (long long)t.row0 * p.out_ld + f;
+            if (!it.split) {
+                for (int c0 = 0; c0 < t.mma_n; c0 += 16) {
+                    float g[16];
+                    tmem_ld16(tacc + c0, g);
+                    if (kSwiGLU) {
+                        float u[16];
+                        tmem_ld16(tacc + kMaxN + c0, u);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
+                    }
+                    if (fvalid) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * p.out_ld, g[i]);
+                    }
+                }
+            } else {
+                // stream-K: publish this block's partial tile
+                const long long slot_floats = 128LL * C::kAccCols;
+                float* mine = p.partials + ((long long)blockIdx.x * 2 + it.slot) * slot_floats;
+                for (int c0 = 0; c0 < t.mma_n; c0 += 16) {
+                    float g[16];
+                    tmem_ld16(tacc + c0, g);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) mine[(long long)(c0 + i) * 128 + r] = g[i];
+                    if (kSwiGLU) {
+                        tmem_ld16(tacc + kMaxN + c0, g);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) mine[(long long)(kMaxN + c0 + i) * 128 + r] = g[i];
+                    }
+                }
+                __threadfence();
+                named_sync(1, 128);
+                if (r == 0) *bcast = atomicAdd(&p.counters[it.sk_tile], 1);
+                named_sync(1, 128);
+                const int arrived = *bcast;
+                // contributors: blocks whose stream-K range meets this tile
+                const long long q0 = it.sk_tile * sch.KI;
+                const int c_first = sch.owner(q0);
+                const int c_last = sch.owner(q0 + sch.KI - 1);
+                int ncontrib = 0;
+                for (int c = c_first; c <= c_last; ++c)
+                    if (sch.beg(c) < sch.beg(c + 1)) ++ncontrib;
+                if (arrived == ncontrib - 1) {
+                    __threadfence();
+                    for (int c0 = 0; c0 < t.mma_n; c0 += 16) {
+                        float g[16], u[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
+                        for (int c = c_first; c <= c_last; ++c) {
+                            const long long bc = sch.beg(c);
+                            if (bc >= sch.beg(c + 1)) continue;
+                            if (c == (int)blockIdx.x) {
+                                float v[16];
+                                tmem_ld16(tacc + c0, v);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) g[i] += v[i];
+                                if (kSwiGLU) {
+                                    tmem_ld16(tacc + kMaxN + c0, v);
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i) u[i] += v[i];
+                                }
+                            } else {
+                                const int slot = (bc / sch.KI == it.sk_tile) ? 0 : 1;
+                                const float* other = p.partials + ((long long)c * 2 + slot) * slot_floats;
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) g[i] += ld_cg_f32(other + (long long)(c0 + i) * 128 + r);
+                                if (kSwiGLU) {
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i)
+                                        u[i] += ld_cg_f32(other + (long long)(kMaxN + c0 + i) * 128 + r);
+                                }
+                            }
+                        }
+                        if (kSwiGLU) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
+                        }
+                        if (fvalid) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * p.out_ld, g[i]);
+                        }
+                    }
+                    if (r == 0) p.counters[it.sk_tile] = 0;  // leave the counter zero for the next launch
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[b]);
+            ++ac;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace moe

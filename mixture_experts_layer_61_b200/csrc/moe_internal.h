@@ -1,0 +1,78 @@
+// moe_internal.h -- host-side declarations shared by the libmoe translation
+// units (launchers, device properties, the launch counter).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Cached properties of the current device.
+struct DeviceInfo {
+    int device;
+    int num_sms;
+    int cc_major, cc_minor;
+};
+// Returns 0 and fills *info for the current device; -5 if it is not sm_100.
+int current_device(DeviceInfo* info);
+
+// Workspace control block: status word, stream-K counters (2 per SM) and
+// partial-tile slots (2 per SM, each 128 rows x at most 512 fp32 columns).
+constexpr size_t kCtlHeaderBytes = 256;
+constexpr size_t kSlotBytesMax = 128ull * 512ull * 4ull;
+size_t gemm_ctl_bytes(int num_sms);
+// Bytes of the control words that must be zero between calls (status + counters).
+size_t gemm_ctl_zero_bytes(int num_sms);
+
+struct GemmCtl {
+    unsigned* status;
+    int* counters;
+    float* partials;
+};
+GemmCtl gemm_ctl(void* workspace, int num_sms);
+
+// One GEMM launch.  X rows are tokens ([x_rows, kdim]), W rows are output
+// features ([w_rows, kdim]); out[row][feature] with row stride out_ld.
+struct GemmLaunch {
+    const void* x;
+    long long x_rows;
+    const void* w;
+    long long w_rows;
+    int kdim;
+    int n_out;
+    const int32_t* seg_offsets;  // device, n_groups + 1, or nullptr
+    int n_groups;
+    int seg_rows;                // one segment [0, seg_rows) when seg_offsets == nullptr
+    int w_group_stride;
+    int up_offset;
+    bool swiglu;
+    bool out_f32;                // fp32 output (router logits) instead of the activation dtype
+    void* out;
+    int out_ld;
+    int dtype;                   // 0 bf16, 1 fp32
+    int max_n;                   // token-tile cap: 32, 64, 128 or 256
+};
+
+int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
+
+// Token-tile cap for an expected number of rows per group.
+int pick_max_n(double rows_per_group);
+
+// Elementwise / routing kernels.
+int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,
+                cudaStream_t stream);
+int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids, int32_t* counts,
+                 int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
+                 int32_t* stats_copy, cudaStream_t stream);
+int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
+                   const int32_t* scalars, void* x_perm, cudaStream_t stream);
+int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
+                   const void* shared_out, void* out, cudaStream_t stream);
+
+// Launch bookkeeping.
+void count_launch();
+uint64_t wait_limit_ns();
+int take_withhold_flag();
+
+}  // namespace moe

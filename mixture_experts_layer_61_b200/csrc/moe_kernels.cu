@@ -1,0 +1,418 @@
+// moe_kernels.cu -- the non-GEMM stages of the MoE block ("top-K selection",
+// "alignment" and the "local sum" of the talk notes' "Key findings 5", plus
+// the permute that feeds the grouped GEMM).  All bandwidth-light: one warp
+// per token for top-K, one block for the alignment, 16-byte vector copies for
+// permute and combine.
+#include <climits>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ top-K
+// Order: larger logit first, lower expert index on equal logits.
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+    return v > bv || (v == bv && i < bi);
+}
+
+// One warp per token.  Lane l owns experts l, l+32, ...; K passes of a warp
+// arg-max over the experts not yet taken.
+__global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int score_fn, int renorm,
+                                                        const float* __restrict__ logits, int32_t* __restrict__ ids,
+                                                        float* __restrict__ w) {
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const float* l = logits + (size_t)t * E;
+    uint32_t taken = 0;  // bit j: expert lane + 32 j
+    float sel_v[16];
+    int sel_i[16];
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+        for (int j = 0, e = lane; e < E; ++j, e += 32) {
+            if ((taken >> j) & 1u) continue;
+            const float v = l[e];
+            if (better(v, e, bv, bi)) {
+                bv = v;
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (better(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if (bi == INT_MAX) {
+            // only NaN logits remain: take the lowest expert not yet taken so
+            // that every id stays in range
+            int cand = INT_MAX;
+            for (int j = 0, e = lane; e < E; ++j, e += 32)
+                if (!((taken >> j) & 1u)) {
+                    cand = e;
+                    break;
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+            bi = cand;
+            bv = l[bi];
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        sel_v[k] = bv;
+        sel_i[k] = bi;
+    }
+    // gate weights, identical in every lane; lane k stores entry k
+    float wk = 0.f;
+    if (score_fn == 0) {
+        float m, den = 0.f;
+        if (renorm) {
+            m = sel_v[0];
+            for (int k = 1; k < K; ++k) m = fmaxf(m, sel_v[k]);
+            for (int k = 0; k < K; ++k) den += expf(sel_v[k] - m);
+        } else {
+            m = -INFINITY;
+            for (int e = lane; e < E; e += 32) m = fmaxf(m, l[e]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float part = 0.f;
+            for (int e = lane; e < E; e += 32) part += expf(l[e] - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            den = part;
+        }
+        for (int k = 0; k < K; ++k)
+            if (k == lane) wk = expf(sel_v[k] - m) / den;
+    } else {
+        float den = 0.f;
+        for (int k = 0; k < K; ++k) den += 1.f / (1.f + expf(-sel_v[k]));
+        for (int k = 0; k < K; ++k)
+            if (k == lane) {
+                const float s = 1.f / (1.f + expf(-sel_v[k]));
+                wk = renorm ? s / den : s;
+            }
+    }
+    if (lane < K) {
+        int id = 0;
+        for (int k = 0; k < K; ++k)
+            if (k == lane) id = sel_i[k];
+        ids[(size_t)t * K + lane] = id;
+        w[(size_t)t * K + lane] = wk;
+    }
+}
+
+int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,
+                cudaStream_t stream) {
+    if (T == 0) return 0;
+    const int warps_per_block = 8;
+    const int blocks = (T + warps_per_block - 1) / warps_per_block;
+    topk_gate_kernel<<<blocks, warps_per_block * 32, 0, stream>>>(T, E, K, score_fn, renorm, logits, ids, w);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+// -------------------------------------------------------------- alignment
+// One block of 1024 threads.  (1) shared-memory histogram of the expert ids;
+// (2) block scan of the padded counts ceil(N_e/B)*B into offsets;
+// (3) stable scatter in rounds of 1024 assignments: inside a warp the rank
+// among equal ids comes from __match_any_sync, across the 32 warps of a round
+// from a per-(warp, expert) count table scanned over the warps, across rounds
+// from a per-expert cursor -- so assignments keep ascending order within
+// each expert; (4) -1 in the padding slots, block_expert per B-row block.
+constexpr int kAlignThreads = 1024;
+
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int s = warp_tot[lane];
+        int si = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, si, o);
+            if (lane >= o) si += x;
+        }
+        warp_tot[lane] = si - s;  // exclusive prefix of warp totals
+        if (lane == 31) warp_tot[32] = si;
+    }
+    __syncthreads();
+    const int r = warp_tot[warp] + incl - v;
+    total = warp_tot[32];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kAlignThreads, 1)
+    align_kernel(int T, int K, int E, int B, long long P_max, const int32_t* __restrict__ ids,
+                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
+                 int32_t* __restrict__ block_expert, int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
+                 int32_t* __restrict__ stats_copy) {
+    extern __shared__ int sm[];
+    int* cnt = sm;                 // E
+    int* off = cnt + E;            // E + 1
+    int* cursor = off + E + 1;     // E
+    int* rt = cursor + E;          // E
+    int* warp_tot = rt + E;        // 33
+    int* bad = warp_tot + 33;      // 1
+    uint16_t* tbl = reinterpret_cast<uint16_t*>(bad + 1);  // 32 x E
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long A = (long long)T * K;
+
+    for (int e = tid; e < E; e += kAlignThreads) cnt[e] = 0;
+    if (tid == 0) *bad = 0;
+    __syncthreads();
+    for (long long a = tid; a < A; a += kAlignThreads) {
+        const int e = ids[a];
+        if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[e], 1);
+        else atomicOr(bad, 1);
+    }
+    __syncthreads();
+
+    // padded counts -> offsets (E <= 1024: one expert per thread)
+    const int n = tid < E ? cnt[tid] : 0;
+    const int padded = ((n + B - 1) / B) * B;
+    int P = 0;
+    const int excl = block_excl_scan(padded, warp_tot, P);
+    const int n_active = __syncthreads_count(tid < E && n > 0);
+    if (tid < E) {
+        off[tid] = excl;
+        cursor[tid] = excl;
+        counts[tid] = n;
+        offsets[tid] = excl;
+    }
+    if (tid == 0) {
+        off[E] = P;
+        offsets[E] = P;
+        scalars[0] = P;
+        scalars[1] = n_active;
+        scalars[2] = *bad;
+        scalars[3] = 0;
+        if (stats_copy) {
+            stats_copy[0] = P;
+            stats_copy[1] = n_active;
+            stats_copy[2] = *bad;
+            stats_copy[3] = 0;
+        }
+    }
+    __syncthreads();
+
+    // stable scatter
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (long long base = 0; base < A; base += kAlignThreads) {
+        const long long a = base + tid;
+        int e = a < A ? ids[a] : -1;
+        if ((unsigned)e >= (unsigned)E) e = -1;
+        for (int i = tid; i < 32 * E; i += kAlignThreads) tbl[i] = 0;
+        __syncthreads();
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & lt_mask);
+        if (e >= 0 && lane == __ffs(peers) - 1) tbl[warp * E + e] = (uint16_t)__popc(peers);
+        __syncthreads();
+        if (tid < E) {
+            int run = 0;
+            for (int w = 0; w < 32; ++w) {
+                const int c = tbl[w * E + tid];
+                tbl[w * E + tid] = (uint16_t)run;
+                run += c;
+            }
+            rt[tid] = run;
+        }
+        __syncthreads();
+        if (e >= 0) {
+            const int p = cursor[e] + tbl[warp * E + e] + rank;
+            sorted_ids[p] = (int32_t)a;
+            pos[a] = p;
+        }
+        __syncthreads();
+        if (tid < E) cursor[tid] += rt[tid];
+        __syncthreads();
+    }
+
+    // padding slots inside each segment, then everything past P
+    for (int e = warp; e < E; e += kAlignThreads / 32)
+        for (int p = off[e] + cnt[e] + lane; p < off[e + 1]; p += 32) sorted_ids[p] = -1;
+    for (long long p = (long long)P + tid; p < P_max; p += kAlignThreads) sorted_ids[p] = -1;
+    const long long nblk = (P_max + B - 1) / B;
+    for (long long b = tid; b < nblk; b += kAlignThreads) {
+        const long long p = b * B;
+        int r = -1;
+        if (p < P) {
+            int lo = 0, hi = E - 1;  // largest e with off[e] <= p
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (off[mid] <= p) lo = mid;
+                else hi = mid - 1;
+            }
+            r = lo;
+        }
+        block_expert[b] = r;
+    }
+}
+
+int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids, int32_t* counts,
+                 int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
+                 int32_t* stats_copy, cudaStream_t stream) {
+    const size_t smem = sizeof(int) * (4 * (size_t)E + 1 + 34) + sizeof(uint16_t) * 32 * (size_t)E;
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return -3;
+        }
+        attr_done = true;
+    }
+    align_kernel<<<1, kAlignThreads, smem, stream>>>(T, K, E, B, P_max, ids, counts, offsets, sorted_ids,
+                                                     block_expert, pos, scalars, stats_copy);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+// ---------------------------------------------------------------- permute
+// x_perm[p] = x[sorted_ids[p] / K] (zero row for a padding slot), p < P.
+__global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const int4* __restrict__ x,
+                                                      const int32_t* __restrict__ sorted_ids,
+                                                      const int32_t* __restrict__ scalars, int4* __restrict__ x_perm) {
+    const int P = scalars[0];
+    const int rows_per_block = blockDim.x / 64;  // 64 threads per row
+    const int sub = threadIdx.x / 64, l = threadIdx.x % 64;
+    for (long long p = (long long)blockIdx.x * rows_per_block + sub; p < P; p += (long long)gridDim.x * rows_per_block) {
+        const int src = sorted_ids[p];
+        int4* dst = x_perm + p * row_vec;
+        if (src >= 0) {
+            const int4* s = x + (long long)(src / K) * row_vec;
+            for (int v = l; v < row_vec; v += 64) dst[v] = __ldg(s + v);
+        } else {
+            const int4 z = make_int4(0, 0, 0, 0);
+            for (int v = l; v < row_vec; v += 64) dst[v] = z;
+        }
+    }
+}
+
+int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
+                   const int32_t* scalars, void* x_perm, cudaStream_t stream) {
+    if (P_max <= 0) return 0;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    const int elt = dtype == 0 ? 2 : 4;
+    const int row_vec = H * elt / 16;
+    long long rows_per_block = 4;
+    long long blocks = (P_max + rows_per_block - 1) / rows_per_block;
+    const long long cap = (long long)d.num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    permute_kernel<<<(int)blocks, 256, 0, stream>>>(row_vec, K, static_cast<const int4*>(x), sorted_ids, scalars,
+                                                    static_cast<int4*>(x_perm));
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+// ---------------------------------------------------------------- combine
+// out[t] = sum_k w[t,k] * y_perm[pos[t*K+k]] (+ shared[t]), fp32, ascending k.
+template <typename T>
+struct Vec16 {
+    static constexpr int N = 16 / sizeof(T);
+};
+
+__device__ __forceinline__ void unpack(const int4& v, float* f, const __nv_bfloat16*) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+__device__ __forceinline__ void unpack(const int4& v, float* f, const float*) {
+    const float* x = reinterpret_cast<const float*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = x[i];
+}
+__device__ __forceinline__ int4 pack(const float* f, const __nv_bfloat16*) {
+    int4 v;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    return v;
+}
+__device__ __forceinline__ int4 pack(const float* f, const float*) {
+    int4 v;
+    float* x = reinterpret_cast<float*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = f[i];
+    return v;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K, const int4* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ pos, const float* __restrict__ w,
+                                                      const int4* __restrict__ sh, int4* __restrict__ out) {
+    constexpr int N = Vec16<T>::N;
+    __shared__ int s_pos[16];
+    __shared__ float s_w[16];
+    for (int t = blockIdx.x; t < T_; t += gridDim.x) {
+        __syncthreads();
+        if (threadIdx.x < K) {
+            s_pos[threadIdx.x] = pos[(long long)t * K + threadIdx.x];
+            s_w[threadIdx.x] = w[(long long)t * K + threadIdx.x];
+        }
+        __syncthreads();
+        for (int v = threadIdx.x; v < row_vec; v += blockDim.x) {
+            float acc[N];
+#pragma unroll
+            for (int i = 0; i < N; ++i) acc[i] = 0.f;
+            for (int k = 0; k < K; ++k) {
+                float y[N];
+                unpack(__ldg(y_perm + (long long)s_pos[k] * row_vec + v), y, (const T*)nullptr);
+                const float wk = s_w[k];
+#pragma unroll
+                for (int i = 0; i < N; ++i) acc[i] += wk * y[i];
+            }
+            if (sh) {
+                float y[N];
+                unpack(__ldg(sh + (long long)t * row_vec + v), y, (const T*)nullptr);
+#pragma unroll
+                for (int i = 0; i < N; ++i) acc[i] += y[i];
+            }
+            out[(long long)t * row_vec + v] = pack(acc, (const T*)nullptr);
+        }
+    }
+}
+
+int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
+                   const void* shared_out, void* out, cudaStream_t stream) {
+    if (T == 0) return 0;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    const int elt = dtype == 0 ? 2 : 4;
+    const int row_vec = H * elt / 16;
+    const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
+    long long blocks = T;
+    const long long cap = (long long)d.num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    if (dtype == 0)
+        combine_kernel<__nv_bfloat16><<<(int)blocks, threads, 0, stream>>>(
+            T, row_vec, K, static_cast<const int4*>(y_perm), pos, w, static_cast<const int4*>(shared_out),
+            static_cast<int4*>(out));
+    else
+        combine_kernel<float><<<(int)blocks, threads, 0, stream>>>(T, row_vec, K, static_cast<const int4*>(y_perm), pos,
+                                                                   w, static_cast<const int4*>(shared_out),
+                                                                   static_cast<int4*>(out));
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+}  // namespace moe

@@ -49,10 +49,13 @@ def lib():
         L.oracle_gate_weights.argtypes = [i, i, i, i, i, P, P, P]
         L.oracle_align.argtypes = [i, i, i, i, P, ctypes.c_int64, P, P, P, P, P, P, P]
         L.oracle_swiglu_ffn.argtypes = [i, i, i, P, P, P, P]
+        L.oracle_permute.argtypes = [i, i, i, P, P, i, P]
+        L.oracle_combine.argtypes = [i, i, i, i, P, P, P, P, P]
         L.oracle_dense_ffn.argtypes = [i, i, i, i, P, P, P, P, i]
         L.oracle_moe_layer.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, i, P, P, P, i]
         for f in (L.oracle_router_logits, L.oracle_topk, L.oracle_gate_weights, L.oracle_align,
-                  L.oracle_swiglu_ffn, L.oracle_dense_ffn, L.oracle_moe_layer):
+                  L.oracle_swiglu_ffn, L.oracle_dense_ffn, L.oracle_moe_layer, L.oracle_permute,
+                  L.oracle_combine):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -145,6 +148,32 @@ def align(ids, E, B, P_max=None):
            "align")
     return dict(counts=counts, offsets=offsets, sorted_ids=sorted_ids[:P_max],
                 block_expert=block_expert[:nblk], pos=pos[:T * K], P=int(P[0]), E_active=int(ea[0]))
+
+
+def permute(x, sorted_ids, K, P):
+    """x_perm[P,H] (float64): row p is x[sorted_ids[p] // K], zero for -1."""
+    x, dt = _typed(x)
+    sid = np.ascontiguousarray(sorted_ids, dtype=np.int32)
+    H = x.shape[1]
+    out = np.empty((P, H), np.float64)
+    _check(lib().oracle_permute(H, K, dt, _ptr(x), _ptr(sid), P, _ptr(out)), "permute")
+    return out
+
+
+def combine(y, pos, w, shared=None):
+    """out[T,H] (float64) = sum_k w[t,k] * y[pos[t*K+k]] (+ shared[t])."""
+    y, dt = _typed(y)
+    pos = np.ascontiguousarray(pos, dtype=np.int32).ravel()
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    T, K = w.shape
+    H = y.shape[1]
+    sh = None
+    if shared is not None:
+        sh, d2 = _typed(shared)
+        assert d2 == dt
+    out = np.empty((T, H), np.float64)
+    _check(lib().oracle_combine(T, H, K, dt, _ptr(y), _ptr(pos), _ptr(w), _ptr(sh), _ptr(out)), "combine")
+    return out
 
 
 def swiglu_ffn(x_row, w13, w2):

@@ -190,6 +190,40 @@ int oracle_align(int T, int K, int E, int B, const int32_t* ids, int64_t P_max,
     return 0;
 }
 
+/* ---------------------------------------------------------------- permute */
+/* x_perm[p] = x[sorted_ids[p] / K] for p < P; a zero row where sorted_ids[p]
+ * is -1 (a padding slot).  Rows are H elements of `dtype`; the output is
+ * double. */
+int oracle_permute(int H, int K, int dtype, const void* x, const int32_t* sorted_ids, int P,
+                   double* x_perm)
+{
+    if (H <= 0 || K <= 0 || P < 0) return -1;
+    for (int p = 0; p < P; ++p) {
+        int a = sorted_ids[p];
+        for (int h = 0; h < H; ++h)
+            x_perm[(size_t)p * H + h] = a < 0 ? 0.0 : ld(x, (size_t)(a / K) * H + h, dtype);
+    }
+    return 0;
+}
+
+/* --------------------------------------------------------------- combine */
+/* Local sum: out[t] = sum_{k=0..K-1} w[t][k] * y[pos[t*K+k]] + shared[t]
+ * (shared may be NULL).  y and shared rows are H elements of `dtype`. */
+int oracle_combine(int T, int H, int K, int dtype, const void* y, const int32_t* pos,
+                   const double* w, const void* shared, double* out)
+{
+    if (T < 0 || H <= 0 || K <= 0) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h) {
+            double s = 0.0;
+            for (int k = 0; k < K; ++k)
+                s += w[(size_t)t * K + k] * ld(y, (size_t)pos[(size_t)t * K + k] * H + h, dtype);
+            if (shared) s += ld(shared, (size_t)t * H + h, dtype);
+            out[(size_t)t * H + h] = s;
+        }
+    return 0;
+}
+
 /* ------------------------------------------------------------- SwiGLU FFN */
 /* One token through one SwiGLU expert.  w13 is [2I, H]: rows 0..I-1 are the
  * gate projection W1, rows I..2I-1 the up projection W3; w2 is [H, I].

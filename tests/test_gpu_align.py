@@ -1,0 +1,96 @@
+"""Alignment with block-wise padding, permute and combine on the GPU against the
+oracle: every index output bit-exact (counts, offsets, sorted_ids,
+block_expert, pos, P, E_active), the permute an exact row copy, the combine
+within fp32 rounding."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import mixture_experts_layer_61_b200 as moe
+import oracle
+from helpers import host
+
+pytestmark = pytest.mark.gpu
+
+
+def _ids(T, E, K, seed, kind="uniform"):
+    if kind == "uniform":
+        lg = mi.zipf_gumbel_logits(E, T, 0.0, seed).numpy()
+    elif kind == "zipf":
+        lg = mi.zipf_gumbel_logits(E, T, 1.5, seed).numpy()
+    elif kind == "one":       # every token's first choice is expert 0
+        lg = mi.zipf_gumbel_logits(E, T, 0.0, seed).numpy()
+        lg[:, 0] = 1e30
+    else:
+        lg = mi.tie_heavy_logits(T, E, seed, levels=1)
+    return oracle.topk(lg, K)
+
+
+def _check_align(T, E, K, B, ids_np):
+    cfg = moe.config(T, 64, E, K, 64, tile_B=B)
+    ids = torch.from_numpy(ids_np).cuda()
+    g = moe.align_pad(cfg, ids)
+    torch.cuda.synchronize()
+    r = oracle.align(ids_np, E, B)
+    for key in ("counts", "offsets", "sorted_ids", "block_expert", "pos"):
+        assert np.array_equal(g[key].cpu().numpy(), r[key]), key
+    sc = g["scalars"].cpu().numpy()
+    assert sc[0] == r["P"] and sc[1] == r["E_active"] and sc[2] == 0
+    return g, r
+
+
+@pytest.mark.parametrize("T,E,K,B", [(1, 8, 2, 16), (64, 8, 2, 16), (128, 64, 8, 16), (1024, 256, 8, 16),
+                                     (4096, 256, 8, 16), (2048, 8, 2, 128), (333, 64, 8, 32), (50, 1024, 16, 8),
+                                     (7, 5, 5, 1), (129, 8, 2, 256)])
+@pytest.mark.parametrize("kind", ["uniform", "zipf", "one", "ties"])
+def test_align_bit_exact(T, E, K, B, kind):
+    _check_align(T, E, K, B, _ids(T, E, K, seed=T + E + B, kind=kind))
+
+
+def test_align_empty():
+    cfg = moe.config(0, 64, 8, 2, 64)
+    ids = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    g = moe.align_pad(cfg, ids)
+    torch.cuda.synchronize()
+    assert g["counts"].sum().item() == 0 and g["scalars"][0].item() == 0
+    assert g["offsets"].cpu().tolist() == [0] * 9
+
+
+def test_align_flags_bad_ids():
+    cfg = moe.config(3, 64, 4, 2, 64, tile_B=4)
+    ids = torch.tensor([[0, 1], [2, 9], [-1, 3]], dtype=torch.int32, device="cuda")
+    g = moe.align_pad(cfg, ids)
+    torch.cuda.synchronize()
+    assert g["scalars"][2].item() != 0
+    assert g["counts"].cpu().tolist() == [1, 1, 1, 1]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("T,E,K,B,H", [(64, 8, 2, 16, 256), (300, 64, 8, 16, 520), (1, 8, 2, 16, 4096)])
+def test_permute_and_combine(dtype, T, E, K, B, H):
+    ids_np = _ids(T, E, K, seed=T * 3 + E)
+    g, r = _check_align(T, E, K, B, ids_np)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    cfg = moe.config(T, H, E, K, 64, tile_B=B, dtype=tdt)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(T)
+    x = torch.randn((T, H), generator=gen, device="cuda").to(tdt)
+    Pm = moe.padded_rows_max(cfg)
+    xp = torch.full((Pm, H), 7.0, dtype=tdt, device="cuda")
+    moe.permute(cfg, x, g["sorted_ids"], g["scalars"], xp)
+    torch.cuda.synchronize()
+    P = r["P"]
+    ref = oracle.permute(host(x), r["sorted_ids"], K, P)
+    assert np.array_equal(xp[:P].float().cpu().numpy().astype(np.float64), ref)
+    assert torch.all(xp[P:] == 7.0)          # rows past P untouched
+    # combine with random gate weights and a shared term
+    y = torch.randn((Pm, H), generator=gen, device="cuda").to(tdt)
+    w = torch.rand((T, K), generator=gen, device="cuda")
+    sh = torch.randn((T, H), generator=gen, device="cuda").to(tdt)
+    for shared in (None, sh):
+        out = moe.combine(cfg, y, g["pos"], w, shared)
+        torch.cuda.synchronize()
+        refc = oracle.combine(host(y), r["pos"], w.cpu().double().numpy(), None if shared is None else host(sh))
+        err = np.abs(out.float().cpu().numpy() - refc).max() / np.abs(refc).max()
+        assert err < (8e-3 if dtype == "bf16" else 1e-6), err

@@ -1,0 +1,112 @@
+"""The tcgen05 grouped GEMM path (gate/up + SwiGLU, down) and the dense FFN on
+the GPU against the oracle, across token-tile caps (32..256 tokens), data-
+parallel and stream-K schedules, ragged feature blocks and skewed groups.
+Bound: max|out - ref| / max|ref| <= 2e-2."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import mixture_experts_layer_61_b200 as moe
+import oracle
+from helpers import OUT_TOL, cfg_for, host, rel_err, sample_tokens, small_shape
+
+pytestmark = pytest.mark.gpu
+
+
+def _grouped(shape, T, seed, kind="uniform", n_check=96):
+    w = mi.make_weights(shape, seed, device="cuda", shared=False)
+    x = mi.make_x(shape, T, seed, device="cuda")
+    if kind == "uniform":
+        lg = mi.zipf_gumbel_logits(shape.E, T, 0.0, seed).numpy()
+    else:
+        lg = mi.zipf_gumbel_logits(shape.E, T, 1.5, seed).numpy()
+        lg[: T // 2, 0] = 1e30
+    cfg = cfg_for(shape, T)
+    ids = oracle.topk(lg, shape.K)
+    g = moe.align_pad(cfg, torch.from_numpy(ids).cuda())
+    xp = moe.permute(cfg, x, g["sorted_ids"], g["scalars"])
+    ws = moe.alloc_workspace(moe.gemm_workspace_size())
+    y, act = moe.grouped_ffn(cfg, xp, w["w13"], w["w2"], g["offsets"], ws)
+    moe.check_status(ws)
+    # oracle: each checked row through its expert (rows of one token are independent)
+    r = oracle.align(ids, shape.E, shape.tile_B)
+    sid = r["sorted_ids"]
+    rows = np.nonzero(sid >= 0)[0]
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(rows, size=min(n_check, len(rows)), replace=False))
+    xh = host(x)
+    w13h, w2h = host(w["w13"]), host(w["w2"])
+    yh = y.float().cpu().numpy()
+    ref = np.stack([oracle.swiglu_ffn(xh[sid[p] // shape.K], w13h[ids.ravel()[sid[p]]], w2h[ids.ravel()[sid[p]]])
+                    for p in rows])
+    return rel_err(yh[rows], ref)
+
+
+@pytest.mark.parametrize("T", [1, 5, 64, 200, 400, 1200])
+def test_grouped_bf16_tile_caps(T):
+    # rows per expert T*K/E picks the token-tile cap: <=24 -> 32, <=56 -> 64, <=112 -> 128, else 256
+    shape = small_shape(H=512, E=8, K=2, I=1024)
+    assert _grouped(shape, T, seed=T) < OUT_TOL
+
+
+def test_grouped_fp32_tiny_config():
+    shape = mi.SHAPES["tiny"]
+    assert _grouped(shape, 64, seed=0, n_check=128) < OUT_TOL
+
+
+@pytest.mark.parametrize("kind", ["uniform", "skew"])
+def test_grouped_many_experts(kind):
+    shape = small_shape(H=1024, E=64, K=8, I=512)
+    assert _grouped(shape, 150, seed=11, kind=kind) < OUT_TOL
+
+
+def test_grouped_ragged_features():
+    # I and H not multiples of the 128-row weight block, H not of the 64-element K step
+    shape = small_shape(H=264, E=6, K=2, I=200)
+    assert _grouped(shape, 77, seed=5) < OUT_TOL
+
+
+def test_grouped_one_hot_expert_many_chunks():
+    # half the tokens on expert 0: several token chunks share one weight block
+    shape = small_shape(H=256, E=4, K=1, I=384)
+    assert _grouped(shape, 1000, seed=2, kind="skew") < OUT_TOL
+
+
+@pytest.mark.parametrize("T,H,I", [(1, 512, 1024), (16, 256, 640), (300, 1024, 2048), (700, 512, 14336)])
+def test_dense_ffn(T, H, I):
+    # (700, 512, 14336): 3 chunks x 112 feature blocks -> data-parallel waves plus a stream-K tail
+    w13, w2 = mi.make_dense_weights(H, I, torch.bfloat16, seed=T + I, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(T)
+    x = torch.randn((T, H), generator=gen, device="cuda").to(torch.bfloat16)
+    ws = moe.alloc_workspace(moe.dense_workspace_size(T, H, I))
+    out = moe.dense_ffn(x, w13, w2, ws)
+    moe.check_status(ws)
+    tok = sample_tokens(T, 48, seed=T)
+    ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
+    assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
+
+
+def test_dense_ffn_fp32_tf32():
+    T, H, I = 40, 256, 512
+    w13, w2 = mi.make_dense_weights(H, I, torch.float32, seed=1, device="cuda")
+    x = torch.randn((T, H), device="cuda")
+    ws = moe.alloc_workspace(moe.dense_workspace_size(T, H, I, moe.FP32))
+    out = moe.dense_ffn(x, w13, w2, ws)
+    moe.check_status(ws)
+    ref = oracle.dense_ffn(host(x), host(w13), host(w2))
+    assert rel_err(out.cpu().numpy(), ref) < OUT_TOL
+
+
+def test_deterministic_repeat():
+    # the stream-K fixup sums partial tiles in a fixed order: bitwise-equal reruns
+    shape = small_shape(H=1024, E=8, K=2, I=2048)
+    w = mi.make_weights(shape, 4, device="cuda", shared=False)
+    x = mi.make_x(shape, 3, 4, device="cuda")
+    cfg = cfg_for(shape, 3)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    o1 = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws).clone()
+    o2 = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws).clone()
+    moe.check_status(ws)
+    assert torch.equal(o1, o2)

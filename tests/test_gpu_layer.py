@@ -1,0 +1,95 @@
+"""Whole-layer parity: moe_layer_forward on the GPU against the oracle's layer
+(router -> top-K -> gate weights -> SwiGLU experts -> weighted sum + shared).
+The oracle routes on the GPU's own fp32 logits, so that a near-tie flipped by
+fp32 rounding of x.W_r cannot diverge the two (the logits themselves are
+checked in test_gpu_route).  Small shapes are checked on every token; the
+full Mixtral-, Qwen2-MoE- and DeepSeek-V3-shaped layers on a seeded sample of
+256 tokens (the layer is token-wise independent given the logits), in the
+launch configuration the benchmark times."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import mixture_experts_layer_61_b200 as moe
+import oracle
+from helpers import OUT_TOL, cfg_for, host, rel_err, sample_tokens, small_shape
+
+pytestmark = pytest.mark.gpu
+
+N_SAMPLE = int(os.environ.get("MOE_TEST_SAMPLE", "256"))
+
+
+def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True):
+    w = mi.make_weights(shape, seed, device="cuda")
+    x = mi.make_x(shape, T, seed, device="cuda")
+    cfg = cfg_for(shape, T)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    stats = torch.zeros(4, dtype=torch.int32, device="cuda")
+    out = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w.get("w13_sh"), w.get("w2_sh"),
+                            logits_override=override, stats=stats)
+    moe.check_status(ws)
+    if override is None:
+        gws = moe.alloc_workspace(moe.gemm_workspace_size())
+        logits = moe.router_gemm(cfg, x, w["w_r"], gws)
+        moe.check_status(gws)
+        lg = logits.cpu().numpy()
+    else:
+        lg = override.cpu().numpy()
+    ids = oracle.topk(lg, shape.K)
+    if check_stats:
+        r = oracle.align(ids, shape.E, shape.tile_B)
+        st = stats.cpu().numpy()
+        assert st[0] == r["P"] and st[1] == r["E_active"] and st[2] == 0
+    tok = sample_tokens(T, n_sample or T, seed)
+    sh = {}
+    if shape.I_sh:
+        sh = dict(w13_sh=host(w["w13_sh"]), w2_sh=host(w["w2_sh"]))
+    ref = oracle.moe_layer(host(x), None, host(w["w13"]), host(w["w2"]), shape.K, shape.score_fn,
+                           shape.renorm, logits=lg, tokens=tok, **sh)
+    return rel_err(out.float().cpu().numpy()[tok], ref)
+
+
+def test_layer_tiny_fp32_all_tokens():
+    assert _run_layer(mi.SHAPES["tiny"], 64, seed=0) < OUT_TOL
+
+
+@pytest.mark.parametrize("score_fn,renorm", [(0, 1), (0, 0), (1, 1), (1, 0)])
+def test_layer_small_gating_variants(score_fn, renorm):
+    shape = small_shape(H=512, E=16, K=4, I=768, I_sh=256, score_fn=score_fn, renorm=renorm)
+    assert _run_layer(shape, 96, seed=score_fn * 2 + renorm) < OUT_TOL
+
+
+@pytest.mark.parametrize("T", [1, 3, 130])
+def test_layer_small_shapes_ragged_T(T):
+    shape = small_shape(H=256, E=8, K=2, I=512, B=16)
+    assert _run_layer(shape, T, seed=T) < OUT_TOL
+
+
+@pytest.mark.parametrize("B", [1, 8, 128])
+def test_layer_padding_tiles(B):
+    shape = small_shape(H=256, E=8, K=2, I=512, B=B)
+    assert _run_layer(shape, 100, seed=B) < OUT_TOL
+
+
+def test_layer_skewed_logits_override():
+    shape = small_shape(H=1024, E=64, K=8, I=256, I_sh=512, score_fn=1)
+    lg = mi.zipf_gumbel_logits(64, 200, 1.5, seed=3, device="cuda")
+    assert _run_layer(shape, 200, seed=3, override=lg) < OUT_TOL
+
+
+@pytest.mark.parametrize("name,T", [("mixtral", 1), ("mixtral", 32), ("mixtral", 2048), ("qwen2moe", 128),
+                                    ("qwen2moe", 1024), ("deepseekv3", 32), ("deepseekv3", 1024)])
+def test_layer_full_size_sampled(name, T):
+    shape = mi.SHAPES[name]
+    assert _run_layer(shape, T, seed=mi.seed_for(shape, T), n_sample=N_SAMPLE) < OUT_TOL
+
+
+@pytest.mark.parametrize("s", [0.0, 1.5])
+def test_layer_deepseek_skew_sweep_point(s):
+    shape = mi.SHAPES["deepseekv3"]
+    T = 256
+    lg = mi.zipf_gumbel_logits(shape.E, T, s, seed=4000 + T, device="cuda")
+    assert _run_layer(shape, T, seed=mi.seed_for(shape, T, 5), override=lg, n_sample=64) < OUT_TOL

@@ -216,6 +216,43 @@ def test_align_rejects_bad_ids():
         oracle.align(np.array([[0, 5]], np.int32), 4, 4)
 
 
+# ----------------------------------------------------- permute / combine
+
+def test_permute_then_combine_with_unit_weights_is_identity():
+    # un-permuting the permuted rows by pos with w = 1 and K = 1 returns x;
+    # padding rows of the permuted matrix are zero.
+    rng = np.random.default_rng(7)
+    T, E, B = 23, 5, 4
+    x = rng.standard_normal((T, 6)).astype(np.float32)
+    ids = rng.integers(0, E, size=(T, 1)).astype(np.int32)
+    r = oracle.align(ids, E, B)
+    xp = oracle.permute(x, r["sorted_ids"], 1, r["P"])
+    pad = r["sorted_ids"][:r["P"]] < 0
+    assert np.all(xp[pad] == 0.0)
+    back = oracle.combine(xp.astype(np.float32), r["pos"], np.ones((T, 1)))
+    assert np.array_equal(back, x.astype(np.float64))
+
+
+def test_combine_closed_form_and_shared():
+    # K = 2 rows with weights 3/4, 1/4 of constant rows c1, c2 give 3/4 c1 + 1/4 c2,
+    # and the shared row is added once.
+    y = np.array([[1.0, 1.0], [5.0, 5.0], [-2.0, 4.0]], np.float32)
+    pos = np.array([[1, 0], [2, 1]], np.int32)
+    w = np.array([[0.75, 0.25], [0.5, 0.5]])
+    sh = np.array([[10.0, 0.0], [0.0, -1.0]], np.float32)
+    out = oracle.combine(y, pos, w, sh)
+    assert out.tolist() == [[0.75 * 5 + 0.25 * 1 + 10.0, 0.75 * 5 + 0.25 * 1], [0.5 * -2 + 0.5 * 5, 0.5 * 4 + 0.5 * 5 - 1.0]]
+
+
+def test_permute_golden():
+    g = _load("align_small.json")
+    T, K = g["T"], g["K"]
+    x = np.arange(T * 3, dtype=np.float32).reshape(T, 3)
+    xp = oracle.permute(x, np.array(g["sorted_ids"], np.int32), K, g["P"])
+    for p, a in enumerate(g["sorted_ids"][:g["P"]]):
+        assert xp[p].tolist() == ([0.0] * 3 if a < 0 else x[a // K].tolist())
+
+
 # -------------------------------------------------------------- FFN math
 
 def _perm_matrix(perm):
