@@ -70,12 +70,9 @@ class ClockSampler:
         try:
             import pynvml
             pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id if hasattr(
-                torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
-            if bus:
-                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-            else:
-                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08X:%02X:%02X.0" % (int(props.pci_domain_id), int(props.pci_bus_id), int(props.pci_device_id))
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
             self._nv = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:
@@ -86,7 +83,9 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                r = get(self._h)
                 for bit, name in self.REASONS.items():
                     if r & bit:
                         self.reasons.add(name)
