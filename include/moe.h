@@ -104,6 +104,24 @@ size_t moe_gemm_workspace_size(void);
 int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router,
                     float* logits, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* Router GEMM for callers that cannot allocate device memory when they
+ * enqueue work -- for example a plugin inside another engine whose enqueue
+ * step must not allocate, or code captured into a CUDA graph under a mode
+ * that forbids cudaMalloc.  The pages have no counterpart: this is a library
+ * convenience, not a step of the method.
+ *   Same result and arguments as moe_router_gemm, minus the workspace: the
+ *   scratch (status word, stream-K counters, partial tiles) lives in a fixed
+ *   ~5 MiB array in the library's device memory, present on every GPU that
+ *   loads the library until the process exits.  No allocation is made.
+ *   Limits: T <= 32 (larger T returns MOE_ERR_ARG: use moe_router_gemm) and
+ *   at most 160 SMs.  The first call on each device looks up the array's
+ *   device address (cudaGetSymbolAddress); make that first call before any
+ *   stream capture.  Each call clears the shared control words before its
+ *   launch; calls that overlap on the GPU (unordered streams) race on the
+ *   shared array.  A device wait that runs out leaves logits unwritten. */
+int moe_router_gemm_noalloc(const moe_config_t* cfg, const void* x, const void* w_router,
+                            float* logits, moe_stream_t stream);
+
 /* Top-K gating (stage "top-K selection"), one token per warp:
  *   topk_ids[T,K]: the K largest logits[t,:], descending, the lower expert
  *     index first on equal values (IEEE comparison: -0.0 ties +0.0; +-inf are
