@@ -150,6 +150,22 @@ class Workload:
         self.s_sh = torch.empty((T, shape.H), dtype=dt, device=device) if shape.I_sh else None
         self.s_shws = (moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, shape.I_sh, self.cfg.dtype), device)
                        if shape.I_sh else None)
+        self.s_al = moe.align_buffers(self.cfg, device)
+
+    def capture(self):
+        """Record one forward into a CUDA graph (the library makes no allocation
+        or synchronisation inside a call, so the whole layer is capturable)."""
+        self.step()  # first call outside capture: one-time kernel attribute setup
+        torch.cuda.synchronize()
+        n0 = self.moe.kernel_launch_count()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        self.launches_per_step = self.moe.kernel_launch_count() - n0
+        torch.cuda.synchronize()
+
+    def replay(self):
+        self.graph.replay()
 
     def step(self):
         m = self.moe
@@ -164,7 +180,7 @@ class Workload:
         ev[1].record()
         m.route(c, self.logits if self.logits is not None else self.s_logits, self.s_ids, self.s_w)
         ev[2].record()
-        self.al = m.align_pad(c, self.s_ids)
+        self.al = m.align_pad(c, self.s_ids, self.s_al)
         ev[3].record()
         m.permute(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
         ev[4].record()
@@ -182,7 +198,9 @@ class Workload:
 
 
 def l2_flush_buffer(device):
-    size = max(512 << 20, 4 * torch.cuda.get_device_properties(device).L2_cache_size)
+    """2 GiB (16x the L2): writing it evicts the L2, and it keeps the GPU busy
+    long enough for the host to enqueue a whole step behind it."""
+    size = max(2 << 30, 16 * torch.cuda.get_device_properties(device).L2_cache_size)
     return torch.empty(size // 4, dtype=torch.float32, device=device)
 
 
@@ -226,11 +244,15 @@ def dense_times(shape, T, I_d, steps, warmup, flush, device, seed):
     x = mi.make_x(shape, T, seed, device=device)
     ws = moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, I_d, 0 if shape.dtype == "bf16" else 1), device)
     out = torch.empty_like(x)
-    fn = lambda: moe.dense_ffn(x, w13, w2, ws, out)
-    for _ in range(warmup):
-        fn()
+    moe.dense_ffn(x, w13, w2, ws, out)
     torch.cuda.synchronize()
-    t = time_steps(fn, steps, flush)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.dense_ffn(x, w13, w2, ws, out)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    t = time_steps(g.replay, steps, flush)
     moe.check_status(ws)
     del w13, w2, ws
     return statistics.median(t)
@@ -289,6 +311,11 @@ def main():
     ap.add_argument("--no-tau", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="also time every configured workload")
     ap.add_argument("--sweep-out", default=None)
+    ap.add_argument("--quick", action="store_true",
+                    help="only the timed region (for profiler captures): no breakdown, e2e, tau or CPU baseline")
+    ap.add_argument("--no-graph", action="store_true", help="launch each step from the host instead of a CUDA graph")
+    ap.add_argument("--token-tile-cap", type=int, default=0, help="grouped GEMM token-tile cap (0 = automatic)")
+    ap.add_argument("--no-pdl", action="store_true", help="plain stream order between kernels")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -309,10 +336,20 @@ def main():
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     pk, pk_kind = peaks()
+    import mixture_experts_layer_61_b200 as moe
+    if args.token_tile_cap:
+        moe.set_token_tile_cap(args.token_tile_cap)
+    if args.no_pdl:
+        moe.set_programmatic_launch(False)
     wl = Workload(shape, T, rank, device, skew=args.skew)
     flush = l2_flush_buffer(device)
+    if args.no_graph:
+        run_step, wl.launches_per_step = wl.step, None
+    else:
+        wl.capture()
+        run_step = wl.replay
     for _ in range(args.warmup):
-        wl.step()
+        run_step()
     torch.cuda.synchronize()
     wl.moe.check_status(wl.ws)
 
@@ -322,9 +359,11 @@ def main():
     torch.cuda.synchronize()
     n0 = wl.moe.kernel_launch_count()
     with ClockSampler(local) as clk:
-        times = time_steps(wl.step, args.steps, flush)
+        times = time_steps(run_step, args.steps, flush)
     torch.cuda.synchronize()
     launches = wl.moe.kernel_launch_count() - n0
+    if not args.no_graph:
+        launches = wl.launches_per_step * args.steps  # graph replays launch the captured kernels
     if dist:
         dist.barrier()
     total_ms = sum(times)
@@ -337,7 +376,6 @@ def main():
     P, E_active = stats[0], stats[1]
     ms_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms / 1e3)
-
     # ---- per-stage breakdown (same kernels, one ABI call per stage)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
     stage_ms = {s: [] for s in Workload.STAGES}
@@ -350,6 +388,19 @@ def main():
                 stage_ms[s].append(ev[j].elapsed_time(ev[j + 1]))
     wl.moe.check_status(wl.gws)
     stages = {s: round(statistics.median(v), 4) for s, v in stage_ms.items()}
+
+    if args.quick:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+                              "quick": True, "config": {"workload": f"{shape.name}:{T}",
+                                                        "token_tile_cap": args.token_tile_cap,
+                                                        "pdl": not args.no_pdl},
+                              "stages_ms": stages, "E_active": E_active, "P": P}), flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # ---- roofline of the dominant kernel (grouped gate/up + SwiGLU)
     gu_bytes, gu_flops = gate_up_work(shape, T, E_active)
@@ -379,7 +430,7 @@ def main():
 
     def e2e_step():
         wl.x.copy_(x_host, non_blocking=True)
-        wl.step()
+        run_step()
         out_host.copy_(wl.out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -434,7 +485,8 @@ def main():
                    "E": shape.E, "K": shape.K, "I": shape.I, "I_shared": shape.I_sh, "tile_B": shape.tile_B,
                    "score_fn": "softmax" if shape.score_fn == 0 else "sigmoid", "global_batch": T * world,
                    "parallelism": f"replicas x{world} (data parallel, no collective)",
-                   "l2": "flushed between steps (512 MiB write outside the events); weights exceed L2"},
+                   "launch": "host launches" if args.no_graph else "CUDA graph replay of moe_layer_forward",
+                   "l2": "flushed between steps (2 GiB write outside the events); weights exceed L2"},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - T * shape.K) / max(P, 1), 4),
                   "bytes_alg": B_alg, "flops_alg": F_alg, "roofline_frac": round(layer_roof, 4),
@@ -473,10 +525,11 @@ def run_sweep(args, device, flush, pk):
     fa_cache = {}
     for sh, T, s in plan:
         wl = Workload(sh, T, 0, device, skew=s)
+        wl.capture()
         for _ in range(3):
-            wl.step()
+            wl.replay()
         torch.cuda.synchronize()
-        t = statistics.median(time_steps(wl.step, steps, flush))
+        t = statistics.median(time_steps(wl.replay, steps, flush))
         moe.check_status(wl.ws)
         st = wl.stats.cpu().tolist()
         B, F = algorithmic(sh, T, st[1])

@@ -213,6 +213,18 @@ int moe_check_status(void* workspace, moe_stream_t stream);
  * 2e9 = 2 s; 0 restores the default).  Process-wide. */
 void moe_set_wait_limit_ns(uint64_t ns);
 
+/* Tuning: force the grouped GEMM's token-tile cap (tokens per MMA tile) to
+ * 32, 64, 128 or 256 for subsequent launches; 0 (default) picks it from the
+ * expected rows per expert, T*K/E.  Results are unchanged; only speed
+ * differs.  Process-wide.  Returns MOE_ERR_ARG for other values. */
+int moe_set_token_tile_cap(int n);
+
+/* Programmatic dependent launch (default on): each kernel may start its
+ * prologue while the previous kernel on the stream drains, and waits for it
+ * before touching its output.  0 turns it off (plain stream order) for
+ * subsequent launches.  Process-wide; results are identical either way. */
+void moe_set_programmatic_launch(int enable);
+
 /* Test hook: when nonzero, the next GEMM launch withholds the first operand
  * load of block 0, so that block's waits run out and report
  * MOE_ERR_TIMEOUT through moe_check_status().  Cleared after one launch. */

@@ -74,6 +74,8 @@ def lib():
             "moe_check_status": (I, [P, P]),
             "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
             "moe_debug_withhold_first_load": (None, [I]),
+            "moe_set_token_tile_cap": (I, [I]),
+            "moe_set_programmatic_launch": (None, [I]),
             "moe_kernel_launch_count": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
@@ -161,17 +163,25 @@ def route(cfg, logits, ids=None, w=None):
     return ids, w
 
 
-def align_pad(cfg, ids):
-    _need_cuda(ids)
-    dev = ids.device
+def align_buffers(cfg, device):
+    """Output buffers of align_pad for this configuration."""
     Pm = padded_rows_max(cfg)
     nblk = (Pm + cfg.tile_B - 1) // cfg.tile_B
-    out = dict(counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
-               offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
-               sorted_ids=torch.empty(max(Pm, 1), dtype=torch.int32, device=dev),
-               block_expert=torch.empty(max(nblk, 1), dtype=torch.int32, device=dev),
-               pos=torch.empty(max(cfg.T * cfg.K, 1), dtype=torch.int32, device=dev),
-               scalars=torch.zeros(4, dtype=torch.int32, device=dev))
+    return dict(counts=torch.empty(cfg.E, dtype=torch.int32, device=device),
+                offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=device),
+                sorted_ids=torch.empty(max(Pm, 1), dtype=torch.int32, device=device),
+                block_expert=torch.empty(max(nblk, 1), dtype=torch.int32, device=device),
+                pos=torch.empty(max(cfg.T * cfg.K, 1), dtype=torch.int32, device=device),
+                scalars=torch.zeros(4, dtype=torch.int32, device=device))
+
+
+def align_pad(cfg, ids, out=None):
+    _need_cuda(ids)
+    Pm = padded_rows_max(cfg)
+    nblk = (Pm + cfg.tile_B - 1) // cfg.tile_B
+    if out is None:
+        out = align_buffers(cfg, ids.device)
+    out = dict(out)
     _check(lib().moe_align_pad(ctypes.byref(cfg), _p(ids), _p(out["counts"]), _p(out["offsets"]),
                                _p(out["sorted_ids"]), _p(out["block_expert"]), _p(out["pos"]),
                                _p(out["scalars"]), _stream()), "moe_align_pad")
@@ -255,6 +265,16 @@ def check_status(ws):
 
 def set_wait_limit_ns(ns):
     lib().moe_set_wait_limit_ns(int(ns))
+
+
+def set_token_tile_cap(n):
+    """Force the grouped GEMM's token-tile cap (32/64/128/256; 0 = automatic)."""
+    _check(lib().moe_set_token_tile_cap(int(n)), "moe_set_token_tile_cap")
+
+
+def set_programmatic_launch(enable=True):
+    """Programmatic dependent launch between the layer's kernels (default on)."""
+    lib().moe_set_programmatic_launch(1 if enable else 0)
 
 
 def debug_withhold_first_load(enable=True):

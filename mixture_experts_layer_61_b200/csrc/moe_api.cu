@@ -22,6 +22,10 @@ int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, -1 unsupported
 std::mutex g_dev_mu;
 }  // namespace
 
+std::atomic<bool> g_pdl{true};
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed); }
+void set_pdl(bool on) { g_pdl.store(on); }
+
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t wait_limit_ns() { return g_wait_limit.load(std::memory_order_relaxed); }
 int take_withhold_flag() { return g_withhold.exchange(0); }
@@ -186,6 +190,14 @@ int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_g
     return launch_gemm(down_launch(act, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w2, y, max_n), ctl, s);
 }
 
+// The router's output has only E features, so its tiles are few: cut the
+// tokens into 64-row tiles (32 for decode batches) and let up to 8 blocks
+// share a tile, so that more SMs stream x.
+void router_tiling(GemmLaunch& g, int T) {
+    g.max_n = T > 32 ? 64 : 32;
+    g.max_split = 8;
+}
+
 int routed_max_n(const moe_config_t* c) {
     return pick_max_n((double)c->T * c->K / (double)c->E);
 }
@@ -256,7 +268,7 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
     g.out = logits;
     g.out_ld = cfg->E;
     g.dtype = cfg->dtype;
-    g.max_n = pick_max_n(cfg->T);
+    router_tiling(g, cfg->T);
     return status_of(launch_gemm(g, gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
 }
 
@@ -399,7 +411,7 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
         g.out = logits;
         g.out_ld = cfg->E;
         g.dtype = cfg->dtype;
-        g.max_n = pick_max_n(cfg->T);
+        router_tiling(g, cfg->T);
         if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
     }
     if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, logits_override ? logits_override : logits,
@@ -469,6 +481,14 @@ int moe_check_status(void* workspace, moe_stream_t stream) {
 }
 
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit.store(ns ? ns : 2000000000ull); }
+
+int moe_set_token_tile_cap(int n) {
+    if (n != 0 && n != 32 && n != 64 && n != 128 && n != 256) return MOE_ERR_ARG;
+    set_token_tile_cap(n);
+    return MOE_OK;
+}
+
+void moe_set_programmatic_launch(int enable) { set_pdl(enable != 0); }
 
 void moe_debug_withhold_first_load(int enable) { g_withhold.store(enable ? 1 : 0); }
 

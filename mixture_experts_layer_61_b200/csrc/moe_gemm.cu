@@ -44,10 +44,10 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void*
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, typename OutT, bool kSwiGLU, int kMaxN>
+template <typename T, typename OutT, int kEpi, int kMaxN>
 int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t stream) {
-    using C = GemmCfg<T, kSwiGLU, kMaxN>;
-    auto kern = moe_gemm_kernel<T, OutT, kSwiGLU, kMaxN>;
+    using C = GemmCfg<T, kEpi, kMaxN>;
+    auto kern = moe_gemm_kernel<T, OutT, kEpi, kMaxN>;
     static bool attr_done = false;  // per instantiation
     if (!attr_done) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
@@ -56,9 +56,11 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
         }
         attr_done = true;
     }
-    CUtensorMap tm_w, tm_x;
+    CUtensorMap tm_w, tm_x, tm_x64, tm_xbig;
     if (!make_map(&tm_w, Elt<T>::kTma, Elt<T>::kBytes, L.w, L.w_rows, L.kdim, 128)) return -3;
     if (!make_map(&tm_x, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxRows)) return -3;
+    if (!make_map(&tm_x64, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxMid)) return -3;
+    if (!make_map(&tm_xbig, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, kMaxN)) return -3;
     GemmParams p;
     p.seg_offsets = L.seg_offsets;
     p.n_groups = L.n_groups;
@@ -75,20 +77,32 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
     p.wait_limit_ns = wait_limit_ns();
     p.withhold_first_load = take_withhold_flag();
     p.sk_min_units = 4;
-    kern<<<num_sms, kGemmThreads, C::kSmemBytes, stream>>>(tm_w, tm_x, p);
+    p.max_split = L.max_split > 0 ? L.max_split : 4;
+    cudaError_t e = launch_kernel(kern, dim3(num_sms), dim3(kGemmThreads), C::kSmemBytes, stream, tm_w, tm_x, tm_x64,
+                                  tm_xbig, p);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+    if (e != cudaSuccess) cudaGetLastError();
+    return e == cudaSuccess ? 0 : -3;
 }
 
-template <typename T, typename OutT, bool kSwiGLU>
+template <typename T, typename OutT, int kEpi>
 int dispatch_n(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t s) {
     switch (L.max_n) {
-        case 32: return launch_variant<T, OutT, kSwiGLU, 32>(L, ctl, num_sms, s);
-        case 64: return launch_variant<T, OutT, kSwiGLU, 64>(L, ctl, num_sms, s);
-        case 128: return launch_variant<T, OutT, kSwiGLU, 128>(L, ctl, num_sms, s);
-        case 256: return launch_variant<T, OutT, kSwiGLU, 256>(L, ctl, num_sms, s);
+        case 32: return launch_variant<T, OutT, kEpi, 32>(L, ctl, num_sms, s);
+        case 64: return launch_variant<T, OutT, kEpi, 64>(L, ctl, num_sms, s);
+        case 128: return launch_variant<T, OutT, kEpi, 128>(L, ctl, num_sms, s);
+        case 256: return launch_variant<T, OutT, kEpi, 256>(L, ctl, num_sms, s);
         default: return -1;
     }
+}
+
+// Plain epilogue: 256-feature tiles (two weight tiles per stage, halving the
+// token-tile bytes per flop) once token tiles are large; 128 otherwise.
+template <typename T, typename OutT>
+int dispatch_plain(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t s) {
+    if (L.max_n == 128 && L.n_out >= 256) return launch_variant<T, OutT, kEpiWide, 128>(L, ctl, num_sms, s);
+    if (L.max_n == 256 && L.n_out >= 256) return launch_variant<T, OutT, kEpiWide, 256>(L, ctl, num_sms, s);
+    return dispatch_n<T, OutT, kEpiPlain>(L, ctl, num_sms, s);
 }
 
 }  // namespace
@@ -110,7 +124,15 @@ GemmCtl gemm_ctl(void* workspace, int num_sms) {
     return c;
 }
 
+namespace {
+int g_token_tile_cap = 0;  // 0: automatic
+}
+
+void set_token_tile_cap(int n) { g_token_tile_cap = n; }
+
 int pick_max_n(double rows_per_group) {
+    if (g_token_tile_cap == 32 || g_token_tile_cap == 64 || g_token_tile_cap == 128 || g_token_tile_cap == 256)
+        return g_token_tile_cap;
     if (rows_per_group <= 24.0) return 32;
     if (rows_per_group <= 56.0) return 64;
     if (rows_per_group <= 112.0) return 128;
@@ -126,14 +148,14 @@ int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream) {
     if (L.dtype == 0) {
         if (L.out_f32) {
             if (L.swiglu) return -1;
-            return dispatch_n<__nv_bfloat16, float, false>(L, ctl, d.num_sms, stream);
+            return dispatch_n<__nv_bfloat16, float, kEpiPlain>(L, ctl, d.num_sms, stream);
         }
-        return L.swiglu ? dispatch_n<__nv_bfloat16, __nv_bfloat16, true>(L, ctl, d.num_sms, stream)
-                        : dispatch_n<__nv_bfloat16, __nv_bfloat16, false>(L, ctl, d.num_sms, stream);
+        return L.swiglu ? dispatch_n<__nv_bfloat16, __nv_bfloat16, kEpiSwiGLU>(L, ctl, d.num_sms, stream)
+                        : dispatch_plain<__nv_bfloat16, __nv_bfloat16>(L, ctl, d.num_sms, stream);
     }
     if (L.dtype == 1) {
-        return L.swiglu ? dispatch_n<float, float, true>(L, ctl, d.num_sms, stream)
-                        : dispatch_n<float, float, false>(L, ctl, d.num_sms, stream);
+        return L.swiglu ? dispatch_n<float, float, kEpiSwiGLU>(L, ctl, d.num_sms, stream)
+                        : dispatch_plain<float, float>(L, ctl, d.num_sms, stream);
     }
     return -1;
 }

@@ -43,6 +43,11 @@ namespace moe {
 constexpr int kMaxGroups = 1024;
 constexpr int kGemmThreads = 192;
 
+// Partial-tile slot layout: column c of row r (r < 128) at float index
+// ((c / 4) * 128 + r) * 4 + c % 4, so that a warp moves 32 consecutive
+// float4 (512 contiguous bytes) per access.
+__device__ __forceinline__ long long slot_f4(int c4, int r) { return (long long)c4 * 128 + r; }
+
 struct GemmParams {
     const int32_t* seg_offsets;  // [n_groups + 1] row offsets into X, or nullptr: one group [0, seg_rows)
     int n_groups;
@@ -59,19 +64,27 @@ struct GemmParams {
     uint64_t wait_limit_ns;
     int withhold_first_load;
     int sk_min_units;     // minimum k-iterations per stream-K block
+    int max_split;        // stream-K: most blocks contributing to one tile
 };
 
-template <typename T, bool kSwiGLU, int kMaxN>
+// Epilogue kinds: one 128-row weight tile per stage (plain store); gate and
+// up tiles of the same 128 features (SwiGLU); two adjacent 128-feature
+// blocks sharing one token tile (wide plain store, 256 features per tile).
+constexpr int kEpiPlain = 0, kEpiSwiGLU = 1, kEpiWide = 2;
+
+template <typename T, int kEpi, int kMaxN>
 struct GemmCfg {
     static constexpr int kBK = 128 / Elt<T>::kBytes;   // K elements per stage (one swizzle row)
     static constexpr int kMmaK = 32 / Elt<T>::kBytes;  // K per MMA instruction
-    static constexpr int kNW = kSwiGLU ? 2 : 1;        // weight tiles per stage (gate, up)
+    static constexpr int kNW = kEpi == kEpiPlain ? 1 : 2;  // weight tiles per stage
+    static constexpr int kFeat = kEpi == kEpiWide ? 256 : 128;  // output features per tile
     static constexpr int kWTileBytes = 128 * 128;
-    static constexpr int kXBoxRows = 16;
+    static constexpr int kXBoxRows = 16;       // token rows per TMA box: 16, 64 and kMaxN
+    static constexpr int kXBoxMid = 64;
     static constexpr int kXBoxBytes = kXBoxRows * 128;
     static constexpr int kXTileBytes = kMaxN * 128;
     static constexpr int kStageBytes = kNW * kWTileBytes + kXTileBytes;
-    static constexpr int kAccCols = kSwiGLU ? 2 * kMaxN : kMaxN;
+    static constexpr int kAccCols = kNW * kMaxN;
     static constexpr int kNumAcc = (512 / kAccCols) >= 2 ? 2 : 1;
     static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
     static constexpr int kMiscBytes = 512;
@@ -86,7 +99,7 @@ struct GemmCfg {
 
 // ------------------------------------------------------------- scheduling
 struct Tile {
-    int group, f0, row0, nrows, mma_n, wrow;
+    int group, f0, row0, nrows, mma_n, wrow, nch;
 };
 
 struct Sched {
@@ -122,7 +135,10 @@ __device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int to
     s.dp_tiles = s.dp_waves * s.G;
     s.sk_tiles = s.total_tiles - s.dp_tiles;
     s.U = s.sk_tiles * KI;
-    long long gsk = p.sk_min_units > 0 ? s.U / p.sk_min_units : s.U;
+    // at most max_split blocks share one tile: every block takes >= KI / kMaxSplit k-iterations
+    long long min_units = (KI + p.max_split - 1) / p.max_split;
+    if (min_units < p.sk_min_units) min_units = p.sk_min_units;
+    long long gsk = s.U / min_units;
     if (gsk < 1) gsk = 1;
     if (gsk > s.G) gsk = s.G;
     s.G_sk = (int)gsk;
@@ -185,7 +201,7 @@ __device__ __forceinline__ int chunks_of(int rows, int max_n) {
 }
 
 __device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, const int* cbase, int n_groups, int NF,
-                                            const GemmParams& p) {
+                                            int feat, const GemmParams& p) {
     // group: largest g with cbase[g] * NF <= tile
     int lo = 0, hi = n_groups - 1;
     while (lo < hi) {
@@ -202,11 +218,12 @@ __device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, cons
     int start, n, mn;
     chunk_rows(seg[g + 1] - seg[g], nch, j, start, n, mn);
     t.group = g;
-    t.f0 = f * 128;
+    t.f0 = f * feat;
     t.row0 = seg[g] + start;
     t.nrows = n;
     t.mma_n = mn;
-    t.wrow = g * p.w_group_stride + f * 128;
+    t.wrow = g * p.w_group_stride + f * feat;
+    t.nch = nch;
     return t;
 }
 
@@ -222,11 +239,14 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* ptr, flo
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
 // ------------------------------------------------------------------ kernel
-template <typename T, typename OutT, bool kSwiGLU, int kMaxN>
+template <typename T, typename OutT, int kEpi, int kMaxN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                    const __grid_constant__ CUtensorMap tm_x64, const __grid_constant__ CUtensorMap tm_xbig,
                     const GemmParams p) {
-    using C = GemmCfg<T, kSwiGLU, kMaxN>;
+    using C = GemmCfg<T, kEpi, kMaxN>;
+    constexpr bool kSwiGLU = kEpi == kEpiSwiGLU;
+    constexpr bool kTwo = C::kNW == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_base = smem;
@@ -247,6 +267,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int n_groups = p.n_groups;
     const uint64_t deadline = p.wait_limit_ns;  // per-wait limit
 
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -261,8 +282,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *abort_flag = 0;
         tma_prefetch_desc(&tm_w);
         tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_x64);
+        tma_prefetch_desc(&tm_xbig);
     }
     if (warp == 1) tmem_alloc(tmem_holder, 512);
+    pdl_wait();  // everything below reads or writes data shared with earlier kernels
     // segment table
     for (int g = threadIdx.x; g <= n_groups; g += blockDim.x)
         seg[g] = p.seg_offsets ? p.seg_offsets[g] : (g == 0 ? 0 : p.seg_rows);
@@ -288,7 +312,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    const int NF = (p.n_out + 127) / 128;
+    const int NF = (p.n_out + C::kFeat - 1) / C::kFeat;
     const int KI = (p.kdim + C::kBK - 1) / C::kBK;
     Sched sch;
     sched_init(sch, p, cbase[n_groups], NF, KI);
@@ -296,7 +320,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
+            // weights read by one tile only are streamed with evict-first; weight
+            // blocks that several token chunks share stay at normal priority
+            const uint64_t pol_w_once = policy_evict_first();
+            const uint64_t pol_w_shared = policy_evict_normal();
             const uint64_t pol_x = policy_evict_last();
             int fills[C::kStages];
 #pragma unroll
@@ -306,8 +333,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             Item it;
             while (ok && sched_next(sch, it)) {
-                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, p);
+                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeat, p);
                 const uint32_t bytes = C::kNW * C::kWTileBytes + (t.mma_n / 16) * C::kXBoxBytes;
+                const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
                     const uint32_t ph = (kc / C::kStages) & 1u;
@@ -323,9 +351,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     mbar_arrive_expect_tx(&full[s], bytes);
                     const int kx = k * C::kBK;
                     tma_load_2d(st, &tm_w, &full[s], kx, t.wrow, pol_w);
-                    if (kSwiGLU) tma_load_2d(st + C::kWTileBytes, &tm_w, &full[s], kx, t.wrow + p.up_offset, pol_w);
+                    if (kTwo)
+                        tma_load_2d(st + C::kWTileBytes, &tm_w, &full[s], kx, t.wrow + (kSwiGLU ? p.up_offset : 128),
+                                    pol_w);
                     uint8_t* xs = st + C::kNW * C::kWTileBytes;
-                    for (int r = 0; r < t.mma_n; r += C::kXBoxRows)
+                    int r = 0;
+                    if (kMaxN > C::kXBoxMid && t.mma_n == kMaxN) {
+                        tma_load_2d(xs, &tm_xbig, &full[s], kx, t.row0, pol_x);
+                        r = kMaxN;
+                    }
+                    if (kMaxN >= C::kXBoxMid)
+                        for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
+                            tma_load_2d(xs + r * 128, &tm_x64, &full[s], kx, t.row0 + r, pol_x);
+                    for (; r < t.mma_n; r += C::kXBoxRows)
                         tma_load_2d(xs + r * 128, &tm_x, &full[s], kx, t.row0 + r, pol_x);
                     ++fills[s];
                 }
@@ -345,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             Item it;
             while (ok && sched_next(sch, it)) {
-                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, p);
+                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeat, p);
                 const int b = ac % C::kNumAcc;
                 const uint32_t aph = (ac / C::kNumAcc) & 1u;
                 if (!mbar_wait_bounded(&tempty[b], aph ^ 1u, deadline, abort_flag)) {
@@ -372,7 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
                         umma<T>(d_gate, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
-                        if (kSwiGLU) umma<T>(d_up, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        if (kTwo) umma<T>(d_up, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
                     }
                     umma_commit(&empty[s]);
                 }
@@ -390,12 +428,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else {
         // -------------------------------------------------------- epilogue
         const int quad = warp & 3;
-        const int r = quad * 32 + lane;  // TMEM lane = feature row within the tile
+        const int r = quad * 32 + lane;  // TMEM lane = feature row within a 128-row block
         OutT* out = reinterpret_cast<OutT*>(p.out);
         uint32_t ac = 0;
         Item it;
         while (sched_next(sch, it)) {
-            Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, p);
+            Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeat, p);
             const int b = ac % C::kNumAcc;
             const uint32_t aph = (ac / C::kNumAcc) & 1u;
             if (!mbar_wait_bounded(&tfull[b], aph, deadline, abort_flag)) {
@@ -406,37 +444,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * C::kAccCols;
             const int f = t.f0 + r;
-            const bool fvalid = f < p.n_out;
+            // valid rows of the first and second accumulator
+            const bool v0 = f < p.n_out;
+            const bool v1 = kEpi == kEpiWide ? (f + 128 < p.n_out) : (kSwiGLU && v0);
             OutT* orow = out + (long long)t.row0 * p.out_ld + f;
+            // g: first accumulator, u: second (up projection, or features f + 128)
+            auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {
+                if (kSwiGLU) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
+                }
+                if (v0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * p.out_ld, g[i]);
+                }
+                if (kEpi == kEpiWide && v1) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.nrows) store_out<OutT>(orow + 128 + (long long)(c0 + i) * p.out_ld, u[i]);
+                }
+            };
             if (!it.split) {
-                for (int c0 = 0; c0 < t.mma_n; c0 += 16) {
-                    float g[16];
+                for (int c0 = 0; c0 < t.nrows; c0 += 16) {
+                    float g[16], u[16];
                     tmem_ld16(tacc + c0, g);
-                    if (kSwiGLU) {
-                        float u[16];
-                        tmem_ld16(tacc + kMaxN + c0, u);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
-                    }
-                    if (fvalid) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * p.out_ld, g[i]);
-                    }
+                    if (kTwo) tmem_ld16(tacc + kMaxN + c0, u);
+                    emit(c0, g, u);
                 }
             } else {
-                // stream-K: publish this block's partial tile
+                // stream-K: publish this block's partial tile (rows of real
+                // output features and columns of real tokens only)
                 const long long slot_floats = 128LL * C::kAccCols;
-                float* mine = p.partials + ((long long)blockIdx.x * 2 + it.slot) * slot_floats;
-                for (int c0 = 0; c0 < t.mma_n; c0 += 16) {
+                float4* mine = reinterpret_cast<float4*>(p.partials + ((long long)blockIdx.x * 2 + it.slot) * slot_floats);
+                for (int c0 = 0; c0 < t.nrows; c0 += 16) {
                     float g[16];
                     tmem_ld16(tacc + c0, g);
+                    if (v0) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) mine[(long long)(c0 + i) * 128 + r] = g[i];
-                    if (kSwiGLU) {
+                        for (int q = 0; q < 4; ++q)
+                            mine[slot_f4((c0 >> 2) + q, r)] =
+                                make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                    }
+                    if (kTwo) {
                         tmem_ld16(tacc + kMaxN + c0, g);
+                        if (v1) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) mine[(long long)(kMaxN + c0 + i) * 128 + r] = g[i];
+                            for (int q = 0; q < 4; ++q)
+                                mine[slot_f4(((kMaxN + c0) >> 2) + q, r)] =
+                                    make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                        }
                     }
                 }
                 __threadfence();
@@ -452,8 +509,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int c = c_first; c <= c_last; ++c)
                     if (sch.beg(c) < sch.beg(c + 1)) ++ncontrib;
                 if (arrived == ncontrib - 1) {
+                    // last to arrive: sum every contribution in block order, then the epilogue
                     __threadfence();
-                    for (int c0 = 0; c0 < t.mma_n; c0 += 16) {
+                    for (int c0 = 0; c0 < t.nrows; c0 += 16) {
                         float g[16], u[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
@@ -465,32 +523,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 tmem_ld16(tacc + c0, v);
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) g[i] += v[i];
-                                if (kSwiGLU) {
+                                if (kTwo) {
                                     tmem_ld16(tacc + kMaxN + c0, v);
 #pragma unroll
                                     for (int i = 0; i < 16; ++i) u[i] += v[i];
                                 }
                             } else {
                                 const int slot = (bc / sch.KI == it.sk_tile) ? 0 : 1;
-                                const float* other = p.partials + ((long long)c * 2 + slot) * slot_floats;
+                                const float4* other =
+                                    reinterpret_cast<const float4*>(p.partials + ((long long)c * 2 + slot) * slot_floats);
+                                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                                float4 a4[4], b4[4];
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) g[i] += ld_cg_f32(other + (long long)(c0 + i) * 128 + r);
-                                if (kSwiGLU) {
+                                for (int q = 0; q < 4; ++q) a4[q] = v0 ? __ldcg(other + slot_f4((c0 >> 2) + q, r)) : z;
+                                if (kTwo) {
 #pragma unroll
-                                    for (int i = 0; i < 16; ++i)
-                                        u[i] += ld_cg_f32(other + (long long)(kMaxN + c0 + i) * 128 + r);
+                                    for (int q = 0; q < 4; ++q)
+                                        b4[q] = v1 ? __ldcg(other + slot_f4(((kMaxN + c0) >> 2) + q, r)) : z;
+                                }
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    g[4 * q] += a4[q].x;
+                                    g[4 * q + 1] += a4[q].y;
+                                    g[4 * q + 2] += a4[q].z;
+                                    g[4 * q + 3] += a4[q].w;
+                                }
+                                if (kTwo) {
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        u[4 * q] += b4[q].x;
+                                        u[4 * q + 1] += b4[q].y;
+                                        u[4 * q + 2] += b4[q].z;
+                                        u[4 * q + 3] += b4[q].w;
+                                    }
                                 }
                             }
                         }
-                        if (kSwiGLU) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
-                        }
-                        if (fvalid) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * p.out_ld, g[i]);
-                        }
+                        emit(c0, g, u);
                     }
                     if (r == 0) p.counters[it.sk_tile] = 0;  // leave the counter zero for the next launch
                 }

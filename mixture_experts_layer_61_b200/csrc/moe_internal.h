@@ -6,7 +6,31 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
+
+// Programmatic dependent launch (on by default): kernels may begin while the
+// previous kernel on the stream drains; each kernel waits (griddepcontrol)
+// before it touches data a predecessor produced.
+bool pdl_enabled();
+void set_pdl(bool on);
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Cached properties of the current device.
 struct DeviceInfo {
@@ -52,12 +76,15 @@ struct GemmLaunch {
     int out_ld;
     int dtype;                   // 0 bf16, 1 fp32
     int max_n;                   // token-tile cap: 32, 64, 128 or 256
+    int max_split;               // stream-K: most blocks per tile (0 = default 4)
 };
 
 int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 
-// Token-tile cap for an expected number of rows per group.
+// Token-tile cap for an expected number of rows per group (or the cap forced
+// by set_token_tile_cap, 0 = automatic).
 int pick_max_n(double rows_per_group);
+void set_token_tile_cap(int n);
 
 // Elementwise / routing kernels.
 int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,

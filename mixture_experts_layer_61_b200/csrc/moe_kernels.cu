@@ -10,6 +10,16 @@
 
 namespace moe {
 
+namespace {
+int launched(cudaError_t e) {
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return -3;
+    }
+    return 0;
+}
+}  // namespace
+
 // ------------------------------------------------------------------ top-K
 // Order: larger logit first, lower expert index on equal logits.
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
@@ -21,6 +31,8 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 __global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int score_fn, int renorm,
                                                         const float* __restrict__ logits, int32_t* __restrict__ ids,
                                                         float* __restrict__ w) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
@@ -111,9 +123,10 @@ int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logi
     if (T == 0) return 0;
     const int warps_per_block = 8;
     const int blocks = (T + warps_per_block - 1) / warps_per_block;
-    topk_gate_kernel<<<blocks, warps_per_block * 32, 0, stream>>>(T, E, K, score_fn, renorm, logits, ids, w);
+    cudaError_t e = launch_kernel(topk_gate_kernel, dim3(blocks), dim3(warps_per_block * 32), 0, stream, T, E, K,
+                                  score_fn, renorm, logits, ids, w);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+    return launched(e);
 }
 
 // -------------------------------------------------------------- alignment
@@ -169,6 +182,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     uint16_t* tbl = reinterpret_cast<uint16_t*>(bad + 1);  // 32 x E
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long A = (long long)T * K;
+    pdl_launch_dependents();
+    pdl_wait();
 
     for (int e = tid; e < E; e += kAlignThreads) cnt[e] = 0;
     if (tid == 0) *bad = 0;
@@ -274,10 +289,10 @@ int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids
         }
         attr_done = true;
     }
-    align_kernel<<<1, kAlignThreads, smem, stream>>>(T, K, E, B, P_max, ids, counts, offsets, sorted_ids,
-                                                     block_expert, pos, scalars, stats_copy);
+    cudaError_t e = launch_kernel(align_kernel, dim3(1), dim3(kAlignThreads), smem, stream, T, K, E, B, P_max, ids,
+                                  counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+    return launched(e);
 }
 
 // ---------------------------------------------------------------- permute
@@ -285,6 +300,8 @@ int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids
 __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const int4* __restrict__ x,
                                                       const int32_t* __restrict__ sorted_ids,
                                                       const int32_t* __restrict__ scalars, int4* __restrict__ x_perm) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int P = scalars[0];
     const int rows_per_block = blockDim.x / 64;  // 64 threads per row
     const int sub = threadIdx.x / 64, l = threadIdx.x % 64;
@@ -313,10 +330,10 @@ int launch_permute(int H, int K, int dtype, long long P_max, const void* x, cons
     long long blocks = (P_max + rows_per_block - 1) / rows_per_block;
     const long long cap = (long long)d.num_sms * 8;
     if (blocks > cap) blocks = cap;
-    permute_kernel<<<(int)blocks, 256, 0, stream>>>(row_vec, K, static_cast<const int4*>(x), sorted_ids, scalars,
-                                                    static_cast<int4*>(x_perm));
+    cudaError_t e = launch_kernel(permute_kernel, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
+                                  static_cast<const int4*>(x), sorted_ids, scalars, static_cast<int4*>(x_perm));
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+    return launched(e);
 }
 
 // ---------------------------------------------------------------- combine
@@ -362,6 +379,8 @@ __global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K
     constexpr int N = Vec16<T>::N;
     __shared__ int s_pos[16];
     __shared__ float s_w[16];
+    pdl_launch_dependents();
+    pdl_wait();
     for (int t = blockIdx.x; t < T_; t += gridDim.x) {
         __syncthreads();
         if (threadIdx.x < K) {
@@ -403,16 +422,15 @@ int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int
     long long blocks = T;
     const long long cap = (long long)d.num_sms * 16;
     if (blocks > cap) blocks = cap;
-    if (dtype == 0)
-        combine_kernel<__nv_bfloat16><<<(int)blocks, threads, 0, stream>>>(
-            T, row_vec, K, static_cast<const int4*>(y_perm), pos, w, static_cast<const int4*>(shared_out),
-            static_cast<int4*>(out));
-    else
-        combine_kernel<float><<<(int)blocks, threads, 0, stream>>>(T, row_vec, K, static_cast<const int4*>(y_perm), pos,
-                                                                   w, static_cast<const int4*>(shared_out),
-                                                                   static_cast<int4*>(out));
+    const int4* y4 = static_cast<const int4*>(y_perm);
+    const int4* s4 = static_cast<const int4*>(shared_out);
+    int4* o4 = static_cast<int4*>(out);
+    cudaError_t e = dtype == 0 ? launch_kernel(combine_kernel<__nv_bfloat16>, dim3((int)blocks), dim3(threads), 0,
+                                               stream, T, row_vec, K, y4, pos, w, s4, o4)
+                               : launch_kernel(combine_kernel<float>, dim3((int)blocks), dim3(threads), 0, stream, T,
+                                               row_vec, K, y4, pos, w, s4, o4);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? 0 : -3;
+    return launched(e);
 }
 
 }  // namespace moe

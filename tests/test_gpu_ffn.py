@@ -73,7 +73,8 @@ def test_grouped_one_hot_expert_many_chunks():
     assert _grouped(shape, 1000, seed=2, kind="skew") < OUT_TOL
 
 
-@pytest.mark.parametrize("T,H,I", [(1, 512, 1024), (16, 256, 640), (300, 1024, 2048), (700, 512, 14336)])
+@pytest.mark.parametrize("T,H,I", [(1, 512, 1024), (16, 256, 640), (300, 1024, 2048), (700, 512, 14336),
+                                   (300, 264, 640), (130, 392, 376)])
 def test_dense_ffn(T, H, I):
     # (700, 512, 14336): 3 chunks x 112 feature blocks -> data-parallel waves plus a stream-K tail
     w13, w2 = mi.make_dense_weights(H, I, torch.bfloat16, seed=T + I, device="cuda")
@@ -86,6 +87,18 @@ def test_dense_ffn(T, H, I):
     tok = sample_tokens(T, 48, seed=T)
     ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
     assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
+
+
+@pytest.mark.parametrize("cap", [32, 64, 128, 256])
+def test_grouped_every_token_tile_cap(cap):
+    # the same grouped problem through every kernel variant: plain or 256-feature
+    # (wide) down tiles, SwiGLU gate/up, token tiles of 32..256
+    shape = small_shape(H=520, E=6, K=2, I=392)
+    moe.set_token_tile_cap(cap)
+    try:
+        assert _grouped(shape, 700, seed=cap) < OUT_TOL
+    finally:
+        moe.set_token_tile_cap(0)
 
 
 def test_dense_ffn_fp32_tf32():
