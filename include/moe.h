@@ -225,6 +225,12 @@ int moe_set_token_tile_cap(int n);
  * subsequent launches.  Process-wide; results are identical either way. */
 void moe_set_programmatic_launch(int enable);
 
+/* CTA pairs (default on): bf16 grouped/dense GEMMs at the 256-token tile
+ * cap run on pairs of SMs (thread-block clusters of 2, 2-SM tensor-core MMA
+ * with 256 weight rows per pair).  0 keeps single-SM tiles.  Process-wide;
+ * results are identical up to fp32 summation order. */
+void moe_set_cta_pairs(int enable);
+
 /* Test hook: when nonzero, the next GEMM launch withholds the first operand
  * load of block 0, so that block's waits run out and report
  * MOE_ERR_TIMEOUT through moe_check_status().  Cleared after one launch. */

@@ -76,6 +76,7 @@ def lib():
             "moe_debug_withhold_first_load": (None, [I]),
             "moe_set_token_tile_cap": (I, [I]),
             "moe_set_programmatic_launch": (None, [I]),
+            "moe_set_cta_pairs": (None, [I]),
             "moe_kernel_launch_count": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
@@ -275,6 +276,11 @@ def set_token_tile_cap(n):
 def set_programmatic_launch(enable=True):
     """Programmatic dependent launch between the layer's kernels (default on)."""
     lib().moe_set_programmatic_launch(1 if enable else 0)
+
+
+def set_cta_pairs(enable=True):
+    """2-SM (CTA pair) GEMM tiles for bf16 at the 256-token cap (default on)."""
+    lib().moe_set_cta_pairs(1 if enable else 0)
 
 
 def debug_withhold_first_load(enable=True):

@@ -490,6 +490,8 @@ int moe_set_token_tile_cap(int n) {
 
 void moe_set_programmatic_launch(int enable) { set_pdl(enable != 0); }
 
+void moe_set_cta_pairs(int enable) { set_cta_pairs(enable != 0); }
+
 void moe_debug_withhold_first_load(int enable) { g_withhold.store(enable ? 1 : 0); }
 
 uint64_t moe_kernel_launch_count(void) { return g_launches.load(); }

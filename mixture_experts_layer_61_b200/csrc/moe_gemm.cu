@@ -44,15 +44,38 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void*
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, typename OutT, int kEpi, int kMaxN>
+template <typename T, typename OutT, int kEpi, int kMaxN, int kCta = 1>
 int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t stream) {
-    using C = GemmCfg<T, kEpi, kMaxN>;
-    auto kern = moe_gemm_kernel<T, OutT, kEpi, kMaxN>;
+    using C = GemmCfg<T, kEpi, kMaxN, kCta>;
+    auto kern = moe_gemm_kernel<T, OutT, kEpi, kMaxN, kCta>;
+    if (kCta == 2 && (num_sms & 1)) return -1;
+    static int grid_blocks = 0;  // per instantiation: CTAs that can be resident at once
     static bool attr_done = false;  // per instantiation
     if (!attr_done) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return -3;
+        }
+        grid_blocks = num_sms;
+        if (kCta > 1) {
+            // pairs must sit in one GPC: size the persistent grid by the clusters that fit
+            cudaLaunchConfig_t oc = {};
+            oc.gridDim = dim3(num_sms);
+            oc.blockDim = dim3(kGemmThreads);
+            oc.dynamicSmemBytes = C::kSmemBytes;
+            cudaLaunchAttribute ca;
+            ca.id = cudaLaunchAttributeClusterDimension;
+            ca.val.clusterDim.x = kCta;
+            ca.val.clusterDim.y = 1;
+            ca.val.clusterDim.z = 1;
+            oc.attrs = &ca;
+            oc.numAttrs = 1;
+            int nclusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &oc) != cudaSuccess || nclusters <= 0) {
+                cudaGetLastError();
+                return -3;
+            }
+            grid_blocks = nclusters * kCta < num_sms ? nclusters * kCta : num_sms;
         }
         attr_done = true;
     }
@@ -60,7 +83,7 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
     if (!make_map(&tm_w, Elt<T>::kTma, Elt<T>::kBytes, L.w, L.w_rows, L.kdim, 128)) return -3;
     if (!make_map(&tm_x, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxRows)) return -3;
     if (!make_map(&tm_x64, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxMid)) return -3;
-    if (!make_map(&tm_xbig, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, kMaxN)) return -3;
+    if (!make_map(&tm_xbig, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, kMaxN / kCta)) return -3;
     GemmParams p;
     p.seg_offsets = L.seg_offsets;
     p.n_groups = L.n_groups;
@@ -78,8 +101,8 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
     p.withhold_first_load = take_withhold_flag();
     p.sk_min_units = 4;
     p.max_split = L.max_split > 0 ? L.max_split : 4;
-    cudaError_t e = launch_kernel(kern, dim3(num_sms), dim3(kGemmThreads), C::kSmemBytes, stream, tm_w, tm_x, tm_x64,
-                                  tm_xbig, p);
+    cudaError_t e = launch_kernel_cluster(kern, dim3(grid_blocks), dim3(kGemmThreads), C::kSmemBytes, stream, kCta,
+                                          tm_w, tm_x, tm_x64, tm_xbig, p);
     count_launch();
     if (e != cudaSuccess) cudaGetLastError();
     return e == cudaSuccess ? 0 : -3;
@@ -96,6 +119,8 @@ int dispatch_n(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_
     }
 }
 
+bool g_cta_pairs = true;
+
 // Plain epilogue: 256-feature tiles (two weight tiles per stage, halving the
 // token-tile bytes per flop) once token tiles are large; 128 otherwise.
 template <typename T, typename OutT>
@@ -103,6 +128,18 @@ int dispatch_plain(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
     if (L.max_n == 128 && L.n_out >= 256) return launch_variant<T, OutT, kEpiWide, 128>(L, ctl, num_sms, s);
     if (L.max_n == 256 && L.n_out >= 256) return launch_variant<T, OutT, kEpiWide, 256>(L, ctl, num_sms, s);
     return dispatch_n<T, OutT, kEpiPlain>(L, ctl, num_sms, s);
+}
+
+// bf16 at the 256-token cap: CTA pairs (2-SM MMA, M = 256 weight rows per
+// pair, each CTA staging half of the 256 token rows).
+int dispatch_bf16(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t s) {
+    using bf = __nv_bfloat16;
+    if (g_cta_pairs && L.max_n == 256 && !L.out_f32 && (num_sms % 2) == 0) {
+        if (L.swiglu) return launch_variant<bf, bf, kEpiSwiGLU, 256, 2>(L, ctl, num_sms, s);
+        if (L.n_out >= 512) return launch_variant<bf, bf, kEpiWide, 256, 2>(L, ctl, num_sms, s);
+    }
+    if (L.out_f32) return dispatch_n<bf, float, kEpiPlain>(L, ctl, num_sms, s);
+    return L.swiglu ? dispatch_n<bf, bf, kEpiSwiGLU>(L, ctl, num_sms, s) : dispatch_plain<bf, bf>(L, ctl, num_sms, s);
 }
 
 }  // namespace
@@ -129,6 +166,7 @@ int g_token_tile_cap = 0;  // 0: automatic
 }
 
 void set_token_tile_cap(int n) { g_token_tile_cap = n; }
+void set_cta_pairs(bool on) { g_cta_pairs = on; }
 
 int pick_max_n(double rows_per_group) {
     if (g_token_tile_cap == 32 || g_token_tile_cap == 64 || g_token_tile_cap == 128 || g_token_tile_cap == 256)
@@ -146,12 +184,8 @@ int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream) {
     if (L.n_groups < 1 || L.n_groups > kMaxGroups || L.kdim <= 0 || L.n_out <= 0) return -1;
     if (L.x_rows <= 0 || L.w_rows <= 0) return 0;
     if (L.dtype == 0) {
-        if (L.out_f32) {
-            if (L.swiglu) return -1;
-            return dispatch_n<__nv_bfloat16, float, kEpiPlain>(L, ctl, d.num_sms, stream);
-        }
-        return L.swiglu ? dispatch_n<__nv_bfloat16, __nv_bfloat16, kEpiSwiGLU>(L, ctl, d.num_sms, stream)
-                        : dispatch_plain<__nv_bfloat16, __nv_bfloat16>(L, ctl, d.num_sms, stream);
+        if (L.out_f32 && L.swiglu) return -1;
+        return dispatch_bf16(L, ctl, d.num_sms, stream);
     }
     if (L.dtype == 1) {
         return L.swiglu ? dispatch_n<float, float, kEpiSwiGLU>(L, ctl, d.num_sms, stream)

@@ -72,17 +72,19 @@ struct GemmParams {
 // blocks sharing one token tile (wide plain store, 256 features per tile).
 constexpr int kEpiPlain = 0, kEpiSwiGLU = 1, kEpiWide = 2;
 
-template <typename T, int kEpi, int kMaxN>
+template <typename T, int kEpi, int kMaxN, int kCta = 1>
 struct GemmCfg {
     static constexpr int kBK = 128 / Elt<T>::kBytes;   // K elements per stage (one swizzle row)
     static constexpr int kMmaK = 32 / Elt<T>::kBytes;  // K per MMA instruction
     static constexpr int kNW = kEpi == kEpiPlain ? 1 : 2;  // weight tiles per stage
-    static constexpr int kFeat = kEpi == kEpiWide ? 256 : 128;  // output features per tile
+    static constexpr int kFeat = kEpi == kEpiWide ? 256 : 128;  // output features per CTA and tile
+    static constexpr int kFeatTile = kFeat * kCta;                 // output features per tile
+    static constexpr int kUnit = 16 * kCta;                        // token-row granularity of the MMA
     static constexpr int kWTileBytes = 128 * 128;
     static constexpr int kXBoxRows = 16;       // token rows per TMA box: 16, 64 and kMaxN
     static constexpr int kXBoxMid = 64;
     static constexpr int kXBoxBytes = kXBoxRows * 128;
-    static constexpr int kXTileBytes = kMaxN * 128;
+    static constexpr int kXTileBytes = (kMaxN / kCta) * 128;  // this CTA's share of the token tile
     static constexpr int kStageBytes = kNW * kWTileBytes + kXTileBytes;
     static constexpr int kAccCols = kNW * kMaxN;
     static constexpr int kNumAcc = (512 / kAccCols) >= 2 ? 2 : 1;
@@ -93,7 +95,8 @@ struct GemmCfg {
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
     static_assert(kStages >= 2, "pipeline needs two stages");
-    static_assert(kMaxN % 16 == 0 && kMaxN >= 16 && kMaxN <= 256, "MMA N range");
+    static_assert(kMaxN % kUnit == 0 && kMaxN >= kUnit && kMaxN <= 256, "MMA N range");
+    static_assert(kCta == 1 || kCta == 2, "one CTA or a CTA pair");
     static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
 };
 
@@ -124,12 +127,13 @@ struct Item {
     long long sk_tile;
 };
 
-__device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int total_chunks, int NF, int KI) {
+// Scheduling unit: one CTA, or one CTA pair (cluster of 2) sharing each tile.
+__device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int total_chunks, int NF, int KI, int ncta) {
     s.n_groups = p.n_groups;
     s.NF = NF;
     s.KI = KI;
-    s.G = gridDim.x;
-    s.cta = blockIdx.x;
+    s.G = gridDim.x / ncta;
+    s.cta = blockIdx.x / ncta;
     s.total_tiles = (long long)total_chunks * NF;
     s.dp_waves = s.total_tiles >= 2LL * s.G ? s.total_tiles / s.G - 1 : 0;
     s.dp_tiles = s.dp_waves * s.G;
@@ -181,27 +185,27 @@ __device__ __forceinline__ bool sched_next(Sched& s, Item& it) {
     return false;
 }
 
-// Rows of chunk j of a group of `rows` rows cut into `nch` chunks, in units of 16.
-__device__ __forceinline__ void chunk_rows(int rows, int nch, int j, int& start, int& n, int& mma_n) {
-    int units = (rows + 15) >> 4;
+// Rows of chunk j of a group of `rows` rows cut into `nch` chunks, in units of `unit` rows.
+__device__ __forceinline__ void chunk_rows(int rows, int nch, int j, int unit, int& start, int& n, int& mma_n) {
+    int units = (rows + unit - 1) / unit;
     int base = units / nch, extra = units % nch;
     int su = j * base + (j < extra ? j : extra);
     int mu = base + (j < extra ? 1 : 0);
-    start = su * 16;
-    mma_n = mu * 16;
+    start = su * unit;
+    mma_n = mu * unit;
     int left = rows - start;
     n = mma_n < left ? mma_n : left;
 }
 
-__device__ __forceinline__ int chunks_of(int rows, int max_n) {
+__device__ __forceinline__ int chunks_of(int rows, int max_n, int unit) {
     if (rows <= 0) return 0;
-    int units = (rows + 15) >> 4;
-    int per = max_n >> 4;
+    int units = (rows + unit - 1) / unit;
+    int per = max_n / unit;
     return (units + per - 1) / per;
 }
 
 __device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, const int* cbase, int n_groups, int NF,
-                                            int feat, const GemmParams& p) {
+                                            int feat, int unit, const GemmParams& p) {
     // group: largest g with cbase[g] * NF <= tile
     int lo = 0, hi = n_groups - 1;
     while (lo < hi) {
@@ -216,7 +220,7 @@ __device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, cons
     int j = (int)(local - (long long)f * nch);
     Tile t;
     int start, n, mn;
-    chunk_rows(seg[g + 1] - seg[g], nch, j, start, n, mn);
+    chunk_rows(seg[g + 1] - seg[g], nch, j, unit, start, n, mn);
     t.group = g;
     t.f0 = f * feat;
     t.row0 = seg[g] + start;
@@ -236,17 +240,18 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* ptr, flo
     *ptr = __float2bfloat16_rn(v);
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // ------------------------------------------------------------------ kernel
-template <typename T, typename OutT, int kEpi, int kMaxN>
+template <typename T, typename OutT, int kEpi, int kMaxN, int kCta>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                     const __grid_constant__ CUtensorMap tm_x64, const __grid_constant__ CUtensorMap tm_xbig,
                     const GemmParams p) {
-    using C = GemmCfg<T, kEpi, kMaxN>;
+    using C = GemmCfg<T, kEpi, kMaxN, kCta>;
     constexpr bool kSwiGLU = kEpi == kEpiSwiGLU;
     constexpr bool kTwo = C::kNW == 2;
+    constexpr bool kPair = kCta == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_base = smem;
@@ -266,6 +271,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int lane = threadIdx.x & 31;
     const int n_groups = p.n_groups;
     const uint64_t deadline = p.wait_limit_ns;  // per-wait limit
+    // CTA pair: rank 0 (the leader) issues the MMAs for both; each CTA stages
+    // its own 128 weight rows and half of the token rows, and holds in TMEM
+    // the accumulators of its own 128 weight rows.
+    const uint32_t rank = kPair ? cluster_rank() : 0u;
 
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < C::kNumAcc; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], 128 * kCta);
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
@@ -285,7 +294,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_prefetch_desc(&tm_x64);
         tma_prefetch_desc(&tm_xbig);
     }
-    if (warp == 1) tmem_alloc(tmem_holder, 512);
+    if (warp == 1) {
+        if (kPair) tmem_alloc_pair(tmem_holder, 512);
+        else tmem_alloc(tmem_holder, 512);
+    }
+    if (kPair) cluster_sync_all();  // the peer's barriers are initialised before any TMA or commit targets them
     pdl_wait();  // everything below reads or writes data shared with earlier kernels
     // segment table
     for (int g = threadIdx.x; g <= n_groups; g += blockDim.x)
@@ -295,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int running = 0;
         for (int base = 0; base < n_groups; base += 32) {
             int g = base + lane;
-            int n = g < n_groups ? chunks_of(seg[g + 1] - seg[g], kMaxN) : 0;
+            int n = g < n_groups ? chunks_of(seg[g + 1] - seg[g], kMaxN, C::kUnit) : 0;
             int incl = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -312,10 +325,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    const int NF = (p.n_out + C::kFeat - 1) / C::kFeat;
+    const int NF = (p.n_out + C::kFeatTile - 1) / C::kFeatTile;
     const int KI = (p.kdim + C::kBK - 1) / C::kBK;
     Sched sch;
-    sched_init(sch, p, cbase[n_groups], NF, KI);
+    sched_init(sch, p, cbase[n_groups], NF, KI, kCta);
 
     if (warp == 0) {
         // ---------------------------------------------------- TMA producer
@@ -333,8 +346,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             Item it;
             while (ok && sched_next(sch, it)) {
-                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeat, p);
-                const uint32_t bytes = C::kNW * C::kWTileBytes + (t.mma_n / 16) * C::kXBoxBytes;
+                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeatTile, C::kUnit, p);
+                // this CTA's weight rows and token rows of the tile
+                const int wrow = t.wrow + (int)rank * C::kFeat;
+                const int xn = t.mma_n / kCta;
+                const int xrow = t.row0 + (int)rank * xn;
+                // bytes landing on the (leader's) full barrier per stage: both CTAs' shares
+                const uint32_t bytes = kCta * (C::kNW * C::kWTileBytes + xn * 128);
                 const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
@@ -348,23 +366,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         continue;
                     }
                     uint8_t* st = stage_base + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], bytes);
-                    const int kx = k * C::kBK;
-                    tma_load_2d(st, &tm_w, &full[s], kx, t.wrow, pol_w);
-                    if (kTwo)
-                        tma_load_2d(st + C::kWTileBytes, &tm_w, &full[s], kx, t.wrow + (kSwiGLU ? p.up_offset : 128),
-                                    pol_w);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
+                    const uint32_t fb = kPair ? map_to_rank(smem_u32(&full[s]), 0) : 0u;
+                    auto load = [&](void* dst, const CUtensorMap* m, int c1, uint64_t pol) {
+                        if (kPair) tma_load_2d_pair(dst, m, fb, k * C::kBK, c1, pol);
+                        else tma_load_2d(dst, m, &full[s], k * C::kBK, c1, pol);
+                    };
+                    load(st, &tm_w, wrow, pol_w);
+                    if (kTwo) load(st + C::kWTileBytes, &tm_w, wrow + (kSwiGLU ? p.up_offset : 128), pol_w);
                     uint8_t* xs = st + C::kNW * C::kWTileBytes;
                     int r = 0;
-                    if (kMaxN > C::kXBoxMid && t.mma_n == kMaxN) {
-                        tma_load_2d(xs, &tm_xbig, &full[s], kx, t.row0, pol_x);
-                        r = kMaxN;
+                    if (kMaxN / kCta > C::kXBoxMid && xn == kMaxN / kCta) {
+                        load(xs, &tm_xbig, xrow, pol_x);
+                        r = xn;
                     }
-                    if (kMaxN >= C::kXBoxMid)
-                        for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
-                            tma_load_2d(xs + r * 128, &tm_x64, &full[s], kx, t.row0 + r, pol_x);
-                    for (; r < t.mma_n; r += C::kXBoxRows)
-                        tma_load_2d(xs + r * 128, &tm_x, &full[s], kx, t.row0 + r, pol_x);
+                    if (kMaxN / kCta >= C::kXBoxMid)
+                        for (; r + C::kXBoxMid <= xn; r += C::kXBoxMid) load(xs + r * 128, &tm_x64, xrow + r, pol_x);
+                    for (; r < xn; r += C::kXBoxRows) load(xs + r * 128, &tm_x, xrow + r, pol_x);
                     ++fills[s];
                 }
             }
@@ -372,18 +390,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 *abort_flag = 1;
                 atomicOr(p.status, kStatusTimeout);
             }
-            // every issued copy lands before the block exits
-            for (int s = 0; s < C::kStages; ++s)
-                if (fills[s] > 0) mbar_drain(&full[s], (uint32_t)(fills[s] - 1) & 1u, p.wait_limit_ns);
+            // every issued copy lands before the block exits (the leader's full
+            // barriers count both CTAs' copies; the pair leaves together)
+            if (rank == 0)
+                for (int s = 0; s < C::kStages; ++s)
+                    if (fills[s] > 0) mbar_drain(&full[s], (uint32_t)(fills[s] - 1) & 1u, p.wait_limit_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             uint32_t kc = 0, ac = 0;
             bool ok = true;
             Item it;
             while (ok && sched_next(sch, it)) {
-                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeat, p);
+                Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeatTile, C::kUnit, p);
                 const int b = ac % C::kNumAcc;
                 const uint32_t aph = (ac / C::kNumAcc) & 1u;
                 if (!mbar_wait_bounded(&tempty[b], aph ^ 1u, deadline, abort_flag)) {
@@ -393,7 +413,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_fence_after();
                 const uint32_t d_gate = tmem_base + b * C::kAccCols;
                 const uint32_t d_up = d_gate + kMaxN;
-                const uint32_t idesc = umma_idesc(Elt<T>::kMmaFmt, 128, t.mma_n);
+                const uint32_t idesc = umma_idesc(Elt<T>::kMmaFmt, 128 * kCta, t.mma_n);
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
                     const uint32_t ph = (kc / C::kStages) & 1u;
@@ -409,19 +429,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
-                        umma<T>(d_gate, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
-                        if (kTwo) umma<T>(d_up, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        if (kPair) {
+                            umma_pair_bf16(d_gate, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                            if (kTwo) umma_pair_bf16(d_up, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        } else {
+                            umma<T>(d_gate, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                            if (kTwo) umma<T>(d_up, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        }
                     }
-                    umma_commit(&empty[s]);
+                    if (kPair) {  // the stage is free in both CTAs
+                        umma_commit_pair(smem_u32(&empty[s]));
+                        umma_commit_pair(map_to_rank(smem_u32(&empty[s]), 1));
+                    } else {
+                        umma_commit(&empty[s]);
+                    }
                 }
                 if (!ok) break;
-                umma_commit(&tfull[b]);
+                if (kPair) {
+                    umma_commit_pair(smem_u32(&tfull[b]));
+                    umma_commit_pair(map_to_rank(smem_u32(&tfull[b]), 1));
+                } else {
+                    umma_commit(&tfull[b]);
+                }
                 ++ac;
             }
             if (!ok) {
                 *abort_flag = 1;
                 atomicOr(p.status, kStatusTimeout);
-                umma_commit(drain_bar);
+                if (kPair) umma_commit_pair(smem_u32(drain_bar));
+                else umma_commit(drain_bar);
                 mbar_drain(drain_bar, 0, p.wait_limit_ns);
             }
         }
@@ -433,7 +469,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t ac = 0;
         Item it;
         while (sched_next(sch, it)) {
-            Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeat, p);
+            Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeatTile, C::kUnit, p);
             const int b = ac % C::kNumAcc;
             const uint32_t aph = (ac / C::kNumAcc) & 1u;
             if (!mbar_wait_bounded(&tfull[b], aph, deadline, abort_flag)) {
@@ -443,7 +479,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_after();
             const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * C::kAccCols;
-            const int f = t.f0 + r;
+            const int f = t.f0 + (int)rank * C::kFeat + r;
             // valid rows of the first and second accumulator
             const bool v0 = f < p.n_out;
             const bool v1 = kEpi == kEpiWide ? (f + 128 < p.n_out) : (kSwiGLU && v0);
@@ -466,17 +502,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             };
             if (!it.split) {
-                for (int c0 = 0; c0 < t.nrows; c0 += 16) {
-                    float g[16], u[16];
-                    tmem_ld16(tacc + c0, g);
-                    if (kTwo) tmem_ld16(tacc + kMaxN + c0, u);
-                    emit(c0, g, u);
+                // 32 columns of both accumulators per round, one wait for both loads
+                for (int c0 = 0; c0 < t.nrows; c0 += 32) {
+                    uint32_t ga[32], ua[32];
+                    tmem_ld32_nowait(tacc + c0, ga);
+                    if (kTwo) tmem_ld32_nowait(tacc + kMaxN + c0, ua);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float g[16], u[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            g[i] = __uint_as_float(ga[16 * h + i]);
+                            u[i] = kTwo ? __uint_as_float(ua[16 * h + i]) : 0.f;
+                        }
+                        if (c0 + 16 * h < t.nrows) emit(c0 + 16 * h, g, u);
+                    }
                 }
             } else {
                 // stream-K: publish this block's partial tile (rows of real
                 // output features and columns of real tokens only)
                 const long long slot_floats = 128LL * C::kAccCols;
                 float4* mine = reinterpret_cast<float4*>(p.partials + ((long long)blockIdx.x * 2 + it.slot) * slot_floats);
+                const long long counter = it.sk_tile * kCta + rank;  // one counter per tile half
                 for (int c0 = 0; c0 < t.nrows; c0 += 16) {
                     float g[16];
                     tmem_ld16(tacc + c0, g);
@@ -498,7 +546,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 __threadfence();
                 named_sync(1, 128);
-                if (r == 0) *bcast = atomicAdd(&p.counters[it.sk_tile], 1);
+                if (r == 0) *bcast = atomicAdd(&p.counters[counter], 1);
                 named_sync(1, 128);
                 const int arrived = *bcast;
                 // contributors: blocks whose stream-K range meets this tile
@@ -518,7 +566,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int c = c_first; c <= c_last; ++c) {
                             const long long bc = sch.beg(c);
                             if (bc >= sch.beg(c + 1)) continue;
-                            if (c == (int)blockIdx.x) {
+                            if (c == sch.cta) {
                                 float v[16];
                                 tmem_ld16(tacc + c0, v);
 #pragma unroll
@@ -531,7 +579,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             } else {
                                 const int slot = (bc / sch.KI == it.sk_tile) ? 0 : 1;
                                 const float4* other =
-                                    reinterpret_cast<const float4*>(p.partials + ((long long)c * 2 + slot) * slot_floats);
+                                    reinterpret_cast<const float4*>(p.partials + (((long long)c * kCta + rank) * 2 + slot) *
+                                                                                     slot_floats);
                                 const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
                                 float4 a4[4], b4[4];
 #pragma unroll
@@ -561,21 +610,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                         emit(c0, g, u);
                     }
-                    if (r == 0) p.counters[it.sk_tile] = 0;  // leave the counter zero for the next launch
+                    if (r == 0) p.counters[counter] = 0;  // leave the counter zero for the next launch
                 }
             }
             tc_fence_before();
-            mbar_arrive(&tempty[b]);
+            if (kPair && rank != 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[b]), 0));
+            else mbar_arrive(&tempty[b]);
             ++ac;
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    if (kPair) cluster_sync_all();  // neither CTA frees TMEM or leaves while the pair's MMAs may run
+    else __syncthreads();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        if (kPair) tmem_dealloc_pair(tmem_base, 512);
+        else tmem_dealloc(tmem_base, 512);
     }
 }
 

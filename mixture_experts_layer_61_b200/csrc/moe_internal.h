@@ -16,20 +16,39 @@ namespace moe {
 bool pdl_enabled();
 void set_pdl(bool on);
 
+// Launch with programmatic dependent launch (when enabled) and, for
+// cluster_x > 1, thread-block clusters of cluster_x CTAs along x.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                          Args&&... args) {
+cudaError_t launch_kernel_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  int cluster_x, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+    return launch_kernel_cluster(kern, grid, block, smem, s, 1, std::forward<Args>(args)...);
 }
 
 // Cached properties of the current device.
@@ -85,6 +104,8 @@ int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 // by set_token_tile_cap, 0 = automatic).
 int pick_max_n(double rows_per_group);
 void set_token_tile_cap(int n);
+// CTA-pair (2-SM MMA) tiles for bf16 launches at the 256-token cap (default on).
+void set_cta_pairs(bool on);
 
 // Elementwise / routing kernels.
 int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,

@@ -123,3 +123,36 @@ def test_deterministic_repeat():
     o2 = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws).clone()
     moe.check_status(ws)
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("pairs", [True, False])
+@pytest.mark.parametrize("T,H,I", [(700, 512, 1024), (300, 1024, 2048), (260, 520, 392)])
+def test_dense_ffn_cta_pairs(pairs, T, H, I):
+    # 2-SM (CTA pair) tiles at the 256-token cap against the oracle, and
+    # against single-SM tiles on the same inputs
+    w13, w2 = mi.make_dense_weights(H, I, torch.bfloat16, seed=T, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(H)
+    x = torch.randn((T, H), generator=gen, device="cuda").to(torch.bfloat16)
+    ws = moe.alloc_workspace(moe.dense_workspace_size(T, H, I))
+    moe.set_cta_pairs(pairs)
+    try:
+        out = moe.dense_ffn(x, w13, w2, ws)
+        moe.check_status(ws)
+    finally:
+        moe.set_cta_pairs(True)
+    tok = sample_tokens(T, 40, seed=1)
+    ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
+    assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
+
+
+@pytest.mark.parametrize("kind", ["uniform", "skew"])
+def test_grouped_cta_pairs_match_single(kind):
+    shape = small_shape(H=1024, E=4, K=2, I=1536)
+    e_pair = _grouped(shape, 900, seed=3, kind=kind)
+    moe.set_cta_pairs(False)
+    try:
+        e_single = _grouped(shape, 900, seed=3, kind=kind)
+    finally:
+        moe.set_cta_pairs(True)
+    assert e_pair < OUT_TOL and e_single < OUT_TOL
