@@ -219,6 +219,13 @@ void moe_set_wait_limit_ns(uint64_t ns);
  * differs.  Process-wide.  Returns MOE_ERR_ARG for other values. */
 int moe_set_token_tile_cap(int n);
 
+/* 1 when moe_grouped_ffn / moe_layer_forward run this configuration's
+ * expert FFN as one fused launch (gate/up + SwiGLU and down in a persistent
+ * kernel with dynamic work fetching; decode-sized T*K/E), 0 when as two
+ * grouped-GEMM launches.  moe_grouped_gate_up / moe_grouped_down always
+ * launch the two GEMMs separately. */
+int moe_ffn_fused(const moe_config_t* cfg);
+
 /* Programmatic dependent launch (default on): each kernel may start its
  * prologue while the previous kernel on the stream drains, and waits for it
  * before touching its output.  0 turns it off (plain stream order) for

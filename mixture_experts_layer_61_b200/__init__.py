@@ -77,6 +77,7 @@ def lib():
             "moe_set_token_tile_cap": (I, [I]),
             "moe_set_programmatic_launch": (None, [I]),
             "moe_set_cta_pairs": (None, [I]),
+            "moe_ffn_fused": (I, [C]),
             "moe_kernel_launch_count": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
@@ -276,6 +277,11 @@ def set_token_tile_cap(n):
 def set_programmatic_launch(enable=True):
     """Programmatic dependent launch between the layer's kernels (default on)."""
     lib().moe_set_programmatic_launch(1 if enable else 0)
+
+
+def ffn_fused(cfg):
+    """True when the layer's expert FFN runs as one fused (decode) launch."""
+    return bool(lib().moe_ffn_fused(ctypes.byref(cfg)))
 
 
 def set_cta_pairs(enable=True):

@@ -109,7 +109,7 @@ Layout layout(const moe_config_t* c, int num_sms) {
         o = align256(o + bytes);
         return r;
     };
-    L.ctl = take(gemm_ctl_bytes(num_sms));
+    L.ctl = take(ctl_block_bytes(num_sms));
     L.logits = take(sizeof(float) * (size_t)c->T * c->E);
     L.ids = take(sizeof(int32_t) * (size_t)A);
     L.w = take(sizeof(float) * (size_t)A);
@@ -180,10 +180,31 @@ GemmLaunch down_launch(const void* act, long long x_rows, const int32_t* seg_off
     return d;
 }
 
-// gate/up (SwiGLU) + down over `n_groups` segments of X
+// gate/up (SwiGLU) + down over `n_groups` segments of X: one fused launch at
+// decode sizes (token-tile cap 32 or 64), else two GEMM launches.
+// `max_chunks` bounds the number of token chunks the segments can form.
 int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows, int H, int I,
             int dtype, const void* w13, const void* w2, void* act, void* y, int max_n, const GemmCtl& ctl,
-            cudaStream_t s) {
+            cudaStream_t s, long long max_chunks) {
+    if (max_n <= 64) {
+        FfnLaunch f;
+        f.x = x;
+        f.x_rows = x_rows;
+        f.w13 = w13;
+        f.w2 = w2;
+        f.H = H;
+        f.I = I;
+        f.seg_offsets = seg_offsets;
+        f.n_groups = n_groups;
+        f.seg_rows = seg_rows;
+        f.act = act;
+        f.y = y;
+        f.dtype = dtype;
+        f.max_n = max_n;
+        f.max_chunks = max_chunks;
+        int rc = launch_ffn_stream(f, ctl, s);
+        if (rc != 1) return rc;  // 1: not handled, use two launches
+    }
     int rc = launch_gemm(gate_up_launch(x, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w13, act, max_n),
                          ctl, s);
     if (rc != 0) return rc;
@@ -201,6 +222,11 @@ void router_tiling(GemmLaunch& g, int T) {
 int routed_max_n(const moe_config_t* c) {
     return pick_max_n((double)c->T * c->K / (double)c->E);
 }
+
+// Upper bounds on the token chunks of the routed segments (every chunk holds
+// at least one 16-row unit) and of a dense segment of T rows.
+long long routed_max_chunks(const moe_config_t* c) { return (long long)c->E + p_max(c) / 16 + 1; }
+long long dense_max_chunks(long long T) { return T / 16 + 1; }
 
 }  // namespace
 
@@ -233,7 +259,7 @@ size_t moe_workspace_size(const moe_config_t* cfg) {
 size_t moe_gemm_workspace_size(void) {
     DeviceInfo d;
     if (current_device(&d) != 0) return 0;
-    return gemm_ctl_bytes(d.num_sms);
+    return ctl_block_bytes(d.num_sms);
 }
 
 size_t dense_ffn_workspace_size(int T, int H, int I, int dtype) {
@@ -241,7 +267,7 @@ size_t dense_ffn_workspace_size(int T, int H, int I, int dtype) {
     if (eb == 0 || T < 0 || H <= 0 || I <= 0) return 0;
     DeviceInfo d;
     if (current_device(&d) != 0) return 0;
-    return align256(gemm_ctl_bytes(d.num_sms)) + align256((size_t)eb * T * I);
+    return align256(ctl_block_bytes(d.num_sms)) + align256((size_t)eb * T * I);
 }
 
 int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router, float* logits, void* workspace,
@@ -253,7 +279,7 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
     if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
-    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
     GemmLaunch g{};
     g.x = x;
     g.x_rows = cfg->T;
@@ -317,9 +343,10 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const void* w13
         return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
-    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
     return status_of(run_ffn(x_perm, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act,
-                             y_perm, routed_max_n(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+                             y_perm, routed_max_n(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream,
+                             routed_max_chunks(cfg)));
 }
 
 int moe_grouped_gate_up(const moe_config_t* cfg, const void* x_perm, const void* w13, const int32_t* offsets,
@@ -331,7 +358,7 @@ int moe_grouped_gate_up(const moe_config_t* cfg, const void* x_perm, const void*
     if (!aligned16(x_perm) || !aligned16(w13) || !aligned16(act) || !aligned16(workspace)) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
-    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
     return status_of(launch_gemm(gate_up_launch(x_perm, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype,
                                                 w13, act, routed_max_n(cfg)),
                                  gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
@@ -346,7 +373,7 @@ int moe_grouped_down(const moe_config_t* cfg, const void* act, const void* w2, c
     if (!aligned16(act) || !aligned16(w2) || !aligned16(y_perm) || !aligned16(workspace)) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
-    if (ws_bytes < gemm_ctl_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
     return status_of(launch_gemm(down_launch(act, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w2,
                                              y_perm, routed_max_n(cfg)),
                                  gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
@@ -423,14 +450,14 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
     if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s)) != 0)
         return status_of(rc);
     if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
-                      routed_max_n(cfg), ctl, s)) != 0)
+                      routed_max_n(cfg), ctl, s, routed_max_chunks(cfg))) != 0)
         return status_of(rc);
     const void* sh = nullptr;
     if (I_sh > 0) {
         void* act_sh = at<void>(workspace, L.act_sh);
         void* sh_out = at<void>(workspace, L.sh_out);
         if ((rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared, act_sh,
-                          sh_out, pick_max_n(cfg->T), ctl, s)) != 0)
+                          sh_out, pick_max_n(cfg->T), ctl, s, dense_max_chunks(cfg->T))) != 0)
             return status_of(rc);
         sh = sh_out;
     }
@@ -449,11 +476,11 @@ int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13, co
     DeviceInfo d;
     int rc = current_device(&d);
     if (rc != 0) return status_of(rc);
-    const size_t ctl_bytes = align256(gemm_ctl_bytes(d.num_sms));
+    const size_t ctl_bytes = align256(ctl_block_bytes(d.num_sms));
     if (ws_bytes < ctl_bytes + (size_t)eb * T * I) return MOE_ERR_WORKSPACE;
     void* act = at<void>(workspace, ctl_bytes);
     return status_of(run_ffn(x, T, nullptr, 1, T, H, I, dtype, w13, w2, act, out, pick_max_n(T),
-                             gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
+                             gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream, dense_max_chunks(T)));
 }
 
 int moe_check_status(void* workspace, moe_stream_t stream) {
@@ -471,7 +498,11 @@ int moe_check_status(void* workspace, moe_stream_t stream) {
         return MOE_ERR_CUDA;
     }
     if (st & kStatusTimeout) {
-        if (cudaMemset(workspace, 0, gemm_ctl_zero_bytes(d.num_sms)) != cudaSuccess) {
+        // re-zero the control words: status and stream-K counters, and the fused FFN's counters
+        const GemmCtl c = gemm_ctl(workspace, d.num_sms);
+        if (cudaMemset(workspace, 0, gemm_ctl_zero_bytes(d.num_sms)) != cudaSuccess ||
+            cudaMemset(c.ffn_ctl, 0, ctl_block_bytes(d.num_sms) - ((uint8_t*)c.ffn_ctl - (uint8_t*)workspace)) !=
+                cudaSuccess) {
             cudaGetLastError();
             return MOE_ERR_CUDA;
         }
@@ -489,6 +520,11 @@ int moe_set_token_tile_cap(int n) {
 }
 
 void moe_set_programmatic_launch(int enable) { set_pdl(enable != 0); }
+
+int moe_ffn_fused(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return routed_max_n(cfg) <= 64 ? 1 : 0;
+}
 
 void moe_set_cta_pairs(int enable) { set_cta_pairs(enable != 0); }
 

@@ -1,0 +1,550 @@
+// moe_ffn_stream.cuh -- the expert FFN for small per-expert batches (decode):
+// gate/up + SwiGLU and down in ONE persistent tcgen05 kernel with dynamic work
+// fetching.
+//
+// At decode sizes the layer is bound by streaming the activated experts'
+// weights from HBM (the "weight amplification" of the talk notes' "Decode
+// phase").  Two separate GEMM launches each pay a prologue, a pipeline ramp
+// and a tail in which the SMs that drew slower HBM service finish last.  Here
+// every block repeatedly takes the next work item from a global counter
+// (faster SMs simply take more), and the down projection's items follow the
+// gate/up items in the same launch, so the down weights start streaming while
+// the last gate/up tiles drain.
+//
+// Work items.  Phase A: gate/up tiles (expert chunk x 128 features), phase B:
+// down tiles (expert chunk x 256 features, two weight tiles per stage).  When
+// a phase has fewer tiles than about twice the SMs, each tile is cut into S
+// K-slices; the slice that completes a tile last (per-tile counter) sums all
+// slices' fp32 partials in slice order (deterministic) and runs the epilogue.
+// A phase-B item reads the SwiGLU activations of its token chunk, so before
+// loading them its producer waits (bounded) until every phase-A tile of that
+// chunk has been stored (per-chunk counter).  No block waits on work that is
+// not already held by a running block, so the wait always ends.
+//
+// Roles as in the grouped GEMM (warp 0 TMA, warp 1 TMEM + MMA, warps 2..5
+// epilogue); the producer publishes each item id to the other roles through a
+// small shared-memory ring.
+#pragma once
+
+#include "moe_gemm.cuh"
+
+namespace moe {
+
+constexpr int kFfnMaxChunks = 4096;   // token chunks (per-chunk phase-A counters)
+constexpr int kFfnTileCtrs = 4096;    // split-tile counters (phase A, then phase B)
+constexpr int kFfnRing = 4;
+// control ints: [0] work counter, [1] finished blocks, [2, 2+kFfnMaxChunks) chunk
+// counters, then kFfnTileCtrs tile counters
+constexpr int kFfnCtlInts = 2 + kFfnMaxChunks + kFfnTileCtrs;
+
+struct FfnParams {
+    const int32_t* seg_offsets;  // [n_groups + 1] row offsets, or nullptr: one group [0, seg_rows)
+    int n_groups;
+    int seg_rows;
+    int H, I;
+    void* act;           // [rows, I] SwiGLU activations (written in phase A, read in phase B)
+    void* y;             // [rows, H] output
+    int* ctl;            // kFfnCtlInts, zero on entry, left zero
+    float* partials;     // split-tile partial slots (up to 8 x gridDim.x)
+    unsigned* status;
+    uint64_t wait_limit_ns;
+    int withhold_first_load;
+};
+
+template <typename T, int kMaxN>
+struct FfnCfg {
+    static constexpr int kBK = 128 / Elt<T>::kBytes;
+    static constexpr int kWTileBytes = 128 * 128;
+    static constexpr int kXBoxRows = 16, kXBoxMid = 64;
+    static constexpr int kXTileBytes = kMaxN * 128;
+    static constexpr int kStageBytes = 2 * kWTileBytes + kXTileBytes;
+    static constexpr int kAccCols = 2 * kMaxN;
+    static constexpr int kNumAcc = 2;
+    static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
+    static constexpr int kMiscBytes = 768;
+    static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes;
+    static constexpr int kStagesRaw = kBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
+    static constexpr int kSlotFloats = 128 * kAccCols;
+    static_assert(kMaxN == 32 || kMaxN == 64, "decode token tiles");
+    static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
+};
+
+// One phase's split: S slices per tile (S = 1: whole tiles).
+__device__ __forceinline__ int ffn_slices(long long tiles, int KI, int G) {
+    if (tiles <= 0 || tiles >= 2LL * G) return 1;
+    long long s = (2LL * G + tiles - 1) / tiles;
+    long long cap = 4LL * G / tiles;
+    if (s > cap) s = cap;
+    if (s > 8) s = 8;
+    if (s > KI / 4) s = KI / 4;
+    return s < 1 ? 1 : (int)s;
+}
+
+struct FfnItem {
+    int phase;      // 0 gate/up, 1 down
+    long long tile; // within the phase
+    int slice, S;
+    int kb, ke;
+    long long slot;  // partial slot (split tiles)
+    long long ctr;   // tile counter index (split tiles)
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const int* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <typename T, int kMaxN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_ffn_stream_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_constant__ CUtensorMap tm_w2,
+                          const __grid_constant__ CUtensorMap tm_xa, const __grid_constant__ CUtensorMap tm_xa64,
+                          const __grid_constant__ CUtensorMap tm_xb, const __grid_constant__ CUtensorMap tm_xb64,
+                          const FfnParams p) {
+    using C = FfnCfg<T, kMaxN>;
+    using OutT = T;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stage_base = smem;
+    int* seg = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes);
+    int* cbase = seg + (kMaxGroups + 1);
+    uint8_t* misc = reinterpret_cast<uint8_t*>(cbase + (kMaxGroups + 1));
+    uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + C::kNumAcc;
+    uint64_t* ring_full = tempty + C::kNumAcc;
+    uint64_t* ring_empty = ring_full + kFfnRing;
+    uint64_t* drain_bar = ring_empty + kFfnRing;
+    int* ring = reinterpret_cast<int*>(drain_bar + 1);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kFfnRing);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    int* bcast = const_cast<int*>(abort_flag) + 1;
+    int* last_block = bcast + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_groups = p.n_groups;
+    const uint64_t limit = p.wait_limit_ns;
+    int* work_ctr = p.ctl;
+    int* done_ctr = p.ctl + 1;
+    int* chunk_done = p.ctl + 2;
+    int* tile_ctr = p.ctl + 2 + kFfnMaxChunks;
+
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < C::kNumAcc; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        for (int r = 0; r < kFfnRing; ++r) {
+            mbar_init(&ring_full[r], 1);
+            mbar_init(&ring_empty[r], 1 + 128);  // the MMA thread and every epilogue thread
+        }
+        mbar_init(drain_bar, 1);
+        fence_barrier_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&tm_w13);
+        tma_prefetch_desc(&tm_w2);
+        tma_prefetch_desc(&tm_xa);
+        tma_prefetch_desc(&tm_xa64);
+        tma_prefetch_desc(&tm_xb);
+        tma_prefetch_desc(&tm_xb64);
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, 512);
+    pdl_wait();
+    for (int g = threadIdx.x; g <= n_groups; g += blockDim.x)
+        seg[g] = p.seg_offsets ? p.seg_offsets[g] : (g == 0 ? 0 : p.seg_rows);
+    __syncthreads();
+    if (warp == 0) {
+        int running = 0;
+        for (int base = 0; base < n_groups; base += 32) {
+            int g = base + lane;
+            int n = g < n_groups ? chunks_of(seg[g + 1] - seg[g], kMaxN, 16) : 0;
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (g < n_groups) cbase[g] = running + incl - n;
+            running += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) cbase[n_groups] = running;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    // ---- the item space (identical in every thread)
+    const int G = gridDim.x;
+    const long long n_chunks = cbase[n_groups];
+    const int NFA = (p.I + 127) / 128, NFB = (p.H + 255) / 256;
+    const int KIA = (p.H + C::kBK - 1) / C::kBK, KIB = (p.I + C::kBK - 1) / C::kBK;
+    const long long tilesA = n_chunks * NFA, tilesB = n_chunks * NFB;
+    const int SA = ffn_slices(tilesA, KIA, G), SB = ffn_slices(tilesB, KIB, G);
+    const long long nA = tilesA * SA, nB = tilesB * SB;
+    const long long total = nA + nB;
+    const long long slotsA = SA > 1 ? nA : 0;
+    const bool oversize = n_chunks > kFfnMaxChunks || (SA > 1 && tilesA > kFfnTileCtrs / 2) ||
+                          (SB > 1 && tilesB > kFfnTileCtrs / 2);
+
+    auto item_of = [&](long long id, FfnItem& it, Tile& t) {
+        if (id < nA) {
+            it.phase = 0;
+            it.tile = id / SA;
+            it.slice = (int)(id - it.tile * SA);
+            it.S = SA;
+            it.kb = (int)((long long)it.slice * KIA / SA);
+            it.ke = (int)((long long)(it.slice + 1) * KIA / SA);
+            it.slot = id;
+            it.ctr = it.tile;
+            t = decode_tile_w(it.tile, seg, cbase, n_groups, NFA, 128, 16, 2 * p.I);
+        } else {
+            const long long j = id - nA;
+            it.phase = 1;
+            it.tile = j / SB;
+            it.slice = (int)(j - it.tile * SB);
+            it.S = SB;
+            it.kb = (int)((long long)it.slice * KIB / SB);
+            it.ke = (int)((long long)(it.slice + 1) * KIB / SB);
+            it.slot = slotsA + j;
+            it.ctr = kFfnTileCtrs / 2 + it.tile;
+            t = decode_tile_w(it.tile, seg, cbase, n_groups, NFB, 256, 16, p.H);
+        }
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------- item fetch + TMA loads
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            int fills[C::kStages];
+#pragma unroll
+            for (int s = 0; s < C::kStages; ++s) fills[s] = 0;
+            uint32_t kc = 0, n = 0;
+            bool withhold = p.withhold_first_load && blockIdx.x == 0;
+            bool ok = !oversize;
+            if (oversize) atomicOr(p.status, kStatusTimeout);
+            while (true) {
+                const int rs = n % kFfnRing;
+                const uint32_t rph = (n / kFfnRing) & 1u;
+                long long id = -1;
+                if (ok) {
+                    if (!mbar_wait_bounded(&ring_empty[rs], rph ^ 1u, limit, abort_flag)) {
+                        ok = false;
+                    } else {
+                        id = atomicAdd(work_ctr, 1);
+                        if (id >= total) id = -1;
+                    }
+                }
+                if (!ok) {
+                    // wake the consumers with the end marker (they may also give up on their own)
+                    ring[rs] = -1;
+                    mbar_arrive(&ring_full[rs]);
+                    break;
+                }
+                ring[rs] = (int)id;
+                mbar_arrive(&ring_full[rs]);
+                ++n;
+                if (id < 0) break;
+                FfnItem it;
+                Tile t;
+                item_of(id, it, t);
+                if (it.phase == 1) {
+                    // the activations of this token chunk: all NFA gate/up tiles stored
+                    const uint64_t t0 = global_ns();
+                    while ((int)ld_acquire_u32(&chunk_done[t.chunk]) < NFA) {
+                        if (*abort_flag || global_ns() - t0 > limit) {
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    if (!ok) continue;  // next turn publishes the end marker
+                    fence_proxy_async_global();
+                }
+                const CUtensorMap* tw = it.phase == 0 ? &tm_w13 : &tm_w2;
+                const CUtensorMap* tx = it.phase == 0 ? &tm_xa : &tm_xb;
+                const CUtensorMap* tx64 = it.phase == 0 ? &tm_xa64 : &tm_xb64;
+                const int second = it.phase == 0 ? p.I : 128;  // up rows, or the next 128 features
+                const uint32_t bytes = 2 * C::kWTileBytes + t.mma_n * 128;
+                for (int k = it.kb; k < it.ke; ++k, ++kc) {
+                    const int s = kc % C::kStages;
+                    const uint32_t ph = (kc / C::kStages) & 1u;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (withhold) {
+                        withhold = false;
+                        continue;
+                    }
+                    uint8_t* st = stage_base + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    const int kx = k * C::kBK;
+                    tma_load_2d(st, tw, &full[s], kx, t.wrow, pol_w);
+                    tma_load_2d(st + C::kWTileBytes, tw, &full[s], kx, t.wrow + second, pol_w);
+                    uint8_t* xs = st + 2 * C::kWTileBytes;
+                    int r = 0;
+                    if (kMaxN >= C::kXBoxMid)
+                        for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
+                            tma_load_2d(xs + r * 128, tx64, &full[s], kx, t.row0 + r, pol_x);
+                    for (; r < t.mma_n; r += C::kXBoxRows)
+                        tma_load_2d(xs + r * 128, tx, &full[s], kx, t.row0 + r, pol_x);
+                    ++fills[s];
+                }
+                if (!ok) continue;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+            }
+            for (int s = 0; s < C::kStages; ++s)
+                if (fills[s] > 0) mbar_drain(&full[s], (uint32_t)(fills[s] - 1) & 1u, limit);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t kc = 0, ac = 0, n = 0;
+            bool ok = true;
+            while (true) {
+                const int rs = n % kFfnRing;
+                const uint32_t rph = (n / kFfnRing) & 1u;
+                if (!mbar_wait_bounded(&ring_full[rs], rph, limit, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const long long id = ring[rs];
+                mbar_arrive(&ring_empty[rs]);
+                ++n;
+                if (id < 0) break;
+                FfnItem it;
+                Tile t;
+                item_of(id, it, t);
+                const int b = ac % C::kNumAcc;
+                const uint32_t aph = (ac / C::kNumAcc) & 1u;
+                if (!mbar_wait_bounded(&tempty[b], aph ^ 1u, limit, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + b * C::kAccCols;
+                const uint32_t d1 = d0 + kMaxN;
+                const uint32_t idesc = umma_idesc(Elt<T>::kMmaFmt, 128, t.mma_n);
+                for (int k = it.kb; k < it.ke; ++k, ++kc) {
+                    const int s = kc % C::kStages;
+                    const uint32_t ph = (kc / C::kStages) & 1u;
+                    if (!mbar_wait_bounded(&full[s], ph, limit, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t* st = stage_base + s * C::kStageBytes;
+                    const uint64_t a0 = umma_desc_sw128(smem_u32(st));
+                    const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
+                    const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kWTileBytes));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
+                        umma<T>(d0, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        umma<T>(d1, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&tfull[b]);
+                ++ac;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+                umma_commit(drain_bar);
+                mbar_drain(drain_bar, 0, limit);
+            }
+        }
+    } else {
+        // --------------------------------------------------------- epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        uint32_t ac = 0, n = 0;
+        while (true) {
+            const int rs = n % kFfnRing;
+            const uint32_t rph = (n / kFfnRing) & 1u;
+            if (!mbar_wait_bounded(&ring_full[rs], rph, limit, abort_flag)) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+                break;
+            }
+            const long long id = ring[rs];
+            mbar_arrive(&ring_empty[rs]);
+            ++n;
+            if (id < 0) break;
+            FfnItem it;
+            Tile t;
+            item_of(id, it, t);
+            const int b = ac % C::kNumAcc;
+            const uint32_t aph = (ac / C::kNumAcc) & 1u;
+            if (!mbar_wait_bounded(&tfull[b], aph, limit, abort_flag)) {
+                *abort_flag = 1;
+                atomicOr(p.status, kStatusTimeout);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * C::kAccCols;
+            const bool gate_up = it.phase == 0;
+            const int n_out = gate_up ? p.I : p.H;
+            const int f = t.f0 + r;
+            const bool v0 = f < n_out;
+            const bool v1 = gate_up ? v0 : (f + 128 < n_out);
+            OutT* orow = reinterpret_cast<OutT*>(gate_up ? p.act : p.y) + (long long)t.row0 * n_out + f;
+            auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {
+                if (gate_up) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
+                }
+                if (v0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * n_out, g[i]);
+                }
+                if (!gate_up && v1) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.nrows) store_out<OutT>(orow + 128 + (long long)(c0 + i) * n_out, u[i]);
+                }
+            };
+            bool finished = true;  // this item completed its tile
+            if (it.S == 1) {
+                for (int c0 = 0; c0 < t.nrows; c0 += 32) {
+                    uint32_t ga[32], ua[32];
+                    tmem_ld32_nowait(tacc + c0, ga);
+                    tmem_ld32_nowait(tacc + kMaxN + c0, ua);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float g[16], u[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            g[i] = __uint_as_float(ga[16 * h + i]);
+                            u[i] = __uint_as_float(ua[16 * h + i]);
+                        }
+                        if (c0 + 16 * h < t.nrows) emit(c0 + 16 * h, g, u);
+                    }
+                }
+            } else {
+                // split tile: publish this slice, the last slice sums them all in order
+                float4* mine = reinterpret_cast<float4*>(p.partials + it.slot * C::kSlotFloats);
+                for (int c0 = 0; c0 < t.nrows; c0 += 16) {
+                    float g[16];
+                    tmem_ld16(tacc + c0, g);
+                    if (v0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            mine[slot_f4((c0 >> 2) + q, r)] = make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                    }
+                    tmem_ld16(tacc + kMaxN + c0, g);
+                    if (v1) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            mine[slot_f4(((kMaxN + c0) >> 2) + q, r)] =
+                                make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                    }
+                }
+                __threadfence();
+                named_sync(1, 128);
+                if (r == 0) *bcast = atomicAdd(&tile_ctr[it.ctr], 1);
+                named_sync(1, 128);
+                finished = *bcast == it.S - 1;
+                if (finished) {
+                    __threadfence();
+                    const long long slot0 = it.slot - it.slice;  // slot of slice 0 of this tile
+                    for (int c0 = 0; c0 < t.nrows; c0 += 16) {
+                        float g[16], u[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
+                        for (int sl = 0; sl < it.S; ++sl) {
+                            if (sl == it.slice) {
+                                float v[16];
+                                tmem_ld16(tacc + c0, v);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) g[i] += v[i];
+                                tmem_ld16(tacc + kMaxN + c0, v);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) u[i] += v[i];
+                            } else {
+                                const float4* other =
+                                    reinterpret_cast<const float4*>(p.partials + (slot0 + sl) * C::kSlotFloats);
+                                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                                float4 a4[4], b4[4];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    a4[q] = v0 ? __ldcg(other + slot_f4((c0 >> 2) + q, r)) : z;
+                                    b4[q] = v1 ? __ldcg(other + slot_f4(((kMaxN + c0) >> 2) + q, r)) : z;
+                                }
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    g[4 * q] += a4[q].x;
+                                    g[4 * q + 1] += a4[q].y;
+                                    g[4 * q + 2] += a4[q].z;
+                                    g[4 * q + 3] += a4[q].w;
+                                    u[4 * q] += b4[q].x;
+                                    u[4 * q + 1] += b4[q].y;
+                                    u[4 * q + 2] += b4[q].z;
+                                    u[4 * q + 3] += b4[q].w;
+                                }
+                            }
+                        }
+                        emit(c0, g, u);
+                    }
+                    if (r == 0) tile_ctr[it.ctr] = 0;
+                }
+            }
+            if (gate_up && finished) {
+                // this gate/up tile's activations are stored: count it for its token chunk
+                fence_proxy_async_global();
+                __threadfence();
+                named_sync(1, 128);
+                if (r == 0) atomicAdd(&chunk_done[t.chunk], 1);
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[b]);
+            ++ac;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // the last block to finish re-zeroes the control words for the next launch
+    if (threadIdx.x == 0) {
+        __threadfence();
+        *last_block = atomicAdd(done_ctr, 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (*last_block) {
+        __threadfence();
+        const long long nc = n_chunks < kFfnMaxChunks ? n_chunks : kFfnMaxChunks;
+        for (long long c = threadIdx.x; c < nc; c += blockDim.x) chunk_done[c] = 0;
+        if (threadIdx.x == 0) {
+            *work_ctr = 0;
+            *done_ctr = 0;
+        }
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace moe

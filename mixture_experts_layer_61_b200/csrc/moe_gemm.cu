@@ -3,6 +3,7 @@
 // and the persistent launch.
 #include <mutex>
 
+#include "moe_ffn_stream.cuh"
 #include "moe_gemm.cuh"
 #include "moe_internal.h"
 
@@ -158,7 +159,81 @@ GemmCtl gemm_ctl(void* workspace, int num_sms) {
     size_t off = kCtlHeaderBytes + sizeof(int) * 2 * (size_t)num_sms;
     off = (off + 255) & ~size_t(255);
     c.partials = reinterpret_cast<float*>(b + off);
+    c.ffn_ctl = reinterpret_cast<int*>(b + ((gemm_ctl_bytes(num_sms) + 255) & ~size_t(255)));
     return c;
+}
+
+size_t ctl_block_bytes(int num_sms) {
+    return ((gemm_ctl_bytes(num_sms) + 255) & ~size_t(255)) + ((sizeof(int) * kFfnCtlInts + 255) & ~size_t(255));
+}
+
+namespace {
+
+template <typename T, int kMaxN>
+int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t stream) {
+    using C = FfnCfg<T, kMaxN>;
+    auto kern = moe_ffn_stream_kernel<T, kMaxN>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return -3;
+        }
+        attr_done = true;
+    }
+    // partial slots: up to 8 per SM of 128 x (2 * kMaxN) fp32 within the GEMM slot area
+    if ((size_t)8 * C::kSlotFloats * 4 > kSlotBytesMax * 2) return -1;
+    CUtensorMap w13, w2, xa, xa64, xb, xb64;
+    const int eb = Elt<T>::kBytes;
+    const CUtensorMapDataType dt = Elt<T>::kTma;
+    if (!make_map(&w13, dt, eb, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128)) return -3;
+    if (!make_map(&w2, dt, eb, L.w2, (long long)L.n_groups * L.H, L.I, 128)) return -3;
+    if (!make_map(&xa, dt, eb, L.x, L.x_rows, L.H, 16)) return -3;
+    if (!make_map(&xa64, dt, eb, L.x, L.x_rows, L.H, 64)) return -3;
+    if (!make_map(&xb, dt, eb, L.act, L.x_rows, L.I, 16)) return -3;
+    if (!make_map(&xb64, dt, eb, L.act, L.x_rows, L.I, 64)) return -3;
+    FfnParams p;
+    p.seg_offsets = L.seg_offsets;
+    p.n_groups = L.n_groups;
+    p.seg_rows = L.seg_rows;
+    p.H = L.H;
+    p.I = L.I;
+    p.act = L.act;
+    p.y = L.y;
+    p.ctl = ctl.ffn_ctl;
+    p.partials = ctl.partials;
+    p.status = ctl.status;
+    p.wait_limit_ns = wait_limit_ns();
+    p.withhold_first_load = take_withhold_flag();
+    cudaError_t e = launch_kernel(kern, dim3(num_sms), dim3(kGemmThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
+                                  xb, xb64, p);
+    count_launch();
+    if (e != cudaSuccess) cudaGetLastError();
+    return e == cudaSuccess ? 0 : -3;
+}
+
+}  // namespace
+
+int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t stream) {
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    if (L.max_n != 32 && L.max_n != 64) return 1;
+    if (L.n_groups < 1 || L.n_groups > kMaxGroups || L.max_chunks > kFfnMaxChunks) return 1;
+    // split-tile counters: each phase's tiles must fit half the counter array when split
+    const long long ntiles_a = L.max_chunks * ((L.I + 127) / 128);
+    const long long ntiles_b = L.max_chunks * ((L.H + 255) / 256);
+    if ((ntiles_a < 2LL * d.num_sms && ntiles_a > kFfnTileCtrs / 2) ||
+        (ntiles_b < 2LL * d.num_sms && ntiles_b > kFfnTileCtrs / 2))
+        return 1;
+    if (L.x_rows <= 0) return 0;
+    if (L.dtype == 0)
+        return L.max_n == 32 ? launch_ffn_variant<__nv_bfloat16, 32>(L, ctl, d.num_sms, stream)
+                             : launch_ffn_variant<__nv_bfloat16, 64>(L, ctl, d.num_sms, stream);
+    if (L.dtype == 1)
+        return L.max_n == 32 ? launch_ffn_variant<float, 32>(L, ctl, d.num_sms, stream)
+                             : launch_ffn_variant<float, 64>(L, ctl, d.num_sms, stream);
+    return -1;
 }
 
 namespace {

@@ -102,7 +102,7 @@ struct GemmCfg {
 
 // ------------------------------------------------------------- scheduling
 struct Tile {
-    int group, f0, row0, nrows, mma_n, wrow, nch;
+    int group, f0, row0, nrows, mma_n, wrow, nch, chunk;
 };
 
 struct Sched {
@@ -204,8 +204,8 @@ __device__ __forceinline__ int chunks_of(int rows, int max_n, int unit) {
     return (units + per - 1) / per;
 }
 
-__device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, const int* cbase, int n_groups, int NF,
-                                            int feat, int unit, const GemmParams& p) {
+__device__ __forceinline__ Tile decode_tile_w(long long tile, const int* seg, const int* cbase, int n_groups, int NF,
+                                              int feat, int unit, int w_group_stride) {
     // group: largest g with cbase[g] * NF <= tile
     int lo = 0, hi = n_groups - 1;
     while (lo < hi) {
@@ -226,9 +226,15 @@ __device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, cons
     t.row0 = seg[g] + start;
     t.nrows = n;
     t.mma_n = mn;
-    t.wrow = g * p.w_group_stride + f * feat;
+    t.wrow = g * w_group_stride + f * feat;
     t.nch = nch;
+    t.chunk = cbase[g] + j;
     return t;
+}
+
+__device__ __forceinline__ Tile decode_tile(long long tile, const int* seg, const int* cbase, int n_groups, int NF,
+                                            int feat, int unit, const GemmParams& p) {
+    return decode_tile_w(tile, seg, cbase, n_groups, NF, feat, unit, p.w_group_stride);
 }
 
 template <typename OutT>

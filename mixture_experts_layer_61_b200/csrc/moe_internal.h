@@ -72,8 +72,12 @@ struct GemmCtl {
     unsigned* status;
     int* counters;
     float* partials;
+    int* ffn_ctl;  // control words of the fused decode FFN kernel
 };
 GemmCtl gemm_ctl(void* workspace, int num_sms);
+// Bytes of the whole control block at the start of a workspace: the GEMM
+// control words and partial slots, then the fused FFN's control words.
+size_t ctl_block_bytes(int num_sms);
 
 // One GEMM launch.  X rows are tokens ([x_rows, kdim]), W rows are output
 // features ([w_rows, kdim]); out[row][feature] with row stride out_ld.
@@ -99,6 +103,27 @@ struct GemmLaunch {
 };
 
 int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
+
+// The expert FFN (gate/up + SwiGLU, then down) over n_groups segments of X in
+// one launch, for token-tile caps 32 and 64 (decode).  Returns 1 when the
+// configuration is outside what the fused kernel handles (caller falls back
+// to two GEMM launches).
+struct FfnLaunch {
+    const void* x;
+    long long x_rows;
+    const void* w13;
+    const void* w2;
+    int H, I;
+    const int32_t* seg_offsets;
+    int n_groups;
+    int seg_rows;
+    void* act;
+    void* y;
+    int dtype;
+    int max_n;
+    long long max_chunks;  // upper bound on token chunks (host side)
+};
+int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 
 // Token-tile cap for an expected number of rows per group (or the cap forced
 // by set_token_tile_cap, 0 = automatic).

@@ -156,3 +156,30 @@ def test_grouped_cta_pairs_match_single(kind):
     finally:
         moe.set_cta_pairs(True)
     assert e_pair < OUT_TOL and e_single < OUT_TOL
+
+
+@pytest.mark.parametrize("shape_kw,T", [(dict(H=512, E=8, K=2, I=1024), 1), (dict(H=1024, E=64, K=8, I=512), 40),
+                                        (dict(H=264, E=6, K=2, I=200), 77), (dict(H=2048, E=16, K=4, I=768), 200)])
+def test_fused_decode_ffn_matches_two_launch_path(shape_kw, T):
+    # the fused decode kernel (one launch, dynamic work, K-sliced tiles) against
+    # the separate gate/up and down GEMM launches on the same permuted rows
+    shape = small_shape(**shape_kw)
+    cfg = cfg_for(shape, T)
+    assert moe.ffn_fused(cfg)
+    w = mi.make_weights(shape, T, device="cuda", shared=False)
+    x = mi.make_x(shape, T, T, device="cuda")
+    ids = oracle.topk(mi.zipf_gumbel_logits(shape.E, T, 0.5, T).numpy(), shape.K)
+    g = moe.align_pad(cfg, torch.from_numpy(ids).cuda())
+    xp = moe.permute(cfg, x, g["sorted_ids"], g["scalars"])
+    ws = moe.alloc_workspace(moe.gemm_workspace_size())
+    y1, _ = moe.grouped_ffn(cfg, xp, w["w13"], w["w2"], g["offsets"], ws)
+    act = torch.empty_like(_)
+    y2 = torch.empty_like(y1)
+    moe.grouped_gate_up(cfg, xp, w["w13"], g["offsets"], ws, act)
+    moe.grouped_down(cfg, act, w["w2"], g["offsets"], ws, y2)
+    moe.check_status(ws)
+    P = int(g["scalars"][0].item())
+    valid = (g["sorted_ids"][:P] >= 0).cpu().numpy()
+    a = y1[:P].float().cpu().numpy()[valid]
+    b = y2[:P].float().cpu().numpy()[valid]
+    assert rel_err(a, b) < 1e-2
