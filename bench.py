@@ -39,9 +39,13 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 HBM_NOMINAL_GBS = 8000.0
 METRIC = "MoE layer tokens/s; % HBM BW (decode) / % tensor peak (prefill); tau vs DenseFA"
-# DRAM bytes per launch of the dominant kernel from ncu (dram__bytes_read.sum + dram__bytes_write.sum);
-# None until a capture of the current kernel exists.
-NCU_TRAFFIC = {}
+# DRAM bytes per launch of the dominant kernel from one ncu capture of the
+# current kernels (dram__bytes_read.sum + dram__bytes_write.sum); workloads
+# without a capture report None.  Summaries of the captures are in profiles/.
+NCU_TRAFFIC = {
+    "mixtral:2048": 2.181456e9 + 0.167618e9,   # moe_gemm_kernel gate/up + SwiGLU, CTA pairs
+    "mixtral:32": 2.824073e9 + 0.008427e9,     # moe_ffn_stream_kernel, fused decode FFN
+}
 
 
 def peaks():
@@ -119,12 +123,12 @@ def parse_workload(s):
 
 
 class Workload:
-    def __init__(self, shape, T, rank=0, device="cuda", skew=None):
+    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None):
         import mixture_experts_layer_61_b200 as moe
         self.moe = moe
         self.shape, self.T = shape, T
         seed = mi.seed_for(shape, T)
-        self.w = mi.make_weights(shape, seed, device=device)
+        self.w = weights if weights is not None else mi.make_weights(shape, seed, device=device)
         self.x = mi.make_x(shape, T, seed + 100 * rank, device=device)
         self.logits = None
         if skew is not None:
@@ -151,6 +155,7 @@ class Workload:
         self.s_shws = (moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, shape.I_sh, self.cfg.dtype), device)
                        if shape.I_sh else None)
         self.s_al = moe.align_buffers(self.cfg, device)
+        self.fused = moe.ffn_fused(self.cfg)
 
     def capture(self):
         """Record one forward into a CUDA graph (the library makes no allocation
@@ -184,9 +189,15 @@ class Workload:
         ev[3].record()
         m.permute(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
         ev[4].record()
-        m.grouped_gate_up(c, self.s_xp, self.w["w13"], self.al["offsets"], self.gws, self.s_act)
-        ev[5].record()
-        m.grouped_down(c, self.s_act, self.w["w2"], self.al["offsets"], self.gws, self.s_y)
+        if self.fused:
+            # the layer's expert FFN is one fused launch (gate/up + SwiGLU + down)
+            m.grouped_ffn(c, self.s_xp, self.w["w13"], self.w["w2"], self.al["offsets"], self.gws, self.s_act,
+                          self.s_y)
+            ev[5].record()
+        else:
+            m.grouped_gate_up(c, self.s_xp, self.w["w13"], self.al["offsets"], self.gws, self.s_act)
+            ev[5].record()
+            m.grouped_down(c, self.s_act, self.w["w2"], self.al["offsets"], self.gws, self.s_y)
         ev[6].record()
         if self.s_sh is not None:
             m.dense_ffn(self.x, self.w["w13_sh"], self.w["w2_sh"], self.s_shws, self.s_sh)
@@ -195,6 +206,8 @@ class Workload:
         ev[8].record()
 
     STAGES = ("router", "topk", "align", "permute", "gate_up", "down", "shared", "combine")
+    # names when the expert FFN is one fused launch ("down" is then empty)
+    STAGES_FUSED = ("router", "topk", "align", "permute", "ffn", "down", "shared", "combine")
 
 
 def l2_flush_buffer(device):
@@ -218,6 +231,23 @@ def time_steps(fn, steps, flush, stream_sync=True):
     return times
 
 
+# ------------------------------------------------------- multi-rank timing
+
+def max_over_ranks(total_ms, dist, device):
+    """The slowest rank's device time (ms); replicas run their own batches, so
+    whole-job throughput is set by the slowest one."""
+    if dist is None:
+        return float(total_ms)
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens_per_s(world, T, steps, max_total_ms):
+    """Whole-job tokens/s: every rank processes T tokens per step."""
+    return world * T * steps / (max_total_ms / 1e3)
+
+
 # ------------------------------------------------------------ accounting
 
 def algorithmic(shape, T, E_active):
@@ -236,6 +266,13 @@ def gate_up_work(shape, T, E_active):
     experts' W1/W3, flops 2 * T K * H * 2I."""
     eb = 2 if shape.dtype == "bf16" else 4
     return E_active * 2 * shape.I * shape.H * eb, 2.0 * T * shape.K * shape.H * 2 * shape.I
+
+
+def ffn_work(shape, T, E_active):
+    """Fused expert FFN: weight bytes of the activated experts' W1/W3/W2,
+    flops 2 * T K * 3 * H * I."""
+    eb = 2 if shape.dtype == "bf16" else 4
+    return E_active * 3 * shape.I * shape.H * eb, 2.0 * T * shape.K * 3 * shape.H * shape.I
 
 
 def dense_times(shape, T, I_d, steps, warmup, flush, device, seed):
@@ -366,28 +403,25 @@ def main():
         launches = wl.launches_per_step * args.steps  # graph replays launch the captured kernels
     if dist:
         dist.barrier()
-    total_ms = sum(times)
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(times), dist, device)
     wl.moe.check_status(wl.ws)
     stats = wl.stats.cpu().tolist()
     P, E_active = stats[0], stats[1]
     ms_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    value = replica_tokens_per_s(world, T, args.steps, total_ms)
     # ---- per-stage breakdown (same kernels, one ABI call per stage)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
-    stage_ms = {s: [] for s in Workload.STAGES}
+    names = Workload.STAGES_FUSED if wl.fused else Workload.STAGES
+    stage_ms = {s: [] for s in names}
     for i in range(args.warmup + args.steps):
         flush.zero_()
         wl.staged_step(ev)
         ev[8].synchronize()
         if i >= args.warmup:
-            for j, s in enumerate(Workload.STAGES):
+            for j, s in enumerate(names):
                 stage_ms[s].append(ev[j].elapsed_time(ev[j + 1]))
     wl.moe.check_status(wl.gws)
-    stages = {s: round(statistics.median(v), 4) for s, v in stage_ms.items()}
+    stages = {s: round(statistics.median(v), 4) for s, v in stage_ms.items() if not (wl.fused and s == "down")}
 
     if args.quick:
         if rank == 0:
@@ -402,9 +436,14 @@ def main():
             dist.destroy_process_group()
         return
 
-    # ---- roofline of the dominant kernel (grouped gate/up + SwiGLU)
-    gu_bytes, gu_flops = gate_up_work(shape, T, E_active)
-    t_gu = stages["gate_up"] * 1e-3
+    # ---- roofline of the dominant kernel: the grouped gate/up + SwiGLU GEMM,
+    # or the fused expert FFN when the layer runs it as one launch
+    if wl.fused:
+        gu_bytes, gu_flops = ffn_work(shape, T, E_active)
+        t_gu = stages["ffn"] * 1e-3
+    else:
+        gu_bytes, gu_flops = gate_up_work(shape, T, E_active)
+        t_gu = stages["gate_up"] * 1e-3
     hbm_peak = pk["hbm_gbs"]
     tc_peak = pk["bf16_tflops"] * (0.5 if shape.dtype == "fp32" else 1.0)  # tf32 is half the bf16 rate
     bound = "tensor" if gu_flops / (tc_peak * 1e12) > gu_bytes / (hbm_peak * 1e9) else "hbm"
@@ -416,7 +455,8 @@ def main():
         ach = gu_flops / t_gu / 1e12
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": round(ach / tc_peak, 4), "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4)}
-    roof["kernel"] = "moe_gemm_kernel (grouped gate/up + SwiGLU)"
+    roof["kernel"] = ("moe_ffn_stream_kernel (fused expert FFN: gate/up + SwiGLU + down)" if wl.fused
+                      else "moe_gemm_kernel (grouped gate/up + SwiGLU)")
     roof["peak_source"] = f"{pk_kind} ({'MEASURED_PEAKS.json' if pk_kind == 'measured' else 'fallback'})"
     roof["traffic"] = NCU_TRAFFIC.get(f"{shape.name}:{T}")
     B_alg, F_alg = algorithmic(shape, T, E_active)
@@ -439,12 +479,8 @@ def main():
     if dist:
         dist.barrier()
     e2e_times = time_steps(e2e_step, args.steps, flush)
-    e2e_total = sum(e2e_times)
-    if dist:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e = {"value": world * T * args.steps / (e2e_total / 1e3), "unit": "tokens/s",
+    e2e_total = max_over_ranks(sum(e2e_times), dist, device)
+    e2e = {"value": replica_tokens_per_s(world, T, args.steps, e2e_total), "unit": "tokens/s",
            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
            "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
 
@@ -509,46 +545,50 @@ def main():
 
 
 def run_sweep(args, device, flush, pk):
-    """Every configured workload (decode and prefill T of each layer shape, and
-    the DeepSeek-V3 routing-skew sweep): tokens/s, roofline fractions and tau."""
+    """Every configured workload (decode and prefill T of each layer shape) and
+    the DeepSeek-V3-shaped routing-skew sweep (Zipf s in {0, 0.5, 1, 1.5},
+    T = 1 .. 4096 in powers of two): tokens/s, activated experts, padded
+    fraction, roofline fractions and tau against DenseFA (same T, same
+    library).  Weights are generated once per layer shape."""
     import mixture_experts_layer_61_b200 as moe
     rows = []
-    plan = []
+    steps = max(5, args.steps // 2)
     for name in ("mixtral", "qwen2moe", "deepseekv3"):
         sh = mi.SHAPES[name]
-        for T in sh.decode_T + sh.prefill_T:
-            plan.append((sh, T, None))
-    for s in (0.0, 0.5, 1.0, 1.5):
-        for T in (1, 8, 64, 512, 4096):
-            plan.append((mi.SHAPES["deepseekv3"], T, s))
-    steps = max(5, args.steps // 2)
-    fa_cache = {}
-    for sh, T, s in plan:
-        wl = Workload(sh, T, 0, device, skew=s)
-        wl.capture()
-        for _ in range(3):
-            wl.replay()
-        torch.cuda.synchronize()
-        t = statistics.median(time_steps(wl.replay, steps, flush))
-        moe.check_status(wl.ws)
-        st = wl.stats.cpu().tolist()
-        B, F = algorithmic(sh, T, st[1])
-        key = (sh.name, T)
-        if key not in fa_cache:
-            fa_cache[key] = dense_times(sh, T, sh.I_FA, steps, 3, flush, device, mi.seed_for(sh, T, 50))
-        row = {"layer": sh.name, "T": T, "skew": s, "ms": round(t, 4), "tokens_per_s": round(T / t * 1e3, 1),
-               "E_active": st[1], "P": st[0], "padded_fraction": round((st[0] - T * sh.K) / max(st[0], 1), 4),
-               "hbm_frac_8TBs": round(B / (t * 1e-3) / 8e12, 4),
-               "hbm_frac_measured": round(B / (t * 1e-3) / (pk["hbm_gbs"] * 1e9), 4),
-               "tensor_frac": round(F / (t * 1e-3) / (pk["bf16_tflops"] * 1e12), 4),
-               "tau_FA": round(t / fa_cache[key], 4)}
-        rows.append(row)
-        del wl
+        weights = mi.make_weights(sh, mi.seed_for(sh, 0), device=device)
+        plan = [(T, None) for T in sh.decode_T + sh.prefill_T]
+        if name == "deepseekv3":
+            plan += [(2 ** k, s) for s in (0.0, 0.5, 1.0, 1.5) for k in range(13)]
+        fa_cache = {}
+        for T, s in plan:
+            wl = Workload(sh, T, 0, device, skew=s, weights=weights)
+            wl.capture()
+            for _ in range(3):
+                wl.replay()
+            torch.cuda.synchronize()
+            t = statistics.median(time_steps(wl.replay, steps, flush))
+            moe.check_status(wl.ws)
+            st = wl.stats.cpu().tolist()
+            B, F = algorithmic(sh, T, st[1])
+            if T not in fa_cache:
+                fa_cache[T] = dense_times(sh, T, sh.I_FA, steps, 3, flush, device, mi.seed_for(sh, T, 50))
+            row = {"layer": sh.name, "T": T, "skew": s, "ms": round(t, 4), "tokens_per_s": round(T / t * 1e3, 1),
+                   "E_active": st[1], "P": st[0],
+                   "padded_fraction": round((st[0] - T * sh.K) / max(st[0], 1), 4),
+                   "hbm_frac_8TBs": round(B / (t * 1e-3) / 8e12, 4),
+                   "hbm_frac_measured": round(B / (t * 1e-3) / (pk["hbm_gbs"] * 1e9), 4),
+                   "tensor_frac": round(F / (t * 1e-3) / (pk["bf16_tflops"] * 1e12), 4),
+                   "roofline_frac": round(max(F / (pk["bf16_tflops"] * 1e12), B / (pk["hbm_gbs"] * 1e9)) /
+                                          (t * 1e-3), 4),
+                   "tau_FA": round(t / fa_cache[T], 4), "fused_ffn": bool(wl.fused)}
+            rows.append(row)
+            if args.sweep_out:
+                with open(args.sweep_out, "a") as f:
+                    f.write(json.dumps(row) + "\n")
+            del wl
+            torch.cuda.empty_cache()
+        del weights
         torch.cuda.empty_cache()
-    if args.sweep_out:
-        with open(args.sweep_out, "w") as f:
-            for r in rows:
-                f.write(json.dumps(r) + "\n")
     return rows
 
 

@@ -93,6 +93,14 @@ int64_t moe_padded_rows_max(const moe_config_t* cfg);
  * control words zero after every call that completes without a timeout. */
 size_t moe_workspace_size(const moe_config_t* cfg);
 
+/* Byte offset, inside the moe_layer_forward workspace, of the fp32 router
+ * logits [T,E] the last forward computed (-1 on a bad configuration).  For
+ * T <= 64 the forward computes them on the CUDA cores (fp32 sums of exact
+ * products) in the same launch as top-K and alignment, otherwise with the
+ * tensor-core router GEMM; either way they are what top-K selected on unless
+ * logits_override was given. */
+int64_t moe_layer_logits_offset(const moe_config_t* cfg);
+
 /* Bytes of workspace moe_router_gemm / moe_grouped_ffn / dense_ffn need (the
  * control words and stream-K partial tiles only), same zeroing rule. */
 size_t moe_gemm_workspace_size(void);
@@ -238,9 +246,10 @@ void moe_set_programmatic_launch(int enable);
  * results are identical up to fp32 summation order. */
 void moe_set_cta_pairs(int enable);
 
-/* Test hook: when nonzero, the next GEMM launch withholds the first operand
- * load of block 0, so that block's waits run out and report
- * MOE_ERR_TIMEOUT through moe_check_status().  Cleared after one launch. */
+/* Test hook: when nonzero, the next GEMM or fused-FFN launch withholds one
+ * operand load (the first load of block 0, or of work item 0 in the fused
+ * FFN), so the waits that depend on it run out and report MOE_ERR_TIMEOUT
+ * through moe_check_status().  Cleared after one launch. */
 void moe_debug_withhold_first_load(int enable);
 
 /* Number of kernels this library launched since load (all entry points). */

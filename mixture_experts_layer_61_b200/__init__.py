@@ -78,6 +78,7 @@ def lib():
             "moe_set_programmatic_launch": (None, [I]),
             "moe_set_cta_pairs": (None, [I]),
             "moe_ffn_fused": (I, [C]),
+            "moe_layer_logits_offset": (ctypes.c_int64, [C]),
             "moe_kernel_launch_count": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
@@ -277,6 +278,15 @@ def set_token_tile_cap(n):
 def set_programmatic_launch(enable=True):
     """Programmatic dependent launch between the layer's kernels (default on)."""
     lib().moe_set_programmatic_launch(1 if enable else 0)
+
+
+def layer_logits(cfg, ws):
+    """View of the fp32 router logits [T,E] of the last layer_forward in `ws`."""
+    off = int(lib().moe_layer_logits_offset(ctypes.byref(cfg)))
+    if off < 0:
+        raise MoeError(-1, "moe_layer_logits_offset")
+    n = cfg.T * cfg.E * 4
+    return ws[off:off + n].view(torch.float32).view(cfg.T, cfg.E)
 
 
 def ffn_fused(cfg):

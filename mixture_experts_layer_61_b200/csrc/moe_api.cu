@@ -93,7 +93,8 @@ long long p_max(const moe_config_t* c) {
 }
 
 struct Layout {
-    size_t ctl, logits, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm, act, act_sh, sh_out;
+    size_t ctl, logits, route_part, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm, act, act_sh,
+        sh_out;
     size_t total;
 };
 
@@ -111,6 +112,8 @@ Layout layout(const moe_config_t* c, int num_sms) {
     };
     L.ctl = take(ctl_block_bytes(num_sms));
     L.logits = take(sizeof(float) * (size_t)c->T * c->E);
+    // partial router sums of the small-batch routing kernel (slices of 256 hidden elements)
+    L.route_part = take(c->T <= kSmallRouteMaxT ? sizeof(float) * ((size_t)c->H / 256 + 1) * c->T * c->E : 0);
     L.ids = take(sizeof(int32_t) * (size_t)A);
     L.w = take(sizeof(float) * (size_t)A);
     L.counts = take(sizeof(int32_t) * (size_t)c->E);
@@ -186,7 +189,7 @@ GemmLaunch down_launch(const void* act, long long x_rows, const int32_t* seg_off
 int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows, int H, int I,
             int dtype, const void* w13, const void* w2, void* act, void* y, int max_n, const GemmCtl& ctl,
             cudaStream_t s, long long max_chunks) {
-    if (max_n <= 64) {
+    if (max_n <= 128) {
         FfnLaunch f;
         f.x = x;
         f.x_rows = x_rows;
@@ -254,6 +257,13 @@ size_t moe_workspace_size(const moe_config_t* cfg) {
     DeviceInfo d;
     if (current_device(&d) != 0) return 0;
     return layout(cfg, d.num_sms).total;
+}
+
+int64_t moe_layer_logits_offset(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return -1;
+    DeviceInfo d;
+    if (current_device(&d) != 0) return -1;
+    return (int64_t)layout(cfg, d.num_sms).logits;
 }
 
 size_t moe_gemm_workspace_size(void) {
@@ -423,8 +433,15 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
     void* y_perm = x_perm;
     const long long P = p_max(cfg);
 
-    // router
-    {
+    if (cfg->T <= kSmallRouteMaxT && cfg->H % 8 == 0) {
+        // router logits, top-K and alignment in one launch (decode-sized batches)
+        int* route_ctr = reinterpret_cast<int*>(at<uint8_t>(workspace, L.ctl)) + 16;  // in the control header
+        if ((rc = launch_route_small(cfg->T, cfg->H, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, cfg->tile_B, P,
+                                     cfg->dtype, x, w_router, logits_override, at<float>(workspace, L.route_part),
+                                     logits, ids, w, counts, offsets, sorted_ids, block_expert, pos, scalars,
+                                     stats_out, route_ctr, s)) != 0)
+            return status_of(rc);
+    } else {
         GemmLaunch g{};
         g.x = x;
         g.x_rows = cfg->T;
@@ -440,13 +457,13 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
         g.dtype = cfg->dtype;
         router_tiling(g, cfg->T);
         if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
+        if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm,
+                              logits_override ? logits_override : logits, ids, w, s)) != 0)
+            return status_of(rc);
+        if ((rc = launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, P, ids, counts, offsets, sorted_ids, block_expert,
+                               pos, scalars, stats_out, s)) != 0)
+            return status_of(rc);
     }
-    if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, logits_override ? logits_override : logits,
-                          ids, w, s)) != 0)
-        return status_of(rc);
-    if ((rc = launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, P, ids, counts, offsets, sorted_ids, block_expert, pos,
-                           scalars, stats_out, s)) != 0)
-        return status_of(rc);
     if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s)) != 0)
         return status_of(rc);
     if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
@@ -523,7 +540,7 @@ void moe_set_programmatic_launch(int enable) { set_pdl(enable != 0); }
 
 int moe_ffn_fused(const moe_config_t* cfg) {
     if (check_cfg(cfg) != MOE_OK) return 0;
-    return routed_max_n(cfg) <= 64 ? 1 : 0;
+    return routed_max_n(cfg) <= 128 ? 1 : 0;
 }
 
 void moe_set_cta_pairs(int enable) { set_cta_pairs(enable != 0); }

@@ -49,6 +49,7 @@ struct FfnParams {
     unsigned* status;
     uint64_t wait_limit_ns;
     int withhold_first_load;
+    int max_slots_phase;  // partial slots available to each phase
 };
 
 template <typename T, int kMaxN>
@@ -67,15 +68,15 @@ struct FfnCfg {
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
     static constexpr int kSlotFloats = 128 * kAccCols;
-    static_assert(kMaxN == 32 || kMaxN == 64, "decode token tiles");
+    static_assert(kMaxN == 32 || kMaxN == 64 || kMaxN == 128, "decode token tiles");
     static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
 };
 
 // One phase's split: S slices per tile (S = 1: whole tiles).
-__device__ __forceinline__ int ffn_slices(long long tiles, int KI, int G) {
+__device__ __forceinline__ int ffn_slices(long long tiles, int KI, int G, int max_slots) {
     if (tiles <= 0 || tiles >= 2LL * G) return 1;
     long long s = (2LL * G + tiles - 1) / tiles;
-    long long cap = 4LL * G / tiles;
+    long long cap = (4LL * G < max_slots ? 4LL * G : max_slots) / tiles;
     if (s > cap) s = cap;
     if (s > 8) s = 8;
     if (s > KI / 4) s = KI / 4;
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int NFA = (p.I + 127) / 128, NFB = (p.H + 255) / 256;
     const int KIA = (p.H + C::kBK - 1) / C::kBK, KIB = (p.I + C::kBK - 1) / C::kBK;
     const long long tilesA = n_chunks * NFA, tilesB = n_chunks * NFB;
-    const int SA = ffn_slices(tilesA, KIA, G), SB = ffn_slices(tilesB, KIB, G);
+    const int SA = ffn_slices(tilesA, KIA, G, p.max_slots_phase), SB = ffn_slices(tilesB, KIB, G, p.max_slots_phase);
     const long long nA = tilesA * SA, nB = tilesB * SB;
     const long long total = nA + nB;
     const long long slotsA = SA > 1 ? nA : 0;
@@ -227,13 +228,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         // ------------------------------------------- item fetch + TMA loads
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_w_once = policy_evict_first();
+            const uint64_t pol_w_shared = policy_evict_normal();
             const uint64_t pol_x = policy_evict_last();
             int fills[C::kStages];
 #pragma unroll
             for (int s = 0; s < C::kStages; ++s) fills[s] = 0;
             uint32_t kc = 0, n = 0;
-            bool withhold = p.withhold_first_load && blockIdx.x == 0;
+            bool withhold = false;  // test hook: armed for work item 0, whichever block takes it
             bool ok = !oversize;
             if (oversize) atomicOr(p.status, kStatusTimeout);
             while (true) {
@@ -261,6 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 FfnItem it;
                 Tile t;
                 item_of(id, it, t);
+                if (id == 0 && p.withhold_first_load) withhold = true;
                 if (it.phase == 1) {
                     // the activations of this token chunk: all NFA gate/up tiles stored
                     const uint64_t t0 = global_ns();
@@ -279,6 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const CUtensorMap* tx64 = it.phase == 0 ? &tm_xa64 : &tm_xb64;
                 const int second = it.phase == 0 ? p.I : 128;  // up rows, or the next 128 features
                 const uint32_t bytes = 2 * C::kWTileBytes + t.mma_n * 128;
+                const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
                     const uint32_t ph = (kc / C::kStages) & 1u;

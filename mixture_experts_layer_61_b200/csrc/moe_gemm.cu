@@ -181,8 +181,8 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
         }
         attr_done = true;
     }
-    // partial slots: up to 8 per SM of 128 x (2 * kMaxN) fp32 within the GEMM slot area
-    if ((size_t)8 * C::kSlotFloats * 4 > kSlotBytesMax * 2) return -1;
+    // partial slots of 128 x (2 * kMaxN) fp32 share the GEMM slot area (2 x 256 KB per SM)
+    const int slots_total = (int)((kSlotBytesMax * 2 * (size_t)num_sms) / ((size_t)C::kSlotFloats * 4));
     CUtensorMap w13, w2, xa, xa64, xb, xb64;
     const int eb = Elt<T>::kBytes;
     const CUtensorMapDataType dt = Elt<T>::kTma;
@@ -205,6 +205,7 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     p.status = ctl.status;
     p.wait_limit_ns = wait_limit_ns();
     p.withhold_first_load = take_withhold_flag();
+    p.max_slots_phase = slots_total / 2;
     cudaError_t e = launch_kernel(kern, dim3(num_sms), dim3(kGemmThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
                                   xb, xb64, p);
     count_launch();
@@ -218,7 +219,7 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
     DeviceInfo d;
     int rc = current_device(&d);
     if (rc != 0) return rc;
-    if (L.max_n != 32 && L.max_n != 64) return 1;
+    if (L.max_n != 32 && L.max_n != 64 && L.max_n != 128) return 1;
     if (L.n_groups < 1 || L.n_groups > kMaxGroups || L.max_chunks > kFfnMaxChunks) return 1;
     // split-tile counters: each phase's tiles must fit half the counter array when split
     const long long ntiles_a = L.max_chunks * ((L.I + 127) / 128);
@@ -227,12 +228,16 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
         (ntiles_b < 2LL * d.num_sms && ntiles_b > kFfnTileCtrs / 2))
         return 1;
     if (L.x_rows <= 0) return 0;
-    if (L.dtype == 0)
-        return L.max_n == 32 ? launch_ffn_variant<__nv_bfloat16, 32>(L, ctl, d.num_sms, stream)
-                             : launch_ffn_variant<__nv_bfloat16, 64>(L, ctl, d.num_sms, stream);
-    if (L.dtype == 1)
-        return L.max_n == 32 ? launch_ffn_variant<float, 32>(L, ctl, d.num_sms, stream)
-                             : launch_ffn_variant<float, 64>(L, ctl, d.num_sms, stream);
+    if (L.dtype == 0) {
+        if (L.max_n == 32) return launch_ffn_variant<__nv_bfloat16, 32>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 64) return launch_ffn_variant<__nv_bfloat16, 64>(L, ctl, d.num_sms, stream);
+        return launch_ffn_variant<__nv_bfloat16, 128>(L, ctl, d.num_sms, stream);
+    }
+    if (L.dtype == 1) {
+        if (L.max_n == 32) return launch_ffn_variant<float, 32>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 64) return launch_ffn_variant<float, 64>(L, ctl, d.num_sms, stream);
+        return launch_ffn_variant<float, 128>(L, ctl, d.num_sms, stream);
+    }
     return -1;
 }
 
@@ -248,7 +253,7 @@ int pick_max_n(double rows_per_group) {
         return g_token_tile_cap;
     if (rows_per_group <= 24.0) return 32;
     if (rows_per_group <= 56.0) return 64;
-    if (rows_per_group <= 112.0) return 128;
+    if (rows_per_group <= 128.0) return 128;
     return 256;
 }
 

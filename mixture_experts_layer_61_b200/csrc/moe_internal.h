@@ -105,7 +105,7 @@ struct GemmLaunch {
 int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 
 // The expert FFN (gate/up + SwiGLU, then down) over n_groups segments of X in
-// one launch, for token-tile caps 32 and 64 (decode).  Returns 1 when the
+// one launch, for token-tile caps 32, 64 and 128 (memory-bound sizes).  Returns 1 when the
 // configuration is outside what the fused kernel handles (caller falls back
 // to two GEMM launches).
 struct FfnLaunch {
@@ -138,6 +138,14 @@ int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logi
 int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids, int32_t* counts,
                  int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
                  int32_t* stats_copy, cudaStream_t stream);
+// Router logits (CUDA cores) + top-K + alignment in one launch, for small T.
+constexpr int kSmallRouteMaxT = 64;
+// `part` holds (H/256 + 1) * T * E floats of partial router sums.
+int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, long long P_max, int dtype,
+                       const void* x, const void* w_r, const float* logits_override, float* part, float* logits,
+                       int32_t* ids, float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                       int32_t* block_expert, int32_t* pos, int32_t* scalars, int32_t* stats_copy, int* done_ctr,
+                       cudaStream_t stream);
 int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
                    const int32_t* scalars, void* x_perm, cudaStream_t stream);
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,

@@ -27,16 +27,10 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 }
 
 // One warp per token.  Lane l owns experts l, l+32, ...; K passes of a warp
-// arg-max over the experts not yet taken.
-__global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int score_fn, int renorm,
-                                                        const float* __restrict__ logits, int32_t* __restrict__ ids,
-                                                        float* __restrict__ w) {
-    pdl_launch_dependents();
-    pdl_wait();
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (t >= T) return;
-    const float* l = logits + (size_t)t * E;
+// arg-max over the experts not yet taken.  Logits are read through L2 (they
+// may have been written by other blocks of the same kernel).
+__device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int E, int K, int score_fn, int renorm,
+                                               int32_t* __restrict__ ids_t, float* __restrict__ w_t, int lane) {
     uint32_t taken = 0;  // bit j: expert lane + 32 j
     float sel_v[16];
     int sel_i[16];
@@ -46,7 +40,7 @@ __global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int
         int bi = INT_MAX;
         for (int j = 0, e = lane; e < E; ++j, e += 32) {
             if ((taken >> j) & 1u) continue;
-            const float v = l[e];
+            const float v = __ldcg(l + e);
             if (better(v, e, bv, bi)) {
                 bv = v;
                 bi = e;
@@ -73,7 +67,7 @@ __global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
             bi = cand;
-            bv = l[bi];
+            bv = __ldcg(l + bi);
         }
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
         sel_v[k] = bv;
@@ -89,11 +83,11 @@ __global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int
             for (int k = 0; k < K; ++k) den += expf(sel_v[k] - m);
         } else {
             m = -INFINITY;
-            for (int e = lane; e < E; e += 32) m = fmaxf(m, l[e]);
+            for (int e = lane; e < E; e += 32) m = fmaxf(m, __ldcg(l + e));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             float part = 0.f;
-            for (int e = lane; e < E; e += 32) part += expf(l[e] - m);
+            for (int e = lane; e < E; e += 32) part += expf(__ldcg(l + e) - m);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
             den = part;
@@ -113,9 +107,20 @@ __global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int
         int id = 0;
         for (int k = 0; k < K; ++k)
             if (k == lane) id = sel_i[k];
-        ids[(size_t)t * K + lane] = id;
-        w[(size_t)t * K + lane] = wk;
+        ids_t[lane] = id;
+        w_t[lane] = wk;
     }
+}
+
+__global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int score_fn, int renorm,
+                                                        const float* __restrict__ logits, int32_t* __restrict__ ids,
+                                                        float* __restrict__ w) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    topk_one_token(logits + (size_t)t * E, E, K, score_fn, renorm, ids + (size_t)t * K, w + (size_t)t * K, lane);
 }
 
 int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,
@@ -167,12 +172,13 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
     return r;
 }
 
-__global__ void __launch_bounds__(kAlignThreads, 1)
-    align_kernel(int T, int K, int E, int B, long long P_max, const int32_t* __restrict__ ids,
-                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
-                 int32_t* __restrict__ block_expert, int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
-                 int32_t* __restrict__ stats_copy) {
-    extern __shared__ int sm[];
+// The alignment of T*K assignments by one block of kAlignThreads threads;
+// `sm` is dynamic shared memory of align_smem_bytes(E) bytes.
+__device__ __forceinline__ void align_block(int T, int K, int E, int B, long long P_max, const int32_t* ids,
+                                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                            int32_t* __restrict__ sorted_ids, int32_t* __restrict__ block_expert,
+                                            int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
+                                            int32_t* __restrict__ stats_copy, int* sm) {
     int* cnt = sm;                 // E
     int* off = cnt + E;            // E + 1
     int* cursor = off + E + 1;     // E
@@ -182,8 +188,6 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     uint16_t* tbl = reinterpret_cast<uint16_t*>(bad + 1);  // 32 x E
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long A = (long long)T * K;
-    pdl_launch_dependents();
-    pdl_wait();
 
     for (int e = tid; e < E; e += kAlignThreads) cnt[e] = 0;
     if (tid == 0) *bad = 0;
@@ -276,10 +280,173 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     }
 }
 
+__global__ void __launch_bounds__(kAlignThreads, 1)
+    align_kernel(int T, int K, int E, int B, long long P_max, const int32_t* __restrict__ ids,
+                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
+                 int32_t* __restrict__ block_expert, int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
+                 int32_t* __restrict__ stats_copy) {
+    extern __shared__ int sm[];
+    pdl_launch_dependents();
+    pdl_wait();
+    align_block(T, K, E, B, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy, sm);
+}
+
+size_t align_smem_bytes(int E) { return sizeof(int) * (4 * (size_t)E + 1 + 34) + sizeof(uint16_t) * 32 * (size_t)E; }
+
+// ----------------------------------------------------- small-batch routing
+// Router logits, top-K gating and alignment in one launch for small T.
+// Stage 1 (every block): partial dot products of the router GEMV on the CUDA
+// cores -- one warp per (expert, group of 8 tokens, slice of the hidden
+// dimension), fp32 sums of the exact products -- written to `part`.
+// Stage 2 (the last block to finish, found with a counter; no block waits):
+// logits[t][e] = sum over slices in slice order (deterministic), then top-K
+// for every token and the alignment.  `logits_override` (nullable) replaces
+// the computed logits in the routing decision.
+constexpr int kRouteTokGroup = 8;
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
+    const int4 v = __ldg(reinterpret_cast<const int4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* p, float* f) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+    f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kAlignThreads, 1)
+    route_small_kernel(int T_, int H, int E, int K, int score_fn, int renorm, int B, long long P_max, int nslices,
+                       int slice_w, const T* __restrict__ x, const T* __restrict__ w_r,
+                       const float* __restrict__ logits_override, float* __restrict__ part, float* __restrict__ logits,
+                       int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ counts,
+                       int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
+                       int32_t* __restrict__ block_expert, int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
+                       int32_t* __restrict__ stats_copy, int* __restrict__ done_ctr) {
+    extern __shared__ int sm[];
+    __shared__ int is_last;
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ngroups = (T_ + kRouteTokGroup - 1) / kRouteTokGroup;
+    const long long units = (long long)E * ngroups * nslices;
+    const long long u = (long long)blockIdx.x * (kAlignThreads / 32) + warp;
+    if (u < units) {
+        const int e = (int)(u % E);
+        const int tg = (int)((u / E) % ngroups);
+        const int sl = (int)(u / ((long long)E * ngroups));
+        const int t0 = tg * kRouteTokGroup;
+        const int nt = T_ - t0 < kRouteTokGroup ? T_ - t0 : kRouteTokGroup;
+        const int h0 = sl * slice_w;
+        const int h1 = h0 + slice_w < H ? h0 + slice_w : H;
+        float acc[kRouteTokGroup];
+#pragma unroll
+        for (int i = 0; i < kRouteTokGroup; ++i) acc[i] = 0.f;
+        const T* wrow = w_r + (size_t)e * H;
+        for (int h = h0 + lane * 8; h < h1; h += 256) {
+            float wv[8];
+            load8(wrow + h, wv);
+#pragma unroll
+            for (int i = 0; i < kRouteTokGroup; ++i) {
+                if (i < nt) {
+                    float xv[8];
+                    load8(x + (size_t)(t0 + i) * H + h, xv);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i] = fmaf(wv[j], xv[j], acc[i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kRouteTokGroup; ++i) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+        }
+        if (lane == 0)
+            for (int i = 0; i < nt; ++i) part[((size_t)sl * T_ + t0 + i) * E + e] = acc[i];
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(done_ctr, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (long long i = threadIdx.x; i < (long long)T_ * E; i += kAlignThreads) {
+        float v = 0.f;
+        for (int sl = 0; sl < nslices; ++sl) v += __ldcg(part + (size_t)sl * T_ * E + i);
+        logits[i] = v;
+    }
+    __syncthreads();
+    const float* src = logits_override ? logits_override : logits;
+    for (int t = warp; t < T_; t += kAlignThreads / 32)
+        topk_one_token(src + (size_t)t * E, E, K, score_fn, renorm, ids + (size_t)t * K, w + (size_t)t * K, lane);
+    __syncthreads();
+    align_block(T_, K, E, B, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy, sm);
+    if (threadIdx.x == 0) *done_ctr = 0;  // ready for the next launch
+}
+
+// Slices of the hidden dimension (multiples of 256 elements) so that the
+// router GEMV covers about one wave of warps on the device.
+void route_small_slices(int T, int H, int E, int num_sms, int* nslices, int* slice_w) {
+    const long long pairs = (long long)E * ((T + kRouteTokGroup - 1) / kRouteTokGroup);
+    const long long target = (long long)num_sms * (kAlignThreads / 32);
+    const int max_sl = (H + 255) / 256;
+    long long ns = (target + pairs - 1) / pairs;
+    if (ns > max_sl) ns = max_sl;
+    if (ns < 1) ns = 1;
+    const int w = (int)(((H + ns - 1) / ns + 255) / 256 * 256);
+    *slice_w = w;
+    *nslices = (H + w - 1) / w;
+}
+
+int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, long long P_max, int dtype,
+                       const void* x, const void* w_r, const float* logits_override, float* part, float* logits,
+                       int32_t* ids, float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                       int32_t* block_expert, int32_t* pos, int32_t* scalars, int32_t* stats_copy, int* done_ctr,
+                       cudaStream_t stream) {
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    const size_t smem = align_smem_bytes(E);
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(route_small_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(route_small_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return -3;
+        }
+        attr_done = true;
+    }
+    int ns, sw;
+    route_small_slices(T, H, E, d.num_sms, &ns, &sw);
+    const long long units = (long long)E * ((T + kRouteTokGroup - 1) / kRouteTokGroup) * ns;
+    const int blocks = (int)((units + kAlignThreads / 32 - 1) / (kAlignThreads / 32));
+    cudaError_t e;
+    if (dtype == 0)
+        e = launch_kernel(route_small_kernel<__nv_bfloat16>, dim3(blocks), dim3(kAlignThreads), smem, stream, T, H, E,
+                          K, score_fn, renorm, B, P_max, ns, sw, static_cast<const __nv_bfloat16*>(x),
+                          static_cast<const __nv_bfloat16*>(w_r), logits_override, part, logits, ids, w, counts,
+                          offsets, sorted_ids, block_expert, pos, scalars, stats_copy, done_ctr);
+    else
+        e = launch_kernel(route_small_kernel<float>, dim3(blocks), dim3(kAlignThreads), smem, stream, T, H, E, K,
+                          score_fn, renorm, B, P_max, ns, sw, static_cast<const float*>(x),
+                          static_cast<const float*>(w_r), logits_override, part, logits, ids, w, counts, offsets,
+                          sorted_ids, block_expert, pos, scalars, stats_copy, done_ctr);
+    count_launch();
+    return launched(e);
+}
+
 int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids, int32_t* counts,
                  int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
                  int32_t* stats_copy, cudaStream_t stream) {
-    const size_t smem = sizeof(int) * (4 * (size_t)E + 1 + 34) + sizeof(uint16_t) * 32 * (size_t)E;
+    const size_t smem = align_smem_bytes(E);
     static bool attr_done = false;
     if (!attr_done) {
         if (cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=

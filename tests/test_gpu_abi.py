@@ -63,9 +63,24 @@ def test_launch_count_of_a_forward():
     before = moe.kernel_launch_count()
     moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws)
     moe.check_status(ws)
-    # router, top-K, align, permute, expert FFN (one fused launch at this size), combine
+    # decode size: routing (router + top-K + alignment), permute, expert FFN, combine
     assert moe.ffn_fused(cfg)
-    assert moe.kernel_launch_count() - before == 6
+    assert moe.kernel_launch_count() - before == 4
+
+
+def test_launch_count_of_a_prefill_forward():
+    shape = small_shape(H=256, E=8, K=2, I=512)
+    T = 1500
+    w = mi.make_weights(shape, 2, device="cuda")
+    x = mi.make_x(shape, T, 2, device="cuda")
+    cfg = cfg_for(shape, T)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    before = moe.kernel_launch_count()
+    moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws)
+    moe.check_status(ws)
+    # router GEMM, top-K, align, permute, gate/up, down, combine
+    assert not moe.ffn_fused(cfg)
+    assert moe.kernel_launch_count() - before == 7
 
 
 def test_wait_timeout_is_reported_and_recoverable():
