@@ -353,6 +353,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch each step from the host instead of a CUDA graph")
     ap.add_argument("--token-tile-cap", type=int, default=0, help="grouped GEMM token-tile cap (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream order between kernels")
+    ap.add_argument("--shared-sms", type=int, default=0,
+                    help="SMs for the shared experts beside the routed ones (0 = cost model, -1 = serial)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -378,6 +380,8 @@ def main():
         moe.set_token_tile_cap(args.token_tile_cap)
     if args.no_pdl:
         moe.set_programmatic_launch(False)
+    if args.shared_sms:
+        moe.set_shared_sms(args.shared_sms)
     wl = Workload(shape, T, rank, device, skew=args.skew)
     flush = l2_flush_buffer(device)
     if args.no_graph:
@@ -429,7 +433,8 @@ def main():
                               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
                               "quick": True, "config": {"workload": f"{shape.name}:{T}",
                                                         "token_tile_cap": args.token_tile_cap,
-                                                        "pdl": not args.no_pdl},
+                                                        "pdl": not args.no_pdl,
+                                                        "shared_sms": moe.shared_sms(wl.cfg)},
                               "stages_ms": stages, "E_active": E_active, "P": P}), flush=True)
         if dist:
             dist.barrier()
@@ -522,7 +527,8 @@ def main():
                    "score_fn": "softmax" if shape.score_fn == 0 else "sigmoid", "global_batch": T * world,
                    "parallelism": f"replicas x{world} (data parallel, no collective)",
                    "launch": "host launches" if args.no_graph else "CUDA graph replay of moe_layer_forward",
-                   "l2": "flushed between steps (2 GiB write outside the events); weights exceed L2"},
+                   "l2": "flushed between steps (2 GiB write outside the events); weights exceed L2",
+                   "shared_sms": moe.shared_sms(wl.cfg)},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - T * shape.K) / max(P, 1), 4),
                   "bytes_alg": B_alg, "flops_alg": F_alg, "roofline_frac": round(layer_roof, 4),
@@ -580,7 +586,8 @@ def run_sweep(args, device, flush, pk):
                    "tensor_frac": round(F / (t * 1e-3) / (pk["bf16_tflops"] * 1e12), 4),
                    "roofline_frac": round(max(F / (pk["bf16_tflops"] * 1e12), B / (pk["hbm_gbs"] * 1e9)) /
                                           (t * 1e-3), 4),
-                   "tau_FA": round(t / fa_cache[T], 4), "fused_ffn": bool(wl.fused)}
+                   "tau_FA": round(t / fa_cache[T], 4), "fused_ffn": bool(wl.fused),
+                   "shared_sms": moe.shared_sms(wl.cfg)}
             rows.append(row)
             if args.sweep_out:
                 with open(args.sweep_out, "a") as f:

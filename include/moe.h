@@ -195,7 +195,10 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* pos,
  * n_shared > 0), combine.  out[T,H].  logits_override (nullable, fp32 [T,E])
  * replaces the router output for the routing decision; the router GEMM still
  * runs so its cost is kept.  stats_out (nullable, device int32[4]) receives
- * {P, E_active, bad_ids, 0}.  Nothing is synchronised. */
+ * {P, E_active, bad_ids, 0}.  Nothing is synchronised.  The shared FFN runs
+ * concurrently on a library stream forked from and joined back into `stream`
+ * (see moe_set_shared_sms); the call is capturable into a CUDA graph, and
+ * concurrent calls on one device are serialised while they enqueue. */
 int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router,
                       const void* w13, const void* w2, const void* w13_shared,
                       const void* w2_shared, const float* logits_override, void* out,
@@ -212,7 +215,8 @@ int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13,
               const void* w2, void* out, void* workspace, size_t ws_bytes,
               moe_stream_t stream);
 
-/* Synchronise `stream`, then read and clear the workspace status word.
+/* Synchronise `stream`, then read and clear the workspace status words
+ * (the caller's-stream kernels' and the concurrent shared FFN's).
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a device wait ran out; the control words
  * are re-zeroed so the workspace stays usable) or MOE_ERR_CUDA. */
 int moe_check_status(void* workspace, moe_stream_t stream);
@@ -245,6 +249,22 @@ void moe_set_programmatic_launch(int enable);
  * with 256 weight rows per pair).  0 keeps single-SM tiles.  Process-wide;
  * results are identical up to fp32 summation order. */
 void moe_set_cta_pairs(int enable);
+
+/* Shared experts beside the routed experts.  With n_shared > 0,
+ * moe_layer_forward launches the shared FFN first, on a second stream that
+ * the library owns (one per device, created on first use), forked from and
+ * joined back into the caller's stream with events; it runs concurrently with
+ * routing and the routed experts on its own share of the SMs.  n = 0
+ * (default): the share comes from a bytes/flops cost model; n > 0: n SMs
+ * (rounded down to even, clamped to [2, SMs - 2]); n = -1: no side stream,
+ * the shared FFN runs after the routed experts on the caller's stream.
+ * Process-wide.  Results agree up to fp32 summation order (the grid size
+ * sets the K-splits).  Returns MOE_ERR_ARG for n < -1. */
+int moe_set_shared_sms(int n);
+
+/* SMs the shared experts of this configuration get under the current
+ * setting (0: they run serially, or there are none). */
+int moe_shared_sms(const moe_config_t* cfg);
 
 /* Test hook: when nonzero, the next GEMM or fused-FFN launch withholds one
  * operand load (the first load of block 0, or of work item 0 in the fused

@@ -77,6 +77,8 @@ def lib():
             "moe_set_token_tile_cap": (I, [I]),
             "moe_set_programmatic_launch": (None, [I]),
             "moe_set_cta_pairs": (None, [I]),
+            "moe_set_shared_sms": (I, [I]),
+            "moe_shared_sms": (I, [C]),
             "moe_ffn_fused": (I, [C]),
             "moe_layer_logits_offset": (ctypes.c_int64, [C]),
             "moe_kernel_launch_count": (ctypes.c_uint64, []),
@@ -297,6 +299,17 @@ def ffn_fused(cfg):
 def set_cta_pairs(enable=True):
     """2-SM (CTA pair) GEMM tiles for bf16 at the 256-token cap (default on)."""
     lib().moe_set_cta_pairs(1 if enable else 0)
+
+
+def set_shared_sms(n=0):
+    """SMs for the shared experts running beside the routed ones: 0 = cost
+    model (default), n > 0 = fixed share, -1 = run them after, serially."""
+    _check(lib().moe_set_shared_sms(int(n)), "moe_set_shared_sms")
+
+
+def shared_sms(cfg):
+    """SMs the shared experts of `cfg` get (0 = serial or none)."""
+    return int(lib().moe_shared_sms(ctypes.byref(cfg)))
 
 
 def debug_withhold_first_load(enable=True):

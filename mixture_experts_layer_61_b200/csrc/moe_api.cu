@@ -3,6 +3,7 @@
 // the MoE layer forward.  Every compute step runs in the kernels of
 // moe_kernels.cu and moe_gemm.cu; nothing here touches tensor data.
 #include <atomic>
+#include <cmath>
 #include <mutex>
 
 #include "../../include/moe.h"
@@ -93,8 +94,8 @@ long long p_max(const moe_config_t* c) {
 }
 
 struct Layout {
-    size_t ctl, logits, route_part, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm, act, act_sh,
-        sh_out;
+    size_t ctl, ctl_sh, logits, route_part, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm,
+        act, act_sh, sh_out;
     size_t total;
 };
 
@@ -111,6 +112,8 @@ Layout layout(const moe_config_t* c, int num_sms) {
         return r;
     };
     L.ctl = take(ctl_block_bytes(num_sms));
+    // the shared experts' own control block: they run beside the routed experts
+    L.ctl_sh = take(I_sh > 0 ? ctl_block_bytes(num_sms) : 0);
     L.logits = take(sizeof(float) * (size_t)c->T * c->E);
     // partial router sums of the small-batch routing kernel (slices of 256 hidden elements)
     L.route_part = take(c->T <= kSmallRouteMaxT ? sizeof(float) * ((size_t)c->H / 256 + 1) * c->T * c->E : 0);
@@ -184,11 +187,13 @@ GemmLaunch down_launch(const void* act, long long x_rows, const int32_t* seg_off
 }
 
 // gate/up (SwiGLU) + down over `n_groups` segments of X: one fused launch at
-// decode sizes (token-tile cap 32 or 64), else two GEMM launches.
-// `max_chunks` bounds the number of token chunks the segments can form.
+// decode sizes (token-tile cap 32, 64 or 128), else two GEMM launches.
+// `max_chunks` bounds the number of token chunks the segments can form;
+// `sms` / `ffn_sms` cap the persistent grid of the GEMMs / of the fused
+// kernel (0 = one block per SM).
 int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows, int H, int I,
             int dtype, const void* w13, const void* w2, void* act, void* y, int max_n, const GemmCtl& ctl,
-            cudaStream_t s, long long max_chunks) {
+            cudaStream_t s, long long max_chunks, int sms = 0, int ffn_sms = 0) {
     if (max_n <= 128) {
         FfnLaunch f;
         f.x = x;
@@ -205,13 +210,81 @@ int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_g
         f.dtype = dtype;
         f.max_n = max_n;
         f.max_chunks = max_chunks;
+        f.sms = ffn_sms;
         int rc = launch_ffn_stream(f, ctl, s);
         if (rc != 1) return rc;  // 1: not handled, use two launches
     }
-    int rc = launch_gemm(gate_up_launch(x, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w13, act, max_n),
-                         ctl, s);
+    GemmLaunch g = gate_up_launch(x, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w13, act, max_n);
+    g.sms = sms;
+    int rc = launch_gemm(g, ctl, s);
     if (rc != 0) return rc;
-    return launch_gemm(down_launch(act, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w2, y, max_n), ctl, s);
+    g = down_launch(act, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w2, y, max_n);
+    g.sms = sms;
+    return launch_gemm(g, ctl, s);
+}
+
+// ------------------------------------------ shared experts beside the routed ones
+// The shared experts read only x, so they run from the start of the layer on a
+// second stream, concurrently with routing and the routed experts, on their
+// own share of the SMs and with their own control block; the combine waits
+// for both.  One side stream and a fork/join event pair per device, created on
+// first use; the mutex keeps the record/wait pairs of concurrent callers apart.
+struct SideStream {
+    std::mutex mu;
+    int state = 0;  // 0 not yet created, 1 ready, -1 creation failed (run serially)
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream g_side[kMaxDevices];
+std::atomic<int> g_shared_sms{0};  // 0 automatic, -1 serial, n > 0 fixed share
+
+// Called with side.mu held.
+bool side_ready(SideStream& side) {
+    if (side.state == 0) {
+        side.state = -1;
+        if (cudaStreamCreateWithFlags(&side.s, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&side.fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&side.join, cudaEventDisableTiming) == cudaSuccess)
+            side.state = 1;
+        else
+            cudaGetLastError();
+    }
+    return side.state == 1;
+}
+
+// SMs given to the shared experts (even, for CTA pairs), or 0 to run them after
+// the routed experts on the caller's stream.  Calibrated on B200 with the
+// Qwen2-MoE- and DeepSeek-V3-shaped layers (a sweep of the share per T):
+//  * T <= 128 (the shared FFN is one fused launch): the shared experts start
+//    with a large share while routing runs, and the routed FFN's blocks take
+//    over their SMs as they exit: 0.35 N + 0.4 N f, at most 0.55 N, where f is
+//    the shared experts' fraction of the weight bytes.
+//  * larger T (the shared FFN is a GEMM pair, near per-SM tensor peak on a
+//    few SMs, beside the routed stream at HBM speed): 12 + rho / 2 SMs, at most
+//    40, with rho = shared flops / routed weight bytes; serially once the
+//    routed experts reach 128 rows each, where they need every SM.
+int shared_sms(const moe_config_t* c, int num_sms) {
+    const int forced = g_shared_sms.load(std::memory_order_relaxed);
+    if (forced < 0 || num_sms < 8) return 0;
+    if (forced > 0) {
+        const int n = forced & ~1;
+        return n < 2 ? 2 : (n > num_sms - 2 ? num_sms - 2 : n);
+    }
+    const double eb = elt_bytes(c->dtype), T = c->T, H = c->H, I = c->I, E = c->E, K = c->K;
+    const double I_sh = (double)c->n_shared * c->I_shared;
+    const double e_act = E * (1.0 - std::pow(1.0 - K / E, T));
+    const double B_r = e_act * 3.0 * H * I * eb, B_s = 3.0 * H * I_sh * eb;
+    double n;
+    if (pick_max_n(T) <= 128) {
+        const double f = B_s / (B_s + B_r);
+        n = num_sms * std::fmin(0.55, 0.35 + 0.4 * f);
+    } else {
+        if (T * K / E >= 128.0) return 0;
+        const double rho = 6.0 * T * H * I_sh / B_r;
+        n = std::fmin(40.0, 12.0 + 0.5 * rho);
+    }
+    int ni = 2 * (int)std::lround(n / 2.0);
+    return ni < 2 ? 2 : (ni > num_sms - 2 ? num_sms - 2 : ni);
 }
 
 // The router's output has only E features, so its tiles are few: cut the
@@ -433,6 +506,57 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
     void* y_perm = x_perm;
     const long long P = p_max(cfg);
 
+    // shared experts first, on the side stream, when they run beside the routed ones
+    SideStream* side = nullptr;
+    std::unique_lock<std::mutex> side_lock;
+    const void* sh = nullptr;
+    int n_sh = 0;
+    if (I_sh > 0) {
+        SideStream& sd = g_side[d.device];
+        side_lock = std::unique_lock<std::mutex>(sd.mu);
+        n_sh = shared_sms(cfg, d.num_sms);
+        if (n_sh > 0 && side_ready(sd)) {
+            if (cudaEventRecord(sd.fork, s) != cudaSuccess || cudaStreamWaitEvent(sd.s, sd.fork, 0) != cudaSuccess) {
+                cudaGetLastError();
+                return MOE_ERR_CUDA;
+            }
+            GemmCtl ctl_sh = gemm_ctl(at<uint8_t>(workspace, L.ctl_sh), d.num_sms);
+            ctl_sh.status = ctl.status + 1;  // the header's second status word
+            void* sh_out = at<void>(workspace, L.sh_out);
+            rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
+                         at<void>(workspace, L.act_sh), sh_out, pick_max_n(cfg->T), ctl_sh, sd.s,
+                         dense_max_chunks(cfg->T), n_sh, n_sh);
+            if (cudaEventRecord(sd.join, sd.s) != cudaSuccess) {
+                cudaGetLastError();
+                return MOE_ERR_CUDA;
+            }
+            side = &sd;
+            if (rc != 0) {
+                cudaStreamWaitEvent(s, sd.join, 0);
+                return status_of(rc);
+            }
+            sh = sh_out;
+        } else {
+            side_lock.unlock();
+        }
+    }
+    // Every return from here on makes the caller's stream wait for the side
+    // stream first, so that a capturing caller stream stays joined.
+    struct JoinOnExit {
+        SideStream* side;
+        cudaStream_t s;
+        ~JoinOnExit() {
+            if (side && cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) cudaGetLastError();
+        }
+    };
+    JoinOnExit join_guard{side, s};
+    // The router and routed GEMMs take the SMs the shared experts leave.  The
+    // routed fused FFN fetches its work dynamically: beside a fused (one-launch)
+    // shared FFN it launches a block per SM, and those that find no free SM
+    // start when the shared experts' blocks exit; beside the shared GEMM pair it
+    // keeps to its share, so that the shared down GEMM finds its SMs free.
+    const int n_routed = side ? d.num_sms - n_sh : 0;
+    const int n_routed_ffn = side && pick_max_n(cfg->T) > 128 ? n_routed : 0;
     if (cfg->T <= kSmallRouteMaxT && cfg->H % 8 == 0) {
         // router logits, top-K and alignment in one launch (decode-sized batches)
         int* route_ctr = reinterpret_cast<int*>(at<uint8_t>(workspace, L.ctl)) + 16;  // in the control header
@@ -456,6 +580,7 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
         g.out_ld = cfg->E;
         g.dtype = cfg->dtype;
         router_tiling(g, cfg->T);
+        g.sms = n_routed;
         if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
         if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm,
                               logits_override ? logits_override : logits, ids, w, s)) != 0)
@@ -467,16 +592,22 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
     if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s)) != 0)
         return status_of(rc);
     if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
-                      routed_max_n(cfg), ctl, s, routed_max_chunks(cfg))) != 0)
+                      routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn)) != 0)
         return status_of(rc);
-    const void* sh = nullptr;
-    if (I_sh > 0) {
-        void* act_sh = at<void>(workspace, L.act_sh);
+    if (I_sh > 0 && !side) {
         void* sh_out = at<void>(workspace, L.sh_out);
-        if ((rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared, act_sh,
-                          sh_out, pick_max_n(cfg->T), ctl, s, dense_max_chunks(cfg->T))) != 0)
+        if ((rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
+                          at<void>(workspace, L.act_sh), sh_out, pick_max_n(cfg->T), ctl, s,
+                          dense_max_chunks(cfg->T))) != 0)
             return status_of(rc);
         sh = sh_out;
+    }
+    if (side) {
+        join_guard.side = nullptr;
+        if (cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
     }
     return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, w, sh, out, s));
 }
@@ -509,20 +640,27 @@ int moe_check_status(void* workspace, moe_stream_t stream) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    unsigned st = 0;
-    if (cudaMemcpy(&st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    // word 0: every kernel on the caller's stream; word 1: the shared experts'
+    // kernels of moe_layer_forward, whose control block follows the first
+    unsigned st[2] = {0, 0};
+    if (cudaMemcpy(st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    if (st & kStatusTimeout) {
-        // re-zero the control words: status and stream-K counters, and the fused FFN's counters
-        const GemmCtl c = gemm_ctl(workspace, d.num_sms);
-        if (cudaMemset(workspace, 0, gemm_ctl_zero_bytes(d.num_sms)) != cudaSuccess ||
-            cudaMemset(c.ffn_ctl, 0, ctl_block_bytes(d.num_sms) - ((uint8_t*)c.ffn_ctl - (uint8_t*)workspace)) !=
-                cudaSuccess) {
-            cudaGetLastError();
+    auto rezero = [&](void* block) {
+        // status and stream-K counters, and the fused FFN's counters
+        const GemmCtl c = gemm_ctl(block, d.num_sms);
+        const bool ok =
+            cudaMemset(block, 0, gemm_ctl_zero_bytes(d.num_sms)) == cudaSuccess &&
+            cudaMemset(c.ffn_ctl, 0, ctl_block_bytes(d.num_sms) - ((uint8_t*)c.ffn_ctl - (uint8_t*)block)) ==
+                cudaSuccess;
+        if (!ok) cudaGetLastError();
+        return ok;
+    };
+    if ((st[0] | st[1]) & kStatusTimeout) {
+        if (!rezero(workspace)) return MOE_ERR_CUDA;
+        if ((st[1] & kStatusTimeout) && !rezero(static_cast<uint8_t*>(workspace) + align256(ctl_block_bytes(d.num_sms))))
             return MOE_ERR_CUDA;
-        }
         return MOE_ERR_TIMEOUT;
     }
     return MOE_OK;
@@ -537,6 +675,19 @@ int moe_set_token_tile_cap(int n) {
 }
 
 void moe_set_programmatic_launch(int enable) { set_pdl(enable != 0); }
+
+int moe_set_shared_sms(int n) {
+    if (n < -1) return MOE_ERR_ARG;
+    g_shared_sms.store(n);
+    return MOE_OK;
+}
+
+int moe_shared_sms(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK || (long long)cfg->n_shared * cfg->I_shared == 0) return 0;
+    DeviceInfo d;
+    if (current_device(&d) != 0) return 0;
+    return shared_sms(cfg, d.num_sms);
+}
 
 int moe_ffn_fused(const moe_config_t* cfg) {
     if (check_cfg(cfg) != MOE_OK) return 0;

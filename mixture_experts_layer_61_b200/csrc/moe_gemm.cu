@@ -102,7 +102,9 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
     p.withhold_first_load = take_withhold_flag();
     p.sk_min_units = 4;
     p.max_split = L.max_split > 0 ? L.max_split : 4;
-    cudaError_t e = launch_kernel_cluster(kern, dim3(grid_blocks), dim3(kGemmThreads), C::kSmemBytes, stream, kCta,
+    int grid = grid_blocks;
+    if (L.sms > 0 && L.sms < grid) grid = L.sms >= 2 * kCta ? L.sms - L.sms % kCta : kCta;
+    cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(kGemmThreads), C::kSmemBytes, stream, kCta,
                                           tm_w, tm_x, tm_x64, tm_xbig, p);
     count_launch();
     if (e != cudaSuccess) cudaGetLastError();
@@ -206,7 +208,8 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     p.wait_limit_ns = wait_limit_ns();
     p.withhold_first_load = take_withhold_flag();
     p.max_slots_phase = slots_total / 2;
-    cudaError_t e = launch_kernel(kern, dim3(num_sms), dim3(kGemmThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
+    const int grid = L.sms > 0 && L.sms < num_sms ? L.sms : num_sms;
+    cudaError_t e = launch_kernel(kern, dim3(grid), dim3(kGemmThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
                                   xb, xb64, p);
     count_launch();
     if (e != cudaSuccess) cudaGetLastError();
@@ -224,8 +227,8 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
     // split-tile counters: each phase's tiles must fit half the counter array when split
     const long long ntiles_a = L.max_chunks * ((L.I + 127) / 128);
     const long long ntiles_b = L.max_chunks * ((L.H + 255) / 256);
-    if ((ntiles_a < 2LL * d.num_sms && ntiles_a > kFfnTileCtrs / 2) ||
-        (ntiles_b < 2LL * d.num_sms && ntiles_b > kFfnTileCtrs / 2))
+    const long long G = L.sms > 0 && L.sms < d.num_sms ? L.sms : d.num_sms;
+    if ((ntiles_a < 2LL * G && ntiles_a > kFfnTileCtrs / 2) || (ntiles_b < 2LL * G && ntiles_b > kFfnTileCtrs / 2))
         return 1;
     if (L.x_rows <= 0) return 0;
     if (L.dtype == 0) {

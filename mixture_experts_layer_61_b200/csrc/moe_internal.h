@@ -100,6 +100,7 @@ struct GemmLaunch {
     int dtype;                   // 0 bf16, 1 fp32
     int max_n;                   // token-tile cap: 32, 64, 128 or 256
     int max_split;               // stream-K: most blocks per tile (0 = default 4)
+    int sms;                     // persistent blocks at most (0 = one per SM): an SM share
 };
 
 int launch_gemm(const GemmLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
@@ -122,6 +123,7 @@ struct FfnLaunch {
     int dtype;
     int max_n;
     long long max_chunks;  // upper bound on token chunks (host side)
+    int sms;               // persistent blocks at most (0 = one per SM)
 };
 int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 

@@ -101,3 +101,35 @@ def test_wait_timeout_is_reported_and_recoverable():
     out = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws)
     moe.check_status(ws)
     assert torch.equal(out, ref)
+
+
+def test_wait_timeout_in_shared_experts_is_reported_and_recoverable():
+    # the withheld load lands in the shared FFN, launched first on the side
+    # stream: its status word (the header's second) reports the timeout and
+    # its own control block is re-zeroed
+    shape = small_shape(H=256, E=8, K=2, I=512, I_sh=768)
+    T = 40
+    w = mi.make_weights(shape, 3, device="cuda")
+    x = mi.make_x(shape, T, 3, device="cuda")
+    cfg = cfg_for(shape, T)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    fwd = lambda: moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w["w13_sh"], w["w2_sh"])
+    moe.set_shared_sms(16)
+    try:
+        ref = fwd().clone()
+        moe.check_status(ws)
+        moe.set_wait_limit_ns(20_000_000)  # 20 ms
+        try:
+            moe.debug_withhold_first_load(True)
+            fwd()
+            with pytest.raises(moe.MoeError) as e:
+                moe.check_status(ws)
+            assert e.value.code == -4
+        finally:
+            moe.debug_withhold_first_load(False)
+            moe.set_wait_limit_ns(0)
+        out = fwd()
+        moe.check_status(ws)
+        assert torch.equal(out, ref)
+    finally:
+        moe.set_shared_sms(0)

@@ -92,3 +92,47 @@ def test_layer_deepseek_skew_sweep_point(s):
     T = 256
     lg = mi.zipf_gumbel_logits(shape.E, T, s, seed=4000 + T, device="cuda")
     assert _run_layer(shape, T, seed=mi.seed_for(shape, T, 5), override=lg, n_sample=64) < OUT_TOL
+
+
+@pytest.mark.parametrize("T", [5, 100, 700])
+@pytest.mark.parametrize("n_sh", [-1, 16, 0])
+def test_layer_shared_experts_beside_routed(T, n_sh):
+    # the shared FFN on the library's side stream with a fixed SM share (16),
+    # with the cost model's share (0), and serially after the routed experts
+    # (-1); T = 5 / 100 run fused FFN kernels, T = 700 the CTA-pair GEMMs
+    shape = small_shape(H=512, E=16, K=4, I=384, I_sh=1024)
+    moe.set_shared_sms(n_sh)
+    try:
+        cfg = cfg_for(shape, T)
+        if n_sh < 0:
+            assert moe.shared_sms(cfg) == 0
+        elif n_sh > 0:
+            assert moe.shared_sms(cfg) == n_sh
+        assert _run_layer(shape, T, seed=T + 7) < OUT_TOL
+    finally:
+        moe.set_shared_sms(0)
+
+
+@pytest.mark.parametrize("T", [24, 400])
+def test_layer_side_stream_captured_in_cuda_graph(T):
+    # the fork/join of the shared experts' stream inside a CUDA graph capture
+    # (T = 24: fused shared and routed FFNs; T = 400: the shared GEMM pair
+    # beside the routed fused FFN): replays equal an eager call bit for bit
+    shape = small_shape(H=512, E=16, K=4, I=384, I_sh=1024)
+    w = mi.make_weights(shape, T, device="cuda")
+    x = mi.make_x(shape, T, T, device="cuda")
+    cfg = cfg_for(shape, T)
+    assert moe.shared_sms(cfg) > 0
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    args = (cfg, x, w["w_r"], w["w13"], w["w2"], ws, w["w13_sh"], w["w2_sh"])
+    ref = moe.layer_forward(*args).clone()
+    moe.check_status(ws)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        out = moe.layer_forward(*args)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    moe.check_status(ws)
+    assert torch.equal(out, ref)
+    del g
