@@ -43,7 +43,7 @@ METRIC = "MoE layer tokens/s; % HBM BW (decode) / % tensor peak (prefill); tau v
 # current kernels (dram__bytes_read.sum + dram__bytes_write.sum); workloads
 # without a capture report None.  Summaries of the captures are in profiles/.
 NCU_TRAFFIC = {
-    "mixtral:2048": 2.181456e9 + 0.167618e9,   # moe_gemm_kernel gate/up + SwiGLU, CTA pairs
+    "mixtral:2048": 2.290887e9 + 0.177937e9,   # moe_gemm_kernel gate/up + SwiGLU, CTA pairs
     "mixtral:32": 2.824073e9 + 0.008427e9,     # moe_ffn_stream_kernel, fused decode FFN
 }
 

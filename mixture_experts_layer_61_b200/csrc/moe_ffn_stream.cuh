@@ -102,7 +102,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 
 template <typename T, int kMaxN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kFfnThreads, 1)
     moe_ffn_stream_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_constant__ CUtensorMap tm_w2,
                           const __grid_constant__ CUtensorMap tm_xa, const __grid_constant__ CUtensorMap tm_xa64,
                           const __grid_constant__ CUtensorMap tm_xb, const __grid_constant__ CUtensorMap tm_xb64,

@@ -29,18 +29,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, kdim] row-major, box = box_rows x (128 bytes), 128-byte swizzle,
-// out-of-range elements read as zero.
+// [rows, kdim] row-major, box = box_rows x row_bytes (128 or 64) with the
+// swizzle of that width, out-of-range elements read as zero.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void* base, long long rows, int kdim,
-              int box_rows) {
+              int box_rows, int row_bytes = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(kdim), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(kdim) * elt_bytes};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt_bytes), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes / elt_bytes), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -81,10 +82,11 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
         attr_done = true;
     }
     CUtensorMap tm_w, tm_x, tm_x64, tm_xbig;
-    if (!make_map(&tm_w, Elt<T>::kTma, Elt<T>::kBytes, L.w, L.w_rows, L.kdim, 128)) return -3;
-    if (!make_map(&tm_x, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxRows)) return -3;
-    if (!make_map(&tm_x64, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxMid)) return -3;
-    if (!make_map(&tm_xbig, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, kMaxN / kCta)) return -3;
+    constexpr int rb = C::kRowBytes;
+    if (!make_map(&tm_w, Elt<T>::kTma, Elt<T>::kBytes, L.w, L.w_rows, L.kdim, 128, rb)) return -3;
+    if (!make_map(&tm_x, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxRows, rb)) return -3;
+    if (!make_map(&tm_x64, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, C::kXBoxMid, rb)) return -3;
+    if (!make_map(&tm_xbig, Elt<T>::kTma, Elt<T>::kBytes, L.x, L.x_rows, L.kdim, kMaxN / kCta, rb)) return -3;
     GemmParams p;
     p.seg_offsets = L.seg_offsets;
     p.n_groups = L.n_groups;
@@ -134,7 +136,8 @@ int dispatch_plain(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
 }
 
 // bf16 at the 256-token cap: CTA pairs (2-SM MMA, M = 256 weight rows per
-// pair, each CTA staging half of the 256 token rows).
+// pair, each CTA staging half of the 256 token rows); without SwiGLU a pair
+// takes 512 output features (wide) when there are that many.
 int dispatch_bf16(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t s) {
     using bf = __nv_bfloat16;
     if (g_cta_pairs && L.max_n == 256 && !L.out_f32 && (num_sms % 2) == 0) {
@@ -209,7 +212,7 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     p.withhold_first_load = take_withhold_flag();
     p.max_slots_phase = slots_total / 2;
     const int grid = L.sms > 0 && L.sms < num_sms ? L.sms : num_sms;
-    cudaError_t e = launch_kernel(kern, dim3(grid), dim3(kGemmThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
+    cudaError_t e = launch_kernel(kern, dim3(grid), dim3(kFfnThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
                                   xb, xb64, p);
     count_launch();
     if (e != cudaSuccess) cudaGetLastError();

@@ -21,8 +21,9 @@
 // reuse it from L2.  Each tile reduces over K = kdim in steps of 128 bytes.
 //
 // Schedule.  gridDim.x persistent blocks (one per SM).  Whole waves of tiles
-// are dealt round-robin; the remaining one to two waves are split evenly by
-// k-iterations across the blocks (stream-K), so every block streams the same
+// are dealt round-robin; the remaining one to two waves (all but the first
+// wave, with fewer than two) are split evenly by k-iterations across the
+// blocks (stream-K), so every block streams the same
 // number of weight bytes even when there are fewer tiles than SMs (decode).
 // A tile split across blocks is finished by the last block to arrive: each
 // contributor stores its fp32 partial tile, then increments the tile's
@@ -30,8 +31,11 @@
 // sums all partials in block order (deterministic) and runs the epilogue.
 // No block ever waits on another block.
 //
-// Roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// the MMAs, warps 2..5 run the epilogue (TMEM -> registers -> global).  All
+// Roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// the MMAs, warps 2..9 run the epilogue (TMEM -> registers -> global), two
+// warps per TMEM lane quadrant, each on half of the tile's token columns.
+// Where the packed results fit in registers, the epilogue reads the whole
+// accumulator, frees it for the next tile's MMAs and only then stores.  All
 // waits are bounded by a deadline; a wait that runs out sets the status word
 // and every role winds down (in-flight copies and MMAs are drained first).
 #pragma once
@@ -41,7 +45,9 @@
 namespace moe {
 
 constexpr int kMaxGroups = 1024;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmEpiWarps = 8;                      // two per TMEM lane quadrant
+constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;  // producer warp, MMA warp, epilogue
+constexpr int kFfnThreads = 192;
 
 // Partial-tile slot layout: column c of row r (r < 128) at float index
 // ((c / 4) * 128 + r) * 4 + c % 4, so that a warp moves 32 consecutive
@@ -74,30 +80,38 @@ constexpr int kEpiPlain = 0, kEpiSwiGLU = 1, kEpiWide = 2;
 
 template <typename T, int kEpi, int kMaxN, int kCta = 1>
 struct GemmCfg {
-    static constexpr int kBK = 128 / Elt<T>::kBytes;   // K elements per stage (one swizzle row)
-    static constexpr int kMmaK = 32 / Elt<T>::kBytes;  // K per MMA instruction
+    // Operand tiles are K-major rows of kRowBytes with the swizzle of that
+    // width.  128-byte rows: 64-byte rows (twice the stages in the same
+    // shared memory) measured slower on B200, the per-stage barrier and TMA
+    // overhead outweighing the deeper lookahead.
+    static constexpr int kRowBytes = 128;
+    static constexpr int kBK = kRowBytes / Elt<T>::kBytes;  // K elements per stage
+    static constexpr int kMmaK = 32 / Elt<T>::kBytes;       // K per MMA instruction
+    static constexpr int kKSteps = kBK / kMmaK;             // MMAs per operand pair and stage
     static constexpr int kNW = kEpi == kEpiPlain ? 1 : 2;  // weight tiles per stage
     static constexpr int kFeat = kEpi == kEpiWide ? 256 : 128;  // output features per CTA and tile
     static constexpr int kFeatTile = kFeat * kCta;                 // output features per tile
     static constexpr int kUnit = 16 * kCta;                        // token-row granularity of the MMA
-    static constexpr int kWTileBytes = 128 * 128;
+    static constexpr int kWTileBytes = 128 * kRowBytes;
     static constexpr int kXBoxRows = 16;       // token rows per TMA box: 16, 64 and kMaxN
     static constexpr int kXBoxMid = 64;
-    static constexpr int kXBoxBytes = kXBoxRows * 128;
-    static constexpr int kXTileBytes = (kMaxN / kCta) * 128;  // this CTA's share of the token tile
+    static constexpr int kXTileBytes = (kMaxN / kCta) * kRowBytes;  // this CTA's share of the token tile
     static constexpr int kStageBytes = kNW * kWTileBytes + kXTileBytes;
     static constexpr int kAccCols = kNW * kMaxN;
     static constexpr int kNumAcc = (512 / kAccCols) >= 2 ? 2 : 1;
     static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
     static constexpr int kMiscBytes = 512;
+    static constexpr int kMaxStages = 16;
     static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes;
     static constexpr int kStagesRaw = kBudget / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kStages = kStagesRaw > kMaxStages ? kMaxStages : kStagesRaw;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
     static_assert(kStages >= 2, "pipeline needs two stages");
     static_assert(kMaxN % kUnit == 0 && kMaxN >= kUnit && kMaxN <= 256, "MMA N range");
     static_assert(kCta == 1 || kCta == 2, "one CTA or a CTA pair");
     static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
+    static_assert(2 * kMaxStages * 8 + 2 * kNumAcc * 8 + 8 + 12 <= kMiscBytes, "barriers fit");
+    static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzle atoms");
 };
 
 // ------------------------------------------------------------- scheduling
@@ -135,7 +149,11 @@ __device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int to
     s.G = gridDim.x / ncta;
     s.cta = blockIdx.x / ncta;
     s.total_tiles = (long long)total_chunks * NF;
-    s.dp_waves = s.total_tiles >= 2LL * s.G ? s.total_tiles / s.G - 1 : 0;
+    // Whole waves first, keeping one to two waves for the stream-K tail; with
+    // fewer than two waves of tiles, one whole wave and the rest as stream-K,
+    // so that the token chunks sharing a weight block (adjacent tiles) stream
+    // it together at least in that wave.
+    s.dp_waves = s.total_tiles >= 2LL * s.G ? s.total_tiles / s.G - 1 : (s.total_tiles >= s.G ? 1 : 0);
     s.dp_tiles = s.dp_waves * s.G;
     s.sk_tiles = s.total_tiles - s.dp_tiles;
     s.U = s.sk_tiles * KI;
@@ -290,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < C::kNumAcc; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128 * kCta);
+            mbar_init(&tempty[b], 32 * kGemmEpiWarps * kCta);
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
@@ -358,7 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int xn = t.mma_n / kCta;
                 const int xrow = t.row0 + (int)rank * xn;
                 // bytes landing on the (leader's) full barrier per stage: both CTAs' shares
-                const uint32_t bytes = kCta * (C::kNW * C::kWTileBytes + xn * 128);
+                const uint32_t bytes = kCta * (C::kNW * C::kWTileBytes + xn * C::kRowBytes);
                 const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
@@ -387,8 +405,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         r = xn;
                     }
                     if (kMaxN / kCta >= C::kXBoxMid)
-                        for (; r + C::kXBoxMid <= xn; r += C::kXBoxMid) load(xs + r * 128, &tm_x64, xrow + r, pol_x);
-                    for (; r < xn; r += C::kXBoxRows) load(xs + r * 128, &tm_x, xrow + r, pol_x);
+                        for (; r + C::kXBoxMid <= xn; r += C::kXBoxMid)
+                            load(xs + r * C::kRowBytes, &tm_x64, xrow + r, pol_x);
+                    for (; r < xn; r += C::kXBoxRows) load(xs + r * C::kRowBytes, &tm_x, xrow + r, pol_x);
                     ++fills[s];
                 }
             }
@@ -429,11 +448,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     tc_fence_after();
                     uint8_t* st = stage_base + s * C::kStageBytes;
-                    const uint64_t a0 = umma_desc_sw128(smem_u32(st));
-                    const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
-                    const uint64_t bx = umma_desc_sw128(smem_u32(st + C::kNW * C::kWTileBytes));
+                    auto desc = [](uint32_t a) { return C::kRowBytes == 128 ? umma_desc_sw128(a) : umma_desc_sw64(a); };
+                    const uint64_t a0 = desc(smem_u32(st));
+                    const uint64_t a1 = desc(smem_u32(st + C::kWTileBytes));
+                    const uint64_t bx = desc(smem_u32(st + C::kNW * C::kWTileBytes));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
+                    for (int kk = 0; kk < C::kKSteps; ++kk) {
                         const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
                         if (kPair) {
                             umma_pair_bf16(d_gate, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
@@ -469,8 +489,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // -------------------------------------------------------- epilogue
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;  // TMEM lane = feature row within a 128-row block
+        const int quad = warp & 3;                // TMEM lane quadrant this warp may access
+        const int half = (warp - 2) >> 2;         // which share of the token columns
+        const int r = quad * 32 + lane;           // TMEM lane = feature row within a 128-row block
+        const int e = (warp - 2) * 32 + lane;     // epilogue thread 0 .. 255
+        constexpr int kEpiThreads = 32 * kGemmEpiWarps;
+        constexpr int kHalfN = kMaxN / (kGemmEpiWarps / 4);  // token columns per warp
+        constexpr int kCh = kHalfN >= 32 ? 32 : 16;
+        constexpr bool kBf16Out = sizeof(OutT) == 2;
+        constexpr int kRegs = kBf16Out ? kHalfN / 2 : kHalfN;  // packed results of one accumulator
+        constexpr bool kEarly = kEpi != kEpiWide && kRegs <= 64;
+        const int cbeg = half * kHalfN;
         OutT* out = reinterpret_cast<OutT*>(p.out);
         uint32_t ac = 0;
         Item it;
@@ -490,70 +519,159 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool v0 = f < p.n_out;
             const bool v1 = kEpi == kEpiWide ? (f + 128 < p.n_out) : (kSwiGLU && v0);
             OutT* orow = out + (long long)t.row0 * p.out_ld + f;
-            // g: first accumulator, u: second (up projection, or features f + 128)
-            auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {
-                if (kSwiGLU) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
-                }
-                if (v0) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * p.out_ld, g[i]);
-                }
-                if (kEpi == kEpiWide && v1) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < t.nrows) store_out<OutT>(orow + 128 + (long long)(c0 + i) * p.out_ld, u[i]);
-                }
-            };
-            if (!it.split) {
-                // 32 columns of both accumulators per round, one wait for both loads
-                for (int c0 = 0; c0 < t.nrows; c0 += 32) {
-                    uint32_t ga[32], ua[32];
+            const int cend = t.nrows < cbeg + kHalfN ? t.nrows : cbeg + kHalfN;  // this half's real columns
+            // kCh columns of the first (and second) accumulator from column c0, one wait
+            auto load_cols = [&](int c0, float (&g)[kCh], float (&u)[kCh]) {
+                uint32_t ga[kCh], ua[kCh];
+                if constexpr (kCh == 32) {
                     tmem_ld32_nowait(tacc + c0, ga);
                     if (kTwo) tmem_ld32_nowait(tacc + kMaxN + c0, ua);
+                } else {
+                    tmem_ld16_nowait(tacc + c0, ga);
+                    if (kTwo) tmem_ld16_nowait(tacc + kMaxN + c0, ua);
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < kCh; ++i) {
+                    g[i] = __uint_as_float(ga[i]);
+                    u[i] = kTwo ? __uint_as_float(ua[i]) : 0.f;
+                }
+            };
+            auto release = [&]() {
+                tc_fence_before();
+                if (kPair && rank != 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[b]), 0));
+                else mbar_arrive(&tempty[b]);
+            };
+            // g: first accumulator, u: second (up projection, or features f + 128)
+            const int nrows = t.nrows;
+            const long long out_ld = p.out_ld;
+            // (callers skip blocks that start past the last real column; whole
+            // blocks store without per-element predicates, which measured
+            // markedly faster than predicating every store)
+            auto emit = [orow, nrows, out_ld, v0, v1](int c0, float (&g)[16], float (&u)[16]) {
+                const int n = nrows - c0 < 16 ? nrows - c0 : 16;
+                if (n == 16) {
+                    if (v0) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) store_out<OutT>(orow + (c0 + i) * out_ld, g[i]);
+                    }
+                    if (kEpi == kEpiWide && v1) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) store_out<OutT>(orow + 128 + (c0 + i) * out_ld, u[i]);
+                    }
+                } else {
+                    if (v0) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (i < n) store_out<OutT>(orow + (c0 + i) * out_ld, g[i]);
+                    }
+                    if (kEpi == kEpiWide && v1) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (i < n) store_out<OutT>(orow + 128 + (c0 + i) * out_ld, u[i]);
+                    }
+                }
+            };
+            if (!it.split && kEarly) {
+                // whole half into registers (SwiGLU applied, packed), accumulator freed, then stores
+                uint32_t res[kRegs];
+#pragma unroll
+                for (int j = 0; j < kHalfN / kCh; ++j) {
+                    const int c0 = cbeg + j * kCh;
+                    if (c0 < cend) {
+                        float g[kCh], u[kCh];
+                        load_cols(c0, g, u);
+#pragma unroll
+                        for (int i = 0; i < kCh; ++i)
+                            if (kSwiGLU) g[i] = silu_mul(g[i], u[i]);
+                        if constexpr (kBf16Out) {
+#pragma unroll
+                            for (int i = 0; i < kCh; i += 2) {
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(g[i], g[i + 1]);
+                                res[(j * kCh + i) / 2] = *reinterpret_cast<uint32_t*>(&h2);
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < kCh; ++i) res[j * kCh + i] = __float_as_uint(g[i]);
+                        }
+                    }
+                }
+                release();
+                // column i of this warp's share from the packed registers
+                auto store_res = [&](int i) {
+                    OutT* dst = orow + (long long)(cbeg + i) * out_ld;
+                    if constexpr (kBf16Out) {
+                        const uint32_t w2 = res[i / 2];
+                        *reinterpret_cast<uint16_t*>(dst) = (i & 1) ? (uint16_t)(w2 >> 16) : (uint16_t)(w2 & 0xffffu);
+                    } else {
+                        *reinterpret_cast<float*>(dst) = __uint_as_float(res[i]);
+                    }
+                };
+                if (v0) {
+#pragma unroll
+                    for (int j = 0; j < kHalfN / 16; ++j) {
+                        const int c0 = cbeg + 16 * j;
+                        if (c0 + 16 <= cend) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) store_res(16 * j + i);
+                        } else if (c0 < cend) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (c0 + i < cend) store_res(16 * j + i);
+                        }
+                    }
+                }
+            } else if (!it.split) {
+                // kCh columns of both accumulators per TMEM round trip, stored 16 at a time
+                for (int c0 = cbeg; c0 < cend; c0 += kCh) {
+                    uint32_t ga[kCh], ua[kCh];
+                    if constexpr (kCh == 32) {
+                        tmem_ld32_nowait(tacc + c0, ga);
+                        if (kTwo) tmem_ld32_nowait(tacc + kMaxN + c0, ua);
+                    } else {
+                        tmem_ld16_nowait(tacc + c0, ga);
+                        if (kTwo) tmem_ld16_nowait(tacc + kMaxN + c0, ua);
+                    }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int h = 0; h < kCh / 16; ++h) {
                         float g[16], u[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             g[i] = __uint_as_float(ga[16 * h + i]);
                             u[i] = kTwo ? __uint_as_float(ua[16 * h + i]) : 0.f;
+                            if (kSwiGLU) g[i] = silu_mul(g[i], u[i]);
                         }
-                        if (c0 + 16 * h < t.nrows) emit(c0 + 16 * h, g, u);
+                        if (c0 + 16 * h < cend) emit(c0 + 16 * h, g, u);
                     }
                 }
+                release();
             } else {
                 // stream-K: publish this block's partial tile (rows of real
                 // output features and columns of real tokens only)
                 const long long slot_floats = 128LL * C::kAccCols;
                 float4* mine = reinterpret_cast<float4*>(p.partials + ((long long)blockIdx.x * 2 + it.slot) * slot_floats);
                 const long long counter = it.sk_tile * kCta + rank;  // one counter per tile half
-                for (int c0 = 0; c0 < t.nrows; c0 += 16) {
-                    float g[16];
-                    tmem_ld16(tacc + c0, g);
+                for (int c0 = cbeg; c0 < cend; c0 += kCh) {
+                    float g[kCh], u[kCh];
+                    load_cols(c0, g, u);
                     if (v0) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
+                        for (int q = 0; q < kCh / 4; ++q)
                             mine[slot_f4((c0 >> 2) + q, r)] =
                                 make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
                     }
-                    if (kTwo) {
-                        tmem_ld16(tacc + kMaxN + c0, g);
-                        if (v1) {
+                    if (kTwo && v1) {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                mine[slot_f4(((kMaxN + c0) >> 2) + q, r)] =
-                                    make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
-                        }
+                        for (int q = 0; q < kCh / 4; ++q)
+                            mine[slot_f4(((kMaxN + c0) >> 2) + q, r)] =
+                                make_float4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
                     }
                 }
                 __threadfence();
-                named_sync(1, 128);
-                if (r == 0) *bcast = atomicAdd(&p.counters[counter], 1);
-                named_sync(1, 128);
+                named_sync(1, kEpiThreads);
+                if (e == 0) *bcast = atomicAdd(&p.counters[counter], 1);
+                named_sync(1, kEpiThreads);
                 const int arrived = *bcast;
                 // contributors: blocks whose stream-K range meets this tile
                 const long long q0 = it.sk_tile * sch.KI;
@@ -565,7 +683,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (arrived == ncontrib - 1) {
                     // last to arrive: sum every contribution in block order, then the epilogue
                     __threadfence();
-                    for (int c0 = 0; c0 < t.nrows; c0 += 16) {
+                    for (int c0 = cbeg; c0 < cend; c0 += 16) {
                         float g[16], u[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
@@ -573,14 +691,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             const long long bc = sch.beg(c);
                             if (bc >= sch.beg(c + 1)) continue;
                             if (c == sch.cta) {
-                                float v[16];
-                                tmem_ld16(tacc + c0, v);
+                                uint32_t va[16], vb[16];
+                                tmem_ld16_nowait(tacc + c0, va);
+                                if (kTwo) tmem_ld16_nowait(tacc + kMaxN + c0, vb);
+                                tmem_wait_ld();
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) g[i] += v[i];
-                                if (kTwo) {
-                                    tmem_ld16(tacc + kMaxN + c0, v);
-#pragma unroll
-                                    for (int i = 0; i < 16; ++i) u[i] += v[i];
+                                for (int i = 0; i < 16; ++i) {
+                                    g[i] += __uint_as_float(va[i]);
+                                    if (kTwo) u[i] += __uint_as_float(vb[i]);
                                 }
                             } else {
                                 const int slot = (bc / sch.KI == it.sk_tile) ? 0 : 1;
@@ -614,14 +732,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 }
                             }
                         }
+                        if (kSwiGLU) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
+                        }
                         emit(c0, g, u);
                     }
-                    if (r == 0) p.counters[counter] = 0;  // leave the counter zero for the next launch
+                    if (e == 0) p.counters[counter] = 0;  // leave the counter zero for the next launch
                 }
+                release();
             }
-            tc_fence_before();
-            if (kPair && rank != 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[b]), 0));
-            else mbar_arrive(&tempty[b]);
             ++ac;
         }
     }

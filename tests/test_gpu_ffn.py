@@ -183,3 +183,19 @@ def test_fused_decode_ffn_matches_two_launch_path(shape_kw, T):
     a = y1[:P].float().cpu().numpy()[valid]
     b = y2[:P].float().cpu().numpy()[valid]
     assert rel_err(a, b) < 1e-2
+
+
+def test_dense_ffn_wide_pair_tiles():
+    # 64 token chunks x 4 blocks of 512 output features: enough tiles for the
+    # 512-feature (wide) CTA-pair down GEMM; fewer tiles take 256-feature pairs
+    T, H, I = 16384, 2048, 1024
+    w13, w2 = mi.make_dense_weights(H, I, torch.bfloat16, seed=7, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    x = torch.randn((T, H), generator=gen, device="cuda").to(torch.bfloat16)
+    ws = moe.alloc_workspace(moe.dense_workspace_size(T, H, I))
+    out = moe.dense_ffn(x, w13, w2, ws)
+    moe.check_status(ws)
+    tok = sample_tokens(T, 24, seed=7)
+    ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
+    assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
