@@ -47,7 +47,7 @@ def lib():
         L.oracle_router_logits.argtypes = [i, i, i, i, P, P, P]
         L.oracle_topk.argtypes = [i, i, i, P, P]
         L.oracle_gate_weights.argtypes = [i, i, i, i, i, P, P, P]
-        L.oracle_align.argtypes = [i, i, i, i, P, ctypes.c_int64, P, P, P, P, P, P, P]
+        L.oracle_align.argtypes = [i, i, i, i, i, P, ctypes.c_int64, P, P, P, P, P, P, P]
         L.oracle_swiglu_ffn.argtypes = [i, i, i, P, P, P, P]
         L.oracle_permute.argtypes = [i, i, i, P, P, i, P]
         L.oracle_combine.argtypes = [i, i, i, i, P, P, P, P, P]
@@ -123,18 +123,23 @@ def expected_active(E: int, K: int, m: int) -> float:
     return E * (1.0 - (1.0 - K / E) ** m)
 
 
-def p_max(T, K, E, B):
-    """Upper bound on padded rows: A + min(E, A) * (B - 1), A = T*K."""
+def p_max(T, K, E, B, mode=0):
+    """Upper bound on padded rows.  Block-wise (mode 0): A + min(E, A) * (B - 1),
+    A = T*K.  Max-value (mode 1): E * ceil(min(T, A) / B) * B (an expert holds at
+    most one assignment per token)."""
     A = T * K
+    if mode == 1:
+        return E * ((min(T, A) + B - 1) // B) * B
     return A + min(E, A) * (B - 1)
 
 
-def align(ids, E, B, P_max=None):
-    """Block-wise alignment of the assignments; returns a dict of int32 arrays."""
+def align(ids, E, B, P_max=None, mode=0):
+    """Alignment of the assignments with block-wise (mode 0) or max-value
+    (mode 1) padding; returns a dict of int32 arrays."""
     ids = np.ascontiguousarray(ids, dtype=np.int32)
     T, K = ids.shape
     if P_max is None:
-        P_max = p_max(T, K, E, B)
+        P_max = p_max(T, K, E, B, mode)
     nblk = (P_max + B - 1) // B
     counts = np.empty(E, np.int32)
     offsets = np.empty(E + 1, np.int32)
@@ -143,7 +148,7 @@ def align(ids, E, B, P_max=None):
     pos = np.empty(max(T * K, 1), np.int32)
     P = np.zeros(1, np.int32)
     ea = np.zeros(1, np.int32)
-    _check(lib().oracle_align(T, K, E, B, _ptr(ids), P_max, _ptr(counts), _ptr(offsets),
+    _check(lib().oracle_align(T, K, E, B, mode, _ptr(ids), P_max, _ptr(counts), _ptr(offsets),
                               _ptr(sorted_ids), _ptr(block_expert), _ptr(pos), _ptr(P), _ptr(ea)),
            "align")
     return dict(counts=counts, offsets=offsets, sorted_ids=sorted_ids[:P_max],

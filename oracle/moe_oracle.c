@@ -142,28 +142,35 @@ int oracle_gate_weights(int T, int E, int K, int score_fn, int renorm,
 /* ---------------------------------------------------------- align + pad */
 /* Assignments a = t*K + k, expert e(a) = ids[a], A = T*K.
  *   counts[e]  = N_e = #{a : e(a) = e}
- *   padded N^_e = ceil(N_e / B) * B                    (block-wise padding)
+ *   padded N^_e = ceil(N_e / B) * B                    (mode 0, block-wise padding)
+ *              = ceil(max_i N_i / B) * B for every e    (mode 1, max-value padding:
+ *                all experts take the size of the most loaded one; same page,
+ *                "Padding model (Section 5.1)", P_g = E_g * ceil(max N_i / B) * B
+ *                with E_g = E on one GPU)
  *   offsets    = exclusive scan of N^, offsets[E] = P = sum_e N^_e
  *   sorted_ids[p] = a, a ascending within each expert's segment; -1 elsewhere
  *   pos[a]     = the slot p holding a
  *   block_expert[b] = e for b in [offsets[e]/B, offsets[e+1]/B), -1 for b >= P/B
  *   E_active   = #{e : N_e > 0}
  * sorted_ids has P_max slots, block_expert ceil(P_max/B) entries. */
-int oracle_align(int T, int K, int E, int B, const int32_t* ids, int64_t P_max,
+int oracle_align(int T, int K, int E, int B, int mode, const int32_t* ids, int64_t P_max,
                  int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                  int32_t* block_expert, int32_t* pos, int32_t* P_out,
                  int32_t* E_active_out)
 {
-    if (T < 0 || K <= 0 || E <= 0 || B <= 0) return -1;
+    if (T < 0 || K <= 0 || E <= 0 || B <= 0 || (mode != 0 && mode != 1)) return -1;
     int64_t A = (int64_t)T * K;
     for (int e = 0; e < E; ++e) counts[e] = 0;
     for (int64_t a = 0; a < A; ++a) {
         if (ids[a] < 0 || ids[a] >= E) return -1;
         counts[ids[a]] += 1;
     }
+    int32_t n_max = 0;
+    for (int e = 0; e < E; ++e) if (counts[e] > n_max) n_max = counts[e];
     offsets[0] = 0;
     for (int e = 0; e < E; ++e) {
-        int32_t padded = ((counts[e] + B - 1) / B) * B;
+        int32_t n = mode == 0 ? counts[e] : n_max;
+        int32_t padded = ((n + B - 1) / B) * B;
         offsets[e + 1] = offsets[e] + padded;
     }
     int32_t P = offsets[E];

@@ -211,6 +211,64 @@ def test_align_single_expert_closed_form():
         assert r["sorted_ids"][:T].tolist() == list(range(T))
 
 
+def _check_max_value_invariants(ids, E, B, r):
+    # max-value padding (Section 5.1): every expert's segment has the padded
+    # size of the most loaded expert, P = E * ceil(max N_i / B) * B
+    T, K = ids.shape
+    A = T * K
+    counts, offsets, sid, be, pos = r["counts"], r["offsets"], r["sorted_ids"], r["block_expert"], r["pos"]
+    assert np.array_equal(counts, np.bincount(ids.ravel(), minlength=E))
+    M = -(-int(counts.max()) // B) * B if A else 0
+    assert np.all(np.diff(offsets) == M)
+    assert r["P"] == E * M == offsets[E]
+    assert len(sid) == oracle.p_max(T, K, E, B, mode=1) >= r["P"]
+    assert np.array_equal(np.sort(sid[sid >= 0]), np.arange(A))
+    for a in range(A):
+        assert sid[pos[a]] == a
+    for e in range(E):
+        seg = sid[offsets[e]:offsets[e + 1]]
+        assert np.all(np.diff(seg[:counts[e]]) > 0) and np.all(ids.ravel()[seg[:counts[e]]] == e)
+        assert np.all(seg[counts[e]:] == -1)
+        assert np.all(be[offsets[e] // B:offsets[e + 1] // B] == e)
+    assert np.all(be[r["P"] // B:] == -1)
+    assert r["E_active"] == int((counts > 0).sum())
+
+
+def test_align_max_value_worked_example():
+    # T = 3, K = 2, E = 4, B = 4: counts (2, 1, 3, 0), the largest 3 pads to 4,
+    # so every expert gets 4 rows and P = 16 (block-wise: 4 + 4 + 4 + 0 = 12)
+    ids = np.array([[0, 2], [2, 1], [2, 0]], np.int32)
+    r = oracle.align(ids, 4, 4, mode=1)
+    assert r["counts"].tolist() == [2, 1, 3, 0]
+    assert r["offsets"].tolist() == [0, 4, 8, 12, 16] and r["P"] == 16
+    assert r["sorted_ids"][:16].tolist() == [0, 5, -1, -1, 3, -1, -1, -1, 1, 2, 4, -1, -1, -1, -1, -1]
+    assert r["pos"].tolist() == [0, 8, 9, 4, 10, 1]
+    assert r["block_expert"][:4].tolist() == [0, 1, 2, 3]
+    assert r["E_active"] == 3
+    assert oracle.align(ids, 4, 4)["P"] == 12
+
+
+@pytest.mark.parametrize("B", [1, 4, 16, 128])
+def test_align_max_value_invariants_random(B):
+    rng = np.random.default_rng(100 + B)
+    for T, E, K in [(1, 8, 2), (37, 8, 2), (64, 64, 8), (50, 256, 8), (3, 5, 5), (0, 4, 2)]:
+        lg = rng.standard_normal((T, E)).astype(np.float32)
+        ids = oracle.topk(lg, K) if T else np.zeros((0, K), np.int32)
+        _check_max_value_invariants(ids, E, B, oracle.align(ids, E, B, mode=1))
+
+
+def test_align_padding_schemes_extremes():
+    # the two schemes' worst cases (Section 5.1): a concentrated distribution
+    # (all tokens on one expert) costs max-value padding E times block-wise,
+    # a dispersed one (each expert a single token) costs them the same
+    E, B = 8, 16
+    hot = np.zeros((40, 1), np.int32)
+    assert oracle.align(hot, E, B)["P"] == 48
+    assert oracle.align(hot, E, B, mode=1)["P"] == E * 48
+    spread = np.arange(E, dtype=np.int32).reshape(E, 1)
+    assert oracle.align(spread, E, B)["P"] == oracle.align(spread, E, B, mode=1)["P"] == E * B
+
+
 def test_align_rejects_bad_ids():
     with pytest.raises(ValueError):
         oracle.align(np.array([[0, 5]], np.int32), 4, 4)
