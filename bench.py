@@ -123,7 +123,7 @@ def parse_workload(s):
 
 
 class Workload:
-    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None):
+    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None, pad_mode=0):
         import mixture_experts_layer_61_b200 as moe
         self.moe = moe
         self.shape, self.T = shape, T
@@ -136,7 +136,7 @@ class Workload:
         n_sh, I_s = (1, shape.I_sh) if shape.I_sh else (0, 0)
         self.cfg = moe.config(T, shape.H, shape.E, shape.K, shape.I, n_shared=n_sh, I_shared=I_s,
                               tile_B=shape.tile_B, score_fn=shape.score_fn, renorm=shape.renorm,
-                              dtype=moe.BF16 if shape.dtype == "bf16" else moe.FP32)
+                              dtype=moe.BF16 if shape.dtype == "bf16" else moe.FP32, pad_mode=pad_mode)
         self.ws = moe.alloc_workspace(moe.workspace_size(self.cfg), device)
         self.stats = torch.zeros(4, dtype=torch.int32, device=device)
         self.out = torch.empty((T, shape.H), dtype=shape.torch_dtype, device=device)
@@ -353,6 +353,10 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch each step from the host instead of a CUDA graph")
     ap.add_argument("--token-tile-cap", type=int, default=0, help="grouped GEMM token-tile cap (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream order between kernels")
+    ap.add_argument("--pad-mode", type=int, default=0, choices=[0, 1],
+                    help="alignment padding: 0 block-wise, 1 max-value")
+    ap.add_argument("--padding-model", action="store_true",
+                    help="time the expert FFN over routings and fit the padding and max-affine latency models")
     ap.add_argument("--shared-sms", type=int, default=0,
                     help="SMs for the shared experts beside the routed ones (0 = cost model, -1 = serial)")
     args = ap.parse_args()
@@ -382,8 +386,15 @@ def main():
         moe.set_programmatic_launch(False)
     if args.shared_sms:
         moe.set_shared_sms(args.shared_sms)
-    wl = Workload(shape, T, rank, device, skew=args.skew)
     flush = l2_flush_buffer(device)
+    if args.padding_model:
+        if rank == 0:
+            print(json.dumps(run_padding_model(args, device, flush)), flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    wl = Workload(shape, T, rank, device, skew=args.skew, pad_mode=args.pad_mode)
     if args.no_graph:
         run_step, wl.launches_per_step = wl.step, None
     else:
@@ -528,7 +539,8 @@ def main():
                    "parallelism": f"replicas x{world} (data parallel, no collective)",
                    "launch": "host launches" if args.no_graph else "CUDA graph replay of moe_layer_forward",
                    "l2": "flushed between steps (2 GiB write outside the events); weights exceed L2",
-                   "shared_sms": moe.shared_sms(wl.cfg)},
+                   "shared_sms": moe.shared_sms(wl.cfg),
+                   "padding": "max-value" if args.pad_mode == 1 else "block-wise"},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - T * shape.K) / max(P, 1), 4),
                   "bytes_alg": B_alg, "flops_alg": F_alg, "roofline_frac": round(layer_roof, 4),
@@ -597,6 +609,93 @@ def run_sweep(args, device, flush, pk):
         del weights
         torch.cuda.empty_cache()
     return rows
+
+
+def ffn_time(wl, steps, flush):
+    """Median device time (ms) of the routed expert FFN alone (the fused
+    launch, or gate/up + down), from the per-stage events of staged steps."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+    names = Workload.STAGES_FUSED if wl.fused else Workload.STAGES
+    out = []
+    for i in range(3 + steps):
+        flush.zero_()
+        wl.staged_step(ev)
+        ev[8].synchronize()
+        if i >= 3:
+            st = {s: ev[j].elapsed_time(ev[j + 1]) for j, s in enumerate(names)}
+            out.append(st["ffn"] if wl.fused else st["gate_up"] + st["down"])
+    wl.moe.check_status(wl.gws)
+    return statistics.median(out)
+
+
+def fit_latency_models(rows):
+    """Least-squares fits of the expert-FFN time t (ms) over the sweep points:
+    the padding model t = c + beta * P on the points in the compute regime
+    (Demystifying the MoE Serving Tax, "Padding model (Section 5.1)": latency
+    from the padded rows P), and the max-affine profile
+    t = max(a + b * G, c + beta * N) of the TEMPO write-up (G activated
+    experts, N rows the kernel computes = P) on all points.  G counts the
+    experts whose weights the kernel streams: the activated ones under
+    block-wise padding, all E under max-value padding."""
+    import numpy as np
+    from scipy.optimize import least_squares
+    G = np.array([r["G"] for r in rows], float)
+    P = np.array([r["P"] for r in rows], float)
+    t = np.array([r["ffn_ms"] for r in rows], float)
+
+    def r2(pred):
+        return float(1.0 - ((t - pred) ** 2).sum() / max(((t - t.mean()) ** 2).sum(), 1e-30))
+
+    mem = np.polyfit(G, t, 1)      # t ~ a + b G
+    comp = np.polyfit(P, t, 1)     # t ~ c + beta P
+    x0 = [mem[1], mem[0], comp[1], comp[0]]
+    f = lambda q: np.maximum(q[0] + q[1] * G, q[2] + q[3] * P) - t
+    q = least_squares(f, x0).x
+    pred = np.maximum(q[0] + q[1] * G, q[2] + q[3] * P)
+    compute = (q[2] + q[3] * P) > (q[0] + q[1] * G)
+    out = {"max_affine": {"a_ms": q[0], "b_ms_per_expert": q[1], "c_ms": q[2], "beta_ms_per_row": q[3],
+                          "r2": r2(pred), "points": int(len(t)), "compute_regime_points": int(compute.sum())},
+           "linear_in_P_all_points": {"r2": r2(np.polyval(comp, P))}}
+    if compute.sum() >= 3:
+        pc = np.polyfit(P[compute], t[compute], 1)
+        tc = t[compute]
+        out["padding_model_compute_regime"] = {
+            "c_ms": pc[1], "beta_ms_per_row": pc[0],
+            "r2": float(1.0 - ((tc - np.polyval(pc, P[compute])) ** 2).sum() / max(((tc - tc.mean()) ** 2).sum(), 1e-30))}
+    return out
+
+
+def run_padding_model(args, device, flush):
+    """Expert-FFN time over routings of the DeepSeek-V3-shaped layer: T = 1..4096
+    with Zipf(s) Gumbel logits, s in {0, 0.5, 1, 1.5}, block-wise padding; and
+    T = 1..128 with max-value padding.  Each point records E_active, P and the
+    FFN time; the fits follow (fit_latency_models)."""
+    import mixture_experts_layer_61_b200 as moe
+    sh = mi.SHAPES["deepseekv3"]
+    weights = mi.make_weights(sh, mi.seed_for(sh, 0), device=device)
+    plan = [(0, 2 ** k, s) for s in (0.0, 0.5, 1.0, 1.5) for k in range(13)]
+    plan += [(1, 2 ** k, s) for s in (0.0, 1.5) for k in range(8)]
+    rows = []
+    for mode, T, s in plan:
+        wl = Workload(sh, T, 0, device, skew=s, weights=weights, pad_mode=mode)
+        t = ffn_time(wl, max(3, args.steps // 4), flush)
+        st = wl.al["scalars"].cpu().tolist()
+        G = int((torch.diff(wl.al["offsets"]) > 0).sum().item())  # segments with rows: experts streamed
+        row = {"layer": sh.name, "pad_mode": mode, "T": T, "skew": s, "E_active": st[1], "G": G, "P": st[0],
+               "A": T * sh.K, "ffn_ms": round(t, 4), "fused_ffn": bool(wl.fused)}
+        rows.append(row)
+        if args.sweep_out:
+            with open(args.sweep_out, "a") as f:
+                f.write(json.dumps(row) + "\n")
+        del wl
+        torch.cuda.empty_cache()
+    fits = {"block-wise": fit_latency_models([r for r in rows if r["pad_mode"] == 0]),
+            "all": fit_latency_models(rows)}
+    mv = [r for r in rows if r["pad_mode"] == 1]
+    bw = {(r["T"], r["skew"]): r for r in rows if r["pad_mode"] == 0}
+    compare = [{"T": r["T"], "skew": r["skew"], "P_block": bw[(r["T"], r["skew"])]["P"], "P_max_value": r["P"],
+                "ms_block": bw[(r["T"], r["skew"])]["ffn_ms"], "ms_max_value": r["ffn_ms"]} for r in mv]
+    return {"padding_model": fits, "max_value_vs_block": compare, "layer": sh.name, "points": len(rows)}
 
 
 def reference_arm(args, shape, T, rank, world, local, dist):

@@ -79,6 +79,10 @@ typedef struct {
     int score_fn;   /* 0 = softmax, 1 = sigmoid */
     int renorm;     /* 1: weights normalised over the selected K */
     int dtype;      /* 0 = bf16, 1 = fp32 (activations and weights) */
+    int pad_mode;   /* 0 = block-wise padding: each expert's rows rounded up to
+                       tile_B; 1 = max-value padding: every expert gets the
+                       rounded row count of the most loaded expert (Demystifying
+                       the MoE Serving Tax, "Padding model (Section 5.1)") */
 } moe_config_t;
 
 /* Text for a status code (static storage). */

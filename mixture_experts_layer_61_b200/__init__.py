@@ -33,16 +33,21 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     """moe_config_t (include/moe.h)."""
     _fields_ = [(n, ctypes.c_int) for n in
-                ("T", "H", "E", "K", "I", "n_shared", "I_shared", "tile_B", "score_fn", "renorm", "dtype")]
+                ("T", "H", "E", "K", "I", "n_shared", "I_shared", "tile_B", "score_fn", "renorm", "dtype",
+                 "pad_mode")]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
-def config(T, H, E, K, I, n_shared=0, I_shared=0, tile_B=16, score_fn=SOFTMAX, renorm=1, dtype=BF16):
+BLOCKWISE, MAXVALUE = 0, 1  # padding schemes of the alignment
+
+
+def config(T, H, E, K, I, n_shared=0, I_shared=0, tile_B=16, score_fn=SOFTMAX, renorm=1, dtype=BF16,
+           pad_mode=BLOCKWISE):
     if isinstance(dtype, torch.dtype):
         dtype = BF16 if dtype == torch.bfloat16 else FP32
-    return MoeConfig(T, H, E, K, I, n_shared, I_shared, tile_B, score_fn, renorm, dtype)
+    return MoeConfig(T, H, E, K, I, n_shared, I_shared, tile_B, score_fn, renorm, dtype, pad_mode)
 
 
 def lib():

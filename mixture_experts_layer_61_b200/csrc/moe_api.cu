@@ -79,6 +79,7 @@ int check_cfg(const moe_config_t* c) {
     if (c->tile_B < 1 || c->tile_B > 256) return MOE_ERR_ARG;
     if (c->score_fn != 0 && c->score_fn != 1) return MOE_ERR_ARG;
     if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_ARG;
+    if (c->pad_mode != 0 && c->pad_mode != 1) return MOE_ERR_ARG;
     if (c->H % vec != 0 || c->I % vec != 0) return MOE_ERR_ARG;
     const long long I_sh = (long long)c->n_shared * c->I_shared;
     if (I_sh % vec != 0 || I_sh > (1LL << 30)) return MOE_ERR_ARG;
@@ -90,6 +91,11 @@ int check_cfg(const moe_config_t* c) {
 
 long long p_max(const moe_config_t* c) {
     const long long A = (long long)c->T * c->K;
+    if (c->pad_mode == 1) {
+        // an expert holds at most one assignment per token
+        const long long n = A < c->T ? A : c->T;
+        return (long long)c->E * ((n + c->tile_B - 1) / c->tile_B) * c->tile_B;
+    }
     return A + (A < c->E ? A : c->E) * (long long)(c->tile_B - 1);
 }
 
@@ -400,7 +406,8 @@ int moe_align_pad(const moe_config_t* cfg, const int32_t* topk_ids, int32_t* cou
     if (cfg->T > 0 && (!topk_ids || !sorted_ids || !pos)) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
-    return status_of(launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, p_max(cfg), topk_ids, counts, offsets,
+    return status_of(launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, cfg->pad_mode, p_max(cfg), topk_ids,
+                                  counts, offsets,
                                   sorted_ids, block_expert, pos, scalars, nullptr, (cudaStream_t)stream));
 }
 
@@ -560,7 +567,8 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
     if (cfg->T <= kSmallRouteMaxT && cfg->H % 8 == 0) {
         // router logits, top-K and alignment in one launch (decode-sized batches)
         int* route_ctr = reinterpret_cast<int*>(at<uint8_t>(workspace, L.ctl)) + 16;  // in the control header
-        if ((rc = launch_route_small(cfg->T, cfg->H, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, cfg->tile_B, P,
+        if ((rc = launch_route_small(cfg->T, cfg->H, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, cfg->tile_B,
+                                     cfg->pad_mode, P,
                                      cfg->dtype, x, w_router, logits_override, at<float>(workspace, L.route_part),
                                      logits, ids, w, counts, offsets, sorted_ids, block_expert, pos, scalars,
                                      stats_out, route_ctr, s)) != 0)
@@ -585,7 +593,8 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
         if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm,
                               logits_override ? logits_override : logits, ids, w, s)) != 0)
             return status_of(rc);
-        if ((rc = launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, P, ids, counts, offsets, sorted_ids, block_expert,
+        if ((rc = launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, cfg->pad_mode, P, ids, counts, offsets,
+                               sorted_ids, block_expert,
                                pos, scalars, stats_out, s)) != 0)
             return status_of(rc);
     }

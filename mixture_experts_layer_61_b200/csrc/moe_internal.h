@@ -137,13 +137,16 @@ void set_cta_pairs(bool on);
 // Elementwise / routing kernels.
 int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,
                 cudaStream_t stream);
-int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids, int32_t* counts,
+// mode 0: block-wise padding, 1: max-value padding (every expert padded to the
+// most loaded one's rounded count).
+int launch_align(int T, int K, int E, int B, int mode, long long P_max, const int32_t* ids, int32_t* counts,
                  int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
                  int32_t* stats_copy, cudaStream_t stream);
 // Router logits (CUDA cores) + top-K + alignment in one launch, for small T.
 constexpr int kSmallRouteMaxT = 64;
 // `part` holds (H/256 + 1) * T * E floats of partial router sums.
-int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, long long P_max, int dtype,
+int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
+                       int dtype,
                        const void* x, const void* w_r, const float* logits_override, float* part, float* logits,
                        int32_t* ids, float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                        int32_t* block_expert, int32_t* pos, int32_t* scalars, int32_t* stats_copy, int* done_ctr,

@@ -174,7 +174,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
 
 // The alignment of T*K assignments by one block of kAlignThreads threads;
 // `sm` is dynamic shared memory of align_smem_bytes(E) bytes.
-__device__ __forceinline__ void align_block(int T, int K, int E, int B, long long P_max, const int32_t* ids,
+__device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode, long long P_max, const int32_t* ids,
                                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                             int32_t* __restrict__ sorted_ids, int32_t* __restrict__ block_expert,
                                             int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
@@ -185,12 +185,13 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, long lon
     int* rt = cursor + E;          // E
     int* warp_tot = rt + E;        // 33
     int* bad = warp_tot + 33;      // 1
-    uint16_t* tbl = reinterpret_cast<uint16_t*>(bad + 1);  // 32 x E
+    int* nmax = bad + 1;           // 1
+    uint16_t* tbl = reinterpret_cast<uint16_t*>(nmax + 1);  // 32 x E
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long A = (long long)T * K;
 
     for (int e = tid; e < E; e += kAlignThreads) cnt[e] = 0;
-    if (tid == 0) *bad = 0;
+    if (tid == 0) *bad = 0, *nmax = 0;
     __syncthreads();
     for (long long a = tid; a < A; a += kAlignThreads) {
         const int e = ids[a];
@@ -199,9 +200,17 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, long lon
     }
     __syncthreads();
 
-    // padded counts -> offsets (E <= 1024: one expert per thread)
+    // padded counts -> offsets (E <= 1024: one expert per thread).  Block-wise
+    // padding rounds each count up to B; max-value padding gives every expert
+    // the rounded size of the most loaded one.
     const int n = tid < E ? cnt[tid] : 0;
-    const int padded = ((n + B - 1) / B) * B;
+    int padded = ((n + B - 1) / B) * B;
+    if (mode == 1) {
+        const int wmax = __reduce_max_sync(0xffffffffu, n);
+        if (lane == 0 && wmax > 0) atomicMax(nmax, wmax);
+        __syncthreads();
+        padded = tid < E ? ((*nmax + B - 1) / B) * B : 0;
+    }
     int P = 0;
     const int excl = block_excl_scan(padded, warp_tot, P);
     const int n_active = __syncthreads_count(tid < E && n > 0);
@@ -281,17 +290,18 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, long lon
 }
 
 __global__ void __launch_bounds__(kAlignThreads, 1)
-    align_kernel(int T, int K, int E, int B, long long P_max, const int32_t* __restrict__ ids,
+    align_kernel(int T, int K, int E, int B, int mode, long long P_max, const int32_t* __restrict__ ids,
                  int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
                  int32_t* __restrict__ block_expert, int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
                  int32_t* __restrict__ stats_copy) {
     extern __shared__ int sm[];
     pdl_launch_dependents();
     pdl_wait();
-    align_block(T, K, E, B, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy, sm);
+    align_block(T, K, E, B, mode, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy,
+                sm);
 }
 
-size_t align_smem_bytes(int E) { return sizeof(int) * (4 * (size_t)E + 1 + 34) + sizeof(uint16_t) * 32 * (size_t)E; }
+size_t align_smem_bytes(int E) { return sizeof(int) * (4 * (size_t)E + 1 + 35) + sizeof(uint16_t) * 32 * (size_t)E; }
 
 // ----------------------------------------------------- small-batch routing
 // Router logits, top-K gating and alignment in one launch for small T.
@@ -322,7 +332,8 @@ __device__ __forceinline__ void load8(const float* p, float* f) {
 
 template <typename T>
 __global__ void __launch_bounds__(kAlignThreads, 1)
-    route_small_kernel(int T_, int H, int E, int K, int score_fn, int renorm, int B, long long P_max, int nslices,
+    route_small_kernel(int T_, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
+                       int nslices,
                        int slice_w, const T* __restrict__ x, const T* __restrict__ w_r,
                        const float* __restrict__ logits_override, float* __restrict__ part, float* __restrict__ logits,
                        int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ counts,
@@ -386,7 +397,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     for (int t = warp; t < T_; t += kAlignThreads / 32)
         topk_one_token(src + (size_t)t * E, E, K, score_fn, renorm, ids + (size_t)t * K, w + (size_t)t * K, lane);
     __syncthreads();
-    align_block(T_, K, E, B, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy, sm);
+    align_block(T_, K, E, B, mode, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy,
+                sm);
     if (threadIdx.x == 0) *done_ctr = 0;  // ready for the next launch
 }
 
@@ -404,7 +416,8 @@ void route_small_slices(int T, int H, int E, int num_sms, int* nslices, int* sli
     *nslices = (H + w - 1) / w;
 }
 
-int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, long long P_max, int dtype,
+int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
+                       int dtype,
                        const void* x, const void* w_r, const float* logits_override, float* part, float* logits,
                        int32_t* ids, float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                        int32_t* block_expert, int32_t* pos, int32_t* scalars, int32_t* stats_copy, int* done_ctr,
@@ -431,19 +444,19 @@ int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int
     cudaError_t e;
     if (dtype == 0)
         e = launch_kernel(route_small_kernel<__nv_bfloat16>, dim3(blocks), dim3(kAlignThreads), smem, stream, T, H, E,
-                          K, score_fn, renorm, B, P_max, ns, sw, static_cast<const __nv_bfloat16*>(x),
+                          K, score_fn, renorm, B, mode, P_max, ns, sw, static_cast<const __nv_bfloat16*>(x),
                           static_cast<const __nv_bfloat16*>(w_r), logits_override, part, logits, ids, w, counts,
                           offsets, sorted_ids, block_expert, pos, scalars, stats_copy, done_ctr);
     else
         e = launch_kernel(route_small_kernel<float>, dim3(blocks), dim3(kAlignThreads), smem, stream, T, H, E, K,
-                          score_fn, renorm, B, P_max, ns, sw, static_cast<const float*>(x),
+                          score_fn, renorm, B, mode, P_max, ns, sw, static_cast<const float*>(x),
                           static_cast<const float*>(w_r), logits_override, part, logits, ids, w, counts, offsets,
                           sorted_ids, block_expert, pos, scalars, stats_copy, done_ctr);
     count_launch();
     return launched(e);
 }
 
-int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids, int32_t* counts,
+int launch_align(int T, int K, int E, int B, int mode, long long P_max, const int32_t* ids, int32_t* counts,
                  int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
                  int32_t* stats_copy, cudaStream_t stream) {
     const size_t smem = align_smem_bytes(E);
@@ -456,7 +469,7 @@ int launch_align(int T, int K, int E, int B, long long P_max, const int32_t* ids
         }
         attr_done = true;
     }
-    cudaError_t e = launch_kernel(align_kernel, dim3(1), dim3(kAlignThreads), smem, stream, T, K, E, B, P_max, ids,
+    cudaError_t e = launch_kernel(align_kernel, dim3(1), dim3(kAlignThreads), smem, stream, T, K, E, B, mode, P_max, ids,
                                   counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy);
     count_launch();
     return launched(e);

@@ -36,11 +36,11 @@ def make_layer(shape, T, seed, device="cuda"):
     return x, w
 
 
-def cfg_for(shape, T, B=None):
+def cfg_for(shape, T, B=None, pad_mode=0):
     n_sh, I_s = (1, shape.I_sh) if shape.I_sh else (0, 0)
     return moe.config(T, shape.H, shape.E, shape.K, shape.I, n_shared=n_sh, I_shared=I_s,
                       tile_B=B or shape.tile_B, score_fn=shape.score_fn, renorm=shape.renorm,
-                      dtype=moe.BF16 if shape.dtype == "bf16" else moe.FP32)
+                      dtype=moe.BF16 if shape.dtype == "bf16" else moe.FP32, pad_mode=pad_mode)
 
 
 def sample_tokens(T, n, seed):

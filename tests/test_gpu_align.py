@@ -1,7 +1,7 @@
-"""Alignment with block-wise padding, permute and combine on the GPU against the
-oracle: every index output bit-exact (counts, offsets, sorted_ids,
-block_expert, pos, P, E_active), the permute an exact row copy, the combine
-within fp32 rounding."""
+"""Alignment with block-wise and max-value padding, permute and combine on the
+GPU against the oracle: every index output bit-exact (counts, offsets,
+sorted_ids, block_expert, pos, P, E_active), the permute an exact row copy,
+the combine within fp32 rounding."""
 import numpy as np
 import pytest
 import torch
@@ -27,12 +27,13 @@ def _ids(T, E, K, seed, kind="uniform"):
     return oracle.topk(lg, K)
 
 
-def _check_align(T, E, K, B, ids_np):
-    cfg = moe.config(T, 64, E, K, 64, tile_B=B)
+def _check_align(T, E, K, B, ids_np, mode=0):
+    cfg = moe.config(T, 64, E, K, 64, tile_B=B, pad_mode=mode)
     ids = torch.from_numpy(ids_np).cuda()
     g = moe.align_pad(cfg, ids)
     torch.cuda.synchronize()
-    r = oracle.align(ids_np, E, B)
+    r = oracle.align(ids_np, E, B, mode=mode)
+    assert moe.padded_rows_max(cfg) == oracle.p_max(T, K, E, B, mode)
     for key in ("counts", "offsets", "sorted_ids", "block_expert", "pos"):
         assert np.array_equal(g[key].cpu().numpy(), r[key]), key
     sc = g["scalars"].cpu().numpy()
@@ -46,6 +47,14 @@ def _check_align(T, E, K, B, ids_np):
 @pytest.mark.parametrize("kind", ["uniform", "zipf", "one", "ties"])
 def test_align_bit_exact(T, E, K, B, kind):
     _check_align(T, E, K, B, _ids(T, E, K, seed=T + E + B, kind=kind))
+
+
+@pytest.mark.parametrize("T,E,K,B", [(1, 8, 2, 16), (64, 8, 2, 16), (128, 64, 8, 16), (32, 256, 8, 16),
+                                     (512, 256, 8, 16), (333, 64, 8, 32), (50, 1024, 16, 8), (7, 5, 5, 1),
+                                     (129, 8, 2, 256)])
+@pytest.mark.parametrize("kind", ["uniform", "zipf", "one", "ties"])
+def test_align_max_value_bit_exact(T, E, K, B, kind):
+    _check_align(T, E, K, B, _ids(T, E, K, seed=T + E + B + 1, kind=kind), mode=1)
 
 
 def test_align_empty():

@@ -22,10 +22,10 @@ pytestmark = pytest.mark.gpu
 N_SAMPLE = int(os.environ.get("MOE_TEST_SAMPLE", "256"))
 
 
-def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True):
+def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True, pad_mode=0):
     w = mi.make_weights(shape, seed, device="cuda")
     x = mi.make_x(shape, T, seed, device="cuda")
-    cfg = cfg_for(shape, T)
+    cfg = cfg_for(shape, T, pad_mode=pad_mode)
     ws = moe.alloc_workspace(moe.workspace_size(cfg))
     stats = torch.zeros(4, dtype=torch.int32, device="cuda")
     out = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w.get("w13_sh"), w.get("w2_sh"),
@@ -39,7 +39,7 @@ def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True):
     lg = layer_lg if override is None else override.cpu().numpy()
     ids = oracle.topk(lg, shape.K)
     if check_stats:
-        r = oracle.align(ids, shape.E, shape.tile_B)
+        r = oracle.align(ids, shape.E, shape.tile_B, mode=pad_mode)
         st = stats.cpu().numpy()
         assert st[0] == r["P"] and st[1] == r["E_active"] and st[2] == 0
     tok = sample_tokens(T, n_sample or T, seed)
@@ -136,3 +136,17 @@ def test_layer_side_stream_captured_in_cuda_graph(T):
     moe.check_status(ws)
     assert torch.equal(out, ref)
     del g
+
+
+@pytest.mark.parametrize("T", [1, 20, 64, 200])
+def test_layer_max_value_padding(T):
+    # every expert padded to the most loaded one's rows: the padding slots are
+    # zero rows, so the outputs equal the oracle's (which does not pad); T <= 64
+    # runs the fused small-batch routing kernel, larger T the separate launches
+    shape = small_shape(H=512, E=16, K=4, I=384, I_sh=256)
+    assert _run_layer(shape, T, seed=T + 50, pad_mode=1) < OUT_TOL
+
+
+def test_layer_max_value_padding_deepseek_decode():
+    shape = mi.SHAPES["deepseekv3"]
+    assert _run_layer(shape, 32, seed=mi.seed_for(shape, 32), n_sample=64, pad_mode=1) < OUT_TOL
