@@ -46,13 +46,15 @@ def lib():
         i = ctypes.c_int
         L.oracle_router_logits.argtypes = [i, i, i, i, P, P, P]
         L.oracle_topk.argtypes = [i, i, i, P, P]
+        L.oracle_topk_k.argtypes = [i, i, i, P, P, P]
+        L.oracle_topk_k.restype = ctypes.c_int
         L.oracle_gate_weights.argtypes = [i, i, i, i, i, P, P, P]
         L.oracle_align.argtypes = [i, i, i, i, i, P, ctypes.c_int64, P, P, P, P, P, P, P]
         L.oracle_swiglu_ffn.argtypes = [i, i, i, P, P, P, P]
         L.oracle_permute.argtypes = [i, i, i, P, P, i, P]
         L.oracle_combine.argtypes = [i, i, i, i, P, P, P, P, P]
         L.oracle_dense_ffn.argtypes = [i, i, i, i, P, P, P, P, i]
-        L.oracle_moe_layer.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, i, P, P, P, i]
+        L.oracle_moe_layer.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, i, P, P, P, i]
         for f in (L.oracle_router_logits, L.oracle_topk, L.oracle_gate_weights, L.oracle_align,
                   L.oracle_swiglu_ffn, L.oracle_dense_ffn, L.oracle_moe_layer, L.oracle_permute,
                   L.oracle_combine):
@@ -96,12 +98,15 @@ def router_logits(x, w_r):
     return out
 
 
-def topk(logits, K):
-    """ids[T,K] int32: K largest fp32 logits per token, lower index on ties."""
+def topk(logits, K, k=None):
+    """ids[T,K] int32: K largest fp32 logits per token, lower index on ties.
+    With k (int32 [T], 0 <= k[t] <= K) token t takes its k[t] largest and the
+    slots from k[t] on hold -1 (per-token dynamic K)."""
     logits = np.ascontiguousarray(logits, dtype=np.float32)
     T, E = logits.shape
     ids = np.empty((T, K), np.int32)
-    _check(lib().oracle_topk(T, E, K, _ptr(logits), _ptr(ids)), "topk")
+    kk = None if k is None else np.ascontiguousarray(k, dtype=np.int32)
+    _check(lib().oracle_topk_k(T, E, K, _ptr(kk), _ptr(logits), _ptr(ids)), "topk")
     return ids
 
 
@@ -207,7 +212,7 @@ def dense_ffn(x, w13, w2, nthreads=None):
 
 
 def moe_layer(x, w_r, w13, w2, K, score_fn=0, renorm=1, w13_sh=None, w2_sh=None,
-              logits=None, tokens=None, nthreads=None, return_routing=False):
+              logits=None, tokens=None, nthreads=None, return_routing=False, k=None):
     """MoE layer output rows (float64) for the listed tokens (all if None).
 
     w13 / w2: either stacked arrays [E,2I,H] / [E,H,I], or lists of per-expert
@@ -257,8 +262,9 @@ def moe_layer(x, w_r, w13, w2, K, score_fn=0, renorm=1, w13_sh=None, w2_sh=None,
     out = np.empty((n, H), np.float64)
     ids = np.empty((n, K), np.int32)
     w = np.empty((n, K), np.float64)
+    kk = None if k is None else np.ascontiguousarray(k, dtype=np.int32)
     rc = lib().oracle_moe_layer(T, H, E, K, I, I_sh, score_fn, renorm, dt, _ptr(x), _ptr(w_r_c),
-                                p13, p2, _ptr(w13_sh), _ptr(w2_sh), _ptr(lg), _ptr(tok), n,
+                                p13, p2, _ptr(w13_sh), _ptr(w2_sh), _ptr(lg), _ptr(kk), _ptr(tok), n,
                                 _ptr(out), _ptr(ids), _ptr(w), nthreads or nthreads_default())
     _check(rc, "moe_layer")
     if return_routing:

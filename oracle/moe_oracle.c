@@ -21,7 +21,9 @@
  *     P = sum_i ceil(N_i / B) * B);
  *   - same page, "Balls-Bins-Buckets" (token-count vector N = [N_1..N_E],
  *     m tokens x K assignments);
- *   - same page, Table 2 (shared experts).
+ *   - same page, Table 2 (shared experts);
+ *   - the MoE-Prism write-up (routing top-k as a per-request runtime knob):
+ *     per-token dynamic K, k_t <= K, unused slots -1.
  * Concrete gating (softmax renormalised over the selected K, or sigmoid
  * normalised over the selected K), SwiGLU experts and the tile size come from
  * the layer definitions of the workloads (Mixtral-, Qwen2-MoE-,
@@ -79,18 +81,25 @@ int oracle_router_logits(int T, int H, int E, int dtype, const void* x,
 /* ------------------------------------------------------------------ top-K */
 /* K passes; each pass picks the not-yet-selected expert with the largest
  * logit, the lowest index winning a tie.  ids[t][0..K-1] in selection order. */
-int oracle_topk(int T, int E, int K, const float* logits, int32_t* ids)
+/* Per-token dynamic K (the MoE-Prism write-up: the routing top-k as a
+ * runtime control knob, per request): token t selects its k_t largest logits,
+ * 0 <= k_t <= K, in the same order; slots k >= k_t hold -1 (no assignment).
+ * k_per_token == NULL means k_t = K for every token. */
+int oracle_topk_k(int T, int E, int K, const int32_t* k_per_token, const float* logits, int32_t* ids)
 {
     if (T < 0 || E <= 0 || K <= 0 || K > E) return -1;
     char* taken = (char*)malloc((size_t)E);
     if (!taken) return -2;
     for (int t = 0; t < T; ++t) {
         const float* l = logits + (size_t)t * E;
+        int kt = k_per_token ? k_per_token[t] : K;
+        if (kt < 0 || kt > K) { free(taken); return -1; }
         for (int e = 0; e < E; ++e) {
             if (isnan(l[e])) { free(taken); return -1; }
             taken[e] = 0;
         }
-        for (int k = 0; k < K; ++k) {
+        for (int k = kt; k < K; ++k) ids[(size_t)t * K + k] = -1;
+        for (int k = 0; k < kt; ++k) {
             int best = -1;
             for (int e = 0; e < E; ++e) {
                 if (taken[e]) continue;
@@ -102,6 +111,11 @@ int oracle_topk(int T, int E, int K, const float* logits, int32_t* ids)
     }
     free(taken);
     return 0;
+}
+
+int oracle_topk(int T, int E, int K, const float* logits, int32_t* ids)
+{
+    return oracle_topk_k(T, E, K, NULL, logits, ids);
 }
 
 /* ---------------------------------------------------------------- weights */
@@ -119,21 +133,23 @@ int oracle_gate_weights(int T, int E, int K, int score_fn, int renorm,
         const float* l = logits + (size_t)t * E;
         const int32_t* id = ids + (size_t)t * K;
         double* wt = w + (size_t)t * K;
+        /* slots with id -1 (no assignment) get weight 0 and stay out of the sums */
+        for (int k = 0; k < K; ++k) if (id[k] >= E || id[k] < -1) return -1;
         if (score_fn == 0) {
             double m = -INFINITY, den = 0.0;
             if (renorm) {
-                for (int k = 0; k < K; ++k) if ((double)l[id[k]] > m) m = l[id[k]];
-                for (int k = 0; k < K; ++k) den += exp((double)l[id[k]] - m);
+                for (int k = 0; k < K; ++k) if (id[k] >= 0 && (double)l[id[k]] > m) m = l[id[k]];
+                for (int k = 0; k < K; ++k) if (id[k] >= 0) den += exp((double)l[id[k]] - m);
             } else {
                 for (int e = 0; e < E; ++e) if ((double)l[e] > m) m = l[e];
                 for (int e = 0; e < E; ++e) den += exp((double)l[e] - m);
             }
-            for (int k = 0; k < K; ++k) wt[k] = exp((double)l[id[k]] - m) / den;
+            for (int k = 0; k < K; ++k) wt[k] = id[k] >= 0 ? exp((double)l[id[k]] - m) / den : 0.0;
         } else {
             double den = 0.0;
-            for (int k = 0; k < K; ++k) den += sigmoid((double)l[id[k]]);
+            for (int k = 0; k < K; ++k) if (id[k] >= 0) den += sigmoid((double)l[id[k]]);
             for (int k = 0; k < K; ++k)
-                wt[k] = renorm ? sigmoid((double)l[id[k]]) / den : sigmoid((double)l[id[k]]);
+                wt[k] = id[k] < 0 ? 0.0 : (renorm ? sigmoid((double)l[id[k]]) / den : sigmoid((double)l[id[k]]));
         }
     }
     return 0;
@@ -162,6 +178,7 @@ int oracle_align(int T, int K, int E, int B, int mode, const int32_t* ids, int64
     int64_t A = (int64_t)T * K;
     for (int e = 0; e < E; ++e) counts[e] = 0;
     for (int64_t a = 0; a < A; ++a) {
+        if (ids[a] == -1) continue;  /* an empty slot (dynamic K): no assignment */
         if (ids[a] < 0 || ids[a] >= E) return -1;
         counts[ids[a]] += 1;
     }
@@ -181,6 +198,7 @@ int oracle_align(int T, int K, int E, int B, int mode, const int32_t* ids, int64
     for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
     for (int64_t a = 0; a < A; ++a) {
         int e = ids[a];
+        if (e < 0) { pos[a] = -1; continue; }
         sorted_ids[cursor[e]] = (int32_t)a;
         pos[a] = cursor[e];
         cursor[e] += 1;
@@ -223,8 +241,10 @@ int oracle_combine(int T, int H, int K, int dtype, const void* y, const int32_t*
     for (int t = 0; t < T; ++t)
         for (int h = 0; h < H; ++h) {
             double s = 0.0;
-            for (int k = 0; k < K; ++k)
-                s += w[(size_t)t * K + k] * ld(y, (size_t)pos[(size_t)t * K + k] * H + h, dtype);
+            for (int k = 0; k < K; ++k) {
+                int32_t p = pos[(size_t)t * K + k];
+                if (p >= 0) s += w[(size_t)t * K + k] * ld(y, (size_t)p * H + h, dtype);
+            }
             if (shared) s += ld(shared, (size_t)t * H + h, dtype);
             out[(size_t)t * H + h] = s;
         }
@@ -327,6 +347,7 @@ int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
                      int renorm, int dtype, const void* x, const void* w_r,
                      const void* const* w13, const void* const* w2,
                      const void* w13_sh, const void* w2_sh, const float* logits_in,
+                     const int32_t* k_per_token,
                      const int32_t* tokens, int n_tok, double* out,
                      int32_t* ids_out, double* w_out, int nthreads)
 {
@@ -366,7 +387,7 @@ int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
                         l[e] = (float)s;
                     }
                 }
-                if (oracle_topk(1, E, K, l, id) != 0 ||
+                if (oracle_topk_k(1, E, K, k_per_token ? k_per_token + t : NULL, l, id) != 0 ||
                     oracle_gate_weights(1, E, K, score_fn, renorm, l, id, w) != 0) {
 #pragma omp atomic write
                     err = -1;
@@ -376,6 +397,7 @@ int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
                 for (int h = 0; h < H; ++h) o[h] = 0.0;
                 for (int k = 0; k < K; ++k) {
                     int e = id[k];
+                    if (e < 0) continue;  /* empty slot */
                     if (!w13[e] || !w2[e]) {
 #pragma omp atomic write
                         err = -1;

@@ -523,3 +523,82 @@ def test_router_generator_is_near_uniform():
     counts = np.bincount(oracle.topk(lg, shape.K).ravel(), minlength=shape.E)
     expect = 256 * shape.K / shape.E
     assert np.all(np.abs(counts - expect) < 5 * math.sqrt(expect)), counts
+
+
+# --------------------------------------------------- per-token dynamic K
+
+def test_dynamic_k_topk_matches_bruteforce_prefix():
+    # token t takes the first k_t experts of the (logit desc, index asc) order;
+    # slots from k_t on are -1
+    rng = np.random.default_rng(21)
+    T, E, K = 40, 12, 5
+    lg = mi.tie_heavy_logits(T, E, 3, levels=4)
+    k = rng.integers(0, K + 1, size=T).astype(np.int32)
+    ids = oracle.topk(lg, K, k)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-float(lg[t, e]), e))
+        assert ids[t].tolist() == order[:k[t]] + [-1] * (K - k[t])
+
+
+def test_dynamic_k_equal_to_K_is_static_topk():
+    lg = np.random.default_rng(22).standard_normal((30, 16)).astype(np.float32)
+    assert np.array_equal(oracle.topk(lg, 4, np.full(30, 4, np.int32)), oracle.topk(lg, 4))
+
+
+@pytest.mark.parametrize("score_fn", [0, 1])
+def test_dynamic_k_gate_weights_closed_forms(score_fn):
+    # k_t = 1: the single weight is 1 (renormalised); k_t = 2 under softmax:
+    # the pair's weights are sigma(l1 - l2) and sigma(l2 - l1); empty slots 0
+    lg = np.array([[0.5, 2.0, -1.0, 1.0], [3.0, -2.0, 0.25, 1.5]], np.float32)
+    k = np.array([1, 2], np.int32)
+    ids = oracle.topk(lg, 3, k)
+    assert ids.tolist() == [[1, -1, -1], [0, 3, -1]]
+    w = oracle.gate_weights(lg, ids, score_fn=score_fn, renorm=1)
+    assert w[0].tolist() == [1.0, 0.0, 0.0] and w[1, 2] == 0.0
+    if score_fn == 0:
+        assert math.isclose(w[1, 0], 1 / (1 + math.exp(-1.5)), rel_tol=1e-15)
+        assert math.isclose(w[1, 1], 1 / (1 + math.exp(1.5)), rel_tol=1e-15)
+    else:
+        s0, s3 = 1 / (1 + math.exp(-3.0)), 1 / (1 + math.exp(-1.5))
+        assert math.isclose(w[1, 0], s0 / (s0 + s3), rel_tol=1e-15)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_dynamic_k_align_skips_empty_slots(mode):
+    rng = np.random.default_rng(23)
+    T, E, K, B = 33, 8, 4, 4
+    k = rng.integers(0, K + 1, size=T).astype(np.int32)
+    ids = oracle.topk(rng.standard_normal((T, E)).astype(np.float32), K, k)
+    r = oracle.align(ids, E, B, mode=mode)
+    real = ids.ravel() >= 0
+    assert np.array_equal(r["counts"], np.bincount(ids.ravel()[real], minlength=E))
+    assert np.all(r["pos"][~real] == -1)
+    sid = r["sorted_ids"]
+    assert np.array_equal(np.sort(sid[sid >= 0]), np.nonzero(real)[0])
+    for a in np.nonzero(real)[0]:
+        assert sid[r["pos"][a]] == a
+    n = r["counts"]
+    P = int(sum(-(-int(c) // B) * B for c in n)) if mode == 0 else E * (-(-int(n.max()) // B) * B)
+    assert r["P"] == P
+
+
+def test_dynamic_k_combine_skips_empty_slots():
+    y = np.array([[1.0, 2.0], [10.0, 20.0]], np.float32)
+    pos = np.array([[1, -1], [-1, -1]], np.int32)
+    out = oracle.combine(y, pos, np.array([[0.5, 0.0], [0.0, 0.0]]))
+    assert out.tolist() == [[5.0, 10.0], [0.0, 0.0]]
+
+
+def test_dynamic_k_layer_is_static_layer_per_token():
+    # each token with k_t equals the same token through the layer with K = k_t
+    # (k_t = 0: the shared FFN alone)
+    x, w_r, w13, w2, sh = _small_layer(24, T=9, E=6, K=3, I_sh=16)
+    k = np.array([3, 0, 1, 2, 3, 1, 0, 2, 2], np.int32)
+    out = oracle.moe_layer(x, w_r, w13, w2, K=3, k=k, **sh)
+    shared = oracle.dense_ffn(x, sh["w13_sh"], sh["w2_sh"])
+    for t in range(9):
+        if k[t] == 0:
+            assert np.allclose(out[t], shared[t], rtol=1e-14, atol=1e-15)
+        else:
+            ref = oracle.moe_layer(x, w_r, w13, w2, K=int(k[t]), tokens=np.array([t], np.int32), **sh)[0]
+            assert np.allclose(out[t], ref, rtol=1e-13, atol=1e-14)
