@@ -123,7 +123,7 @@ def parse_workload(s):
 
 
 class Workload:
-    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None, pad_mode=0):
+    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None, pad_mode=0, dyn_k=False):
         import mixture_experts_layer_61_b200 as moe
         self.moe = moe
         self.shape, self.T = shape, T
@@ -131,6 +131,14 @@ class Workload:
         self.w = weights if weights is not None else mi.make_weights(shape, seed, device=device)
         self.x = mi.make_x(shape, T, seed + 100 * rank, device=device)
         self.logits = None
+        # per-token dynamic K: each token's count drawn uniformly from 1..K (seeded)
+        self.k = None
+        self.A = T * shape.K
+        if dyn_k:
+            g = torch.Generator(device="cpu")
+            g.manual_seed(seed + 31)
+            self.k = torch.randint(1, shape.K + 1, (T,), generator=g, dtype=torch.int32).to(device)
+            self.A = int(self.k.sum().item())
         if skew is not None:
             self.logits = mi.zipf_gumbel_logits(shape.E, T, skew, seed=seed + 17 + 100 * rank, device=device)
         n_sh, I_s = (1, shape.I_sh) if shape.I_sh else (0, 0)
@@ -175,7 +183,7 @@ class Workload:
     def step(self):
         m = self.moe
         m.layer_forward(self.cfg, self.x, self.w["w_r"], self.w["w13"], self.w["w2"], self.ws,
-                        self.w.get("w13_sh"), self.w.get("w2_sh"), self.logits, self.out, self.stats)
+                        self.w.get("w13_sh"), self.w.get("w2_sh"), self.logits, self.out, self.stats, k=self.k)
 
     def staged_step(self, ev):
         """The same kernels as step(), one ABI call per stage, events in between."""
@@ -183,7 +191,7 @@ class Workload:
         ev[0].record()
         m.router_gemm(c, self.x, self.w["w_r"], self.gws, self.s_logits)
         ev[1].record()
-        m.route(c, self.logits if self.logits is not None else self.s_logits, self.s_ids, self.s_w)
+        m.route(c, self.logits if self.logits is not None else self.s_logits, self.s_ids, self.s_w, k=self.k)
         ev[2].record()
         self.al = m.align_pad(c, self.s_ids, self.s_al)
         ev[3].record()
@@ -250,29 +258,33 @@ def replica_tokens_per_s(world, T, steps, max_total_ms):
 
 # ------------------------------------------------------------ accounting
 
-def algorithmic(shape, T, E_active):
+def algorithmic(shape, T, E_active, A=None):
     """Algorithmic bytes and flops of one layer forward (padding excluded):
     bytes = weights of the activated experts + shared weights + router weights,
-    flops = 2 T (H E + K 3 H I + 3 H I_sh)."""
+    flops = 2 T (H E + 3 H I_sh) + 2 A 3 H I with A = T K assignments (or
+    the sum of the per-token counts under dynamic K)."""
     eb = 2 if shape.dtype == "bf16" else 4
     H, I, E, K = shape.H, shape.I, shape.E, shape.K
+    A = T * K if A is None else A
     B = E_active * 3 * H * I * eb + 3 * H * shape.I_sh * eb + E * H * eb
-    F = 2.0 * T * (H * E + K * 3 * H * I + 3 * H * shape.I_sh)
+    F = 2.0 * T * (H * E + 3 * H * shape.I_sh) + 2.0 * A * 3 * H * I
     return B, F
 
 
-def gate_up_work(shape, T, E_active):
+def gate_up_work(shape, T, E_active, A=None):
     """Dominant kernel (grouped gate/up + SwiGLU): weight bytes of the activated
-    experts' W1/W3, flops 2 * T K * H * 2I."""
+    experts' W1/W3, flops 2 * A * H * 2I (A = T K assignments)."""
     eb = 2 if shape.dtype == "bf16" else 4
-    return E_active * 2 * shape.I * shape.H * eb, 2.0 * T * shape.K * shape.H * 2 * shape.I
+    A = T * shape.K if A is None else A
+    return E_active * 2 * shape.I * shape.H * eb, 2.0 * A * shape.H * 2 * shape.I
 
 
-def ffn_work(shape, T, E_active):
+def ffn_work(shape, T, E_active, A=None):
     """Fused expert FFN: weight bytes of the activated experts' W1/W3/W2,
-    flops 2 * T K * 3 * H * I."""
+    flops 2 * A * 3 * H * I (A = T K assignments)."""
     eb = 2 if shape.dtype == "bf16" else 4
-    return E_active * 3 * shape.I * shape.H * eb, 2.0 * T * shape.K * 3 * shape.H * shape.I
+    A = T * shape.K if A is None else A
+    return E_active * 3 * shape.I * shape.H * eb, 2.0 * A * 3 * shape.H * shape.I
 
 
 def dense_times(shape, T, I_d, steps, warmup, flush, device, seed):
@@ -355,6 +367,8 @@ def main():
     ap.add_argument("--no-pdl", action="store_true", help="plain stream order between kernels")
     ap.add_argument("--pad-mode", type=int, default=0, choices=[0, 1],
                     help="alignment padding: 0 block-wise, 1 max-value")
+    ap.add_argument("--dynamic-k", action="store_true",
+                    help="per-token dynamic K: each token's expert count uniform in 1..K (seeded)")
     ap.add_argument("--padding-model", action="store_true",
                     help="time the expert FFN over routings and fit the padding and max-affine latency models")
     ap.add_argument("--shared-sms", type=int, default=0,
@@ -394,7 +408,7 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return
-    wl = Workload(shape, T, rank, device, skew=args.skew, pad_mode=args.pad_mode)
+    wl = Workload(shape, T, rank, device, skew=args.skew, pad_mode=args.pad_mode, dyn_k=args.dynamic_k)
     if args.no_graph:
         run_step, wl.launches_per_step = wl.step, None
     else:
@@ -445,7 +459,8 @@ def main():
                               "quick": True, "config": {"workload": f"{shape.name}:{T}",
                                                         "token_tile_cap": args.token_tile_cap,
                                                         "pdl": not args.no_pdl,
-                                                        "shared_sms": moe.shared_sms(wl.cfg)},
+                                                        "shared_sms": moe.shared_sms(wl.cfg),
+                                                        "pad_mode": args.pad_mode, "dynamic_k": args.dynamic_k},
                               "stages_ms": stages, "E_active": E_active, "P": P}), flush=True)
         if dist:
             dist.barrier()
@@ -455,10 +470,10 @@ def main():
     # ---- roofline of the dominant kernel: the grouped gate/up + SwiGLU GEMM,
     # or the fused expert FFN when the layer runs it as one launch
     if wl.fused:
-        gu_bytes, gu_flops = ffn_work(shape, T, E_active)
+        gu_bytes, gu_flops = ffn_work(shape, T, E_active, wl.A)
         t_gu = stages["ffn"] * 1e-3
     else:
-        gu_bytes, gu_flops = gate_up_work(shape, T, E_active)
+        gu_bytes, gu_flops = gate_up_work(shape, T, E_active, wl.A)
         t_gu = stages["gate_up"] * 1e-3
     hbm_peak = pk["hbm_gbs"]
     tc_peak = pk["bf16_tflops"] * (0.5 if shape.dtype == "fp32" else 1.0)  # tf32 is half the bf16 rate
@@ -475,7 +490,7 @@ def main():
                       else "moe_gemm_kernel (grouped gate/up + SwiGLU)")
     roof["peak_source"] = f"{pk_kind} ({'MEASURED_PEAKS.json' if pk_kind == 'measured' else 'fallback'})"
     roof["traffic"] = NCU_TRAFFIC.get(f"{shape.name}:{T}")
-    B_alg, F_alg = algorithmic(shape, T, E_active)
+    B_alg, F_alg = algorithmic(shape, T, E_active, wl.A)
     t_layer = ms_step * 1e-3
     layer_roof = max(F_alg / (tc_peak * 1e12), B_alg / (hbm_peak * 1e9)) / t_layer
 
@@ -540,9 +555,11 @@ def main():
                    "launch": "host launches" if args.no_graph else "CUDA graph replay of moe_layer_forward",
                    "l2": "flushed between steps (2 GiB write outside the events); weights exceed L2",
                    "shared_sms": moe.shared_sms(wl.cfg),
-                   "padding": "max-value" if args.pad_mode == 1 else "block-wise"},
+                   "padding": "max-value" if args.pad_mode == 1 else "block-wise",
+                   "top_k": (f"per-token dynamic, uniform 1..{shape.K} (sum {wl.A})" if args.dynamic_k
+                             else f"{shape.K} for every token")},
         "roofline": roof,
-        "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - T * shape.K) / max(P, 1), 4),
+        "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - wl.A) / max(P, 1), 4),
                   "bytes_alg": B_alg, "flops_alg": F_alg, "roofline_frac": round(layer_roof, 4),
                   "hbm_GBs_alg": round(B_alg / t_layer / 1e9, 1), "tflops_alg": round(F_alg / t_layer / 1e12, 2)},
         "stages_ms": stages,

@@ -145,16 +145,29 @@ int moe_router_gemm_noalloc(const moe_config_t* cfg, const void* x, const void* 
 int moe_route(const moe_config_t* cfg, const float* logits, int32_t* topk_ids,
               float* topk_w, moe_stream_t stream);
 
-/* Token-to-expert alignment with block-wise padding (stage "alignment",
- * Section 5.1 padding model).  With e(a) = topk_ids[a]:
+/* Per-token dynamic K (the routing top-k as a per-request runtime knob: the
+ * MoE-Prism write-up).  As moe_route, with token t selecting its
+ * k_per_token[t] largest logits (device int32 [T]; values clamped to
+ * [0, cfg->K]); slots k >= k_per_token[t] get id -1 and weight 0, and the
+ * weights are renormalised over the k_per_token[t] selected.  NULL: K for
+ * every token (= moe_route).  The alignment treats id -1 as an empty slot
+ * (no row, pos -1, not flagged) and the combine skips it. */
+int moe_route_k(const moe_config_t* cfg, const float* logits, const int32_t* k_per_token,
+                int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/* Token-to-expert alignment (stage "alignment", Section 5.1 padding model).
+ * With e(a) = topk_ids[a]:
  *   counts[E]        N_e = #{a : e(a) = e}
- *   offsets[E+1]     exclusive scan of ceil(N_e / B) * B; offsets[E] = P
+ *   offsets[E+1]     exclusive scan of the padded counts; offsets[E] = P.
+ *                    cfg->pad_mode 0 (block-wise): ceil(N_e / B) * B;
+ *                    1 (max-value): ceil(max_i N_i / B) * B for every expert
  *   sorted_ids[P_max] the assignments of expert e in ascending a at
  *                    offsets[e] .. offsets[e] + N_e - 1; every other slot -1
  *   block_expert[ceil(P_max/B)]  e for blocks inside expert e's segment, -1 after P
- *   pos[A]           the slot p with sorted_ids[p] = a
+ *   pos[A]           the slot p with sorted_ids[p] = a (-1 for an empty slot)
  *   scalars[4]       {P, E_active = #{e : N_e > 0}, 0, 0}
- * Bit-exact and deterministic.  Out-of-range ids are skipped and flagged in
+ * Bit-exact and deterministic.  Id -1 is an empty slot (per-token dynamic K):
+ * no row, pos -1.  Other out-of-range ids are skipped and flagged in
  * scalars[2] (nonzero = bad input). */
 int moe_align_pad(const moe_config_t* cfg, const int32_t* topk_ids, int32_t* counts,
                   int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert,
@@ -208,6 +221,15 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
                       const void* w2_shared, const float* logits_override, void* out,
                       void* workspace, size_t ws_bytes, int32_t* stats_out,
                       moe_stream_t stream);
+
+/* moe_layer_forward with per-token dynamic K (see moe_route_k): token t is
+ * routed to its k_per_token[t] top experts (0 = shared experts only);
+ * NULL = K for every token.  Same workspace. */
+int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_router,
+                        const void* w13, const void* w2, const void* w13_shared,
+                        const void* w2_shared, const float* logits_override,
+                        const int32_t* k_per_token, void* out, void* workspace,
+                        size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
 
 /* Bytes of workspace dense_ffn needs for T tokens of width I (0 if invalid). */
 size_t dense_ffn_workspace_size(int T, int H, int I, int dtype);

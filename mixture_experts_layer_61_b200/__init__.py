@@ -67,6 +67,7 @@ def lib():
             "moe_gemm_workspace_size": (S, []),
             "moe_router_gemm": (I, [C, P, P, P, P, S, P]),
             "moe_route": (I, [C, P, P, P, P]),
+            "moe_route_k": (I, [C, P, P, P, P, P]),
             "moe_align_pad": (I, [C, P, P, P, P, P, P, P, P]),
             "moe_permute": (I, [C, P, P, P, P, P]),
             "moe_grouped_ffn": (I, [C, P, P, P, P, P, P, P, S, P]),
@@ -74,6 +75,7 @@ def lib():
             "moe_grouped_down": (I, [C, P, P, P, P, P, S, P]),
             "moe_combine": (I, [C, P, P, P, P, P, P]),
             "moe_layer_forward": (I, [C, P, P, P, P, P, P, P, P, P, S, P, P]),
+            "moe_layer_forward_k": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P, P]),
             "dense_ffn_workspace_size": (S, [I, I, I, I]),
             "dense_ffn": (I, [I, I, I, I, P, P, P, P, P, S, P]),
             "moe_check_status": (I, [P, P]),
@@ -164,12 +166,14 @@ def router_gemm(cfg, x, w_r, ws, logits=None):
     return logits
 
 
-def route(cfg, logits, ids=None, w=None):
-    _need_cuda(logits)
+def route(cfg, logits, ids=None, w=None, k=None):
+    """Top-K ids and gate weights; k (device int32 [T], optional) gives each
+    token its own expert count (per-token dynamic K, empty slots -1)."""
+    _need_cuda(logits, k)
     if ids is None:
         ids = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device=logits.device)
         w = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device=logits.device)
-    _check(lib().moe_route(ctypes.byref(cfg), _p(logits), _p(ids), _p(w), _stream()), "moe_route")
+    _check(lib().moe_route_k(ctypes.byref(cfg), _p(logits), _p(k), _p(ids), _p(w), _stream()), "moe_route_k")
     return ids, w
 
 
@@ -246,13 +250,15 @@ def combine(cfg, y_perm, pos, w, shared_out=None, out=None):
 
 
 def layer_forward(cfg, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, logits_override=None, out=None,
-                  stats=None):
-    _need_cuda(x, w_r, w13, w2, ws, w13_sh, w2_sh, logits_override, stats)
+                  stats=None, k=None):
+    """The whole layer; k (device int32 [T], optional): per-token dynamic K."""
+    _need_cuda(x, w_r, w13, w2, ws, w13_sh, w2_sh, logits_override, stats, k)
     if out is None:
         out = torch.empty((cfg.T, cfg.H), dtype=x.dtype, device=x.device)
-    _check(lib().moe_layer_forward(ctypes.byref(cfg), _p(x), _p(w_r), _p(w13), _p(w2), _p(w13_sh), _p(w2_sh),
-                                   _p(logits_override), _p(out), _p(ws), ws.numel(), _p(stats), _stream()),
-           "moe_layer_forward")
+    _check(lib().moe_layer_forward_k(ctypes.byref(cfg), _p(x), _p(w_r), _p(w13), _p(w2), _p(w13_sh), _p(w2_sh),
+                                     _p(logits_override), _p(k), _p(out), _p(ws), ws.numel(), _p(stats),
+                                     _stream()),
+           "moe_layer_forward_k")
     return out
 
 

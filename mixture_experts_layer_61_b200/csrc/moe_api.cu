@@ -387,15 +387,20 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
     return status_of(launch_gemm(g, gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream));
 }
 
-int moe_route(const moe_config_t* cfg, const float* logits, int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
+int moe_route_k(const moe_config_t* cfg, const float* logits, const int32_t* k_per_token, int32_t* topk_ids,
+                float* topk_w, moe_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->T == 0) return MOE_OK;
     if (!logits || !topk_ids || !topk_w) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
-    return status_of(launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, logits, topk_ids, topk_w,
-                                 (cudaStream_t)stream));
+    return status_of(launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, logits, k_per_token, topk_ids,
+                                 topk_w, (cudaStream_t)stream));
+}
+
+int moe_route(const moe_config_t* cfg, const float* logits, int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
+    return moe_route_k(cfg, logits, nullptr, topk_ids, topk_w, stream);
 }
 
 int moe_align_pad(const moe_config_t* cfg, const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
@@ -484,6 +489,14 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* pos,
 int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13, const void* w2,
                       const void* w13_shared, const void* w2_shared, const float* logits_override, void* out,
                       void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
+    return moe_layer_forward_k(cfg, x, w_router, w13, w2, w13_shared, w2_shared, logits_override, nullptr, out,
+                               workspace, ws_bytes, stats_out, stream);
+}
+
+int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
+                        const void* w2, const void* w13_shared, const void* w2_shared, const float* logits_override,
+                        const int32_t* k_per_token, void* out, void* workspace, size_t ws_bytes, int32_t* stats_out,
+                        moe_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->T == 0) return MOE_OK;
@@ -569,7 +582,8 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
         int* route_ctr = reinterpret_cast<int*>(at<uint8_t>(workspace, L.ctl)) + 16;  // in the control header
         if ((rc = launch_route_small(cfg->T, cfg->H, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, cfg->tile_B,
                                      cfg->pad_mode, P,
-                                     cfg->dtype, x, w_router, logits_override, at<float>(workspace, L.route_part),
+                                     cfg->dtype, x, w_router, logits_override, k_per_token,
+                                     at<float>(workspace, L.route_part),
                                      logits, ids, w, counts, offsets, sorted_ids, block_expert, pos, scalars,
                                      stats_out, route_ctr, s)) != 0)
             return status_of(rc);
@@ -591,7 +605,7 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
         g.sms = n_routed;
         if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
         if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm,
-                              logits_override ? logits_override : logits, ids, w, s)) != 0)
+                              logits_override ? logits_override : logits, k_per_token, ids, w, s)) != 0)
             return status_of(rc);
         if ((rc = launch_align(cfg->T, cfg->K, cfg->E, cfg->tile_B, cfg->pad_mode, P, ids, counts, offsets,
                                sorted_ids, block_expert,

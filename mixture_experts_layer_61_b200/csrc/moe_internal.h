@@ -135,8 +135,10 @@ void set_token_tile_cap(int n);
 void set_cta_pairs(bool on);
 
 // Elementwise / routing kernels.
-int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,
-                cudaStream_t stream);
+// k_per_token (nullable): per-token expert count, clamped to [0, K]; slots
+// from it on get id -1 and weight 0.
+int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, const int32_t* k_per_token,
+                int32_t* ids, float* w, cudaStream_t stream);
 // mode 0: block-wise padding, 1: max-value padding (every expert padded to the
 // most loaded one's rounded count).
 int launch_align(int T, int K, int E, int B, int mode, long long P_max, const int32_t* ids, int32_t* counts,
@@ -146,11 +148,10 @@ int launch_align(int T, int K, int E, int B, int mode, long long P_max, const in
 constexpr int kSmallRouteMaxT = 64;
 // `part` holds (H/256 + 1) * T * E floats of partial router sums.
 int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
-                       int dtype,
-                       const void* x, const void* w_r, const float* logits_override, float* part, float* logits,
-                       int32_t* ids, float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
-                       int32_t* block_expert, int32_t* pos, int32_t* scalars, int32_t* stats_copy, int* done_ctr,
-                       cudaStream_t stream);
+                       int dtype, const void* x, const void* w_r, const float* logits_override,
+                       const int32_t* k_per_token, float* part, float* logits, int32_t* ids, float* w,
+                       int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos,
+                       int32_t* scalars, int32_t* stats_copy, int* done_ctr, cudaStream_t stream);
 int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
                    const int32_t* scalars, void* x_perm, cudaStream_t stream);
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,

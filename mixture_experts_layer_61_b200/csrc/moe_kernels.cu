@@ -26,16 +26,19 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
     return v > bv || (v == bv && i < bi);
 }
 
-// One warp per token.  Lane l owns experts l, l+32, ...; K passes of a warp
-// arg-max over the experts not yet taken.  Logits are read through L2 (they
-// may have been written by other blocks of the same kernel).
-__device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int E, int K, int score_fn, int renorm,
-                                               int32_t* __restrict__ ids_t, float* __restrict__ w_t, int lane) {
+// One warp per token.  Lane l owns experts l, l+32, ...; kt passes of a warp
+// arg-max over the experts not yet taken (kt = K, or the token's own count
+// 0..K under per-token dynamic K; slots kt..K-1 get id -1 and weight 0).
+// Logits are read through L2 (they may have been written by other blocks of
+// the same kernel).
+__device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int E, int K, int kt, int score_fn,
+                                               int renorm, int32_t* __restrict__ ids_t, float* __restrict__ w_t,
+                                               int lane) {
     uint32_t taken = 0;  // bit j: expert lane + 32 j
     float sel_v[16];
     int sel_i[16];
 #pragma unroll 1
-    for (int k = 0; k < K; ++k) {
+    for (int k = 0; k < kt; ++k) {
         float bv = -INFINITY;
         int bi = INT_MAX;
         for (int j = 0, e = lane; e < E; ++j, e += 32) {
@@ -78,9 +81,9 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int 
     if (score_fn == 0) {
         float m, den = 0.f;
         if (renorm) {
-            m = sel_v[0];
-            for (int k = 1; k < K; ++k) m = fmaxf(m, sel_v[k]);
-            for (int k = 0; k < K; ++k) den += expf(sel_v[k] - m);
+            m = kt > 0 ? sel_v[0] : 0.f;
+            for (int k = 1; k < kt; ++k) m = fmaxf(m, sel_v[k]);
+            for (int k = 0; k < kt; ++k) den += expf(sel_v[k] - m);
         } else {
             m = -INFINITY;
             for (int e = lane; e < E; e += 32) m = fmaxf(m, __ldcg(l + e));
@@ -92,44 +95,53 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int 
             for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
             den = part;
         }
-        for (int k = 0; k < K; ++k)
+        for (int k = 0; k < kt; ++k)
             if (k == lane) wk = expf(sel_v[k] - m) / den;
     } else {
         float den = 0.f;
-        for (int k = 0; k < K; ++k) den += 1.f / (1.f + expf(-sel_v[k]));
-        for (int k = 0; k < K; ++k)
+        for (int k = 0; k < kt; ++k) den += 1.f / (1.f + expf(-sel_v[k]));
+        for (int k = 0; k < kt; ++k)
             if (k == lane) {
                 const float s = 1.f / (1.f + expf(-sel_v[k]));
                 wk = renorm ? s / den : s;
             }
     }
     if (lane < K) {
-        int id = 0;
-        for (int k = 0; k < K; ++k)
+        int id = -1;
+        for (int k = 0; k < kt; ++k)
             if (k == lane) id = sel_i[k];
         ids_t[lane] = id;
         w_t[lane] = wk;
     }
 }
 
+// The token's expert count: K, or k_per_token[t] clamped to [0, K].
+__device__ __forceinline__ int token_k(const int32_t* __restrict__ k_per_token, int t, int K) {
+    if (!k_per_token) return K;
+    const int k = __ldg(k_per_token + t);
+    return k < 0 ? 0 : (k > K ? K : k);
+}
+
 __global__ void __launch_bounds__(256) topk_gate_kernel(int T, int E, int K, int score_fn, int renorm,
-                                                        const float* __restrict__ logits, int32_t* __restrict__ ids,
-                                                        float* __restrict__ w) {
+                                                        const float* __restrict__ logits,
+                                                        const int32_t* __restrict__ k_per_token,
+                                                        int32_t* __restrict__ ids, float* __restrict__ w) {
     pdl_launch_dependents();
     pdl_wait();
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
-    topk_one_token(logits + (size_t)t * E, E, K, score_fn, renorm, ids + (size_t)t * K, w + (size_t)t * K, lane);
+    topk_one_token(logits + (size_t)t * E, E, K, token_k(k_per_token, t, K), score_fn, renorm, ids + (size_t)t * K,
+                   w + (size_t)t * K, lane);
 }
 
-int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, int32_t* ids, float* w,
-                cudaStream_t stream) {
+int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logits, const int32_t* k_per_token,
+                int32_t* ids, float* w, cudaStream_t stream) {
     if (T == 0) return 0;
     const int warps_per_block = 8;
     const int blocks = (T + warps_per_block - 1) / warps_per_block;
     cudaError_t e = launch_kernel(topk_gate_kernel, dim3(blocks), dim3(warps_per_block * 32), 0, stream, T, E, K,
-                                  score_fn, renorm, logits, ids, w);
+                                  score_fn, renorm, logits, k_per_token, ids, w);
     count_launch();
     return launched(e);
 }
@@ -196,7 +208,7 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     for (long long a = tid; a < A; a += kAlignThreads) {
         const int e = ids[a];
         if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[e], 1);
-        else atomicOr(bad, 1);
+        else if (e != -1) atomicOr(bad, 1);  // -1: an empty slot (per-token dynamic K)
     }
     __syncthreads();
 
@@ -262,6 +274,8 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
             const int p = cursor[e] + tbl[warp * E + e] + rank;
             sorted_ids[p] = (int32_t)a;
             pos[a] = p;
+        } else if (a < A) {
+            pos[a] = -1;  // empty slot (or an out-of-range id, flagged above)
         }
         __syncthreads();
         if (tid < E) cursor[tid] += rt[tid];
@@ -335,7 +349,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     route_small_kernel(int T_, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
                        int nslices,
                        int slice_w, const T* __restrict__ x, const T* __restrict__ w_r,
-                       const float* __restrict__ logits_override, float* __restrict__ part, float* __restrict__ logits,
+                       const float* __restrict__ logits_override, const int32_t* __restrict__ k_per_token,
+                       float* __restrict__ part, float* __restrict__ logits,
                        int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ counts,
                        int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
                        int32_t* __restrict__ block_expert, int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
@@ -395,7 +410,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     __syncthreads();
     const float* src = logits_override ? logits_override : logits;
     for (int t = warp; t < T_; t += kAlignThreads / 32)
-        topk_one_token(src + (size_t)t * E, E, K, score_fn, renorm, ids + (size_t)t * K, w + (size_t)t * K, lane);
+        topk_one_token(src + (size_t)t * E, E, K, token_k(k_per_token, t, K), score_fn, renorm, ids + (size_t)t * K,
+                       w + (size_t)t * K, lane);
     __syncthreads();
     align_block(T_, K, E, B, mode, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy,
                 sm);
@@ -418,10 +434,10 @@ void route_small_slices(int T, int H, int E, int num_sms, int* nslices, int* sli
 
 int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
                        int dtype,
-                       const void* x, const void* w_r, const float* logits_override, float* part, float* logits,
-                       int32_t* ids, float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
-                       int32_t* block_expert, int32_t* pos, int32_t* scalars, int32_t* stats_copy, int* done_ctr,
-                       cudaStream_t stream) {
+                       const void* x, const void* w_r, const float* logits_override, const int32_t* k_per_token,
+                       float* part, float* logits, int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                       int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
+                       int32_t* stats_copy, int* done_ctr, cudaStream_t stream) {
     DeviceInfo d;
     int rc = current_device(&d);
     if (rc != 0) return rc;
@@ -445,12 +461,14 @@ int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int
     if (dtype == 0)
         e = launch_kernel(route_small_kernel<__nv_bfloat16>, dim3(blocks), dim3(kAlignThreads), smem, stream, T, H, E,
                           K, score_fn, renorm, B, mode, P_max, ns, sw, static_cast<const __nv_bfloat16*>(x),
-                          static_cast<const __nv_bfloat16*>(w_r), logits_override, part, logits, ids, w, counts,
+                          static_cast<const __nv_bfloat16*>(w_r), logits_override, k_per_token, part, logits, ids, w,
+                          counts,
                           offsets, sorted_ids, block_expert, pos, scalars, stats_copy, done_ctr);
     else
         e = launch_kernel(route_small_kernel<float>, dim3(blocks), dim3(kAlignThreads), smem, stream, T, H, E, K,
                           score_fn, renorm, B, mode, P_max, ns, sw, static_cast<const float*>(x),
-                          static_cast<const float*>(w_r), logits_override, part, logits, ids, w, counts, offsets,
+                          static_cast<const float*>(w_r), logits_override, k_per_token, part, logits, ids, w, counts,
+                          offsets,
                           sorted_ids, block_expert, pos, scalars, stats_copy, done_ctr);
     count_launch();
     return launched(e);
@@ -573,6 +591,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K
 #pragma unroll
             for (int i = 0; i < N; ++i) acc[i] = 0.f;
             for (int k = 0; k < K; ++k) {
+                if (s_pos[k] < 0) continue;  // empty slot (per-token dynamic K)
                 float y[N];
                 unpack(__ldg(y_perm + (long long)s_pos[k] * row_vec + v), y, (const T*)nullptr);
                 const float wk = s_w[k];

@@ -57,6 +57,17 @@ def test_align_max_value_bit_exact(T, E, K, B, kind):
     _check_align(T, E, K, B, _ids(T, E, K, seed=T + E + B + 1, kind=kind), mode=1)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("T,E,K,B", [(64, 8, 2, 16), (300, 64, 8, 16), (1000, 256, 8, 16), (40, 16, 4, 4)])
+def test_align_dynamic_k_empty_slots(mode, T, E, K, B):
+    # ids -1 (per-token dynamic K) are empty slots: no row, pos -1, not flagged
+    rng = np.random.default_rng(T + E)
+    k = rng.integers(0, K + 1, size=T).astype(np.int32)
+    ids_np = oracle.topk(mi.zipf_gumbel_logits(E, T, 0.5, T + 1).numpy(), K, k)
+    g, r = _check_align(T, E, K, B, ids_np, mode=mode)
+    assert np.all(g["pos"].cpu().numpy()[ids_np.ravel() < 0] == -1)
+
+
 def test_align_empty():
     cfg = moe.config(0, 64, 8, 2, 64)
     ids = torch.empty((0, 2), dtype=torch.int32, device="cuda")

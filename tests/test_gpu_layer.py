@@ -22,14 +22,15 @@ pytestmark = pytest.mark.gpu
 N_SAMPLE = int(os.environ.get("MOE_TEST_SAMPLE", "256"))
 
 
-def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True, pad_mode=0):
+def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True, pad_mode=0, k=None):
     w = mi.make_weights(shape, seed, device="cuda")
     x = mi.make_x(shape, T, seed, device="cuda")
     cfg = cfg_for(shape, T, pad_mode=pad_mode)
     ws = moe.alloc_workspace(moe.workspace_size(cfg))
     stats = torch.zeros(4, dtype=torch.int32, device="cuda")
+    kt = None if k is None else torch.from_numpy(np.asarray(k, np.int32)).cuda()
     out = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w.get("w13_sh"), w.get("w2_sh"),
-                            logits_override=override, stats=stats)
+                            logits_override=override, stats=stats, k=kt)
     moe.check_status(ws)
     # the logits the layer computed (checked against the oracle's below)
     layer_lg = moe.layer_logits(cfg, ws).cpu().numpy()
@@ -37,7 +38,7 @@ def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True, p
     tol = 4e-3 if shape.dtype == "fp32" and T > 64 else 1e-5
     assert np.abs(layer_lg[:min(T, 64)] - ref_lg).max() / np.abs(ref_lg).max() < tol
     lg = layer_lg if override is None else override.cpu().numpy()
-    ids = oracle.topk(lg, shape.K)
+    ids = oracle.topk(lg, shape.K, k)
     if check_stats:
         r = oracle.align(ids, shape.E, shape.tile_B, mode=pad_mode)
         st = stats.cpu().numpy()
@@ -47,7 +48,7 @@ def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True, p
     if shape.I_sh:
         sh = dict(w13_sh=host(w["w13_sh"]), w2_sh=host(w["w2_sh"]))
     ref = oracle.moe_layer(host(x), None, host(w["w13"]), host(w["w2"]), shape.K, shape.score_fn,
-                           shape.renorm, logits=lg, tokens=tok, **sh)
+                           shape.renorm, logits=lg, tokens=tok, k=k, **sh)
     return rel_err(out.float().cpu().numpy()[tok], ref)
 
 
@@ -150,3 +151,19 @@ def test_layer_max_value_padding(T):
 def test_layer_max_value_padding_deepseek_decode():
     shape = mi.SHAPES["deepseekv3"]
     assert _run_layer(shape, 32, seed=mi.seed_for(shape, 32), n_sample=64, pad_mode=1) < OUT_TOL
+
+
+@pytest.mark.parametrize("T,pad_mode", [(7, 0), (48, 0), (300, 0), (48, 1)])
+def test_layer_dynamic_k(T, pad_mode):
+    # per-token dynamic K (0..K experts per token; 0 = shared experts only)
+    shape = small_shape(H=512, E=16, K=4, I=384, I_sh=256)
+    k = np.random.default_rng(T).integers(0, shape.K + 1, size=T).astype(np.int32)
+    k[0] = 0
+    assert _run_layer(shape, T, seed=T + 70, pad_mode=pad_mode, k=k) < OUT_TOL
+
+
+def test_layer_dynamic_k_qwen_full_size():
+    shape = mi.SHAPES["qwen2moe"]
+    T = 128
+    k = np.random.default_rng(11).integers(1, shape.K + 1, size=T).astype(np.int32)
+    assert _run_layer(shape, T, seed=mi.seed_for(shape, T, 9), n_sample=64, k=k) < OUT_TOL

@@ -91,3 +91,34 @@ def test_router_logits(dtype, H, E, T):
     err = np.abs(lg.cpu().numpy() - ref).max() / np.abs(ref).max()
     # bf16 inputs: exact products, fp32 sums; fp32 inputs run as tf32 products
     assert err < (1e-5 if dtype == "bf16" else 4e-3), err
+
+
+@pytest.mark.parametrize("E,K", [(8, 2), (64, 8), (256, 8), (1024, 16), (5, 5)])
+def test_dynamic_k_topk_bit_exact(E, K):
+    # per-token dynamic K: token t takes its k[t] top experts (0..K), empty
+    # slots -1 with weight 0, weights renormalised over the selected
+    T = 300
+    rng = np.random.default_rng(E + K)
+    lg = mi.tie_heavy_logits(T, E, seed=E * 3 + K, levels=3)
+    k = rng.integers(0, K + 1, size=T).astype(np.int32)
+    ref = oracle.topk(lg, K, k)
+    kt = torch.from_numpy(k).cuda()
+    for score_fn in (0, 1):
+        for renorm in (0, 1):
+            cfg = moe.config(T, 64, E, K, 64, score_fn=score_fn, renorm=renorm)
+            ids, w = moe.route(cfg, torch.from_numpy(lg).cuda(), k=kt)
+            torch.cuda.synchronize()
+            assert np.array_equal(ids.cpu().numpy(), ref)
+            wr = oracle.gate_weights(lg, ref, score_fn, renorm)
+            assert np.allclose(w.cpu().numpy(), wr, rtol=2e-6, atol=1e-7)
+
+
+def test_dynamic_k_is_clamped():
+    # counts outside [0, K] act as the nearest bound
+    T, E, K = 6, 8, 3
+    lg = np.random.default_rng(5).standard_normal((T, E)).astype(np.float32)
+    k = np.array([-4, 0, 1, 3, 7, 100], np.int32)
+    cfg = moe.config(T, 64, E, K, 64)
+    ids, _ = moe.route(cfg, torch.from_numpy(lg).cuda(), k=torch.from_numpy(k).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(ids.cpu().numpy(), oracle.topk(lg, K, np.clip(k, 0, K)))
