@@ -55,6 +55,15 @@ def lib():
         L.oracle_combine.argtypes = [i, i, i, i, P, P, P, P, P]
         L.oracle_dense_ffn.argtypes = [i, i, i, i, P, P, P, P, i]
         L.oracle_moe_layer.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, i, P, P, P, i]
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_quantize_fp8.argtypes = [i, i, i, P, P, P]
+        L.oracle_quantize_fp8.restype = ctypes.c_int
+        L.oracle_moe_layer_fp8.argtypes = [i, i, i, i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P, P, i,
+                                           P, i]
+        L.oracle_moe_layer_fp8.restype = ctypes.c_int
         for f in (L.oracle_router_logits, L.oracle_topk, L.oracle_gate_weights, L.oracle_align,
                   L.oracle_swiglu_ffn, L.oracle_dense_ffn, L.oracle_moe_layer, L.oracle_permute,
                   L.oracle_combine):
@@ -269,4 +278,73 @@ def moe_layer(x, w_r, w13, w2, K, score_fn=0, renorm=1, w13_sh=None, w2_sh=None,
     _check(rc, "moe_layer")
     if return_routing:
         return out, ids, w
+    return out
+
+
+# ------------------------------------------------------------- FP8 weights
+
+def e4m3_value(codes):
+    """Values (float64) of E4M3 codes (uint8 array), from the format definition."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib().oracle_e4m3_value(c) for c in range(256)], np.float64)
+    return table[codes]
+
+
+def e4m3_encode(v):
+    """Nearest E4M3 codes (ties to even, saturating at +-448) of fp32 values."""
+    v = np.asarray(v, dtype=np.float32)
+    f = lib().oracle_e4m3_encode
+    return np.array([f(float(a)) for a in v.ravel()], np.uint8).reshape(v.shape)
+
+
+def quantize_fp8(w):
+    """Row-wise FP8 quantisation of a 2-D weight matrix (bf16 as uint16 bit
+    patterns, or fp32): returns (codes uint8 [rows, cols], scales fp32 [rows])."""
+    w, dt = _typed(w)
+    rows, cols = w.shape
+    q = np.empty((rows, cols), np.uint8)
+    sc = np.empty(rows, np.float32)
+    _check(lib().oracle_quantize_fp8(rows, cols, dt, _ptr(w), _ptr(q), _ptr(sc)), "quantize_fp8")
+    return q, sc
+
+
+def moe_layer_fp8(x, w_r, q13, s13, q2, s2, K, score_fn=0, renorm=1, q13_sh=None, s13_sh=None, q2_sh=None,
+                  s2_sh=None, logits=None, tokens=None, k=None, nthreads=None):
+    """MoE layer output rows (float64) with FP8 expert weights: q13 [E,2I,H] /
+    q2 [E,H,I] uint8 codes, s13 [E,2I] / s2 [E,H] fp32 row scales (shared FFN
+    likewise, optional); x (and w_r) bf16 bit patterns or fp32."""
+    x, dt = _typed(x)
+    T, H = x.shape
+    E = q13.shape[0]
+    I = q2.shape[2]
+    keep = []
+
+    def table(arrs, ctype=ctypes.c_void_p):
+        tab = (ctype * E)()
+        for e in range(E):
+            a = np.ascontiguousarray(arrs[e])
+            keep.append(a)
+            tab[e] = a.ctypes.data
+        return tab
+
+    p13, p2 = table(q13), table(q2)
+    ps13, ps2 = table(np.asarray(s13, np.float32)), table(np.asarray(s2, np.float32))
+    w_r_c = None
+    if w_r is not None:
+        w_r_c, d = _typed(w_r)
+        assert d == dt
+    I_sh = 0 if q13_sh is None else q2_sh.shape[1]
+    sh = [None if a is None else np.ascontiguousarray(a) for a in (q13_sh, q2_sh)]
+    ssh = [None if a is None else np.ascontiguousarray(a, np.float32) for a in (s13_sh, s2_sh)]
+    lg = None if logits is None else np.ascontiguousarray(logits, dtype=np.float32)
+    if lg is None and w_r_c is None:
+        raise ValueError("need router weights or logits")
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    n = T if tok is None else tok.shape[0]
+    kk = None if k is None else np.ascontiguousarray(k, dtype=np.int32)
+    out = np.empty((n, H), np.float64)
+    _check(lib().oracle_moe_layer_fp8(T, H, E, K, I, I_sh, score_fn, renorm, dt, _ptr(x), _ptr(w_r_c), p13, p2,
+                                      ps13, ps2, _ptr(sh[0]), _ptr(sh[1]), _ptr(ssh[0]), _ptr(ssh[1]), _ptr(lg),
+                                      _ptr(kk), _ptr(tok), n, _ptr(out), nthreads or nthreads_default()),
+           "moe_layer_fp8")
     return out

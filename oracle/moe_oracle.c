@@ -23,7 +23,10 @@
  *     m tokens x K assignments);
  *   - same page, Table 2 (shared experts);
  *   - the MoE-Prism write-up (routing top-k as a per-request runtime knob):
- *     per-token dynamic K, k_t <= K, unused slots -1.
+ *     per-token dynamic K, k_t <= K, unused slots -1;
+ *   - talk notes, "Reduction techniques" (decode: weight quantisation cuts
+ *     the expert weights loaded from HBM): FP8 E4M3 expert weights with row
+ *     scales (format and scaling are this oracle's reading, stated below).
  * Concrete gating (softmax renormalised over the selected K, or sigmoid
  * normalised over the selected K), SwiGLU experts and the tile size come from
  * the layer definitions of the workloads (Mixtral-, Qwen2-MoE-,
@@ -258,6 +261,87 @@ int oracle_combine(int T, int H, int K, int dtype, const void* y, const int32_t*
  *   a_i = silu(g_i) * u_i,      silu(v) = v * sigmoid(v)
  *   y_h = sum_i W2[h][i] a_i
  * x is given as an element offset into a typed array. */
+/* --------------------------------------------------------- FP8 weights */
+/* Quantised expert weights for the decode streaming path (talk notes,
+ * "Reduction techniques / decode optimisation": weight quantisation cuts the
+ * expert weights loaded from HBM, more so for MoE than for dense models).
+ * The pages fix no format; the reading is FP8 E4M3 with one fp32 scale per
+ * output row:
+ *   E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent
+ *   field 0 holds subnormals m/8 * 2^-6; no infinities; S.1111.111 is NaN;
+ *   the largest finite value is 448 (S.1111.110).
+ *   Row scale s_r = max_c |w[r][c]| / 448 (fp32; 1 for an all-zero row);
+ *   code q[r][c] = E4M3(w[r][c] / s_r), the fp32 quotient rounded to the
+ *   nearest E4M3 value, ties to the even mantissa, saturating at +-448;
+ *   dequantised weight = value(q) * s_r. */
+double oracle_e4m3_value(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10); /* (1 + m/8) 2^(e-7) */
+    return sgn ? -v : v;
+}
+
+uint8_t oracle_e4m3_encode(float v)
+{
+    if (isnan(v)) return 0x7F;
+    uint8_t sgn = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return sgn | 0x7E;
+    if (a == 0.0) return sgn;
+    int k;
+    frexp(a, &k);             /* a in [2^(k-1), 2^k) */
+    int eb = k - 1;           /* binade exponent */
+    double step = eb < -6 ? ldexp(1.0, -9) : ldexp(1.0, eb - 3);
+    double q = nearbyint(a / step) * step; /* exact quotient; ties to even (default rounding) */
+    if (q == 0.0) return sgn;
+    frexp(q, &k);
+    eb = k - 1;
+    if (eb < -6) return sgn | (uint8_t)(q / ldexp(1.0, -9));      /* subnormal: m = q / 2^-9 */
+    int m = (int)((q / ldexp(1.0, eb) - 1.0) * 8.0);
+    return sgn | (uint8_t)((eb + 7) << 3) | (uint8_t)m;
+}
+
+/* Row-wise quantisation of w [rows, cols] (dtype 0 bf16 / 1 fp32). */
+int oracle_quantize_fp8(int rows, int cols, int dtype, const void* w, uint8_t* q, float* scales)
+{
+    if (rows < 0 || cols <= 0 || (dtype != 0 && dtype != 1)) return -1;
+    for (int r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int c = 0; c < cols; ++c) {
+            float a = fabsf((float)ld(w, (size_t)r * cols + c, dtype));
+            if (a > amax) amax = a;
+        }
+        float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scales[r] = sc;
+        for (int c = 0; c < cols; ++c) {
+            float v = (float)ld(w, (size_t)r * cols + c, dtype) / sc;
+            q[(size_t)r * cols + c] = oracle_e4m3_encode(v);
+        }
+    }
+    return 0;
+}
+
+/* One token through one FP8 expert: as ffn_one with w = value(q) * s_row. */
+static void ffn_one_fp8(int H, int I, int dtype, const void* x, size_t x_off, const uint8_t* q13,
+                        const float* s13, const uint8_t* q2, const float* s2, double* a_scratch, double* y)
+{
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = ld(x, x_off + h, dtype);
+            g += oracle_e4m3_value(q13[(size_t)i * H + h]) * (double)s13[i] * xv;
+            u += oracle_e4m3_value(q13[(size_t)(I + i) * H + h]) * (double)s13[I + i] * xv;
+        }
+        a_scratch[i] = g * sigmoid(g) * u;
+    }
+    for (int h = 0; h < H; ++h) {
+        double acc = 0.0;
+        for (int i = 0; i < I; ++i) acc += oracle_e4m3_value(q2[(size_t)h * I + i]) * (double)s2[h] * a_scratch[i];
+        y[h] = acc;
+    }
+}
+
 static void ffn_one(int H, int I, int dtype, const void* x, size_t x_off,
                     const void* w13, const void* w2, double* a_scratch, double* y)
 {
@@ -343,13 +427,16 @@ int oracle_dense_ffn(int T, int H, int I, int dtype, const void* x,
  * experts no listed token selects may be NULL).  ids_out / w_out (nullable)
  * receive the routing of each listed token.  Returns -1 on bad input
  * (NaN logit, NULL weight of a selected expert). */
-int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
-                     int renorm, int dtype, const void* x, const void* w_r,
-                     const void* const* w13, const void* const* w2,
-                     const void* w13_sh, const void* w2_sh, const float* logits_in,
-                     const int32_t* k_per_token,
-                     const int32_t* tokens, int n_tok, double* out,
-                     int32_t* ids_out, double* w_out, int nthreads)
+/* wfmt 0: weights of `dtype`; wfmt 1: FP8 codes (uint8) with fp32 row scales
+ * s13 / s2 (per expert) and s13_sh / s2_sh. */
+static int layer_impl(int T, int H, int E, int K, int I, int I_sh, int score_fn,
+                      int renorm, int dtype, int wfmt, const void* x, const void* w_r,
+                      const void* const* w13, const void* const* w2,
+                      const float* const* s13, const float* const* s2,
+                      const void* w13_sh, const void* w2_sh, const float* s13_sh, const float* s2_sh,
+                      const float* logits_in, const int32_t* k_per_token,
+                      const int32_t* tokens, int n_tok, double* out,
+                      int32_t* ids_out, double* w_out, int nthreads)
 {
     if (T < 0 || H <= 0 || E <= 0 || K <= 0 || K > E || I <= 0 || I_sh < 0) return -1;
     if (n_tok < 0) return -1;
@@ -398,16 +485,24 @@ int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
                 for (int k = 0; k < K; ++k) {
                     int e = id[k];
                     if (e < 0) continue;  /* empty slot */
-                    if (!w13[e] || !w2[e]) {
+                    if (!w13[e] || !w2[e] || (wfmt == 1 && (!s13[e] || !s2[e]))) {
 #pragma omp atomic write
                         err = -1;
                         break;
                     }
-                    ffn_one(H, I, dtype, x, xo, w13[e], w2[e], a, y);
+                    if (wfmt == 1)
+                        ffn_one_fp8(H, I, dtype, x, xo, (const uint8_t*)w13[e], s13[e], (const uint8_t*)w2[e],
+                                    s2[e], a, y);
+                    else
+                        ffn_one(H, I, dtype, x, xo, w13[e], w2[e], a, y);
                     for (int h = 0; h < H; ++h) o[h] += w[k] * y[h];
                 }
                 if (I_sh > 0) {
-                    ffn_one(H, I_sh, dtype, x, xo, w13_sh, w2_sh, a, y);
+                    if (wfmt == 1)
+                        ffn_one_fp8(H, I_sh, dtype, x, xo, (const uint8_t*)w13_sh, s13_sh, (const uint8_t*)w2_sh,
+                                    s2_sh, a, y);
+                    else
+                        ffn_one(H, I_sh, dtype, x, xo, w13_sh, w2_sh, a, y);
                     for (int h = 0; h < H; ++h) o[h] += y[h];
                 }
                 if (ids_out)
@@ -424,4 +519,31 @@ int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
         free(y);
     }
     return err;
+}
+
+int oracle_moe_layer(int T, int H, int E, int K, int I, int I_sh, int score_fn,
+                     int renorm, int dtype, const void* x, const void* w_r,
+                     const void* const* w13, const void* const* w2,
+                     const void* w13_sh, const void* w2_sh, const float* logits_in,
+                     const int32_t* k_per_token,
+                     const int32_t* tokens, int n_tok, double* out,
+                     int32_t* ids_out, double* w_out, int nthreads)
+{
+    return layer_impl(T, H, E, K, I, I_sh, score_fn, renorm, dtype, 0, x, w_r, w13, w2, NULL, NULL, w13_sh,
+                      w2_sh, NULL, NULL, logits_in, k_per_token, tokens, n_tok, out, ids_out, w_out, nthreads);
+}
+
+/* The layer with FP8 expert weights (routed and shared): q13[e] / q2[e] the
+ * E4M3 codes of expert e ([2I,H], [H,I]), s13[e] / s2[e] its row scales ([2I],
+ * [H]); x and the router are of `dtype`. */
+int oracle_moe_layer_fp8(int T, int H, int E, int K, int I, int I_sh, int score_fn,
+                         int renorm, int dtype, const void* x, const void* w_r,
+                         const void* const* q13, const void* const* q2,
+                         const float* const* s13, const float* const* s2,
+                         const void* q13_sh, const void* q2_sh, const float* s13_sh, const float* s2_sh,
+                         const float* logits_in, const int32_t* k_per_token,
+                         const int32_t* tokens, int n_tok, double* out, int nthreads)
+{
+    return layer_impl(T, H, E, K, I, I_sh, score_fn, renorm, dtype, 1, x, w_r, q13, q2, s13, s2, q13_sh,
+                      q2_sh, s13_sh, s2_sh, logits_in, k_per_token, tokens, n_tok, out, NULL, NULL, nthreads);
 }

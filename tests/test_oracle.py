@@ -602,3 +602,69 @@ def test_dynamic_k_layer_is_static_layer_per_token():
         else:
             ref = oracle.moe_layer(x, w_r, w13, w2, K=int(k[t]), tokens=np.array([t], np.int32), **sh)[0]
             assert np.allclose(out[t], ref, rtol=1e-13, atol=1e-14)
+
+
+# -------------------------------------------------------- FP8 expert weights
+
+def test_e4m3_value_table_from_the_format():
+    # 1 sign, 4 exponent bits (bias 7), 3 mantissa bits; subnormals at exponent 0
+    v = oracle.e4m3_value(np.arange(256, dtype=np.uint8))
+    assert v[0x38] == 1.0 and v[0x7E] == 448.0 and v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9
+    assert v[0x30] == 0.5 and v[0x3C] == 1.5 and v[0x07] == 7 * 2.0 ** -9
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert np.array_equal(v[0x80:0xFF], -v[0x00:0x7F])
+    assert np.all(np.diff(v[0x00:0x7F]) > 0)                   # codes order the values
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_value(codes).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(vals), codes)     # every finite code, -0 included
+    # ties go to the even mantissa; magnitudes past 448 saturate
+    cases = {1.0625: 0x38, 1.1875: 0x3A, 2.0 ** -10: 0x00, 3 * 2.0 ** -10: 0x02, 2.0 ** -6 - 2.0 ** -10: 0x08,
+             464.0: 0x7E, 1000.0: 0x7E, -1e9: 0xFE, 0.3: 0x2A}
+    for v, c in cases.items():
+        assert int(oracle.e4m3_encode(np.float32(v))) == c, v
+
+
+def test_e4m3_encode_matches_torch_inside_the_finite_range():
+    # torch's float8_e4m3fn cast (round to nearest even) is an independent
+    # implementation; it turns magnitudes >= 464 into NaN, so compare below that
+    rng = np.random.default_rng(31)
+    v = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1.0, 30.0, 200.0)]).astype(np.float32)
+    v = v[np.abs(v) < 464]
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(v), ref)
+
+
+def test_quantize_fp8_rows():
+    rng = np.random.default_rng(32)
+    w = (rng.standard_normal((7, 300)) * np.array([1e-3, 0.1, 1, 3, 0, 50, 1e4])[:, None]).astype(np.float32)
+    q, s = oracle.quantize_fp8(w)
+    assert s[4] == 1.0 and np.all(oracle.e4m3_value(q[4]) == 0)       # an all-zero row (signed zeros kept)
+    amax = np.abs(w).max(1)
+    for r in (0, 1, 2, 3, 5, 6):
+        assert s[r] == np.float32(amax[r]) / np.float32(448.0)
+        assert abs(oracle.e4m3_value(q[r][np.abs(w[r]).argmax()])) == 448.0   # the largest maps to +-448
+        deq = oracle.e4m3_value(q[r]) * s[r]
+        # normal range: relative error at most half a mantissa step (2^-4); below it, half the subnormal step
+        bound = np.maximum(np.abs(w[r]) * 2.0 ** -4, 2.0 ** -10 * s[r]) * (1 + 1e-6)
+        assert np.all(np.abs(deq - w[r]) <= bound)
+
+
+def test_fp8_layer_equals_float_layer_on_representable_weights():
+    # with unit scales the dequantised weights are the codes' values, exactly
+    # fp32; the FP8 layer must then equal the float layer (another code path)
+    rng = np.random.default_rng(33)
+    T, H, E, K, I, I_sh = 9, 32, 5, 2, 24, 16
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w_r = rng.standard_normal((E, H)).astype(np.float32)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    codes = lambda *sh: rng.choice(finite, size=sh).astype(np.uint8)
+    q13, q2, q13s, q2s = codes(E, 2 * I, H), codes(E, H, I), codes(2 * I_sh, H), codes(H, I_sh)
+    scale = lambda *sh: np.full(sh, 1.0 / 64, np.float32)            # a power of two: still exact
+    s13, s2, s13s, s2s = scale(E, 2 * I), scale(E, H), scale(2 * I_sh), scale(H)
+    out = oracle.moe_layer_fp8(x, w_r, q13, s13, q2, s2, K, q13_sh=q13s, s13_sh=s13s, q2_sh=q2s, s2_sh=s2s)
+    f = lambda q, s: (oracle.e4m3_value(q) * s[..., None]).astype(np.float32)
+    ref = oracle.moe_layer(x, w_r, f(q13, s13), f(q2, s2), K, w13_sh=f(q13s, s13s), w2_sh=f(q2s, s2s))
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
