@@ -123,12 +123,16 @@ def parse_workload(s):
 
 
 class Workload:
-    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None, pad_mode=0, dyn_k=False):
+    def __init__(self, shape, T, rank=0, device="cuda", skew=None, weights=None, pad_mode=0, dyn_k=False,
+                 fp8=False):
         import mixture_experts_layer_61_b200 as moe
         self.moe = moe
         self.shape, self.T = shape, T
         seed = mi.seed_for(shape, T)
         self.w = weights if weights is not None else mi.make_weights(shape, seed, device=device)
+        # FP8 expert weights (decode sizes): E4M3 codes + row scales, quantised once here (not timed)
+        self.fp8 = fp8
+        self.q = {n: moe.quantize_fp8(self.w[n]) for n in ("w13", "w2", "w13_sh", "w2_sh") if fp8 and n in self.w}
         self.x = mi.make_x(shape, T, seed + 100 * rank, device=device)
         self.logits = None
         # per-token dynamic K: each token's count drawn uniformly from 1..K (seeded)
@@ -160,8 +164,11 @@ class Workload:
         self.s_act = torch.empty((Pm, shape.I), dtype=dt, device=device)
         self.s_y = torch.empty((Pm, shape.H), dtype=dt, device=device)
         self.s_sh = torch.empty((T, shape.H), dtype=dt, device=device) if shape.I_sh else None
-        self.s_shws = (moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, shape.I_sh, self.cfg.dtype), device)
-                       if shape.I_sh else None)
+        self.s_shws = None
+        if shape.I_sh:
+            n = (moe.dense_fp8_workspace_size(T, shape.H, shape.I_sh) if fp8
+                 else moe.dense_workspace_size(T, shape.H, shape.I_sh, self.cfg.dtype))
+            self.s_shws = moe.alloc_workspace(n, device)
         self.s_al = moe.align_buffers(self.cfg, device)
         self.fused = moe.ffn_fused(self.cfg)
 
@@ -182,6 +189,13 @@ class Workload:
 
     def step(self):
         m = self.moe
+        if self.fp8:
+            q, sh = self.q, {}
+            if "w13_sh" in q:
+                sh = dict(q13_sh=q["w13_sh"][0], s13_sh=q["w13_sh"][1], q2_sh=q["w2_sh"][0], s2_sh=q["w2_sh"][1])
+            m.layer_forward_fp8(self.cfg, self.x, self.w["w_r"], q["w13"][0], q["w13"][1], q["w2"][0], q["w2"][1],
+                                self.ws, logits_override=self.logits, out=self.out, stats=self.stats, k=self.k, **sh)
+            return
         m.layer_forward(self.cfg, self.x, self.w["w_r"], self.w["w13"], self.w["w2"], self.ws,
                         self.w.get("w13_sh"), self.w.get("w2_sh"), self.logits, self.out, self.stats, k=self.k)
 
@@ -195,9 +209,17 @@ class Workload:
         ev[2].record()
         self.al = m.align_pad(c, self.s_ids, self.s_al)
         ev[3].record()
-        m.permute(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
+        if self.fp8:
+            m.permute_f16(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
+        else:
+            m.permute(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
         ev[4].record()
-        if self.fused:
+        if self.fp8:
+            q = self.q
+            m.grouped_ffn_fp8(c, self.s_xp, q["w13"][0], q["w13"][1], q["w2"][0], q["w2"][1], self.al["offsets"],
+                              self.gws, self.s_act, self.s_y)
+            ev[5].record()
+        elif self.fused:
             # the layer's expert FFN is one fused launch (gate/up + SwiGLU + down)
             m.grouped_ffn(c, self.s_xp, self.w["w13"], self.w["w2"], self.al["offsets"], self.gws, self.s_act,
                           self.s_y)
@@ -207,7 +229,11 @@ class Workload:
             ev[5].record()
             m.grouped_down(c, self.s_act, self.w["w2"], self.al["offsets"], self.gws, self.s_y)
         ev[6].record()
-        if self.s_sh is not None:
+        if self.s_sh is not None and self.fp8:
+            q = self.q
+            m.dense_ffn_fp8(self.x, q["w13_sh"][0], q["w13_sh"][1], q["w2_sh"][0], q["w2_sh"][1], self.s_shws,
+                            self.s_sh)
+        elif self.s_sh is not None:
             m.dense_ffn(self.x, self.w["w13_sh"], self.w["w2_sh"], self.s_shws, self.s_sh)
         ev[7].record()
         m.combine(c, self.s_y, self.al["pos"], self.s_w, self.s_sh, self.out)
@@ -258,7 +284,7 @@ def replica_tokens_per_s(world, T, steps, max_total_ms):
 
 # ------------------------------------------------------------ accounting
 
-def algorithmic(shape, T, E_active, A=None):
+def algorithmic(shape, T, E_active, A=None, fp8=False):
     """Algorithmic bytes and flops of one layer forward (padding excluded):
     bytes = weights of the activated experts + shared weights + router weights,
     flops = 2 T (H E + 3 H I_sh) + 2 A 3 H I with A = T K assignments (or
@@ -266,7 +292,11 @@ def algorithmic(shape, T, E_active, A=None):
     eb = 2 if shape.dtype == "bf16" else 4
     H, I, E, K = shape.H, shape.I, shape.E, shape.K
     A = T * K if A is None else A
-    B = E_active * 3 * H * I * eb + 3 * H * shape.I_sh * eb + E * H * eb
+    if fp8:  # 1-byte codes + fp32 row scales for the expert weights; the router stays bf16
+        B = E_active * (3 * H * I + 4 * (2 * I + H)) + (3 * H * shape.I_sh + 4 * (2 * shape.I_sh + H)) * (
+            shape.I_sh > 0) + E * H * eb
+    else:
+        B = E_active * 3 * H * I * eb + 3 * H * shape.I_sh * eb + E * H * eb
     F = 2.0 * T * (H * E + 3 * H * shape.I_sh) + 2.0 * A * 3 * H * I
     return B, F
 
@@ -279,25 +309,34 @@ def gate_up_work(shape, T, E_active, A=None):
     return E_active * 2 * shape.I * shape.H * eb, 2.0 * A * shape.H * 2 * shape.I
 
 
-def ffn_work(shape, T, E_active, A=None):
+def ffn_work(shape, T, E_active, A=None, fp8=False):
     """Fused expert FFN: weight bytes of the activated experts' W1/W3/W2,
     flops 2 * A * 3 * H * I (A = T K assignments)."""
     eb = 2 if shape.dtype == "bf16" else 4
     A = T * shape.K if A is None else A
-    return E_active * 3 * shape.I * shape.H * eb, 2.0 * A * 3 * shape.H * shape.I
+    B = E_active * (3 * shape.I * shape.H + 4 * (2 * shape.I + shape.H)) if fp8 else E_active * 3 * shape.I * shape.H * eb
+    return B, 2.0 * A * 3 * shape.H * shape.I
 
 
-def dense_times(shape, T, I_d, steps, warmup, flush, device, seed):
+def dense_times(shape, T, I_d, steps, warmup, flush, device, seed, fp8=False):
     import mixture_experts_layer_61_b200 as moe
     w13, w2 = mi.make_dense_weights(shape.H, I_d, shape.torch_dtype, seed=seed, device=device)
     x = mi.make_x(shape, T, seed, device=device)
-    ws = moe.alloc_workspace(moe.dense_workspace_size(T, shape.H, I_d, 0 if shape.dtype == "bf16" else 1), device)
+    ws = moe.alloc_workspace(moe.dense_fp8_workspace_size(T, shape.H, I_d) if fp8 else
+                             moe.dense_workspace_size(T, shape.H, I_d, 0 if shape.dtype == "bf16" else 1), device)
     out = torch.empty_like(x)
-    moe.dense_ffn(x, w13, w2, ws, out)
+    if fp8:
+        (q13, s13), (q2, s2) = moe.quantize_fp8(w13), moe.quantize_fp8(w2)
+        del w13, w2
+        w13 = w2 = None
+        run = lambda: moe.dense_ffn_fp8(x, q13, s13, q2, s2, ws, out)
+    else:
+        run = lambda: moe.dense_ffn(x, w13, w2, ws, out)
+    run()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        moe.dense_ffn(x, w13, w2, ws, out)
+        run()
     for _ in range(warmup):
         g.replay()
     torch.cuda.synchronize()
@@ -367,6 +406,8 @@ def main():
     ap.add_argument("--no-pdl", action="store_true", help="plain stream order between kernels")
     ap.add_argument("--pad-mode", type=int, default=0, choices=[0, 1],
                     help="alignment padding: 0 block-wise, 1 max-value")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 E4M3 expert weights with row scales (decode sizes)")
     ap.add_argument("--dynamic-k", action="store_true",
                     help="per-token dynamic K: each token's expert count uniform in 1..K (seeded)")
     ap.add_argument("--padding-model", action="store_true",
@@ -408,7 +449,8 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return
-    wl = Workload(shape, T, rank, device, skew=args.skew, pad_mode=args.pad_mode, dyn_k=args.dynamic_k)
+    wl = Workload(shape, T, rank, device, skew=args.skew, pad_mode=args.pad_mode, dyn_k=args.dynamic_k,
+                  fp8=args.fp8)
     if args.no_graph:
         run_step, wl.launches_per_step = wl.step, None
     else:
@@ -460,7 +502,8 @@ def main():
                                                         "token_tile_cap": args.token_tile_cap,
                                                         "pdl": not args.no_pdl,
                                                         "shared_sms": moe.shared_sms(wl.cfg),
-                                                        "pad_mode": args.pad_mode, "dynamic_k": args.dynamic_k},
+                                                        "pad_mode": args.pad_mode, "dynamic_k": args.dynamic_k,
+                                                        "fp8": args.fp8},
                               "stages_ms": stages, "E_active": E_active, "P": P}), flush=True)
         if dist:
             dist.barrier()
@@ -470,7 +513,7 @@ def main():
     # ---- roofline of the dominant kernel: the grouped gate/up + SwiGLU GEMM,
     # or the fused expert FFN when the layer runs it as one launch
     if wl.fused:
-        gu_bytes, gu_flops = ffn_work(shape, T, E_active, wl.A)
+        gu_bytes, gu_flops = ffn_work(shape, T, E_active, wl.A, fp8=args.fp8)
         t_gu = stages["ffn"] * 1e-3
     else:
         gu_bytes, gu_flops = gate_up_work(shape, T, E_active, wl.A)
@@ -487,10 +530,10 @@ def main():
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": round(ach / tc_peak, 4), "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4)}
     roof["kernel"] = ("moe_ffn_stream_kernel (fused expert FFN: gate/up + SwiGLU + down)" if wl.fused
-                      else "moe_gemm_kernel (grouped gate/up + SwiGLU)")
+                      else "moe_gemm_kernel (grouped gate/up + SwiGLU)") + (", FP8 weights" if args.fp8 else "")
     roof["peak_source"] = f"{pk_kind} ({'MEASURED_PEAKS.json' if pk_kind == 'measured' else 'fallback'})"
-    roof["traffic"] = NCU_TRAFFIC.get(f"{shape.name}:{T}")
-    B_alg, F_alg = algorithmic(shape, T, E_active, wl.A)
+    roof["traffic"] = NCU_TRAFFIC.get(f"{shape.name}:{T}" + (":fp8" if args.fp8 else ""))
+    B_alg, F_alg = algorithmic(shape, T, E_active, wl.A, fp8=args.fp8)
     t_layer = ms_step * 1e-3
     layer_roof = max(F_alg / (tc_peak * 1e12), B_alg / (hbm_peak * 1e9)) / t_layer
 
@@ -519,8 +562,8 @@ def main():
     tau = None
     if not args.no_tau:
         seed = mi.seed_for(shape, T, 50)
-        t_fa = dense_times(shape, T, shape.I_FA, args.steps, args.warmup, flush, device, seed)
-        t_pa = dense_times(shape, T, shape.I_PA, args.steps, args.warmup, flush, device, seed + 1)
+        t_fa = dense_times(shape, T, shape.I_FA, args.steps, args.warmup, flush, device, seed, fp8=args.fp8)
+        t_pa = dense_times(shape, T, shape.I_PA, args.steps, args.warmup, flush, device, seed + 1, fp8=args.fp8)
         t_moe = statistics.median(times)
         tau = {"tau_FA": round(t_moe / t_fa, 4), "tau_PA": round(t_moe / t_pa, 4),
                "t_moe_ms": round(t_moe, 4), "t_DenseFA_ms": round(t_fa, 4), "t_DensePA_ms": round(t_pa, 4),
@@ -557,7 +600,9 @@ def main():
                    "shared_sms": moe.shared_sms(wl.cfg),
                    "padding": "max-value" if args.pad_mode == 1 else "block-wise",
                    "top_k": (f"per-token dynamic, uniform 1..{shape.K} (sum {wl.A})" if args.dynamic_k
-                             else f"{shape.K} for every token")},
+                             else f"{shape.K} for every token"),
+                   "expert_weights": ("FP8 E4M3 codes + fp32 row scales (widened to bf16 in shared memory)"
+                                      if args.fp8 else shape.dtype)},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - wl.A) / max(P, 1), 4),
                   "bytes_alg": B_alg, "flops_alg": F_alg, "roofline_frac": round(layer_roof, 4),

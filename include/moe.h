@@ -231,6 +231,60 @@ int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_ro
                         const int32_t* k_per_token, void* out, void* workspace,
                         size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
 
+/* FP8 expert weights for the decode streaming path (talk notes, "Reduction
+ * techniques": weight quantisation cuts the expert bytes loaded from HBM).
+ * Row-wise E4M3 quantisation of w [rows, cols] (dtype 0 bf16, 1 fp32):
+ *   scales[r] = max_c |w[r][c]| / 448 (1 for an all-zero row, fp32),
+ *   q[r][c]   = E4M3(w[r][c] / scales[r]), nearest with ties to even,
+ *               saturating at +-448 (E4M3: 1 sign, 4 exponent bits with bias
+ *               7, 3 mantissa bits, no infinities).
+ * cols must be a multiple of 16 (16-byte rows of codes).  Apply it to each
+ * expert's w13 rows ([E*2I, H]) and w2 rows ([E*H, I]), and to the shared
+ * FFN's; one block per row. */
+int moe_quantize_fp8(int64_t rows, int cols, int dtype, const void* w, uint8_t* q,
+                     float* scales, moe_stream_t stream);
+
+/* moe_layer_forward_k with FP8 routed (and shared) expert weights: codes
+ * w13_q [E,2I,H], w2_q [E,H,I] with row scales w13_s [E,2I], w2_s [E,H]
+ * (shared likewise, [2*I_sh,H] / [H,I_sh] with [2*I_sh] / [H]); x, the router
+ * and the output stay bf16 (cfg->dtype 0).  The codes stream from HBM and are
+ * widened to f16 in shared memory (exact); the expert MMAs run on f16
+ * operands (x and the SwiGLU activations converted to f16, so |x| and the
+ * activations must stay within the f16 range) with fp32 accumulation, and
+ * each output row is multiplied by its fp32 scale.  Decode sizes only: the expert FFNs
+ * must run as the fused kernel (at most 128 rows per routed expert and, with
+ * shared experts, T <= 128); otherwise MOE_ERR_ARG.  H, I, S*I_s multiples of
+ * 16.  Same workspace as moe_layer_forward. */
+int moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_router,
+                          const uint8_t* w13_q, const float* w13_s, const uint8_t* w2_q,
+                          const float* w2_s, const uint8_t* w13_shared_q,
+                          const float* w13_shared_s, const uint8_t* w2_shared_q,
+                          const float* w2_shared_s, const float* logits_override,
+                          const int32_t* k_per_token, void* out, void* workspace,
+                          size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
+
+/* moe_permute writing the permuted rows as f16 (the FP8-weight path computes
+ * on f16 operands; E4M3 values are exact in f16); bf16 x (cfg->dtype 0). */
+int moe_permute_f16(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids,
+                    const int32_t* scalars, void* x_perm, moe_stream_t stream);
+
+/* moe_grouped_ffn with FP8 routed expert weights (codes and row scales as
+ * for moe_layer_forward_fp8); decode sizes only (at most 128 rows per
+ * expert).  x_perm is f16 (moe_permute_f16); `act` is f16 scratch
+ * ([P_max, I]); y_perm is bf16. */
+int moe_grouped_ffn_fp8(const moe_config_t* cfg, const void* x_perm, const uint8_t* w13_q,
+                        const float* w13_s, const uint8_t* w2_q, const float* w2_s,
+                        const int32_t* offsets, void* act, void* y_perm, void* workspace,
+                        size_t ws_bytes, moe_stream_t stream);
+
+/* dense_ffn with FP8 weights (codes [2I,H] / [H,I] and row scales [2I] /
+ * [H]), bf16 x and out; decode sizes only (T <= 128); workspace of
+ * dense_ffn_fp8_workspace_size bytes (x is widened to f16 there). */
+size_t dense_ffn_fp8_workspace_size(int T, int H, int I);
+int dense_ffn_fp8(int T, int H, int I, const void* x, const uint8_t* w13_q, const float* w13_s,
+                  const uint8_t* w2_q, const float* w2_s, void* out, void* workspace,
+                  size_t ws_bytes, moe_stream_t stream);
+
 /* Bytes of workspace dense_ffn needs for T tokens of width I (0 if invalid). */
 size_t dense_ffn_workspace_size(int T, int H, int I, int dtype);
 

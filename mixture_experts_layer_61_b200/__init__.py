@@ -76,6 +76,12 @@ def lib():
             "moe_combine": (I, [C, P, P, P, P, P, P]),
             "moe_layer_forward": (I, [C, P, P, P, P, P, P, P, P, P, S, P, P]),
             "moe_layer_forward_k": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P, P]),
+            "moe_quantize_fp8": (I, [ctypes.c_int64, I, I, P, P, P, P]),
+            "moe_grouped_ffn_fp8": (I, [C, P, P, P, P, P, P, P, P, P, S, P]),
+            "dense_ffn_fp8": (I, [I, I, I, P, P, P, P, P, P, P, S, P]),
+            "dense_ffn_fp8_workspace_size": (S, [I, I, I]),
+            "moe_permute_f16": (I, [C, P, P, P, P, P]),
+            "moe_layer_forward_fp8": (I, [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P, P]),
             "dense_ffn_workspace_size": (S, [I, I, I, I]),
             "dense_ffn": (I, [I, I, I, I, P, P, P, P, P, S, P]),
             "moe_check_status": (I, [P, P]),
@@ -259,6 +265,65 @@ def layer_forward(cfg, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, logits_over
                                      _p(logits_override), _p(k), _p(out), _p(ws), ws.numel(), _p(stats),
                                      _stream()),
            "moe_layer_forward_k")
+    return out
+
+
+def quantize_fp8(w):
+    """Row-wise FP8 E4M3 codes and fp32 scales of a weight tensor whose last
+    dimension is the input features (rows = everything else), on the device:
+    returns (codes uint8 of w's shape, scales float32 of w.shape[:-1])."""
+    _need_cuda(w)
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    sc = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    dt = BF16 if w.dtype == torch.bfloat16 else FP32
+    _check(lib().moe_quantize_fp8(rows, cols, dt, _p(w), _p(q), _p(sc), _stream()), "moe_quantize_fp8")
+    return q, sc
+
+
+def dense_ffn_fp8(x, q13, s13, q2, s2, ws, out=None):
+    _need_cuda(x, q13, s13, q2, s2, ws)
+    T, H = x.shape
+    I = q2.shape[1]
+    if out is None:
+        out = torch.empty((T, H), dtype=x.dtype, device=x.device)
+    _check(lib().dense_ffn_fp8(T, H, I, _p(x), _p(q13), _p(s13), _p(q2), _p(s2), _p(out), _p(ws), ws.numel(),
+                               _stream()), "dense_ffn_fp8")
+    return out
+
+
+def dense_fp8_workspace_size(T, H, I):
+    return int(lib().dense_ffn_fp8_workspace_size(T, H, I))
+
+
+def permute_f16(cfg, x, sorted_ids, scalars, x_perm=None):
+    """moe_permute writing f16 rows (the FP8-weight path's token operand)."""
+    _need_cuda(x, sorted_ids, scalars)
+    if x_perm is None:
+        x_perm = torch.empty((max(padded_rows_max(cfg), 1), cfg.H), dtype=torch.float16, device=x.device)
+    _check(lib().moe_permute_f16(ctypes.byref(cfg), _p(x), _p(sorted_ids), _p(scalars), _p(x_perm), _stream()),
+           "moe_permute_f16")
+    return x_perm
+
+
+def grouped_ffn_fp8(cfg, x_perm, q13, s13, q2, s2, offsets, ws, act, y_perm):
+    _need_cuda(x_perm, q13, s13, q2, s2, offsets, ws, act, y_perm)
+    _check(lib().moe_grouped_ffn_fp8(ctypes.byref(cfg), _p(x_perm), _p(q13), _p(s13), _p(q2), _p(s2), _p(offsets),
+                                     _p(act), _p(y_perm), _p(ws), ws.numel(), _stream()), "moe_grouped_ffn_fp8")
+    return y_perm, act
+
+
+def layer_forward_fp8(cfg, x, w_r, q13, s13, q2, s2, ws, q13_sh=None, s13_sh=None, q2_sh=None, s2_sh=None,
+                      logits_override=None, out=None, stats=None, k=None):
+    """The layer with FP8 expert weights (codes and row scales from quantize_fp8)."""
+    _need_cuda(x, w_r, q13, s13, q2, s2, ws, q13_sh, s13_sh, q2_sh, s2_sh, logits_override, stats, k)
+    if out is None:
+        out = torch.empty((cfg.T, cfg.H), dtype=x.dtype, device=x.device)
+    _check(lib().moe_layer_forward_fp8(ctypes.byref(cfg), _p(x), _p(w_r), _p(q13), _p(s13), _p(q2), _p(s2),
+                                       _p(q13_sh), _p(s13_sh), _p(q2_sh), _p(s2_sh), _p(logits_override), _p(k),
+                                       _p(out), _p(ws), ws.numel(), _p(stats), _stream()),
+           "moe_layer_forward_fp8")
     return out
 
 

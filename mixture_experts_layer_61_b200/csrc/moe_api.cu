@@ -3,6 +3,7 @@
 // the MoE layer forward.  Every compute step runs in the kernels of
 // moe_kernels.cu and moe_gemm.cu; nothing here touches tensor data.
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <mutex>
 
@@ -101,7 +102,7 @@ long long p_max(const moe_config_t* c) {
 
 struct Layout {
     size_t ctl, ctl_sh, logits, route_part, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm,
-        act, act_sh, sh_out;
+        act, act_sh, sh_out, x16;
     size_t total;
 };
 
@@ -135,6 +136,8 @@ Layout layout(const moe_config_t* c, int num_sms) {
     L.act = take(eb * (size_t)P * c->I);
     L.act_sh = take(I_sh > 0 ? eb * (size_t)c->T * I_sh : 0);
     L.sh_out = take(I_sh > 0 ? eb * (size_t)c->T * c->H : 0);
+    // x in f16 for the shared FFN on FP8 weights (bf16 layers only)
+    L.x16 = take(I_sh > 0 && c->dtype == 0 ? 2 * (size_t)c->T * c->H : 0);
     L.total = o;
     return L;
 }
@@ -199,7 +202,10 @@ GemmLaunch down_launch(const void* act, long long x_rows, const int32_t* seg_off
 // kernel (0 = one block per SM).
 int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows, int H, int I,
             int dtype, const void* w13, const void* w2, void* act, void* y, int max_n, const GemmCtl& ctl,
-            cudaStream_t s, long long max_chunks, int sms = 0, int ffn_sms = 0) {
+            cudaStream_t s, long long max_chunks, int sms = 0, int ffn_sms = 0, const float* s13 = nullptr,
+            const float* s2 = nullptr) {
+    const bool fp8 = s13 != nullptr;  // w13 / w2 hold E4M3 codes with these row scales
+    if (fp8 && max_n > 128) return -1;  // FP8 weights run on the fused (decode-size) kernel only
     if (max_n <= 128) {
         FfnLaunch f;
         f.x = x;
@@ -217,8 +223,12 @@ int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_g
         f.max_n = max_n;
         f.max_chunks = max_chunks;
         f.sms = ffn_sms;
+        f.fp8 = fp8;
+        f.s13 = s13;
+        f.s2 = s2;
         int rc = launch_ffn_stream(f, ctl, s);
         if (rc != 1) return rc;  // 1: not handled, use two launches
+        if (fp8) return -1;
     }
     GemmLaunch g = gate_up_launch(x, x_rows, seg_offsets, n_groups, seg_rows, H, I, dtype, w13, act, max_n);
     g.sms = sms;
@@ -444,6 +454,27 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const void* w13
                              routed_max_chunks(cfg)));
 }
 
+int moe_grouped_ffn_fp8(const moe_config_t* cfg, const void* x_perm, const uint8_t* w13_q, const float* w13_s,
+                        const uint8_t* w2_q, const float* w2_s, const int32_t* offsets, void* act, void* y_perm,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->dtype != 0 || cfg->H % 16 || cfg->I % 16) return MOE_ERR_ARG;
+    if (cfg->T == 0) return MOE_OK;
+    if (!x_perm || !w13_q || !w13_s || !w2_q || !w2_s || !offsets || !act || !y_perm || !workspace)
+        return MOE_ERR_ARG;
+    if (!aligned16(x_perm) || !aligned16(w13_q) || !aligned16(w2_q) || !aligned16(act) || !aligned16(y_perm) ||
+        !aligned16(workspace))
+        return MOE_ERR_ARG;
+    if (routed_max_n(cfg) > 128) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    return status_of(run_ffn(x_perm, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13_q, w2_q, act,
+                             y_perm, routed_max_n(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream,
+                             routed_max_chunks(cfg), 0, 0, w13_s, w2_s));
+}
+
 int moe_grouped_gate_up(const moe_config_t* cfg, const void* x_perm, const void* w13, const int32_t* offsets,
                         void* act, void* workspace, size_t ws_bytes, moe_stream_t stream) {
     int rc = check_cfg(cfg);
@@ -493,10 +524,50 @@ int moe_layer_forward(const moe_config_t* cfg, const void* x, const void* w_rout
                                workspace, ws_bytes, stats_out, stream);
 }
 
+namespace {
+struct Fp8Scales {
+    const float *s13, *s2, *s13_sh, *s2_sh;
+};
+}  // namespace
+
+static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
+                              const void* w2, const void* w13_shared, const void* w2_shared,
+                              const Fp8Scales* fp8, const float* logits_override, const int32_t* k_per_token,
+                              void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
+
 int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
                         const void* w2, const void* w13_shared, const void* w2_shared, const float* logits_override,
                         const int32_t* k_per_token, void* out, void* workspace, size_t ws_bytes, int32_t* stats_out,
                         moe_stream_t stream) {
+    return layer_forward_impl(cfg, x, w_router, w13, w2, w13_shared, w2_shared, nullptr, logits_override,
+                              k_per_token, out, workspace, ws_bytes, stats_out, stream);
+}
+
+int moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_router, const uint8_t* w13_q,
+                          const float* w13_s, const uint8_t* w2_q, const float* w2_s, const uint8_t* w13_shared_q,
+                          const float* w13_shared_s, const uint8_t* w2_shared_q, const float* w2_shared_s,
+                          const float* logits_override, const int32_t* k_per_token, void* out, void* workspace,
+                          size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->dtype != 0) return MOE_ERR_ARG;  // bf16 activations
+    if (cfg->T == 0) return MOE_OK;
+    const long long I_sh = (long long)cfg->n_shared * cfg->I_shared;
+    if (!w13_s || !w2_s || (I_sh > 0 && (!w13_shared_s || !w2_shared_s))) return MOE_ERR_ARG;
+    if (cfg->H % 16 || cfg->I % 16 || I_sh % 16) return MOE_ERR_ARG;  // 16-byte rows of codes
+    // decode sizes: the routed and shared FFNs must run on the fused kernel
+    if (routed_max_n(cfg) > 128 || (I_sh > 0 && pick_max_n(cfg->T) > 128)) return MOE_ERR_ARG;
+    const Fp8Scales sc{w13_s, w2_s, w13_shared_s, w2_shared_s};
+    return layer_forward_impl(cfg, x, w_router, w13_q, w2_q, w13_shared_q, w2_shared_q, &sc, logits_override,
+                              k_per_token, out, workspace, ws_bytes, stats_out, stream);
+}
+
+}  // extern "C"
+
+static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
+                              const void* w2, const void* w13_shared, const void* w2_shared,
+                              const Fp8Scales* fp8, const float* logits_override, const int32_t* k_per_token,
+                              void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->T == 0) return MOE_OK;
@@ -543,9 +614,19 @@ int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_ro
             GemmCtl ctl_sh = gemm_ctl(at<uint8_t>(workspace, L.ctl_sh), d.num_sms);
             ctl_sh.status = ctl.status + 1;  // the header's second status word
             void* sh_out = at<void>(workspace, L.sh_out);
-            rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
+            const void* x_sh = x;
+            if (fp8) {  // the FP8 path's token operand is f16
+                x_sh = at<void>(workspace, L.x16);
+                if ((rc = launch_bf16_to_f16((long long)cfg->T * cfg->H, x, at<void>(workspace, L.x16), sd.s)) != 0) {
+                    cudaEventRecord(sd.join, sd.s);
+                    cudaStreamWaitEvent(s, sd.join, 0);
+                    return status_of(rc);
+                }
+            }
+            rc = run_ffn(x_sh, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
                          at<void>(workspace, L.act_sh), sh_out, pick_max_n(cfg->T), ctl_sh, sd.s,
-                         dense_max_chunks(cfg->T), n_sh, n_sh);
+                         dense_max_chunks(cfg->T), n_sh, n_sh, fp8 ? fp8->s13_sh : nullptr,
+                         fp8 ? fp8->s2_sh : nullptr);
             if (cudaEventRecord(sd.join, sd.s) != cudaSuccess) {
                 cudaGetLastError();
                 return MOE_ERR_CUDA;
@@ -612,16 +693,24 @@ int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_ro
                                pos, scalars, stats_out, s)) != 0)
             return status_of(rc);
     }
-    if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s)) != 0)
+    if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s, fp8 != nullptr)) != 0)
         return status_of(rc);
     if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
-                      routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn)) != 0)
+                      routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn,
+                      fp8 ? fp8->s13 : nullptr, fp8 ? fp8->s2 : nullptr)) != 0)
         return status_of(rc);
     if (I_sh > 0 && !side) {
         void* sh_out = at<void>(workspace, L.sh_out);
-        if ((rc = run_ffn(x, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
+        const void* x_sh = x;
+        if (fp8) {
+            x_sh = at<void>(workspace, L.x16);
+            if ((rc = launch_bf16_to_f16((long long)cfg->T * cfg->H, x, at<void>(workspace, L.x16), s)) != 0)
+                return status_of(rc);
+        }
+        if ((rc = run_ffn(x_sh, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
                           at<void>(workspace, L.act_sh), sh_out, pick_max_n(cfg->T), ctl, s,
-                          dense_max_chunks(cfg->T))) != 0)
+                          dense_max_chunks(cfg->T), 0, 0, fp8 ? fp8->s13_sh : nullptr,
+                          fp8 ? fp8->s2_sh : nullptr)) != 0)
             return status_of(rc);
         sh = sh_out;
     }
@@ -634,6 +723,9 @@ int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_ro
     }
     return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, w, sh, out, s));
 }
+
+extern "C" {
+
 
 int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13, const void* w2, void* out,
               void* workspace, size_t ws_bytes, moe_stream_t stream) {
@@ -652,6 +744,58 @@ int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13, co
     void* act = at<void>(workspace, ctl_bytes);
     return status_of(run_ffn(x, T, nullptr, 1, T, H, I, dtype, w13, w2, act, out, pick_max_n(T),
                              gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream, dense_max_chunks(T)));
+}
+
+int dense_ffn_fp8(int T, int H, int I, const void* x, const uint8_t* w13_q, const float* w13_s, const uint8_t* w2_q,
+                  const float* w2_s, void* out, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    if (T < 0 || H <= 0 || I <= 0 || H % 16 || I % 16) return MOE_ERR_ARG;
+    if ((long long)2 * I >= (1LL << 31)) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (pick_max_n(T) > 128) return MOE_ERR_ARG;  // decode sizes: the fused kernel
+    if (!x || !w13_q || !w13_s || !w2_q || !w2_s || !out || !workspace) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w13_q) || !aligned16(w2_q) || !aligned16(out) || !aligned16(workspace))
+        return MOE_ERR_ARG;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return status_of(rc);
+    const size_t ctl_bytes = align256(ctl_block_bytes(d.num_sms));
+    const size_t act_bytes = align256((size_t)2 * T * I);
+    if (ws_bytes < ctl_bytes + act_bytes + (size_t)2 * T * H) return MOE_ERR_WORKSPACE;
+    void* act = at<void>(workspace, ctl_bytes);
+    void* x16 = at<void>(workspace, ctl_bytes + act_bytes);  // the FP8 path's token operand is f16
+    if ((rc = launch_bf16_to_f16((long long)T * H, x, x16, (cudaStream_t)stream)) != 0) return status_of(rc);
+    return status_of(run_ffn(x16, T, nullptr, 1, T, H, I, 0, w13_q, w2_q, act, out, pick_max_n(T),
+                             gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream, dense_max_chunks(T), 0, 0, w13_s,
+                             w2_s));
+}
+
+size_t dense_ffn_fp8_workspace_size(int T, int H, int I) {
+    if (T < 0 || H <= 0 || I <= 0) return 0;
+    DeviceInfo d;
+    if (current_device(&d) != 0) return 0;
+    return align256(ctl_block_bytes(d.num_sms)) + align256((size_t)2 * T * I) + align256((size_t)2 * T * H);
+}
+
+int moe_permute_f16(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids, const int32_t* scalars,
+                    void* x_perm, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->dtype != 0) return MOE_ERR_ARG;
+    if (cfg->T == 0) return MOE_OK;
+    if (!x || !sorted_ids || !scalars || !x_perm || !aligned16(x) || !aligned16(x_perm)) return MOE_ERR_ARG;
+    return status_of(launch_permute(cfg->H, cfg->K, cfg->dtype, p_max(cfg), x, sorted_ids, scalars, x_perm,
+                                    (cudaStream_t)stream, true));
+}
+
+int moe_quantize_fp8(int64_t rows, int cols, int dtype, const void* w, uint8_t* q, float* scales,
+                     moe_stream_t stream) {
+    if (rows < 0 || rows > INT32_MAX || cols <= 0 || cols % 16 || (dtype != 0 && dtype != 1)) return MOE_ERR_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!w || !q || !scales) return MOE_ERR_ARG;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return status_of(rc);
+    return status_of(launch_quantize_fp8(rows, cols, dtype, w, q, scales, (cudaStream_t)stream));
 }
 
 int moe_check_status(void* workspace, moe_stream_t stream) {

@@ -6,6 +6,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,6 +28,13 @@ template <> struct Elt<__nv_bfloat16> {
     static constexpr uint32_t kMmaFmt = 1;  // BF16 in the instruction descriptor
     __device__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
     __device__ static __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+template <> struct Elt<__half> {
+    static constexpr int kBytes = 2;
+    static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    static constexpr uint32_t kMmaFmt = 0;  // F16 in the instruction descriptor
+    __device__ static float to_f(__half v) { return __half2float(v); }
+    __device__ static __half from_f(float v) { return __float2half_rn(v); }
 };
 template <> struct Elt<float> {
     static constexpr int kBytes = 4;
@@ -226,6 +235,13 @@ __device__ __forceinline__ void umma<__nv_bfloat16>(uint32_t d_tmem, uint64_t a_
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// f16 operands: the same kind::f16 MMA, the format is in the instruction descriptor
+template <>
+__device__ __forceinline__ void umma<__half>(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    umma<__nv_bfloat16>(d_tmem, a_desc, b_desc, idesc, accumulate);
 }
 
 template <>

@@ -24,7 +24,17 @@
 // Roles as in the grouped GEMM (warp 0 TMA, warp 1 TMEM + MMA, warps 2..5
 // epilogue); the producer publishes each item id to the other roles through a
 // small shared-memory ring.
+//
+// FP8 weights (kFp8): the weight tiles stream as E4M3 codes (half the bytes),
+// 128 rows x 64 codes per tile without swizzle; warps 6..9 widen each stage's
+// two tiles to f16 (one cvt per pair of codes; E4M3 values are exact in f16)
+// into a ring of conversion buffers in the 128-byte swizzled layout the MMA
+// reads, and the epilogue multiplies each output row by its fp32 row scale.
+// The MMAs then run on f16 operands: x_perm arrives in f16 and the SwiGLU
+// activations are stored in f16 (the output stays in the activation dtype).
 #pragma once
+
+#include <type_traits>
 
 #include "moe_gemm.cuh"
 
@@ -50,23 +60,36 @@ struct FfnParams {
     uint64_t wait_limit_ns;
     int withhold_first_load;
     int max_slots_phase;  // partial slots available to each phase
+    const float* s13;     // FP8 weights: row scales [n_groups * 2I] (gate rows, then up rows), else nullptr
+    const float* s2;      // FP8 weights: row scales [n_groups * H], else nullptr
 };
 
-template <typename T, int kMaxN>
+template <typename T, int kMaxN, bool kFp8 = false>
 struct FfnCfg {
     static constexpr int kBK = 128 / Elt<T>::kBytes;
-    static constexpr int kWTileBytes = 128 * 128;
+    static constexpr int kWTileBytes = 128 * 128;                        // a bf16 weight tile as the MMA reads it
+    static constexpr int kRawWBytes = kFp8 ? 128 * kBK : kWTileBytes;  // a weight tile as it streams in
     static constexpr int kXBoxRows = 16, kXBoxMid = 64;
     static constexpr int kXTileBytes = kMaxN * 128;
-    static constexpr int kStageBytes = 2 * kWTileBytes + kXTileBytes;
+    static constexpr int kStageBytes = 2 * kRawWBytes + kXTileBytes;
+    static constexpr int kConv = kFp8 ? (kMaxN <= 64 ? 3 : 2) : 0;       // f16 conversion buffers
+    static constexpr int kConvBytes = 2 * kWTileBytes;
+    static constexpr int kThreads = kFp8 ? 320 : kFfnThreads;
     static constexpr int kAccCols = 2 * kMaxN;
     static constexpr int kNumAcc = 2;
     static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
     static constexpr int kMiscBytes = 768;
-    static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes;
+    static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes - kConv * kConvBytes;
     static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
+    static constexpr int kSmemBytes =
+        1024 + kStages * kStageBytes + kConv * kConvBytes + kTableBytes + kMiscBytes;
+    static_assert(kStageBytes % 1024 == 0, "stages keep the swizzle atoms aligned");
+    static_assert(!kFp8 || sizeof(T) == 2, "FP8 weights: 16-bit activations");
+    // barriers (full/empty per stage, 2 TMEM pairs, the item ring, the conversion
+    // ring, the drain barrier) and the ring / TMEM / flag words fit the misc area
+    static_assert((2 * kStages + 2 * kNumAcc + 2 * kFfnRing + 2 * kConv + 1) * 8 + 4 * kFfnRing + 16 <= kMiscBytes,
+                  "misc area");
     static constexpr int kSlotFloats = 128 * kAccCols;
     static_assert(kMaxN == 32 || kMaxN == 64 || kMaxN == 128, "decode token tiles");
     static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
@@ -101,18 +124,29 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-template <typename T, int kMaxN>
-__global__ void __launch_bounds__(kFfnThreads, 1)
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Two E4M3 codes (low byte first) -> two f16 (exact), one conversion instruction.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+    return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+}
+
+template <typename T, int kMaxN, bool kFp8 = false>
+__global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     moe_ffn_stream_kernel(const __grid_constant__ CUtensorMap tm_w13, const __grid_constant__ CUtensorMap tm_w2,
                           const __grid_constant__ CUtensorMap tm_xa, const __grid_constant__ CUtensorMap tm_xa64,
                           const __grid_constant__ CUtensorMap tm_xb, const __grid_constant__ CUtensorMap tm_xb64,
                           const FfnParams p) {
-    using C = FfnCfg<T, kMaxN>;
+    using C = FfnCfg<T, kMaxN, kFp8>;
     using OutT = T;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_base = smem;
-    int* seg = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes);
+    uint8_t* conv_base = smem + C::kStages * C::kStageBytes;
+    int* seg = reinterpret_cast<int*>(conv_base + C::kConv * C::kConvBytes);
     int* cbase = seg + (kMaxGroups + 1);
     uint8_t* misc = reinterpret_cast<uint8_t*>(cbase + (kMaxGroups + 1));
     uint64_t* full = reinterpret_cast<uint64_t*>(misc);
@@ -121,7 +155,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     uint64_t* tempty = tfull + C::kNumAcc;
     uint64_t* ring_full = tempty + C::kNumAcc;
     uint64_t* ring_empty = ring_full + kFfnRing;
-    uint64_t* drain_bar = ring_empty + kFfnRing;
+    uint64_t* conv_full = ring_empty + kFfnRing;  // C::kConv barriers each (none without FP8 weights)
+    uint64_t* conv_empty = conv_full + C::kConv;
+    uint64_t* drain_bar = conv_empty + C::kConv;
     int* ring = reinterpret_cast<int*>(drain_bar + 1);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kFfnRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -149,7 +185,12 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         }
         for (int r = 0; r < kFfnRing; ++r) {
             mbar_init(&ring_full[r], 1);
-            mbar_init(&ring_empty[r], 1 + 128);  // the MMA thread and every epilogue thread
+            // the MMA thread, every epilogue thread and (FP8) every converter thread
+            mbar_init(&ring_empty[r], 1 + 128 + (kFp8 ? 128 : 0));
+        }
+        for (int c = 0; c < C::kConv; ++c) {
+            mbar_init(&conv_full[c], 128);
+            mbar_init(&conv_empty[c], 1);
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
@@ -281,7 +322,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                 const CUtensorMap* tx = it.phase == 0 ? &tm_xa : &tm_xb;
                 const CUtensorMap* tx64 = it.phase == 0 ? &tm_xa64 : &tm_xb64;
                 const int second = it.phase == 0 ? p.I : 128;  // up rows, or the next 128 features
-                const uint32_t bytes = 2 * C::kWTileBytes + t.mma_n * 128;
+                const uint32_t bytes = 2 * C::kRawWBytes + t.mma_n * 128;
                 const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
@@ -298,8 +339,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                     mbar_arrive_expect_tx(&full[s], bytes);
                     const int kx = k * C::kBK;
                     tma_load_2d(st, tw, &full[s], kx, t.wrow, pol_w);
-                    tma_load_2d(st + C::kWTileBytes, tw, &full[s], kx, t.wrow + second, pol_w);
-                    uint8_t* xs = st + 2 * C::kWTileBytes;
+                    tma_load_2d(st + C::kRawWBytes, tw, &full[s], kx, t.wrow + second, pol_w);
+                    uint8_t* xs = st + 2 * C::kRawWBytes;
                     int r = 0;
                     if (kMaxN >= C::kXBoxMid)
                         for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
@@ -345,7 +386,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + b * C::kAccCols;
                 const uint32_t d1 = d0 + kMaxN;
-                const uint32_t idesc = umma_idesc(Elt<T>::kMmaFmt, 128, t.mma_n);
+                const uint32_t idesc = umma_idesc(kFp8 ? Elt<__half>::kMmaFmt : Elt<T>::kMmaFmt, 128, t.mma_n);
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
                     const uint32_t ph = (kc / C::kStages) & 1u;
@@ -353,11 +394,22 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     uint8_t* st = stage_base + s * C::kStageBytes;
-                    const uint64_t a0 = umma_desc_sw128(smem_u32(st));
-                    const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
-                    const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kWTileBytes));
+                    uint8_t* wt = st;  // the weight tiles the MMA reads
+                    int cv = 0;
+                    if constexpr (kFp8) {
+                        // ... widened to bf16 by the converter warps
+                        cv = (int)(kc % C::kConv);
+                        if (!mbar_wait_bounded(&conv_full[cv], (kc / C::kConv) & 1u, limit, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        wt = conv_base + cv * C::kConvBytes;
+                    }
+                    tc_fence_after();
+                    const uint64_t a0 = umma_desc_sw128(smem_u32(wt));
+                    const uint64_t a1 = umma_desc_sw128(smem_u32(wt + C::kWTileBytes));
+                    const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
@@ -365,6 +417,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                         umma<T>(d1, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
                     }
                     umma_commit(&empty[s]);
+                    if constexpr (kFp8) umma_commit(&conv_empty[cv]);
                 }
                 if (!ok) break;
                 umma_commit(&tfull[b]);
@@ -376,6 +429,64 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                 umma_commit(drain_bar);
                 mbar_drain(drain_bar, 0, limit);
             }
+        }
+    } else if (kFp8 && warp >= 6) {
+        // ------------------------------------------- FP8 -> f16 converters
+        // a stage's two tiles are 2 x 128 rows x 4 chunks of 16 codes; pass j
+        // of thread i takes chunk (j * 128 + i): consecutive lanes read
+        // consecutive 16-byte chunks (8 rows x 64 bytes per warp, no bank
+        // conflict) and write the two f16 chunks at the 128-byte swizzle's
+        // positions (chunk c of row r at c ^ (r mod 8))
+        const int i = (int)threadIdx.x - 192;
+        uint32_t kc = 0, n = 0;
+        bool ok = true;
+        while (ok) {
+            const int rs = n % kFfnRing;
+            const uint32_t rph = (n / kFfnRing) & 1u;
+            if (!mbar_wait_bounded(&ring_full[rs], rph, limit, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const long long id = ring[rs];
+            mbar_arrive(&ring_empty[rs]);
+            ++n;
+            if (id < 0) break;
+            FfnItem it;
+            Tile t;
+            item_of(id, it, t);
+            for (int k = it.kb; k < it.ke; ++k, ++kc) {
+                const int s = kc % C::kStages;
+                const int cv = (int)(kc % C::kConv);
+                if (!mbar_wait_bounded(&full[s], (kc / C::kStages) & 1u, limit, abort_flag) ||
+                    !mbar_wait_bounded(&conv_empty[cv], ((kc / C::kConv) & 1u) ^ 1u, limit, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* src = stage_base + s * C::kStageBytes;
+                uint8_t* dst = conv_base + cv * C::kConvBytes;
+                constexpr int kChunks = C::kBK / 16;  // 16-code chunks per row
+#pragma unroll
+                for (int j = 0; j < 2 * 128 * kChunks / 128; ++j) {
+                    const int idx = j * 128 + i;
+                    const int tt = idx / (128 * kChunks);
+                    const int row = (idx % (128 * kChunks)) / kChunks;
+                    const int q = idx % kChunks;
+                    const uint4 v = *reinterpret_cast<const uint4*>(src + tt * C::kRawWBytes + row * C::kBK + 16 * q);
+                    const uint4 lo = make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
+                                                e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
+                    const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
+                                                e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+                    uint8_t* orow = dst + tt * C::kWTileBytes + row * 128;
+                    *reinterpret_cast<uint4*>(orow + (((2 * q) ^ (row & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(orow + (((2 * q + 1) ^ (row & 7)) << 4)) = hi;
+                }
+                fence_proxy_async_shared();  // the tensor core reads what these generic stores wrote
+                mbar_arrive(&conv_full[cv]);
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            atomicOr(p.status, kStatusTimeout);
         }
     } else {
         // --------------------------------------------------------- epilogue
@@ -411,13 +522,40 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
             const int f = t.f0 + r;
             const bool v0 = f < n_out;
             const bool v1 = gate_up ? v0 : (f + 128 < n_out);
-            OutT* orow = reinterpret_cast<OutT*>(gate_up ? p.act : p.y) + (long long)t.row0 * n_out + f;
+            // FP8 weights: the activations are f16 (the next MMA's operand)
+            using ActT = typename std::conditional<kFp8, __half, OutT>::type;
+            OutT* orow = reinterpret_cast<OutT*>(p.y) + (long long)t.row0 * n_out + f;
+            ActT* arow = reinterpret_cast<ActT*>(p.act) + (long long)t.row0 * n_out + f;
+            // FP8 weights: the row scales of the two accumulators' weight rows
+            float sc0 = 1.f, sc1 = 1.f;
+            if constexpr (kFp8) {
+                if (gate_up) {
+                    const float* sr = p.s13 + (long long)t.group * 2 * p.I;
+                    sc0 = v0 ? __ldg(sr + f) : 0.f;
+                    sc1 = v0 ? __ldg(sr + p.I + f) : 0.f;
+                } else {
+                    const float* sr = p.s2 + (long long)t.group * p.H;
+                    sc0 = v0 ? __ldg(sr + f) : 0.f;
+                    sc1 = v1 ? __ldg(sr + f + 128) : 0.f;
+                }
+            }
             auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {
+                if constexpr (kFp8) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        g[i] *= sc0;
+                        u[i] *= sc1;
+                    }
+                }
                 if (gate_up) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
                 }
-                if (v0) {
+                if (v0 && gate_up) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.nrows) store_out<ActT>(arow + (long long)(c0 + i) * n_out, g[i]);
+                } else if (v0) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         if (c0 + i < t.nrows) store_out<OutT>(orow + (long long)(c0 + i) * n_out, g[i]);

@@ -30,9 +30,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // [rows, kdim] row-major, box = box_rows x row_bytes (128 or 64) with the
-// swizzle of that width, out-of-range elements read as zero.
+// swizzle of that width (or none), out-of-range elements read as zero.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void* base, long long rows, int kdim,
-              int box_rows, int row_bytes = 128) {
+              int box_rows, int row_bytes = 128, bool swizzled = true) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(kdim), static_cast<cuuint64_t>(rows)};
@@ -40,7 +40,8 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void*
     cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes / elt_bytes), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    !swizzled ? CU_TENSOR_MAP_SWIZZLE_NONE
+                              : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B),
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -174,10 +175,10 @@ size_t ctl_block_bytes(int num_sms) {
 
 namespace {
 
-template <typename T, int kMaxN>
+template <typename T, int kMaxN, bool kFp8>
 int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t stream) {
-    using C = FfnCfg<T, kMaxN>;
-    auto kern = moe_ffn_stream_kernel<T, kMaxN>;
+    using C = FfnCfg<T, kMaxN, kFp8>;
+    auto kern = moe_ffn_stream_kernel<T, kMaxN, kFp8>;
     static bool attr_done = false;
     if (!attr_done) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
@@ -191,12 +192,24 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     CUtensorMap w13, w2, xa, xa64, xb, xb64;
     const int eb = Elt<T>::kBytes;
     const CUtensorMapDataType dt = Elt<T>::kTma;
-    if (!make_map(&w13, dt, eb, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128)) return -3;
-    if (!make_map(&w2, dt, eb, L.w2, (long long)L.n_groups * L.H, L.I, 128)) return -3;
-    if (!make_map(&xa, dt, eb, L.x, L.x_rows, L.H, 16)) return -3;
-    if (!make_map(&xa64, dt, eb, L.x, L.x_rows, L.H, 64)) return -3;
-    if (!make_map(&xb, dt, eb, L.act, L.x_rows, L.I, 16)) return -3;
-    if (!make_map(&xb64, dt, eb, L.act, L.x_rows, L.I, 64)) return -3;
+    if (kFp8) {
+        // E4M3 codes: 64-code rows (one stage's K), no swizzle; the converters re-lay them out
+        if (!make_map(&w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128,
+                      C::kBK, false))
+            return -3;
+        if (!make_map(&w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w2, (long long)L.n_groups * L.H, L.I, 128, C::kBK,
+                      false))
+            return -3;
+    } else {
+        if (!make_map(&w13, dt, eb, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128)) return -3;
+        if (!make_map(&w2, dt, eb, L.w2, (long long)L.n_groups * L.H, L.I, 128)) return -3;
+    }
+    // token operands: f16 on the FP8 path (x_perm and the activations), else the activation dtype
+    const CUtensorMapDataType xdt = kFp8 ? Elt<__half>::kTma : dt;
+    if (!make_map(&xa, xdt, eb, L.x, L.x_rows, L.H, 16)) return -3;
+    if (!make_map(&xa64, xdt, eb, L.x, L.x_rows, L.H, 64)) return -3;
+    if (!make_map(&xb, xdt, eb, L.act, L.x_rows, L.I, 16)) return -3;
+    if (!make_map(&xb64, xdt, eb, L.act, L.x_rows, L.I, 64)) return -3;
     FfnParams p;
     p.seg_offsets = L.seg_offsets;
     p.n_groups = L.n_groups;
@@ -211,8 +224,10 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     p.wait_limit_ns = wait_limit_ns();
     p.withhold_first_load = take_withhold_flag();
     p.max_slots_phase = slots_total / 2;
+    p.s13 = L.s13;
+    p.s2 = L.s2;
     const int grid = L.sms > 0 && L.sms < num_sms ? L.sms : num_sms;
-    cudaError_t e = launch_kernel(kern, dim3(grid), dim3(kFfnThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
+    cudaError_t e = launch_kernel(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
                                   xb, xb64, p);
     count_launch();
     if (e != cudaSuccess) cudaGetLastError();
@@ -234,15 +249,21 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
     if ((ntiles_a < 2LL * G && ntiles_a > kFfnTileCtrs / 2) || (ntiles_b < 2LL * G && ntiles_b > kFfnTileCtrs / 2))
         return 1;
     if (L.x_rows <= 0) return 0;
+    if (L.fp8) {
+        if (L.dtype != 0 || !L.s13 || !L.s2) return -1;
+        if (L.max_n == 32) return launch_ffn_variant<__nv_bfloat16, 32, true>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 64) return launch_ffn_variant<__nv_bfloat16, 64, true>(L, ctl, d.num_sms, stream);
+        return launch_ffn_variant<__nv_bfloat16, 128, true>(L, ctl, d.num_sms, stream);
+    }
     if (L.dtype == 0) {
-        if (L.max_n == 32) return launch_ffn_variant<__nv_bfloat16, 32>(L, ctl, d.num_sms, stream);
-        if (L.max_n == 64) return launch_ffn_variant<__nv_bfloat16, 64>(L, ctl, d.num_sms, stream);
-        return launch_ffn_variant<__nv_bfloat16, 128>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 32) return launch_ffn_variant<__nv_bfloat16, 32, false>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 64) return launch_ffn_variant<__nv_bfloat16, 64, false>(L, ctl, d.num_sms, stream);
+        return launch_ffn_variant<__nv_bfloat16, 128, false>(L, ctl, d.num_sms, stream);
     }
     if (L.dtype == 1) {
-        if (L.max_n == 32) return launch_ffn_variant<float, 32>(L, ctl, d.num_sms, stream);
-        if (L.max_n == 64) return launch_ffn_variant<float, 64>(L, ctl, d.num_sms, stream);
-        return launch_ffn_variant<float, 128>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 32) return launch_ffn_variant<float, 32, false>(L, ctl, d.num_sms, stream);
+        if (L.max_n == 64) return launch_ffn_variant<float, 64, false>(L, ctl, d.num_sms, stream);
+        return launch_ffn_variant<float, 128, false>(L, ctl, d.num_sms, stream);
     }
     return -1;
 }

@@ -260,6 +260,10 @@ __device__ __forceinline__ void store_out(OutT* ptr, float v);
 template <>
 __device__ __forceinline__ void store_out<float>(float* ptr, float v) { *ptr = v; }
 template <>
+__device__ __forceinline__ void store_out<__half>(__half* ptr, float v) {
+    *ptr = __float2half_rn(v);
+}
+template <>
 __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* ptr, float v) {
     *ptr = __float2bfloat16_rn(v);
 }

@@ -124,6 +124,9 @@ struct FfnLaunch {
     int max_n;
     long long max_chunks;  // upper bound on token chunks (host side)
     int sms;               // persistent blocks at most (0 = one per SM)
+    bool fp8 = false;      // w13 / w2 are E4M3 codes with fp32 row scales s13 [n_groups*2I], s2 [n_groups*H]
+    const float* s13 = nullptr;
+    const float* s2 = nullptr;
 };
 int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 
@@ -152,10 +155,17 @@ int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int
                        const int32_t* k_per_token, float* part, float* logits, int32_t* ids, float* w,
                        int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos,
                        int32_t* scalars, int32_t* stats_copy, int* done_ctr, cudaStream_t stream);
+// to_f16: bf16 x written to x_perm as f16 (the FP8-weight path's operand type)
 int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
-                   const int32_t* scalars, void* x_perm, cudaStream_t stream);
+                   const int32_t* scalars, void* x_perm, cudaStream_t stream, bool to_f16 = false);
+// n bf16 values -> f16 (n a multiple of 8)
+int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stream);
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
                    const void* shared_out, void* out, cudaStream_t stream);
+
+// Row-wise FP8 E4M3 quantisation: q [rows, cols] codes, scales [rows].
+int launch_quantize_fp8(long long rows, int cols, int dtype, const void* w, uint8_t* q, float* scales,
+                        cudaStream_t stream);
 
 // Launch bookkeeping.
 void count_launch();

@@ -495,6 +495,17 @@ int launch_align(int T, int K, int E, int B, int mode, long long P_max, const in
 
 // ---------------------------------------------------------------- permute
 // x_perm[p] = x[sorted_ids[p] / K] (zero row for a padding slot), p < P.
+// 8 bf16 -> 8 f16 (the FP8-weight path computes on f16 operands)
+__device__ __forceinline__ int4 bf16x8_to_f16x8(int4 v) {
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+    int4 o;
+    __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(__bfloat1622float2(b[i]));
+    return o;
+}
+
+template <bool kToF16>
 __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const int4* __restrict__ x,
                                                       const int32_t* __restrict__ sorted_ids,
                                                       const int32_t* __restrict__ scalars, int4* __restrict__ x_perm) {
@@ -508,7 +519,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const 
         int4* dst = x_perm + p * row_vec;
         if (src >= 0) {
             const int4* s = x + (long long)(src / K) * row_vec;
-            for (int v = l; v < row_vec; v += 64) dst[v] = __ldg(s + v);
+            for (int v = l; v < row_vec; v += 64) dst[v] = kToF16 ? bf16x8_to_f16x8(__ldg(s + v)) : __ldg(s + v);
         } else {
             const int4 z = make_int4(0, 0, 0, 0);
             for (int v = l; v < row_vec; v += 64) dst[v] = z;
@@ -517,7 +528,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const 
 }
 
 int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
-                   const int32_t* scalars, void* x_perm, cudaStream_t stream) {
+                   const int32_t* scalars, void* x_perm, cudaStream_t stream, bool to_f16) {
     if (P_max <= 0) return 0;
     DeviceInfo d;
     int rc = current_device(&d);
@@ -528,8 +539,34 @@ int launch_permute(int H, int K, int dtype, long long P_max, const void* x, cons
     long long blocks = (P_max + rows_per_block - 1) / rows_per_block;
     const long long cap = (long long)d.num_sms * 8;
     if (blocks > cap) blocks = cap;
-    cudaError_t e = launch_kernel(permute_kernel, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
-                                  static_cast<const int4*>(x), sorted_ids, scalars, static_cast<int4*>(x_perm));
+    if (to_f16 && dtype != 0) return -1;
+    cudaError_t e = to_f16 ? launch_kernel(permute_kernel<true>, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
+                                           static_cast<const int4*>(x), sorted_ids, scalars,
+                                           static_cast<int4*>(x_perm))
+                           : launch_kernel(permute_kernel<false>, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
+                                           static_cast<const int4*>(x), sorted_ids, scalars,
+                                           static_cast<int4*>(x_perm));
+    count_launch();
+    return launched(e);
+}
+
+// bf16 rows -> f16 rows (n_vec vectors of 8), for the shared FFN on FP8 weights
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(long long n_vec, const int4* __restrict__ in,
+                                                          int4* __restrict__ out) {
+    pdl_launch_dependents();
+    pdl_wait();
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += (long long)gridDim.x * blockDim.x)
+        out[i] = bf16x8_to_f16x8(__ldg(in + i));
+}
+
+int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stream) {
+    if (n <= 0) return 0;
+    if (n % 8) return -1;
+    const long long n_vec = n / 8;
+    long long blocks = (n_vec + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    cudaError_t e = launch_kernel(bf16_to_f16_kernel, dim3((int)blocks), dim3(256), 0, stream, n_vec,
+                                  static_cast<const int4*>(in), static_cast<int4*>(out));
     count_launch();
     return launched(e);
 }
@@ -628,6 +665,42 @@ int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int
                                                stream, T, row_vec, K, y4, pos, w, s4, o4)
                                : launch_kernel(combine_kernel<float>, dim3((int)blocks), dim3(threads), 0, stream, T,
                                                row_vec, K, y4, pos, w, s4, o4);
+    count_launch();
+    return launched(e);
+}
+
+// ------------------------------------------------------ FP8 quantisation
+// Row-wise E4M3 codes for the decode weight stream: one block per row, the
+// row's max |w| by a block reduction, scale = max / 448 (1 for an all-zero
+// row), code = E4M3(w / scale) rounded to nearest even with saturation.  The
+// divisions are IEEE (correctly rounded) so that the codes are reproducible.
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_fp8_kernel(int cols, const T* __restrict__ w,
+                                                           uint8_t* __restrict__ q, float* __restrict__ scales) {
+    __shared__ float red[8];
+    const long long row = blockIdx.x;
+    const T* wr = w + row * cols;
+    float amax = 0.f;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) amax = fmaxf(amax, fabsf(Elt<T>::to_f(wr[c])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) amax = fmaxf(amax, red[i]);
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    if (threadIdx.x == 0) scales[row] = sc;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x)
+        q[row * cols + c] = __nv_cvt_float_to_fp8(__fdiv_rn(Elt<T>::to_f(wr[c]), sc), __NV_SATFINITE, __NV_E4M3);
+}
+
+int launch_quantize_fp8(long long rows, int cols, int dtype, const void* w, uint8_t* q, float* scales,
+                        cudaStream_t stream) {
+    if (rows == 0) return 0;
+    cudaError_t e = dtype == 0 ? launch_kernel(quantize_fp8_kernel<__nv_bfloat16>, dim3((unsigned)rows), dim3(256), 0,
+                                               stream, cols, static_cast<const __nv_bfloat16*>(w), q, scales)
+                               : launch_kernel(quantize_fp8_kernel<float>, dim3((unsigned)rows), dim3(256), 0, stream,
+                                               cols, static_cast<const float*>(w), q, scales);
     count_launch();
     return launched(e);
 }
