@@ -26,10 +26,11 @@
 // small shared-memory ring.
 //
 // FP8 weights (kFp8): the weight tiles stream as E4M3 codes (half the bytes),
-// 128 rows x 64 codes per tile without swizzle; warps 6..9 widen each stage's
-// two tiles to f16 (one cvt per pair of codes; E4M3 values are exact in f16)
-// into a ring of conversion buffers in the 128-byte swizzled layout the MMA
-// reads, and the epilogue multiplies each output row by its fp32 row scale.
+// 128 rows x 64 codes per tile without swizzle; warps 6..13 widen each
+// stage's two tiles to f16 by moving the code's bits into an f16 pattern
+// (value x 2^-8, exact: E4M3 subnormals land on f16 subnormals) into a ring of
+// conversion buffers in the 128-byte swizzled layout the MMA reads, and the
+// epilogue multiplies each output row by its fp32 row scale x 2^8.
 // The MMAs then run on f16 operands: x_perm arrives in f16 and the SwiGLU
 // activations are stored in f16 (the output stays in the activation dtype).
 #pragma once
@@ -74,7 +75,8 @@ struct FfnCfg {
     static constexpr int kStageBytes = 2 * kRawWBytes + kXTileBytes;
     static constexpr int kConv = kFp8 ? (kMaxN <= 64 ? 3 : 2) : 0;       // f16 conversion buffers
     static constexpr int kConvBytes = 2 * kWTileBytes;
-    static constexpr int kThreads = kFp8 ? 320 : kFfnThreads;
+    static constexpr int kConvThreads = kFp8 ? 256 : 0;   // converter warps 6..13
+    static constexpr int kThreads = kFfnThreads + kConvThreads;
     static constexpr int kAccCols = 2 * kMaxN;
     static constexpr int kNumAcc = 2;
     static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
@@ -128,10 +130,23 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Two E4M3 codes (low byte first) -> two f16 (exact), one conversion instruction.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-    return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+// Two E4M3 codes at bits [7:0] and [23:16] -> two f16 holding value x 2^-8:
+// the sign moves to bit 15, the 4 exponent and 3 mantissa bits to bits 13:7,
+// so an E4M3 exponent field e becomes the f16 exponent field e (bias 15 vs 7)
+// and e = 0 (subnormal) stays subnormal -- exact for every finite code.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t two) {
+    return ((two << 8) & 0x80008000u) | ((two << 7) & 0x3F803F80u);
+}
+// 16 codes -> 16 f16 (value x 2^-8) in two 16-byte chunks
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, uint4& lo, uint4& hi) {
+    lo = make_uint4(e4m3x2_to_f16x2_scaled(__byte_perm(v.x, 0, 0x4140)),
+                    e4m3x2_to_f16x2_scaled(__byte_perm(v.x, 0, 0x4342)),
+                    e4m3x2_to_f16x2_scaled(__byte_perm(v.y, 0, 0x4140)),
+                    e4m3x2_to_f16x2_scaled(__byte_perm(v.y, 0, 0x4342)));
+    hi = make_uint4(e4m3x2_to_f16x2_scaled(__byte_perm(v.z, 0, 0x4140)),
+                    e4m3x2_to_f16x2_scaled(__byte_perm(v.z, 0, 0x4342)),
+                    e4m3x2_to_f16x2_scaled(__byte_perm(v.w, 0, 0x4140)),
+                    e4m3x2_to_f16x2_scaled(__byte_perm(v.w, 0, 0x4342)));
 }
 
 template <typename T, int kMaxN, bool kFp8 = false>
@@ -186,10 +201,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         for (int r = 0; r < kFfnRing; ++r) {
             mbar_init(&ring_full[r], 1);
             // the MMA thread, every epilogue thread and (FP8) every converter thread
-            mbar_init(&ring_empty[r], 1 + 128 + (kFp8 ? 128 : 0));
+            mbar_init(&ring_empty[r], 1 + 128 + C::kConvThreads);
         }
         for (int c = 0; c < C::kConv; ++c) {
-            mbar_init(&conv_full[c], 128);
+            mbar_init(&conv_full[c], C::kConvThreads);
             mbar_init(&conv_empty[c], 1);
         }
         mbar_init(drain_bar, 1);
@@ -430,10 +445,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 mbar_drain(drain_bar, 0, limit);
             }
         }
-    } else if (kFp8 && warp >= 6) {
+    } else if (kFp8 && warp >= 6) {  // converter warps 6 .. 5 + kConvThreads / 32
         // ------------------------------------------- FP8 -> f16 converters
         // a stage's two tiles are 2 x 128 rows x 4 chunks of 16 codes; pass j
-        // of thread i takes chunk (j * 128 + i): consecutive lanes read
+        // of thread i takes chunk (j * kConvThreads + i): consecutive lanes read
         // consecutive 16-byte chunks (8 rows x 64 bytes per warp, no bank
         // conflict) and write the two f16 chunks at the 128-byte swizzle's
         // positions (chunk c of row r at c ^ (r mod 8))
@@ -466,16 +481,14 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 uint8_t* dst = conv_base + cv * C::kConvBytes;
                 constexpr int kChunks = C::kBK / 16;  // 16-code chunks per row
 #pragma unroll
-                for (int j = 0; j < 2 * 128 * kChunks / 128; ++j) {
-                    const int idx = j * 128 + i;
+                for (int j = 0; j < 2 * 128 * kChunks / C::kConvThreads; ++j) {
+                    const int idx = j * C::kConvThreads + i;
                     const int tt = idx / (128 * kChunks);
                     const int row = (idx % (128 * kChunks)) / kChunks;
                     const int q = idx % kChunks;
                     const uint4 v = *reinterpret_cast<const uint4*>(src + tt * C::kRawWBytes + row * C::kBK + 16 * q);
-                    const uint4 lo = make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
-                                                e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
-                    const uint4 hi = make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
-                                                e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+                    uint4 lo, hi;
+                    e4m3x16_to_f16(v, lo, hi);
                     uint8_t* orow = dst + tt * C::kWTileBytes + row * 128;
                     *reinterpret_cast<uint4*>(orow + (((2 * q) ^ (row & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(orow + (((2 * q + 1) ^ (row & 7)) << 4)) = hi;
@@ -526,17 +539,18 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             using ActT = typename std::conditional<kFp8, __half, OutT>::type;
             OutT* orow = reinterpret_cast<OutT*>(p.y) + (long long)t.row0 * n_out + f;
             ActT* arow = reinterpret_cast<ActT*>(p.act) + (long long)t.row0 * n_out + f;
-            // FP8 weights: the row scales of the two accumulators' weight rows
+            // FP8 weights: the row scales of the two accumulators' weight rows,
+            // times 2^8 (the widened codes hold value x 2^-8)
             float sc0 = 1.f, sc1 = 1.f;
             if constexpr (kFp8) {
                 if (gate_up) {
                     const float* sr = p.s13 + (long long)t.group * 2 * p.I;
-                    sc0 = v0 ? __ldg(sr + f) : 0.f;
-                    sc1 = v0 ? __ldg(sr + p.I + f) : 0.f;
+                    sc0 = v0 ? __ldg(sr + f) * 256.f : 0.f;
+                    sc1 = v0 ? __ldg(sr + p.I + f) * 256.f : 0.f;
                 } else {
                     const float* sr = p.s2 + (long long)t.group * p.H;
-                    sc0 = v0 ? __ldg(sr + f) : 0.f;
-                    sc1 = v1 ? __ldg(sr + f + 128) : 0.f;
+                    sc0 = v0 ? __ldg(sr + f) * 256.f : 0.f;
+                    sc1 = v1 ? __ldg(sr + f + 128) * 256.f : 0.f;
                 }
             }
             auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {

@@ -100,3 +100,31 @@ def test_fp8_layer_rejects_prefill_sizes():
     with pytest.raises(moe.MoeError) as e:
         moe.layer_forward_fp8(cfg, x, w["w_r"], q13, s13, q2, s2, ws)
     assert e.value.code == -1
+
+
+def test_fp8_subnormal_codes_are_kept():
+    # gate/up rows of one large weight (it sets the scale) and many tiny ones
+    # that quantise to E4M3 subnormals; the large weights meet x = 0, so the
+    # output comes from the subnormal codes alone and would vanish if the
+    # widening or the tensor core dropped them
+    T, H, I = 16, 256, 128
+    rng = np.random.default_rng(77)
+    w13 = rng.uniform(-0.03, 0.03, (2 * I, H)).astype(np.float32)
+    w13[:, 0] = 1000.0                       # scale 1000/448: the rest are below 2^-6 x scale
+    w2 = (rng.standard_normal((H, I)) / np.sqrt(I)).astype(np.float32)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    x[:, 0] = 0.0
+    dev = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)
+    w13_d, w2_d, x_d = dev(w13), dev(w2), dev(x)
+    q13, s13 = moe.quantize_fp8(w13_d)
+    q2, s2 = moe.quantize_fp8(w2_d)
+    codes = q13.cpu().numpy()[:, 1:]
+    assert np.mean((codes & 0x78) == 0) > 0.95              # exponent field 0: subnormal (or zero)
+    ws = moe.alloc_workspace(moe.dense_fp8_workspace_size(T, H, I))
+    out = moe.dense_ffn_fp8(x_d, q13, s13, q2, s2, ws)
+    moe.check_status(ws)
+    c = lambda t: t.cpu().numpy()
+    ref = oracle.moe_layer_fp8(host(x_d), None, c(q13)[None], c(s13)[None], c(q2)[None], c(s2)[None], 1,
+                               logits=np.zeros((T, 1), np.float32))
+    assert np.abs(ref).max() > 0
+    assert rel_err(out.float().cpu().numpy(), ref) < OUT_TOL
