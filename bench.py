@@ -602,7 +602,7 @@ def main():
                    "padding": "max-value" if args.pad_mode == 1 else "block-wise",
                    "top_k": (f"per-token dynamic, uniform 1..{shape.K} (sum {wl.A})" if args.dynamic_k
                              else f"{shape.K} for every token"),
-                   "expert_weights": ("FP8 E4M3 codes + fp32 row scales (widened to bf16 in shared memory)"
+                   "expert_weights": ("FP8 E4M3 codes + fp32 row scales (widened to f16 in shared memory, f16 MMAs)"
                                       if args.fp8 else shape.dtype)},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - wl.A) / max(P, 1), 4),
