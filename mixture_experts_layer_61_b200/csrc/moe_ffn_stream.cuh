@@ -26,12 +26,16 @@
 // small shared-memory ring.
 //
 // FP8 weights (kFp8): the weight tiles stream as E4M3 codes (half the bytes),
-// 128 rows x 64 codes per tile without swizzle; warps 6..13 widen each
-// stage's two tiles to f16 by moving the code's bits into an f16 pattern
-// (value x 2^-8, exact: E4M3 subnormals land on f16 subnormals) into a ring of
-// conversion buffers in the 128-byte swizzled layout the MMA reads, and the
-// epilogue multiplies each output row by its fp32 row scale x 2^8.
-// The MMAs then run on f16 operands: x_perm arrives in f16 and the SwiGLU
+// 128 rows x 64 codes per tile with the 64-byte swizzle; warps 6..13 widen
+// each stage's two tiles to f16 in registers by moving the code's bits into an
+// f16 pattern (value x 2^-8, exact: E4M3 subnormals land on f16 subnormals)
+// and store them into a ring of TMEM buffers, from which the MMA takes its A
+// operand; the epilogue multiplies each output row by its fp32 row scale x 2^8.
+// Widening through shared memory instead costs 6 bytes of shared-memory
+// traffic per weight (TMA write, read, f16 write, tensor-core read) against 2
+// for bf16 weights, which caps the stream below the bf16 rate; through TMEM
+// the shared-memory traffic stays at 2 bytes per weight.
+// The MMAs run on f16 operands: x_perm arrives in f16 and the SwiGLU
 // activations are stored in f16 (the output stays in the activation dtype).
 #pragma once
 
@@ -73,19 +77,19 @@ struct FfnCfg {
     static constexpr int kXBoxRows = 16, kXBoxMid = 64;
     static constexpr int kXTileBytes = kMaxN * 128;
     static constexpr int kStageBytes = 2 * kRawWBytes + kXTileBytes;
-    static constexpr int kConv = kFp8 ? (kMaxN <= 64 ? 3 : 2) : 0;       // f16 conversion buffers
-    static constexpr int kConvBytes = 2 * kWTileBytes;
+    static constexpr int kConv = kFp8 ? (kMaxN <= 64 ? 3 : 2) : 0;  // TMEM buffers of widened weights
+    static constexpr int kConvCols = 64;   // a stage's two 128 x 64 f16 tiles: 2 x 32 TMEM columns
     static constexpr int kConvThreads = kFp8 ? 256 : 0;   // converter warps 6..13
     static constexpr int kThreads = kFfnThreads + kConvThreads;
     static constexpr int kAccCols = 2 * kMaxN;
-    static constexpr int kNumAcc = 2;
+    static constexpr int kNumAcc = (kFp8 && kMaxN == 128) ? 1 : 2;  // leaves TMEM room for the weight buffers
+    static constexpr int kConvCol0 = kNumAcc * kAccCols;
     static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
     static constexpr int kMiscBytes = 768;
-    static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes - kConv * kConvBytes;
+    static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes;
     static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kSmemBytes =
-        1024 + kStages * kStageBytes + kConv * kConvBytes + kTableBytes + kMiscBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
     static_assert(kStageBytes % 1024 == 0, "stages keep the swizzle atoms aligned");
     static_assert(!kFp8 || sizeof(T) == 2, "FP8 weights: 16-bit activations");
     // barriers (full/empty per stage, 2 TMEM pairs, the item ring, the conversion
@@ -94,7 +98,7 @@ struct FfnCfg {
                   "misc area");
     static constexpr int kSlotFloats = 128 * kAccCols;
     static_assert(kMaxN == 32 || kMaxN == 64 || kMaxN == 128, "decode token tiles");
-    static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
+    static_assert(kAccCols * kNumAcc + kConv * kConvCols <= 512, "TMEM columns");
 };
 
 // One phase's split: S slices per tile (S = 1: whole tiles).
@@ -124,10 +128,6 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const int* p) {
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_shared() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Two E4M3 codes at bits [7:0] and [23:16] -> two f16 holding value x 2^-8:
@@ -160,8 +160,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_base = smem;
-    uint8_t* conv_base = smem + C::kStages * C::kStageBytes;
-    int* seg = reinterpret_cast<int*>(conv_base + C::kConv * C::kConvBytes);
+    int* seg = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes);
     int* cbase = seg + (kMaxGroups + 1);
     uint8_t* misc = reinterpret_cast<uint8_t*>(cbase + (kMaxGroups + 1));
     uint64_t* full = reinterpret_cast<uint64_t*>(misc);
@@ -204,7 +203,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             mbar_init(&ring_empty[r], 1 + 128 + C::kConvThreads);
         }
         for (int c = 0; c < C::kConv; ++c) {
-            mbar_init(&conv_full[c], C::kConvThreads);
+            mbar_init(&conv_full[c], C::kConvThreads / 32);  // one arrival per converter warp
             mbar_init(&conv_empty[c], 1);
         }
         mbar_init(drain_bar, 1);
@@ -410,26 +409,33 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         break;
                     }
                     uint8_t* st = stage_base + s * C::kStageBytes;
-                    uint8_t* wt = st;  // the weight tiles the MMA reads
+                    const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
                     int cv = 0;
                     if constexpr (kFp8) {
-                        // ... widened to bf16 by the converter warps
+                        // A: the stage's two tiles, widened to f16 in TMEM by the converter warps
                         cv = (int)(kc % C::kConv);
                         if (!mbar_wait_bounded(&conv_full[cv], (kc / C::kConv) & 1u, limit, abort_flag)) {
                             ok = false;
                             break;
                         }
-                        wt = conv_base + cv * C::kConvBytes;
-                    }
-                    tc_fence_after();
-                    const uint64_t a0 = umma_desc_sw128(smem_u32(wt));
-                    const uint64_t a1 = umma_desc_sw128(smem_u32(wt + C::kWTileBytes));
-                    const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
+                        tc_fence_after();
+                        const uint32_t a0 = tmem_base + C::kConvCol0 + cv * C::kConvCols;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
-                        umma<T>(d0, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
-                        umma<T>(d1, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
+                            umma_f16_tmem_a(d0, a0 + 8 * kk, bx + 2 * kk, idesc, acc);
+                            umma_f16_tmem_a(d1, a0 + 32 + 8 * kk, bx + 2 * kk, idesc, acc);
+                        }
+                    } else {
+                        tc_fence_after();
+                        const uint64_t a0 = umma_desc_sw128(smem_u32(st));
+                        const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
+                            umma<T>(d0, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                            umma<T>(d1, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                        }
                     }
                     umma_commit(&empty[s]);
                     if constexpr (kFp8) umma_commit(&conv_empty[cv]);
@@ -447,12 +453,16 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         }
     } else if (kFp8 && warp >= 6) {  // converter warps 6 .. 5 + kConvThreads / 32
         // ------------------------------------------- FP8 -> f16 converters
-        // a stage's two tiles are 2 x 128 rows x 4 chunks of 16 codes; pass j
-        // of thread i takes chunk (j * kConvThreads + i): consecutive lanes read
-        // consecutive 16-byte chunks (8 rows x 64 bytes per warp, no bank
-        // conflict) and write the two f16 chunks at the 128-byte swizzle's
-        // positions (chunk c of row r at c ^ (r mod 8))
-        const int i = (int)threadIdx.x - 192;
+        // warps 6..9 widen a stage's first weight tile, warps 10..13 its second;
+        // a warp may only store to its TMEM lane quadrant (warp mod 4), so each
+        // thread takes one row (quadrant x 32 + lane): its 64 codes are four
+        // 16-byte chunks, chunk c of row r at chunk position c ^ ((r / 2) mod 4)
+        // under the 64-byte swizzle (8 consecutive rows hit 8 distinct bank
+        // groups), widened to 32 f16 pairs and stored as 32 TMEM columns
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int tt = (warp - 6) >> 2;
+        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
         uint32_t kc = 0, n = 0;
         bool ok = true;
         while (ok) {
@@ -472,29 +482,34 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             for (int k = it.kb; k < it.ke; ++k, ++kc) {
                 const int s = kc % C::kStages;
                 const int cv = (int)(kc % C::kConv);
-                if (!mbar_wait_bounded(&full[s], (kc / C::kStages) & 1u, limit, abort_flag) ||
-                    !mbar_wait_bounded(&conv_empty[cv], ((kc / C::kConv) & 1u) ^ 1u, limit, abort_flag)) {
+                const bool got = mbar_wait_bounded(&full[s], (kc / C::kStages) & 1u, limit, abort_flag) &&
+                                 mbar_wait_bounded(&conv_empty[cv], ((kc / C::kConv) & 1u) ^ 1u, limit, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) {  // the whole warp leaves together (warp-wide TMEM stores)
                     ok = false;
                     break;
                 }
-                const uint8_t* src = stage_base + s * C::kStageBytes;
-                uint8_t* dst = conv_base + cv * C::kConvBytes;
-                constexpr int kChunks = C::kBK / 16;  // 16-code chunks per row
+                tc_fence_after();  // the MMAs that read this buffer before have completed
+                const uint8_t* src = stage_base + s * C::kStageBytes + tt * C::kRawWBytes + row * C::kBK;
+                uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 2 * 128 * kChunks / C::kConvThreads; ++j) {
-                    const int idx = j * C::kConvThreads + i;
-                    const int tt = idx / (128 * kChunks);
-                    const int row = (idx % (128 * kChunks)) / kChunks;
-                    const int q = idx % kChunks;
-                    const uint4 v = *reinterpret_cast<const uint4*>(src + tt * C::kRawWBytes + row * C::kBK + 16 * q);
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(src + ((c ^ ((row >> 1) & 3)) << 4));
                     uint4 lo, hi;
                     e4m3x16_to_f16(v, lo, hi);
-                    uint8_t* orow = dst + tt * C::kWTileBytes + row * 128;
-                    *reinterpret_cast<uint4*>(orow + (((2 * q) ^ (row & 7)) << 4)) = lo;
-                    *reinterpret_cast<uint4*>(orow + (((2 * q + 1) ^ (row & 7)) << 4)) = hi;
+                    w[8 * c + 0] = lo.x;
+                    w[8 * c + 1] = lo.y;
+                    w[8 * c + 2] = lo.z;
+                    w[8 * c + 3] = lo.w;
+                    w[8 * c + 4] = hi.x;
+                    w[8 * c + 5] = hi.y;
+                    w[8 * c + 6] = hi.z;
+                    w[8 * c + 7] = hi.w;
                 }
-                fence_proxy_async_shared();  // the tensor core reads what these generic stores wrote
-                mbar_arrive(&conv_full[cv]);
+                tmem_st32(tmem_base + lane_base + C::kConvCol0 + cv * C::kConvCols + tt * 32, w);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&conv_full[cv]);
             }
         }
         if (!ok) {

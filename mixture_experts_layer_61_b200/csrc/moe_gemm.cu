@@ -193,12 +193,12 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     const int eb = Elt<T>::kBytes;
     const CUtensorMapDataType dt = Elt<T>::kTma;
     if (kFp8) {
-        // E4M3 codes: 64-code rows (one stage's K), no swizzle; the converters re-lay them out
+        // E4M3 codes: 64-code rows (one stage's K) with the 64-byte swizzle, which
+        // spreads the converters' row-per-thread reads over all banks
         if (!make_map(&w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128,
-                      C::kBK, false))
+                      C::kBK))
             return -3;
-        if (!make_map(&w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w2, (long long)L.n_groups * L.H, L.I, 128, C::kBK,
-                      false))
+        if (!make_map(&w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w2, (long long)L.n_groups * L.H, L.I, 128, C::kBK))
             return -3;
     } else {
         if (!make_map(&w13, dt, eb, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128)) return -3;
