@@ -348,3 +348,51 @@ def moe_layer_fp8(x, w_r, q13, s13, q2, s2, K, score_fn=0, renorm=1, q13_sh=None
                                       _ptr(kk), _ptr(tok), n, _ptr(out), nthreads or nthreads_default()),
            "moe_layer_fp8")
     return out
+
+
+# ------------------------------------------------ tensor parallelism over I
+
+def tp_shard(w13, w2, rank, n_ranks):
+    """Rank `rank` of `n_ranks` of a layer split over the expert intermediate
+    dimension I (talk notes, "Demystifying the Mixture of Experts Serving
+    Tax", "Balls-Bins-Buckets framework": under TP the buckets are the n_tp
+    GPUs, each holding a share of every expert).  Reading: every GPU holds,
+    for every expert, the gate rows [r*I/n, (r+1)*I/n) of W1, the same rows of
+    W3 (rows I + that range of the packed [2I, H] matrix) and the same columns
+    of W2, so the FFN of the slice yields W2[:, slice] (silu(W1[slice] x) *
+    W3[slice] x), and the slices' outputs sum to the expert's output.
+
+    w13 [E, 2I, H] / w2 [E, H, I] (or one dense FFN [2I, H] / [H, I]);
+    returns (w13 slice [E, 2I/n, H], w2 slice [E, H, I/n]) as new arrays."""
+    w13 = np.asarray(w13)
+    w2 = np.asarray(w2)
+    I = w2.shape[-1]
+    if n_ranks < 1 or not 0 <= rank < n_ranks or I % n_ranks:
+        raise ValueError("I must split evenly over the ranks")
+    n = I // n_ranks
+    lo, hi = rank * n, (rank + 1) * n
+    g = w13[..., lo:hi, :]
+    u = w13[..., I + lo:I + hi, :]
+    return np.ascontiguousarray(np.concatenate([g, u], axis=-2)), np.ascontiguousarray(w2[..., lo:hi])
+
+
+def moe_layer_tp(x, w_r, w13, w2, K, n_ranks, score_fn=0, renorm=1, w13_sh=None, w2_sh=None, logits=None,
+                 tokens=None, k=None, nthreads=None, partials=False):
+    """The layer under TP over I: every rank routes the same tokens the same
+    way (the router weights are whole on every rank), runs its slice of every
+    expert and of the shared FFN and combines with the gate weights; the
+    all-reduce (talk notes, "Key findings" 3: the AllReduce after the MoE
+    block under TP) sums the ranks' outputs, here in rank order in float64.
+    Returns the sum [n, H], or the list of the ranks' outputs if `partials`."""
+    parts = []
+    for r in range(n_ranks):
+        a13, a2 = tp_shard(w13, w2, r, n_ranks)
+        s13, s2 = (None, None) if w13_sh is None else tp_shard(w13_sh, w2_sh, r, n_ranks)
+        parts.append(moe_layer(x, w_r, a13, a2, K, score_fn=score_fn, renorm=renorm, w13_sh=s13, w2_sh=s2,
+                               logits=logits, tokens=tokens, k=k, nthreads=nthreads))
+    if partials:
+        return parts
+    out = np.zeros_like(parts[0])
+    for p in parts:
+        out += p
+    return out

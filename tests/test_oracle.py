@@ -668,3 +668,65 @@ def test_fp8_layer_equals_float_layer_on_representable_weights():
     f = lambda q, s: (oracle.e4m3_value(q) * s[..., None]).astype(np.float32)
     ref = oracle.moe_layer(x, w_r, f(q13, s13), f(q2, s2), K, w13_sh=f(q13s, s13s), w2_sh=f(q2s, s2s))
     assert np.allclose(out, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+# ------------------------------------------- tensor parallelism over I (oracle)
+
+def test_tp_shard_takes_the_reading_rows_and_columns():
+    # weights whose entries encode their own indices: rank 1 of 3 over I = 6
+    # holds gate rows 2, 3, up rows 6 + 2, 6 + 3 and W2 columns 2, 3
+    E, I, H = 2, 6, 3
+    w13 = np.array([[[1000 * e + 10 * j + h for h in range(H)] for j in range(2 * I)] for e in range(E)],
+                   np.float32)
+    w2 = np.array([[[1000 * e + 10 * h + i for i in range(I)] for h in range(H)] for e in range(E)], np.float32)
+    s13, s2 = oracle.tp_shard(w13, w2, 1, 3)
+    assert s13.shape == (E, 4, H) and s2.shape == (E, H, 2)
+    for e in range(E):
+        assert np.array_equal(s13[e], w13[e][[2, 3, 8, 9]])
+        assert np.array_equal(s2[e], w2[e][:, [2, 3]])
+    d13, d2 = oracle.tp_shard(w13[1], w2[1], 2, 3)  # one dense FFN: rows 4, 5, 10, 11
+    assert np.array_equal(d13, w13[1][[4, 5, 10, 11]]) and np.array_equal(d2, w2[1][:, [4, 5]])
+    one13, one2 = oracle.tp_shard(w13, w2, 0, 1)
+    assert np.array_equal(one13, w13) and np.array_equal(one2, w2)
+    with pytest.raises(ValueError):
+        oracle.tp_shard(w13, w2, 0, 4)  # 6 does not split over 4 ranks
+    with pytest.raises(ValueError):
+        oracle.tp_shard(w13, w2, 3, 3)
+
+
+@pytest.mark.parametrize("n_ranks", [1, 2, 4])
+@pytest.mark.parametrize("score_fn", [0, 1])
+def test_tp_layer_sums_to_the_whole_layer(n_ranks, score_fn):
+    # linearity of the FFN output in the slices of I: the ranks' outputs add
+    # up to the unsplit layer (routed and shared), up to float64 rounding
+    x, w_r, w13, w2, sh = _small_layer(11, T=9, E=6, K=2, I=40, I_sh=24)
+    full = oracle.moe_layer(x, w_r, w13, w2, K=2, score_fn=score_fn, **sh)
+    tp = oracle.moe_layer_tp(x, w_r, w13, w2, 2, n_ranks, score_fn=score_fn, **sh)
+    assert np.allclose(tp, full, rtol=1e-12, atol=1e-13 * np.abs(full).max())
+    if n_ranks > 1:
+        parts = oracle.moe_layer_tp(x, w_r, w13, w2, 2, n_ranks, score_fn=score_fn, partials=True, **sh)
+        assert len(parts) == n_ranks
+        assert all(np.abs(p - full).max() > 1e-3 * np.abs(full).max() for p in parts)
+
+
+def test_tp_dense_slices_sum_and_routing_is_replicated():
+    x, w_r, w13, w2, sh = _small_layer(12, T=7, E=5, K=3, I=32, I_sh=16)
+    d = sum(oracle.dense_ffn(x, *oracle.tp_shard(sh["w13_sh"], sh["w2_sh"], r, 4)) for r in range(4))
+    ref = oracle.dense_ffn(x, sh["w13_sh"], sh["w2_sh"])
+    assert np.allclose(d, ref, rtol=1e-12, atol=1e-13 * np.abs(ref).max())
+    routes = [oracle.moe_layer(x, w_r, *oracle.tp_shard(w13, w2, r, 2), K=3, return_routing=True)[1:]
+              for r in range(2)]
+    assert np.array_equal(routes[0][0], routes[1][0]) and np.array_equal(routes[0][1], routes[1][1])
+
+
+def test_tp_pin_catches_a_misaligned_up_slice():
+    # a plausible slicing mistake (up rows taken without the +I offset, i.e.
+    # the next gate rows) must break the sum: the pin above would catch it
+    x, w_r, w13, w2, _ = _small_layer(13, T=6, E=4, K=2, I=16)
+    full = oracle.moe_layer(x, w_r, w13, w2, K=2)
+    wrong = np.zeros_like(full)
+    for r in range(2):
+        lo, hi = 8 * r, 8 * r + 8
+        bad13 = np.ascontiguousarray(np.concatenate([w13[:, lo:hi], w13[:, (lo + 8) % 16:(lo + 8) % 16 + 8]], 1))
+        wrong += oracle.moe_layer(x, w_r, bad13, np.ascontiguousarray(w2[..., lo:hi]), K=2)
+    assert np.abs(wrong - full).max() > 1e-2 * np.abs(full).max()
