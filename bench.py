@@ -413,6 +413,9 @@ def main():
                     help="per-token dynamic K: each token's expert count uniform in 1..K (seeded)")
     ap.add_argument("--padding-model", action="store_true",
                     help="time the expert FFN over routings and fit the padding and max-affine latency models")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor parallelism over I across the ranks: every rank holds I/N of every expert and "
+                         "runs the same tokens; one NCCL all-reduce of the fp32 partial output per layer")
     ap.add_argument("--shared-sms", type=int, default=0,
                     help="SMs for the shared experts beside the routed ones (0 = cost model, -1 = serial)")
     args = ap.parse_args()
@@ -446,6 +449,14 @@ def main():
     if args.padding_model:
         if rank == 0:
             print(json.dumps(run_padding_model(args, device, flush)), flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if args.tp:
+        line = run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
         if dist:
             dist.barrier()
             dist.destroy_process_group()
@@ -602,7 +613,7 @@ def main():
                    "padding": "max-value" if args.pad_mode == 1 else "block-wise",
                    "top_k": (f"per-token dynamic, uniform 1..{shape.K} (sum {wl.A})" if args.dynamic_k
                              else f"{shape.K} for every token"),
-                   "expert_weights": ("FP8 E4M3 codes + fp32 row scales (widened to f16 in shared memory, f16 MMAs)"
+                   "expert_weights": ("FP8 E4M3 codes + fp32 row scales (widened to f16 in TMEM, f16 MMAs)"
                                       if args.fp8 else shape.dtype)},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "padded_fraction": round((P - wl.A) / max(P, 1), 4),
@@ -623,6 +634,129 @@ def main():
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def tp_tokens_per_s(T, steps, max_total_ms):
+    """TP: every rank works on the same T tokens, so the job's throughput is
+    T per step over the slowest rank's device time."""
+    return T * steps / (max_total_ms * 1e-3)
+
+
+def run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind):
+    """The layer under tensor parallelism over I on `world` ranks (strong
+    scaling): each rank slices every expert and the shared FFN, computes its
+    fp32 partial output (one CUDA graph of the layer's kernels), NCCL sums the
+    partials across the ranks, and one kernel rounds the sum."""
+    import mixture_experts_layer_61_b200 as moe
+    seed = mi.seed_for(shape, T)
+    w = mi.make_weights(shape, seed, device=device)
+    x = mi.make_x(shape, T, seed, device=device)           # the same tokens on every rank
+    n_sh, I_s = (1, shape.I_sh) if shape.I_sh else (0, 0)
+    cfg = moe.config(T, shape.H, shape.E, shape.K, shape.I, n_shared=n_sh, I_shared=I_s, tile_B=shape.tile_B,
+                     score_fn=shape.score_fn, renorm=shape.renorm,
+                     dtype=moe.BF16 if shape.dtype == "bf16" else moe.FP32, pad_mode=args.pad_mode)
+    cl = moe.tp_config(cfg, world)
+    w13, w2 = moe.tp_shard(w["w13"], w["w2"], rank, world)
+    sh = moe.tp_shard(w["w13_sh"], w["w2_sh"], rank, world) if shape.I_sh else (None, None)
+    w_r = w["w_r"]
+    del w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    ws = moe.alloc_workspace(moe.workspace_size(cl), device)
+    stats = torch.zeros(4, dtype=torch.int32, device=device)
+    partial = torch.empty((T, shape.H), dtype=torch.float32, device=device)
+    out = torch.empty((T, shape.H), dtype=x.dtype, device=device)
+
+    def layer():
+        moe.layer_forward_partial(cl, x, w_r, w13, w2, ws, sh[0], sh[1], out=partial, stats=stats)
+
+    layer()
+    torch.cuda.synchronize()
+    n0 = moe.kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer()
+    per_graph = moe.kernel_launch_count() - n0
+    torch.cuda.synchronize()
+
+    def step():
+        graph.replay()
+        moe.tp_allreduce(partial)             # NCCL all-reduce (no-op on one rank)
+        moe.tp_reduce([partial], out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    moe.check_status(ws)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = time_steps(step, args.steps, flush)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    total_ms = max_over_ranks(sum(times), dist, device)
+    moe.check_status(ws)
+    P, E_active = stats.cpu().tolist()[:2]
+    ms_step = total_ms / args.steps
+    # per-rank algorithmic work: this rank's slice of the layer's weights and flops
+    B_alg, F_alg = algorithmic(shape, T, E_active)
+    eb = 2 if shape.dtype == "bf16" else 4
+    B_r, F_r = shape.E * shape.H * eb, 2.0 * T * shape.H * shape.E    # the router, whole on every rank
+    B_rank, F_rank = (B_alg - B_r) / world + B_r, (F_alg - F_r) / world + F_r
+    hbm_peak = pk["hbm_gbs"]
+    tc_peak = pk["bf16_tflops"] * (0.5 if shape.dtype == "fp32" else 1.0)
+    t = ms_step * 1e-3
+    if F_rank / (tc_peak * 1e12) > B_rank / (hbm_peak * 1e9):
+        ach = F_rank / t / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": round(ach / tc_peak, 4)}
+    else:
+        ach = B_rank / t / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(ach / hbm_peak, 4)}
+    roof.update({"kernel": "whole TP step per rank (slice of the layer + all-reduce + rounding)",
+                 "peak_source": f"{pk_kind} ({'MEASURED_PEAKS.json' if pk_kind == 'measured' else 'fallback'})",
+                 "traffic": None})
+    # e2e: tokens from pinned host memory, the rounded output back
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x)
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e2e_total = max_over_ranks(sum(time_steps(e2e_step, args.steps, flush)), dist, device)
+    del graph
+    return {
+        "metric": METRIC, "value": round(tp_tokens_per_s(T, args.steps, total_ms), 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16" if shape.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded Gaussian weights/activations of the layer's shape; router logits x.W_r)",
+        "config": {"workload": f"{shape.name}-shaped MoE layer forward, T={T}", "T": T, "H": shape.H,
+                   "E": shape.E, "K": shape.K, "I": shape.I, "I_per_rank": cl.I, "I_shared": shape.I_sh,
+                   "tile_B": shape.tile_B, "global_batch": T,
+                   "parallelism": f"TP over I x{world} (one all-reduce of the fp32 partial output per layer)",
+                   "launch": "CUDA graph of the partial layer, then the all-reduce and the rounding kernel",
+                   "l2": "flushed between steps (2 GiB write outside the events)"},
+        "roofline": roof,
+        "layer": {"P": P, "E_active": E_active, "bytes_alg_per_rank": B_rank, "flops_alg_per_rank": F_rank},
+        "e2e": {"value": tp_tokens_per_s(T, args.steps, e2e_total), "unit": "tokens/s",
+                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+        "gpu_launches": (per_graph + 1) * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": None,
+    }
 
 
 def run_sweep(args, device, flush, pk):

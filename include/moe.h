@@ -346,6 +346,45 @@ int moe_set_shared_sms(int n);
  * setting (0: they run serially, or there are none). */
 int moe_shared_sms(const moe_config_t* cfg);
 
+/* Tensor parallelism over the expert intermediate dimension I (talk notes,
+ * "Demystifying the Mixture of Experts Serving Tax": under TP the buckets of
+ * the Balls-Bins-Buckets model are the n_tp GPUs; "Key findings" 3: the
+ * AllReduce that follows the MoE block).  Rank r of n holds, for every routed
+ * expert and for the shared FFN, the gate rows [r*I/n, (r+1)*I/n) of W1, the
+ * same rows of W3 and the same columns of W2; the router weights are whole on
+ * every rank, so every rank routes identically.  The sum over ranks of the
+ * partial outputs is the layer output.
+ *
+ * moe_tp_shard: rank `rank`'s slice of w13 [E, 2I, H] / w2 [E, H, I] (dtype
+ * 0 bf16, 1 fp32) into caller-owned w13_local [E, 2I/n, H] (gate slice, then
+ * up slice, per expert) and w2_local [E, H, I/n]; E = 1 slices one dense FFN
+ * (the shared experts).  Device-to-device copies enqueued on `stream`.
+ * MOE_ERR_ARG unless I % n_ranks == 0 and 0 <= rank < n_ranks. */
+int moe_tp_shard(int E, int H, int I, int dtype, int rank, int n_ranks, const void* w13,
+                 const void* w2, void* w13_local, void* w2_local, moe_stream_t stream);
+
+/* moe_layer_forward_k on one rank's slice (cfg->I = I/n, cfg->n_shared *
+ * cfg->I_shared = the shared FFN's I_sh/n): the same routing, the same
+ * kernels, but the combine writes the fp32 sums unrounded into out_partial
+ * [T, H] (fp32), ready for the all-reduce.  Same workspace as
+ * moe_layer_forward for cfg. */
+int moe_layer_forward_partial(const moe_config_t* cfg, const void* x, const void* w_router,
+                              const void* w13, const void* w2, const void* w13_shared,
+                              const void* w2_shared, const float* logits_override,
+                              const int32_t* k_per_token, float* out_partial, void* workspace,
+                              size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
+
+/* The reduction of the ranks' partial outputs: out[i] = sum over r of
+ * parts[r][i] for i < count, fp32 in rank order, one rounding to dtype (0
+ * bf16, 1 fp32).  `parts` is a HOST array of n_parts (1..16) device
+ * pointers, each 16-byte aligned; they may point into other GPUs' memory
+ * mapped into this one (peer access), which the kernel reads with plain
+ * loads.  With n_parts = 1 it rounds an all-reduced sum.  count % 4 == 0.
+ * The caller orders the writes of every part before this call (on other
+ * GPUs: an event or a barrier) and keeps the parts alive until it ends. */
+int moe_tp_reduce(int n_parts, const float* const* parts, long long count, int dtype, void* out,
+                  moe_stream_t stream);
+
 /* Test hook: when nonzero, the next GEMM or fused-FFN launch withholds one
  * operand load (the first load of block 0, or of work item 0 in the fused
  * FFN), so the waits that depend on it run out and report MOE_ERR_TIMEOUT

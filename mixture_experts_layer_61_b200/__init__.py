@@ -95,6 +95,9 @@ def lib():
             "moe_ffn_fused": (I, [C]),
             "moe_layer_logits_offset": (ctypes.c_int64, [C]),
             "moe_kernel_launch_count": (ctypes.c_uint64, []),
+            "moe_tp_shard": (I, [I, I, I, I, I, I, P, P, P, P, P]),
+            "moe_layer_forward_partial": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P, P]),
+            "moe_tp_reduce": (I, [I, ctypes.POINTER(ctypes.c_void_p), ctypes.c_longlong, I, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -408,3 +411,85 @@ class MoELayer:
     def forward(self, x, logits_override=None, out=None):
         return layer_forward(self.cfg, x, self.w["w_r"], self.w["w13"], self.w["w2"], self.ws,
                              self.w.get("w13_sh"), self.w.get("w2_sh"), logits_override, out, self.stats)
+
+
+# ------------------------------------------------ tensor parallelism over I
+# Rank r of n holds, for every routed expert and for the shared FFN, the gate
+# rows [r*I/n, (r+1)*I/n) of W1, the same rows of W3 and the same columns of
+# W2 (talk notes, "Demystifying the Mixture of Experts Serving Tax",
+# "Balls-Bins-Buckets framework": the n_tp GPUs are the buckets under TP); the
+# router is whole on every rank.  Each rank computes an fp32 partial output,
+# one all-reduce sums them ("Key findings" 3), and one rounding follows.
+
+def tp_config(cfg, n_ranks):
+    """The per-rank configuration of `cfg` split over I into n_ranks."""
+    I_sh = cfg.n_shared * cfg.I_shared
+    if n_ranks < 1 or cfg.I % n_ranks or I_sh % n_ranks:
+        raise ValueError("I and the shared FFN's width must split evenly over the ranks")
+    return MoeConfig(cfg.T, cfg.H, cfg.E, cfg.K, cfg.I // n_ranks, 1 if I_sh else 0, I_sh // n_ranks,
+                     cfg.tile_B, cfg.score_fn, cfg.renorm, cfg.dtype, cfg.pad_mode)
+
+
+def tp_shard(w13, w2, rank, n_ranks):
+    """Rank `rank`'s slice of w13 [E,2I,H] / w2 [E,H,I] (or one dense FFN
+    [2I,H] / [H,I]): new device tensors [E,2I/n,H] / [E,H,I/n]."""
+    _need_cuda(w13, w2)
+    dense = w13.dim() == 2
+    E = 1 if dense else w13.shape[0]
+    H, I = w2.shape[-2], w2.shape[-1]
+    n = I // n_ranks if n_ranks > 0 else 0
+    lead = () if dense else (E,)
+    a = torch.empty(lead + (2 * n, H), dtype=w13.dtype, device=w13.device)
+    b = torch.empty(lead + (H, n), dtype=w2.dtype, device=w2.device)
+    dt = BF16 if w13.dtype == torch.bfloat16 else FP32
+    _check(lib().moe_tp_shard(E, H, I, dt, rank, n_ranks, _p(w13), _p(w2), _p(a), _p(b), _stream()),
+           "moe_tp_shard")
+    return a, b
+
+
+def layer_forward_partial(cfg, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, logits_override=None, out=None,
+                          stats=None, k=None):
+    """This rank's fp32 partial output [T,H] for its slice (cfg from tp_config)."""
+    _need_cuda(x, w_r, w13, w2, ws, w13_sh, w2_sh, logits_override, out, stats, k)
+    if out is None:
+        out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device=x.device)
+    _check(lib().moe_layer_forward_partial(ctypes.byref(cfg), _p(x), _p(w_r), _p(w13), _p(w2), _p(w13_sh),
+                                           _p(w2_sh), _p(logits_override), _p(k), _p(out), _p(ws), ws.numel(),
+                                           _p(stats), _stream()),
+           "moe_layer_forward_partial")
+    return out
+
+
+def tp_reduce(parts, out=None, dtype=torch.bfloat16):
+    """out = sum of the fp32 partial outputs in list order, rounded once to
+    dtype (the parts may be other GPUs' memory mapped here)."""
+    _need_cuda(out, *parts)
+    count = parts[0].numel()
+    if any(p_.numel() != count or p_.dtype != torch.float32 for p_ in parts):
+        raise ValueError("parts must be fp32 tensors of one size")
+    if out is None:
+        out = torch.empty(parts[0].shape, dtype=dtype, device=parts[0].device)
+    ptrs = (ctypes.c_void_p * len(parts))(*[p_.data_ptr() for p_ in parts])
+    dt = BF16 if out.dtype == torch.bfloat16 else FP32
+    _check(lib().moe_tp_reduce(len(parts), ptrs, count, dt, _p(out), _stream()), "moe_tp_reduce")
+    return out
+
+
+def tp_allreduce(partial, group=None):
+    """Sums the ranks' fp32 partial outputs in place across `group` (the
+    collective step of TP over I; NCCL on GPUs)."""
+    import torch.distributed as dist
+
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(partial, op=dist.ReduceOp.SUM, group=group)
+    return partial
+
+
+def tp_layer_forward(cfg_local, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, logits_override=None,
+                     partial=None, out=None, group=None, k=None):
+    """One layer under TP over I on this rank: partial output (kernels), the
+    all-reduce over `group`, then the rounding (kernel)."""
+    partial = layer_forward_partial(cfg_local, x, w_r, w13, w2, ws, w13_sh, w2_sh, logits_override, partial,
+                                    k=k)
+    tp_allreduce(partial, group)
+    return tp_reduce([partial], out, dtype=x.dtype)

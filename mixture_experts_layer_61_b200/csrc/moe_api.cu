@@ -533,7 +533,8 @@ struct Fp8Scales {
 static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
                               const void* w2, const void* w13_shared, const void* w2_shared,
                               const Fp8Scales* fp8, const float* logits_override, const int32_t* k_per_token,
-                              void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
+                              void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream,
+                              bool out_f32 = false);
 
 int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
                         const void* w2, const void* w13_shared, const void* w2_shared, const float* logits_override,
@@ -567,7 +568,8 @@ int moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_
 static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
                               const void* w2, const void* w13_shared, const void* w2_shared,
                               const Fp8Scales* fp8, const float* logits_override, const int32_t* k_per_token,
-                              void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
+                              void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream,
+                              bool out_f32) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->T == 0) return MOE_OK;
@@ -721,10 +723,55 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
             return MOE_ERR_CUDA;
         }
     }
-    return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, w, sh, out, s));
+    return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, w, sh, out, s, out_f32));
 }
 
 extern "C" {
+
+// ------------------------------------------------ tensor parallelism over I
+
+int moe_layer_forward_partial(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
+                              const void* w2, const void* w13_shared, const void* w2_shared,
+                              const float* logits_override, const int32_t* k_per_token, float* out_partial,
+                              void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
+    return layer_forward_impl(cfg, x, w_router, w13, w2, w13_shared, w2_shared, nullptr, logits_override,
+                              k_per_token, out_partial, workspace, ws_bytes, stats_out, stream, true);
+}
+
+int moe_tp_reduce(int n_parts, const float* const* parts, long long count, int dtype, void* out,
+                  moe_stream_t stream) {
+    if (n_parts < 1 || n_parts > kTpMaxParts || count < 0 || count % 4 || !parts || !out) return MOE_ERR_ARG;
+    if (dtype != 0 && dtype != 1) return MOE_ERR_ARG;
+    if (count == 0) return MOE_OK;
+    for (int r = 0; r < n_parts; ++r)
+        if (!parts[r] || !aligned16(parts[r])) return MOE_ERR_ARG;
+    if (!aligned16(out)) return MOE_ERR_ARG;
+    return status_of(launch_tp_reduce(n_parts, parts, count, dtype, out, (cudaStream_t)stream));
+}
+
+int moe_tp_shard(int E, int H, int I, int dtype, int rank, int n_ranks, const void* w13, const void* w2,
+                 void* w13_local, void* w2_local, moe_stream_t stream) {
+    const int eb = elt_bytes(dtype);
+    if (eb == 0 || E < 1 || H < 1 || I < 1 || n_ranks < 1 || rank < 0 || rank >= n_ranks || I % n_ranks)
+        return MOE_ERR_ARG;
+    if (!w13 || !w2 || !w13_local || !w2_local) return MOE_ERR_ARG;
+    const size_t n = (size_t)(I / n_ranks);
+    const size_t row = (size_t)H * eb;
+    cudaStream_t s = (cudaStream_t)stream;
+    // w13: the 2E blocks [gate of e, up of e] are I rows apart; each gives its
+    // n rows starting at rank * n
+    cudaError_t e = cudaMemcpy2DAsync(w13_local, n * row, static_cast<const uint8_t*>(w13) + rank * n * row,
+                                      (size_t)I * row, n * row, (size_t)2 * E, cudaMemcpyDeviceToDevice, s);
+    // w2: the E*H rows of I columns each give columns [rank * n, rank * n + n)
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(w2_local, n * eb, static_cast<const uint8_t*>(w2) + rank * n * eb, (size_t)I * eb,
+                              n * eb, (size_t)E * H, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
 
 
 int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13, const void* w2, void* out,

@@ -161,7 +161,9 @@ int launch_permute(int H, int K, int dtype, long long P_max, const void* x, cons
 // n bf16 values -> f16 (n a multiple of 8)
 int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stream);
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
-                   const void* shared_out, void* out, cudaStream_t stream);
+                   const void* shared_out, void* out, cudaStream_t stream, bool out_f32 = false);
+constexpr int kTpMaxParts = 16;  // ranks of one TP reduction
+int launch_tp_reduce(int n, const float* const* parts, long long count, int dtype, void* out, cudaStream_t stream);
 
 // Row-wise FP8 E4M3 quantisation: q [rows, cols] codes, scales [rows].
 int launch_quantize_fp8(long long rows, int cols, int dtype, const void* w, uint8_t* q, float* scales,

@@ -607,10 +607,23 @@ __device__ __forceinline__ int4 pack(const float* f, const float*) {
     return v;
 }
 
-template <typename T>
+// Stores the N fp32 sums of one 16-byte input vector: rounded once to the
+// activation dtype, or (TP partials, which an all-reduce sums next) unrounded.
+template <int N>
+__device__ __forceinline__ void store_sums(const float* acc, __nv_bfloat16* out) {
+    *reinterpret_cast<int4*>(out) = pack(acc, (const __nv_bfloat16*)nullptr);
+}
+template <int N>
+__device__ __forceinline__ void store_sums(const float* acc, float* out) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4)
+        *reinterpret_cast<float4*>(out + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+}
+
+template <typename T, typename TOut>
 __global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K, const int4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ pos, const float* __restrict__ w,
-                                                      const int4* __restrict__ sh, int4* __restrict__ out) {
+                                                      const int4* __restrict__ sh, TOut* __restrict__ out) {
     constexpr int N = Vec16<T>::N;
     __shared__ int s_pos[16];
     __shared__ float s_w[16];
@@ -641,13 +654,13 @@ __global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K
 #pragma unroll
                 for (int i = 0; i < N; ++i) acc[i] += y[i];
             }
-            out[(long long)t * row_vec + v] = pack(acc, (const T*)nullptr);
+            store_sums<N>(acc, out + ((long long)t * row_vec + v) * N);
         }
     }
 }
 
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
-                   const void* shared_out, void* out, cudaStream_t stream) {
+                   const void* shared_out, void* out, cudaStream_t stream, bool out_f32) {
     if (T == 0) return 0;
     DeviceInfo d;
     int rc = current_device(&d);
@@ -660,11 +673,76 @@ int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int
     if (blocks > cap) blocks = cap;
     const int4* y4 = static_cast<const int4*>(y_perm);
     const int4* s4 = static_cast<const int4*>(shared_out);
-    int4* o4 = static_cast<int4*>(out);
-    cudaError_t e = dtype == 0 ? launch_kernel(combine_kernel<__nv_bfloat16>, dim3((int)blocks), dim3(threads), 0,
-                                               stream, T, row_vec, K, y4, pos, w, s4, o4)
-                               : launch_kernel(combine_kernel<float>, dim3((int)blocks), dim3(threads), 0, stream, T,
-                                               row_vec, K, y4, pos, w, s4, o4);
+    cudaError_t e;
+    if (dtype == 0 && !out_f32)
+        e = launch_kernel(combine_kernel<__nv_bfloat16, __nv_bfloat16>, dim3((int)blocks), dim3(threads), 0, stream,
+                          T, row_vec, K, y4, pos, w, s4, static_cast<__nv_bfloat16*>(out));
+    else if (dtype == 0)
+        e = launch_kernel(combine_kernel<__nv_bfloat16, float>, dim3((int)blocks), dim3(threads), 0, stream, T,
+                          row_vec, K, y4, pos, w, s4, static_cast<float*>(out));
+    else
+        e = launch_kernel(combine_kernel<float, float>, dim3((int)blocks), dim3(threads), 0, stream, T, row_vec, K,
+                          y4, pos, w, s4, static_cast<float*>(out));
+    count_launch();
+    return launched(e);
+}
+
+// ------------------------------------------------------------ TP reduction
+// out[i] = sum over r of parts[r][i], fp32 in rank order, one rounding to the
+// output dtype.  parts[r] may live on another GPU (a peer mapping): plain
+// coalesced 16-byte loads, 4 elements per thread per step, grid-stride over
+// the whole vector with a grid of a few blocks per SM.
+struct TpParts {
+    const float4* p[kTpMaxParts];
+};
+
+template <typename TOut>
+__device__ __forceinline__ void store4(TOut* out, long long i, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* out, long long i, float4 v) {
+    reinterpret_cast<float4*>(out)[i] = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* out, long long i, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    reinterpret_cast<uint2*>(out)[i] = u;
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(256) tp_reduce_kernel(TpParts parts, int n, long long n4, TOut* __restrict__ out) {
+    pdl_launch_dependents();
+    pdl_wait();
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+        float4 acc = __ldcs(parts.p[0] + i);
+        for (int r = 1; r < n; ++r) {
+            const float4 v = __ldcs(parts.p[r] + i);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        store4<TOut>(out, i, acc);
+    }
+}
+
+int launch_tp_reduce(int n, const float* const* parts, long long count, int dtype, void* out, cudaStream_t stream) {
+    if (count == 0) return 0;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    TpParts tp{};
+    for (int r = 0; r < n; ++r) tp.p[r] = reinterpret_cast<const float4*>(parts[r]);
+    const long long n4 = count / 4;
+    long long blocks = (n4 + 255) / 256;
+    const long long cap = (long long)d.num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    cudaError_t e = dtype == 0 ? launch_kernel(tp_reduce_kernel<__nv_bfloat16>, dim3((int)blocks), dim3(256), 0,
+                                               stream, tp, n, n4, static_cast<__nv_bfloat16*>(out))
+                               : launch_kernel(tp_reduce_kernel<float>, dim3((int)blocks), dim3(256), 0, stream, tp,
+                                               n, n4, static_cast<float*>(out));
     count_launch();
     return launched(e);
 }

@@ -46,3 +46,9 @@ def test_max_over_ranks_and_whole_job_throughput_gloo():
 def test_single_rank_is_identity():
     assert bench.max_over_ranks(12.5, None, torch.device("cpu")) == 12.5
     assert bench.replica_tokens_per_s(1, 100, 10, 1000.0) == pytest.approx(1000.0)
+
+
+def test_tp_throughput_counts_the_shared_tokens_once():
+    # under TP every rank works on the same T tokens: the job's rate is T per
+    # step over the slowest rank's time, whatever the number of ranks
+    assert bench.tp_tokens_per_s(32, 10, 5.0) == pytest.approx(32 * 10 / 0.005)
