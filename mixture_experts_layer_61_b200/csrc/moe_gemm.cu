@@ -30,9 +30,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // [rows, kdim] row-major, box = box_rows x row_bytes (128 or 64) with the
-// swizzle of that width (or none), out-of-range elements read as zero.
+// swizzle of that width, out-of-range elements read as zero.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void* base, long long rows, int kdim,
-              int box_rows, int row_bytes = 128, bool swizzled = true) {
+              int box_rows, int row_bytes = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(kdim), static_cast<cuuint64_t>(rows)};
@@ -40,8 +40,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elt_bytes, const void*
     cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes / elt_bytes), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    !swizzled ? CU_TENSOR_MAP_SWIZZLE_NONE
-                              : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B),
+                    row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;

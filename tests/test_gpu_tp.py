@@ -19,26 +19,29 @@ from helpers import OUT_TOL, cfg_for, host, rel_err, sample_tokens, small_shape
 pytestmark = pytest.mark.gpu
 
 
-def _run_tp(shape, T, n_ranks, seed, n_sample=None, check_rank=None):
+def _run_tp(shape, T, n_ranks, seed, n_sample=None, check_rank=None, pad_mode=0, k=None, override=None):
     w = mi.make_weights(shape, seed, device="cuda")
     x = mi.make_x(shape, T, seed, device="cuda")
-    cl = moe.tp_config(cfg_for(shape, T), n_ranks)
+    cl = moe.tp_config(cfg_for(shape, T, pad_mode=pad_mode), n_ranks)
+    kt = None if k is None else torch.from_numpy(np.asarray(k, np.int32)).cuda()
     ws = moe.alloc_workspace(moe.workspace_size(cl))
     parts, lgs = [], []
     for r in range(n_ranks):
         a13, a2 = moe.tp_shard(w["w13"], w["w2"], r, n_ranks)
         s13, s2 = moe.tp_shard(w["w13_sh"], w["w2_sh"], r, n_ranks) if shape.I_sh else (None, None)
-        parts.append(moe.layer_forward_partial(cl, x, w["w_r"], a13, a2, ws, s13, s2))
+        parts.append(moe.layer_forward_partial(cl, x, w["w_r"], a13, a2, ws, s13, s2, logits_override=override,
+                                               k=kt))
         moe.check_status(ws)
         lgs.append(moe.layer_logits(cl, ws).clone())
         del a13, a2, s13, s2
     assert all(torch.equal(lgs[0], lg) for lg in lgs[1:])  # every rank routes identically
     out = moe.tp_reduce(parts, dtype=x.dtype)
-    lg = lgs[0].cpu().numpy()
+    lg = lgs[0].cpu().numpy() if override is None else override.cpu().numpy()
     tok = sample_tokens(T, n_sample or T, seed)
     hx, h13, h2 = host(x), host(w["w13"]), host(w["w2"])
     sh = dict(w13_sh=host(w["w13_sh"]), w2_sh=host(w["w2_sh"])) if shape.I_sh else {}
-    ref = oracle.moe_layer(hx, None, h13, h2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok, **sh)
+    ref = oracle.moe_layer(hx, None, h13, h2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok, k=k,
+                           **sh)
     errs = {"out": rel_err(out.float().cpu().numpy()[tok], ref)}
     ranks = range(n_ranks) if check_rank is None else [check_rank]
     for r in ranks:
@@ -48,7 +51,7 @@ def _run_tp(shape, T, n_ranks, seed, n_sample=None, check_rank=None):
             a, b = oracle.tp_shard(sh["w13_sh"], sh["w2_sh"], r, n_ranks)
             osh = dict(w13_sh=a, w2_sh=b)
         ref_r = oracle.moe_layer(hx, None, o13, o2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok,
-                                 **osh)
+                                 k=k, **osh)
         errs[f"part{r}"] = rel_err(parts[r].cpu().numpy()[tok], ref_r)
     return errs
 
@@ -70,6 +73,17 @@ def test_tp_shard_is_the_oracle_slice():
 def test_tp_small_layer_with_shared(n_ranks, T):
     shape = small_shape(H=512, E=16, K=4, I=768, I_sh=256)
     errs = _run_tp(shape, T, n_ranks, seed=T + n_ranks)
+    assert max(errs.values()) < OUT_TOL, errs
+
+
+@pytest.mark.parametrize("T", [24, 200])
+def test_tp_dynamic_k_max_value_padding_and_supplied_logits(T):
+    # per-token expert counts 0..K (0 = shared experts only), max-value padding,
+    # skewed supplied logits: the same on every rank
+    shape = small_shape(H=512, E=16, K=4, I=768, I_sh=256, score_fn=1)
+    k = np.random.default_rng(T).integers(0, 5, T).astype(np.int32)
+    lg = mi.zipf_gumbel_logits(16, T, 1.2, seed=T, device="cuda")
+    errs = _run_tp(shape, T, 2, seed=T, pad_mode=1, k=k, override=lg)
     assert max(errs.values()) < OUT_TOL, errs
 
 
