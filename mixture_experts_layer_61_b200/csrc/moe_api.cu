@@ -379,6 +379,9 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
     if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
+    if (router_cc_fits(cfg->H, cfg->E, cfg->dtype))  // a small router matrix: CUDA cores, w_r in shared memory
+        return status_of(launch_router_cc(cfg->T, cfg->H, cfg->E, cfg->dtype, x, w_router, logits,
+                                          (cudaStream_t)stream));
     GemmLaunch g{};
     g.x = x;
     g.x_rows = cfg->T;
@@ -671,22 +674,28 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
                                      stats_out, route_ctr, s)) != 0)
             return status_of(rc);
     } else {
-        GemmLaunch g{};
-        g.x = x;
-        g.x_rows = cfg->T;
-        g.w = w_router;
-        g.w_rows = cfg->E;
-        g.kdim = cfg->H;
-        g.n_out = cfg->E;
-        g.n_groups = 1;
-        g.seg_rows = cfg->T;
-        g.out_f32 = true;
-        g.out = logits;
-        g.out_ld = cfg->E;
-        g.dtype = cfg->dtype;
-        router_tiling(g, cfg->T);
-        g.sms = n_routed;
-        if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
+        if (router_cc_fits(cfg->H, cfg->E, cfg->dtype)) {
+            // a small router matrix (E * H fits shared memory): CUDA cores, one read of x
+            if ((rc = launch_router_cc(cfg->T, cfg->H, cfg->E, cfg->dtype, x, w_router, logits, s)) != 0)
+                return status_of(rc);
+        } else {
+            GemmLaunch g{};
+            g.x = x;
+            g.x_rows = cfg->T;
+            g.w = w_router;
+            g.w_rows = cfg->E;
+            g.kdim = cfg->H;
+            g.n_out = cfg->E;
+            g.n_groups = 1;
+            g.seg_rows = cfg->T;
+            g.out_f32 = true;
+            g.out = logits;
+            g.out_ld = cfg->E;
+            g.dtype = cfg->dtype;
+            router_tiling(g, cfg->T);
+            g.sms = n_routed;
+            if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
+        }
         if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm,
                               logits_override ? logits_override : logits, k_per_token, ids, w, s)) != 0)
             return status_of(rc);

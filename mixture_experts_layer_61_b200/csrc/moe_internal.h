@@ -163,6 +163,12 @@ int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stre
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
                    const void* shared_out, void* out, cudaStream_t stream, bool out_f32 = false);
 constexpr int kTpMaxParts = 16;  // ranks of one TP reduction
+// router logits on the CUDA cores for small router matrices (E <= 16, E*H*elt
+// bytes <= kRouterCcMaxBytes, H % 8 == 0); -1 when the shape does not fit
+constexpr int kRouterCcMaxBytes = 96 * 1024;
+bool router_cc_fits(int H, int E, int dtype);
+int launch_router_cc(int T, int H, int E, int dtype, const void* x, const void* w_r, float* logits,
+                     cudaStream_t stream);
 int launch_tp_reduce(int n, const float* const* parts, long long count, int dtype, void* out, cudaStream_t stream);
 
 // Row-wise FP8 E4M3 quantisation: q [rows, cols] codes, scales [rows].

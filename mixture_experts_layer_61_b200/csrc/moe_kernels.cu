@@ -418,6 +418,123 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     if (threadIdx.x == 0) *done_ctr = 0;  // ready for the next launch
 }
 
+// ------------------------------------------------ router on the CUDA cores
+// logits[t][e] = sum over h of x[t][h] * w_r[e][h] in fp32, for layers whose
+// router matrix fits shared memory (E <= 16, E * H * elt <= kRouterCcMaxBytes;
+// the Mixtral-shaped layer's is 64 KB).  Every block keeps w_r in shared
+// memory and each warp takes whole tokens: lane l reads 16-byte chunks l,
+// l + 32, ... of the token row (each row is read once, coalesced), multiplies
+// them with the E weight chunks at the same position (consecutive lanes,
+// consecutive chunks: no bank conflict) and the E per-lane sums go through a
+// shuffle tree.  The tensor-core GEMM would fill 8 of the 128 rows of each
+// MMA here and pay a pipeline ramp and split-K fixups for what is one read of x.
+__device__ __forceinline__ void load8_shared(const __nv_bfloat16* p, float* f) {
+    const int4 v = *reinterpret_cast<const int4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+__device__ __forceinline__ void load8_shared(const float* p, float* f) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+
+template <typename T, int kE>
+__global__ void __launch_bounds__(256) router_cc_kernel(int T_, int H, const T* __restrict__ x,
+                                                        const T* __restrict__ w_r, float* __restrict__ logits) {
+    extern __shared__ int4 router_sm[];
+    const T* ws = reinterpret_cast<const T*>(router_sm);
+    pdl_launch_dependents();
+    // the router weights are not written by the previous kernel: stage them before waiting for it
+    const int n16 = (int)((long long)kE * H * sizeof(T) / 16);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) router_sm[i] = __ldg(reinterpret_cast<const int4*>(w_r) + i);
+    pdl_wait();
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int warps = blockDim.x >> 5;
+    for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T_; t += gridDim.x * warps) {
+        float acc[kE];
+#pragma unroll
+        for (int e = 0; e < kE; ++e) acc[e] = 0.f;
+        const T* xr = x + (size_t)t * H;
+#pragma unroll 2
+        for (int h = lane * 8; h < H; h += 256) {
+            float xv[8];
+            load8(xr + h, xv);
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                float wv[8];
+                load8_shared(ws + (size_t)e * H + h, wv);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[e] = fmaf(wv[j], xv[j], acc[e]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < kE; ++e) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        }
+#pragma unroll
+        for (int e = 0; e < kE; ++e)
+            if (lane == e) logits[(size_t)t * kE + e] = acc[e];
+    }
+}
+
+bool router_cc_fits(int H, int E, int dtype) {
+    const long long eb = dtype == 0 ? 2 : 4;
+    return E >= 1 && E <= 16 && H > 0 && H % 8 == 0 && (long long)E * H * eb <= kRouterCcMaxBytes;
+}
+
+template <typename T, int kE>
+cudaError_t launch_router_cc_e(int n_tok, int H, const void* x, const void* w_r, float* logits, int num_sms,
+                               cudaStream_t stream) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(router_cc_kernel<T, kE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kRouterCcMaxBytes);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    long long blocks = (n_tok + 7) / 8;
+    if (blocks > 2LL * num_sms) blocks = 2LL * num_sms;
+    const size_t smem = (size_t)kE * H * sizeof(T);
+    return launch_kernel(router_cc_kernel<T, kE>, dim3((int)blocks), dim3(256), smem, stream, n_tok, H,
+                         static_cast<const T*>(x), static_cast<const T*>(w_r), logits);
+}
+
+template <typename T>
+cudaError_t launch_router_cc_t(int n_tok, int H, int E, const void* x, const void* w_r, float* logits, int num_sms,
+                               cudaStream_t s) {
+    switch (E) {
+#define MOE_ROUTER_CC_CASE(n) \
+    case n: return launch_router_cc_e<T, n>(n_tok, H, x, w_r, logits, num_sms, s);
+        MOE_ROUTER_CC_CASE(1) MOE_ROUTER_CC_CASE(2) MOE_ROUTER_CC_CASE(3) MOE_ROUTER_CC_CASE(4)
+        MOE_ROUTER_CC_CASE(5) MOE_ROUTER_CC_CASE(6) MOE_ROUTER_CC_CASE(7) MOE_ROUTER_CC_CASE(8)
+        MOE_ROUTER_CC_CASE(9) MOE_ROUTER_CC_CASE(10) MOE_ROUTER_CC_CASE(11) MOE_ROUTER_CC_CASE(12)
+        MOE_ROUTER_CC_CASE(13) MOE_ROUTER_CC_CASE(14) MOE_ROUTER_CC_CASE(15) MOE_ROUTER_CC_CASE(16)
+#undef MOE_ROUTER_CC_CASE
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+int launch_router_cc(int T, int H, int E, int dtype, const void* x, const void* w_r, float* logits,
+                     cudaStream_t stream) {
+    if (T == 0) return 0;
+    if (!router_cc_fits(H, E, dtype)) return -1;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    cudaError_t e = dtype == 0 ? launch_router_cc_t<__nv_bfloat16>(T, H, E, x, w_r, logits, d.num_sms, stream)
+                               : launch_router_cc_t<float>(T, H, E, x, w_r, logits, d.num_sms, stream);
+    count_launch();
+    return launched(e);
+}
+
 // Slices of the hidden dimension (multiples of 256 elements) so that the
 // router GEMV covers about one wave of warps on the device.
 void route_small_slices(int T, int H, int E, int num_sms, int* nslices, int* slice_w) {
