@@ -450,9 +450,19 @@ __global__ void __launch_bounds__(256) router_cc_kernel(int T_, int H, const T* 
     extern __shared__ int4 router_sm[];
     const T* ws = reinterpret_cast<const T*>(router_sm);
     pdl_launch_dependents();
-    // the router weights are not written by the previous kernel: stage them before waiting for it
+    // the router weights are not written by the previous kernel: stage them
+    // before waiting for it, 8 independent 16-byte loads per thread in flight
     const int n16 = (int)((long long)kE * H * sizeof(T) / 16);
-    for (int i = threadIdx.x; i < n16; i += blockDim.x) router_sm[i] = __ldg(reinterpret_cast<const int4*>(w_r) + i);
+    const int4* wsrc = reinterpret_cast<const int4*>(w_r);
+    for (int i0 = threadIdx.x; i0 < n16; i0 += 8 * blockDim.x) {
+        int4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + j * (int)blockDim.x < n16) v[j] = __ldg(wsrc + i0 + j * blockDim.x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + j * (int)blockDim.x < n16) router_sm[i0 + j * blockDim.x] = v[j];
+    }
     pdl_wait();
     __syncthreads();
     const int lane = threadIdx.x & 31;
@@ -462,16 +472,24 @@ __global__ void __launch_bounds__(256) router_cc_kernel(int T_, int H, const T* 
 #pragma unroll
         for (int e = 0; e < kE; ++e) acc[e] = 0.f;
         const T* xr = x + (size_t)t * H;
-#pragma unroll 2
-        for (int h = lane * 8; h < H; h += 256) {
-            float xv[8];
-            load8(xr + h, xv);
+        // the token row in groups of 8 chunks per lane, all 8 loads issued before the first use
+        for (int h0 = lane * 8; h0 < H; h0 += 8 * 256) {
+            float xv[8][8];
 #pragma unroll
-            for (int e = 0; e < kE; ++e) {
-                float wv[8];
-                load8_shared(ws + (size_t)e * H + h, wv);
+            for (int c = 0; c < 8; ++c)
+                if (h0 + c * 256 < H) load8(xr + h0 + c * 256, xv[c]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[e] = fmaf(wv[j], xv[j], acc[e]);
+            for (int c = 0; c < 8; ++c) {
+                const int h = h0 + c * 256;
+                if (h < H) {
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) {
+                        float wv[8];
+                        load8_shared(ws + (size_t)e * H + h, wv);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[e] = fmaf(wv[j], xv[c][j], acc[e]);
+                    }
+                }
             }
         }
 #pragma unroll
