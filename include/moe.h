@@ -100,8 +100,8 @@ size_t moe_workspace_size(const moe_config_t* cfg);
 /* Byte offset, inside the moe_layer_forward workspace, of the fp32 router
  * logits [T,E] the last forward computed (-1 on a bad configuration).  For
  * T <= 64 the forward computes them on the CUDA cores (fp32 sums of exact
- * products) in the same launch as top-K and alignment, otherwise with the
- * tensor-core router GEMM; either way they are what top-K selected on unless
+ * products) in the same launch as top-K and alignment, otherwise as
+ * moe_router_gemm does; either way they are what top-K selected on unless
  * logits_override was given. */
 int64_t moe_layer_logits_offset(const moe_config_t* cfg);
 
@@ -110,9 +110,12 @@ int64_t moe_layer_logits_offset(const moe_config_t* cfg);
 size_t moe_gemm_workspace_size(void);
 
 /* Router GEMM (stage "router"): logits[T,E] (fp32) = x[T,H] . w_router[E,H]^T,
- * products of the inputs accumulated in fp32 on the tensor cores (fp32
- * inputs: tf32 products).  `workspace` as returned by
- * moe_gemm_workspace_size(). */
+ * products of the inputs accumulated in fp32.  A router matrix that fits
+ * shared memory (E <= 16, E*H*elt <= 96 KB, H % 8 == 0) runs on the CUDA cores
+ * with exact products (fp32 inputs too); larger ones on the tensor cores (fp32
+ * inputs: tf32 products).  The summation order differs between the two, so
+ * results agree to fp32 rounding.  `workspace` as returned by
+ * moe_gemm_workspace_size() (unused by the CUDA-core form). */
 int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router,
                     float* logits, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
@@ -121,7 +124,9 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
  * step must not allocate, or code captured into a CUDA graph under a mode
  * that forbids cudaMalloc.  The pages have no counterpart: this is a library
  * convenience, not a step of the method.
- *   Same result and arguments as moe_router_gemm, minus the workspace: the
+ *   Same arguments as moe_router_gemm, minus the workspace, and always the
+ *   tensor-core form (equal to moe_router_gemm's result up to fp32 rounding
+ *   where that one takes the CUDA-core form): the
  *   scratch (status word, stream-K counters, partial tiles) lives in a fixed
  *   ~5 MiB array in the library's device memory, present on every GPU that
  *   loads the library until the process exits.  No allocation is made.
