@@ -636,6 +636,16 @@ def main():
         dist.destroy_process_group()
 
 
+def tp_rank_work(shape, T, E_active, world):
+    """Algorithmic bytes and flops of one rank under TP over I: its 1/world
+    share of the experts' and the shared FFN's, plus the whole router (every
+    rank routes all tokens)."""
+    B_alg, F_alg = algorithmic(shape, T, E_active)
+    eb = 2 if shape.dtype == "bf16" else 4
+    B_r, F_r = shape.E * shape.H * eb, 2.0 * T * shape.H * shape.E
+    return (B_alg - B_r) / world + B_r, (F_alg - F_r) / world + F_r
+
+
 def tp_tokens_per_s(T, steps, max_total_ms):
     """TP: every rank works on the same T tokens, so the job's throughput is
     T per step over the slowest rank's device time."""
@@ -701,10 +711,7 @@ def run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind)
     P, E_active = stats.cpu().tolist()[:2]
     ms_step = total_ms / args.steps
     # per-rank algorithmic work: this rank's slice of the layer's weights and flops
-    B_alg, F_alg = algorithmic(shape, T, E_active)
-    eb = 2 if shape.dtype == "bf16" else 4
-    B_r, F_r = shape.E * shape.H * eb, 2.0 * T * shape.H * shape.E    # the router, whole on every rank
-    B_rank, F_rank = (B_alg - B_r) / world + B_r, (F_alg - F_r) / world + F_r
+    B_rank, F_rank = tp_rank_work(shape, T, E_active, world)
     hbm_peak = pk["hbm_gbs"]
     tc_peak = pk["bf16_tflops"] * (0.5 if shape.dtype == "fp32" else 1.0)
     t = ms_step * 1e-3
