@@ -39,6 +39,7 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 HBM_NOMINAL_GBS = 8000.0
 METRIC = "MoE layer tokens/s; % HBM BW (decode) / % tensor peak (prefill); tau vs DenseFA"
+N_INPUT_SETS = 4  # seeded token sets rotated through the timed steps (different routings)
 # DRAM bytes per launch of the dominant kernel from one ncu capture of the
 # current kernels (dram__bytes_read.sum + dram__bytes_write.sum); workloads
 # without a capture report None.  Summaries of the captures are in profiles/.
@@ -252,11 +253,14 @@ def l2_flush_buffer(device):
     return torch.empty(size // 4, dtype=torch.float32, device=device)
 
 
-def time_steps(fn, steps, flush, stream_sync=True):
-    """Per-step CUDA-event durations (ms), L2 flushed before each step (outside the events)."""
+def time_steps(fn, steps, flush, stream_sync=True, before=None):
+    """Per-step CUDA-event durations (ms), L2 flushed before each step (outside
+    the events); before(i) (optional) runs after the flush, also outside."""
     times = []
-    for _ in range(steps):
+    for i in range(steps):
         flush.zero_()
+        if before is not None:
+            before(i)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
@@ -264,6 +268,18 @@ def time_steps(fn, steps, flush, stream_sync=True):
         b.synchronize()
         times.append(a.elapsed_time(b))
     return times
+
+
+def step_percentiles(times):
+    """Median, p10 and p90 of the per-step times (ms), nearest-rank."""
+    v = sorted(times)
+    n = len(v)
+
+    def pct(q):
+        return v[min(n - 1, max(0, math.ceil(q * n) - 1))]
+
+    return {"ms_median": round(statistics.median(v), 4), "ms_p10": round(pct(0.10), 4),
+            "ms_p90": round(pct(0.90), 4)}
 
 
 # ------------------------------------------------------- multi-rank timing
@@ -473,13 +489,22 @@ def main():
     torch.cuda.synchronize()
     wl.moe.check_status(wl.ws)
 
-    # ---- timed region: K steps of the fused layer call
+    # ---- timed region: K steps of the fused layer call, rotating R seeded token
+    # sets (different routings) into the input buffer before each step, outside
+    # the events like the L2 flush
+    seed = mi.seed_for(shape, T)
+    x_sets = [wl.x.clone()] + [mi.make_x(shape, T, seed + 100 * rank + 10 * j, device=device)
+                               for j in range(1, N_INPUT_SETS)]
+
+    def rotate(i):
+        wl.x.copy_(x_sets[i % N_INPUT_SETS])
+
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     n0 = wl.moe.kernel_launch_count()
     with ClockSampler(local) as clk:
-        times = time_steps(run_step, args.steps, flush)
+        times = time_steps(run_step, args.steps, flush, before=rotate)
     torch.cuda.synchronize()
     launches = wl.moe.kernel_launch_count() - n0
     if not args.no_graph:
@@ -597,6 +622,7 @@ def main():
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4),
+        **step_percentiles(times),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -609,6 +635,7 @@ def main():
                    "parallelism": f"replicas x{world} (data parallel, no collective)",
                    "launch": "host launches" if args.no_graph else "CUDA graph replay of moe_layer_forward",
                    "l2": "flushed between steps (2 GiB write outside the events); weights exceed L2",
+                   "inputs": f"{N_INPUT_SETS} seeded token sets rotated step by step (copied in outside the events)",
                    "shared_sms": moe.shared_sms(wl.cfg),
                    "padding": "max-value" if args.pad_mode == 1 else "block-wise",
                    "top_k": (f"per-token dynamic, uniform 1..{shape.K} (sum {wl.A})" if args.dynamic_k

@@ -40,3 +40,10 @@ def test_tp_rank_work_splits_all_but_the_router(world):
     router_b, router_f = 8 * 4096 * 2, 2 * 32 * 4096 * 8
     assert world * b == pytest.approx(B + (world - 1) * router_b)
     assert world * f == pytest.approx(F + (world - 1) * router_f)
+
+
+def test_step_percentiles_nearest_rank():
+    t = [float(v) for v in range(1, 21)]          # 1 .. 20 ms
+    p = bench.step_percentiles(list(reversed(t)))
+    assert p == {"ms_median": 10.5, "ms_p10": 2.0, "ms_p90": 18.0}
+    assert bench.step_percentiles([3.0]) == {"ms_median": 3.0, "ms_p10": 3.0, "ms_p90": 3.0}
