@@ -365,41 +365,52 @@ def dense_times(shape, T, I_d, steps, warmup, flush, device, seed, fp8=False):
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_tokens_per_s(wl, budget_s=15.0, max_tokens=None):
+def oracle_tokens_per_s(wl, budget_s=15.0, max_tokens=None, budget_1core_s=5.0):
     """The oracle as it stands on a bounded sample of the workload's tokens,
-    all host cores, routing on the GPU path's logits (read back)."""
-    import numpy as np
-    import oracle
+    all host cores and one core, routing on the GPU path's logits (read back)."""
     shape = wl.shape
-    nthreads = os.cpu_count() or 1
     logits = wl.logits
     if logits is None:
         logits = wl.moe.router_gemm(wl.cfg, wl.x, wl.w["w_r"], wl.gws, wl.s_logits)
     lg = logits.float().cpu().numpy()
-    xh = mi.to_oracle(wl.x)
-    w13 = mi.to_oracle(wl.w["w13"])
-    w2 = mi.to_oracle(wl.w["w2"])
     sh = {}
     if shape.I_sh:
         sh = dict(w13_sh=mi.to_oracle(wl.w["w13_sh"]), w2_sh=mi.to_oracle(wl.w["w2_sh"]))
-    T = wl.T
+    return time_oracle(shape, mi.to_oracle(wl.x), mi.to_oracle(wl.w["w13"]), mi.to_oracle(wl.w["w2"]), sh, lg,
+                       budget_s, max_tokens, budget_1core_s)
 
-    def run(n):
+
+def time_oracle(shape, xh, w13, w2, sh, lg, budget_s=15.0, max_tokens=None, budget_1core_s=5.0,
+                nthreads=None):
+    """Oracle tokens/s on the first tokens of host inputs: a sample sized for
+    about budget_s of work on all threads, then one sized for budget_1core_s
+    on one thread."""
+    import numpy as np
+    import oracle
+    nthreads = nthreads or os.cpu_count() or 1
+    T = xh.shape[0]
+
+    def run(n, threads):
         tok = np.arange(n, dtype=np.int32)
         t0 = time.perf_counter()
         oracle.moe_layer(xh, None, w13, w2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok,
-                         nthreads=nthreads, **sh)
+                         nthreads=threads, **sh)
         return time.perf_counter() - t0
 
     n = min(T, nthreads)
-    t1 = run(n)
+    t1 = run(n, nthreads)
     per_tok = t1 / n
     n2 = int(max(1, min(T if max_tokens is None else max_tokens, budget_s / max(per_tok, 1e-9))))
     n2 = max(n2 - n2 % nthreads, min(T, nthreads)) if n2 >= nthreads else n2
-    t2 = run(n2)
+    t2 = run(n2, nthreads)
+    # one core: a token costs about nthreads times the all-threads time per token
+    n1 = int(max(1, min(T, budget_1core_s / max(t2 / n2 * nthreads, 1e-9))))
+    t3 = run(n1, 1)
     return {"value": n2 / t2, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
             "sample": f"first {n2} of the {T} tokens of the workload (all {nthreads} host threads, "
-                      f"{t2:.1f} s), routing on the GPU path's fp32 logits"}
+                      f"{t2:.1f} s), routing on the GPU path's fp32 logits",
+            "value_1core": n1 / t3,
+            "sample_1core": f"first {n1} tokens on one host thread ({t3:.1f} s)"}
 
 
 # ------------------------------------------------------------------- main

@@ -47,3 +47,20 @@ def test_step_percentiles_nearest_rank():
     p = bench.step_percentiles(list(reversed(t)))
     assert p == {"ms_median": 10.5, "ms_p10": 2.0, "ms_p90": 18.0}
     assert bench.step_percentiles([3.0]) == {"ms_median": 3.0, "ms_p10": 3.0, "ms_p90": 3.0}
+
+
+def test_cpu_baseline_timer_reports_all_threads_and_one_core():
+    import numpy as np
+    import oracle
+    shape = mi.SHAPES["tiny"]
+    rng = np.random.default_rng(0)
+    T, H, E, I = 16, shape.H, shape.E, shape.I
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w_r = (rng.standard_normal((E, H)) / np.sqrt(H)).astype(np.float32)
+    w13 = (rng.standard_normal((E, 2 * I, H)) / np.sqrt(H)).astype(np.float32)
+    w2 = (rng.standard_normal((E, H, I)) / np.sqrt(I)).astype(np.float32)
+    lg = oracle.router_logits(x, w_r).astype(np.float32)
+    r = bench.time_oracle(shape, x, w13, w2, {}, lg, budget_s=0.2, budget_1core_s=0.1, nthreads=2)
+    assert r["kind"] == "oracle" and r["cores"] == 2 and r["unit"] == "tokens/s"
+    assert r["value"] > 0 and r["value_1core"] > 0
+    assert "one host thread" in r["sample_1core"]
