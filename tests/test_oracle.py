@@ -730,3 +730,16 @@ def test_tp_pin_catches_a_misaligned_up_slice():
         bad13 = np.ascontiguousarray(np.concatenate([w13[:, lo:hi], w13[:, (lo + 8) % 16:(lo + 8) % 16 + 8]], 1))
         wrong += oracle.moe_layer(x, w_r, bad13, np.ascontiguousarray(w2[..., lo:hi]), K=2)
     assert np.abs(wrong - full).max() > 1e-2 * np.abs(full).max()
+
+
+# -------------------------------------------- workload shapes (input recipe)
+
+def test_layer_shapes_are_the_pages_models():
+    with open(os.path.join(GOLDEN, "layer_shapes.json")) as f:
+        g = json.load(f)
+    for name in ("mixtral", "qwen2moe", "deepseekv3"):
+        s, want = mi.SHAPES[name], g[name]
+        assert (s.H, s.I, s.E, s.K) == (want["H"], want["I"], want["E"], want["K"]), name
+        assert s.I_sh == want["shared"] * want["I"], name
+        assert s.dtype == "bf16"
+    assert mi.SHAPES["deepseekv3"].score_fn == 1 and mi.SHAPES["mixtral"].score_fn == 0
