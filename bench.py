@@ -241,9 +241,47 @@ class Workload:
         m.combine(c, self.s_y, self.al["pos"], self.s_w, self.s_sh, self.out)
         ev[8].record()
 
+    def capture_staged(self):
+        """The staged step in one CUDA graph with timing events between the
+        stages (event record nodes), so that each stage is timed in the same
+        launch context as the step: graph replay, no host launch gaps.
+        Returns (replay, events); on a torch without graph event nodes, the
+        eager staged step and host-launch events."""
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(9)]
+        try:
+            self.staged_step(ev)  # outside capture first: one-time kernel attribute setup
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.staged_step(ev)
+            torch.cuda.synchronize()
+            self.staged_graph = g
+            return g.replay, ev, "CUDA graph replay of the staged calls (event nodes between stages)"
+        except Exception:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+            return (lambda: self.staged_step(ev)), ev, "host launches of the staged calls"
+
     STAGES = ("router", "topk", "align", "permute", "gate_up", "down", "shared", "combine")
     # names when the expert FFN is one fused launch ("down" is then empty)
     STAGES_FUSED = ("router", "topk", "align", "permute", "ffn", "down", "shared", "combine")
+
+
+def staged_breakdown(wl, warmup, steps, flush):
+    """Median per-stage device times (ms) of the staged step, L2 flushed
+    before each replay, and how the stages were launched."""
+    run, ev, how = wl.capture_staged()
+    names = Workload.STAGES_FUSED if wl.fused else Workload.STAGES
+    stage_ms = {s: [] for s in names}
+    for i in range(warmup + steps):
+        flush.zero_()
+        run()
+        ev[8].synchronize()
+        if i >= warmup:
+            for j, s in enumerate(names):
+                stage_ms[s].append(ev[j].elapsed_time(ev[j + 1]))
+    wl.moe.check_status(wl.gws)
+    wl.staged_graph = None
+    return {s: round(statistics.median(v), 4) for s, v in stage_ms.items() if not (wl.fused and s == "down")}, how
 
 
 def l2_flush_buffer(device):
@@ -425,6 +463,8 @@ def main():
     ap.add_argument("--skew", type=float, default=None, help="Zipf exponent of Gumbel router logits")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tau", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode block (Mixtral-shaped T=32, DeepSeek-V3-shaped T=128) of the default line")
     ap.add_argument("--sweep", action="store_true", help="also time every configured workload")
     ap.add_argument("--sweep-out", default=None)
     ap.add_argument("--quick", action="store_true",
@@ -438,6 +478,8 @@ def main():
                     help="FP8 E4M3 expert weights with row scales (decode sizes)")
     ap.add_argument("--dynamic-k", action="store_true",
                     help="per-token dynamic K: each token's expert count uniform in 1..K (seeded)")
+    ap.add_argument("--tax-model", action="store_true",
+                    help="time every configured workload and its DenseFA, and compare tau with the analytic model")
     ap.add_argument("--padding-model", action="store_true",
                     help="time the expert FFN over routings and fit the padding and max-affine latency models")
     ap.add_argument("--tp", action="store_true",
@@ -476,6 +518,15 @@ def main():
     if args.padding_model:
         if rank == 0:
             print(json.dumps(run_padding_model(args, device, flush)), flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if args.tax_model:
+        if rank == 0:
+            rows = run_sweep(args, device, flush, pk, skew=False)
+            print(json.dumps({"tax_model": tax_model_report(rows, pk["hbm_gbs"], pk["bf16_tflops"]),
+                              "peak_source": pk_kind, "rows": rows}), flush=True)
         if dist:
             dist.barrier()
             dist.destroy_process_group()
@@ -528,19 +579,9 @@ def main():
     P, E_active = stats[0], stats[1]
     ms_step = total_ms / args.steps
     value = replica_tokens_per_s(world, T, args.steps, total_ms)
-    # ---- per-stage breakdown (same kernels, one ABI call per stage)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
-    names = Workload.STAGES_FUSED if wl.fused else Workload.STAGES
-    stage_ms = {s: [] for s in names}
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        wl.staged_step(ev)
-        ev[8].synchronize()
-        if i >= args.warmup:
-            for j, s in enumerate(names):
-                stage_ms[s].append(ev[j].elapsed_time(ev[j + 1]))
-    wl.moe.check_status(wl.gws)
-    stages = {s: round(statistics.median(v), 4) for s, v in stage_ms.items() if not (wl.fused and s == "down")}
+    # ---- per-stage breakdown (same kernels, one ABI call per stage, replayed
+    # from a CUDA graph with event nodes between the stages)
+    stages, staged_launch = staged_breakdown(wl, args.warmup, args.steps, flush)
 
     if args.quick:
         if rank == 0:
@@ -617,6 +658,10 @@ def main():
                "t_moe_ms": round(t_moe, 4), "t_DenseFA_ms": round(t_fa, 4), "t_DensePA_ms": round(t_pa, 4),
                "I_FA": shape.I_FA, "I_PA": shape.I_PA}
 
+    decode = None
+    if not args.no_decode:
+        decode = decode_block(device, flush, pk, args.steps, args.warmup, rank)
+
     sweep = None
     if args.sweep:
         sweep = run_sweep(args, device, flush, pk)
@@ -659,7 +704,9 @@ def main():
                   "hbm_GBs_alg": round(B_alg / t_layer / 1e9, 1), "tflops_alg": round(F_alg / t_layer / 1e12, 2)},
         "stages_ms": stages,
         "staged_total_ms": round(sum(stages.values()), 4),
+        "staged_launch": staged_launch,
         "tau": tau,
+        "decode": decode,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
@@ -672,6 +719,51 @@ def main():
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+DECODE_POINTS = (("mixtral", 32), ("deepseekv3", 128))
+
+
+def decode_block(device, flush, pk, steps, warmup, rank=0):
+    """The HBM-bound half of the metric on the default line: decode-sized
+    layers (the Mixtral-8x7B-shaped layer at T = 32 and the largest
+    single-GPU configuration, the DeepSeek-V3-shaped layer at T = 128), each
+    timed like the headline (CUDA graph replay, L2 flushed before every step,
+    four rotated token sets), with the fused expert FFN's stage time, the
+    fractions of the measured copy bandwidth and of 8 TB/s, and tau against
+    DenseFA at the same T."""
+    out = []
+    for name, T in DECODE_POINTS:
+        sh = mi.SHAPES[name]
+        wl = Workload(sh, T, rank, device)
+        wl.capture()
+        for _ in range(warmup):
+            wl.replay()
+        torch.cuda.synchronize()
+        seed = mi.seed_for(sh, T)
+        xs = [wl.x.clone()] + [mi.make_x(sh, T, seed + 100 * rank + 10 * j, device=device)
+                               for j in range(1, N_INPUT_SETS)]
+        times = time_steps(wl.replay, steps, flush, before=lambda i: wl.x.copy_(xs[i % N_INPUT_SETS]))
+        wl.moe.check_status(wl.ws)
+        st = wl.stats.cpu().tolist()
+        stages, _ = staged_breakdown(wl, 3, max(5, steps // 2), flush)
+        t = statistics.median(times)
+        B, F = algorithmic(sh, T, st[1])
+        fb, _ = ffn_work(sh, T, st[1])
+        t_ffn = stages.get("ffn") or (stages["gate_up"] + stages["down"])
+        del wl, xs
+        torch.cuda.empty_cache()
+        t_fa = dense_times(sh, T, sh.I_FA, max(5, steps // 2), 3, flush, device, mi.seed_for(sh, T, 50))
+        out.append({"workload": f"{name}:{T}", "ms_median": round(t, 4), "tokens_per_s": round(T / t * 1e3, 1),
+                    "E_active": st[1], "P": st[0], "bytes_alg": B,
+                    "hbm_GBs_alg": round(B / t / 1e6, 1),
+                    "hbm_frac_measured": round(B / (t * 1e-3) / (pk["hbm_gbs"] * 1e9), 4),
+                    "hbm_frac_8TBs": round(B / (t * 1e-3) / (HBM_NOMINAL_GBS * 1e9), 4),
+                    "ffn_ms": round(t_ffn, 4),
+                    "ffn_hbm_frac_measured": round(fb / (t_ffn * 1e-3) / (pk["hbm_gbs"] * 1e9), 4),
+                    "tau_FA": round(t / t_fa, 4), "t_DenseFA_ms": round(t_fa, 4)})
+        torch.cuda.empty_cache()
+    return out
 
 
 def tp_rank_work(shape, T, E_active, world):
@@ -804,7 +896,100 @@ def run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind)
     }
 
 
-def run_sweep(args, device, flush, pk):
+# ---------------------------------------------------- analytic tax model
+# Demystifying the MoE Serving Tax, "Validation of the analytic model
+# (Section 5.3)": the pages give the model's parameters for A100-40GB
+# (HBM 1500 GB/s, 312 TFLOP/s bf16, padding overhead eta = 1.05 in decode and
+# 1.25 in prefill), its three regimes (memory-bound, compute-bound and the
+# transition between them) and its accuracy (within 10-30 % of measured), not
+# its formula.  Reading taken here, the plainest one the printed endpoints
+# support: each layer takes the roofline time of its algorithmic bytes and
+# flops, the MoE layer's multiplied by the phase's eta,
+#   t_MoE = eta * max(B_MoE / BW, F_MoE / FLOPS),  t_FA = max(B_FA / BW, F_FA / FLOPS),
+#   tau = t_MoE / t_FA,
+# with B_MoE counting the expected activated experts E (1 - (1 - K/E)^T)
+# ("Balls-Bins-Buckets").  At T = 1 both layers read the same expert bytes and
+# tau = eta_decode (the pages: 1.05x for Mixtral at one request); at large T
+# both are compute-bound with equal flops and tau = eta_prefill (the pages:
+# about 1.28x at 1024-2048 tokens).
+PAGES_TAX_MODEL = {"hardware": "A100-40GB (the pages' validation)", "bw_gbs": 1500.0, "tflops": 312.0,
+                   "eta_decode": 1.05, "eta_prefill": 1.25}
+
+
+def expected_active(E, K, T):
+    """E[E_active] = E (1 - (1 - K/E)^T) under uniform routing (talk notes,
+    "Balls-Bins-Buckets" model construction)."""
+    return E * (1.0 - (1.0 - K / E) ** T)
+
+
+def dense_fa_work(shape, T):
+    """DenseFA's algorithmic bytes (its weights, read once) and flops: a dense
+    SwiGLU FFN of width I_FA = K I + S I_s, no router."""
+    eb = 2 if shape.dtype == "bf16" else 4
+    return 3.0 * shape.H * shape.I_FA * eb, 2.0 * T * 3 * shape.H * shape.I_FA
+
+
+def tax_model(shape, T, bw_gbs, tflops, eta, E_active=None):
+    """Predicted MoE and DenseFA layer times (s), tau and the regime."""
+    if E_active is None:
+        E_active = expected_active(shape.E, shape.K, T)
+    B_m, F_m = algorithmic(shape, T, E_active)
+    B_d, F_d = dense_fa_work(shape, T)
+    bw, fl = bw_gbs * 1e9, tflops * 1e12
+    mem_m, cmp_m = B_m / bw, F_m / fl
+    mem_d, cmp_d = B_d / bw, F_d / fl
+    t_m, t_d = eta * max(mem_m, cmp_m), max(mem_d, cmp_d)
+    if mem_m >= cmp_m and mem_d >= cmp_d:
+        regime = "memory"
+    elif mem_m < cmp_m and mem_d < cmp_d:
+        regime = "compute"
+    else:
+        regime = "transition"
+    return {"t_moe_s": t_m, "t_fa_s": t_d, "tau": t_m / t_d, "regime": regime, "E_active": E_active}
+
+
+def phase_of(shape, T):
+    return "prefill" if T in shape.prefill_T else "decode"
+
+
+def fit_eta(taus, ratios):
+    """Least-squares eta of tau = eta * ratio (ratio: the roofline tau with
+    eta = 1) over a phase's points."""
+    num = sum(t * r for t, r in zip(taus, ratios))
+    den = sum(r * r for r in ratios)
+    return num / den if den > 0 else float("nan")
+
+
+def tax_model_report(rows, bw_gbs, tflops):
+    """Predicted against measured tau_FA for every measured configuration
+    (rows: layer, T, tau_FA), with the pages' eta constants on this GPU's
+    peaks and with eta fitted per phase to the measurements."""
+    pts = []
+    for r in rows:
+        sh = mi.SHAPES[r["layer"]]
+        ph = phase_of(sh, r["T"])
+        base = tax_model(sh, r["T"], bw_gbs, tflops, 1.0)
+        pts.append((r, sh, ph, base))
+    eta_fit = {}
+    for ph in ("decode", "prefill"):
+        sel = [(r["tau_FA"], b["tau"]) for r, sh, p, b in pts if p == ph]
+        eta_fit[ph] = fit_eta([a for a, _ in sel], [b for _, b in sel]) if sel else None
+    table = []
+    for r, sh, ph, b in pts:
+        e_pages = PAGES_TAX_MODEL["eta_" + ph]
+        tp, tf = e_pages * b["tau"], eta_fit[ph] * b["tau"]
+        table.append({"layer": r["layer"], "T": r["T"], "phase": ph, "regime": b["regime"],
+                      "tau_measured": r["tau_FA"], "tau_model_pages_eta": round(tp, 4),
+                      "err_pages_eta_pct": round(100.0 * (tp - r["tau_FA"]) / r["tau_FA"], 1),
+                      "tau_model_fitted_eta": round(tf, 4),
+                      "err_fitted_eta_pct": round(100.0 * (tf - r["tau_FA"]) / r["tau_FA"], 1),
+                      "E_active_model": round(b["E_active"], 2), "E_active_measured": r.get("E_active")})
+    return {"bw_gbs": bw_gbs, "tflops": tflops, "eta_pages": {"decode": PAGES_TAX_MODEL["eta_decode"],
+                                                               "prefill": PAGES_TAX_MODEL["eta_prefill"]},
+            "eta_fitted": eta_fit, "points": table}
+
+
+def run_sweep(args, device, flush, pk, skew=True):
     """Every configured workload (decode and prefill T of each layer shape) and
     the DeepSeek-V3-shaped routing-skew sweep (Zipf s in {0, 0.5, 1, 1.5},
     T = 1 .. 4096 in powers of two): tokens/s, activated experts, padded
@@ -817,7 +1002,7 @@ def run_sweep(args, device, flush, pk):
         sh = mi.SHAPES[name]
         weights = mi.make_weights(sh, mi.seed_for(sh, 0), device=device)
         plan = [(T, None) for T in sh.decode_T + sh.prefill_T]
-        if name == "deepseekv3":
+        if name == "deepseekv3" and skew:
             plan += [(2 ** k, s) for s in (0.0, 0.5, 1.0, 1.5) for k in range(13)]
         fa_cache = {}
         for T, s in plan:
@@ -856,12 +1041,12 @@ def run_sweep(args, device, flush, pk):
 def ffn_time(wl, steps, flush):
     """Median device time (ms) of the routed expert FFN alone (the fused
     launch, or gate/up + down), from the per-stage events of staged steps."""
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+    run, ev, _ = wl.capture_staged()
     names = Workload.STAGES_FUSED if wl.fused else Workload.STAGES
     out = []
     for i in range(3 + steps):
         flush.zero_()
-        wl.staged_step(ev)
+        run()
         ev[8].synchronize()
         if i >= 3:
             st = {s: ev[j].elapsed_time(ev[j + 1]) for j, s in enumerate(names)}

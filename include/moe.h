@@ -88,7 +88,13 @@ typedef struct {
 /* Text for a status code (static storage). */
 const char* moe_status_string(int status);
 
-/* Upper bound on padded rows: P_max = A + min(E, A) * (B - 1), A = T * K. */
+/* Upper bound on padded rows, the length callers give sorted_ids and the
+ * permuted buffers (-1 on a bad configuration), A = T * K:
+ *   pad_mode 0 (block-wise): P_max = A + min(E, A) * (B - 1);
+ *   pad_mode 1 (max-value):  P_max = E * ceil(min(T, A) / B) * B, which
+ *     assumes an expert holds at most one assignment per token (true of every
+ *     top-K routing); ids that repeat within a token are flagged by the
+ *     alignment instead (see moe_align_pad). */
 int64_t moe_padded_rows_max(const moe_config_t* cfg);
 
 /* Bytes of workspace moe_layer_forward needs for this configuration on the
@@ -121,8 +127,8 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
 
 /* Router GEMM for callers that cannot allocate device memory when they
  * enqueue work -- for example a plugin inside another engine whose enqueue
- * step must not allocate, or code captured into a CUDA graph under a mode
- * that forbids cudaMalloc.  The pages have no counterpart: this is a library
+ * step must not allocate, or a runtime that plans every byte of device memory
+ * before it starts.  The pages have no counterpart: this is a library
  * convenience, not a step of the method.
  *   Same arguments as moe_router_gemm, minus the workspace, and always the
  *   tensor-core form (equal to moe_router_gemm's result up to fp32 rounding
@@ -135,9 +141,19 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
  *   device address (cudaGetSymbolAddress); make that first call before any
  *   stream capture.  Each call clears the shared control words before its
  *   launch; calls that overlap on the GPU (unordered streams) race on the
- *   shared array.  A device wait that runs out leaves logits unwritten. */
+ *   shared array.  A device wait that runs out sets a status word in the
+ *   array and may leave logits partly written (the tiles whose blocks gave up);
+ *   moe_router_gemm_noalloc_status reports it. */
 int moe_router_gemm_noalloc(const moe_config_t* cfg, const void* x, const void* w_router,
                             float* logits, moe_stream_t stream);
+
+/* Status of the moe_router_gemm_noalloc calls enqueued on `stream` so far:
+ * synchronises the stream, reads the status word of the fixed array and
+ * clears it.  MOE_ERR_TIMEOUT when a device wait ran out (the logits of that
+ * call are not to be used), MOE_OK otherwise, MOE_ERR_CUDA on a CUDA error.
+ * The next moe_router_gemm_noalloc call also clears the word, so call this
+ * before it.  No allocation.  The pages have no counterpart. */
+int moe_router_gemm_noalloc_status(moe_stream_t stream);
 
 /* Top-K gating (stage "top-K selection"), one token per warp:
  *   topk_ids[T,K]: the K largest logits[t,:], descending, the lower expert
@@ -173,7 +189,11 @@ int moe_route_k(const moe_config_t* cfg, const float* logits, const int32_t* k_p
  *   scalars[4]       {P, E_active = #{e : N_e > 0}, 0, 0}
  * Bit-exact and deterministic.  Id -1 is an empty slot (per-token dynamic K):
  * no row, pos -1.  Other out-of-range ids are skipped and flagged in
- * scalars[2] (nonzero = bad input). */
+ * scalars[2] (bit 1; nonzero = bad input).  Max-value padding with ids that
+ * repeat within a token (no top-K produces them) can need more than P_max rows:
+ * the alignment then sets bit 2 of scalars[2] and writes an empty routing
+ * (P = 0, E_active = 0, offsets 0, every pos -1, sorted_ids and block_expert
+ * -1), writing nothing at or past P_max. */
 int moe_align_pad(const moe_config_t* cfg, const int32_t* topk_ids, int32_t* counts,
                   int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert,
                   int32_t* pos, int32_t* scalars, moe_stream_t stream);
@@ -253,7 +273,7 @@ int moe_quantize_fp8(int64_t rows, int cols, int dtype, const void* w, uint8_t* 
  * w13_q [E,2I,H], w2_q [E,H,I] with row scales w13_s [E,2I], w2_s [E,H]
  * (shared likewise, [2*I_sh,H] / [H,I_sh] with [2*I_sh] / [H]); x, the router
  * and the output stay bf16 (cfg->dtype 0).  The codes stream from HBM and are
- * widened to f16 in shared memory (exact); the expert MMAs run on f16
+ * widened to f16 in tensor memory (exact); the expert MMAs run on f16
  * operands (x and the SwiGLU activations converted to f16, so |x| and the
  * activations must stay within the f16 range) with fp32 accumulation, and
  * each output row is multiplied by its fp32 scale.  Decode sizes only: the expert FFNs
@@ -303,7 +323,10 @@ int dense_ffn(int T, int H, int I, int dtype, const void* x, const void* w13,
 /* Synchronise `stream`, then read and clear the workspace status words
  * (the caller's-stream kernels' and the concurrent shared FFN's).
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a device wait ran out; the control words
- * are re-zeroed so the workspace stays usable) or MOE_ERR_CUDA. */
+ * are re-zeroed so the workspace stays usable), MOE_ERR_ARG (a fused expert
+ * FFN launch was handed segment offsets that form more token chunks than its
+ * tables hold -- offsets inconsistent with the configuration; it did no work)
+ * or MOE_ERR_CUDA. */
 int moe_check_status(void* workspace, moe_stream_t stream);
 
 /* Device-side wait limit in nanoseconds for subsequent launches (default
@@ -315,6 +338,18 @@ void moe_set_wait_limit_ns(uint64_t ns);
  * expected rows per expert, T*K/E.  Results are unchanged; only speed
  * differs.  Process-wide.  Returns MOE_ERR_ARG for other values. */
 int moe_set_token_tile_cap(int n);
+
+/* Tuning: how the grouped GEMM shares out the tiles left after its whole
+ * waves of one tile per SM (or SM pair), for subsequent launches.
+ *   1: every whole wave data-parallel; the tiles of the last
+ *     partial wave cut into equal k-slices, taken slice-major, so that tiles
+ *     sharing a weight block or a token chunk stream the same slice together;
+ *   0 (default): stream-K over the last one to two waves, in contiguous ranges of
+ *     (tile, k-iteration) units.
+ * Split tiles are summed in a fixed order by the last contributor; results
+ * agree up to fp32 summation order.  Process-wide.  MOE_ERR_ARG for other
+ * values. */
+int moe_set_split_tail(int mode);
 
 /* 1 when moe_grouped_ffn / moe_layer_forward run this configuration's
  * expert FFN as one fused launch (gate/up + SwiGLU and down in a persistent

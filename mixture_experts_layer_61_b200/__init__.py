@@ -89,6 +89,7 @@ def lib():
             "moe_debug_withhold_first_load": (None, [I]),
             "moe_set_token_tile_cap": (I, [I]),
             "moe_set_programmatic_launch": (None, [I]),
+            "moe_set_split_tail": (I, [I]),
             "moe_set_cta_pairs": (None, [I]),
             "moe_set_shared_sms": (I, [I]),
             "moe_shared_sms": (I, [C]),
@@ -354,6 +355,12 @@ def set_wait_limit_ns(ns):
 def set_token_tile_cap(n):
     """Force the grouped GEMM's token-tile cap (32/64/128/256; 0 = automatic)."""
     _check(lib().moe_set_token_tile_cap(int(n)), "moe_set_token_tile_cap")
+
+
+def set_split_tail(mode=1):
+    """GEMM tail schedule: 1 aligned k-slices of the last partial wave, 0
+    contiguous stream-K over the last one to two waves (the library default)."""
+    _check(lib().moe_set_split_tail(int(mode)), "moe_set_split_tail")
 
 
 def set_programmatic_launch(enable=True):

@@ -880,11 +880,14 @@ int moe_check_status(void* workspace, moe_stream_t stream) {
         if (!ok) cudaGetLastError();
         return ok;
     };
-    if ((st[0] | st[1]) & kStatusTimeout) {
+    const unsigned kBad = kStatusTimeout | kStatusCapacity;
+    if ((st[0] | st[1]) & kBad) {
         if (!rezero(workspace)) return MOE_ERR_CUDA;
-        if ((st[1] & kStatusTimeout) && !rezero(static_cast<uint8_t*>(workspace) + align256(ctl_block_bytes(d.num_sms))))
+        if ((st[1] & kBad) && !rezero(static_cast<uint8_t*>(workspace) + align256(ctl_block_bytes(d.num_sms))))
             return MOE_ERR_CUDA;
-        return MOE_ERR_TIMEOUT;
+        // a wait that ran out is a timeout; work that did not fit the kernel's
+        // tables came from segment offsets inconsistent with the configuration
+        return ((st[0] | st[1]) & kStatusTimeout) ? MOE_ERR_TIMEOUT : MOE_ERR_ARG;
     }
     return MOE_OK;
 }
@@ -898,6 +901,12 @@ int moe_set_token_tile_cap(int n) {
 }
 
 void moe_set_programmatic_launch(int enable) { set_pdl(enable != 0); }
+
+int moe_set_split_tail(int mode) {
+    if (mode != 0 && mode != 1) return MOE_ERR_ARG;
+    set_split_tail(mode);
+    return MOE_OK;
+}
 
 int moe_set_shared_sms(int n) {
     if (n < -1) return MOE_ERR_ARG;

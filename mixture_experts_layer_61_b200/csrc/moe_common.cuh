@@ -18,6 +18,7 @@ namespace moe {
 enum : unsigned {
     kStatusTimeout = 1u,   // a bounded wait ran out
     kStatusBadIds = 2u,    // an expert id outside [0, E) reached the alignment
+    kStatusCapacity = 4u,  // a launch's work exceeded a kernel's fixed tables (inconsistent segment offsets)
 };
 
 // ------------------------------------------------------------ type traits

@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             uint32_t kc = 0, n = 0;
             bool withhold = false;  // test hook: armed for work item 0, whichever block takes it
             bool ok = !oversize;
-            if (oversize) atomicOr(p.status, kStatusTimeout);
+            if (oversize) atomicOr(p.status, kStatusCapacity);  // not a wait: the item space does not fit
             while (true) {
                 const int rs = n % kFfnRing;
                 const uint32_t rph = (n / kFfnRing) & 1u;
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             }
             if (!ok) {
                 *abort_flag = 1;
-                atomicOr(p.status, kStatusTimeout);
+                if (!oversize) atomicOr(p.status, kStatusTimeout);
             }
             for (int s = 0; s < C::kStages; ++s)
                 if (fills[s] > 0) mbar_drain(&full[s], (uint32_t)(fills[s] - 1) & 1u, limit);

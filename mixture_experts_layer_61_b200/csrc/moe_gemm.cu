@@ -104,6 +104,7 @@ int launch_variant(const GemmLaunch& L, const GemmCtl& ctl, int num_sms, cudaStr
     p.withhold_first_load = take_withhold_flag();
     p.sk_min_units = 4;
     p.max_split = L.max_split > 0 ? L.max_split : 4;
+    p.split_tail = split_tail_mode();
     int grid = grid_blocks;
     if (L.sms > 0 && L.sms < grid) grid = L.sms >= 2 * kCta ? L.sms - L.sms % kCta : kCta;
     cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(kGemmThreads), C::kSmemBytes, stream, kCta,
@@ -269,9 +270,12 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
 
 namespace {
 int g_token_tile_cap = 0;  // 0: automatic
+int g_split_tail = 0;      // contiguous stream-K over the last one to two waves
 }
 
 void set_token_tile_cap(int n) { g_token_tile_cap = n; }
+void set_split_tail(int mode) { g_split_tail = mode; }
+int split_tail_mode() { return g_split_tail; }
 void set_cta_pairs(bool on) { g_cta_pairs = on; }
 
 int pick_max_n(double rows_per_group) {

@@ -71,6 +71,7 @@ struct GemmParams {
     int withhold_first_load;
     int sk_min_units;     // minimum k-iterations per stream-K block
     int max_split;        // stream-K: most blocks contributing to one tile
+    int split_tail;       // 1: whole waves data-parallel, the last partial wave in aligned k-slices
 };
 
 // Epilogue kinds: one 128-row weight tile per stage (plain store); gate and
@@ -119,19 +120,52 @@ struct Tile {
     int group, f0, row0, nrows, mma_n, wrow, nch, chunk;
 };
 
+// Two ways to share out the tiles left after the whole data-parallel waves:
+//  * contiguous stream-K (split_tail 0): the last one to two waves of tiles
+//    as one range of (tile, k-iteration) units cut evenly across the blocks;
+//  * aligned slices (split_tail 1): every whole wave data-parallel, and the
+//    tiles of the last partial wave each cut into S equal k-slices, taken
+//    slice-major and dealt round-robin (block c takes units c and c + G).
+//    Tiles that share a weight block (adjacent token chunks) or a token chunk
+//    (feature blocks of one expert) then stream the same k-slice at the same
+//    time, so the shared operand is read from DRAM once; with contiguous
+//    ranges the sharing tiles sit at different k-offsets and each reads it.
 struct Sched {
     int n_groups, NF, KI, G, cta;
     long long total_tiles, dp_waves, dp_tiles, sk_tiles, U;
     int G_sk;
+    int S;              // aligned slices per tail tile (0: contiguous stream-K)
     // iteration state
     long long w;        // next DP wave
     long long u, u_end; // stream-K cursor
     bool sk_first;
+    int next_unit;      // aligned slices: this block's next local unit (0 or 1)
 
     __device__ long long beg(int c) const { return (long long)c * U / G_sk; }
     // block owning stream-K unit q
     __device__ int owner(long long q) const { return (int)(((q + 1) * (long long)G_sk - 1) / U); }
 };
+
+// Slices per tail tile for the aligned split: at most 2 units per block (the
+// two partial slots), at least min_units k-iterations per slice, at most
+// max_split contributors per tile; among those, the fewest slices with the
+// shortest tail, ceil(tail * S / G) / S tile-times.
+__device__ __forceinline__ int aligned_slices(long long tail, int G, int KI, long long min_units, int max_split) {
+    if (tail <= 0) return 1;
+    long long smax = (2LL * G) / tail;
+    if (smax > max_split) smax = max_split;
+    if (smax > KI / min_units) smax = KI / min_units;
+    int best = 1;
+    double best_t = (double)((tail + G - 1) / G);
+    for (int s = 2; s <= smax; ++s) {
+        const double t = (double)((tail * s + G - 1) / G) / s;
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = s;
+        }
+    }
+    return best;
+}
 
 struct Item {
     long long tile;
@@ -149,6 +183,23 @@ __device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int to
     s.G = gridDim.x / ncta;
     s.cta = blockIdx.x / ncta;
     s.total_tiles = (long long)total_chunks * NF;
+    // at most max_split blocks share one tile: every block takes >= KI / kMaxSplit k-iterations
+    long long min_units = (KI + p.max_split - 1) / p.max_split;
+    if (min_units < p.sk_min_units) min_units = p.sk_min_units;
+    s.S = 0;
+    s.next_unit = 0;
+    if (p.split_tail) {
+        s.dp_waves = s.total_tiles / s.G;
+        s.dp_tiles = s.dp_waves * s.G;
+        s.sk_tiles = s.total_tiles - s.dp_tiles;  // < G: fits the counters and two slots per block
+        s.S = aligned_slices(s.sk_tiles, s.G, KI, min_units, p.max_split);
+        s.U = 0;
+        s.G_sk = s.G;
+        s.w = 0;
+        s.u = s.u_end = 0;
+        s.sk_first = true;
+        return;
+    }
     // Whole waves first, keeping one to two waves for the stream-K tail; with
     // fewer than two waves of tiles, one whole wave and the rest as stream-K,
     // so that the token chunks sharing a weight block (adjacent tiles) stream
@@ -157,9 +208,6 @@ __device__ __forceinline__ void sched_init(Sched& s, const GemmParams& p, int to
     s.dp_tiles = s.dp_waves * s.G;
     s.sk_tiles = s.total_tiles - s.dp_tiles;
     s.U = s.sk_tiles * KI;
-    // at most max_split blocks share one tile: every block takes >= KI / kMaxSplit k-iterations
-    long long min_units = (KI + p.max_split - 1) / p.max_split;
-    if (min_units < p.sk_min_units) min_units = p.sk_min_units;
     long long gsk = s.U / min_units;
     if (gsk < 1) gsk = 1;
     if (gsk > s.G) gsk = s.G;
@@ -198,6 +246,21 @@ __device__ __forceinline__ bool sched_next(Sched& s, Item& it) {
         it.slot = s.sk_first ? 0 : 1;
         s.sk_first = false;
         s.u += ke - kb;
+        return true;
+    }
+    if (s.S > 0 && s.next_unit < 2) {
+        // aligned slices: unit q = cta + j G is slice q / tail of tail tile q % tail
+        const long long q = (long long)s.cta + (long long)s.next_unit * s.G;
+        if (q >= s.sk_tiles * s.S) return false;
+        const long long st = q % s.sk_tiles;
+        const int sl = (int)(q / s.sk_tiles);
+        it.tile = s.dp_tiles + st;
+        it.kb = (int)((long long)sl * s.KI / s.S);
+        it.ke = (int)((long long)(sl + 1) * s.KI / s.S);
+        it.sk_tile = st;
+        it.split = s.S > 1;
+        it.slot = s.next_unit;
+        ++s.next_unit;
         return true;
     }
     return false;
@@ -677,13 +740,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (e == 0) *bcast = atomicAdd(&p.counters[counter], 1);
                 named_sync(1, kEpiThreads);
                 const int arrived = *bcast;
-                // contributors: blocks whose stream-K range meets this tile
+                // contributors: blocks whose stream-K range meets this tile, or
+                // (aligned slices) the S slices' units
+                const bool aligned = sch.S > 0;
                 const long long q0 = it.sk_tile * sch.KI;
-                const int c_first = sch.owner(q0);
-                const int c_last = sch.owner(q0 + sch.KI - 1);
+                const int c_first = aligned ? 0 : sch.owner(q0);
+                const int c_last = aligned ? sch.S - 1 : sch.owner(q0 + sch.KI - 1);
                 int ncontrib = 0;
-                for (int c = c_first; c <= c_last; ++c)
-                    if (sch.beg(c) < sch.beg(c + 1)) ++ncontrib;
+                if (aligned) {
+                    ncontrib = sch.S;
+                } else {
+                    for (int c = c_first; c <= c_last; ++c)
+                        if (sch.beg(c) < sch.beg(c + 1)) ++ncontrib;
+                }
                 if (arrived == ncontrib - 1) {
                     // last to arrive: sum every contribution in block order, then the epilogue
                     __threadfence();
@@ -691,10 +760,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         float g[16], u[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
-                        for (int c = c_first; c <= c_last; ++c) {
-                            const long long bc = sch.beg(c);
-                            if (bc >= sch.beg(c + 1)) continue;
-                            if (c == sch.cta) {
+                        for (int i = c_first; i <= c_last; ++i) {
+                            // contributor i: a block (contiguous) or a slice (aligned), in k order
+                            int c, slot;
+                            if (aligned) {
+                                const long long q = it.sk_tile + (long long)i * sch.sk_tiles;
+                                c = (int)(q % sch.G);
+                                slot = (int)(q / sch.G);
+                            } else {
+                                c = i;
+                                const long long bc = sch.beg(c);
+                                if (bc >= sch.beg(c + 1)) continue;
+                                slot = (bc / sch.KI == it.sk_tile) ? 0 : 1;
+                            }
+                            if (c == sch.cta && slot == it.slot) {
                                 uint32_t va[16], vb[16];
                                 tmem_ld16_nowait(tacc + c0, va);
                                 if (kTwo) tmem_ld16_nowait(tacc + kMaxN + c0, vb);
@@ -705,7 +784,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                     if (kTwo) u[i] += __uint_as_float(vb[i]);
                                 }
                             } else {
-                                const int slot = (bc / sch.KI == it.sk_tile) ? 0 : 1;
                                 const float4* other =
                                     reinterpret_cast<const float4*>(p.partials + (((long long)c * kCta + rank) * 2 + slot) *
                                                                                      slot_floats);

@@ -134,6 +134,11 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
 // by set_token_tile_cap, 0 = automatic).
 int pick_max_n(double rows_per_group);
 void set_token_tile_cap(int n);
+// How the GEMM shares out the tiles after its whole data-parallel waves:
+// 0 contiguous stream-K over the last one to two waves (default), 1 aligned
+// k-slices of the last partial wave.
+void set_split_tail(int mode);
+int split_tail_mode();
 // CTA-pair (2-SM MMA) tiles for bf16 launches at the 256-token cap (default on).
 void set_cta_pairs(bool on);
 

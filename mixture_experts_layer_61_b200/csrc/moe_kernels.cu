@@ -217,15 +217,25 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     // the rounded size of the most loaded one.
     const int n = tid < E ? cnt[tid] : 0;
     int padded = ((n + B - 1) / B) * B;
+    // Block-wise padding stays within P_max for any ids (at most min(E, A)
+    // experts each add fewer than B rows).  Max-value padding assumes an
+    // expert holds at most one assignment per token; ids that repeat within a
+    // token can push E * ceil(max N / B) * B past P_max.  Such a routing is
+    // flagged (bit 2 of the bad-input word) and aligned as empty: no rows, no
+    // write at or past P_max.
+    bool overflow = false;
     if (mode == 1) {
         const int wmax = __reduce_max_sync(0xffffffffu, n);
         if (lane == 0 && wmax > 0) atomicMax(nmax, wmax);
         __syncthreads();
-        padded = tid < E ? ((*nmax + B - 1) / B) * B : 0;
+        const long long rows = ((long long)*nmax + B - 1) / B * B;
+        overflow = (long long)E * rows > P_max;
+        padded = tid < E && !overflow ? (int)rows : 0;
+        if (overflow && tid == 0) *bad |= 2;
     }
     int P = 0;
     const int excl = block_excl_scan(padded, warp_tot, P);
-    const int n_active = __syncthreads_count(tid < E && n > 0);
+    const int n_active = overflow ? 0 : __syncthreads_count(tid < E && n > 0);
     if (tid < E) {
         off[tid] = excl;
         cursor[tid] = excl;
@@ -252,7 +262,7 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     const unsigned lt_mask = (1u << lane) - 1u;
     for (long long base = 0; base < A; base += kAlignThreads) {
         const long long a = base + tid;
-        int e = a < A ? ids[a] : -1;
+        int e = a < A && !overflow ? ids[a] : -1;
         if ((unsigned)e >= (unsigned)E) e = -1;
         for (int i = tid; i < 32 * E; i += kAlignThreads) tbl[i] = 0;
         __syncthreads();
@@ -283,8 +293,9 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     }
 
     // padding slots inside each segment, then everything past P
-    for (int e = warp; e < E; e += kAlignThreads / 32)
-        for (int p = off[e] + cnt[e] + lane; p < off[e + 1]; p += 32) sorted_ids[p] = -1;
+    if (!overflow)
+        for (int e = warp; e < E; e += kAlignThreads / 32)
+            for (int p = off[e] + cnt[e] + lane; p < off[e + 1]; p += 32) sorted_ids[p] = -1;
     for (long long p = (long long)P + tid; p < P_max; p += kAlignThreads) sorted_ids[p] = -1;
     const long long nblk = (P_max + B - 1) / B;
     for (long long b = tid; b < nblk; b += kAlignThreads) {

@@ -3,8 +3,7 @@
 //
 // Some callers cannot allocate device memory at the moment they enqueue
 // work: a plugin inside another inference engine whose enqueue hook must not
-// allocate, code recorded into a CUDA graph under a capture mode that forbids
-// cudaMalloc, or a runtime that plans every byte of device memory up front.
+// allocate, or a runtime that plans every byte of device memory up front.
 // For them, moe_router_gemm_noalloc runs the same tensor-core router GEMM as
 // moe_router_gemm but keeps its scratch -- the status word, the stream-K tile
 // counters and the partial tiles -- in a fixed array in the library's own
@@ -15,6 +14,10 @@
 // keep each partial tile at 128 x 32 fp32) and at most kMaxSms SMs.  All calls
 // share the one array: two calls that overlap on the GPU (different streams,
 // no ordering between them) race on it.
+//
+// A bounded device wait that runs out sets the status word inside the array.
+// moe_router_gemm_noalloc_status() reads and clears it; the next
+// moe_router_gemm_noalloc call clears it too, so read it before that call.
 #include "../../include/moe.h"
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -95,4 +98,31 @@ extern "C" int moe_router_gemm_noalloc(const moe_config_t* cfg, const void* x, c
     g.max_n = kTokenTile;
     rc = moe::launch_gemm(g, moe::gemm_ctl(scratch, d.num_sms), s);
     return rc == 0 ? MOE_OK : (rc == -1 ? MOE_ERR_ARG : MOE_ERR_CUDA);
+}
+
+extern "C" int moe_router_gemm_noalloc_status(moe_stream_t stream) {
+    moe::DeviceInfo d;
+    int rc = moe::current_device(&d);
+    if (rc != 0) return rc == -5 ? MOE_ERR_DEVICE : MOE_ERR_CUDA;
+    if (d.num_sms > kMaxSms || d.device >= kMaxDevices) return MOE_ERR_DEVICE;
+    void* scratch = nullptr;
+    if ((rc = scratch_for(d.device, &scratch)) != MOE_OK) return rc;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    unsigned st = 0;
+    if (cudaMemcpy(&st, scratch, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (st & moe::kStatusTimeout) {
+        // the timed-out launch may have left stream-K counters set: clear them with the status word
+        if (cudaMemset(scratch, 0, moe::gemm_ctl_zero_bytes(d.num_sms)) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        return MOE_ERR_TIMEOUT;
+    }
+    return MOE_OK;
 }

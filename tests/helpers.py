@@ -48,3 +48,44 @@ def sample_tokens(T, n, seed):
         return np.arange(T, dtype=np.int32)
     rng = np.random.default_rng(seed)
     return np.sort(rng.choice(T, size=n, replace=False)).astype(np.int32)
+
+
+def layer_case(shape, T, w, x, wh=None, override=None, n_sample=None, sample_seed=0, check_stats=True, pad_mode=0,
+               k=None):
+    """One moe_layer_forward on the GPU against the oracle's layer.
+
+    w / x: device weights and tokens; wh: host copies of the weights (made here
+    when None).  The oracle routes on the logits the layer computed (read back
+    from the workspace), or on `override`; the layer's logits are checked
+    against the oracle's router on the same sampled tokens, spread over all of
+    T.  Returns max|out - ref| / max|ref| over the sampled tokens."""
+    import oracle
+
+    cfg = cfg_for(shape, T, pad_mode=pad_mode)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    stats = torch.zeros(4, dtype=torch.int32, device="cuda")
+    kt = None if k is None else torch.from_numpy(np.asarray(k, np.int32)).cuda()
+    out = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w.get("w13_sh"), w.get("w2_sh"),
+                            logits_override=override, stats=stats, k=kt)
+    moe.check_status(ws)
+    if wh is None:
+        wh = {n: host(t) for n, t in w.items()}
+    tok = sample_tokens(T, n_sample or T, sample_seed)
+    xh = host(x)
+    layer_lg = moe.layer_logits(cfg, ws).cpu().numpy()
+    ref_lg = oracle.router_logits(xh[tok], wh["w_r"])
+    # fp32 tiny layer above the fused routing's 64 tokens: tf32 router products
+    tol = 4e-3 if shape.dtype == "fp32" and T > 64 else 1e-5
+    assert np.abs(layer_lg[tok] - ref_lg).max() / np.abs(ref_lg).max() < tol
+    lg = layer_lg if override is None else override.cpu().numpy()
+    if check_stats:
+        ids = oracle.topk(lg, shape.K, k)
+        r = oracle.align(ids, shape.E, shape.tile_B, mode=pad_mode)
+        st = stats.cpu().numpy()
+        assert st[0] == r["P"] and st[1] == r["E_active"] and st[2] == 0
+    sh = {}
+    if shape.I_sh:
+        sh = dict(w13_sh=wh["w13_sh"], w2_sh=wh["w2_sh"])
+    ref = oracle.moe_layer(xh, None, wh["w13"], wh["w2"], shape.K, shape.score_fn, shape.renorm, logits=lg,
+                           tokens=tok, k=k, **sh)
+    return rel_err(out.float().cpu().numpy()[tok], ref)

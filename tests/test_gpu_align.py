@@ -57,6 +57,35 @@ def test_align_max_value_bit_exact(T, E, K, B, kind):
     _check_align(T, E, K, B, _ids(T, E, K, seed=T + E + B + 1, kind=kind), mode=1)
 
 
+def test_align_max_value_repeated_ids_are_flagged_and_stay_in_bounds():
+    # ids repeating within a token (no top-K produces them) would need
+    # E * ceil(80 / 16) * 16 = 1280 max-value rows against P_max = 768: the
+    # alignment flags bit 2 of scalars[2], aligns nothing and writes nothing at
+    # or past P_max (guard words after every buffer stay untouched)
+    T, K, E, B = 40, 4, 16, 16
+    ids_np = np.zeros((T, K), np.int32)
+    ids_np[:, 2], ids_np[:, 3] = 5, 7
+    cfg = moe.config(T, 64, E, K, 64, tile_B=B, pad_mode=1)
+    Pm = moe.padded_rows_max(cfg)
+    assert Pm == 768
+    nblk, guard = Pm // B, 4096
+    buf = lambda n: torch.full((n + guard,), -7, dtype=torch.int32, device="cuda")
+    out = dict(counts=buf(E), offsets=buf(E + 1), sorted_ids=buf(Pm), block_expert=buf(nblk), pos=buf(T * K),
+               scalars=torch.zeros(4, dtype=torch.int32, device="cuda"))
+    g = moe.align_pad(cfg, torch.from_numpy(ids_np).cuda(), out)
+    torch.cuda.synchronize()
+    sc = g["scalars"].cpu().numpy()
+    assert sc[0] == 0 and sc[1] == 0 and (sc[2] & 2)
+    assert np.array_equal(out["counts"][:E].cpu().numpy(), np.bincount(ids_np.ravel(), minlength=E))
+    assert np.all(out["offsets"][:E + 1].cpu().numpy() == 0)
+    assert np.all(g["pos"].cpu().numpy() == -1)
+    assert np.all(g["sorted_ids"].cpu().numpy() == -1)
+    assert np.all(g["block_expert"].cpu().numpy() == -1)
+    n = {"counts": E, "offsets": E + 1, "sorted_ids": Pm, "block_expert": nblk, "pos": T * K}
+    for key, length in n.items():
+        assert np.all(out[key][length:].cpu().numpy() == -7), key
+
+
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("T,E,K,B", [(64, 8, 2, 16), (300, 64, 8, 16), (1000, 256, 8, 16), (40, 16, 4, 4)])
 def test_align_dynamic_k_empty_slots(mode, T, E, K, B):

@@ -1,8 +1,8 @@
 """FP8 expert weights on the GPU against the oracle: the row quantiser's
 codes and scales bit-exact, and the layer with FP8 routed and shared weights
-(the fused decode FFN widening E4M3 tiles to bf16 in shared memory) within
-the output bound of the bf16 layer, against the oracle's layer computed on
-the same codes and scales."""
+(the fused decode FFN widening E4M3 codes to f16 in tensor memory, f16 MMAs)
+within the output bound of the bf16 layer, against the oracle's layer
+computed on the same codes and scales."""
 import numpy as np
 import pytest
 import torch
@@ -82,10 +82,13 @@ def test_fp8_layer_ragged_and_dynamic_k():
     assert _run_fp8_layer(shape, 28, seed=3, k=k) < OUT_TOL
 
 
-@pytest.mark.parametrize("name,T", [("mixtral", 32), ("qwen2moe", 32), ("deepseekv3", 32)])
+@pytest.mark.parametrize("name,T", [("mixtral", 32), ("qwen2moe", 32), ("deepseekv3", 32), ("mixtral", 256),
+                                    ("qwen2moe", 128), ("deepseekv3", 128)])
 def test_fp8_layer_full_size_sampled(name, T):
+    # every token up to 256 (the FP8 path runs decode sizes: at most 128 rows
+    # per routed expert, and T <= 128 with shared experts)
     shape = mi.SHAPES[name]
-    assert _run_fp8_layer(shape, T, seed=mi.seed_for(shape, T, 3), n_sample=32) < OUT_TOL
+    assert _run_fp8_layer(shape, T, seed=mi.seed_for(shape, T, 3), n_sample=256) < OUT_TOL
 
 
 def test_fp8_layer_rejects_prefill_sizes():

@@ -2,54 +2,25 @@
 (router -> top-K -> gate weights -> SwiGLU experts -> weighted sum + shared).
 The oracle routes on the logits the layer itself computed (read back from the
 workspace), so that a near-tie flipped by fp32 rounding of x.W_r cannot
-diverge the two; those logits are checked against the oracle's here.  Small shapes are checked on every token; the
-full Mixtral-, Qwen2-MoE- and DeepSeek-V3-shaped layers on a seeded sample of
-256 tokens (the layer is token-wise independent given the logits), in the
-launch configuration the benchmark times."""
-import os
-
+diverge the two; those logits are checked against the oracle's here.  Small
+shapes are checked on every token; the full-size layers of every benchmarked
+configuration are in test_gpu_fullsize.py."""
 import numpy as np
 import pytest
 import torch
 
 import moe_inputs as mi
 import mixture_experts_layer_61_b200 as moe
-import oracle
-from helpers import OUT_TOL, cfg_for, host, rel_err, sample_tokens, small_shape
+from helpers import OUT_TOL, cfg_for, layer_case, small_shape
 
 pytestmark = pytest.mark.gpu
-
-N_SAMPLE = int(os.environ.get("MOE_TEST_SAMPLE", "256"))
 
 
 def _run_layer(shape, T, seed, override=None, n_sample=None, check_stats=True, pad_mode=0, k=None):
     w = mi.make_weights(shape, seed, device="cuda")
     x = mi.make_x(shape, T, seed, device="cuda")
-    cfg = cfg_for(shape, T, pad_mode=pad_mode)
-    ws = moe.alloc_workspace(moe.workspace_size(cfg))
-    stats = torch.zeros(4, dtype=torch.int32, device="cuda")
-    kt = None if k is None else torch.from_numpy(np.asarray(k, np.int32)).cuda()
-    out = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w.get("w13_sh"), w.get("w2_sh"),
-                            logits_override=override, stats=stats, k=kt)
-    moe.check_status(ws)
-    # the logits the layer computed (checked against the oracle's below)
-    layer_lg = moe.layer_logits(cfg, ws).cpu().numpy()
-    ref_lg = oracle.router_logits(host(x)[:min(T, 64)], host(w["w_r"]))
-    tol = 4e-3 if shape.dtype == "fp32" and T > 64 else 1e-5
-    assert np.abs(layer_lg[:min(T, 64)] - ref_lg).max() / np.abs(ref_lg).max() < tol
-    lg = layer_lg if override is None else override.cpu().numpy()
-    ids = oracle.topk(lg, shape.K, k)
-    if check_stats:
-        r = oracle.align(ids, shape.E, shape.tile_B, mode=pad_mode)
-        st = stats.cpu().numpy()
-        assert st[0] == r["P"] and st[1] == r["E_active"] and st[2] == 0
-    tok = sample_tokens(T, n_sample or T, seed)
-    sh = {}
-    if shape.I_sh:
-        sh = dict(w13_sh=host(w["w13_sh"]), w2_sh=host(w["w2_sh"]))
-    ref = oracle.moe_layer(host(x), None, host(w["w13"]), host(w["w2"]), shape.K, shape.score_fn,
-                           shape.renorm, logits=lg, tokens=tok, k=k, **sh)
-    return rel_err(out.float().cpu().numpy()[tok], ref)
+    return layer_case(shape, T, w, x, override=override, n_sample=n_sample, sample_seed=seed,
+                      check_stats=check_stats, pad_mode=pad_mode, k=k)
 
 
 def test_layer_tiny_fp32_all_tokens():
@@ -78,21 +49,6 @@ def test_layer_skewed_logits_override():
     shape = small_shape(H=1024, E=64, K=8, I=256, I_sh=512, score_fn=1)
     lg = mi.zipf_gumbel_logits(64, 200, 1.5, seed=3, device="cuda")
     assert _run_layer(shape, 200, seed=3, override=lg) < OUT_TOL
-
-
-@pytest.mark.parametrize("name,T", [("mixtral", 1), ("mixtral", 32), ("mixtral", 2048), ("qwen2moe", 128),
-                                    ("qwen2moe", 1024), ("deepseekv3", 32), ("deepseekv3", 1024)])
-def test_layer_full_size_sampled(name, T):
-    shape = mi.SHAPES[name]
-    assert _run_layer(shape, T, seed=mi.seed_for(shape, T), n_sample=N_SAMPLE) < OUT_TOL
-
-
-@pytest.mark.parametrize("s", [0.0, 1.5])
-def test_layer_deepseek_skew_sweep_point(s):
-    shape = mi.SHAPES["deepseekv3"]
-    T = 256
-    lg = mi.zipf_gumbel_logits(shape.E, T, s, seed=4000 + T, device="cuda")
-    assert _run_layer(shape, T, seed=mi.seed_for(shape, T, 5), override=lg, n_sample=64) < OUT_TOL
 
 
 @pytest.mark.parametrize("T", [5, 100, 700])

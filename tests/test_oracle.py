@@ -274,6 +274,20 @@ def test_align_rejects_bad_ids():
         oracle.align(np.array([[0, 5]], np.int32), 4, 4)
 
 
+def test_align_max_value_rejects_rows_past_the_bound():
+    # max-value padding's bound E * ceil(min(T, A) / B) * B holds when an
+    # expert has at most one assignment per token (every top-K routing); ids
+    # that repeat within a token can need more rows, and the oracle rejects
+    # them.  Block-wise padding stays within A + min(E, A) (B - 1) for any ids.
+    T, K, E, B = 4, 2, 4, 4
+    ids = np.zeros((T, K), np.int32)         # expert 0 twice per token: N_0 = 8 > T
+    assert oracle.p_max(T, K, E, B, 1) == 16
+    with pytest.raises(ValueError):
+        oracle.align(ids, E, B, mode=1)      # would need E * 8 = 32 rows
+    r = oracle.align(ids, E, B)
+    assert r["P"] == 8 and r["P"] <= oracle.p_max(T, K, E, B, 0)
+
+
 # ----------------------------------------------------- permute / combine
 
 def test_permute_then_combine_with_unit_weights_is_identity():
