@@ -472,6 +472,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch each step from the host instead of a CUDA graph")
     ap.add_argument("--token-tile-cap", type=int, default=0, help="grouped GEMM token-tile cap (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true", help="plain stream order between kernels")
+    ap.add_argument("--split-tail", type=int, default=-1, choices=[-1, 0, 1],
+                    help="GEMM tail schedule: 0 contiguous stream-K, 1 aligned k-slices (-1 = library default)")
     ap.add_argument("--pad-mode", type=int, default=0, choices=[0, 1],
                     help="alignment padding: 0 block-wise, 1 max-value")
     ap.add_argument("--fp8", action="store_true",
@@ -512,6 +514,8 @@ def main():
         moe.set_token_tile_cap(args.token_tile_cap)
     if args.no_pdl:
         moe.set_programmatic_launch(False)
+    if args.split_tail >= 0:
+        moe.set_split_tail(args.split_tail)
     if args.shared_sms:
         moe.set_shared_sms(args.shared_sms)
     flush = l2_flush_buffer(device)
@@ -592,7 +596,7 @@ def main():
                                                         "pdl": not args.no_pdl,
                                                         "shared_sms": moe.shared_sms(wl.cfg),
                                                         "pad_mode": args.pad_mode, "dynamic_k": args.dynamic_k,
-                                                        "fp8": args.fp8},
+                                                        "fp8": args.fp8, "split_tail": args.split_tail},
                               "stages_ms": stages, "E_active": E_active, "P": P}), flush=True)
         if dist:
             dist.barrier()

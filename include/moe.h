@@ -341,10 +341,10 @@ int moe_set_token_tile_cap(int n);
 
 /* Tuning: how the grouped GEMM shares out the tiles left after its whole
  * waves of one tile per SM (or SM pair), for subsequent launches.
- *   1: every whole wave data-parallel; the tiles of the last
+ *   1 (default): every whole wave data-parallel; the tiles of the last
  *     partial wave cut into equal k-slices, taken slice-major, so that tiles
  *     sharing a weight block or a token chunk stream the same slice together;
- *   0 (default): stream-K over the last one to two waves, in contiguous ranges of
+ *   0: stream-K over the last one to two waves, in contiguous ranges of
  *     (tile, k-iteration) units.
  * Split tiles are summed in a fixed order by the last contributor; results
  * agree up to fp32 summation order.  Process-wide.  MOE_ERR_ARG for other

@@ -358,8 +358,8 @@ def set_token_tile_cap(n):
 
 
 def set_split_tail(mode=1):
-    """GEMM tail schedule: 1 aligned k-slices of the last partial wave, 0
-    contiguous stream-K over the last one to two waves (the library default)."""
+    """GEMM tail schedule: 1 aligned k-slices of the last partial wave (the
+    library default), 0 contiguous stream-K over the last one to two waves."""
     _check(lib().moe_set_split_tail(int(mode)), "moe_set_split_tail")
 
 

@@ -270,7 +270,7 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
 
 namespace {
 int g_token_tile_cap = 0;  // 0: automatic
-int g_split_tail = 0;      // contiguous stream-K over the last one to two waves
+int g_split_tail = 1;      // aligned k-slices for the last partial wave
 }
 
 void set_token_tile_cap(int n) { g_token_tile_cap = n; }

@@ -199,3 +199,35 @@ def test_dense_ffn_wide_pair_tiles():
     tok = sample_tokens(T, 24, seed=7)
     ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
     assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
+
+
+@pytest.fixture
+def split_tail_mode(request):
+    moe.set_split_tail(request.param)
+    yield request.param
+    moe.set_split_tail(1)
+
+
+# the tiles after the whole waves: contiguous stream-K (0) or aligned k-slices
+# taken slice-major (1).  (1200 tokens, 8 experts): 64 gate/up pair tiles, all
+# of them a tail of 2 slices, and 16 down tiles of 4 slices; (2048, I = 8192):
+# 3 whole waves of 74 pairs and a 34-tile tail; (300, ragged 264 / 640): the
+# single-CTA 128-token tiles.
+@pytest.mark.parametrize("split_tail_mode", [0, 1], indirect=True)
+@pytest.mark.parametrize("T", [1200, 400])
+def test_grouped_split_tail_modes(split_tail_mode, T):
+    shape = small_shape(H=512, E=8, K=2, I=1024)
+    assert _grouped(shape, T, seed=T + 3, n_check=128) < OUT_TOL
+
+
+@pytest.mark.parametrize("split_tail_mode", [0, 1], indirect=True)
+@pytest.mark.parametrize("T,H,I", [(2048, 1024, 8192), (700, 512, 14336), (300, 264, 640)])
+def test_dense_ffn_split_tail_modes(split_tail_mode, T, H, I):
+    w13, w2 = mi.make_dense_weights(H, I, torch.bfloat16, seed=T + I + 1, device="cuda")
+    x = mi.make_x(small_shape(H, 1, 1, I), T, T, device="cuda")
+    ws = moe.alloc_workspace(moe.dense_workspace_size(T, H, I))
+    out = moe.dense_ffn(x, w13, w2, ws)
+    moe.check_status(ws)
+    tok = sample_tokens(T, 64, seed=T)
+    ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
+    assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
