@@ -487,6 +487,9 @@ def main():
     ap.add_argument("--tp", action="store_true",
                     help="tensor parallelism over I across the ranks: every rank holds I/N of every expert and "
                          "runs the same tokens; one NCCL all-reduce of the fp32 partial output per layer")
+    ap.add_argument("--tp-chunks", type=int, default=0,
+                    help="with --tp: overlap the all-reduce with the down projection in this many blocks of output "
+                         "features (0 = one all-reduce after the whole partial layer)")
     ap.add_argument("--shared-sms", type=int, default=0,
                     help="SMs for the shared experts beside the routed ones (0 = cost model, -1 = serial)")
     args = ap.parse_args()
@@ -811,8 +814,16 @@ def run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind)
     partial = torch.empty((T, shape.H), dtype=torch.float32, device=device)
     out = torch.empty((T, shape.H), dtype=x.dtype, device=device)
 
+    overlap = args.tp_chunks > 0 and not moe.ffn_fused(cl)
+    n_chunks = args.tp_chunks if overlap else 0
+    parts = [torch.empty((T, shape.H // n_chunks), dtype=torch.float32, device=device)
+             for _ in range(n_chunks)]
+
     def layer():
-        moe.layer_forward_partial(cl, x, w_r, w13, w2, ws, sh[0], sh[1], out=partial, stats=stats)
+        if overlap:   # routing, permute, gate/up and the shared FFN; the down blocks follow per step
+            moe.layer_forward_partial_front(cl, x, w_r, w13, ws, sh[0], sh[1], stats=stats)
+        else:
+            moe.layer_forward_partial(cl, x, w_r, w13, w2, ws, sh[0], sh[1], out=partial, stats=stats)
 
     layer()
     torch.cuda.synchronize()
@@ -820,13 +831,20 @@ def run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         layer()
-    per_graph = moe.kernel_launch_count() - n0
+    per_graph = moe.kernel_launch_count() - n0 + (2 * n_chunks + 1 if overlap else 1)
     torch.cuda.synchronize()
 
     def step():
         graph.replay()
-        moe.tp_allreduce(partial)             # NCCL all-reduce (no-op on one rank)
-        moe.tp_reduce([partial], out)
+        if overlap:
+            # each block's down projection + combine, its all-reduce started
+            # beside the next block's kernels; then the blocks side by side, rounded
+            moe.tp_overlapped_allreduce(
+                parts, lambda c: moe.layer_forward_partial_down(cl, w2, c, n_chunks, ws, parts[c]))
+            moe.tp_gather(parts, out)
+        else:
+            moe.tp_allreduce(partial)             # NCCL all-reduce (no-op on one rank)
+            moe.tp_reduce([partial], out)
 
     for _ in range(args.warmup):
         step()
@@ -886,15 +904,19 @@ def run_tp(args, shape, T, rank, world, local, dist, device, flush, pk, pk_kind)
         "config": {"workload": f"{shape.name}-shaped MoE layer forward, T={T}", "T": T, "H": shape.H,
                    "E": shape.E, "K": shape.K, "I": shape.I, "I_per_rank": cl.I, "I_shared": shape.I_sh,
                    "tile_B": shape.tile_B, "global_batch": T,
-                   "parallelism": f"TP over I x{world} (one all-reduce of the fp32 partial output per layer)",
-                   "launch": "CUDA graph of the partial layer, then the all-reduce and the rounding kernel",
+                   "parallelism": (f"TP over I x{world} (all-reduce of the fp32 partial output in {n_chunks} blocks "
+                                   "of output features, each beside the next block's down projection)" if overlap else
+                                   f"TP over I x{world} (one all-reduce of the fp32 partial output per layer)"),
+                   "launch": ("CUDA graph of the front part (routing, gate/up, shared FFN), then per block the down "
+                              "projection + combine and an async all-reduce, then the gather kernel" if overlap else
+                              "CUDA graph of the partial layer, then the all-reduce and the rounding kernel"),
                    "l2": "flushed between steps (2 GiB write outside the events)"},
         "roofline": roof,
         "layer": {"P": P, "E_active": E_active, "bytes_alg_per_rank": B_rank, "flops_alg_per_rank": F_rank},
         "e2e": {"value": tp_tokens_per_s(T, args.steps, e2e_total), "unit": "tokens/s",
                 "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
-        "gpu_launches": (per_graph + 1) * args.steps,
+        "gpu_launches": per_graph * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": None,
     }

@@ -370,6 +370,15 @@ void moe_set_programmatic_launch(int enable);
  * results are identical up to fp32 summation order. */
 void moe_set_cta_pairs(int enable);
 
+/* FP8 expert weights on CTA pairs (default off): the fused decode FFN of
+ * moe_layer_forward_fp8 / moe_grouped_ffn_fp8 / dense_ffn_fp8 runs on pairs of
+ * SMs (thread-block clusters of 2), each CTA widening its own 128 weight rows
+ * into its own tensor memory and one 2-SM MMA covering both (M = 256): half
+ * the MMA instructions per weight byte.  Needs H and I multiples of 64; token
+ * tiles are then multiples of 32 rows.  0 keeps one CTA per tile.
+ * Process-wide; results agree up to fp32 summation order. */
+void moe_set_fp8_pairs(int enable);
+
 /* Shared experts beside the routed experts.  With n_shared > 0,
  * moe_layer_forward launches the shared FFN first, on a second stream that
  * the library owns (one per device, created on first use), forked from and
@@ -413,6 +422,41 @@ int moe_layer_forward_partial(const moe_config_t* cfg, const void* x, const void
                               const void* w2_shared, const float* logits_override,
                               const int32_t* k_per_token, float* out_partial, void* workspace,
                               size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
+
+/* TP over I with the all-reduce overlapped with the down projection (talk
+ * notes, "Key findings" 3: the AllReduce that follows the MoE block).  The
+ * layer on this rank's slice (cfg as for moe_layer_forward_partial) in two
+ * parts, so that the all-reduce of one block of output features can run
+ * while the down projection of the next block computes:
+ *   moe_layer_forward_partial_front: routing, permute, the routed experts'
+ *     gate/up + SwiGLU and the whole shared FFN, all into the workspace (the
+ *     shared experts' side stream is joined back before it returns);
+ *   moe_layer_forward_partial_down: for output features
+ *     [chunk * H/n_chunks, (chunk + 1) * H/n_chunks): the routed experts' down
+ *     projection and the combine (fp32 sums in ascending k, the shared output
+ *     added last, unrounded) into part [T, H/n_chunks] fp32, contiguous and
+ *     ready for that block's all-reduce.
+ * Call front once, then down for every chunk, on the same stream and
+ * workspace (front's results stay there until the next front call).  The sum
+ * over ranks of the parts, placed side by side, is the layer output (see
+ * moe_tp_gather).  Needs the two-launch expert FFN (moe_ffn_fused(cfg) == 0:
+ * more than 128 rows per expert); H/n_chunks a multiple of 8 (bf16) or 4
+ * (fp32).  MOE_ERR_ARG otherwise.  Same workspace size as moe_layer_forward. */
+int moe_layer_forward_partial_front(const moe_config_t* cfg, const void* x, const void* w_router,
+                                    const void* w13, const void* w13_shared, const void* w2_shared,
+                                    const float* logits_override, const int32_t* k_per_token,
+                                    void* workspace, size_t ws_bytes, int32_t* stats_out,
+                                    moe_stream_t stream);
+int moe_layer_forward_partial_down(const moe_config_t* cfg, const void* w2, int chunk, int n_chunks,
+                                   float* part, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* The layer output from the all-reduced column blocks of
+ * moe_layer_forward_partial_down: out[t][c * Hc + j] = parts[c][t * Hc + j]
+ * rounded once to dtype (0 bf16, 1 fp32), Hc = H / n_chunks.  `parts` is a
+ * HOST array of n_chunks (1..16) device pointers to [T, Hc] fp32 blocks,
+ * 16-byte aligned; Hc % 4 == 0. */
+int moe_tp_gather(int n_chunks, const float* const* parts, int T, int H, int dtype, void* out,
+                  moe_stream_t stream);
 
 /* The reduction of the ranks' partial outputs: out[i] = sum over r of
  * parts[r][i] for i < count, fp32 in rank order, one rounding to dtype (0

@@ -91,6 +91,7 @@ def lib():
             "moe_set_programmatic_launch": (None, [I]),
             "moe_set_split_tail": (I, [I]),
             "moe_set_cta_pairs": (None, [I]),
+            "moe_set_fp8_pairs": (None, [I]),
             "moe_set_shared_sms": (I, [I]),
             "moe_shared_sms": (I, [C]),
             "moe_ffn_fused": (I, [C]),
@@ -99,6 +100,9 @@ def lib():
             "moe_tp_shard": (I, [I, I, I, I, I, I, P, P, P, P, P]),
             "moe_layer_forward_partial": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P, P]),
             "moe_tp_reduce": (I, [I, ctypes.POINTER(ctypes.c_void_p), ctypes.c_longlong, I, P, P]),
+            "moe_layer_forward_partial_front": (I, [C, P, P, P, P, P, P, P, P, S, P, P]),
+            "moe_layer_forward_partial_down": (I, [C, P, I, I, P, P, S, P]),
+            "moe_tp_gather": (I, [I, ctypes.POINTER(ctypes.c_void_p), I, I, I, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -387,6 +391,11 @@ def set_cta_pairs(enable=True):
     lib().moe_set_cta_pairs(1 if enable else 0)
 
 
+def set_fp8_pairs(enable=True):
+    """FP8 decode weights on CTA pairs (2-SM MMAs; off by default)."""
+    lib().moe_set_fp8_pairs(1 if enable else 0)
+
+
 def set_shared_sms(n=0):
     """SMs for the shared experts running beside the routed ones: 0 = cost
     model (default), n > 0 = fixed share, -1 = run them after, serially."""
@@ -490,6 +499,85 @@ def tp_allreduce(partial, group=None):
     if dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(partial, op=dist.ReduceOp.SUM, group=group)
     return partial
+
+
+def layer_forward_partial_front(cfg, x, w_r, w13, ws, w13_sh=None, w2_sh=None, logits_override=None, stats=None,
+                                k=None):
+    """This rank's layer up to the routed gate/up and the shared FFN (results
+    in `ws`), for the down projection by output-feature blocks."""
+    _need_cuda(x, w_r, w13, ws, w13_sh, w2_sh, logits_override, stats, k)
+    _check(lib().moe_layer_forward_partial_front(ctypes.byref(cfg), _p(x), _p(w_r), _p(w13), _p(w13_sh), _p(w2_sh),
+                                                 _p(logits_override), _p(k), _p(ws), ws.numel(), _p(stats),
+                                                 _stream()),
+           "moe_layer_forward_partial_front")
+
+
+def layer_forward_partial_down(cfg, w2, chunk, n_chunks, ws, part=None):
+    """Down projection + combine of output features block `chunk` of
+    n_chunks into part [T, H/n_chunks] fp32 (unrounded)."""
+    _need_cuda(w2, ws, part)
+    if part is None:
+        part = torch.empty((cfg.T, cfg.H // n_chunks), dtype=torch.float32, device=w2.device)
+    _check(lib().moe_layer_forward_partial_down(ctypes.byref(cfg), _p(w2), int(chunk), int(n_chunks), _p(part),
+                                                _p(ws), ws.numel(), _stream()), "moe_layer_forward_partial_down")
+    return part
+
+
+def tp_gather(parts, out):
+    """out [T, H] = the column blocks `parts` ([T, H/n] fp32 each) side by side,
+    rounded once to out's dtype."""
+    _need_cuda(out, *parts)
+    T, H = out.shape
+    ptrs = (ctypes.c_void_p * len(parts))(*[p_.data_ptr() for p_ in parts])
+    dt = BF16 if out.dtype == torch.bfloat16 else FP32
+    _check(lib().moe_tp_gather(len(parts), ptrs, T, H, dt, _p(out), _stream()), "moe_tp_gather")
+    return out
+
+
+def tp_allreduce_async(partial, group=None):
+    """Starts the sum of `partial` across `group` (in place) and returns the
+    pending work, or None when there is nothing to sum (one rank)."""
+    import torch.distributed as dist
+
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        return dist.all_reduce(partial, op=dist.ReduceOp.SUM, group=group, async_op=True)
+    return None
+
+
+def tp_overlapped_allreduce(parts, produce, group=None):
+    """The overlap protocol of TP over I: for each output-feature block c in
+    order, produce(c) enqueues the block's partial into parts[c], then its
+    all-reduce starts (asynchronously, beside the next block's work); all of
+    them are waited for before returning."""
+    works = []
+    for c in range(len(parts)):
+        produce(c)
+        works.append(tp_allreduce_async(parts[c], group))
+    for w_ in works:
+        if w_ is not None:
+            w_.wait()
+    return parts
+
+
+def tp_layer_forward_overlapped(cfg_local, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, n_chunks=4,
+                                logits_override=None, parts=None, out=None, group=None, k=None):
+    """One layer under TP over I with the all-reduce overlapped with the down
+    projection: the front part, then per block of H/n_chunks output features
+    the down projection + combine into its fp32 part and that part's
+    all-reduce, then the concatenation and rounding.  At decode sizes (the
+    fused expert FFN) it is tp_layer_forward."""
+    if ffn_fused(cfg_local):
+        return tp_layer_forward(cfg_local, x, w_r, w13, w2, ws, w13_sh, w2_sh, logits_override, out=out,
+                                group=group, k=k)
+    if parts is None:
+        parts = [torch.empty((cfg_local.T, cfg_local.H // n_chunks), dtype=torch.float32, device=x.device)
+                 for _ in range(n_chunks)]
+    if out is None:
+        out = torch.empty((cfg_local.T, cfg_local.H), dtype=x.dtype, device=x.device)
+    layer_forward_partial_front(cfg_local, x, w_r, w13, ws, w13_sh, w2_sh, logits_override, k=k)
+    tp_overlapped_allreduce(parts, lambda c: layer_forward_partial_down(cfg_local, w2, c, len(parts), ws, parts[c]),
+                            group)
+    return tp_gather(parts, out)
 
 
 def tp_layer_forward(cfg_local, x, w_r, w13, w2, ws, w13_sh=None, w2_sh=None, logits_override=None,

@@ -533,11 +533,14 @@ struct Fp8Scales {
 };
 }  // namespace
 
+// stage 0: the whole layer; stage 1 (TP over I, overlapped all-reduce): up to
+// the routed experts' gate/up and the whole shared FFN, no down projection and
+// no combine (those run per output-feature block in moe_layer_forward_partial_down)
 static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
                               const void* w2, const void* w13_shared, const void* w2_shared,
                               const Fp8Scales* fp8, const float* logits_override, const int32_t* k_per_token,
                               void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream,
-                              bool out_f32 = false);
+                              bool out_f32 = false, int stage = 0);
 
 int moe_layer_forward_k(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
                         const void* w2, const void* w13_shared, const void* w2_shared, const float* logits_override,
@@ -572,15 +575,18 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
                               const void* w2, const void* w13_shared, const void* w2_shared,
                               const Fp8Scales* fp8, const float* logits_override, const int32_t* k_per_token,
                               void* out, void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream,
-                              bool out_f32) {
+                              bool out_f32, int stage) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->T == 0) return MOE_OK;
     const long long I_sh = (long long)cfg->n_shared * cfg->I_shared;
-    if (!x || !w_router || !w13 || !w2 || !out || !workspace) return MOE_ERR_ARG;
+    const bool front = stage == 1;
+    if (front && (fp8 || routed_max_n(cfg) <= 128)) return MOE_ERR_ARG;  // the two-launch expert FFN only
+    if (!x || !w_router || !w13 || (!w2 && !front) || (!out && !front) || !workspace) return MOE_ERR_ARG;
     if (I_sh > 0 && (!w13_shared || !w2_shared)) return MOE_ERR_ARG;
-    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) ||
-        !aligned16(workspace) || (I_sh > 0 && (!aligned16(w13_shared) || !aligned16(w2_shared))))
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || (!front && !aligned16(w2)) ||
+        (!front && !aligned16(out)) || !aligned16(workspace) ||
+        (I_sh > 0 && (!aligned16(w13_shared) || !aligned16(w2_shared))))
         return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
@@ -673,29 +679,54 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
                                      logits, ids, w, counts, offsets, sorted_ids, block_expert, pos, scalars,
                                      stats_out, route_ctr, s)) != 0)
             return status_of(rc);
+    } else if (router_cc_fits(cfg->H, cfg->E, cfg->dtype)) {
+        // a small router matrix (E * H fits shared memory): router logits on the
+        // CUDA cores, top-K and alignment in the same launch
+        RouteCcArgs a{};
+        a.T = cfg->T;
+        a.H = cfg->H;
+        a.E = cfg->E;
+        a.K = cfg->K;
+        a.score_fn = cfg->score_fn;
+        a.renorm = cfg->renorm;
+        a.B = cfg->tile_B;
+        a.mode = cfg->pad_mode;
+        a.dtype = cfg->dtype;
+        a.P_max = P;
+        a.x = x;
+        a.w_r = w_router;
+        a.logits_override = logits_override;
+        a.k_per_token = k_per_token;
+        a.logits = logits;
+        a.ids = ids;
+        a.w = w;
+        a.counts = counts;
+        a.offsets = offsets;
+        a.sorted_ids = sorted_ids;
+        a.block_expert = block_expert;
+        a.pos = pos;
+        a.scalars = scalars;
+        a.stats_copy = stats_out;
+        a.done_ctr = reinterpret_cast<int*>(at<uint8_t>(workspace, L.ctl)) + 16;  // in the control header
+        if ((rc = launch_route_cc(a, s)) != 0) return status_of(rc);
     } else {
-        if (router_cc_fits(cfg->H, cfg->E, cfg->dtype)) {
-            // a small router matrix (E * H fits shared memory): CUDA cores, one read of x
-            if ((rc = launch_router_cc(cfg->T, cfg->H, cfg->E, cfg->dtype, x, w_router, logits, s)) != 0)
-                return status_of(rc);
-        } else {
-            GemmLaunch g{};
-            g.x = x;
-            g.x_rows = cfg->T;
-            g.w = w_router;
-            g.w_rows = cfg->E;
-            g.kdim = cfg->H;
-            g.n_out = cfg->E;
-            g.n_groups = 1;
-            g.seg_rows = cfg->T;
-            g.out_f32 = true;
-            g.out = logits;
-            g.out_ld = cfg->E;
-            g.dtype = cfg->dtype;
-            router_tiling(g, cfg->T);
-            g.sms = n_routed;
-            if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
-        }
+        // the tensor-core router GEMM, then top-K and the alignment
+        GemmLaunch g{};
+        g.x = x;
+        g.x_rows = cfg->T;
+        g.w = w_router;
+        g.w_rows = cfg->E;
+        g.kdim = cfg->H;
+        g.n_out = cfg->E;
+        g.n_groups = 1;
+        g.seg_rows = cfg->T;
+        g.out_f32 = true;
+        g.out = logits;
+        g.out_ld = cfg->E;
+        g.dtype = cfg->dtype;
+        router_tiling(g, cfg->T);
+        g.sms = n_routed;
+        if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
         if ((rc = launch_topk(cfg->T, cfg->E, cfg->K, cfg->score_fn, cfg->renorm,
                               logits_override ? logits_override : logits, k_per_token, ids, w, s)) != 0)
             return status_of(rc);
@@ -706,10 +737,16 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
     }
     if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s, fp8 != nullptr)) != 0)
         return status_of(rc);
-    if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
-                      routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn,
-                      fp8 ? fp8->s13 : nullptr, fp8 ? fp8->s2 : nullptr)) != 0)
+    if (front) {
+        GemmLaunch g = gate_up_launch(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, act,
+                                      routed_max_n(cfg));
+        g.sms = n_routed;
+        if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
+    } else if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
+                             routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn,
+                             fp8 ? fp8->s13 : nullptr, fp8 ? fp8->s2 : nullptr)) != 0) {
         return status_of(rc);
+    }
     if (I_sh > 0 && !side) {
         void* sh_out = at<void>(workspace, L.sh_out);
         const void* x_sh = x;
@@ -732,6 +769,7 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
             return MOE_ERR_CUDA;
         }
     }
+    if (front) return MOE_OK;  // act, the routing and the shared output wait in the workspace
     return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, pos, w, sh, out, s, out_f32));
 }
 
@@ -745,6 +783,57 @@ int moe_layer_forward_partial(const moe_config_t* cfg, const void* x, const void
                               void* workspace, size_t ws_bytes, int32_t* stats_out, moe_stream_t stream) {
     return layer_forward_impl(cfg, x, w_router, w13, w2, w13_shared, w2_shared, nullptr, logits_override,
                               k_per_token, out_partial, workspace, ws_bytes, stats_out, stream, true);
+}
+
+int moe_layer_forward_partial_front(const moe_config_t* cfg, const void* x, const void* w_router, const void* w13,
+                                    const void* w13_shared, const void* w2_shared, const float* logits_override,
+                                    const int32_t* k_per_token, void* workspace, size_t ws_bytes, int32_t* stats_out,
+                                    moe_stream_t stream) {
+    return layer_forward_impl(cfg, x, w_router, w13, nullptr, w13_shared, w2_shared, nullptr, logits_override,
+                              k_per_token, nullptr, workspace, ws_bytes, stats_out, stream, true, 1);
+}
+
+int moe_layer_forward_partial_down(const moe_config_t* cfg, const void* w2, int chunk, int n_chunks, float* part,
+                                   void* workspace, size_t ws_bytes, moe_stream_t stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (n_chunks < 1 || chunk < 0 || chunk >= n_chunks || cfg->H % n_chunks) return MOE_ERR_ARG;
+    const int eb = elt_bytes(cfg->dtype);
+    const int Hc = cfg->H / n_chunks, c0 = chunk * Hc;
+    if ((Hc * eb) % 16 || Hc % 4) return MOE_ERR_ARG;  // 16-byte vectors in, float4 out
+    if (routed_max_n(cfg) <= 128) return MOE_ERR_ARG;   // the two-launch expert FFN only
+    if (cfg->T == 0) return MOE_OK;
+    if (!w2 || !part || !workspace || !aligned16(w2) || !aligned16(part) || !aligned16(workspace)) return MOE_ERR_ARG;
+    DeviceInfo d;
+    if ((rc = current_device(&d)) != 0) return status_of(rc);
+    const Layout L = layout(cfg, d.num_sms);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const GemmCtl ctl = gemm_ctl(at<uint8_t>(workspace, L.ctl), d.num_sms);
+    const long long I_sh = (long long)cfg->n_shared * cfg->I_shared;
+    uint8_t* y_perm = at<uint8_t>(workspace, L.x_perm);
+    // output features [c0, c0 + Hc) of every expert: rows c0 .. of w2 [E, H, I]
+    // with the expert stride kept, into the same columns of y_perm
+    GemmLaunch g = down_launch(at<void>(workspace, L.act), p_max(cfg), at<int32_t>(workspace, L.offsets), cfg->E, 0,
+                               cfg->H, cfg->I, cfg->dtype, static_cast<const uint8_t*>(w2) + (size_t)c0 * cfg->I * eb,
+                               y_perm + (size_t)c0 * eb, routed_max_n(cfg));
+    g.n_out = Hc;
+    g.w_rows = (long long)cfg->E * cfg->H - c0;
+    if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
+    return status_of(launch_combine(cfg->T, cfg->H, cfg->K, cfg->dtype, y_perm, at<int32_t>(workspace, L.pos),
+                                    at<float>(workspace, L.w), I_sh > 0 ? at<void>(workspace, L.sh_out) : nullptr,
+                                    part, s, true, c0, Hc));
+}
+
+int moe_tp_gather(int n_chunks, const float* const* parts, int T, int H, int dtype, void* out, moe_stream_t stream) {
+    if (n_chunks < 1 || n_chunks > kTpMaxParts || T < 0 || H <= 0 || H % n_chunks || (H / n_chunks) % 4 || !parts)
+        return MOE_ERR_ARG;
+    if (dtype != 0 && dtype != 1) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (!out || !aligned16(out)) return MOE_ERR_ARG;
+    for (int c = 0; c < n_chunks; ++c)
+        if (!parts[c] || !aligned16(parts[c])) return MOE_ERR_ARG;
+    return status_of(launch_tp_gather(n_chunks, parts, T, H, dtype, out, (cudaStream_t)stream));
 }
 
 int moe_tp_reduce(int n_parts, const float* const* parts, long long count, int dtype, void* out,
@@ -927,6 +1016,8 @@ int moe_ffn_fused(const moe_config_t* cfg) {
 }
 
 void moe_set_cta_pairs(int enable) { set_cta_pairs(enable != 0); }
+
+void moe_set_fp8_pairs(int enable) { set_fp8_pairs(enable != 0); }
 
 void moe_debug_withhold_first_load(int enable) { g_withhold.store(enable ? 1 : 0); }
 

@@ -107,7 +107,7 @@ __device__ __forceinline__ int ffn_slices(long long tiles, int KI, int G, int ma
     long long s = (2LL * G + tiles - 1) / tiles;
     long long cap = (4LL * G < max_slots ? 4LL * G : max_slots) / tiles;
     if (s > cap) s = cap;
-    if (s > 8) s = 8;
+    if (s > 16) s = 16;
     if (s > KI / 4) s = KI / 4;
     return s < 1 ? 1 : (int)s;
 }
@@ -319,26 +319,63 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 Tile t;
                 item_of(id, it, t);
                 if (id == 0 && p.withhold_first_load) withhold = true;
-                if (it.phase == 1) {
-                    // the activations of this token chunk: all NFA gate/up tiles stored
-                    const uint64_t t0 = global_ns();
-                    while ((int)ld_acquire_u32(&chunk_done[t.chunk]) < NFA) {
-                        if (*abort_flag || global_ns() - t0 > limit) {
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    if (!ok) continue;  // next turn publishes the end marker
-                    fence_proxy_async_global();
-                }
                 const CUtensorMap* tw = it.phase == 0 ? &tm_w13 : &tm_w2;
                 const CUtensorMap* tx = it.phase == 0 ? &tm_xa : &tm_xb;
                 const CUtensorMap* tx64 = it.phase == 0 ? &tm_xa64 : &tm_xb64;
                 const int second = it.phase == 0 ? p.I : 128;  // up rows, or the next 128 features
                 const uint32_t bytes = 2 * C::kRawWBytes + t.mma_n * 128;
                 const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
-                for (int k = it.kb; k < it.ke; ++k, ++kc) {
+                auto load_w = [&](int s, int k) {
+                    uint8_t* st = stage_base + s * C::kStageBytes;
+                    const int kx = k * C::kBK;
+                    tma_load_2d(st, tw, &full[s], kx, t.wrow, pol_w);
+                    tma_load_2d(st + C::kRawWBytes, tw, &full[s], kx, t.wrow + second, pol_w);
+                };
+                auto load_x = [&](int s, int k) {
+                    uint8_t* xs = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes;
+                    const int kx = k * C::kBK;
+                    int r = 0;
+                    if (kMaxN >= C::kXBoxMid)
+                        for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
+                            tma_load_2d(xs + r * 128, tx64, &full[s], kx, t.row0 + r, pol_x);
+                    for (; r < t.mma_n; r += C::kXBoxRows) tma_load_2d(xs + r * 128, tx, &full[s], kx, t.row0 + r, pol_x);
+                };
+                int pre = 0;  // stages of this item whose weight tiles went out before the activation wait
+                if (it.phase == 1) {
+                    // The weights do not depend on phase A: stream the first stages'
+                    // weight tiles now, then wait until every gate/up tile of this
+                    // token chunk has stored its activations, then load those.
+                    const int want = it.ke - it.kb < C::kStages ? it.ke - it.kb : C::kStages;
+                    for (; pre < want; ++pre) {
+                        const int s = (kc + pre) % C::kStages;
+                        const uint32_t ph = ((kc + pre) / C::kStages) & 1u;
+                        if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        load_w(s, it.kb + pre);
+                        ++fills[s];
+                    }
+                    if (ok) {
+                        const uint64_t t0 = global_ns();
+                        while ((int)ld_acquire_u32(&chunk_done[t.chunk]) < NFA) {
+                            if (*abort_flag || global_ns() - t0 > limit) {
+                                ok = false;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                        if (ok) fence_proxy_async_global();
+                    }
+                    // the stages already expecting their activations get them even
+                    // when the wait gave up (in-bounds rows; the launch is reported
+                    // as timed out), so that every started stage completes
+                    for (int j = 0; j < pre; ++j) load_x((kc + j) % C::kStages, it.kb + j);
+                    kc += pre;
+                    if (!ok) continue;  // next turn publishes the end marker
+                }
+                for (int k = it.kb + pre; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
                     const uint32_t ph = (kc / C::kStages) & 1u;
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, abort_flag)) {
@@ -349,18 +386,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         withhold = false;
                         continue;
                     }
-                    uint8_t* st = stage_base + s * C::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], bytes);
-                    const int kx = k * C::kBK;
-                    tma_load_2d(st, tw, &full[s], kx, t.wrow, pol_w);
-                    tma_load_2d(st + C::kRawWBytes, tw, &full[s], kx, t.wrow + second, pol_w);
-                    uint8_t* xs = st + 2 * C::kRawWBytes;
-                    int r = 0;
-                    if (kMaxN >= C::kXBoxMid)
-                        for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
-                            tma_load_2d(xs + r * 128, tx64, &full[s], kx, t.row0 + r, pol_x);
-                    for (; r < t.mma_n; r += C::kXBoxRows)
-                        tma_load_2d(xs + r * 128, tx, &full[s], kx, t.row0 + r, pol_x);
+                    load_w(s, k);
+                    load_x(s, k);
                     ++fills[s];
                 }
                 if (!ok) continue;

@@ -135,12 +135,14 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
 int pick_max_n(double rows_per_group);
 void set_token_tile_cap(int n);
 // How the GEMM shares out the tiles after its whole data-parallel waves:
-// 0 contiguous stream-K over the last one to two waves (default), 1 aligned
-// k-slices of the last partial wave.
+// 0 contiguous stream-K over the last one to two waves, 1 aligned k-slices of
+// the last partial wave (default).
 void set_split_tail(int mode);
 int split_tail_mode();
 // CTA-pair (2-SM MMA) tiles for bf16 launches at the 256-token cap (default on).
 void set_cta_pairs(bool on);
+// The fused FFN with FP8 weights on CTA pairs (default off).
+void set_fp8_pairs(bool on);
 
 // Elementwise / routing kernels.
 // k_per_token (nullable): per-token expert count, clamped to [0, K]; slots
@@ -165,8 +167,13 @@ int launch_permute(int H, int K, int dtype, long long P_max, const void* x, cons
                    const int32_t* scalars, void* x_perm, cudaStream_t stream, bool to_f16 = false);
 // n bf16 values -> f16 (n a multiple of 8)
 int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stream);
+// col0 / ncols (elements, multiples of 16 bytes): only those columns, into
+// rows of ncols; ncols < 0: all H columns
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
-                   const void* shared_out, void* out, cudaStream_t stream, bool out_f32 = false);
+                   const void* shared_out, void* out, cudaStream_t stream, bool out_f32 = false, int col0 = 0,
+                   int ncols = -1);
+// out [T, H] from n column blocks parts[c] [T, H / n] (fp32), rounded to dtype
+int launch_tp_gather(int n, const float* const* parts, int T, int H, int dtype, void* out, cudaStream_t stream);
 constexpr int kTpMaxParts = 16;  // ranks of one TP reduction
 // router logits on the CUDA cores for small router matrices (E <= 16, E*H*elt
 // bytes <= kRouterCcMaxBytes, H % 8 == 0); -1 when the shape does not fit
@@ -175,6 +182,22 @@ bool router_cc_fits(int H, int E, int dtype);
 int launch_router_cc(int T, int H, int E, int dtype, const void* x, const void* w_r, float* logits,
                      cudaStream_t stream);
 int launch_tp_reduce(int n, const float* const* parts, long long count, int dtype, void* out, cudaStream_t stream);
+// Router logits (CUDA cores, router matrix in shared memory) + top-K + gate
+// weights + alignment in one launch, for router_cc_fits shapes at any T.
+struct RouteCcArgs {
+    int T, H, E, K, score_fn, renorm, B, mode, dtype;
+    long long P_max;
+    const void* x;
+    const void* w_r;
+    const float* logits_override;
+    const int32_t* k_per_token;
+    float* logits;
+    int32_t* ids;
+    float* w;
+    int32_t *counts, *offsets, *sorted_ids, *block_expert, *pos, *scalars, *stats_copy;
+    int* done_ctr;
+};
+int launch_route_cc(const RouteCcArgs& a, cudaStream_t stream);
 
 // Row-wise FP8 E4M3 quantisation: q [rows, cols] codes, scales [rows].
 int launch_quantize_fp8(long long rows, int cols, int dtype, const void* w, uint8_t* q, float* scales,

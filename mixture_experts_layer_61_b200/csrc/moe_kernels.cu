@@ -4,6 +4,7 @@
 // per token for top-K, one block for the alignment, 16-byte vector copies for
 // permute and combine.
 #include <climits>
+#include <type_traits>
 
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -147,13 +148,11 @@ int launch_topk(int T, int E, int K, int score_fn, int renorm, const float* logi
 }
 
 // -------------------------------------------------------------- alignment
-// One block of 1024 threads.  (1) shared-memory histogram of the expert ids;
-// (2) block scan of the padded counts ceil(N_e/B)*B into offsets;
-// (3) stable scatter in rounds of 1024 assignments: inside a warp the rank
-// among equal ids comes from __match_any_sync, across the 32 warps of a round
-// from a per-(warp, expert) count table scanned over the warps, across rounds
-// from a per-expert cursor -- so assignments keep ascending order within
-// each expert; (4) -1 in the padding slots, block_expert per B-row block.
+// One block of 1024 threads.  (1) the counts N_e (with the ranks of the fast
+// path below, or a shared-memory histogram); (2) block scan of the padded
+// counts ceil(N_e/B)*B into offsets; (3) stable scatter: every assignment's
+// slot keeps ascending a within its expert; (4) -1 in the padding slots,
+// block_expert per B-row block.
 constexpr int kAlignThreads = 1024;
 
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total) {
@@ -186,6 +185,19 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
 
 // The alignment of T*K assignments by one block of kAlignThreads threads;
 // `sm` is dynamic shared memory of align_smem_bytes(E) bytes.
+//
+// Fast path (A <= kAlignFastItems * kAlignThreads, E <= kAlignFastMaxE): warp
+// w owns the contiguous assignments [w C, (w + 1) C), C = 32 R, each lane R of
+// them held in registers (all loaded up front).  Walking its chunk in order,
+// the warp ranks each assignment among equal ids with __match_any_sync on top
+// of a per-warp running count per expert (a [32][E] table); one scan over the
+// 32 warps per expert then gives every warp's base inside each segment, and
+// the totals are the counts N_e.  Chunks are in assignment order, so the ranks
+// keep ascending a within each expert (stable).  Otherwise the rounds of the
+// general path below.
+constexpr int kAlignFastItems = 16;   // assignments per lane on the fast path
+constexpr int kAlignFastMaxE = 512;   // [32][E] int table within the shared-memory budget
+
 __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode, long long P_max, const int32_t* ids,
                                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                             int32_t* __restrict__ sorted_ids, int32_t* __restrict__ block_expert,
@@ -198,19 +210,71 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     int* warp_tot = rt + E;        // 33
     int* bad = warp_tot + 33;      // 1
     int* nmax = bad + 1;           // 1
-    uint16_t* tbl = reinterpret_cast<uint16_t*>(nmax + 1);  // 32 x E
+    uint16_t* tbl = reinterpret_cast<uint16_t*>(nmax + 1);  // general path: 32 x E per round
+    int* wt = nmax + 1;                                       // fast path: 32 x E running counts
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long A = (long long)T * K;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const bool fast = A <= (long long)kAlignFastItems * kAlignThreads && E <= kAlignFastMaxE;
+    // fast path: item i of this lane is assignment a0 + 32 i; packed as
+    // (rank << 11) | (expert + 1), 0 in the low bits for no expert
+    const int R = fast ? (int)((A + kAlignThreads - 1) / kAlignThreads) : 0;
+    const long long a0 = (long long)warp * 32 * R + lane;
+    uint32_t item[kAlignFastItems];
 
-    for (int e = tid; e < E; e += kAlignThreads) cnt[e] = 0;
-    if (tid == 0) *bad = 0, *nmax = 0;
-    __syncthreads();
-    for (long long a = tid; a < A; a += kAlignThreads) {
-        const int e = ids[a];
-        if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[e], 1);
-        else if (e != -1) atomicOr(bad, 1);  // -1: an empty slot (per-token dynamic K)
+    if (fast) {
+        for (int i = tid; i < 32 * E; i += kAlignThreads) wt[i] = 0;
+        if (tid == 0) *bad = 0, *nmax = 0;
+        // ids may come from other blocks of the same kernel: read through L2
+#pragma unroll
+        for (int i = 0; i < kAlignFastItems; ++i) {
+            const long long a = a0 + 32LL * i;
+            item[i] = (i < R && a < A) ? (uint32_t)__ldcg(ids + a) : 0xFFFFFFFFu;
+        }
+        __syncthreads();
+        int* row = wt + warp * E;
+        int badl = 0;
+#pragma unroll
+        for (int i = 0; i < kAlignFastItems; ++i) {
+            if (i < R) {  // the same R in every lane
+                int e = (int)item[i];
+                if ((unsigned)e >= (unsigned)E) {
+                    if (e != -1) badl = 1;  // -1: an empty slot (per-token dynamic K) or past A
+                    e = -1;
+                }
+                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                const int run = e >= 0 ? row[e] : 0;
+                const int rank = run + __popc(peers & lt_mask);
+                __syncwarp();
+                if (e >= 0 && lane == __ffs(peers) - 1) row[e] = run + __popc(peers);
+                __syncwarp();
+                item[i] = ((uint32_t)rank << 11) | (uint32_t)(e + 1);
+            }
+        }
+        if (badl) atomicOr(bad, 1);
+        __syncthreads();
+        // per expert: exclusive scan of the warps' counts in warp order; the total is N_e
+        for (int e = tid; e < E; e += kAlignThreads) {
+            int run = 0;
+            for (int w = 0; w < 32; ++w) {
+                const int c = wt[w * E + e];
+                wt[w * E + e] = run;
+                run += c;
+            }
+            cnt[e] = run;
+        }
+        __syncthreads();
+    } else {
+        for (int e = tid; e < E; e += kAlignThreads) cnt[e] = 0;
+        if (tid == 0) *bad = 0, *nmax = 0;
+        __syncthreads();
+        for (long long a = tid; a < A; a += kAlignThreads) {
+            const int e = __ldcg(ids + a);
+            if ((unsigned)e < (unsigned)E) atomicAdd(&cnt[e], 1);
+            else if (e != -1) atomicOr(bad, 1);  // -1: an empty slot (per-token dynamic K)
+        }
+        __syncthreads();
     }
-    __syncthreads();
 
     // padded counts -> offsets (E <= 1024: one expert per thread).  Block-wise
     // padding rounds each count up to B; max-value padding gives every expert
@@ -258,38 +322,58 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     }
     __syncthreads();
 
-    // stable scatter
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (long long base = 0; base < A; base += kAlignThreads) {
-        const long long a = base + tid;
-        int e = a < A && !overflow ? ids[a] : -1;
-        if ((unsigned)e >= (unsigned)E) e = -1;
-        for (int i = tid; i < 32 * E; i += kAlignThreads) tbl[i] = 0;
-        __syncthreads();
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & lt_mask);
-        if (e >= 0 && lane == __ffs(peers) - 1) tbl[warp * E + e] = (uint16_t)__popc(peers);
-        __syncthreads();
-        if (tid < E) {
-            int run = 0;
-            for (int w = 0; w < 32; ++w) {
-                const int c = tbl[w * E + tid];
-                tbl[w * E + tid] = (uint16_t)run;
-                run += c;
+    if (fast) {
+        // slot = segment start + this warp's base in the segment + rank in the warp
+#pragma unroll
+        for (int i = 0; i < kAlignFastItems; ++i) {
+            if (i < R) {
+                const long long a = a0 + 32LL * i;
+                const int e = (int)(item[i] & 0x7FFu) - 1;
+                if (e >= 0 && !overflow) {
+                    const int p = off[e] + wt[warp * E + e] + (int)(item[i] >> 11);
+                    sorted_ids[p] = (int32_t)a;
+                    pos[a] = p;
+                } else if (a < A) {
+                    pos[a] = -1;  // empty slot (or an out-of-range id, flagged above)
+                }
             }
-            rt[tid] = run;
         }
-        __syncthreads();
-        if (e >= 0) {
-            const int p = cursor[e] + tbl[warp * E + e] + rank;
-            sorted_ids[p] = (int32_t)a;
-            pos[a] = p;
-        } else if (a < A) {
-            pos[a] = -1;  // empty slot (or an out-of-range id, flagged above)
+    } else {
+        // stable scatter in rounds of kAlignThreads assignments: the rank among
+        // equal ids inside a warp from __match_any_sync, across the warps of a
+        // round from a per-(warp, expert) count table scanned over the warps,
+        // across rounds from a per-expert cursor
+        for (long long base = 0; base < A; base += kAlignThreads) {
+            const long long a = base + tid;
+            int e = a < A && !overflow ? __ldcg(ids + a) : -1;
+            if ((unsigned)e >= (unsigned)E) e = -1;
+            for (int i = tid; i < 32 * E; i += kAlignThreads) tbl[i] = 0;
+            __syncthreads();
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int rank = __popc(peers & lt_mask);
+            if (e >= 0 && lane == __ffs(peers) - 1) tbl[warp * E + e] = (uint16_t)__popc(peers);
+            __syncthreads();
+            if (tid < E) {
+                int run = 0;
+                for (int w = 0; w < 32; ++w) {
+                    const int c = tbl[w * E + tid];
+                    tbl[w * E + tid] = (uint16_t)run;
+                    run += c;
+                }
+                rt[tid] = run;
+            }
+            __syncthreads();
+            if (e >= 0) {
+                const int p = cursor[e] + tbl[warp * E + e] + rank;
+                sorted_ids[p] = (int32_t)a;
+                pos[a] = p;
+            } else if (a < A) {
+                pos[a] = -1;  // empty slot (or an out-of-range id, flagged above)
+            }
+            __syncthreads();
+            if (tid < E) cursor[tid] += rt[tid];
+            __syncthreads();
         }
-        __syncthreads();
-        if (tid < E) cursor[tid] += rt[tid];
-        __syncthreads();
     }
 
     // padding slots inside each segment, then everything past P
@@ -326,7 +410,12 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
                 sm);
 }
 
-size_t align_smem_bytes(int E) { return sizeof(int) * (4 * (size_t)E + 1 + 35) + sizeof(uint16_t) * 32 * (size_t)E; }
+// cnt, off, cursor, rt, the scan words and flags, then the [32][E] table (int
+// counts on the fast path when E allows it, uint16 per round otherwise)
+size_t align_smem_bytes(int E) {
+    const size_t table = E <= kAlignFastMaxE ? sizeof(int) * 32 * (size_t)E : sizeof(uint16_t) * 32 * (size_t)E;
+    return sizeof(int) * (4 * (size_t)E + 1 + 35) + table;
+}
 
 // ----------------------------------------------------- small-batch routing
 // Router logits, top-K gating and alignment in one launch for small T.
@@ -514,6 +603,101 @@ __global__ void __launch_bounds__(256) router_cc_kernel(int T_, int H, const T* 
     }
 }
 
+// Router logits, top-K gating and alignment in one launch for router
+// matrices that fit shared memory (the layer's routing above the small-batch
+// size): blocks of 1024 threads stage w_r in shared memory; each warp takes
+// whole tokens, computes the E logits as router_cc_kernel does (the same
+// products and summation order), stores them, and runs the top-K and gate
+// weights of topk_gate_kernel on the stored row (or on logits_override).  The
+// last block to finish (a counter; no block waits) runs the alignment over all
+// T, reusing its shared memory.
+template <typename T, int kE>
+__global__ void __launch_bounds__(kAlignThreads, 1)
+    route_cc_kernel(int T_, int H, int K, int score_fn, int renorm, int B, int mode, long long P_max,
+                    const T* __restrict__ x, const T* __restrict__ w_r, const float* __restrict__ logits_override,
+                    const int32_t* __restrict__ k_per_token, float* __restrict__ logits, int32_t* __restrict__ ids,
+                    float* __restrict__ w, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                    int32_t* __restrict__ sorted_ids, int32_t* __restrict__ block_expert, int32_t* __restrict__ pos,
+                    int32_t* __restrict__ scalars, int32_t* __restrict__ stats_copy, int* __restrict__ done_ctr) {
+    extern __shared__ int4 route_sm[];
+    __shared__ int is_last;
+    const T* ws = reinterpret_cast<const T*>(route_sm);
+    pdl_launch_dependents();
+    const int n16 = (int)((long long)kE * H * sizeof(T) / 16);
+    const int4* wsrc = reinterpret_cast<const int4*>(w_r);
+    for (int i0 = threadIdx.x; i0 < n16; i0 += 4 * blockDim.x) {
+        int4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i0 + j * (int)blockDim.x < n16) v[j] = __ldg(wsrc + i0 + j * blockDim.x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i0 + j * (int)blockDim.x < n16) route_sm[i0 + j * blockDim.x] = v[j];
+    }
+    pdl_wait();
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int warps = blockDim.x >> 5;
+    // 1024-thread blocks leave 64 registers a thread: the token row's 16-byte
+    // words stay packed while in flight (32 registers: 8 chunks of bf16, 4 of
+    // fp32) and each chunk is widened when it is used; the products and their
+    // order are those of router_cc_kernel
+    constexpr int kChunks = sizeof(T) == 2 ? 8 : 4;
+    constexpr int kWords = 8 * sizeof(T) / 16;  // 16-byte words per chunk of 8 elements
+    for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T_; t += gridDim.x * warps) {
+        float acc[kE];
+#pragma unroll
+        for (int e = 0; e < kE; ++e) acc[e] = 0.f;
+        const T* xr = x + (size_t)t * H;
+        for (int h0 = lane * 8; h0 < H; h0 += kChunks * 256) {
+            int4 raw[kChunks * kWords];
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+                if (h0 + c * 256 < H) {
+#pragma unroll
+                    for (int q = 0; q < kWords; ++q)
+                        raw[c * kWords + q] = __ldg(reinterpret_cast<const int4*>(xr + h0 + c * 256) + q);
+                }
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                const int h = h0 + c * 256;
+                if (h < H) {
+                    float xv[8];
+                    load8_shared(reinterpret_cast<const T*>(&raw[c * kWords]), xv);
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) {
+                        float wv[8];
+                        load8_shared(ws + (size_t)e * H + h, wv);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[e] = fmaf(wv[j], xv[j], acc[e]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < kE; ++e) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        }
+#pragma unroll
+        for (int e = 0; e < kE; ++e)
+            if (lane == e) logits[(size_t)t * kE + e] = acc[e];
+        __syncwarp();  // the row is complete before the warp reads it back
+        const float* src = logits_override ? logits_override + (size_t)t * kE : logits + (size_t)t * kE;
+        topk_one_token(src, kE, K, token_k(k_per_token, t, K), score_fn, renorm, ids + (size_t)t * K,
+                       w + (size_t)t * K, lane);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(done_ctr, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    align_block(T_, K, kE, B, mode, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy,
+                reinterpret_cast<int*>(route_sm));
+    if (threadIdx.x == 0) *done_ctr = 0;  // ready for the next launch
+}
+
 bool router_cc_fits(int H, int E, int dtype) {
     const long long eb = dtype == 0 ? 2 : 4;
     return E >= 1 && E <= 16 && H > 0 && H % 8 == 0 && (long long)E * H * eb <= kRouterCcMaxBytes;
@@ -560,6 +744,52 @@ int launch_router_cc(int T, int H, int E, int dtype, const void* x, const void* 
     if (rc != 0) return rc;
     cudaError_t e = dtype == 0 ? launch_router_cc_t<__nv_bfloat16>(T, H, E, x, w_r, logits, d.num_sms, stream)
                                : launch_router_cc_t<float>(T, H, E, x, w_r, logits, d.num_sms, stream);
+    count_launch();
+    return launched(e);
+}
+
+template <typename T, int kE>
+cudaError_t launch_route_cc_e(const RouteCcArgs& a, int num_sms, cudaStream_t stream) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(route_cc_kernel<T, kE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kRouterCcMaxBytes);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    // one token per warp where T allows, at most two blocks per SM
+    long long blocks = (a.T + 31) / 32;
+    if (blocks > 2LL * num_sms) blocks = 2LL * num_sms;
+    const size_t wr = (size_t)kE * a.H * sizeof(T), al = align_smem_bytes(kE);
+    return launch_kernel(route_cc_kernel<T, kE>, dim3((int)blocks), dim3(kAlignThreads), wr > al ? wr : al, stream,
+                         a.T, a.H, a.K, a.score_fn, a.renorm, a.B, a.mode, a.P_max, static_cast<const T*>(a.x),
+                         static_cast<const T*>(a.w_r), a.logits_override, a.k_per_token, a.logits, a.ids, a.w,
+                         a.counts, a.offsets, a.sorted_ids, a.block_expert, a.pos, a.scalars, a.stats_copy,
+                         a.done_ctr);
+}
+
+template <typename T>
+cudaError_t launch_route_cc_t(const RouteCcArgs& a, int num_sms, cudaStream_t s) {
+    switch (a.E) {
+#define MOE_ROUTE_CC_CASE(n) \
+    case n: return launch_route_cc_e<T, n>(a, num_sms, s);
+        MOE_ROUTE_CC_CASE(1) MOE_ROUTE_CC_CASE(2) MOE_ROUTE_CC_CASE(3) MOE_ROUTE_CC_CASE(4)
+        MOE_ROUTE_CC_CASE(5) MOE_ROUTE_CC_CASE(6) MOE_ROUTE_CC_CASE(7) MOE_ROUTE_CC_CASE(8)
+        MOE_ROUTE_CC_CASE(9) MOE_ROUTE_CC_CASE(10) MOE_ROUTE_CC_CASE(11) MOE_ROUTE_CC_CASE(12)
+        MOE_ROUTE_CC_CASE(13) MOE_ROUTE_CC_CASE(14) MOE_ROUTE_CC_CASE(15) MOE_ROUTE_CC_CASE(16)
+#undef MOE_ROUTE_CC_CASE
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+int launch_route_cc(const RouteCcArgs& a, cudaStream_t stream) {
+    if (a.T == 0) return 0;
+    if (!router_cc_fits(a.H, a.E, a.dtype)) return -1;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    cudaError_t e = a.dtype == 0 ? launch_route_cc_t<__nv_bfloat16>(a, d.num_sms, stream)
+                                 : launch_route_cc_t<float>(a, d.num_sms, stream);
     count_launch();
     return launched(e);
 }
@@ -766,69 +996,93 @@ __device__ __forceinline__ void store_sums(const float* acc, float* out) {
         *reinterpret_cast<float4*>(out + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
 }
 
-template <typename T, typename TOut>
-__global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K, const int4* __restrict__ y_perm,
+// One thread per 16-byte vector of one token's output row: the K expert rows'
+// vectors are all requested before the first is used (K <= 16, unrolled), then
+// summed in fp32 in ascending k (empty slots skipped), the shared output added
+// last, one rounding.  The output holds the columns [col0, col0 + ncol) (in
+// 16-byte vectors of the input rows; ncol vectors per output row).
+template <typename T, typename TOut, int kMaxK>
+__global__ void __launch_bounds__(256) combine_kernel(int T_, int row_vec, int K, int col0, int ncol,
+                                                      const int4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ pos, const float* __restrict__ w,
                                                       const int4* __restrict__ sh, TOut* __restrict__ out) {
     constexpr int N = Vec16<T>::N;
-    __shared__ int s_pos[16];
-    __shared__ float s_w[16];
     pdl_launch_dependents();
     pdl_wait();
-    for (int t = blockIdx.x; t < T_; t += gridDim.x) {
-        __syncthreads();
-        if (threadIdx.x < K) {
-            s_pos[threadIdx.x] = pos[(long long)t * K + threadIdx.x];
-            s_w[threadIdx.x] = w[(long long)t * K + threadIdx.x];
-        }
-        __syncthreads();
-        for (int v = threadIdx.x; v < row_vec; v += blockDim.x) {
-            float acc[N];
+    const long long total = (long long)T_ * ncol;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long t = i / ncol;
+        const int v = col0 + (int)(i - t * ncol);
+        int p[kMaxK];
+        int4 yv[kMaxK];
 #pragma unroll
-            for (int i = 0; i < N; ++i) acc[i] = 0.f;
-            for (int k = 0; k < K; ++k) {
-                if (s_pos[k] < 0) continue;  // empty slot (per-token dynamic K)
+        for (int k = 0; k < kMaxK; ++k)
+            if (k < K) p[k] = __ldg(pos + t * K + k);
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k)
+            if (k < K && p[k] >= 0) yv[k] = __ldcs(y_perm + (long long)p[k] * row_vec + v);
+        int4 sv = make_int4(0, 0, 0, 0);
+        if (sh) sv = __ldcs(sh + t * row_vec + v);
+        float acc[N];
+#pragma unroll
+        for (int j = 0; j < N; ++j) acc[j] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+            if (k < K && p[k] >= 0) {  // empty slot (per-token dynamic K): skipped
                 float y[N];
-                unpack(__ldg(y_perm + (long long)s_pos[k] * row_vec + v), y, (const T*)nullptr);
-                const float wk = s_w[k];
+                unpack(yv[k], y, (const T*)nullptr);
+                const float wk = __ldg(w + t * K + k);
 #pragma unroll
-                for (int i = 0; i < N; ++i) acc[i] += wk * y[i];
+                for (int j = 0; j < N; ++j) acc[j] += wk * y[j];
             }
-            if (sh) {
-                float y[N];
-                unpack(__ldg(sh + (long long)t * row_vec + v), y, (const T*)nullptr);
-#pragma unroll
-                for (int i = 0; i < N; ++i) acc[i] += y[i];
-            }
-            store_sums<N>(acc, out + ((long long)t * row_vec + v) * N);
         }
+        if (sh) {
+            float y[N];
+            unpack(sv, y, (const T*)nullptr);
+#pragma unroll
+            for (int j = 0; j < N; ++j) acc[j] += y[j];
+        }
+        store_sums<N>(acc, out + i * N);
     }
 }
 
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,
-                   const void* shared_out, void* out, cudaStream_t stream, bool out_f32) {
+                   const void* shared_out, void* out, cudaStream_t stream, bool out_f32, int col0, int ncols) {
     if (T == 0) return 0;
     DeviceInfo d;
     int rc = current_device(&d);
     if (rc != 0) return rc;
     const int elt = dtype == 0 ? 2 : 4;
     const int row_vec = H * elt / 16;
-    const int threads = row_vec >= 256 ? 256 : ((row_vec + 31) / 32) * 32;
-    long long blocks = T;
-    const long long cap = (long long)d.num_sms * 16;
-    if (blocks > cap) blocks = cap;
+    if (ncols < 0) col0 = 0, ncols = H;
+    if ((col0 * elt) % 16 || (ncols * elt) % 16 || col0 < 0 || col0 + ncols > H) return -1;
+    const int c0 = col0 * elt / 16, nc = ncols * elt / 16;
+    const int threads = 256;
+    // one thread per output vector (a grid of up to 2^31 - 1 blocks covers
+    // every layer this library accepts; beyond that the threads stride)
+    long long blocks = ((long long)T * nc + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) blocks = 0x7fffffffLL;
     const int4* y4 = static_cast<const int4*>(y_perm);
     const int4* s4 = static_cast<const int4*>(shared_out);
+    const dim3 g((unsigned)blocks), b(threads);
     cudaError_t e;
-    if (dtype == 0 && !out_f32)
-        e = launch_kernel(combine_kernel<__nv_bfloat16, __nv_bfloat16>, dim3((int)blocks), dim3(threads), 0, stream,
-                          T, row_vec, K, y4, pos, w, s4, static_cast<__nv_bfloat16*>(out));
-    else if (dtype == 0)
-        e = launch_kernel(combine_kernel<__nv_bfloat16, float>, dim3((int)blocks), dim3(threads), 0, stream, T,
-                          row_vec, K, y4, pos, w, s4, static_cast<float*>(out));
-    else
-        e = launch_kernel(combine_kernel<float, float>, dim3((int)blocks), dim3(threads), 0, stream, T, row_vec, K,
-                          y4, pos, w, s4, static_cast<float*>(out));
+    // the K expert rows are held in registers: size the array to K's bucket
+    auto go = [&](auto kmax) -> cudaError_t {
+        constexpr int kK = decltype(kmax)::value;
+        if (dtype == 0 && !out_f32)
+            return launch_kernel(combine_kernel<__nv_bfloat16, __nv_bfloat16, kK>, g, b, 0, stream, T, row_vec, K, c0,
+                                 nc, y4, pos, w, s4, static_cast<__nv_bfloat16*>(out));
+        if (dtype == 0)
+            return launch_kernel(combine_kernel<__nv_bfloat16, float, kK>, g, b, 0, stream, T, row_vec, K, c0, nc, y4,
+                                 pos, w, s4, static_cast<float*>(out));
+        return launch_kernel(combine_kernel<float, float, kK>, g, b, 0, stream, T, row_vec, K, c0, nc, y4, pos, w, s4,
+                             static_cast<float*>(out));
+    };
+    if (K <= 2) e = go(std::integral_constant<int, 2>());
+    else if (K <= 4) e = go(std::integral_constant<int, 4>());
+    else if (K <= 8) e = go(std::integral_constant<int, 8>());
+    else e = go(std::integral_constant<int, 16>());
     count_launch();
     return launched(e);
 }
@@ -889,6 +1143,43 @@ int launch_tp_reduce(int n, const float* const* parts, long long count, int dtyp
                                                stream, tp, n, n4, static_cast<__nv_bfloat16*>(out))
                                : launch_kernel(tp_reduce_kernel<float>, dim3((int)blocks), dim3(256), 0, stream, tp,
                                                n, n4, static_cast<float*>(out));
+    count_launch();
+    return launched(e);
+}
+
+// One output row from n all-reduced column blocks: out[t][c * Hc + j] =
+// parts[c][t * Hc + j], rounded once to the output dtype (4 elements per
+// thread, grid-stride over all T * H).
+template <typename TOut>
+__global__ void __launch_bounds__(256) tp_gather_kernel(TpParts parts, int T_, int hc4, int n, TOut* __restrict__ out) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long row4 = (long long)hc4 * n;
+    const long long total = (long long)T_ * row4;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+        const long long t = i / row4;
+        const int rem = (int)(i - t * row4);
+        const int c = rem / hc4, j = rem - c * hc4;
+        store4<TOut>(out, i, __ldcs(parts.p[c] + t * hc4 + j));
+    }
+}
+
+int launch_tp_gather(int n, const float* const* parts, int T, int H, int dtype, void* out, cudaStream_t stream) {
+    if (T == 0) return 0;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    TpParts tp{};
+    for (int r = 0; r < n; ++r) tp.p[r] = reinterpret_cast<const float4*>(parts[r]);
+    const int hc4 = H / n / 4;
+    const long long total = (long long)T * H / 4;
+    long long blocks = (total + 255) / 256;
+    const long long cap = (long long)d.num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    cudaError_t e = dtype == 0 ? launch_kernel(tp_gather_kernel<__nv_bfloat16>, dim3((int)blocks), dim3(256), 0,
+                                               stream, tp, T, hc4, n, static_cast<__nv_bfloat16*>(out))
+                               : launch_kernel(tp_gather_kernel<float>, dim3((int)blocks), dim3(256), 0, stream, tp,
+                                               T, hc4, n, static_cast<float*>(out));
     count_launch();
     return launched(e);
 }

@@ -78,6 +78,22 @@ def test_launch_count_of_a_prefill_forward():
     before = moe.kernel_launch_count()
     moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws)
     moe.check_status(ws)
+    # routing (router logits on the CUDA cores for this 8 x 256 router matrix,
+    # top-K and alignment in one launch), permute, gate/up, down, combine
+    assert not moe.ffn_fused(cfg)
+    assert moe.kernel_launch_count() - before == 5
+
+
+def test_launch_count_of_a_prefill_forward_with_a_tensor_core_router():
+    shape = small_shape(H=256, E=64, K=4, I=512)
+    T = 4000  # 250 rows per expert: the two-launch expert FFN
+    w = mi.make_weights(shape, 2, device="cuda")
+    x = mi.make_x(shape, T, 2, device="cuda")
+    cfg = cfg_for(shape, T)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    before = moe.kernel_launch_count()
+    moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws)
+    moe.check_status(ws)
     # router GEMM, top-K, align, permute, gate/up, down, combine
     assert not moe.ffn_fused(cfg)
     assert moe.kernel_launch_count() - before == 7

@@ -140,3 +140,80 @@ def test_tp_argument_errors():
         moe.tp_shard(w13, w2, 0, 5)                   # 24 does not split over 5
     with pytest.raises(ValueError):
         moe.tp_config(moe.config(4, 16, 2, 1, 24), 5)
+
+
+@pytest.mark.parametrize("n_ranks,n_chunks", [(2, 2), (2, 4), (4, 4), (1, 3)])
+def test_tp_overlapped_down_chunks(n_ranks, n_chunks):
+    # the all-reduce overlapped with the down projection: per rank the front
+    # part, then the down projection + combine of each block of H / n_chunks
+    # output features into its own fp32 part; the parts summed over the ranks
+    # (here in rank order on one GPU, where an all-reduce would run) and placed
+    # side by side are the layer; every rank's blocks side by side are its
+    # slice's partial output.  T = 700 on 16 experts: 175 rows per expert, the
+    # two-launch expert FFN (CTA-pair GEMMs) and the shared GEMM pair.
+    shape = small_shape(H=768, E=16, K=4, I=768, I_sh=384)
+    T, seed = 700, 41 + n_ranks + n_chunks
+    w = mi.make_weights(shape, seed, device="cuda")
+    x = mi.make_x(shape, T, seed, device="cuda")
+    cl = moe.tp_config(cfg_for(shape, T), n_ranks)
+    assert not moe.ffn_fused(cl)
+    ws = moe.alloc_workspace(moe.workspace_size(cl))
+    total = [torch.zeros((T, shape.H // n_chunks), dtype=torch.float32, device="cuda") for _ in range(n_chunks)]
+    tok = sample_tokens(T, 128, seed)
+    hx, h13, h2 = host(x), host(w["w13"]), host(w["w2"])
+    hs13, hs2 = host(w["w13_sh"]), host(w["w2_sh"])
+    lg = None
+    for r in range(n_ranks):
+        a13, a2 = moe.tp_shard(w["w13"], w["w2"], r, n_ranks)
+        s13, s2 = moe.tp_shard(w["w13_sh"], w["w2_sh"], r, n_ranks)
+        moe.layer_forward_partial_front(cl, x, w["w_r"], a13, ws, s13, s2)
+        parts = [moe.layer_forward_partial_down(cl, a2, c, n_chunks, ws) for c in range(n_chunks)]
+        moe.check_status(ws)
+        if lg is None:
+            lg = moe.layer_logits(cl, ws).cpu().numpy()
+        full_r = torch.cat(parts, dim=1).cpu().numpy()
+        o13, o2 = oracle.tp_shard(h13, h2, r, n_ranks)
+        q13, q2 = oracle.tp_shard(hs13, hs2, r, n_ranks)
+        ref_r = oracle.moe_layer(hx, None, o13, o2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok,
+                                 w13_sh=q13, w2_sh=q2)
+        assert rel_err(full_r[tok], ref_r) < OUT_TOL
+        for c in range(n_chunks):
+            total[c] += parts[c]
+    out = moe.tp_gather(total, torch.empty((T, shape.H), dtype=x.dtype, device="cuda"))
+    torch.cuda.synchronize()
+    ref = oracle.moe_layer(hx, None, h13, h2, shape.K, shape.score_fn, shape.renorm, logits=lg, tokens=tok,
+                           w13_sh=hs13, w2_sh=hs2)
+    assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
+
+
+def test_tp_overlapped_one_rank_equals_the_layer():
+    # the whole overlapped step on one rank (the all-reduce has nothing to sum)
+    # against the unsplit layer: the same routing and the same numerics up to
+    # the fp32 order of the down GEMM's split tiles
+    shape = small_shape(H=512, E=8, K=2, I=1024, I_sh=512)
+    T = 1200
+    w = mi.make_weights(shape, 9, device="cuda")
+    x = mi.make_x(shape, T, 9, device="cuda")
+    cfg = cfg_for(shape, T)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    ref = moe.layer_forward(cfg, x, w["w_r"], w["w13"], w["w2"], ws, w["w13_sh"], w["w2_sh"]).float()
+    cl = moe.tp_config(cfg, 1)
+    out = moe.tp_layer_forward_overlapped(cl, x, w["w_r"], w["w13"], w["w2"], ws, w["w13_sh"], w["w2_sh"],
+                                          n_chunks=4)
+    moe.check_status(ws)
+    assert rel_err(out.float().cpu().numpy(), ref.cpu().numpy()) < 1e-2
+
+
+def test_tp_down_chunk_arguments():
+    shape = small_shape(H=512, E=8, K=2, I=512)
+    cfg = cfg_for(shape, 1200)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    w2 = torch.zeros((8, 512, 512), dtype=torch.bfloat16, device="cuda")
+    for chunk, n in [(0, 3), (4, 4), (-1, 2), (0, 0)]:       # 512 / 3 not whole; chunk out of range
+        with pytest.raises(moe.MoeError):
+            moe.layer_forward_partial_down(cfg, w2, chunk, n, ws,
+                                           torch.empty((1200, 128), dtype=torch.float32, device="cuda"))
+    small = cfg_for(shape, 8)                                 # decode size: the fused expert FFN
+    with pytest.raises(moe.MoeError):
+        moe.layer_forward_partial_down(small, w2, 0, 2, moe.alloc_workspace(moe.workspace_size(small)),
+                                       torch.empty((8, 256), dtype=torch.float32, device="cuda"))

@@ -81,3 +81,41 @@ def test_tp_config_splits_I_and_the_shared_width():
     assert moe.tp_config(moe.config(4, 4096, 8, 2, 14336), 8).n_shared == 0
     with pytest.raises(ValueError):
         moe.tp_config(moe.config(4, 4096, 8, 2, 14336), 5)
+
+
+def _rank_overlapped(rank, world, port, n_chunks, out):
+    # the overlap protocol: each block of H / n_chunks output features is
+    # produced, its all-reduce started asynchronously, the next block produced
+    # beside it; the blocks side by side after all waits are the whole layer
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x, w_r, w13, w2, w13_sh, w2_sh, K = _layer(5)
+        a13, a2 = oracle.tp_shard(w13, w2, rank, world)
+        s13, s2 = oracle.tp_shard(w13_sh, w2_sh, rank, world)
+        mine = oracle.moe_layer(x, w_r, a13, a2, K, w13_sh=s13, w2_sh=s2, nthreads=1)
+        Hc = mine.shape[1] // n_chunks
+        parts = [torch.empty((mine.shape[0], Hc), dtype=torch.float64) for _ in range(n_chunks)]
+        order = []
+
+        def produce(c):
+            order.append(c)
+            parts[c].copy_(torch.from_numpy(np.ascontiguousarray(mine[:, c * Hc:(c + 1) * Hc])))
+
+        moe.tp_overlapped_allreduce(parts, produce)
+        out[rank] = (order, torch.cat(parts, dim=1).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,n_chunks", [(2, 2), (2, 4), (4, 4)])
+def test_tp_overlapped_allreduce_protocol_gloo(world, n_chunks):
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_rank_overlapped, args=(world, _free_port(), n_chunks, out), nprocs=world, join=True)
+    x, w_r, w13, w2, w13_sh, w2_sh, K = _layer(5)
+    full = oracle.moe_layer(x, w_r, w13, w2, K, w13_sh=w13_sh, w2_sh=w2_sh)
+    for r in range(world):
+        order, got = out[r]
+        assert order == list(range(n_chunks))
+        assert np.allclose(got, full, rtol=1e-10, atol=1e-10)
