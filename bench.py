@@ -166,6 +166,8 @@ class Workload:
         self.s_act = torch.empty((Pm, shape.I), dtype=dt, device=device)
         self.s_y = torch.empty((Pm, shape.H), dtype=dt, device=device)
         self.s_sh = torch.empty((T, shape.H), dtype=dt, device=device) if shape.I_sh else None
+        # the FP8 path's token operand: E4M3 hi/lo codes (in s_xp's bytes) and row scales
+        self.s_xsc = torch.empty((Pm,), dtype=torch.float32, device=device)
         self.s_shws = None
         if shape.I_sh:
             n = (moe.dense_fp8_workspace_size(T, shape.H, shape.I_sh) if fp8
@@ -212,13 +214,15 @@ class Workload:
         self.al = m.align_pad(c, self.s_ids, self.s_al)
         ev[3].record()
         if self.fp8:
-            m.permute_f16(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
+            m.permute_e4m3x2(c, self.x, self.al["sorted_ids"], self.al["scalars"],
+                             self.s_xp.view(torch.uint8).view(2 * self.s_xp.shape[0], -1), self.s_xsc)
         else:
             m.permute(c, self.x, self.al["sorted_ids"], self.al["scalars"], self.s_xp)
         ev[4].record()
         if self.fp8:
             q = self.q
-            m.grouped_ffn_fp8(c, self.s_xp, q["w13"][0], q["w13"][1], q["w2"][0], q["w2"][1], self.al["offsets"],
+            m.grouped_ffn_fp8(c, self.s_xp.view(torch.uint8).view(2 * self.s_xp.shape[0], -1), self.s_xsc,
+                              q["w13"][0], q["w13"][1], q["w2"][0], q["w2"][1], self.al["offsets"],
                               self.gws, self.s_act, self.s_y)
             ev[5].record()
         elif self.fused:

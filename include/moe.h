@@ -288,23 +288,36 @@ int moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_
                           const int32_t* k_per_token, void* out, void* workspace,
                           size_t ws_bytes, int32_t* stats_out, moe_stream_t stream);
 
-/* moe_permute writing the permuted rows as f16 (the FP8-weight path computes
- * on f16 operands; E4M3 values are exact in f16); bf16 x (cfg->dtype 0). */
-int moe_permute_f16(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids,
-                    const int32_t* scalars, void* x_perm, moe_stream_t stream);
+/* moe_permute for the FP8-weight path (bf16 x, cfg->dtype 0): each permuted
+ * row p < scalars[0] is split exactly into two E4M3 code rows and a power-of-
+ * two scale, x[sorted_ids[p] / K] = x_scales[p] * (hi + lo), with hi the
+ * row's codes x_codes[p] and lo the remainder's codes x_codes[P_max + p]
+ * (P_max = moe_padded_rows_max(cfg)); x_scales[p] is the smallest power of
+ * two with max|row| <= 448 x_scales[p].  The split is exact except where the
+ * remainder is below E4M3's subnormal grid (under 2^-17 of the row's largest
+ * magnitude), which rounds to the nearest grid value.  Padding rows get zero
+ * codes and scale 1.  x_codes: [2 P_max, H] bytes (16-byte aligned); x_scales:
+ * [P_max] floats.  The FP8 gate/up products then run as two E4M3 x E4M3
+ * tensor-core products per weight tile (Blackwell kind::f8f6f4).  Errors:
+ * MOE_ERR_ARG for a bad config, dtype != 0 or a null/misaligned pointer. */
+int moe_permute_e4m3x2(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids,
+                       const int32_t* scalars, uint8_t* x_codes, float* x_scales,
+                       moe_stream_t stream);
 
 /* moe_grouped_ffn with FP8 routed expert weights (codes and row scales as
  * for moe_layer_forward_fp8); decode sizes only (at most 128 rows per
- * expert).  x_perm is f16 (moe_permute_f16); `act` is f16 scratch
- * ([P_max, I]); y_perm is bf16. */
-int moe_grouped_ffn_fp8(const moe_config_t* cfg, const void* x_perm, const uint8_t* w13_q,
-                        const float* w13_s, const uint8_t* w2_q, const float* w2_s,
-                        const int32_t* offsets, void* act, void* y_perm, void* workspace,
-                        size_t ws_bytes, moe_stream_t stream);
+ * expert).  x_codes / x_scales as written by moe_permute_e4m3x2; `act` is
+ * f16 scratch ([P_max, I]); y_perm is bf16 [P_max, H] and must not overlap
+ * x_codes. */
+int moe_grouped_ffn_fp8(const moe_config_t* cfg, const uint8_t* x_codes, const float* x_scales,
+                        const uint8_t* w13_q, const float* w13_s, const uint8_t* w2_q,
+                        const float* w2_s, const int32_t* offsets, void* act, void* y_perm,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* dense_ffn with FP8 weights (codes [2I,H] / [H,I] and row scales [2I] /
  * [H]), bf16 x and out; decode sizes only (T <= 128); workspace of
- * dense_ffn_fp8_workspace_size bytes (x is widened to f16 there). */
+ * dense_ffn_fp8_workspace_size bytes (x's E4M3 hi/lo split, as in
+ * moe_permute_e4m3x2, is written there). */
 size_t dense_ffn_fp8_workspace_size(int T, int H, int I);
 int dense_ffn_fp8(int T, int H, int I, const void* x, const uint8_t* w13_q, const float* w13_s,
                   const uint8_t* w2_q, const float* w2_s, void* out, void* workspace,
@@ -369,15 +382,6 @@ void moe_set_programmatic_launch(int enable);
  * with 256 weight rows per pair).  0 keeps single-SM tiles.  Process-wide;
  * results are identical up to fp32 summation order. */
 void moe_set_cta_pairs(int enable);
-
-/* FP8 expert weights on CTA pairs (default off): the fused decode FFN of
- * moe_layer_forward_fp8 / moe_grouped_ffn_fp8 / dense_ffn_fp8 runs on pairs of
- * SMs (thread-block clusters of 2), each CTA widening its own 128 weight rows
- * into its own tensor memory and one 2-SM MMA covering both (M = 256): half
- * the MMA instructions per weight byte.  Needs H and I multiples of 64; token
- * tiles are then multiples of 32 rows.  0 keeps one CTA per tile.
- * Process-wide; results agree up to fp32 summation order. */
-void moe_set_fp8_pairs(int enable);
 
 /* Shared experts beside the routed experts.  With n_shared > 0,
  * moe_layer_forward launches the shared FFN first, on a second stream that

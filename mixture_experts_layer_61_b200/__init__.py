@@ -77,10 +77,10 @@ def lib():
             "moe_layer_forward": (I, [C, P, P, P, P, P, P, P, P, P, S, P, P]),
             "moe_layer_forward_k": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P, P]),
             "moe_quantize_fp8": (I, [ctypes.c_int64, I, I, P, P, P, P]),
-            "moe_grouped_ffn_fp8": (I, [C, P, P, P, P, P, P, P, P, P, S, P]),
+            "moe_grouped_ffn_fp8": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
             "dense_ffn_fp8": (I, [I, I, I, P, P, P, P, P, P, P, S, P]),
             "dense_ffn_fp8_workspace_size": (S, [I, I, I]),
-            "moe_permute_f16": (I, [C, P, P, P, P, P]),
+            "moe_permute_e4m3x2": (I, [C, P, P, P, P, P, P]),
             "moe_layer_forward_fp8": (I, [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P, P]),
             "dense_ffn_workspace_size": (S, [I, I, I, I]),
             "dense_ffn": (I, [I, I, I, I, P, P, P, P, P, S, P]),
@@ -91,7 +91,6 @@ def lib():
             "moe_set_programmatic_launch": (None, [I]),
             "moe_set_split_tail": (I, [I]),
             "moe_set_cta_pairs": (None, [I]),
-            "moe_set_fp8_pairs": (None, [I]),
             "moe_set_shared_sms": (I, [I]),
             "moe_shared_sms": (I, [C]),
             "moe_ffn_fused": (I, [C]),
@@ -305,20 +304,26 @@ def dense_fp8_workspace_size(T, H, I):
     return int(lib().dense_ffn_fp8_workspace_size(T, H, I))
 
 
-def permute_f16(cfg, x, sorted_ids, scalars, x_perm=None):
-    """moe_permute writing f16 rows (the FP8-weight path's token operand)."""
+def permute_e4m3x2(cfg, x, sorted_ids, scalars, x_codes=None, x_scales=None):
+    """moe_permute for the FP8-weight path: the permuted rows split exactly
+    into E4M3 hi codes (rows [0, P_max)), lo codes (rows [P_max, 2 P_max))
+    and power-of-two row scales."""
     _need_cuda(x, sorted_ids, scalars)
-    if x_perm is None:
-        x_perm = torch.empty((max(padded_rows_max(cfg), 1), cfg.H), dtype=torch.float16, device=x.device)
-    _check(lib().moe_permute_f16(ctypes.byref(cfg), _p(x), _p(sorted_ids), _p(scalars), _p(x_perm), _stream()),
-           "moe_permute_f16")
-    return x_perm
+    Pm = max(padded_rows_max(cfg), 1)
+    if x_codes is None:
+        x_codes = torch.empty((2 * Pm, cfg.H), dtype=torch.uint8, device=x.device)
+    if x_scales is None:
+        x_scales = torch.empty((Pm,), dtype=torch.float32, device=x.device)
+    _check(lib().moe_permute_e4m3x2(ctypes.byref(cfg), _p(x), _p(sorted_ids), _p(scalars), _p(x_codes),
+                                    _p(x_scales), _stream()), "moe_permute_e4m3x2")
+    return x_codes, x_scales
 
 
-def grouped_ffn_fp8(cfg, x_perm, q13, s13, q2, s2, offsets, ws, act, y_perm):
-    _need_cuda(x_perm, q13, s13, q2, s2, offsets, ws, act, y_perm)
-    _check(lib().moe_grouped_ffn_fp8(ctypes.byref(cfg), _p(x_perm), _p(q13), _p(s13), _p(q2), _p(s2), _p(offsets),
-                                     _p(act), _p(y_perm), _p(ws), ws.numel(), _stream()), "moe_grouped_ffn_fp8")
+def grouped_ffn_fp8(cfg, x_codes, x_scales, q13, s13, q2, s2, offsets, ws, act, y_perm):
+    _need_cuda(x_codes, x_scales, q13, s13, q2, s2, offsets, ws, act, y_perm)
+    _check(lib().moe_grouped_ffn_fp8(ctypes.byref(cfg), _p(x_codes), _p(x_scales), _p(q13), _p(s13), _p(q2),
+                                     _p(s2), _p(offsets), _p(act), _p(y_perm), _p(ws), ws.numel(), _stream()),
+           "moe_grouped_ffn_fp8")
     return y_perm, act
 
 
@@ -389,11 +394,6 @@ def ffn_fused(cfg):
 def set_cta_pairs(enable=True):
     """2-SM (CTA pair) GEMM tiles for bf16 at the 256-token cap (default on)."""
     lib().moe_set_cta_pairs(1 if enable else 0)
-
-
-def set_fp8_pairs(enable=True):
-    """FP8 decode weights on CTA pairs (2-SM MMAs; off by default)."""
-    lib().moe_set_fp8_pairs(1 if enable else 0)
 
 
 def set_shared_sms(n=0):

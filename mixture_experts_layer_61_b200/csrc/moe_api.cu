@@ -102,9 +102,14 @@ long long p_max(const moe_config_t* c) {
 
 struct Layout {
     size_t ctl, ctl_sh, logits, route_part, ids, w, counts, offsets, scalars, sorted_ids, block_expert, pos, x_perm,
-        act, act_sh, sh_out, x16;
+        act, act_sh, sh_out, x16, x_scale, y8, sh_scale;
     size_t total;
 };
+
+int routed_max_n(const moe_config_t* c);
+
+// FP8 expert weights run at decode sizes only (the fused expert FFN)
+bool fp8_sized(const moe_config_t* c) { return c->dtype == 0 && routed_max_n(c) <= 128; }
 
 Layout layout(const moe_config_t* c, int num_sms) {
     Layout L;
@@ -132,12 +137,20 @@ Layout layout(const moe_config_t* c, int num_sms) {
     L.sorted_ids = take(sizeof(int32_t) * (size_t)P);
     L.block_expert = take(sizeof(int32_t) * (size_t)((P + c->tile_B - 1) / c->tile_B));
     L.pos = take(sizeof(int32_t) * (size_t)A);
-    L.x_perm = take(eb * (size_t)P * c->H);  // also holds y_perm once x_perm is consumed
+    // also holds y_perm once x_perm is consumed; with FP8 weights the token rows'
+    // E4M3 hi and lo codes (the same 2 bytes an element)
+    L.x_perm = take(eb * (size_t)P * c->H);
     L.act = take(eb * (size_t)P * c->I);
     L.act_sh = take(I_sh > 0 ? eb * (size_t)c->T * I_sh : 0);
     L.sh_out = take(I_sh > 0 ? eb * (size_t)c->T * c->H : 0);
-    // x in f16 for the shared FFN on FP8 weights (bf16 layers only)
+    // the shared FFN on FP8 weights: x's E4M3 hi and lo codes and its row scales
     L.x16 = take(I_sh > 0 && c->dtype == 0 ? 2 * (size_t)c->T * c->H : 0);
+    L.sh_scale = take(I_sh > 0 && c->dtype == 0 ? sizeof(float) * (size_t)c->T : 0);
+    // the routed FFN on FP8 weights: the permuted rows' scales, and its
+    // outputs (x_perm holds the codes, which other chunks still read)
+    const bool f8 = fp8_sized(c);
+    L.x_scale = take(f8 ? sizeof(float) * (size_t)P : 0);
+    L.y8 = take(f8 ? eb * (size_t)P * c->H : 0);
     L.total = o;
     return L;
 }
@@ -203,7 +216,7 @@ GemmLaunch down_launch(const void* act, long long x_rows, const int32_t* seg_off
 int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_groups, int seg_rows, int H, int I,
             int dtype, const void* w13, const void* w2, void* act, void* y, int max_n, const GemmCtl& ctl,
             cudaStream_t s, long long max_chunks, int sms = 0, int ffn_sms = 0, const float* s13 = nullptr,
-            const float* s2 = nullptr) {
+            const float* s2 = nullptr, const float* x_scale = nullptr) {
     const bool fp8 = s13 != nullptr;  // w13 / w2 hold E4M3 codes with these row scales
     if (fp8 && max_n > 128) return -1;  // FP8 weights run on the fused (decode-size) kernel only
     if (max_n <= 128) {
@@ -226,6 +239,7 @@ int run_ffn(const void* x, long long x_rows, const int32_t* seg_offsets, int n_g
         f.fp8 = fp8;
         f.s13 = s13;
         f.s2 = s2;
+        f.x_scale = x_scale;
         int rc = launch_ffn_stream(f, ctl, s);
         if (rc != 1) return rc;  // 1: not handled, use two launches
         if (fp8) return -1;
@@ -311,9 +325,7 @@ void router_tiling(GemmLaunch& g, int T) {
     g.max_split = 8;
 }
 
-int routed_max_n(const moe_config_t* c) {
-    return pick_max_n((double)c->T * c->K / (double)c->E);
-}
+int routed_max_n(const moe_config_t* c) { return pick_max_n((double)c->T * c->K / (double)c->E); }
 
 // Upper bounds on the token chunks of the routed segments (every chunk holds
 // at least one 16-row unit) and of a dense segment of T rows.
@@ -457,25 +469,26 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_perm, const void* w13
                              routed_max_chunks(cfg)));
 }
 
-int moe_grouped_ffn_fp8(const moe_config_t* cfg, const void* x_perm, const uint8_t* w13_q, const float* w13_s,
-                        const uint8_t* w2_q, const float* w2_s, const int32_t* offsets, void* act, void* y_perm,
-                        void* workspace, size_t ws_bytes, moe_stream_t stream) {
+int moe_grouped_ffn_fp8(const moe_config_t* cfg, const uint8_t* x_codes, const float* x_scales,
+                        const uint8_t* w13_q, const float* w13_s, const uint8_t* w2_q, const float* w2_s,
+                        const int32_t* offsets, void* act, void* y_perm, void* workspace, size_t ws_bytes,
+                        moe_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->dtype != 0 || cfg->H % 16 || cfg->I % 16) return MOE_ERR_ARG;
     if (cfg->T == 0) return MOE_OK;
-    if (!x_perm || !w13_q || !w13_s || !w2_q || !w2_s || !offsets || !act || !y_perm || !workspace)
+    if (!x_codes || !x_scales || !w13_q || !w13_s || !w2_q || !w2_s || !offsets || !act || !y_perm || !workspace)
         return MOE_ERR_ARG;
-    if (!aligned16(x_perm) || !aligned16(w13_q) || !aligned16(w2_q) || !aligned16(act) || !aligned16(y_perm) ||
+    if (!aligned16(x_codes) || !aligned16(w13_q) || !aligned16(w2_q) || !aligned16(act) || !aligned16(y_perm) ||
         !aligned16(workspace))
         return MOE_ERR_ARG;
     if (routed_max_n(cfg) > 128) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
     if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
-    return status_of(run_ffn(x_perm, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13_q, w2_q, act,
+    return status_of(run_ffn(x_codes, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13_q, w2_q, act,
                              y_perm, routed_max_n(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream,
-                             routed_max_chunks(cfg), 0, 0, w13_s, w2_s));
+                             routed_max_chunks(cfg), 0, 0, w13_s, w2_s, x_scales));
 }
 
 int moe_grouped_gate_up(const moe_config_t* cfg, const void* x_perm, const void* w13, const int32_t* offsets,
@@ -626,9 +639,10 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
             ctl_sh.status = ctl.status + 1;  // the header's second status word
             void* sh_out = at<void>(workspace, L.sh_out);
             const void* x_sh = x;
-            if (fp8) {  // the FP8 path's token operand is f16
+            if (fp8) {  // the FP8 path's token operand: x split into E4M3 hi and lo codes
                 x_sh = at<void>(workspace, L.x16);
-                if ((rc = launch_bf16_to_f16((long long)cfg->T * cfg->H, x, at<void>(workspace, L.x16), sd.s)) != 0) {
+                if ((rc = launch_split_e4m3(cfg->H, 1, cfg->T, x, nullptr, nullptr, at<uint8_t>(workspace, L.x16),
+                                            cfg->T, at<float>(workspace, L.sh_scale), sd.s)) != 0) {
                     cudaEventRecord(sd.join, sd.s);
                     cudaStreamWaitEvent(s, sd.join, 0);
                     return status_of(rc);
@@ -637,7 +651,7 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
             rc = run_ffn(x_sh, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
                          at<void>(workspace, L.act_sh), sh_out, pick_max_n(cfg->T), ctl_sh, sd.s,
                          dense_max_chunks(cfg->T), n_sh, n_sh, fp8 ? fp8->s13_sh : nullptr,
-                         fp8 ? fp8->s2_sh : nullptr);
+                         fp8 ? fp8->s2_sh : nullptr, fp8 ? at<float>(workspace, L.sh_scale) : nullptr);
             if (cudaEventRecord(sd.join, sd.s) != cudaSuccess) {
                 cudaGetLastError();
                 return MOE_ERR_CUDA;
@@ -735,8 +749,16 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
                                pos, scalars, stats_out, s)) != 0)
             return status_of(rc);
     }
-    if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s, fp8 != nullptr)) != 0)
+    if (fp8) {
+        // the permuted token rows split into E4M3 hi and lo codes with their scales;
+        // the expert outputs get their own rows (other chunks still read the codes)
+        if ((rc = launch_split_e4m3(cfg->H, cfg->K, P, x, sorted_ids, scalars, static_cast<uint8_t*>(x_perm), P,
+                                    at<float>(workspace, L.x_scale), s)) != 0)
+            return status_of(rc);
+        y_perm = at<void>(workspace, L.y8);
+    } else if ((rc = launch_permute(cfg->H, cfg->K, cfg->dtype, P, x, sorted_ids, scalars, x_perm, s)) != 0) {
         return status_of(rc);
+    }
     if (front) {
         GemmLaunch g = gate_up_launch(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, act,
                                       routed_max_n(cfg));
@@ -744,7 +766,8 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
         if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
     } else if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
                              routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn,
-                             fp8 ? fp8->s13 : nullptr, fp8 ? fp8->s2 : nullptr)) != 0) {
+                             fp8 ? fp8->s13 : nullptr, fp8 ? fp8->s2 : nullptr,
+                             fp8 ? at<float>(workspace, L.x_scale) : nullptr)) != 0) {
         return status_of(rc);
     }
     if (I_sh > 0 && !side) {
@@ -752,13 +775,14 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
         const void* x_sh = x;
         if (fp8) {
             x_sh = at<void>(workspace, L.x16);
-            if ((rc = launch_bf16_to_f16((long long)cfg->T * cfg->H, x, at<void>(workspace, L.x16), s)) != 0)
+            if ((rc = launch_split_e4m3(cfg->H, 1, cfg->T, x, nullptr, nullptr, at<uint8_t>(workspace, L.x16), cfg->T,
+                                        at<float>(workspace, L.sh_scale), s)) != 0)
                 return status_of(rc);
         }
         if ((rc = run_ffn(x_sh, cfg->T, nullptr, 1, cfg->T, cfg->H, (int)I_sh, cfg->dtype, w13_shared, w2_shared,
                           at<void>(workspace, L.act_sh), sh_out, pick_max_n(cfg->T), ctl, s,
                           dense_max_chunks(cfg->T), 0, 0, fp8 ? fp8->s13_sh : nullptr,
-                          fp8 ? fp8->s2_sh : nullptr)) != 0)
+                          fp8 ? fp8->s2_sh : nullptr, fp8 ? at<float>(workspace, L.sh_scale) : nullptr)) != 0)
             return status_of(rc);
         sh = sh_out;
     }
@@ -905,31 +929,38 @@ int dense_ffn_fp8(int T, int H, int I, const void* x, const uint8_t* w13_q, cons
     if (rc != 0) return status_of(rc);
     const size_t ctl_bytes = align256(ctl_block_bytes(d.num_sms));
     const size_t act_bytes = align256((size_t)2 * T * I);
-    if (ws_bytes < ctl_bytes + act_bytes + (size_t)2 * T * H) return MOE_ERR_WORKSPACE;
+    const size_t code_bytes = align256((size_t)2 * T * H);
+    if (ws_bytes < ctl_bytes + act_bytes + code_bytes + sizeof(float) * (size_t)T) return MOE_ERR_WORKSPACE;
     void* act = at<void>(workspace, ctl_bytes);
-    void* x16 = at<void>(workspace, ctl_bytes + act_bytes);  // the FP8 path's token operand is f16
-    if ((rc = launch_bf16_to_f16((long long)T * H, x, x16, (cudaStream_t)stream)) != 0) return status_of(rc);
-    return status_of(run_ffn(x16, T, nullptr, 1, T, H, I, 0, w13_q, w2_q, act, out, pick_max_n(T),
+    // the token operand: x split into E4M3 hi and lo codes, and the rows' scales
+    uint8_t* codes = at<uint8_t>(workspace, ctl_bytes + act_bytes);
+    float* scales = at<float>(workspace, ctl_bytes + act_bytes + code_bytes);
+    if ((rc = launch_split_e4m3(H, 1, T, x, nullptr, nullptr, codes, T, scales, (cudaStream_t)stream)) != 0)
+        return status_of(rc);
+    return status_of(run_ffn(codes, T, nullptr, 1, T, H, I, 0, w13_q, w2_q, act, out, pick_max_n(T),
                              gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream, dense_max_chunks(T), 0, 0, w13_s,
-                             w2_s));
+                             w2_s, scales));
 }
 
 size_t dense_ffn_fp8_workspace_size(int T, int H, int I) {
     if (T < 0 || H <= 0 || I <= 0) return 0;
     DeviceInfo d;
     if (current_device(&d) != 0) return 0;
-    return align256(ctl_block_bytes(d.num_sms)) + align256((size_t)2 * T * I) + align256((size_t)2 * T * H);
+    return align256(ctl_block_bytes(d.num_sms)) + align256((size_t)2 * T * I) + align256((size_t)2 * T * H) +
+           sizeof(float) * (size_t)T;
 }
 
-int moe_permute_f16(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids, const int32_t* scalars,
-                    void* x_perm, moe_stream_t stream) {
+int moe_permute_e4m3x2(const moe_config_t* cfg, const void* x, const int32_t* sorted_ids, const int32_t* scalars,
+                       uint8_t* x_codes, float* x_scales, moe_stream_t stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (cfg->dtype != 0) return MOE_ERR_ARG;
     if (cfg->T == 0) return MOE_OK;
-    if (!x || !sorted_ids || !scalars || !x_perm || !aligned16(x) || !aligned16(x_perm)) return MOE_ERR_ARG;
-    return status_of(launch_permute(cfg->H, cfg->K, cfg->dtype, p_max(cfg), x, sorted_ids, scalars, x_perm,
-                                    (cudaStream_t)stream, true));
+    if (!x || !sorted_ids || !scalars || !x_codes || !x_scales || !aligned16(x) || !aligned16(x_codes))
+        return MOE_ERR_ARG;
+    const long long P = p_max(cfg);
+    return status_of(launch_split_e4m3(cfg->H, cfg->K, P, x, sorted_ids, scalars, x_codes, P, x_scales,
+                                       (cudaStream_t)stream));
 }
 
 int moe_quantize_fp8(int64_t rows, int cols, int dtype, const void* w, uint8_t* q, float* scales,
@@ -1016,8 +1047,6 @@ int moe_ffn_fused(const moe_config_t* cfg) {
 }
 
 void moe_set_cta_pairs(int enable) { set_cta_pairs(enable != 0); }
-
-void moe_set_fp8_pairs(int enable) { set_fp8_pairs(enable != 0); }
 
 void moe_debug_withhold_first_load(int enable) { g_withhold.store(enable ? 1 : 0); }
 

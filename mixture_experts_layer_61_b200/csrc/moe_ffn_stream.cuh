@@ -26,11 +26,23 @@
 // small shared-memory ring.
 //
 // FP8 weights (kFp8): the weight tiles stream as E4M3 codes (half the bytes),
-// 128 rows x 64 codes per tile with the 64-byte swizzle; warps 6..13 widen
-// each stage's two tiles to f16 in registers by moving the code's bits into an
-// f16 pattern (value x 2^-8, exact: E4M3 subnormals land on f16 subnormals)
-// and store them into a ring of TMEM buffers, from which the MMA takes its A
-// operand; the epilogue multiplies each output row by its fp32 row scale x 2^8.
+// 128 rows x 128 codes per tile with the 128-byte swizzle (the same 128-byte
+// row pieces as a bf16 tile: 64-code pieces left the weight stream at about
+// half the copy bandwidth).
+//  * gate/up: the token rows arrive split exactly into two E4M3 terms with a
+//    power-of-two scale per row (x = s (hi + lo)); each stage's MMAs are
+//    kind::f8f6f4 with both operands in shared memory -- weights x hi, then
+//    weights x lo into the same accumulator -- so no code is widened; the
+//    epilogue multiplies by the weight row's scale and the token row's s;
+//  * down: warps 6..13 widen each stage's two tiles to f16 in registers by
+//    moving the code's bits into an f16 pattern (value x 2^-8, exact: E4M3
+//    subnormals land on f16 subnormals) and store them into a ring of TMEM
+//    buffers, from which the f16 MMA takes its A operand (the activations are
+//    f16, two 64-column boxes per stage); the epilogue multiplies each output
+//    row by its fp32 row scale x 2^8.
+// Widening costs 4 bytes of tensor-memory traffic per weight byte (the f16
+// store and the MMA's read): at the gate/up projections, two thirds of the
+// bytes, the direct FP8 MMAs avoid it.
 // Widening through shared memory instead costs 6 bytes of shared-memory
 // traffic per weight (TMA write, read, f16 write, tensor-core read) against 2
 // for bf16 weights, which caps the stream below the bf16 rate; through TMEM
@@ -67,18 +79,23 @@ struct FfnParams {
     int max_slots_phase;  // partial slots available to each phase
     const float* s13;     // FP8 weights: row scales [n_groups * 2I] (gate rows, then up rows), else nullptr
     const float* s2;      // FP8 weights: row scales [n_groups * H], else nullptr
+    const float* x_scale; // FP8 weights: the token rows' power-of-two scales (phase A operand)
+    long long lo_rows;    // FP8 weights: rows from a token row's hi codes to its lo codes
 };
 
 template <typename T, int kMaxN, bool kFp8 = false>
 struct FfnCfg {
-    static constexpr int kBK = 128 / Elt<T>::kBytes;
-    static constexpr int kWTileBytes = 128 * 128;                        // a bf16 weight tile as the MMA reads it
-    static constexpr int kRawWBytes = kFp8 ? 128 * kBK : kWTileBytes;  // a weight tile as it streams in
+    // K per stage: 64 bf16 / fp32-as-tf32 elements, or 128 E4M3 codes; either
+    // way a weight tile is 128 rows of 128 bytes
+    static constexpr int kBK = kFp8 ? 128 : 128 / Elt<T>::kBytes;
+    static constexpr int kWTileBytes = 128 * 128;  // a weight tile as it streams in (and, bf16, as the MMA reads it)
+    static constexpr int kRawWBytes = kWTileBytes;
     static constexpr int kXBoxRows = 16, kXBoxMid = 64;
-    static constexpr int kXTileBytes = kMaxN * 128;
+    static constexpr int kXBoxes = kFp8 ? 2 : 1;   // 64-column f16 boxes of the token tile per stage (FP8: K 128)
+    static constexpr int kXTileBytes = kXBoxes * kMaxN * 128;
     static constexpr int kStageBytes = 2 * kRawWBytes + kXTileBytes;
-    static constexpr int kConv = kFp8 ? (kMaxN <= 64 ? 3 : 2) : 0;  // TMEM buffers of widened weights
-    static constexpr int kConvCols = 64;   // a stage's two 128 x 64 f16 tiles: 2 x 32 TMEM columns
+    static constexpr int kConv = kFp8 ? (kMaxN <= 32 ? 3 : 2) : 0;  // TMEM buffers of widened weights
+    static constexpr int kConvCols = 128;  // a stage's two 128 x 128 f16 tiles: 2 x 64 TMEM columns
     static constexpr int kConvThreads = kFp8 ? 256 : 0;   // converter warps 6..13
     static constexpr int kThreads = kFfnThreads + kConvThreads;
     static constexpr int kAccCols = 2 * kMaxN;
@@ -323,7 +340,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 const CUtensorMap* tx = it.phase == 0 ? &tm_xa : &tm_xb;
                 const CUtensorMap* tx64 = it.phase == 0 ? &tm_xa64 : &tm_xb64;
                 const int second = it.phase == 0 ? p.I : 128;  // up rows, or the next 128 features
-                const uint32_t bytes = 2 * C::kRawWBytes + t.mma_n * 128;
+                const uint32_t bytes = 2 * C::kRawWBytes + C::kXBoxes * t.mma_n * 128;
                 const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
                 auto load_w = [&](int s, int k) {
                     uint8_t* st = stage_base + s * C::kStageBytes;
@@ -332,13 +349,21 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                     tma_load_2d(st + C::kRawWBytes, tw, &full[s], kx, t.wrow + second, pol_w);
                 };
                 auto load_x = [&](int s, int k) {
-                    uint8_t* xs = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes;
-                    const int kx = k * C::kBK;
-                    int r = 0;
-                    if (kMaxN >= C::kXBoxMid)
-                        for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
-                            tma_load_2d(xs + r * 128, tx64, &full[s], kx, t.row0 + r, pol_x);
-                    for (; r < t.mma_n; r += C::kXBoxRows) tma_load_2d(xs + r * 128, tx, &full[s], kx, t.row0 + r, pol_x);
+#pragma unroll
+                    for (int xb = 0; xb < C::kXBoxes; ++xb) {
+                        uint8_t* xs = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes + xb * kMaxN * 128;
+                        // FP8 gate/up: box xb holds the hi (0) or lo (1) codes of columns
+                        // k*128..+127; otherwise 64 16-bit columns each
+                        const bool codes = kFp8 && it.phase == 0;
+                        const int kx = codes ? k * C::kBK : k * C::kBK + xb * 64;
+                        const int rbase = codes ? (int)(xb * p.lo_rows) : 0;
+                        int r = 0;
+                        if (kMaxN >= C::kXBoxMid)
+                            for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
+                                tma_load_2d(xs + r * 128, tx64, &full[s], kx, rbase + t.row0 + r, pol_x);
+                        for (; r < t.mma_n; r += C::kXBoxRows)
+                            tma_load_2d(xs + r * 128, tx, &full[s], kx, rbase + t.row0 + r, pol_x);
+                    }
                 };
                 int pre = 0;  // stages of this item whose weight tiles went out before the activation wait
                 if (it.phase == 1) {
@@ -404,6 +429,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
             uint32_t kc = 0, ac = 0, n = 0;
+            uint32_t cc = 0;  // FP8: stages widened so far (the conversion ring's own count)
             bool ok = true;
             while (true) {
                 const int rs = n % kFfnRing;
@@ -428,6 +454,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + b * C::kAccCols;
                 const uint32_t d1 = d0 + kMaxN;
+                // (FP8: f16 operands in phase B; in phase A E4M3 x E4M3, whose format
+                // code in the kind::f8f6f4 descriptor is also 0)
                 const uint32_t idesc = umma_idesc(kFp8 ? Elt<__half>::kMmaFmt : Elt<T>::kMmaFmt, 128, t.mma_n);
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
@@ -438,21 +466,41 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                     }
                     uint8_t* st = stage_base + s * C::kStageBytes;
                     const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
-                    int cv = 0;
-                    if constexpr (kFp8) {
+                    int cv = -1;
+                    if (kFp8 && it.phase == 0) {
+                        // E4M3 weights x the token rows' hi codes, then x their lo codes,
+                        // into the same accumulator: K 32 per MMA, four steps per stage
+                        tc_fence_after();
+                        const uint64_t a0 = umma_desc_sw128(smem_u32(st));
+                        const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
+#pragma unroll
+                        for (int part = 0; part < 2; ++part) {
+                            const uint64_t b = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes + part * kMaxN * 128));
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t acc = (k > it.kb || kk > 0 || part > 0) ? 1u : 0u;
+                                umma_e4m3(d0, a0 + 2 * kk, b + 2 * kk, idesc, acc);
+                                umma_e4m3(d1, a1 + 2 * kk, b + 2 * kk, idesc, acc);
+                            }
+                        }
+                    } else if constexpr (kFp8) {
                         // A: the stage's two tiles, widened to f16 in TMEM by the converter warps
-                        cv = (int)(kc % C::kConv);
-                        if (!mbar_wait_bounded(&conv_full[cv], (kc / C::kConv) & 1u, limit, abort_flag)) {
+                        cv = (int)(cc % C::kConv);
+                        if (!mbar_wait_bounded(&conv_full[cv], (cc / C::kConv) & 1u, limit, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t a0 = tmem_base + C::kConvCol0 + cv * C::kConvCols;
+                        // K 128 per stage: eight 16-deep steps, the token operand's
+                        // first four in its first 64-column box, the rest in the second
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
+                        for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
-                            umma_f16_tmem_a(d0, a0 + 8 * kk, bx + 2 * kk, idesc, acc);
-                            umma_f16_tmem_a(d1, a0 + 32 + 8 * kk, bx + 2 * kk, idesc, acc);
+                            const uint64_t b = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes + (kk >> 2) * kMaxN * 128)) +
+                                               2 * (kk & 3);
+                            umma_f16_tmem_a(d0, a0 + 8 * kk, b, idesc, acc);
+                            umma_f16_tmem_a(d1, a0 + 64 + 8 * kk, b, idesc, acc);
                         }
                     } else {
                         tc_fence_after();
@@ -466,7 +514,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         }
                     }
                     umma_commit(&empty[s]);
-                    if constexpr (kFp8) umma_commit(&conv_empty[cv]);
+                    if (cv >= 0) {  // FP8 down: the conversion buffer is free too
+                        umma_commit(&conv_empty[cv]);
+                        ++cc;
+                    }
                 }
                 if (!ok) break;
                 umma_commit(&tfull[b]);
@@ -483,15 +534,15 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         // ------------------------------------------- FP8 -> f16 converters
         // warps 6..9 widen a stage's first weight tile, warps 10..13 its second;
         // a warp may only store to its TMEM lane quadrant (warp mod 4), so each
-        // thread takes one row (quadrant x 32 + lane): its 64 codes are four
-        // 16-byte chunks, chunk c of row r at chunk position c ^ ((r / 2) mod 4)
-        // under the 64-byte swizzle (8 consecutive rows hit 8 distinct bank
-        // groups), widened to 32 f16 pairs and stored as 32 TMEM columns
+        // thread takes one row (quadrant x 32 + lane): its 128 codes are eight
+        // 16-byte chunks, chunk c of row r at chunk position c ^ (r mod 8) under
+        // the 128-byte swizzle (8 consecutive rows hit 8 distinct bank groups),
+        // widened to 64 f16 pairs and stored as 64 TMEM columns
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const int tt = (warp - 6) >> 2;
         const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        uint32_t kc = 0, n = 0;
+        uint32_t kc = 0, n = 0, cc = 0;  // stages, items, widened stages
         bool ok = true;
         while (ok) {
             const int rs = n % kFfnRing;
@@ -507,33 +558,41 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             FfnItem it;
             Tile t;
             item_of(id, it, t);
-            for (int k = it.kb; k < it.ke; ++k, ++kc) {
+            if (it.phase == 0) {  // gate/up stages use the codes as they are
+                kc += it.ke - it.kb;
+                continue;
+            }
+            for (int k = it.kb; k < it.ke; ++k, ++kc, ++cc) {
                 const int s = kc % C::kStages;
-                const int cv = (int)(kc % C::kConv);
+                const int cv = (int)(cc % C::kConv);
                 const bool got = mbar_wait_bounded(&full[s], (kc / C::kStages) & 1u, limit, abort_flag) &&
-                                 mbar_wait_bounded(&conv_empty[cv], ((kc / C::kConv) & 1u) ^ 1u, limit, abort_flag);
+                                 mbar_wait_bounded(&conv_empty[cv], ((cc / C::kConv) & 1u) ^ 1u, limit, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) {  // the whole warp leaves together (warp-wide TMEM stores)
                     ok = false;
                     break;
                 }
                 tc_fence_after();  // the MMAs that read this buffer before have completed
-                const uint8_t* src = stage_base + s * C::kStageBytes + tt * C::kRawWBytes + row * C::kBK;
-                uint32_t w[32];
+                const uint8_t* src = stage_base + s * C::kStageBytes + tt * C::kRawWBytes + row * 128;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(src + ((c ^ ((row >> 1) & 3)) << 4));
-                    uint4 lo, hi;
-                    e4m3x16_to_f16(v, lo, hi);
-                    w[8 * c + 0] = lo.x;
-                    w[8 * c + 1] = lo.y;
-                    w[8 * c + 2] = lo.z;
-                    w[8 * c + 3] = lo.w;
-                    w[8 * c + 4] = hi.x;
-                    w[8 * c + 5] = hi.y;
-                    w[8 * c + 6] = hi.z;
-                    w[8 * c + 7] = hi.w;
+                for (int h = 0; h < 2; ++h) {  // codes 64 h .. 64 h + 63 -> 32 columns
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int cc = 4 * h + c;
+                        const uint4 v = *reinterpret_cast<const uint4*>(src + ((cc ^ (row & 7)) << 4));
+                        uint4 lo, hi;
+                        e4m3x16_to_f16(v, lo, hi);
+                        w[8 * c + 0] = lo.x;
+                        w[8 * c + 1] = lo.y;
+                        w[8 * c + 2] = lo.z;
+                        w[8 * c + 3] = lo.w;
+                        w[8 * c + 4] = hi.x;
+                        w[8 * c + 5] = hi.y;
+                        w[8 * c + 6] = hi.z;
+                        w[8 * c + 7] = hi.w;
+                    }
+                    tmem_st32(tmem_base + lane_base + C::kConvCol0 + cv * C::kConvCols + tt * 64 + h * 32, w);
                 }
-                tmem_st32(tmem_base + lane_base + C::kConvCol0 + cv * C::kConvCols + tt * 32, w);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -586,10 +645,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             // times 2^8 (the widened codes hold value x 2^-8)
             float sc0 = 1.f, sc1 = 1.f;
             if constexpr (kFp8) {
-                if (gate_up) {
+                if (gate_up) {  // direct E4M3 products: no widening factor; the token scale per column below
                     const float* sr = p.s13 + (long long)t.group * 2 * p.I;
-                    sc0 = v0 ? __ldg(sr + f) * 256.f : 0.f;
-                    sc1 = v0 ? __ldg(sr + p.I + f) * 256.f : 0.f;
+                    sc0 = v0 ? __ldg(sr + f) : 0.f;
+                    sc1 = v0 ? __ldg(sr + p.I + f) : 0.f;
                 } else {
                     const float* sr = p.s2 + (long long)t.group * p.H;
                     sc0 = v0 ? __ldg(sr + f) * 256.f : 0.f;
@@ -600,8 +659,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 if constexpr (kFp8) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        g[i] *= sc0;
-                        u[i] *= sc1;
+                        // the token row's scale (phase A operand), read for real rows only
+                        const float xs = gate_up && c0 + i < t.nrows ? __ldg(p.x_scale + t.row0 + c0 + i) : 1.f;
+                        g[i] *= sc0 * xs;
+                        u[i] *= sc1 * xs;
                     }
                 }
                 if (gate_up) {

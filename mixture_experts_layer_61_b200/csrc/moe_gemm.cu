@@ -3,7 +3,6 @@
 // and the persistent launch.
 #include <mutex>
 
-#include "moe_ffn_pair.cuh"
 #include "moe_ffn_stream.cuh"
 #include "moe_gemm.cuh"
 #include "moe_internal.h"
@@ -205,10 +204,18 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
         if (!make_map(&w13, dt, eb, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128)) return -3;
         if (!make_map(&w2, dt, eb, L.w2, (long long)L.n_groups * L.H, L.I, 128)) return -3;
     }
-    // token operands: f16 on the FP8 path (x_perm and the activations), else the activation dtype
+    // token operands: on the FP8 path the gate/up operand is the rows' E4M3 hi
+    // and lo codes ([2 x_rows, H] bytes, 128-code boxes) and the activations are
+    // f16; otherwise both are in the activation dtype
     const CUtensorMapDataType xdt = kFp8 ? Elt<__half>::kTma : dt;
-    if (!make_map(&xa, xdt, eb, L.x, L.x_rows, L.H, 16)) return -3;
-    if (!make_map(&xa64, xdt, eb, L.x, L.x_rows, L.H, 64)) return -3;
+    if (kFp8) {
+        if (!L.x_scale) return -1;
+        if (!make_map(&xa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.x, 2 * L.x_rows, L.H, 16)) return -3;
+        if (!make_map(&xa64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.x, 2 * L.x_rows, L.H, 64)) return -3;
+    } else {
+        if (!make_map(&xa, xdt, eb, L.x, L.x_rows, L.H, 16)) return -3;
+        if (!make_map(&xa64, xdt, eb, L.x, L.x_rows, L.H, 64)) return -3;
+    }
     if (!make_map(&xb, xdt, eb, L.act, L.x_rows, L.I, 16)) return -3;
     if (!make_map(&xb64, xdt, eb, L.act, L.x_rows, L.I, 64)) return -3;
     FfnParams p;
@@ -227,6 +234,8 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     p.max_slots_phase = slots_total / 2;
     p.s13 = L.s13;
     p.s2 = L.s2;
+    p.x_scale = L.x_scale;
+    p.lo_rows = L.x_rows;
     const int grid = L.sms > 0 && L.sms < num_sms ? L.sms : num_sms;
     cudaError_t e = launch_kernel(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, w13, w2, xa, xa64,
                                   xb, xb64, p);
@@ -235,80 +244,7 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     return e == cudaSuccess ? 0 : -3;
 }
 
-bool g_fp8_pairs = false;  // FP8 decode weights on CTA pairs
-
-// The FP8 fused FFN on CTA pairs (moe_ffn_pair.cuh).  Returns 1 when the
-// item space does not fit its counters (the caller takes the single-CTA kernel).
-template <int kMaxN>
-int launch_ffn_pair_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cudaStream_t stream) {
-    using C = FfnPairCfg<kMaxN>;
-    auto kern = moe_ffn_fp8_pair_kernel<kMaxN>;
-    static int max_blocks = 0;  // CTAs of whole pairs that can be resident at once
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) {
-            cudaGetLastError();
-            return -3;
-        }
-        cudaLaunchConfig_t oc = {};
-        oc.gridDim = dim3(num_sms);
-        oc.blockDim = dim3(C::kThreads);
-        oc.dynamicSmemBytes = C::kSmemBytes;
-        cudaLaunchAttribute ca;
-        ca.id = cudaLaunchAttributeClusterDimension;
-        ca.val.clusterDim.x = 2;
-        ca.val.clusterDim.y = 1;
-        ca.val.clusterDim.z = 1;
-        oc.attrs = &ca;
-        oc.numAttrs = 1;
-        int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &oc) != cudaSuccess || nclusters <= 0) {
-            cudaGetLastError();
-            return -3;
-        }
-        max_blocks = 2 * nclusters < num_sms ? 2 * nclusters : num_sms & ~1;
-        attr_done = true;
-    }
-    int grid = max_blocks;
-    if (L.sms > 0 && L.sms < grid) grid = L.sms >= 4 ? L.sms & ~1 : 2;
-    const long long G = grid / 2;
-    // split-tile counters: 2 per tile (one per CTA half) within each phase's half of the array
-    const long long ta = L.max_chunks * ((L.I + 255) / 256), tb = L.max_chunks * ((L.H + 511) / 512);
-    if ((ta < 2 * G && 2 * ta > kFfnTileCtrs / 2) || (tb < 2 * G && 2 * tb > kFfnTileCtrs / 2)) return 1;
-    const int slots_total = (int)((kSlotBytesMax * 2 * (size_t)num_sms) / ((size_t)C::kSlotFloats * 4));
-    CUtensorMap w13, w2, xa, xb;
-    if (!make_map(&w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w13, (long long)L.n_groups * 2 * L.I, L.H, 128, C::kBK))
-        return -3;
-    if (!make_map(&w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.w2, (long long)L.n_groups * L.H, L.I, 128, C::kBK))
-        return -3;
-    if (!make_map(&xa, Elt<__half>::kTma, 2, L.x, L.x_rows, L.H, 16)) return -3;
-    if (!make_map(&xb, Elt<__half>::kTma, 2, L.act, L.x_rows, L.I, 16)) return -3;
-    FfnParams p;
-    p.seg_offsets = L.seg_offsets;
-    p.n_groups = L.n_groups;
-    p.seg_rows = L.seg_rows;
-    p.H = L.H;
-    p.I = L.I;
-    p.act = L.act;
-    p.y = L.y;
-    p.ctl = ctl.ffn_ctl;
-    p.partials = ctl.partials;
-    p.status = ctl.status;
-    p.wait_limit_ns = wait_limit_ns();
-    p.withhold_first_load = take_withhold_flag();  // not used by the pair kernel
-    p.max_slots_phase = slots_total / 2;
-    p.s13 = L.s13;
-    p.s2 = L.s2;
-    cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, 2, w13, w2, xa,
-                                          xb, p);
-    count_launch();
-    if (e != cudaSuccess) cudaGetLastError();
-    return e == cudaSuccess ? 0 : -3;
-}
-
 }  // namespace
-
-void set_fp8_pairs(bool on) { g_fp8_pairs = on; }
 
 int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t stream) {
     DeviceInfo d;
@@ -325,12 +261,6 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
     if (L.x_rows <= 0) return 0;
     if (L.fp8) {
         if (L.dtype != 0 || !L.s13 || !L.s2) return -1;
-        if (g_fp8_pairs && d.num_sms % 2 == 0 && L.H % 64 == 0 && L.I % 64 == 0) {
-            int rc = L.max_n == 32   ? launch_ffn_pair_variant<32>(L, ctl, d.num_sms, stream)
-                     : L.max_n == 64 ? launch_ffn_pair_variant<64>(L, ctl, d.num_sms, stream)
-                                     : launch_ffn_pair_variant<128>(L, ctl, d.num_sms, stream);
-            if (rc != 1) return rc;  // 1: its counters do not fit, the single-CTA kernel below
-        }
         if (L.max_n == 32) return launch_ffn_variant<__nv_bfloat16, 32, true>(L, ctl, d.num_sms, stream);
         if (L.max_n == 64) return launch_ffn_variant<__nv_bfloat16, 64, true>(L, ctl, d.num_sms, stream);
         return launch_ffn_variant<__nv_bfloat16, 128, true>(L, ctl, d.num_sms, stream);

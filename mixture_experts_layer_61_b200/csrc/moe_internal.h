@@ -127,6 +127,9 @@ struct FfnLaunch {
     bool fp8 = false;      // w13 / w2 are E4M3 codes with fp32 row scales s13 [n_groups*2I], s2 [n_groups*H]
     const float* s13 = nullptr;
     const float* s2 = nullptr;
+    // FP8 weights: x holds the token rows' E4M3 hi codes [x_rows, H], then their
+    // lo codes [x_rows, H]; x_scale [x_rows] their power-of-two scales
+    const float* x_scale = nullptr;
 };
 int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t stream);
 
@@ -141,8 +144,6 @@ void set_split_tail(int mode);
 int split_tail_mode();
 // CTA-pair (2-SM MMA) tiles for bf16 launches at the 256-token cap (default on).
 void set_cta_pairs(bool on);
-// The fused FFN with FP8 weights on CTA pairs (default off).
-void set_fp8_pairs(bool on);
 
 // Elementwise / routing kernels.
 // k_per_token (nullable): per-token expert count, clamped to [0, K]; slots
@@ -162,11 +163,13 @@ int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int
                        const int32_t* k_per_token, float* part, float* logits, int32_t* ids, float* w,
                        int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos,
                        int32_t* scalars, int32_t* stats_copy, int* done_ctr, cudaStream_t stream);
-// to_f16: bf16 x written to x_perm as f16 (the FP8-weight path's operand type)
 int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
-                   const int32_t* scalars, void* x_perm, cudaStream_t stream, bool to_f16 = false);
-// n bf16 values -> f16 (n a multiple of 8)
-int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stream);
+                   const int32_t* scalars, void* x_perm, cudaStream_t stream);
+// The exact two-term E4M3 split of bf16 rows [rows, H] (gathered by
+// sorted_ids with the count in scalars[0] when sorted_ids is given): codes
+// [rows, H] hi then, lo_rows rows on, lo; power-of-two scales [rows].
+int launch_split_e4m3(int H, int K, long long rows, const void* x, const int32_t* sorted_ids, const int32_t* scalars,
+                      uint8_t* codes, long long lo_rows, float* scales, cudaStream_t stream);
 // col0 / ncols (elements, multiples of 16 bytes): only those columns, into
 // rows of ncols; ncols < 0: all H columns
 int launch_combine(int T, int H, int K, int dtype, const void* y_perm, const int32_t* pos, const float* w,

@@ -871,17 +871,6 @@ int launch_align(int T, int K, int E, int B, int mode, long long P_max, const in
 
 // ---------------------------------------------------------------- permute
 // x_perm[p] = x[sorted_ids[p] / K] (zero row for a padding slot), p < P.
-// 8 bf16 -> 8 f16 (the FP8-weight path computes on f16 operands)
-__device__ __forceinline__ int4 bf16x8_to_f16x8(int4 v) {
-    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
-    int4 o;
-    __half2* h = reinterpret_cast<__half2*>(&o);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(__bfloat1622float2(b[i]));
-    return o;
-}
-
-template <bool kToF16>
 __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const int4* __restrict__ x,
                                                       const int32_t* __restrict__ sorted_ids,
                                                       const int32_t* __restrict__ scalars, int4* __restrict__ x_perm) {
@@ -895,7 +884,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const 
         int4* dst = x_perm + p * row_vec;
         if (src >= 0) {
             const int4* s = x + (long long)(src / K) * row_vec;
-            for (int v = l; v < row_vec; v += 64) dst[v] = kToF16 ? bf16x8_to_f16x8(__ldg(s + v)) : __ldg(s + v);
+            for (int v = l; v < row_vec; v += 64) dst[v] = __ldg(s + v);
         } else {
             const int4 z = make_int4(0, 0, 0, 0);
             for (int v = l; v < row_vec; v += 64) dst[v] = z;
@@ -904,7 +893,7 @@ __global__ void __launch_bounds__(256) permute_kernel(int row_vec, int K, const 
 }
 
 int launch_permute(int H, int K, int dtype, long long P_max, const void* x, const int32_t* sorted_ids,
-                   const int32_t* scalars, void* x_perm, cudaStream_t stream, bool to_f16) {
+                   const int32_t* scalars, void* x_perm, cudaStream_t stream) {
     if (P_max <= 0) return 0;
     DeviceInfo d;
     int rc = current_device(&d);
@@ -915,34 +904,111 @@ int launch_permute(int H, int K, int dtype, long long P_max, const void* x, cons
     long long blocks = (P_max + rows_per_block - 1) / rows_per_block;
     const long long cap = (long long)d.num_sms * 8;
     if (blocks > cap) blocks = cap;
-    if (to_f16 && dtype != 0) return -1;
-    cudaError_t e = to_f16 ? launch_kernel(permute_kernel<true>, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
-                                           static_cast<const int4*>(x), sorted_ids, scalars,
-                                           static_cast<int4*>(x_perm))
-                           : launch_kernel(permute_kernel<false>, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
-                                           static_cast<const int4*>(x), sorted_ids, scalars,
-                                           static_cast<int4*>(x_perm));
+    cudaError_t e = launch_kernel(permute_kernel, dim3((int)blocks), dim3(256), 0, stream, row_vec, K,
+                                  static_cast<const int4*>(x), sorted_ids, scalars, static_cast<int4*>(x_perm));
     count_launch();
     return launched(e);
 }
 
-// bf16 rows -> f16 rows (n_vec vectors of 8), for the shared FFN on FP8 weights
-__global__ void __launch_bounds__(256) bf16_to_f16_kernel(long long n_vec, const int4* __restrict__ in,
-                                                          int4* __restrict__ out) {
-    pdl_launch_dependents();
-    pdl_wait();
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += (long long)gridDim.x * blockDim.x)
-        out[i] = bf16x8_to_f16x8(__ldg(in + i));
+// Exact two-term E4M3 split of bf16 token rows, the token operand of the FP8
+// gate/up MMAs: with s the smallest power of two for which max |x| <= 448 s,
+// x / s is exact, hi = E4M3(x / s) keeps its leading four significant bits,
+// and the rest r = x / s - hi (exact in fp32; at most four significant bits
+// for the eight of a bf16 value) is lo = E4M3(r), so x = s (hi + lo) except
+// where r falls below the E4M3 subnormal grid (2^-9, i.e. below 2^-17 of the
+// row's largest value).  One warp per row; rows gathered by sorted_ids
+// (padding slots: zero codes, scale 1) or taken in order.  codes holds the hi
+// rows, then, lo_rows rows further on, the lo rows.
+__device__ __forceinline__ uint8_t e4m3_rn(float v) { return __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3); }
+__device__ __forceinline__ float e4m3_value(uint8_t c) {
+    __nv_fp8_e4m3 f;
+    f.__x = c;
+    return static_cast<float>(f);
 }
 
-int launch_bf16_to_f16(long long n, const void* in, void* out, cudaStream_t stream) {
-    if (n <= 0) return 0;
-    if (n % 8) return -1;
-    const long long n_vec = n / 8;
-    long long blocks = (n_vec + 255) / 256;
-    if (blocks > 4096) blocks = 4096;
-    cudaError_t e = launch_kernel(bf16_to_f16_kernel, dim3((int)blocks), dim3(256), 0, stream, n_vec,
-                                  static_cast<const int4*>(in), static_cast<int4*>(out));
+template <bool kGather>
+__global__ void __launch_bounds__(256) split_e4m3_kernel(int H, int K, long long rows, const int4* __restrict__ x,
+                                                         const int32_t* __restrict__ sorted_ids,
+                                                         const int32_t* __restrict__ scalars, uint8_t* __restrict__ codes,
+                                                         long long lo_rows, float* __restrict__ scales) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nv = H / 8;  // 16-byte vectors of 8 bf16 per row
+    const long long n = kGather ? (long long)scalars[0] : rows;
+    for (long long p = (long long)blockIdx.x * 8 + warp; p < n; p += (long long)gridDim.x * 8) {
+        const int4* src = nullptr;
+        if (kGather) {
+            const int a = sorted_ids[p];
+            if (a >= 0) src = x + (long long)(a / K) * nv;
+        } else {
+            src = x + p * nv;
+        }
+        uint2* hi = reinterpret_cast<uint2*>(codes + p * H);
+        uint2* lo = reinterpret_cast<uint2*>(codes + (lo_rows + p) * H);
+        if (!src) {
+            for (int v = lane; v < nv; v += 32) hi[v] = lo[v] = make_uint2(0u, 0u);
+            if (lane == 0) scales[p] = 1.f;
+            continue;
+        }
+        float amax = 0.f;
+        for (int v = lane; v < nv; v += 32) {
+            const int4 q = __ldg(src + v);
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        // the smallest power of two s with amax <= 448 s (products with 448 s are exact)
+        float sc = 1.f;
+        if (amax > 0.f) {
+            int e;
+            frexpf(amax / 448.f, &e);
+            sc = ldexpf(1.f, e);
+            while (amax > 448.f * sc) sc *= 2.f;
+            while (amax <= 224.f * sc) sc *= 0.5f;
+        }
+        const float inv = 1.f / sc;  // a power of two: exact
+        for (int v = lane; v < nv; v += 32) {
+            const int4 q = __ldg(src + v);
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+            uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                const float y0 = f.x * inv, y1 = f.y * inv;
+                const uint8_t h0 = e4m3_rn(y0), h1 = e4m3_rn(y1);
+                const uint8_t l0 = e4m3_rn(y0 - e4m3_value(h0)), l1 = e4m3_rn(y1 - e4m3_value(h1));
+                const int sh = 16 * (i & 1);
+                hw[i >> 1] |= ((uint32_t)h0 | ((uint32_t)h1 << 8)) << sh;
+                lw[i >> 1] |= ((uint32_t)l0 | ((uint32_t)l1 << 8)) << sh;
+            }
+            hi[v] = make_uint2(hw[0], hw[1]);
+            lo[v] = make_uint2(lw[0], lw[1]);
+        }
+        if (lane == 0) scales[p] = sc;
+    }
+}
+
+int launch_split_e4m3(int H, int K, long long rows, const void* x, const int32_t* sorted_ids, const int32_t* scalars,
+                      uint8_t* codes, long long lo_rows, float* scales, cudaStream_t stream) {
+    if (rows <= 0) return 0;
+    if (H % 8) return -1;
+    DeviceInfo d;
+    int rc = current_device(&d);
+    if (rc != 0) return rc;
+    long long blocks = (rows + 7) / 8;
+    const long long cap = (long long)d.num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    cudaError_t e = sorted_ids
+                        ? launch_kernel(split_e4m3_kernel<true>, dim3((int)blocks), dim3(256), 0, stream, H, K, rows,
+                                        static_cast<const int4*>(x), sorted_ids, scalars, codes, lo_rows, scales)
+                        : launch_kernel(split_e4m3_kernel<false>, dim3((int)blocks), dim3(256), 0, stream, H, K, rows,
+                                        static_cast<const int4*>(x), sorted_ids, scalars, codes, lo_rows, scales);
     count_launch();
     return launched(e);
 }

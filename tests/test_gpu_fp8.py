@@ -1,8 +1,9 @@
 """FP8 expert weights on the GPU against the oracle: the row quantiser's
-codes and scales bit-exact, and the layer with FP8 routed and shared weights
-(the fused decode FFN widening E4M3 codes to f16 in tensor memory, f16 MMAs)
-within the output bound of the bf16 layer, against the oracle's layer
-computed on the same codes and scales."""
+codes and scales bit-exact, the token rows' exact E4M3 hi/lo split checked
+against the format's definition, and the layer with FP8 routed and shared
+weights (the fused decode FFN: E4M3 x E4M3 gate/up products, down products on
+codes widened to f16 in tensor memory) within the output bound of the bf16
+layer, against the oracle's layer computed on the same codes and scales."""
 import numpy as np
 import pytest
 import torch
@@ -83,7 +84,7 @@ def test_fp8_layer_ragged_and_dynamic_k():
 
 
 @pytest.mark.parametrize("name,T", [("mixtral", 32), ("qwen2moe", 32), ("deepseekv3", 32), ("mixtral", 256),
-                                    ("qwen2moe", 128), ("deepseekv3", 128)])
+                                    ("qwen2moe", 128), ("deepseekv3", 128), ("mixtral", 1)])
 def test_fp8_layer_full_size_sampled(name, T):
     # every token up to 256 (the FP8 path runs decode sizes: at most 128 rows
     # per routed expert, and T <= 128 with shared experts)
@@ -131,3 +132,61 @@ def test_fp8_subnormal_codes_are_kept():
                                logits=np.zeros((T, 1), np.float32))
     assert np.abs(ref).max() > 0
     assert rel_err(out.float().cpu().numpy(), ref) < OUT_TOL
+
+
+# ------------------------------------------------ the token rows' E4M3 split
+def _e4m3_values():
+    """All 256 E4M3 code values from the format's definition (OCP FP8: sign,
+    4-bit exponent with bias 7, 3-bit mantissa, subnormals at exponent 0,
+    S.1111.111 NaN, no infinities)."""
+    v = np.empty(256)
+    for c in range(256):
+        e, m = (c >> 3) & 15, c & 7
+        mag = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        v[c] = np.nan if (e == 15 and m == 7) else (-mag if c & 0x80 else mag)
+    return v
+
+
+def test_permute_e4m3x2_is_an_exact_split():
+    # x[sorted_ids[p] / K] = s_p (hi_p + lo_p): s_p the smallest power of two
+    # with max|row| <= 448 s_p, hi the nearest E4M3 value of row / s_p, and the
+    # remainder exact wherever |row / s_p| >= 1/4 (its quantum is then on the
+    # E4M3 grid), else within half the smallest subnormal
+    shape = small_shape(H=272, E=8, K=2, I=208)
+    T = 40
+    cfg = cfg_for(shape, T)
+    Pm = moe.padded_rows_max(cfg)
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((T, shape.H)) * np.logspace(-30, 30, T)[:, None]
+    x[3] = 0.0                                           # an all-zero row
+    x[4, :4] = [448.0, -1e-30, 3e-3, -0.0]
+    x_d = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    P = Pm - 3                                           # rows past P are left alone
+    sid = np.full(Pm, -7, np.int32)
+    sid[:P] = rng.permutation(np.concatenate([np.arange(T * shape.K), -np.ones(P, int)]))[:P]
+    scalars = torch.tensor([P, 0, 0, 0], dtype=torch.int32, device="cuda")
+    codes, scales = moe.permute_e4m3x2(cfg, x_d, torch.from_numpy(sid).cuda(), scalars)
+    torch.cuda.synchronize()
+    codes, scales = codes.cpu().numpy(), scales.cpu().numpy().astype(np.float64)
+    val = _e4m3_values()
+    finite = val[~np.isnan(val)]
+    xb = x_d.float().cpu().numpy().astype(np.float64)
+    for p in range(P):
+        hi, lo = val[codes[p]], val[codes[Pm + p]]
+        if sid[p] < 0:
+            assert not codes[p].any() and not codes[Pm + p].any() and scales[p] == 1.0
+            continue
+        row, s = xb[sid[p] // shape.K], scales[p]
+        assert np.frexp(s)[0] == 0.5                     # a power of two
+        amax = np.abs(row).max()
+        if amax == 0:
+            assert s == 1.0 and not np.any(hi) and not np.any(lo)
+            continue
+        assert amax <= 448 * s and amax > 224 * s
+        y = row / s
+        assert not np.isnan(hi).any() and not np.isnan(lo).any()
+        nearest = np.abs(finite[None, :] - y[:, None]).min(axis=1)
+        assert np.array_equal(np.abs(y - hi), nearest)
+        err = np.abs(y - (hi + lo))
+        assert np.all(err[np.abs(y) >= 0.25] == 0)
+        assert np.all(err <= 2.0 ** -10)
