@@ -343,23 +343,10 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[1
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 lanes x 32 bits, 32 consecutive columns per thread (thread i -> lane
-// base + i); complete with tmem_wait_st before the columns are read.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // kind::f8f6f4 MMA, both operands in shared memory (K-major, 128-byte
 // swizzle), 32 K per instruction; the formats are in the instruction
-// descriptor (E4M3 = 0).
+// descriptor (kFmtE4M3 for both).
+constexpr uint32_t kFmtE4M3 = 0;
 __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
@@ -369,19 +356,56 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
-// kind::f16 MMA with the A operand in tensor memory: A's M = 128 rows in
-// lanes 0..127, K packed two 16-bit values per 32-bit column (the lower K
-// index in the low half), so a K step of 16 spans 8 columns.
-__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
 
 // Named barrier among `nthreads` threads (whole warps) on barrier id `id`.
+// The smallest power of two s >= 2^-126 with amax <= 448 s (1 for amax = 0):
+// the scale of a row split into E4M3 terms, x = s (hi + lo) -- x / s is exact
+// and within E4M3's range; the lower bound keeps 1 / s finite.  Returned as
+// its exponent k (s = 2^k).  For a normal amax = (1 + f) 2^E, 448 = 1.75 x 2^8
+// gives k = E - 8 when 1 + f <= 1.75 (f's 23-bit field <= 0x600000) and
+// E - 7 otherwise; a subnormal amax takes the bound.
+__device__ __forceinline__ int e4m3_pow2_exp(float amax) {
+    const uint32_t u = __float_as_uint(amax) & 0x7FFFFFFFu;
+    if (u == 0u) return 0;
+    const int e = (int)(u >> 23) - 127;
+    int k = e - 8 + ((u & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    if ((u >> 23) == 0u || k < -126) k = -126;
+    return k;
+}
+__device__ __forceinline__ float pow2f_exact(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+__device__ __forceinline__ float e4m3_pow2_scale(float amax) { return pow2f_exact(e4m3_pow2_exp(amax)); }
+__device__ __forceinline__ float e4m3_pow2_inv_scale(float amax) { return pow2f_exact(-e4m3_pow2_exp(amax)); }
+
+// Untiled bulk copy global -> shared, completing on `bar` (16-byte aligned
+// addresses, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Generic-proxy writes to shared memory made visible to the tensor core's
+// (async proxy) reads that follow.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Named barrier over nthreads that also returns whether v held in all of them.
+__device__ __forceinline__ bool named_all(int id, int nthreads, bool v) {
+    __syncwarp();
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

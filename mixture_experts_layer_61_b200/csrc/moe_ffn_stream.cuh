@@ -27,28 +27,26 @@
 //
 // FP8 weights (kFp8): the weight tiles stream as E4M3 codes (half the bytes),
 // 128 rows x 128 codes per tile with the 128-byte swizzle (the same 128-byte
-// row pieces as a bf16 tile: 64-code pieces left the weight stream at about
-// half the copy bandwidth).
-//  * gate/up: the token rows arrive split exactly into two E4M3 terms with a
-//    power-of-two scale per row (x = s (hi + lo)); each stage's MMAs are
-//    kind::f8f6f4 with both operands in shared memory -- weights x hi, then
-//    weights x lo into the same accumulator -- so no code is widened; the
-//    epilogue multiplies by the weight row's scale and the token row's s;
-//  * down: warps 6..13 widen each stage's two tiles to f16 in registers by
-//    moving the code's bits into an f16 pattern (value x 2^-8, exact: E4M3
-//    subnormals land on f16 subnormals) and store them into a ring of TMEM
-//    buffers, from which the f16 MMA takes its A operand (the activations are
-//    f16, two 64-column boxes per stage); the epilogue multiplies each output
-//    row by its fp32 row scale x 2^8.
-// Widening costs 4 bytes of tensor-memory traffic per weight byte (the f16
-// store and the MMA's read): at the gate/up projections, two thirds of the
-// bytes, the direct FP8 MMAs avoid it.
-// Widening through shared memory instead costs 6 bytes of shared-memory
-// traffic per weight (TMA write, read, f16 write, tensor-core read) against 2
-// for bf16 weights, which caps the stream below the bf16 rate; through TMEM
-// the shared-memory traffic stays at 2 bytes per weight.
-// The MMAs run on f16 operands: x_perm arrives in f16 and the SwiGLU
-// activations are stored in f16 (the output stays in the activation dtype).
+// row pieces as a bf16 tile), and every MMA is kind::f8f6f4 with both
+// operands E4M3 in shared memory (K 32 per instruction), fp32 accumulation.
+// The token operand is split exactly into two E4M3 terms with a power-of-two
+// scale per row, x = s (hi + lo), and each stage runs weights x hi, then
+// weights x lo, into the same accumulator; the epilogue multiplies by the
+// weight row's fp32 scale and the token row's s.
+//  * gate/up: the token rows arrive split (hi codes, then lo codes lo_rows
+//    rows further on, and their scales x_scale);
+//  * down: phase A stores the SwiGLU activations in f16 and raises, per token
+//    row, the maximum |activation| (atomicMax on the fp32 bits) before its
+//    chunk counter; a phase-B item's first stage brings those maxima along
+//    (bulk copy on the stage's barrier), and warps 6..13 split each stage's
+//    f16 activation tile in place into hi and lo E4M3 codes (row scale from
+//    the maximum) before the MMA thread issues.  The split keeps about 8
+//    significant bits of each activation (bf16's precision); the weights
+//    meet no rounding at all.
+// Widening the weight codes instead (to f16, in tensor memory, for kind::f16
+// MMAs) cost 4 bytes of tensor-memory traffic per weight byte and ran at half
+// the copy bandwidth; splitting the token operand touches kMaxN x 128 values
+// per stage against 32 K weights.
 #pragma once
 
 #include <type_traits>
@@ -60,9 +58,13 @@ namespace moe {
 constexpr int kFfnMaxChunks = 4096;   // token chunks (per-chunk phase-A counters)
 constexpr int kFfnTileCtrs = 4096;    // split-tile counters (phase A, then phase B)
 constexpr int kFfnRing = 4;
+constexpr int kFfnMaxRows = 1 << 17;  // token rows of an FP8 launch (per-row activation maxima)
 // control ints: [0] work counter, [1] finished blocks, [2, 2+kFfnMaxChunks) chunk
-// counters, then kFfnTileCtrs tile counters
-constexpr int kFfnCtlInts = 2 + kFfnMaxChunks + kFfnTileCtrs;
+// counters, then kFfnTileCtrs tile counters, then (16-byte aligned, for the
+// bulk copies) the FP8 path's per-row activation maxima (fp32 bits) with a
+// margin for the copies' rounding to 16 bytes
+constexpr int kFfnAmaxOff = (2 + kFfnMaxChunks + kFfnTileCtrs + 63) / 64 * 64;
+constexpr int kFfnCtlInts = kFfnAmaxOff + kFfnMaxRows + 256;
 
 struct FfnParams {
     const int32_t* seg_offsets;  // [n_groups + 1] row offsets, or nullptr: one group [0, seg_rows)
@@ -71,7 +73,7 @@ struct FfnParams {
     int H, I;
     void* act;           // [rows, I] SwiGLU activations (written in phase A, read in phase B)
     void* y;             // [rows, H] output
-    int* ctl;            // kFfnCtlInts, zero on entry, left zero
+    int* ctl;            // kFfnCtlInts, zero on entry, left zero (ctl 16-byte aligned)
     float* partials;     // split-tile partial slots (up to 8 x gridDim.x)
     unsigned* status;
     uint64_t wait_limit_ns;
@@ -91,31 +93,49 @@ struct FfnCfg {
     static constexpr int kWTileBytes = 128 * 128;  // a weight tile as it streams in (and, bf16, as the MMA reads it)
     static constexpr int kRawWBytes = kWTileBytes;
     static constexpr int kXBoxRows = 16, kXBoxMid = 64;
-    static constexpr int kXBoxes = kFp8 ? 2 : 1;   // 64-column f16 boxes of the token tile per stage (FP8: K 128)
+    // 128-byte rows of the token tile per stage: one box of 64 16-bit columns,
+    // or (FP8) two: the hi and lo codes of 128 columns (phase B: the two f16
+    // boxes of 64 activation columns, split in place into hi and lo codes)
+    static constexpr int kXBoxes = kFp8 ? 2 : 1;
     static constexpr int kXTileBytes = kXBoxes * kMaxN * 128;
     static constexpr int kStageBytes = 2 * kRawWBytes + kXTileBytes;
-    static constexpr int kConv = kFp8 ? (kMaxN <= 32 ? 3 : 2) : 0;  // TMEM buffers of widened weights
-    static constexpr int kConvCols = 128;  // a stage's two 128 x 128 f16 tiles: 2 x 64 TMEM columns
-    static constexpr int kConvThreads = kFp8 ? 256 : 0;   // converter warps 6..13
-    static constexpr int kThreads = kFfnThreads + kConvThreads;
-    static constexpr int kAccCols = 2 * kMaxN;
-    static constexpr int kNumAcc = (kFp8 && kMaxN == 128) ? 1 : 2;  // leaves TMEM room for the weight buffers
-    static constexpr int kConvCol0 = kNumAcc * kAccCols;
+    static constexpr int kSplitThreads = kFp8 ? 256 : 0;  // activation splitters, warps 6..13
+    static constexpr int kUnits = kMaxN * 8 / 256;         // (row, 16 columns) units per splitter per stage
+    // per stage: the activation maxima of a phase-B item's rows (first stage
+    // only), fetched 16-byte aligned: up to 3 rows before the item's first
+    static constexpr int kSideBytes = kFp8 ? (kMaxN + 8) * 4 : 0;
+    static constexpr int kThreads = kFfnThreads + kSplitThreads;
+    // FP8 with tiles of at most 64 token rows: the hi and lo rows sit one after
+    // the other in the stage (lo at row mma_n) and one MMA with N = 2 mma_n
+    // covers both -- the per-MMA cost is flat up to N = 64 and at the tensor
+    // rate beyond, so this halves the MMAs of a stage; each accumulator then
+    // holds the hi and lo products side by side (2 kMaxN columns each), which
+    // the epilogue adds.  128-row tiles keep two MMAs into one accumulator
+    // (TMEM holds two 2 x 256-column buffers only that way).
+    static constexpr bool kStack = kFp8 && kMaxN <= 64;
+    static constexpr int kUOff = kStack ? 2 * kMaxN : kMaxN;  // the up (or second) accumulator's first column
+    static constexpr int kAccCols = 2 * kUOff;
+    static constexpr int kNumAcc = 2;
+    // FP8: per stage, a barrier on which phase-B fills complete (their own
+    // phases, so the splitters, which skip phase-A stages, wait on exact
+    // phases) and one for the split tile being ready (at most 8 stages)
+    static constexpr int kXReady = kFp8 ? 8 : 0;
     static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
     static constexpr int kMiscBytes = 768;
     static constexpr int kBudget = 227 * 1024 - 1024 - kTableBytes - kMiscBytes;
-    static constexpr int kStagesRaw = kBudget / kStageBytes;
+    static constexpr int kStagesRaw = kBudget / (kStageBytes + kSideBytes);
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTableBytes + kMiscBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * (kStageBytes + kSideBytes) + kTableBytes + kMiscBytes;
     static_assert(kStageBytes % 1024 == 0, "stages keep the swizzle atoms aligned");
+    static_assert(kSideBytes % 16 == 0, "bulk copies land 16-byte aligned");
     static_assert(!kFp8 || sizeof(T) == 2, "FP8 weights: 16-bit activations");
-    // barriers (full/empty per stage, 2 TMEM pairs, the item ring, the conversion
-    // ring, the drain barrier) and the ring / TMEM / flag words fit the misc area
-    static_assert((2 * kStages + 2 * kNumAcc + 2 * kFfnRing + 2 * kConv + 1) * 8 + 4 * kFfnRing + 16 <= kMiscBytes,
+    // barriers (full/empty per stage, 2 TMEM pairs, the item ring, the split
+    // barriers, the drain barrier) and the ring / TMEM / flag words fit the misc area
+    static_assert((2 * kStages + 2 * kNumAcc + 2 * kFfnRing + 2 * kXReady + 1) * 8 + 4 * kFfnRing + 16 <= kMiscBytes,
                   "misc area");
-    static constexpr int kSlotFloats = 128 * kAccCols;
+    static constexpr int kSlotFloats = 128 * 2 * kMaxN;  // a split tile's partial gate and up sums
     static_assert(kMaxN == 32 || kMaxN == 64 || kMaxN == 128, "decode token tiles");
-    static_assert(kAccCols * kNumAcc + kConv * kConvCols <= 512, "TMEM columns");
+    static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
 };
 
 // One phase's split: S slices per tile (S = 1: whole tiles).
@@ -147,23 +167,35 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Two E4M3 codes at bits [7:0] and [23:16] -> two f16 holding value x 2^-8:
-// the sign moves to bit 15, the 4 exponent and 3 mantissa bits to bits 13:7,
-// so an E4M3 exponent field e becomes the f16 exponent field e (bias 15 vs 7)
-// and e = 0 (subnormal) stays subnormal -- exact for every finite code.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t two) {
-    return ((two << 8) & 0x80008000u) | ((two << 7) & 0x3F803F80u);
-}
-// 16 codes -> 16 f16 (value x 2^-8) in two 16-byte chunks
-__device__ __forceinline__ void e4m3x16_to_f16(const uint4 v, uint4& lo, uint4& hi) {
-    lo = make_uint4(e4m3x2_to_f16x2_scaled(__byte_perm(v.x, 0, 0x4140)),
-                    e4m3x2_to_f16x2_scaled(__byte_perm(v.x, 0, 0x4342)),
-                    e4m3x2_to_f16x2_scaled(__byte_perm(v.y, 0, 0x4140)),
-                    e4m3x2_to_f16x2_scaled(__byte_perm(v.y, 0, 0x4342)));
-    hi = make_uint4(e4m3x2_to_f16x2_scaled(__byte_perm(v.z, 0, 0x4140)),
-                    e4m3x2_to_f16x2_scaled(__byte_perm(v.z, 0, 0x4342)),
-                    e4m3x2_to_f16x2_scaled(__byte_perm(v.w, 0, 0x4140)),
-                    e4m3x2_to_f16x2_scaled(__byte_perm(v.w, 0, 0x4342)));
+// 16 activations (two 16-byte chunks of f16) times inv -> their E4M3 hi and
+// lo codes: hi = E4M3(y), lo = E4M3(y - hi), y = a * inv (inv a power of two:
+// exact), y - hi exact in fp32.
+__device__ __forceinline__ void split_f16x16_e4m3(const uint4 a, const uint4 b, float inv, uint4& hi, uint4& lo) {
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t hw = 0, lw = 0;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            __half2_raw raw;
+            raw.x = (unsigned short)(in[2 * q + j] & 0xFFFFu);
+            raw.y = (unsigned short)(in[2 * q + j] >> 16);
+            float2 y = __half22float2(__half2(raw));
+            y.x *= inv;
+            y.y *= inv;
+            const __nv_fp8x2_storage_t hc = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+            const float2 hv = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hc, __NV_E4M3)));
+            const __nv_fp8x2_storage_t lc =
+                __nv_cvt_float2_to_fp8x2(make_float2(y.x - hv.x, y.y - hv.y), __NV_SATFINITE, __NV_E4M3);
+            hw |= (uint32_t)hc << (16 * j);
+            lw |= (uint32_t)lc << (16 * j);
+        }
+        h[q] = hw;
+        l[q] = lw;
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 template <typename T, int kMaxN, bool kFp8 = false>
@@ -177,7 +209,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_base = smem;
-    int* seg = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes);
+    uint8_t* side_base = smem + C::kStages * C::kStageBytes;  // FP8: per-stage activation maxima
+    int* seg = reinterpret_cast<int*>(side_base + C::kStages * C::kSideBytes);
     int* cbase = seg + (kMaxGroups + 1);
     uint8_t* misc = reinterpret_cast<uint8_t*>(cbase + (kMaxGroups + 1));
     uint64_t* full = reinterpret_cast<uint64_t*>(misc);
@@ -186,9 +219,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     uint64_t* tempty = tfull + C::kNumAcc;
     uint64_t* ring_full = tempty + C::kNumAcc;
     uint64_t* ring_empty = ring_full + kFfnRing;
-    uint64_t* conv_full = ring_empty + kFfnRing;  // C::kConv barriers each (none without FP8 weights)
-    uint64_t* conv_empty = conv_full + C::kConv;
-    uint64_t* drain_bar = conv_empty + C::kConv;
+    uint64_t* xready = ring_empty + kFfnRing;  // FP8: a stage's split activation tile is ready
+    uint64_t* bfull = xready + C::kXReady;     // FP8: a phase-B fill of the stage landed
+    uint64_t* drain_bar = bfull + C::kXReady;
     int* ring = reinterpret_cast<int*>(drain_bar + 1);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ring + kFfnRing);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -203,6 +236,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     int* done_ctr = p.ctl + 1;
     int* chunk_done = p.ctl + 2;
     int* tile_ctr = p.ctl + 2 + kFfnMaxChunks;
+    unsigned* act_amax = reinterpret_cast<unsigned*>(p.ctl + kFfnAmaxOff);  // FP8: per-row max |activation|
 
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
@@ -216,12 +250,12 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         }
         for (int r = 0; r < kFfnRing; ++r) {
             mbar_init(&ring_full[r], 1);
-            // the MMA thread, every epilogue thread and (FP8) every converter thread
-            mbar_init(&ring_empty[r], 1 + 128 + C::kConvThreads);
+            // the MMA thread, every epilogue thread and (FP8) every splitter thread
+            mbar_init(&ring_empty[r], 1 + 128 + C::kSplitThreads);
         }
-        for (int c = 0; c < C::kConv; ++c) {
-            mbar_init(&conv_full[c], C::kConvThreads / 32);  // one arrival per converter warp
-            mbar_init(&conv_empty[c], 1);
+        for (int c = 0; c < C::kXReady; ++c) {
+            mbar_init(&xready[c], C::kSplitThreads / 32);  // one arrival per splitter warp
+            mbar_init(&bfull[c], 1);
         }
         mbar_init(drain_bar, 1);
         fence_barrier_init();
@@ -270,7 +304,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     const long long total = nA + nB;
     const long long slotsA = SA > 1 ? nA : 0;
     const bool oversize = n_chunks > kFfnMaxChunks || (SA > 1 && tilesA > kFfnTileCtrs / 2) ||
-                          (SB > 1 && tilesB > kFfnTileCtrs / 2);
+                          (SB > 1 && tilesB > kFfnTileCtrs / 2) || (kFp8 && seg[n_groups] > kFfnMaxRows);
 
     auto item_of = [&](long long id, FfnItem& it, Tile& t) {
         if (id < nA) {
@@ -303,9 +337,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             const uint64_t pol_w_once = policy_evict_first();
             const uint64_t pol_w_shared = policy_evict_normal();
             const uint64_t pol_x = policy_evict_last();
-            int fills[C::kStages];
+            int fills[C::kStages], bfills[C::kStages];  // completions owed on full[s] / bfull[s]
 #pragma unroll
-            for (int s = 0; s < C::kStages; ++s) fills[s] = 0;
+            for (int s = 0; s < C::kStages; ++s) fills[s] = bfills[s] = 0;
             uint32_t kc = 0, n = 0;
             bool withhold = false;  // test hook: armed for work item 0, whichever block takes it
             bool ok = !oversize;
@@ -341,17 +375,35 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 const CUtensorMap* tx64 = it.phase == 0 ? &tm_xa64 : &tm_xb64;
                 const int second = it.phase == 0 ? p.I : 128;  // up rows, or the next 128 features
                 const uint32_t bytes = 2 * C::kRawWBytes + C::kXBoxes * t.mma_n * 128;
+                // FP8 down: the item's first stage also brings its rows' activation
+                // maxima, from the 16-byte boundary at or below row0
+                const uint32_t side_bytes =
+                    kFp8 && it.phase == 1 ? 4u * (uint32_t)(((t.row0 & 3) + t.mma_n + 3) & ~3) : 0u;
                 const uint64_t pol_w = t.nch > 1 ? pol_w_shared : pol_w_once;
+                // FP8 phase B: the stage's loads complete on bfull[s] (the splitters'
+                // barrier); every other stage on full[s] (the MMA thread's)
+                const bool to_b = kFp8 && it.phase == 1;
+                auto bar_of = [&](int s) { return to_b ? &bfull[s] : &full[s]; };
+                auto owe = [&](int s) {
+                    if (to_b)
+                        ++bfills[s];
+                    else
+                        ++fills[s];
+                };
                 auto load_w = [&](int s, int k) {
                     uint8_t* st = stage_base + s * C::kStageBytes;
                     const int kx = k * C::kBK;
-                    tma_load_2d(st, tw, &full[s], kx, t.wrow, pol_w);
-                    tma_load_2d(st + C::kRawWBytes, tw, &full[s], kx, t.wrow + second, pol_w);
+                    tma_load_2d(st, tw, bar_of(s), kx, t.wrow, pol_w);
+                    tma_load_2d(st + C::kRawWBytes, tw, bar_of(s), kx, t.wrow + second, pol_w);
                 };
+                // FP8: the second box (lo codes, or activation columns 64..127)
+                const int box_off = (C::kStack ? t.mma_n : kMaxN) * 128;
                 auto load_x = [&](int s, int k) {
+                    if (to_b && k == it.kb)
+                        bulk_load_g2s(side_base + s * C::kSideBytes, act_amax + (t.row0 & ~3), side_bytes, bar_of(s));
 #pragma unroll
                     for (int xb = 0; xb < C::kXBoxes; ++xb) {
-                        uint8_t* xs = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes + xb * kMaxN * 128;
+                        uint8_t* xs = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes + xb * box_off;
                         // FP8 gate/up: box xb holds the hi (0) or lo (1) codes of columns
                         // k*128..+127; otherwise 64 16-bit columns each
                         const bool codes = kFp8 && it.phase == 0;
@@ -360,9 +412,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         int r = 0;
                         if (kMaxN >= C::kXBoxMid)
                             for (; r + C::kXBoxMid <= t.mma_n; r += C::kXBoxMid)
-                                tma_load_2d(xs + r * 128, tx64, &full[s], kx, rbase + t.row0 + r, pol_x);
+                                tma_load_2d(xs + r * 128, tx64, bar_of(s), kx, rbase + t.row0 + r, pol_x);
                         for (; r < t.mma_n; r += C::kXBoxRows)
-                            tma_load_2d(xs + r * 128, tx, &full[s], kx, rbase + t.row0 + r, pol_x);
+                            tma_load_2d(xs + r * 128, tx, bar_of(s), kx, rbase + t.row0 + r, pol_x);
                     }
                 };
                 int pre = 0;  // stages of this item whose weight tiles went out before the activation wait
@@ -378,9 +430,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&full[s], bytes);
+                        mbar_arrive_expect_tx(bar_of(s), bytes + (pre == 0 ? side_bytes : 0u));
                         load_w(s, it.kb + pre);
-                        ++fills[s];
+                        owe(s);
                     }
                     if (ok) {
                         const uint64_t t0 = global_ns();
@@ -411,10 +463,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         withhold = false;
                         continue;
                     }
-                    mbar_arrive_expect_tx(&full[s], bytes);
+                    mbar_arrive_expect_tx(bar_of(s), bytes + (k == it.kb ? side_bytes : 0u));
                     load_w(s, k);
                     load_x(s, k);
-                    ++fills[s];
+                    owe(s);
                 }
                 if (!ok) continue;
             }
@@ -422,14 +474,16 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 *abort_flag = 1;
                 if (!oversize) atomicOr(p.status, kStatusTimeout);
             }
-            for (int s = 0; s < C::kStages; ++s)
+            for (int s = 0; s < C::kStages; ++s) {
                 if (fills[s] > 0) mbar_drain(&full[s], (uint32_t)(fills[s] - 1) & 1u, limit);
+                if (bfills[s] > 0) mbar_drain(&bfull[s], (uint32_t)(bfills[s] - 1) & 1u, limit);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
             uint32_t kc = 0, ac = 0, n = 0;
-            uint32_t cc = 0;  // FP8: stages widened so far (the conversion ring's own count)
+            uint32_t xpar = 0;  // FP8: per-stage parity of the split barriers (bit s)
             bool ok = true;
             while (true) {
                 const int rs = n % kFfnRing;
@@ -453,59 +507,57 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + b * C::kAccCols;
-                const uint32_t d1 = d0 + kMaxN;
-                // (FP8: f16 operands in phase B; in phase A E4M3 x E4M3, whose format
-                // code in the kind::f8f6f4 descriptor is also 0)
-                const uint32_t idesc = umma_idesc(kFp8 ? Elt<__half>::kMmaFmt : Elt<T>::kMmaFmt, 128, t.mma_n);
+                const uint32_t d1 = d0 + C::kUOff;
+                const uint32_t idesc = umma_idesc(kFp8 ? kFmtE4M3 : Elt<T>::kMmaFmt, 128, C::kStack ? 2 * t.mma_n : t.mma_n);
                 for (int k = it.kb; k < it.ke; ++k, ++kc) {
                     const int s = kc % C::kStages;
                     const uint32_t ph = (kc / C::kStages) & 1u;
-                    if (!mbar_wait_bounded(&full[s], ph, limit, abort_flag)) {
+                    if (kFp8 && it.phase == 1) {
+                        // the splitters' hi / lo codes of the activation tile (they waited
+                        // for the stage's loads; a block's phase-B items follow all of
+                        // its phase-A items, so full[s]'s phases count phase-A fills only)
+                        if (!mbar_wait_bounded(&xready[s], (xpar >> s) & 1u, limit, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        xpar ^= 1u << s;
+                    } else if (!mbar_wait_bounded(&full[s], ph, limit, abort_flag)) {
                         ok = false;
                         break;
                     }
                     uint8_t* st = stage_base + s * C::kStageBytes;
-                    const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
-                    int cv = -1;
-                    if (kFp8 && it.phase == 0) {
-                        // E4M3 weights x the token rows' hi codes, then x their lo codes,
-                        // into the same accumulator: K 32 per MMA, four steps per stage
+                    const uint64_t a0 = umma_desc_sw128(smem_u32(st));
+                    const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
+                    if constexpr (kFp8) {
                         tc_fence_after();
-                        const uint64_t a0 = umma_desc_sw128(smem_u32(st));
-                        const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
-#pragma unroll
-                        for (int part = 0; part < 2; ++part) {
-                            const uint64_t b = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes + part * kMaxN * 128));
+                        if constexpr (C::kStack) {
+                            // E4M3 weights x [hi rows; lo rows] in one MMA (N = 2 mma_n):
+                            // K 32 per MMA, four steps per stage
+                            const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
-                                const uint32_t acc = (k > it.kb || kk > 0 || part > 0) ? 1u : 0u;
-                                umma_e4m3(d0, a0 + 2 * kk, b + 2 * kk, idesc, acc);
-                                umma_e4m3(d1, a1 + 2 * kk, b + 2 * kk, idesc, acc);
+                                const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
+                                umma_e4m3(d0, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                                umma_e4m3(d1, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
                             }
-                        }
-                    } else if constexpr (kFp8) {
-                        // A: the stage's two tiles, widened to f16 in TMEM by the converter warps
-                        cv = (int)(cc % C::kConv);
-                        if (!mbar_wait_bounded(&conv_full[cv], (cc / C::kConv) & 1u, limit, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t a0 = tmem_base + C::kConvCol0 + cv * C::kConvCols;
-                        // K 128 per stage: eight 16-deep steps, the token operand's
-                        // first four in its first 64-column box, the rest in the second
+                        } else {
+                            // E4M3 weights x the hi rows, then x the lo rows, into the same
+                            // accumulator
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
-                            const uint64_t b = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes + (kk >> 2) * kMaxN * 128)) +
-                                               2 * (kk & 3);
-                            umma_f16_tmem_a(d0, a0 + 8 * kk, b, idesc, acc);
-                            umma_f16_tmem_a(d1, a0 + 64 + 8 * kk, b, idesc, acc);
+                            for (int part = 0; part < 2; ++part) {
+                                const uint64_t bx =
+                                    umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes + part * kMaxN * 128));
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk) {
+                                    const uint32_t acc = (k > it.kb || kk > 0 || part > 0) ? 1u : 0u;
+                                    umma_e4m3(d0, a0 + 2 * kk, bx + 2 * kk, idesc, acc);
+                                    umma_e4m3(d1, a1 + 2 * kk, bx + 2 * kk, idesc, acc);
+                                }
+                            }
                         }
                     } else {
                         tc_fence_after();
-                        const uint64_t a0 = umma_desc_sw128(smem_u32(st));
-                        const uint64_t a1 = umma_desc_sw128(smem_u32(st + C::kWTileBytes));
+                        const uint64_t bx = umma_desc_sw128(smem_u32(st + 2 * C::kRawWBytes));
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint32_t acc = (k > it.kb || kk > 0) ? 1u : 0u;
@@ -514,10 +566,6 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         }
                     }
                     umma_commit(&empty[s]);
-                    if (cv >= 0) {  // FP8 down: the conversion buffer is free too
-                        umma_commit(&conv_empty[cv]);
-                        ++cc;
-                    }
                 }
                 if (!ok) break;
                 umma_commit(&tfull[b]);
@@ -530,24 +578,24 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 mbar_drain(drain_bar, 0, limit);
             }
         }
-    } else if (kFp8 && warp >= 6) {  // converter warps 6 .. 5 + kConvThreads / 32
-        // ------------------------------------------- FP8 -> f16 converters
-        // warps 6..9 widen a stage's first weight tile, warps 10..13 its second;
-        // a warp may only store to its TMEM lane quadrant (warp mod 4), so each
-        // thread takes one row (quadrant x 32 + lane): its 128 codes are eight
-        // 16-byte chunks, chunk c of row r at chunk position c ^ (r mod 8) under
-        // the 128-byte swizzle (8 consecutive rows hit 8 distinct bank groups),
-        // widened to 64 f16 pairs and stored as 64 TMEM columns
-        const int quad = warp & 3;
-        const int row = quad * 32 + lane;
-        const int tt = (warp - 6) >> 2;
-        const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-        uint32_t kc = 0, n = 0, cc = 0;  // stages, items, widened stages
+    } else if (kFp8 && warp >= 6) {  // splitter warps 6 .. 13
+        // ------------------------------------- activation splitters (phase B)
+        // Unit u = (row u / 8, columns 16 (u % 8) .. + 15) of a stage's 128
+        // activation columns; thread i takes units i, i + 256, ...  A unit reads
+        // two 16-byte f16 chunks of box (u % 8) / 4 and writes one 16-byte chunk
+        // of hi codes (box 0) and one of lo codes (box 1), all under the 128-byte
+        // swizzle (chunk c of row r at c ^ (r mod 8)).  Every read of the stage
+        // precedes every write (in-place), so the 256 threads meet at a named
+        // barrier in between; every exit is agreed at a reducing barrier first,
+        // so no thread is left waiting at one.
+        const int ct = threadIdx.x - 6 * 32;
+        uint32_t kc = 0, n = 0;
+        uint32_t bpar = 0;  // per-stage parity of bfull (bit s): phase-B fills seen so far
         bool ok = true;
-        while (ok) {
+        while (true) {
             const int rs = n % kFfnRing;
-            const uint32_t rph = (n / kFfnRing) & 1u;
-            if (!mbar_wait_bounded(&ring_full[rs], rph, limit, abort_flag)) {
+            const bool got = mbar_wait_bounded(&ring_full[rs], (n / kFfnRing) & 1u, limit, abort_flag);
+            if (!named_all(2, C::kSplitThreads, got)) {
                 ok = false;
                 break;
             }
@@ -558,46 +606,56 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             FfnItem it;
             Tile t;
             item_of(id, it, t);
-            if (it.phase == 0) {  // gate/up stages use the codes as they are
+            if (it.phase == 0) {  // gate/up stages carry split token rows already
                 kc += it.ke - it.kb;
                 continue;
             }
-            for (int k = it.kb; k < it.ke; ++k, ++kc, ++cc) {
+            float inv[C::kUnits];
+            for (int k = it.kb; k < it.ke; ++k, ++kc) {
                 const int s = kc % C::kStages;
-                const int cv = (int)(cc % C::kConv);
-                const bool got = mbar_wait_bounded(&full[s], (kc / C::kStages) & 1u, limit, abort_flag) &&
-                                 mbar_wait_bounded(&conv_empty[cv], ((cc / C::kConv) & 1u) ^ 1u, limit, abort_flag);
-                if (!__all_sync(0xffffffffu, got)) {  // the whole warp leaves together (warp-wide TMEM stores)
+                const bool g = mbar_wait_bounded(&bfull[s], (bpar >> s) & 1u, limit, abort_flag);
+                bpar ^= 1u << s;
+                if (!named_all(2, C::kSplitThreads, g)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();  // the MMAs that read this buffer before have completed
-                const uint8_t* src = stage_base + s * C::kStageBytes + tt * C::kRawWBytes + row * 128;
+                uint8_t* xt = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes;
+                const int box_off = (C::kStack ? t.mma_n : kMaxN) * 128;  // second box: f16 columns 64.., then lo codes
+                if (k == it.kb) {  // the rows' scales, from the maxima that came with this stage
+                    const unsigned* side = reinterpret_cast<const unsigned*>(side_base + s * C::kSideBytes);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {  // codes 64 h .. 64 h + 63 -> 32 columns
-                    uint32_t w[32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int cc = 4 * h + c;
-                        const uint4 v = *reinterpret_cast<const uint4*>(src + ((cc ^ (row & 7)) << 4));
-                        uint4 lo, hi;
-                        e4m3x16_to_f16(v, lo, hi);
-                        w[8 * c + 0] = lo.x;
-                        w[8 * c + 1] = lo.y;
-                        w[8 * c + 2] = lo.z;
-                        w[8 * c + 3] = lo.w;
-                        w[8 * c + 4] = hi.x;
-                        w[8 * c + 5] = hi.y;
-                        w[8 * c + 6] = hi.z;
-                        w[8 * c + 7] = hi.w;
+                    for (int j = 0; j < C::kUnits; ++j) {
+                        const int r = (ct + 256 * j) >> 3;
+                        inv[j] = r < t.nrows ? e4m3_pow2_inv_scale(__uint_as_float(side[(t.row0 & 3) + r])) : 0.f;
                     }
-                    tmem_st32(tmem_base + lane_base + C::kConvCol0 + cv * C::kConvCols + tt * 64 + h * 32, w);
                 }
-                tmem_wait_st();
-                tc_fence_before();
+                uint4 va[C::kUnits], vb[C::kUnits];
+#pragma unroll
+                for (int j = 0; j < C::kUnits; ++j) {
+                    const int u = ct + 256 * j, r = u >> 3, c = u & 7;
+                    if (r < t.nrows) {
+                        const uint8_t* src = xt + (c >> 2) * box_off + r * 128;
+                        va[j] = *reinterpret_cast<const uint4*>(src + (((2 * (c & 3)) ^ (r & 7)) << 4));
+                        vb[j] = *reinterpret_cast<const uint4*>(src + (((2 * (c & 3) + 1) ^ (r & 7)) << 4));
+                    }
+                }
+                named_sync(2, C::kSplitThreads);
+#pragma unroll
+                for (int j = 0; j < C::kUnits; ++j) {
+                    const int u = ct + 256 * j, r = u >> 3, c = u & 7;
+                    if (r < t.mma_n) {  // rows past the chunk's own: zero codes
+                        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+                        if (r < t.nrows) split_f16x16_e4m3(va[j], vb[j], inv[j], hi, lo);
+                        const int off = r * 128 + ((c ^ (r & 7)) << 4);
+                        *reinterpret_cast<uint4*>(xt + off) = hi;
+                        *reinterpret_cast<uint4*>(xt + box_off + off) = lo;
+                    }
+                }
+                fence_proxy_async_shared();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&conv_full[cv]);
+                if (lane == 0) mbar_arrive(&xready[s]);
             }
+            if (!ok) break;
         }
         if (!ok) {
             *abort_flag = 1;
@@ -641,26 +699,30 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             using ActT = typename std::conditional<kFp8, __half, OutT>::type;
             OutT* orow = reinterpret_cast<OutT*>(p.y) + (long long)t.row0 * n_out + f;
             ActT* arow = reinterpret_cast<ActT*>(p.act) + (long long)t.row0 * n_out + f;
-            // FP8 weights: the row scales of the two accumulators' weight rows,
-            // times 2^8 (the widened codes hold value x 2^-8)
+            // FP8 weights: the row scales of the two accumulators' weight rows
             float sc0 = 1.f, sc1 = 1.f;
             if constexpr (kFp8) {
-                if (gate_up) {  // direct E4M3 products: no widening factor; the token scale per column below
+                if (gate_up) {
                     const float* sr = p.s13 + (long long)t.group * 2 * p.I;
                     sc0 = v0 ? __ldg(sr + f) : 0.f;
                     sc1 = v0 ? __ldg(sr + p.I + f) : 0.f;
                 } else {
                     const float* sr = p.s2 + (long long)t.group * p.H;
-                    sc0 = v0 ? __ldg(sr + f) * 256.f : 0.f;
-                    sc1 = v1 ? __ldg(sr + f + 128) * 256.f : 0.f;
+                    sc0 = v0 ? __ldg(sr + f) : 0.f;
+                    sc1 = v1 ? __ldg(sr + f + 128) : 0.f;
                 }
             }
             auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {
                 if constexpr (kFp8) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        // the token row's scale (phase A operand), read for real rows only
-                        const float xs = gate_up && c0 + i < t.nrows ? __ldg(p.x_scale + t.row0 + c0 + i) : 1.f;
+                        // the token row's scale, read for real rows only: the split of x
+                        // (gate/up), or the one the splitters took from the row's maximum
+                        // activation (down)
+                        float xs = 1.f;
+                        if (c0 + i < t.nrows)
+                            xs = gate_up ? __ldg(p.x_scale + t.row0 + c0 + i)
+                                         : e4m3_pow2_scale(__uint_as_float(__ldcg(act_amax + t.row0 + c0 + i)));
                         g[i] *= sc0 * xs;
                         u[i] *= sc1 * xs;
                     }
@@ -668,6 +730,16 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 if (gate_up) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) g[i] = silu_mul(g[i], u[i]);
+                    if constexpr (kFp8) {
+                        // raise each row's maximum |activation| (as stored, in f16) by
+                        // this warp's 32 features; non-negative floats order as their bits
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float a = v0 && c0 + i < t.nrows ? fabsf(__half2float(__float2half_rn(g[i]))) : 0.f;
+                            const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
+                            if (lane == i && m != 0u) atomicMax(act_amax + t.row0 + c0 + i, m);
+                        }
+                    }
                 }
                 if (v0 && gate_up) {
 #pragma unroll
@@ -684,8 +756,25 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         if (c0 + i < t.nrows) store_out<OutT>(orow + 128 + (long long)(c0 + i) * n_out, u[i]);
                 }
             };
+            // 16 columns of an accumulator (FP8 stacked: its hi and lo products added)
+            auto ld_acc = [&](uint32_t col, float (&v)[16]) {
+                tmem_ld16(col, v);
+                if constexpr (C::kStack) {
+                    float w[16];
+                    tmem_ld16(col + t.mma_n, w);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] += w[i];
+                }
+            };
             bool finished = true;  // this item completed its tile
-            if (it.S == 1) {
+            if (C::kStack && it.S == 1) {
+                for (int c0 = 0; c0 < t.nrows; c0 += 16) {
+                    float g[16], u[16];
+                    ld_acc(tacc + c0, g);
+                    ld_acc(tacc + C::kUOff + c0, u);
+                    emit(c0, g, u);
+                }
+            } else if (it.S == 1) {
                 for (int c0 = 0; c0 < t.nrows; c0 += 32) {
                     uint32_t ga[32], ua[32];
                     tmem_ld32_nowait(tacc + c0, ga);
@@ -707,13 +796,13 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 float4* mine = reinterpret_cast<float4*>(p.partials + it.slot * C::kSlotFloats);
                 for (int c0 = 0; c0 < t.nrows; c0 += 16) {
                     float g[16];
-                    tmem_ld16(tacc + c0, g);
+                    ld_acc(tacc + c0, g);
                     if (v0) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             mine[slot_f4((c0 >> 2) + q, r)] = make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
                     }
-                    tmem_ld16(tacc + kMaxN + c0, g);
+                    ld_acc(tacc + C::kUOff + c0, g);
                     if (v1) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
@@ -736,10 +825,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         for (int sl = 0; sl < it.S; ++sl) {
                             if (sl == it.slice) {
                                 float v[16];
-                                tmem_ld16(tacc + c0, v);
+                                ld_acc(tacc + c0, v);
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) g[i] += v[i];
-                                tmem_ld16(tacc + kMaxN + c0, v);
+                                ld_acc(tacc + C::kUOff + c0, v);
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) u[i] += v[i];
                             } else {
@@ -795,6 +884,10 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         __threadfence();
         const long long nc = n_chunks < kFfnMaxChunks ? n_chunks : kFfnMaxChunks;
         for (long long c = threadIdx.x; c < nc; c += blockDim.x) chunk_done[c] = 0;
+        if (kFp8) {
+            const int rows = seg[n_groups] < kFfnMaxRows ? seg[n_groups] : kFfnMaxRows;
+            for (int r = threadIdx.x; r < rows; r += blockDim.x) act_amax[r] = 0u;
+        }
         if (threadIdx.x == 0) {
             *work_ctr = 0;
             *done_ctr = 0;

@@ -206,10 +206,12 @@ int launch_ffn_variant(const FfnLaunch& L, const GemmCtl& ctl, int num_sms, cuda
     }
     // token operands: on the FP8 path the gate/up operand is the rows' E4M3 hi
     // and lo codes ([2 x_rows, H] bytes, 128-code boxes) and the activations are
-    // f16; otherwise both are in the activation dtype
+    // f16 (split into codes in shared memory); otherwise both are in the
+    // activation dtype
     const CUtensorMapDataType xdt = kFp8 ? Elt<__half>::kTma : dt;
     if (kFp8) {
-        if (!L.x_scale) return -1;
+        // the per-row activation maxima live in the control block
+        if (!L.x_scale || L.x_rows > kFfnMaxRows) return -1;
         if (!make_map(&xa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.x, 2 * L.x_rows, L.H, 16)) return -3;
         if (!make_map(&xa64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L.x, 2 * L.x_rows, L.H, 64)) return -3;
     } else {

@@ -911,7 +911,8 @@ int launch_permute(int H, int K, int dtype, long long P_max, const void* x, cons
 }
 
 // Exact two-term E4M3 split of bf16 token rows, the token operand of the FP8
-// gate/up MMAs: with s the smallest power of two for which max |x| <= 448 s,
+// gate/up MMAs: with s the smallest power of two for which max |x| <= 448 s
+// (at least 2^-126),
 // x / s is exact, hi = E4M3(x / s) keeps its leading four significant bits,
 // and the rest r = x / s - hi (exact in fp32; at most four significant bits
 // for the eight of a bf16 value) is lo = E4M3(r), so x = s (hi + lo) except
@@ -963,16 +964,8 @@ __global__ void __launch_bounds__(256) split_e4m3_kernel(int H, int K, long long
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        // the smallest power of two s with amax <= 448 s (products with 448 s are exact)
-        float sc = 1.f;
-        if (amax > 0.f) {
-            int e;
-            frexpf(amax / 448.f, &e);
-            sc = ldexpf(1.f, e);
-            while (amax > 448.f * sc) sc *= 2.f;
-            while (amax <= 224.f * sc) sc *= 0.5f;
-        }
-        const float inv = 1.f / sc;  // a power of two: exact
+        const float sc = e4m3_pow2_scale(amax);
+        const float inv = e4m3_pow2_inv_scale(amax);
         for (int v = lane; v < nv; v += 32) {
             const int4 q = __ldg(src + v);
             const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
