@@ -138,14 +138,21 @@ struct FfnCfg {
     static_assert(kAccCols * kNumAcc <= 512, "TMEM columns");
 };
 
-// One phase's split: S slices per tile (S = 1: whole tiles).
-__device__ __forceinline__ int ffn_slices(long long tiles, int KI, int G, int max_slots) {
+// One phase's split: S slices per tile (S = 1: whole tiles), about two items
+// per block.  A tile's last slice sums the S partial slots (128 x 2 n fp32
+// each, n token columns) on one SM, so S also balances that sum against the
+// streaming it shortens: a slice streams KI / S stages of 32 KB of weights,
+// the sum reads (S - 1) slots of n KB, and the two balance near
+// S = sqrt(32 KI / n).
+__device__ __forceinline__ int ffn_slices(long long tiles, int KI, int G, int max_slots, int n) {
     if (tiles <= 0 || tiles >= 2LL * G) return 1;
     long long s = (2LL * G + tiles - 1) / tiles;
     long long cap = (4LL * G < max_slots ? 4LL * G : max_slots) / tiles;
     if (s > cap) s = cap;
     if (s > 16) s = 16;
     if (s > KI / 4) s = KI / 4;
+    const long long bal = (long long)sqrtf(32.f * (float)KI / (float)n);
+    if (s > bal) s = bal;
     return s < 1 ? 1 : (int)s;
 }
 
@@ -167,32 +174,56 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// 16 activations (two 16-byte chunks of f16) times inv -> their E4M3 hi and
-// lo codes: hi = E4M3(y), lo = E4M3(y - hi), y = a * inv (inv a power of two:
-// exact), y - hi exact in fp32.
-__device__ __forceinline__ void split_f16x16_e4m3(const uint4 a, const uint4 b, float inv, uint4& hi, uint4& lo) {
+// 16 activations (two 16-byte chunks of f16) times 2^e -> their E4M3 hi and
+// lo codes: hi = E4M3(y), lo = E4M3(y - hi), y = a 2^e.  For e <= 15 in packed
+// f16: a 2^e is exact (it only loses what falls below 2^-24, far under the lo
+// codes' grid) and y - hi is exact (both are multiples of y's unit in the last
+// place and |y - hi| is below hi's); for larger e (rows whose largest
+// activation is below 448 x 2^-16) in fp32, where 2^e is representable.
+__device__ __forceinline__ uint32_t e4m3x2_of_h2(__half2 v) {
+    return (uint32_t)__nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(v), __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ void split_f16x16_e4m3(const uint4 a, const uint4 b, int e, uint4& hi, uint4& lo) {
     const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     uint32_t h[4], l[4];
+    if (e <= 15) {
+        const __half2 m = __half2half2(__ushort_as_half((unsigned short)((e + 15) << 10)));
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t hw = 0, lw = 0;
+        for (int q = 0; q < 4; ++q) {
+            uint32_t hw = 0, lw = 0;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            __half2_raw raw;
-            raw.x = (unsigned short)(in[2 * q + j] & 0xFFFFu);
-            raw.y = (unsigned short)(in[2 * q + j] >> 16);
-            float2 y = __half22float2(__half2(raw));
-            y.x *= inv;
-            y.y *= inv;
-            const __nv_fp8x2_storage_t hc = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
-            const float2 hv = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hc, __NV_E4M3)));
-            const __nv_fp8x2_storage_t lc =
-                __nv_cvt_float2_to_fp8x2(make_float2(y.x - hv.x, y.y - hv.y), __NV_SATFINITE, __NV_E4M3);
-            hw |= (uint32_t)hc << (16 * j);
-            lw |= (uint32_t)lc << (16 * j);
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t w = in[2 * q + j];
+                const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&w), m);
+                const uint32_t hc = e4m3x2_of_h2(y);
+                const __half2 hv(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)hc, __NV_E4M3));
+                hw |= hc << (16 * j);
+                lw |= e4m3x2_of_h2(__hsub2(y, hv)) << (16 * j);
+            }
+            h[q] = hw;
+            l[q] = lw;
         }
-        h[q] = hw;
-        l[q] = lw;
+    } else {
+        const float inv = __uint_as_float((uint32_t)(e + 127) << 23);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t hw = 0, lw = 0;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t w = in[2 * q + j];
+                float2 y = __half22float2(*reinterpret_cast<const __half2*>(&w));
+                y.x *= inv;
+                y.y *= inv;
+                const __nv_fp8x2_storage_t hc = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+                const float2 hv = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hc, __NV_E4M3)));
+                const __nv_fp8x2_storage_t lc =
+                    __nv_cvt_float2_to_fp8x2(make_float2(y.x - hv.x, y.y - hv.y), __NV_SATFINITE, __NV_E4M3);
+                hw |= (uint32_t)hc << (16 * j);
+                lw |= (uint32_t)lc << (16 * j);
+            }
+            h[q] = hw;
+            l[q] = lw;
+        }
     }
     hi = make_uint4(h[0], h[1], h[2], h[3]);
     lo = make_uint4(l[0], l[1], l[2], l[3]);
@@ -299,7 +330,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     const int NFA = (p.I + 127) / 128, NFB = (p.H + 255) / 256;
     const int KIA = (p.H + C::kBK - 1) / C::kBK, KIB = (p.I + C::kBK - 1) / C::kBK;
     const long long tilesA = n_chunks * NFA, tilesB = n_chunks * NFB;
-    const int SA = ffn_slices(tilesA, KIA, G, p.max_slots_phase), SB = ffn_slices(tilesB, KIB, G, p.max_slots_phase);
+    const int SA = ffn_slices(tilesA, KIA, G, p.max_slots_phase, kMaxN),
+              SB = ffn_slices(tilesB, KIB, G, p.max_slots_phase, kMaxN);
     const long long nA = tilesA * SA, nB = tilesB * SB;
     const long long total = nA + nB;
     const long long slotsA = SA > 1 ? nA : 0;
@@ -585,9 +617,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         // two 16-byte f16 chunks of box (u % 8) / 4 and writes one 16-byte chunk
         // of hi codes (box 0) and one of lo codes (box 1), all under the 128-byte
         // swizzle (chunk c of row r at c ^ (r mod 8)).  Every read of the stage
-        // precedes every write (in-place), so the 256 threads meet at a named
-        // barrier in between; every exit is agreed at a reducing barrier first,
-        // so no thread is left waiting at one.
+        // precedes every write (in place), so the 256 threads meet in between at
+        // a reducing barrier, which also decides whether all of them go on: an
+        // exit is always agreed there, so no thread is left waiting at one.
         const int ct = threadIdx.x - 6 * 32;
         uint32_t kc = 0, n = 0;
         uint32_t bpar = 0;  // per-stage parity of bfull (bit s): phase-B fills seen so far
@@ -610,42 +642,45 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 kc += it.ke - it.kb;
                 continue;
             }
-            float inv[C::kUnits];
+            int ex[C::kUnits];  // per unit: the row's scale is 2^-ex
             for (int k = it.kb; k < it.ke; ++k, ++kc) {
                 const int s = kc % C::kStages;
                 const bool g = mbar_wait_bounded(&bfull[s], (bpar >> s) & 1u, limit, abort_flag);
                 bpar ^= 1u << s;
+                uint8_t* xt = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes;
+                const int box_off = (C::kStack ? t.mma_n : kMaxN) * 128;  // second box: f16 columns 64.., then lo codes
+                uint4 va[C::kUnits], vb[C::kUnits];
+                if (g) {
+                    if (k == it.kb) {  // the rows' scales, from the maxima that came with this stage
+                        const unsigned* side = reinterpret_cast<const unsigned*>(side_base + s * C::kSideBytes);
+#pragma unroll
+                        for (int j = 0; j < C::kUnits; ++j) {
+                            const int r = (ct + 256 * j) >> 3;
+                            ex[j] = r < t.nrows ? -e4m3_pow2_exp(__uint_as_float(side[(t.row0 & 3) + r])) : 0;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < C::kUnits; ++j) {
+                        const int u = ct + 256 * j, r = u >> 3, c = u & 7;
+                        if (r < t.nrows) {
+                            const uint8_t* src = xt + (c >> 2) * box_off + r * 128;
+                            va[j] = *reinterpret_cast<const uint4*>(src + (((2 * (c & 3)) ^ (r & 7)) << 4));
+                            vb[j] = *reinterpret_cast<const uint4*>(src + (((2 * (c & 3) + 1) ^ (r & 7)) << 4));
+                        }
+                    }
+                }
+                // every read of the stage precedes every write (in place), and all
+                // leave together if any wait gave up
                 if (!named_all(2, C::kSplitThreads, g)) {
                     ok = false;
                     break;
                 }
-                uint8_t* xt = stage_base + s * C::kStageBytes + 2 * C::kRawWBytes;
-                const int box_off = (C::kStack ? t.mma_n : kMaxN) * 128;  // second box: f16 columns 64.., then lo codes
-                if (k == it.kb) {  // the rows' scales, from the maxima that came with this stage
-                    const unsigned* side = reinterpret_cast<const unsigned*>(side_base + s * C::kSideBytes);
-#pragma unroll
-                    for (int j = 0; j < C::kUnits; ++j) {
-                        const int r = (ct + 256 * j) >> 3;
-                        inv[j] = r < t.nrows ? e4m3_pow2_inv_scale(__uint_as_float(side[(t.row0 & 3) + r])) : 0.f;
-                    }
-                }
-                uint4 va[C::kUnits], vb[C::kUnits];
-#pragma unroll
-                for (int j = 0; j < C::kUnits; ++j) {
-                    const int u = ct + 256 * j, r = u >> 3, c = u & 7;
-                    if (r < t.nrows) {
-                        const uint8_t* src = xt + (c >> 2) * box_off + r * 128;
-                        va[j] = *reinterpret_cast<const uint4*>(src + (((2 * (c & 3)) ^ (r & 7)) << 4));
-                        vb[j] = *reinterpret_cast<const uint4*>(src + (((2 * (c & 3) + 1) ^ (r & 7)) << 4));
-                    }
-                }
-                named_sync(2, C::kSplitThreads);
 #pragma unroll
                 for (int j = 0; j < C::kUnits; ++j) {
                     const int u = ct + 256 * j, r = u >> 3, c = u & 7;
                     if (r < t.mma_n) {  // rows past the chunk's own: zero codes
                         uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-                        if (r < t.nrows) split_f16x16_e4m3(va[j], vb[j], inv[j], hi, lo);
+                        if (r < t.nrows) split_f16x16_e4m3(va[j], vb[j], ex[j], hi, lo);
                         const int off = r * 128 + ((c ^ (r & 7)) << 4);
                         *reinterpret_cast<uint4*>(xt + off) = hi;
                         *reinterpret_cast<uint4*>(xt + box_off + off) = lo;
@@ -818,42 +853,51 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 if (finished) {
                     __threadfence();
                     const long long slot0 = it.slot - it.slice;  // slot of slice 0 of this tile
-                    for (int c0 = 0; c0 < t.nrows; c0 += 16) {
-                        float g[16], u[16];
+                    // acc = sum over slices, in slice order, of one accumulator's 16
+                    // columns: this slice's from TMEM, the others' from their slots,
+                    // loaded kSumBatch slices at a time so their L2 round trips overlap
+                    auto sum_slices = [&](int c0, int col, bool valid, float (&acc)[16]) {
+                        constexpr int kSumBatch = kFp8 ? 2 : 4;  // (FP8: 448 threads, 128 registers each)
+                        float own[16];
+                        ld_acc(tacc + (col ? C::kUOff : 0) + c0, own);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
-                        for (int sl = 0; sl < it.S; ++sl) {
-                            if (sl == it.slice) {
-                                float v[16];
-                                ld_acc(tacc + c0, v);
+                        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                        for (int sl0 = 0; sl0 < it.S; sl0 += kSumBatch) {
+                            float4 a4[kSumBatch][4];
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) g[i] += v[i];
-                                ld_acc(tacc + C::kUOff + c0, v);
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) u[i] += v[i];
-                            } else {
+                            for (int j = 0; j < kSumBatch; ++j) {
+                                const int sl = sl0 + j;
                                 const float4* other =
                                     reinterpret_cast<const float4*>(p.partials + (slot0 + sl) * C::kSlotFloats);
-                                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-                                float4 a4[4], b4[4];
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    a4[q] = v0 ? __ldcg(other + slot_f4((c0 >> 2) + q, r)) : z;
-                                    b4[q] = v1 ? __ldcg(other + slot_f4(((kMaxN + c0) >> 2) + q, r)) : z;
-                                }
+                                for (int q = 0; q < 4; ++q)
+                                    a4[j][q] = valid && sl < it.S && sl != it.slice
+                                                   ? __ldcg(other + slot_f4(((col + c0) >> 2) + q, r))
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    g[4 * q] += a4[q].x;
-                                    g[4 * q + 1] += a4[q].y;
-                                    g[4 * q + 2] += a4[q].z;
-                                    g[4 * q + 3] += a4[q].w;
-                                    u[4 * q] += b4[q].x;
-                                    u[4 * q + 1] += b4[q].y;
-                                    u[4 * q + 2] += b4[q].z;
-                                    u[4 * q + 3] += b4[q].w;
+                            for (int j = 0; j < kSumBatch; ++j) {
+                                const int sl = sl0 + j;
+                                if (sl >= it.S) break;
+                                if (sl == it.slice) {
+#pragma unroll
+                                    for (int i = 0; i < 16; ++i) acc[i] += own[i];
+                                } else {
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        acc[4 * q] += a4[j][q].x;
+                                        acc[4 * q + 1] += a4[j][q].y;
+                                        acc[4 * q + 2] += a4[j][q].z;
+                                        acc[4 * q + 3] += a4[j][q].w;
+                                    }
                                 }
                             }
                         }
+                    };
+                    for (int c0 = 0; c0 < t.nrows; c0 += 16) {
+                        float g[16], u[16];
+                        sum_slices(c0, 0, v0, g);
+                        sum_slices(c0, kMaxN, v1, u);
                         emit(c0, g, u);
                     }
                     if (r == 0) tile_ctr[it.ctr] = 0;
