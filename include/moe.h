@@ -272,11 +272,13 @@ int moe_quantize_fp8(int64_t rows, int cols, int dtype, const void* w, uint8_t* 
 /* moe_layer_forward_k with FP8 routed (and shared) expert weights: codes
  * w13_q [E,2I,H], w2_q [E,H,I] with row scales w13_s [E,2I], w2_s [E,H]
  * (shared likewise, [2*I_sh,H] / [H,I_sh] with [2*I_sh] / [H]); x, the router
- * and the output stay bf16 (cfg->dtype 0).  The codes stream from HBM and are
- * widened to f16 in tensor memory (exact); the expert MMAs run on f16
- * operands (x and the SwiGLU activations converted to f16, so |x| and the
- * activations must stay within the f16 range) with fp32 accumulation, and
- * each output row is multiplied by its fp32 scale.  Decode sizes only: the expert FFNs
+ * and the output stay bf16 (cfg->dtype 0).  The codes stream from HBM and
+ * every expert MMA is E4M3 x E4M3 with fp32 accumulation: the token rows
+ * enter split exactly into two E4M3 terms with a power-of-two row scale
+ * (moe_permute_e4m3x2), the SwiGLU activations are stored in f16 (they must
+ * stay within its range) and split the same way on chip (about 8 significant
+ * bits kept, bf16's precision); each output is multiplied by its weight
+ * row's fp32 scale and its token row's scale.  Decode sizes only: the expert FFNs
  * must run as the fused kernel (at most 128 rows per routed expert and, with
  * shared experts, T <= 128); otherwise MOE_ERR_ARG.  H, I, S*I_s multiples of
  * 16.  Same workspace as moe_layer_forward. */

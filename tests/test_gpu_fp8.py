@@ -1,9 +1,10 @@
 """FP8 expert weights on the GPU against the oracle: the row quantiser's
 codes and scales bit-exact, the token rows' exact E4M3 hi/lo split checked
 against the format's definition, and the layer with FP8 routed and shared
-weights (the fused decode FFN: E4M3 x E4M3 gate/up products, down products on
-codes widened to f16 in tensor memory) within the output bound of the bf16
-layer, against the oracle's layer computed on the same codes and scales."""
+weights (the fused decode FFN: E4M3 x E4M3 products throughout, the
+activations split into E4M3 terms on chip) within the output bound of the
+bf16 layer, against the oracle's layer computed on the same codes and
+scales."""
 import numpy as np
 import pytest
 import torch
@@ -110,7 +111,7 @@ def test_fp8_subnormal_codes_are_kept():
     # gate/up rows of one large weight (it sets the scale) and many tiny ones
     # that quantise to E4M3 subnormals; the large weights meet x = 0, so the
     # output comes from the subnormal codes alone and would vanish if the
-    # widening or the tensor core dropped them
+    # tensor core's E4M3 products dropped them
     T, H, I = 16, 256, 128
     rng = np.random.default_rng(77)
     w13 = rng.uniform(-0.03, 0.03, (2 * I, H)).astype(np.float32)
