@@ -853,42 +853,56 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 if (finished) {
                     __threadfence();
                     const long long slot0 = it.slot - it.slice;  // slot of slice 0 of this tile
-                    // acc = sum over slices, in slice order, of one accumulator's 16
-                    // columns: this slice's from TMEM, the others' from their slots,
-                    // loaded kSumBatch slices at a time so their L2 round trips overlap
-                    auto sum_slices = [&](int c0, int col, bool valid, float (&acc)[16]) {
-                        constexpr int kSumBatch = kFp8 ? 2 : 4;  // (FP8: 448 threads, 128 registers each)
-                        float own[16];
-                        ld_acc(tacc + (col ? C::kUOff : 0) + c0, own);
+                    // g / u = sums over slices, in slice order, of the two accumulators'
+                    // 16 columns: this slice's from TMEM, the others' from their slots,
+                    // requested kSumBatch slices per L2 round trip -- both accumulators
+                    // together, or (FP8: 448 threads at 128 registers each) one at a time
+                    constexpr int kSumBatch = kFp8 ? 2 : 4;
+                    constexpr int kAccs = kFp8 ? 1 : 2;  // accumulators summed per pass
+                    auto sum_pass = [&](int c0, int col, float (&acc0)[16], float (&acc1)[16]) {
+                        float own0[16], own1[16];
+                        ld_acc(tacc + (col ? C::kUOff : 0) + c0, own0);
+                        if (kAccs == 2) ld_acc(tacc + C::kUOff + c0, own1);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                        for (int i = 0; i < 16; ++i) acc0[i] = acc1[i] = 0.f;
                         for (int sl0 = 0; sl0 < it.S; sl0 += kSumBatch) {
-                            float4 a4[kSumBatch][4];
+                            float4 a4[kSumBatch][kAccs][4];
 #pragma unroll
                             for (int j = 0; j < kSumBatch; ++j) {
                                 const int sl = sl0 + j;
+                                const bool other_slice = sl < it.S && sl != it.slice;
                                 const float4* other =
                                     reinterpret_cast<const float4*>(p.partials + (slot0 + sl) * C::kSlotFloats);
 #pragma unroll
-                                for (int q = 0; q < 4; ++q)
-                                    a4[j][q] = valid && sl < it.S && sl != it.slice
-                                                   ? __ldcg(other + slot_f4(((col + c0) >> 2) + q, r))
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                                for (int h = 0; h < kAccs; ++h) {
+                                    const int cb = (h == 1 || col) ? kMaxN : 0;
+                                    const bool valid = (h == 1 || col) ? v1 : v0;
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q)
+                                        a4[j][h][q] = valid && other_slice
+                                                          ? __ldcg(other + slot_f4(((cb + c0) >> 2) + q, r))
+                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                                }
                             }
 #pragma unroll
                             for (int j = 0; j < kSumBatch; ++j) {
                                 const int sl = sl0 + j;
                                 if (sl >= it.S) break;
-                                if (sl == it.slice) {
 #pragma unroll
-                                    for (int i = 0; i < 16; ++i) acc[i] += own[i];
-                                } else {
+                                for (int h = 0; h < kAccs; ++h) {
+                                    float* acc = h == 0 ? acc0 : acc1;
+                                    const float* own = h == 0 ? own0 : own1;
+                                    if (sl == it.slice) {
 #pragma unroll
-                                    for (int q = 0; q < 4; ++q) {
-                                        acc[4 * q] += a4[j][q].x;
-                                        acc[4 * q + 1] += a4[j][q].y;
-                                        acc[4 * q + 2] += a4[j][q].z;
-                                        acc[4 * q + 3] += a4[j][q].w;
+                                        for (int i = 0; i < 16; ++i) acc[i] += own[i];
+                                    } else {
+#pragma unroll
+                                        for (int q = 0; q < 4; ++q) {
+                                            acc[4 * q] += a4[j][h][q].x;
+                                            acc[4 * q + 1] += a4[j][h][q].y;
+                                            acc[4 * q + 2] += a4[j][h][q].z;
+                                            acc[4 * q + 3] += a4[j][h][q].w;
+                                        }
                                     }
                                 }
                             }
@@ -896,8 +910,13 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                     };
                     for (int c0 = 0; c0 < t.nrows; c0 += 16) {
                         float g[16], u[16];
-                        sum_slices(c0, 0, v0, g);
-                        sum_slices(c0, kMaxN, v1, u);
+                        if (kAccs == 2) {
+                            sum_pass(c0, 0, g, u);
+                        } else {
+                            float unused[16];
+                            sum_pass(c0, 0, g, unused);
+                            sum_pass(c0, kMaxN, u, unused);
+                        }
                         emit(c0, g, u);
                     }
                     if (r == 0) tile_ctr[it.ctr] = 0;
