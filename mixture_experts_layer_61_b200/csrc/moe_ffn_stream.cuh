@@ -747,17 +747,30 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                     sc1 = v1 ? __ldg(sr + f + 128) : 0.f;
                 }
             }
+            // FP8: the token rows' scales, one column per lane (column 32 j + lane
+            // in tsc[j]), read once per item for real rows only: the split of x
+            // (gate/up), or the one the splitters took from the row's maximum
+            // activation (down; the MMAs are done, so its chunk's maxima are final)
+            constexpr int kTsc = kFp8 ? kMaxN / 32 : 1;
+            float tsc[kTsc];
+#pragma unroll
+            for (int j = 0; j < kTsc; ++j) {
+                const int c = 32 * j + lane;
+                tsc[j] = 1.f;
+                if (kFp8 && c < t.nrows)
+                    tsc[j] = gate_up ? __ldg(p.x_scale + t.row0 + c)
+                                     : e4m3_pow2_scale(__uint_as_float(__ldcg(act_amax + t.row0 + c)));
+            }
             auto emit = [&](int c0, float (&g)[16], float (&u)[16]) {
                 if constexpr (kFp8) {
+                    // columns c0 .. c0 + 15 sit in one register of the lanes (c0 & 31) + i
+                    float base = tsc[0];
+#pragma unroll
+                    for (int j = 1; j < kTsc; ++j)
+                        if (j == (c0 >> 5)) base = tsc[j];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        // the token row's scale, read for real rows only: the split of x
-                        // (gate/up), or the one the splitters took from the row's maximum
-                        // activation (down)
-                        float xs = 1.f;
-                        if (c0 + i < t.nrows)
-                            xs = gate_up ? __ldg(p.x_scale + t.row0 + c0 + i)
-                                         : e4m3_pow2_scale(__uint_as_float(__ldcg(act_amax + t.row0 + c0 + i)));
+                        const float xs = __shfl_sync(0xffffffffu, base, (c0 & 31) + i);
                         g[i] *= sc0 * xs;
                         u[i] *= sc1 * xs;
                     }
