@@ -107,9 +107,10 @@ struct Layout {
 };
 
 int routed_max_n(const moe_config_t* c);
+int routed_max_n_avg(const moe_config_t* c);
 
 // FP8 expert weights run at decode sizes only (the fused expert FFN)
-bool fp8_sized(const moe_config_t* c) { return c->dtype == 0 && routed_max_n(c) <= 128; }
+bool fp8_sized(const moe_config_t* c) { return c->dtype == 0 && routed_max_n_avg(c) <= 128; }
 
 Layout layout(const moe_config_t* c, int num_sms) {
     Layout L;
@@ -325,7 +326,25 @@ void router_tiling(GemmLaunch& g, int T) {
     g.max_split = 8;
 }
 
-int routed_max_n(const moe_config_t* c) { return pick_max_n((double)c->T * c->K / (double)c->E); }
+// The routed experts' token tile: by the average rows per expert (the FP8
+// path, and every layer but the one case below) ...
+int routed_max_n_avg(const moe_config_t* c) { return pick_max_n((double)c->T * c->K / (double)c->E); }
+
+// ... except that bf16 layers of large experts (H I >= 2^25) whose largest
+// expert is expected past the fused FFN's 128-row chunk (binomial rows under
+// uniform routing: mean + 2.5 standard deviations) take the 256-token
+// CTA-pair GEMMs: there the fused kernel, MMA-issue-bound at 128 rows, would
+// stream and issue a whole large expert once more for each remainder chunk
+// (Mixtral-shaped layer at 128 rows per expert: 0.619 ms fused, 0.573 ms
+// pairs; at 96 rows 0.509 fused, 0.556 pairs; Qwen2-MoE's small experts at
+// 128 rows: 1.152 fused, 1.172 pairs).
+int routed_max_n(const moe_config_t* c) {
+    const int n = routed_max_n_avg(c);
+    if (n != 128 || c->dtype != 0 || token_tile_cap() != 0) return n;
+    const double A = (double)c->T * c->K, pe = 1.0 / c->E;
+    const double hi = A * pe + 2.5 * std::sqrt(A * pe * (1.0 - pe));
+    return (double)c->H * c->I >= 33554432.0 && hi > 128.0 ? 256 : n;
+}
 
 // Upper bounds on the token chunks of the routed segments (every chunk holds
 // at least one 16-row unit) and of a dense segment of T rows.
@@ -482,12 +501,12 @@ int moe_grouped_ffn_fp8(const moe_config_t* cfg, const uint8_t* x_codes, const f
     if (!aligned16(x_codes) || !aligned16(w13_q) || !aligned16(w2_q) || !aligned16(act) || !aligned16(y_perm) ||
         !aligned16(workspace))
         return MOE_ERR_ARG;
-    if (routed_max_n(cfg) > 128) return MOE_ERR_ARG;
+    if (routed_max_n_avg(cfg) > 128) return MOE_ERR_ARG;
     DeviceInfo d;
     if ((rc = current_device(&d)) != 0) return status_of(rc);
     if (ws_bytes < ctl_block_bytes(d.num_sms)) return MOE_ERR_WORKSPACE;
     return status_of(run_ffn(x_codes, p_max(cfg), offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13_q, w2_q, act,
-                             y_perm, routed_max_n(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream,
+                             y_perm, routed_max_n_avg(cfg), gemm_ctl(workspace, d.num_sms), (cudaStream_t)stream,
                              routed_max_chunks(cfg), 0, 0, w13_s, w2_s, x_scales));
 }
 
@@ -576,7 +595,7 @@ int moe_layer_forward_fp8(const moe_config_t* cfg, const void* x, const void* w_
     if (!w13_s || !w2_s || (I_sh > 0 && (!w13_shared_s || !w2_shared_s))) return MOE_ERR_ARG;
     if (cfg->H % 16 || cfg->I % 16 || I_sh % 16) return MOE_ERR_ARG;  // 16-byte rows of codes
     // decode sizes: the routed and shared FFNs must run on the fused kernel
-    if (routed_max_n(cfg) > 128 || (I_sh > 0 && pick_max_n(cfg->T) > 128)) return MOE_ERR_ARG;
+    if (routed_max_n_avg(cfg) > 128 || (I_sh > 0 && pick_max_n(cfg->T) > 128)) return MOE_ERR_ARG;
     const Fp8Scales sc{w13_s, w2_s, w13_shared_s, w2_shared_s};
     return layer_forward_impl(cfg, x, w_router, w13_q, w2_q, w13_shared_q, w2_shared_q, &sc, logits_override,
                               k_per_token, out, workspace, ws_bytes, stats_out, stream);
@@ -765,7 +784,8 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
         g.sms = n_routed;
         if ((rc = launch_gemm(g, ctl, s)) != 0) return status_of(rc);
     } else if ((rc = run_ffn(x_perm, P, offsets, cfg->E, 0, cfg->H, cfg->I, cfg->dtype, w13, w2, act, y_perm,
-                             routed_max_n(cfg), ctl, s, routed_max_chunks(cfg), n_routed, n_routed_ffn,
+                             fp8 ? routed_max_n_avg(cfg) : routed_max_n(cfg), ctl, s, routed_max_chunks(cfg),
+                             n_routed, n_routed_ffn,
                              fp8 ? fp8->s13 : nullptr, fp8 ? fp8->s2 : nullptr,
                              fp8 ? at<float>(workspace, L.x_scale) : nullptr)) != 0) {
         return status_of(rc);

@@ -286,6 +286,7 @@ int g_split_tail = 1;      // aligned k-slices for the last partial wave
 }
 
 void set_token_tile_cap(int n) { g_token_tile_cap = n; }
+int token_tile_cap() { return g_token_tile_cap; }
 void set_split_tail(int mode) { g_split_tail = mode; }
 int split_tail_mode() { return g_split_tail; }
 void set_cta_pairs(bool on) { g_cta_pairs = on; }

@@ -137,6 +137,7 @@ int launch_ffn_stream(const FfnLaunch& L, const GemmCtl& ctl, cudaStream_t strea
 // by set_token_tile_cap, 0 = automatic).
 int pick_max_n(double rows_per_group);
 void set_token_tile_cap(int n);
+int token_tile_cap();  // the forced cap, 0 = automatic
 // How the GEMM shares out the tiles after its whole data-parallel waves:
 // 0 contiguous stream-K over the last one to two waves, 1 aligned k-slices of
 // the last partial wave (default).

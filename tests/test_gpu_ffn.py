@@ -231,3 +231,27 @@ def test_dense_ffn_split_tail_modes(split_tail_mode, T, H, I):
     tok = sample_tokens(T, 64, seed=T)
     ref = oracle.dense_ffn(host(x)[tok], host(w13), host(w2))
     assert rel_err(out.float().cpu().numpy()[tok], ref) < OUT_TOL
+
+
+def test_routed_path_policy_for_large_experts():
+    # bf16 layers of large experts whose largest expert is expected past the
+    # fused FFN's 128-row chunk take the CTA-pair GEMMs; smaller experts and
+    # fewer rows keep the fused kernel; FP8 weights always run fused
+    m = mi.SHAPES["mixtral"]
+    assert not moe.ffn_fused(cfg_for(m, 512))   # 128 rows per expert on average, ~154 at the largest
+    assert moe.ffn_fused(cfg_for(m, 384))       # 96 on average
+    assert moe.ffn_fused(cfg_for(mi.SHAPES["qwen2moe"], 1024))  # small experts at 128 rows
+    moe.set_token_tile_cap(128)                 # a forced cap is kept
+    try:
+        assert moe.ffn_fused(cfg_for(m, 512))
+    finally:
+        moe.set_token_tile_cap(0)
+    T = 512
+    w = mi.make_weights(m, 5, device="cuda", shared=False)
+    x = mi.make_x(m, T, 5, device="cuda")
+    cfg = cfg_for(m, T)
+    q13, s13 = moe.quantize_fp8(w["w13"])
+    q2, s2 = moe.quantize_fp8(w["w2"])
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    moe.layer_forward_fp8(cfg, x, w["w_r"], q13, s13, q2, s2, ws)
+    moe.check_status(ws)
