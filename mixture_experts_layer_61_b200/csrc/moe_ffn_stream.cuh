@@ -704,7 +704,11 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
         while (true) {
             const int rs = n % kFfnRing;
             const uint32_t rph = (n / kFfnRing) & 1u;
-            if (!mbar_wait_bounded(&ring_full[rs], rph, limit, abort_flag)) {
+            // every wait ends in an agreement of the 128 epilogue threads: all go
+            // on or all leave (the split path meets at named barriers, which a
+            // thread that left would never reach)
+            const bool got_item = mbar_wait_bounded(&ring_full[rs], rph, limit, abort_flag);
+            if (!named_all(1, 128, got_item)) {
                 *abort_flag = 1;
                 atomicOr(p.status, kStatusTimeout);
                 break;
@@ -718,7 +722,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             item_of(id, it, t);
             const int b = ac % C::kNumAcc;
             const uint32_t aph = (ac / C::kNumAcc) & 1u;
-            if (!mbar_wait_bounded(&tfull[b], aph, limit, abort_flag)) {
+            const bool got_acc = mbar_wait_bounded(&tfull[b], aph, limit, abort_flag);
+            if (!named_all(1, 128, got_acc)) {
                 *abort_flag = 1;
                 atomicOr(p.status, kStatusTimeout);
                 break;

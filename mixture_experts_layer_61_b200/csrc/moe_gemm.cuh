@@ -574,7 +574,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             Tile t = decode_tile(it.tile, seg, cbase, n_groups, NF, C::kFeatTile, C::kUnit, p);
             const int b = ac % C::kNumAcc;
             const uint32_t aph = (ac / C::kNumAcc) & 1u;
-            if (!mbar_wait_bounded(&tfull[b], aph, deadline, abort_flag)) {
+            // every epilogue thread goes on, or all leave (the split path below
+            // meets at named barriers, which a thread that left would never reach)
+            const bool got = mbar_wait_bounded(&tfull[b], aph, deadline, abort_flag);
+            if (!named_all(1, kEpiThreads, got)) {
                 *abort_flag = 1;
                 atomicOr(p.status, kStatusTimeout);
                 break;
