@@ -236,3 +236,35 @@ def test_fp8_repeated_forwards_are_identical(name, T):
     # the two entry paths may cut the tiles into different K-slices (their own
     # SM counts), so they agree within the output bound, not bit for bit
     assert rel_err(first.float().cpu().numpy(), ref.float().cpu().numpy()) < OUT_TOL
+
+
+def test_fp8_wait_timeout_is_reported_and_recoverable():
+    # the FP8 kernel's abort path: a withheld operand load makes one block's
+    # bounded wait run out (20 ms); every role (producer, MMA thread, activation
+    # splitters, epilogue) winds down, the status reads MOE_ERR_TIMEOUT, the
+    # control words (the per-row activation maxima among them) are zero again
+    # and the next call reproduces the reference bit for bit
+    shape = small_shape(H=512, E=8, K=2, I=512, I_sh=256)
+    T = 40
+    w = mi.make_weights(shape, 8, device="cuda")
+    x = mi.make_x(shape, T, 8, device="cuda")
+    cfg = cfg_for(shape, T)
+    q = _fp8_weights(w)
+    ws = moe.alloc_workspace(moe.workspace_size(cfg))
+    sh = dict(q13_sh=q["w13_sh"][0], s13_sh=q["w13_sh"][1], q2_sh=q["w2_sh"][0], s2_sh=q["w2_sh"][1])
+    fwd = lambda: moe.layer_forward_fp8(cfg, x, w["w_r"], q["w13"][0], q["w13"][1], q["w2"][0], q["w2"][1], ws, **sh)
+    ref = fwd().clone()
+    moe.check_status(ws)
+    moe.set_wait_limit_ns(20_000_000)
+    try:
+        moe.debug_withhold_first_load(True)
+        fwd()
+        with pytest.raises(moe.MoeError) as e:
+            moe.check_status(ws)
+        assert e.value.code == -4
+    finally:
+        moe.debug_withhold_first_load(False)
+        moe.set_wait_limit_ns(0)
+    out = fwd()
+    moe.check_status(ws)
+    assert torch.equal(out, ref)
