@@ -27,14 +27,33 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
     return v > bv || (v == bv && i < bi);
 }
 
-// One warp per token.  Lane l owns experts l, l+32, ...; kt passes of a warp
-// arg-max over the experts not yet taken (kt = K, or the token's own count
-// 0..K under per-token dynamic K; slots kt..K-1 get id -1 and weight 0).
-// Logits are read through L2 (they may have been written by other blocks of
-// the same kernel).
-__device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int E, int K, int kt, int score_fn,
-                                               int renorm, int32_t* __restrict__ ids_t, float* __restrict__ w_t,
-                                               int lane) {
+// One warp per token.  Lane l owns experts l, l+32, ... (at most kPL of them,
+// E <= 32 kPL), read through L2 (they may have been written by other blocks
+// of the same kernel): once into registers, or (kStream, for the largest E in
+// kernels with few registers per thread) again on every pass, all of a lane's
+// loads issued together; kt passes of a warp arg-max over the experts not yet
+// taken (kt = K, or the token's own count 0..K under per-token dynamic K;
+// slots kt..K-1 get id -1 and weight 0).
+template <int kPL, bool kStream = false>
+__device__ __forceinline__ void topk_one_token_r(const float* __restrict__ l, int E, int K, int kt, int score_fn,
+                                                 int renorm, int32_t* __restrict__ ids_t, float* __restrict__ w_t,
+                                                 int lane) {
+    float lv[kStream ? 1 : kPL];
+    if constexpr (!kStream) {
+#pragma unroll
+        for (int j = 0; j < kPL; ++j) {
+            const int e = lane + 32 * j;
+            lv[j] = e < E ? __ldcg(l + e) : 0.f;
+        }
+    }
+    auto val = [&](int j) -> float {
+        if constexpr (kStream)
+            return __ldcg(l + lane + 32 * j);
+        else
+            return lv[j];
+    };
+    // the register variant unrolls fully; the streaming one four loads at a time
+    constexpr int kU = kStream ? 4 : kPL;
     uint32_t taken = 0;  // bit j: expert lane + 32 j
     float sel_v[16];
     int sel_i[16];
@@ -42,12 +61,15 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int 
     for (int k = 0; k < kt; ++k) {
         float bv = -INFINITY;
         int bi = INT_MAX;
-        for (int j = 0, e = lane; e < E; ++j, e += 32) {
-            if ((taken >> j) & 1u) continue;
-            const float v = __ldcg(l + e);
-            if (better(v, e, bv, bi)) {
-                bv = v;
-                bi = e;
+#pragma unroll kU
+        for (int j = 0; j < kPL; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E && !((taken >> j) & 1u)) {
+                const float v = val(j);
+                if (better(v, e, bv, bi)) {
+                    bv = v;
+                    bi = e;
+                }
             }
         }
 #pragma unroll
@@ -63,15 +85,23 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int 
             // only NaN logits remain: take the lowest expert not yet taken so
             // that every id stays in range
             int cand = INT_MAX;
-            for (int j = 0, e = lane; e < E; ++j, e += 32)
-                if (!((taken >> j) & 1u)) {
-                    cand = e;
-                    break;
-                }
+#pragma unroll
+            for (int j = kPL - 1; j >= 0; --j) {
+                const int e = lane + 32 * j;
+                if (e < E && !((taken >> j) & 1u)) cand = e;
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
             bi = cand;
-            bv = __ldcg(l + bi);
+            if constexpr (kStream) {
+                bv = __ldcg(l + bi);
+            } else {
+                float mine = lv[0];
+#pragma unroll
+                for (int j = 1; j < kPL; ++j)
+                    if (j == (bi >> 5)) mine = lv[j];
+                bv = __shfl_sync(0xffffffffu, mine, bi & 31);
+            }
         }
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
         sel_v[k] = bv;
@@ -87,11 +117,15 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int 
             for (int k = 0; k < kt; ++k) den += expf(sel_v[k] - m);
         } else {
             m = -INFINITY;
-            for (int e = lane; e < E; e += 32) m = fmaxf(m, __ldcg(l + e));
+#pragma unroll kU
+            for (int j = 0; j < kPL; ++j)
+                if (lane + 32 * j < E) m = fmaxf(m, val(j));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             float part = 0.f;
-            for (int e = lane; e < E; e += 32) part += expf(__ldcg(l + e) - m);
+#pragma unroll kU
+            for (int j = 0; j < kPL; ++j)
+                if (lane + 32 * j < E) part += expf(val(j) - m);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
             den = part;
@@ -114,6 +148,24 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int 
         ids_t[lane] = id;
         w_t[lane] = wk;
     }
+}
+
+// The same for any E <= 1024: the register count sized by E (E > 512 reloads).
+__device__ __forceinline__ void topk_one_token(const float* __restrict__ l, int E, int K, int kt, int score_fn,
+                                               int renorm, int32_t* __restrict__ ids_t, float* __restrict__ w_t,
+                                               int lane) {
+    if (E <= 32)
+        topk_one_token_r<1>(l, E, K, kt, score_fn, renorm, ids_t, w_t, lane);
+    else if (E <= 64)
+        topk_one_token_r<2>(l, E, K, kt, score_fn, renorm, ids_t, w_t, lane);
+    else if (E <= 128)
+        topk_one_token_r<4>(l, E, K, kt, score_fn, renorm, ids_t, w_t, lane);
+    else if (E <= 256)
+        topk_one_token_r<8>(l, E, K, kt, score_fn, renorm, ids_t, w_t, lane);
+    else if (E <= 512)
+        topk_one_token_r<16>(l, E, K, kt, score_fn, renorm, ids_t, w_t, lane);
+    else
+        topk_one_token_r<32, true>(l, E, K, kt, score_fn, renorm, ids_t, w_t, lane);
 }
 
 // The token's expert count: K, or k_per_token[t] clamped to [0, K].
@@ -684,8 +736,8 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
             if (lane == e) logits[(size_t)t * kE + e] = acc[e];
         __syncwarp();  // the row is complete before the warp reads it back
         const float* src = logits_override ? logits_override + (size_t)t * kE : logits + (size_t)t * kE;
-        topk_one_token(src, kE, K, token_k(k_per_token, t, K), score_fn, renorm, ids + (size_t)t * K,
-                       w + (size_t)t * K, lane);
+        topk_one_token_r<(kE + 31) / 32>(src, kE, K, token_k(k_per_token, t, K), score_fn, renorm,
+                                         ids + (size_t)t * K, w + (size_t)t * K, lane);
     }
     __threadfence();
     __syncthreads();
