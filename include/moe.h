@@ -105,10 +105,10 @@ size_t moe_workspace_size(const moe_config_t* cfg);
 
 /* Byte offset, inside the moe_layer_forward workspace, of the fp32 router
  * logits [T,E] the last forward computed (-1 on a bad configuration).  For
- * T <= 64 the forward computes them on the CUDA cores (fp32 sums of exact
- * products) in the same launch as top-K and alignment, otherwise as
- * moe_router_gemm does; either way they are what top-K selected on unless
- * logits_override was given. */
+ * T <= 64 and a small router matrix (E * H <= 2^17) the forward computes them
+ * on the CUDA cores (fp32 sums of exact products) in the same launch as top-K
+ * and alignment, otherwise as moe_router_gemm does; either way they are what
+ * top-K selected on unless logits_override was given. */
 int64_t moe_layer_logits_offset(const moe_config_t* cfg);
 
 /* Bytes of workspace moe_router_gemm / moe_grouped_ffn / dense_ffn need (the

@@ -109,6 +109,11 @@ struct Layout {
 int routed_max_n(const moe_config_t* c);
 int routed_max_n_avg(const moe_config_t* c);
 
+// The layer's routing runs as one small-batch launch (route_small_kernel).
+bool small_route(const moe_config_t* c) {
+    return c->T <= kSmallRouteMaxT && c->H % 8 == 0 && (long long)c->E * c->H <= kSmallRouteMaxEH;
+}
+
 // FP8 expert weights run at decode sizes only (the fused expert FFN)
 bool fp8_sized(const moe_config_t* c) { return c->dtype == 0 && routed_max_n_avg(c) <= 128; }
 
@@ -129,7 +134,7 @@ Layout layout(const moe_config_t* c, int num_sms) {
     L.ctl_sh = take(I_sh > 0 ? ctl_block_bytes(num_sms) : 0);
     L.logits = take(sizeof(float) * (size_t)c->T * c->E);
     // partial router sums of the small-batch routing kernel (slices of 256 hidden elements)
-    L.route_part = take(c->T <= kSmallRouteMaxT ? sizeof(float) * ((size_t)c->H / 256 + 1) * c->T * c->E : 0);
+    L.route_part = take(small_route(c) ? sizeof(float) * ((size_t)c->H / 256 + 1) * c->T * c->E : 0);
     L.ids = take(sizeof(int32_t) * (size_t)A);
     L.w = take(sizeof(float) * (size_t)A);
     L.counts = take(sizeof(int32_t) * (size_t)c->E);
@@ -702,7 +707,7 @@ static int layer_forward_impl(const moe_config_t* cfg, const void* x, const void
     // keeps to its share, so that the shared down GEMM finds its SMs free.
     const int n_routed = side ? d.num_sms - n_sh : 0;
     const int n_routed_ffn = side && pick_max_n(cfg->T) > 128 ? n_routed : 0;
-    if (cfg->T <= kSmallRouteMaxT && cfg->H % 8 == 0) {
+    if (small_route(cfg)) {
         // router logits, top-K and alignment in one launch (decode-sized batches)
         int* route_ctr = reinterpret_cast<int*>(at<uint8_t>(workspace, L.ctl)) + 16;  // in the control header
         if ((rc = launch_route_small(cfg->T, cfg->H, cfg->E, cfg->K, cfg->score_fn, cfg->renorm, cfg->tile_B,
