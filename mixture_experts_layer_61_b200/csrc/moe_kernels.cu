@@ -250,6 +250,122 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
 constexpr int kAlignFastItems = 16;   // assignments per lane on the fast path
 constexpr int kAlignFastMaxE = 512;   // [32][E] int table within the shared-memory budget
 
+// The same alignment for at most 32 x kAlignTinyItems assignments, by warp 0
+// alone (no block barrier; the other warps have nothing to do): lane l holds
+// assignments l, l + 32, ...; ranks inside an expert follow the assignment
+// index, as in align_block.
+constexpr int kAlignTinyItems = 4;
+__device__ __forceinline__ void align_warp(int A, int E, int B, int mode, long long P_max, const int32_t* ids,
+                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                           int32_t* __restrict__ sorted_ids, int32_t* __restrict__ block_expert,
+                                           int32_t* __restrict__ pos, int32_t* __restrict__ scalars,
+                                           int32_t* __restrict__ stats_copy, int* sm, int lane) {
+    int* run = sm;           // E: assignments per expert so far
+    int* off = run + E;      // E + 1: padded segment starts
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int e = lane; e < E; e += 32) run[e] = 0;
+    __syncwarp();
+    int bad = 0;
+    int ie[kAlignTinyItems], ir[kAlignTinyItems];
+#pragma unroll
+    for (int i = 0; i < kAlignTinyItems; ++i) {
+        const int a = lane + 32 * i;
+        // ids may come from other blocks (or warps) of the same kernel: read through L2
+        int e = a < A ? __ldcg(ids + a) : -1;
+        if ((unsigned)e >= (unsigned)E) {
+            if (e != -1) bad = 1;  // -1: an empty slot (per-token dynamic K)
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int r = (e >= 0 ? run[e] : 0) + __popc(peers & lt_mask);
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+        __syncwarp();
+        ie[i] = e;
+        ir[i] = r;
+    }
+    bad = __any_sync(0xffffffffu, bad) ? 1 : 0;
+    // padded sizes (block-wise, or every expert at the most loaded one's) and
+    // their exclusive scan, 32 experts at a time
+    long long rows = 0;
+    bool overflow = false;
+    if (mode == 1) {
+        int m = 0;
+        for (int e = lane; e < E; e += 32) m = max(m, run[e]);
+        m = __reduce_max_sync(0xffffffffu, m);
+        rows = ((long long)m + B - 1) / B * B;
+        overflow = (long long)E * rows > P_max;
+        if (overflow) bad |= 2;
+    }
+    int carry = 0, n_active = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int n = e < E ? run[e] : 0;
+        int v = e < E ? (mode == 1 ? (overflow ? 0 : (int)rows) : (n + B - 1) / B * B) : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (e < E) {
+            off[e] = carry + incl - v;
+            counts[e] = n;
+            offsets[e] = carry + incl - v;
+        }
+        n_active += __popc(__ballot_sync(0xffffffffu, e < E && n > 0));
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const int P = carry;
+    if (overflow) n_active = 0;
+    if (lane == 0) {
+        off[E] = P;
+        offsets[E] = P;
+        scalars[0] = P;
+        scalars[1] = n_active;
+        scalars[2] = bad;
+        scalars[3] = 0;
+        if (stats_copy) {
+            stats_copy[0] = P;
+            stats_copy[1] = n_active;
+            stats_copy[2] = bad;
+            stats_copy[3] = 0;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kAlignTinyItems; ++i) {
+        const int a = lane + 32 * i;
+        if (ie[i] >= 0 && !overflow) {
+            const int p = off[ie[i]] + ir[i];
+            sorted_ids[p] = (int32_t)a;
+            pos[a] = p;
+        } else if (a < A) {
+            pos[a] = -1;  // empty slot (or an out-of-range id, flagged above)
+        }
+    }
+    // padding slots inside each segment, then everything past P
+    if (!overflow)
+        for (int e = lane; e < E; e += 32)
+            for (int p = off[e] + run[e]; p < off[e + 1]; ++p) sorted_ids[p] = -1;
+    for (long long p = (long long)P + lane; p < P_max; p += 32) sorted_ids[p] = -1;
+    const long long nblk = (P_max + B - 1) / B;
+    for (long long b = lane; b < nblk; b += 32) {
+        const long long p = b * B;
+        int r = -1;
+        if (p < P) {
+            int lo = 0, hi = E - 1;  // largest e with off[e] <= p
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (off[mid] <= p) lo = mid;
+                else hi = mid - 1;
+            }
+            r = lo;
+        }
+        block_expert[b] = r;
+    }
+}
+
 __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode, long long P_max, const int32_t* ids,
                                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                             int32_t* __restrict__ sorted_ids, int32_t* __restrict__ block_expert,
@@ -266,6 +382,12 @@ __device__ __forceinline__ void align_block(int T, int K, int E, int B, int mode
     int* wt = nmax + 1;                                       // fast path: 32 x E running counts
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long A = (long long)T * K;
+    if (A <= 32LL * kAlignTinyItems) {  // a handful of assignments: one warp, no block barrier
+        if (warp == 0)
+            align_warp((int)A, E, B, mode, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars,
+                       stats_copy, sm, lane);
+        return;
+    }
     const unsigned lt_mask = (1u << lane) - 1u;
     const bool fast = A <= (long long)kAlignFastItems * kAlignThreads && E <= kAlignFastMaxE;
     // fast path: item i of this lane is assignment a0 + 32 i; packed as
