@@ -52,6 +52,24 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// ------------------------------------------- cross-block hand-over
+// One thread's gpu-scope read-modify-write with acquire-release semantics.
+// Used as: every thread of the group stores its part, the group meets at a
+// block or named barrier, one thread adds; the release is cumulative over the
+// barrier, so it publishes every part the group stored before it, and (read
+// side) the group's loads after the next barrier see every part published by
+// the additions that came before.  This replaces a fence in every thread,
+// which under a full HBM stream waits microseconds per thread.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+// The release half alone, for a counter that nobody reads back here.
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

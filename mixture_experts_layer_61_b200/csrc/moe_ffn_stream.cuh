@@ -16,10 +16,15 @@
 // a phase has fewer tiles than about twice the SMs, each tile is cut into S
 // K-slices; the slice that completes a tile last (per-tile counter) sums all
 // slices' fp32 partials in slice order (deterministic) and runs the epilogue.
-// A phase-B item reads the SwiGLU activations of its token chunk, so before
-// loading them its producer waits (bounded) until every phase-A tile of that
-// chunk has been stored (per-chunk counter).  No block waits on work that is
-// not already held by a running block, so the wait always ends.
+// A phase-B item reads the SwiGLU activations of its token chunk over its
+// k-slice of features, so before loading them its producer waits (bounded)
+// until the phase-A tiles that produce those features have been stored: a
+// chunk's gate/up feature blocks count in kFfnBands bands, and the item waits
+// for the bands its slice overlaps (FP8: all of them, as its activation split
+// takes each row's maximum over every feature).  Within a token chunk the
+// phase-B items go slice by slice, so the slices that need the chunk's last
+// gate/up tiles come last.  No block waits on work that is not already held
+// by a running block, so the wait always ends.
 //
 // Roles as in the grouped GEMM (warp 0 TMA, warp 1 TMEM + MMA, warps 2..5
 // epilogue); the producer publishes each item id to the other roles through a
@@ -55,7 +60,8 @@
 
 namespace moe {
 
-constexpr int kFfnMaxChunks = 4096;   // token chunks (per-chunk phase-A counters)
+constexpr int kFfnMaxChunks = 4096;   // token chunks
+constexpr int kFfnBands = 8;          // phase-A counters per chunk (bands of its gate/up feature blocks)
 constexpr int kFfnTileCtrs = 4096;    // split-tile counters (phase A, then phase B)
 constexpr int kFfnRing = 4;
 constexpr int kFfnMaxRows = 1 << 17;  // token rows of an FP8 launch (per-row activation maxima)
@@ -63,7 +69,7 @@ constexpr int kFfnMaxRows = 1 << 17;  // token rows of an FP8 launch (per-row ac
 // counters, then kFfnTileCtrs tile counters, then (16-byte aligned, for the
 // bulk copies) the FP8 path's per-row activation maxima (fp32 bits) with a
 // margin for the copies' rounding to 16 bytes
-constexpr int kFfnAmaxOff = (2 + kFfnMaxChunks + kFfnTileCtrs + 63) / 64 * 64;
+constexpr int kFfnAmaxOff = (2 + kFfnMaxChunks * kFfnBands + kFfnTileCtrs + 63) / 64 * 64;
 constexpr int kFfnCtlInts = kFfnAmaxOff + kFfnMaxRows + 256;
 
 struct FfnParams {
@@ -265,8 +271,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     const uint64_t limit = p.wait_limit_ns;
     int* work_ctr = p.ctl;
     int* done_ctr = p.ctl + 1;
-    int* chunk_done = p.ctl + 2;
-    int* tile_ctr = p.ctl + 2 + kFfnMaxChunks;
+    int* band_done = p.ctl + 2;  // [chunk][band]: gate/up tiles stored
+    int* tile_ctr = p.ctl + 2 + kFfnMaxChunks * kFfnBands;
     unsigned* act_amax = reinterpret_cast<unsigned*>(p.ctl + kFfnAmaxOff);  // FP8: per-row max |activation|
 
     pdl_launch_dependents();
@@ -328,6 +334,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     const int G = gridDim.x;
     const long long n_chunks = cbase[n_groups];
     const int NFA = (p.I + 127) / 128, NFB = (p.H + 255) / 256;
+    const int BS = (NFA + kFfnBands - 1) / kFfnBands;  // gate/up feature blocks per band
     const int KIA = (p.H + C::kBK - 1) / C::kBK, KIB = (p.I + C::kBK - 1) / C::kBK;
     const long long tilesA = n_chunks * NFA, tilesB = n_chunks * NFB;
     const int SA = ffn_slices(tilesA, KIA, G, p.max_slots_phase, kMaxN),
@@ -350,14 +357,20 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             it.ctr = it.tile;
             t = decode_tile_w(it.tile, seg, cbase, n_groups, NFA, 128, 16, 2 * p.I);
         } else {
+            // expert by expert (a group's tiles hold its items' range, SB per
+            // tile), and inside an expert slice by slice over its tiles
             const long long j = id - nA;
+            const Tile tg = decode_tile_w(j / SB, seg, cbase, n_groups, NFB, 256, 16, p.H);
+            const long long gt0 = (long long)cbase[tg.group] * NFB;  // the expert's first tile
+            const long long per = (long long)tg.nch * NFB;          // its tiles
+            const long long r = j - gt0 * SB;
             it.phase = 1;
-            it.tile = j / SB;
-            it.slice = (int)(j - it.tile * SB);
+            it.slice = (int)(r / per);
+            it.tile = gt0 + (r - (long long)it.slice * per);
             it.S = SB;
             it.kb = (int)((long long)it.slice * KIB / SB);
             it.ke = (int)((long long)(it.slice + 1) * KIB / SB);
-            it.slot = slotsA + j;
+            it.slot = slotsA + it.tile * SB + it.slice;
             it.ctr = kFfnTileCtrs / 2 + it.tile;
             t = decode_tile_w(it.tile, seg, cbase, n_groups, NFB, 256, 16, p.H);
         }
@@ -452,8 +465,9 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                 int pre = 0;  // stages of this item whose weight tiles went out before the activation wait
                 if (it.phase == 1) {
                     // The weights do not depend on phase A: stream the first stages'
-                    // weight tiles now, then wait until every gate/up tile of this
-                    // token chunk has stored its activations, then load those.
+                    // weight tiles now, then wait until the gate/up tiles of this
+                    // token chunk that produce the slice's features (FP8: all of
+                    // them) have stored their activations, then load those.
                     const int want = it.ke - it.kb < C::kStages ? it.ke - it.kb : C::kStages;
                     for (; pre < want; ++pre) {
                         const int s = (kc + pre) % C::kStages;
@@ -467,13 +481,21 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                         owe(s);
                     }
                     if (ok) {
+                        // the bands of the 128-feature gate/up blocks that hold
+                        // features [kb kBK, ke kBK)
+                        const int fa1 = (it.ke * C::kBK - 1) / 128;
+                        const int b0 = kFp8 ? 0 : (it.kb * C::kBK / 128) / BS;
+                        const int b1 = (kFp8 || fa1 >= NFA ? NFA - 1 : fa1) / BS;
                         const uint64_t t0 = global_ns();
-                        while ((int)ld_acquire_u32(&chunk_done[t.chunk]) < NFA) {
-                            if (*abort_flag || global_ns() - t0 > limit) {
-                                ok = false;
-                                break;
+                        for (int bd = b0; bd <= b1 && ok; ++bd) {
+                            const int need = NFA - bd * BS < BS ? NFA - bd * BS : BS;
+                            while ((int)ld_acquire_u32(&band_done[t.chunk * kFfnBands + bd]) < need) {
+                                if (*abort_flag || global_ns() - t0 > limit) {
+                                    ok = false;
+                                    break;
+                                }
+                                __nanosleep(64);
                             }
-                            __nanosleep(64);
                         }
                         if (ok) fence_proxy_async_global();
                     }
@@ -845,7 +867,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                     }
                 }
             } else {
-                // split tile: publish this slice, the last slice sums them all in order
+                // split tile: publish this slice, the last slice sums them all in
+                // order; only the columns of real token rows travel (4 at a time)
                 float4* mine = reinterpret_cast<float4*>(p.partials + it.slot * C::kSlotFloats);
                 for (int c0 = 0; c0 < t.nrows; c0 += 16) {
                     float g[16];
@@ -853,23 +876,24 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                     if (v0) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            mine[slot_f4((c0 >> 2) + q, r)] = make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                            if (c0 + 4 * q < t.nrows)
+                                mine[slot_f4((c0 >> 2) + q, r)] =
+                                    make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
                     }
                     ld_acc(tacc + C::kUOff + c0, g);
                     if (v1) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            mine[slot_f4(((kMaxN + c0) >> 2) + q, r)] =
-                                make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+                            if (c0 + 4 * q < t.nrows)
+                                mine[slot_f4(((kMaxN + c0) >> 2) + q, r)] =
+                                    make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
                     }
                 }
-                __threadfence();
                 named_sync(1, 128);
-                if (r == 0) *bcast = atomicAdd(&tile_ctr[it.ctr], 1);
+                if (r == 0) *bcast = atomic_add_acq_rel_gpu(&tile_ctr[it.ctr], 1);
                 named_sync(1, 128);
                 finished = *bcast == it.S - 1;
                 if (finished) {
-                    __threadfence();
                     const long long slot0 = it.slot - it.slice;  // slot of slice 0 of this tile
                     // g / u = sums over slices, in slice order, of the two accumulators'
                     // 16 columns: this slice's from TMEM, the others' from their slots,
@@ -897,7 +921,7 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
                                     const bool valid = (h == 1 || col) ? v1 : v0;
 #pragma unroll
                                     for (int q = 0; q < 4; ++q)
-                                        a4[j][h][q] = valid && other_slice
+                                        a4[j][h][q] = valid && other_slice && c0 + 4 * q < t.nrows
                                                           ? __ldcg(other + slot_f4(((cb + c0) >> 2) + q, r))
                                                           : make_float4(0.f, 0.f, 0.f, 0.f);
                                 }
@@ -943,9 +967,8 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
             if (gate_up && finished) {
                 // this gate/up tile's activations are stored: count it for its token chunk
                 fence_proxy_async_global();
-                __threadfence();
                 named_sync(1, 128);
-                if (r == 0) atomicAdd(&chunk_done[t.chunk], 1);
+                if (r == 0) red_add_release_gpu(&band_done[t.chunk * kFfnBands + (t.f0 / 128) / BS], 1);
             }
             tc_fence_before();
             mbar_arrive(&tempty[b]);
@@ -956,15 +979,11 @@ __global__ void __launch_bounds__(FfnCfg<T, kMaxN, kFp8>::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     // the last block to finish re-zeroes the control words for the next launch
-    if (threadIdx.x == 0) {
-        __threadfence();
-        *last_block = atomicAdd(done_ctr, 1) == (int)gridDim.x - 1;
-    }
+    if (threadIdx.x == 0) *last_block = atomic_add_acq_rel_gpu(done_ctr, 1) == (int)gridDim.x - 1;
     __syncthreads();
     if (*last_block) {
-        __threadfence();
         const long long nc = n_chunks < kFfnMaxChunks ? n_chunks : kFfnMaxChunks;
-        for (long long c = threadIdx.x; c < nc; c += blockDim.x) chunk_done[c] = 0;
+        for (long long c = threadIdx.x; c < nc * kFfnBands; c += blockDim.x) band_done[c] = 0;
         if (kFp8) {
             const int rows = seg[n_groups] < kFfnMaxRows ? seg[n_groups] : kFfnMaxRows;
             for (int r = threadIdx.x; r < rows; r += blockDim.x) act_amax[r] = 0u;

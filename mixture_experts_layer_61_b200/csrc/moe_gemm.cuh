@@ -738,9 +738,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 make_float4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
                     }
                 }
-                __threadfence();
                 named_sync(1, kEpiThreads);
-                if (e == 0) *bcast = atomicAdd(&p.counters[counter], 1);
+                if (e == 0) *bcast = atomic_add_acq_rel_gpu(&p.counters[counter], 1);
                 named_sync(1, kEpiThreads);
                 const int arrived = *bcast;
                 // contributors: blocks whose stream-K range meets this tile, or
@@ -758,7 +757,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 if (arrived == ncontrib - 1) {
                     // last to arrive: sum every contribution in block order, then the epilogue
-                    __threadfence();
                     for (int c0 = cbeg; c0 < cend; c0 += 16) {
                         float g[16], u[16];
 #pragma unroll

@@ -27,13 +27,26 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
     return v > bv || (v == bv && i < bi);
 }
 
+// Order-preserving 32-bit key of a logit: a larger value has a larger key,
+// -0 and +0 share one key, and every NaN takes key 0, below every number, so
+// a NaN logit is picked only once nothing else is left.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+    uint32_t u = __float_as_uint(v);
+    if (u == 0x80000000u) u = 0u;
+    const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return v != v ? 0u : k;
+}
+
 // One warp per token.  Lane l owns experts l, l+32, ... (at most kPL of them,
 // E <= 32 kPL), read through L2 (they may have been written by other blocks
 // of the same kernel): once into registers, or (kStream, for the largest E in
-// kernels with few registers per thread) again on every pass, all of a lane's
-// loads issued together; kt passes of a warp arg-max over the experts not yet
-// taken (kt = K, or the token's own count 0..K under per-token dynamic K;
-// slots kt..K-1 get id -1 and weight 0).
+// kernels with few registers per thread) again on every scan.  kt rounds
+// (kt = K, or the token's own count 0..K under per-token dynamic K; slots
+// kt..K-1 get id -1 and weight 0) each take the largest remaining logit, the
+// lower expert index on equal logits: every lane keeps its own best expert not
+// yet taken; a warp max of the lanes' keys, then a warp min of the expert
+// index over the lanes holding that key, name the winner, whose lane alone
+// rescans.  Lane k keeps the k-th pick and computes its weight.
 template <int kPL, bool kStream = false>
 __device__ __forceinline__ void topk_one_token_r(const float* __restrict__ l, int E, int K, int kt, int score_fn,
                                                  int renorm, int32_t* __restrict__ ids_t, float* __restrict__ w_t,
@@ -55,66 +68,58 @@ __device__ __forceinline__ void topk_one_token_r(const float* __restrict__ l, in
     // the register variant unrolls fully; the streaming one four loads at a time
     constexpr int kU = kStream ? 4 : kPL;
     uint32_t taken = 0;  // bit j: expert lane + 32 j
-    float sel_v[16];
-    int sel_i[16];
-#pragma unroll 1
-    for (int k = 0; k < kt; ++k) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
+    // this lane's best expert not yet taken: key, index (INT_MAX: none), logit
+    uint32_t bk = 0;
+    int be = INT_MAX;
+    float bv = 0.f;
+    auto rescan = [&]() {
+        bk = 0;
+        be = INT_MAX;
+        bv = 0.f;
 #pragma unroll kU
         for (int j = 0; j < kPL; ++j) {
             const int e = lane + 32 * j;
             if (e < E && !((taken >> j) & 1u)) {
                 const float v = val(j);
-                if (better(v, e, bv, bi)) {
+                const uint32_t k = logit_key(v);
+                if (be == INT_MAX || k > bk) {  // ascending j: the lower index keeps a tie
+                    bk = k;
+                    be = e;
                     bv = v;
-                    bi = e;
                 }
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (better(ov, oi, bv, bi)) {
-                bv = ov;
-                bi = oi;
-            }
+    };
+    rescan();
+    float my_v = 0.f;  // lane k < kt: the k-th pick's logit and expert
+    int my_i = -1;
+#pragma unroll 1
+    for (int k = 0; k < kt; ++k) {
+        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+        // lanes without a candidate hold INT_MAX; kt <= E leaves a real one
+        const int win = __reduce_min_sync(0xffffffffu, bk == m ? be : INT_MAX);
+        const float wv = __shfl_sync(0xffffffffu, bv, win & 31);
+        if (lane == k) {
+            my_v = wv;
+            my_i = win;
         }
-        if (bi == INT_MAX) {
-            // only NaN logits remain: take the lowest expert not yet taken so
-            // that every id stays in range
-            int cand = INT_MAX;
-#pragma unroll
-            for (int j = kPL - 1; j >= 0; --j) {
-                const int e = lane + 32 * j;
-                if (e < E && !((taken >> j) & 1u)) cand = e;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
-            bi = cand;
-            if constexpr (kStream) {
-                bv = __ldcg(l + bi);
-            } else {
-                float mine = lv[0];
-#pragma unroll
-                for (int j = 1; j < kPL; ++j)
-                    if (j == (bi >> 5)) mine = lv[j];
-                bv = __shfl_sync(0xffffffffu, mine, bi & 31);
-            }
+        if ((win & 31) == lane) {
+            taken |= 1u << (win >> 5);
+            rescan();
         }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        sel_v[k] = bv;
-        sel_i[k] = bi;
     }
-    // gate weights, identical in every lane; lane k stores entry k
+    // gate weights: lane k < kt computes its own
+    const bool mine = lane < kt;
     float wk = 0.f;
     if (score_fn == 0) {
-        float m, den = 0.f;
+        float m, den;
         if (renorm) {
-            m = kt > 0 ? sel_v[0] : 0.f;
-            for (int k = 1; k < kt; ++k) m = fmaxf(m, sel_v[k]);
-            for (int k = 0; k < kt; ++k) den += expf(sel_v[k] - m);
+            // the first pick is the largest selected logit (all NaN if it is)
+            m = __shfl_sync(0xffffffffu, my_v, 0);
+            float e = mine ? expf(my_v - m) : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+            den = e;
         } else {
             m = -INFINITY;
 #pragma unroll kU
@@ -130,22 +135,16 @@ __device__ __forceinline__ void topk_one_token_r(const float* __restrict__ l, in
             for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
             den = part;
         }
-        for (int k = 0; k < kt; ++k)
-            if (k == lane) wk = expf(sel_v[k] - m) / den;
+        if (mine) wk = expf(my_v - m) / den;
     } else {
-        float den = 0.f;
-        for (int k = 0; k < kt; ++k) den += 1.f / (1.f + expf(-sel_v[k]));
-        for (int k = 0; k < kt; ++k)
-            if (k == lane) {
-                const float s = 1.f / (1.f + expf(-sel_v[k]));
-                wk = renorm ? s / den : s;
-            }
+        const float sg = mine ? 1.f / (1.f + expf(-my_v)) : 0.f;
+        float den = sg;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        wk = renorm ? (mine ? sg / den : 0.f) : sg;
     }
     if (lane < K) {
-        int id = -1;
-        for (int k = 0; k < kt; ++k)
-            if (k == lane) id = sel_i[k];
-        ids_t[lane] = id;
+        ids_t[lane] = mine ? my_i : -1;
         w_t[lane] = wk;
     }
 }
@@ -670,12 +669,10 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
         if (lane == 0)
             for (int i = 0; i < nt; ++i) part[((size_t)sl * T_ + t0 + i) * E + e] = acc[i];
     }
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) is_last = atomicAdd(done_ctr, 1) == (int)gridDim.x - 1;
+    if (threadIdx.x == 0) is_last = atomic_add_acq_rel_gpu(done_ctr, 1) == (int)gridDim.x - 1;
     __syncthreads();
     if (!is_last) return;
-    __threadfence();
     for (long long i = threadIdx.x; i < (long long)T_ * E; i += kAlignThreads) {
         float v = 0.f;
         for (int sl = 0; sl < nslices; ++sl) v += __ldcg(part + (size_t)sl * T_ * E + i);
@@ -861,12 +858,10 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
         topk_one_token_r<(kE + 31) / 32>(src, kE, K, token_k(k_per_token, t, K), score_fn, renorm,
                                          ids + (size_t)t * K, w + (size_t)t * K, lane);
     }
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) is_last = atomicAdd(done_ctr, 1) == (int)gridDim.x - 1;
+    if (threadIdx.x == 0) is_last = atomic_add_acq_rel_gpu(done_ctr, 1) == (int)gridDim.x - 1;
     __syncthreads();
     if (!is_last) return;
-    __threadfence();
     align_block(T_, K, kE, B, mode, P_max, ids, counts, offsets, sorted_ids, block_expert, pos, scalars, stats_copy,
                 reinterpret_cast<int*>(route_sm));
     if (threadIdx.x == 0) *done_ctr = 0;  // ready for the next launch
