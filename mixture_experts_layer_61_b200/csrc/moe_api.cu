@@ -111,7 +111,8 @@ int routed_max_n_avg(const moe_config_t* c);
 
 // The layer's routing runs as one small-batch launch (route_small_kernel).
 bool small_route(const moe_config_t* c) {
-    return c->T <= kSmallRouteMaxT && c->H % 8 == 0 && (long long)c->E * c->H <= kSmallRouteMaxEH;
+    return c->T <= kSmallRouteMaxT && c->H % 8 == 0 &&
+           ((long long)c->E * c->H <= kSmallRouteMaxEH || (long long)c->T * c->E <= kSmallRouteMaxTE);
 }
 
 // FP8 expert weights run at decode sizes only (the fused expert FFN)

@@ -157,12 +157,16 @@ int launch_align(int T, int K, int E, int B, int mode, long long P_max, const in
                  int32_t* offsets, int32_t* sorted_ids, int32_t* block_expert, int32_t* pos, int32_t* scalars,
                  int32_t* stats_copy, cudaStream_t stream);
 // Router logits (CUDA cores) + top-K + alignment in one launch, for small T
-// and a small router matrix (E H <= kSmallRouteMaxEH): with a large one the
-// single block that reduces the partial sums and runs top-K and the alignment
-// outlasts the three separate launches (DeepSeek-V3-shaped layer at T = 32:
-// 81 us against 17 + 14 + 8).
+// and a small router matrix (E H <= kSmallRouteMaxEH), or any router matrix
+// with few logits (T E <= kSmallRouteMaxTE): with many logits of a large
+// router the single block that reduces the partial sums and runs top-K and
+// the alignment outlasts the three separate launches (DeepSeek-V3-shaped
+// layer at T = 8: 6 us slower per layer, at T = 32: 56 us), while with one
+// token it saves two launch hand-overs (T = 1: DeepSeek-V3-shaped 8 us,
+// Qwen2-MoE-shaped 7 us faster).
 constexpr int kSmallRouteMaxT = 64;
 constexpr long long kSmallRouteMaxEH = 1 << 17;
+constexpr long long kSmallRouteMaxTE = 256;
 // `part` holds (H/256 + 1) * T * E floats of partial router sums.
 int launch_route_small(int T, int H, int E, int K, int score_fn, int renorm, int B, int mode, long long P_max,
                        int dtype, const void* x, const void* w_r, const float* logits_override,
