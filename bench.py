@@ -44,9 +44,9 @@ N_INPUT_SETS = 4  # seeded token sets rotated through the timed steps (different
 # current kernels (dram__bytes_read.sum + dram__bytes_write.sum); workloads
 # without a capture report None.  Summaries of the captures are in profiles/.
 NCU_TRAFFIC = {
-    "mixtral:2048": 2.086e9 + 0.129e9,         # moe_gemm_kernel gate/up + SwiGLU, CTA pairs, aligned tail split
-    "mixtral:32": 2.824100e9 + 0.006820e9,     # moe_ffn_stream_kernel, fused decode FFN
-    "mixtral:32:fp8": 1.415910e9 + 0.006099e9,  # moe_ffn_stream_kernel, FP8 weights (E4M3 x E4M3 MMAs)
+    "mixtral:2048": 2.264e9 + 0.137e9,         # moe_gemm_kernel gate/up + SwiGLU, CTA pairs, aligned tail split
+    "mixtral:32": 2.824110e9 + 0.006375e9,     # moe_ffn_stream_kernel, fused decode FFN
+    "mixtral:32:fp8": 1.415865e9 + 0.005974e9,  # moe_ffn_stream_kernel, FP8 weights (E4M3 x E4M3 MMAs)
 }
 
 
