@@ -138,10 +138,9 @@ int moe_router_gemm(const moe_config_t* cfg, const void* x, const void* w_router
  *   loads the library until the process exits.  No allocation is made.
  *   Limits: T <= 32 (larger T returns MOE_ERR_ARG: use moe_router_gemm) and
  *   at most 160 SMs.  The first call on each device looks up the array's
- *   device address (cudaGetSymbolAddress); make that first call before any
- *   stream capture.  Each call clears the shared control words before its
- *   launch; calls that overlap on the GPU (unordered streams) race on the
- *   shared array.  A device wait that runs out sets a status word in the
+ *   device address (cudaGetSymbolAddress).  Each call clears the shared
+ *   control words before its launch; calls that overlap on the GPU
+ *   (unordered streams) race on the shared array.  A device wait that runs out sets a status word in the
  *   array and may leave logits partly written (the tiles whose blocks gave up);
  *   moe_router_gemm_noalloc_status reports it. */
 int moe_router_gemm_noalloc(const moe_config_t* cfg, const void* x, const void* w_router,
