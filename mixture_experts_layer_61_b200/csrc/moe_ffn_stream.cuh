@@ -42,7 +42,8 @@
 //    rows further on, and their scales x_scale);
 //  * down: phase A stores the SwiGLU activations in f16 and raises, per token
 //    row, the maximum |activation| (atomicMax on the fp32 bits) before its
-//    chunk counter; a phase-B item's first stage brings those maxima along
+//    band counter; a phase-B item (which waits for every band of its chunk)
+//    brings those maxima along on its first stage
 //    (bulk copy on the stage's barrier), and warps 6..13 split each stage's
 //    f16 activation tile in place into hi and lo E4M3 codes (row scale from
 //    the maximum) before the MMA thread issues.  The split keeps about 8
