@@ -34,7 +34,7 @@ def _rank(rank, world, port, totals, out):
 def test_max_over_ranks_and_whole_job_throughput_gloo():
     world = 2
     totals = [25.0, 31.5]   # ms of K = 20 steps on each rank
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of this multi-threaded process
     out = mgr.dict()
     mp.spawn(_rank, args=(world, _free_port(), totals, out), nprocs=world, join=True)
     for r in range(world):

@@ -53,7 +53,7 @@ def _rank(rank, world, port, out):
 
 @pytest.mark.parametrize("world", [2, 4])
 def test_tp_allreduce_of_rank_partials_is_the_whole_layer_gloo(world):
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of this multi-threaded process
     out = mgr.dict()
     mp.spawn(_rank, args=(world, _free_port(), out), nprocs=world, join=True)
     x, w_r, w13, w2, w13_sh, w2_sh, K = _layer(5)
@@ -110,7 +110,7 @@ def _rank_overlapped(rank, world, port, n_chunks, out):
 
 @pytest.mark.parametrize("world,n_chunks", [(2, 2), (2, 4), (4, 4)])
 def test_tp_overlapped_allreduce_protocol_gloo(world, n_chunks):
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of this multi-threaded process
     out = mgr.dict()
     mp.spawn(_rank_overlapped, args=(world, _free_port(), n_chunks, out), nprocs=world, join=True)
     x, w_r, w13, w2, w13_sh, w2_sh, K = _layer(5)
